@@ -1,0 +1,425 @@
+"""Pins for the CPU oracle: checks that tie it to something other than itself.
+
+Each ``pin_*`` function raises AssertionError when the oracle library passed in
+(``lib``; None = the real one) breaks a fact fixed by the definition of
+decode attention or of the tile plan: closed forms, invariants, special cases
+that reduce to a library routine (torch's scaled_dot_product_attention and
+logsumexp in float64), hand-derived worked examples, and brute force on tiny
+inputs.  The same battery is run against deliberately broken copies of the
+oracle (tests/test_oracle_mutants.py) to show that each plausible mistake is
+caught by at least one pin.
+
+Operation source: "Tencent HPC lands in SGLang, challenging default inference
+kernels", section "Why Tencent HPC matters for online model serving".
+"""
+
+from __future__ import annotations
+
+import json
+import math
+import os
+
+import numpy as np
+import torch
+
+import oracle
+
+GOLDEN = os.path.join(os.path.dirname(os.path.abspath(__file__)), "golden")
+
+
+# ---------------------------------------------------------------------------------------------
+# Small case construction: dense per-request K/V -> pages, in a chosen page order.
+
+
+def bf16(x) -> torch.Tensor:
+    return torch.as_tensor(np.asarray(x, dtype=np.float32)).to(torch.bfloat16)
+
+
+def pack(dense_k, dense_v, page_size: int, rng: np.random.Generator | None = None, spare: int = 1,
+         max_pages: int | None = None):
+    """Lay out per-request dense K/V ([L_b, Hkv, d] bf16) as [pages, Hkv, P, d] with a block table."""
+    Hkv, d = dense_k[0].shape[1], dense_k[0].shape[2]
+    P = page_size
+    used = [-(-k.shape[0] // P) for k in dense_k]
+    n_pages = sum(used) + spare
+    order = rng.permutation(n_pages) if rng is not None else np.arange(n_pages)
+    mp = max_pages or max(1, max(used))
+    bt = np.full((len(dense_k), mp), -1, dtype=np.int32)
+    kc = torch.full((n_pages, Hkv, P, d), float("nan"), dtype=torch.bfloat16)
+    vc = kc.clone()
+    o = 0
+    for b, (k, v) in enumerate(zip(dense_k, dense_v)):
+        for j in range(used[b]):
+            page = int(order[o]); o += 1
+            bt[b, j] = page
+            rows = slice(j * P, min((j + 1) * P, k.shape[0]))
+            n = rows.stop - rows.start
+            kc[page, :, :n, :] = k[rows].permute(1, 0, 2)
+            vc[page, :, :n, :] = v[rows].permute(1, 0, 2)
+    lens = np.array([k.shape[0] for k in dense_k], dtype=np.int32)
+    return kc, vc, bt, lens
+
+
+def random_case(rng, B, Hq, Hkv, d, P, lens, scale=None):
+    q = bf16(rng.standard_normal((B, Hq, d)))
+    dk = [bf16(rng.standard_normal((L, Hkv, d))) for L in lens]
+    dv = [bf16(rng.standard_normal((L, Hkv, d))) for L in lens]
+    kc, vc, bt, sl = pack(dk, dv, P, rng)
+    scale = float(np.float32(1.0 / math.sqrt(d))) if scale is None else scale
+    return q, dk, dv, kc, vc, bt, sl, scale
+
+
+def run(lib, q, kc, vc, bt, sl, scale, **kw):
+    return oracle.attention(q, kc, vc, bt, sl, scale=scale, lib=lib, **kw)
+
+
+# ---------------------------------------------------------------------------------------------
+# Attention pins.
+
+
+def pin_golden_attention(lib=None):
+    with open(os.path.join(GOLDEN, "attention_hand.json")) as f:
+        cases = json.load(f)["cases"]
+    for c in cases:
+        d = len(c["q"])
+        q = bf16(c["q"]).reshape(1, 1, d)
+        k = bf16(c["k"]).reshape(-1, 1, d)
+        v = bf16(c["v"]).reshape(-1, 1, d)
+        assert torch.equal(q.float(), torch.tensor(c["q"]).reshape(1, 1, d)), "fixture not bf16-exact"
+        kc, vc, bt, sl = pack([k], [v], c["page_size"], np.random.default_rng(7))
+        out, lse, st = run(lib, q, kc, vc, bt, sl, c["scale"])
+        assert st == oracle.OK
+        want = np.array([eval(e, {"math": math}) for e in c["out"]])
+        np.testing.assert_allclose(out[0, 0], want, rtol=1e-13, atol=1e-13, err_msg=c["name"])
+        assert abs(lse[0, 0] - eval(c["lse"], {"math": math})) < 1e-13, c["name"]
+
+
+def pin_length_one(lib=None):
+    """One cached token: the softmax weight is 1, so out is that V row and lse is its score."""
+    rng = np.random.default_rng(11)
+    for (Hq, Hkv, d, P) in [(4, 1, 64, 16), (8, 2, 32, 4), (6, 3, 16, 1)]:
+        q, dk, dv, kc, vc, bt, sl, scale = random_case(rng, 3, Hq, Hkv, d, P, [1, 1, 1])
+        out, lse, st = run(lib, q, kc, vc, bt, sl, scale)
+        assert st == oracle.OK
+        G = Hq // Hkv
+        for b in range(3):
+            for h in range(Hq):
+                g = h // G
+                assert np.array_equal(out[b, h], dv[b][0, g].double().numpy())
+                s0 = scale * float(torch.dot(q[b, h].double(), dk[b][0, g].double()))
+                assert abs(lse[b, h] - s0) <= 1e-12 * max(1.0, abs(s0))
+
+
+def pin_constant_v(lib=None):
+    """If every V row equals c, every convex combination of them is c."""
+    rng = np.random.default_rng(12)
+    B, Hq, Hkv, d, P = 3, 8, 2, 16, 4
+    lens = [5, 17, 33]
+    q = bf16(rng.standard_normal((B, Hq, d)) * 3)
+    dk = [bf16(rng.standard_normal((L, Hkv, d)) * 3) for L in lens]
+    c = bf16(rng.standard_normal((Hkv, d)))
+    dv = [c.unsqueeze(0).expand(L, Hkv, d).contiguous() for L in lens]
+    kc, vc, bt, sl = pack(dk, dv, P, rng)
+    out, lse, st = run(lib, q, kc, vc, bt, sl, 0.3)
+    assert st == oracle.OK
+    for b in range(B):
+        for h in range(Hq):
+            np.testing.assert_allclose(out[b, h], c[h // (Hq // Hkv)].double().numpy(), rtol=1e-13, atol=1e-14)
+
+
+def pin_uniform_scores(lib=None):
+    """q = 0 (or scale = 0): all scores are 0, so out is the mean of the V rows and lse = ln L."""
+    rng = np.random.default_rng(13)
+    B, Hq, Hkv, d, P = 3, 4, 2, 8, 3
+    lens = [1, 10, 29]
+    _, dk, dv, kc, vc, bt, sl, _ = random_case(rng, B, Hq, Hkv, d, P, lens)
+    for qv, sc in [(torch.zeros(B, Hq, d, dtype=torch.bfloat16), 0.7),
+                   (bf16(rng.standard_normal((B, Hq, d))), 0.0)]:
+        out, lse, st = run(lib, qv, kc, vc, bt, sl, sc)
+        assert st == oracle.OK
+        for b, L in enumerate(lens):
+            for h in range(Hq):
+                g = h // (Hq // Hkv)
+                np.testing.assert_allclose(out[b, h], dv[b][:, g].double().mean(0).numpy(), rtol=1e-12, atol=1e-13)
+                assert abs(lse[b, h] - math.log(L)) < 1e-13
+
+
+def pin_dominant_key(lib=None):
+    """One key far ahead of the rest: the output tends to its V row, lse to its score."""
+    rng = np.random.default_rng(14)
+    d, L, P = 16, 40, 8
+    q = bf16(np.ones((1, 1, d)))
+    k = torch.zeros(L, 1, d, dtype=torch.bfloat16)
+    k[23, 0, :] = 4.0  # score 64 * scale vs 0 elsewhere
+    v = bf16(rng.standard_normal((L, 1, d)))
+    kc, vc, bt, sl = pack([k], [v], P, rng)
+    out, lse, st = run(lib, q, kc, vc, bt, sl, 1.0)
+    assert st == oracle.OK
+    # exact answer: weight w = e^64 / (e^64 + 39) on row 23, (1 - w)/39 on each other row
+    np.testing.assert_allclose(out[0, 0], v[23, 0].double().numpy(), rtol=1e-15, atol=40 * math.exp(-64) * 4)
+    assert abs(lse[0, 0] - 64.0) < 1e-20 + 39 * math.exp(-64)
+
+
+def pin_page_order_invariance(lib=None):
+    """Moving pages around while rewriting the block table must not change a single bit."""
+    rng = np.random.default_rng(15)
+    B, Hq, Hkv, d, P = 4, 8, 2, 32, 4
+    lens = [3, 4, 9, 30]
+    q = bf16(rng.standard_normal((B, Hq, d)))
+    dk = [bf16(rng.standard_normal((L, Hkv, d))) for L in lens]
+    dv = [bf16(rng.standard_normal((L, Hkv, d))) for L in lens]
+    a = run(lib, q, *pack(dk, dv, P, np.random.default_rng(1)), 0.25)
+    b = run(lib, q, *pack(dk, dv, P, np.random.default_rng(2), spare=5), 0.25)
+    c = run(lib, q, *pack(dk, dv, P, None), 0.25)
+    assert a[2] == b[2] == c[2] == oracle.OK
+    for x in (b, c):
+        assert np.array_equal(a[0], x[0]) and np.array_equal(a[1], x[1])
+
+
+def pin_prefix_sharing(lib=None):
+    """Two requests whose block tables name the same pages (a shared prefix) see the same tokens."""
+    rng = np.random.default_rng(16)
+    Hq, Hkv, d, P = 4, 2, 16, 4
+    q1 = bf16(rng.standard_normal((1, Hq, d)))
+    k = bf16(rng.standard_normal((12, Hkv, d)))
+    v = bf16(rng.standard_normal((12, Hkv, d)))
+    kc, vc, bt, sl = pack([k], [v], P, rng)
+    bt2 = np.concatenate([bt, bt], 0)
+    q2 = torch.cat([q1, q1], 0)
+    out, lse, st = run(lib, q2, kc, vc, bt2, np.array([12, 8], np.int32), 0.25)
+    ref8, lse8, _ = run(lib, q1, *pack([k[:8]], [v[:8]], P, None), 0.25)
+    ref12, lse12, _ = run(lib, q1, *pack([k], [v], P, None), 0.25)
+    assert st == oracle.OK
+    assert np.array_equal(out[0], ref12[0]) and np.array_equal(out[1], ref8[0])
+    assert np.array_equal(lse[1], lse8[0]) and np.array_equal(lse[0], lse12[0])
+
+
+def pin_matches_sdpa(lib=None):
+    """Brute force by a library routine: torch SDPA (float64, GQA) and logsumexp over the gathered cache."""
+    rng = np.random.default_rng(17)
+    for (B, Hq, Hkv, d, P, lens) in [(3, 4, 1, 64, 16, [1, 7, 40]), (2, 8, 2, 8, 3, [13, 26]),
+                                     (2, 6, 3, 16, 1, [5, 9]), (4, 16, 2, 128, 64, [64, 65, 130, 1])]:
+        q, dk, dv, kc, vc, bt, sl, scale = random_case(rng, B, Hq, Hkv, d, P, lens)
+        out, lse, st = run(lib, q, kc, vc, bt, sl, scale)
+        assert st == oracle.OK
+        for b in range(B):
+            qb = q[b].double().unsqueeze(0).unsqueeze(2)  # [1, Hq, 1, d]
+            kb = dk[b].double().permute(1, 0, 2).unsqueeze(0)  # [1, Hkv, L, d]
+            vb = dv[b].double().permute(1, 0, 2).unsqueeze(0)
+            ref = torch.nn.functional.scaled_dot_product_attention(qb, kb, vb, scale=scale, enable_gqa=True)
+            np.testing.assert_allclose(out[b], ref[0, :, 0].numpy(), rtol=1e-11, atol=1e-12)
+            kx = kb.repeat_interleave(Hq // Hkv, dim=1)  # torch's GQA convention
+            s = torch.einsum("hd,htd->ht", qb[0, :, 0], kx[0]) * scale
+            np.testing.assert_allclose(lse[b], torch.logsumexp(s, dim=1).numpy(), rtol=1e-12, atol=1e-12)
+
+
+def pin_split_merge_identity(lib=None):
+    """Attention over [0, a) and [a, L) merged by log-sum-exp equals attention over [0, L).
+
+    The second piece is taken by starting the block table at page a / P.  The
+    merged result is checked both with the oracle's combine and with a
+    weighting written here from the two partial normalisers.
+    """
+    rng = np.random.default_rng(18)
+    Hq, Hkv, d, P = 4, 2, 16, 4
+    L = 37
+    q = bf16(rng.standard_normal((1, Hq, d)))
+    k = bf16(rng.standard_normal((L, Hkv, d)))
+    v = bf16(rng.standard_normal((L, Hkv, d)))
+    kc, vc, bt, sl = pack([k], [v], P, rng)
+    full, full_lse, _ = run(lib, q, kc, vc, bt, sl, 0.4)
+    for a in (4, 8, 20, 36):
+        pieces = [(bt, a), (bt[:, a // P:], L - a)]
+        parts = [run(lib, q, kc, vc, np.ascontiguousarray(t), np.array([n], np.int32), 0.4) for t, n in pieces]
+        for h in range(Hq):
+            o = np.stack([p[0][0, h] for p in parts])
+            l = np.array([p[1][0, h] for p in parts])
+            merged, merged_lse = oracle.combine(o, l, lib=lib)
+            np.testing.assert_allclose(merged, full[0, h], rtol=1e-12, atol=1e-13)
+            assert abs(merged_lse - full_lse[0, h]) < 1e-12
+            # a second, separately written merge: weights e^{lse_i} / e^{lse_full}
+            w = np.exp(l - full_lse[0, h])
+            assert abs(w.sum() - 1.0) < 1e-12
+            np.testing.assert_allclose((w[:, None] * o).sum(0), full[0, h], rtol=1e-12, atol=1e-13)
+    # merging with an empty piece (lse = -inf) changes nothing
+    m, ml = oracle.combine(np.stack([full[0, 0], np.zeros(d)]), np.array([full_lse[0, 0], -np.inf]), lib=lib)
+    assert np.array_equal(m, full[0, 0]) or np.allclose(m, full[0, 0], rtol=1e-15)
+    assert ml == full_lse[0, 0]
+    m, ml = oracle.combine(np.zeros((2, d)), np.array([-np.inf, -np.inf]), lib=lib)
+    assert ml == -np.inf and not m.any()
+
+
+def pin_degenerate_lengths(lib=None):
+    """Length 0 gives out = 0, lse = -inf; out-of-range lengths are reported and count as 0."""
+    rng = np.random.default_rng(19)
+    Hq, Hkv, d, P = 2, 1, 8, 4
+    q, dk, dv, kc, vc, bt, sl, scale = random_case(rng, 2, Hq, Hkv, d, P, [0, 6])
+    out, lse, st = run(lib, q, kc, vc, bt, sl, scale)
+    assert st == oracle.OK
+    assert not out[0].any() and np.all(lse[0] == -np.inf) and np.all(np.isfinite(lse[1]))
+    for bad in (-1, bt.shape[1] * P + 1):
+        out, lse, st = run(lib, q, kc, vc, bt, np.array([bad, 6], np.int32), scale)
+        assert st == oracle.ERR_BAD_SEQLEN
+        assert not out[0].any() and np.all(lse[0] == -np.inf)
+    bt2 = bt.copy()
+    bt2[1, 0] = kc.shape[0]  # page id out of range
+    _, _, st = run(lib, q, kc, vc, bt2, sl, scale)
+    assert st == oracle.ERR_BAD_PAGE
+
+
+def pin_pairs_match_full(lib=None):
+    rng = np.random.default_rng(20)
+    q, dk, dv, kc, vc, bt, sl, scale = random_case(rng, 3, 8, 2, 16, 4, [3, 11, 20])
+    full, full_lse, _ = run(lib, q, kc, vc, bt, sl, scale)
+    pb = np.array([2, 0, 1, 2], np.int32)
+    ph = np.array([7, 0, 3, 4], np.int32)
+    sub, sub_lse, st = run(lib, q, kc, vc, bt, sl, scale, pairs=(pb, ph))
+    assert st == oracle.OK
+    assert np.array_equal(sub, full[pb, ph]) and np.array_equal(sub_lse, full_lse[pb, ph])
+
+
+ATTENTION_PINS = [pin_golden_attention, pin_length_one, pin_constant_v, pin_uniform_scores, pin_dominant_key,
+                  pin_page_order_invariance, pin_prefix_sharing, pin_matches_sdpa, pin_split_merge_identity,
+                  pin_degenerate_lengths, pin_pairs_match_full]
+
+
+# ---------------------------------------------------------------------------------------------
+# Plan pins.
+
+
+def brute_force_plan(seq_lens, T, C, capacity):
+    """The dynamic plan by scanning: for each unit, search the CTA whose range holds it."""
+    n = [(-(-L // T) if 0 <= L <= capacity else 0) for L in seq_lens]
+    U = sum(n)
+    starts = [c * U // C for c in range(C + 1)]
+    segs = []  # [req, cta, tile_begin, tile_end]
+    u = 0
+    for r, nr in enumerate(n):
+        for t in range(nr):
+            cta = next(c for c in range(C) if starts[c] <= u < starts[c + 1])
+            if segs and segs[-1][0] == r and segs[-1][1] == cta:
+                segs[-1][3] = t + 1
+            else:
+                segs.append([r, cta, t, t + 1])
+            u += 1
+    return n, U, segs
+
+
+def check_plan_invariants(p, seq_lens, T, C, capacity):
+    n = [(-(-L // T) if 0 <= L <= capacity else 0) for L in seq_lens]
+    B, U, S = len(seq_lens), sum(n), p["num_segments"]
+    assert p["num_units"] == U
+    assert list(p["req_tile_prefix"]) == list(np.concatenate([[0], np.cumsum(n)]))
+    assert S <= C + max(B, 1) - 1
+    req, cta, tb, te = p["seg_req"], p["seg_cta"], p["seg_tile_begin"], p["seg_tile_end"]
+    assert np.all(te > tb)  # no empty segment in a dynamic plan
+    # segments of each request tile [0, n_b) in order, without gap or overlap
+    for b in range(B):
+        s0, s1 = p["req_seg_begin"][b], p["req_seg_begin"][b + 1]
+        assert np.all(req[s0:s1] == b)
+        cover = [t for s in range(s0, s1) for t in range(tb[s], te[s])]
+        assert cover == list(range(n[b]))
+    # each CTA's load is floor or ceil of U / C, its segments are contiguous and in unit order
+    loads = np.zeros(C, np.int64)
+    for c in range(C):
+        s0, s1 = p["cta_seg_begin"][c], p["cta_seg_begin"][c + 1]
+        assert np.all(cta[s0:s1] == c)
+        loads[c] = int((te[s0:s1] - tb[s0:s1]).sum())
+    assert loads.sum() == U
+    if U:
+        assert loads.min() >= U // C and loads.max() <= -(-U // C)
+    units = [p["req_tile_prefix"][req[s]] + tb[s] for s in range(S)]
+    assert units == sorted(units)
+
+
+def compare_plan(p, want: dict):
+    for key in ("num_units", "num_segments"):
+        assert p[key] == want[key], key
+    for key in ("req_tile_prefix", "req_seg_begin", "cta_seg_begin", "seg_req", "seg_cta", "seg_tile_begin",
+                "seg_tile_end"):
+        assert list(p[key]) == list(want[key]), key
+
+
+def pin_golden_plans(lib=None):
+    with open(os.path.join(GOLDEN, "plan_hand.json")) as f:
+        g = json.load(f)
+    for c in g["dynamic"]:
+        p = oracle.plan(c["seq_lens"], c["tile_tokens"], c["num_ctas"], 1 << 20, lib=lib)
+        compare_plan(p, c)
+    for c in g["static"]:
+        p = oracle.static_plan(c["seq_lens"], c["tile_tokens"], c["splits"], 1 << 20, lib=lib)
+        compare_plan(p, c)
+
+
+def pin_plan_brute_force(lib=None, exhaustive_batch: int = 3, max_len: int = 5):
+    import itertools
+    for B in range(0, exhaustive_batch + 1):
+        for lens in itertools.product(range(max_len + 1), repeat=B):
+            for T in (1, 2, 3):
+                for C in range(1, 7):
+                    p = oracle.plan(list(lens), T, C, 1 << 20, lib=lib)
+                    n, U, segs = brute_force_plan(list(lens), T, C, 1 << 20)
+                    got = list(zip(p["seg_req"], p["seg_cta"], p["seg_tile_begin"], p["seg_tile_end"]))
+                    assert got == [tuple(s) for s in segs], (lens, T, C)
+                    check_plan_invariants(p, list(lens), T, C, 1 << 20)
+
+
+def pin_plan_random(lib=None):
+    rng = np.random.default_rng(21)
+    for _ in range(60):
+        B = int(rng.integers(1, 300))
+        C = int(rng.choice([1, 7, 37, 148, 296, 1000]))
+        T = int(rng.choice([16, 32, 64, 128]))
+        lens = rng.integers(0, 5000, size=B)
+        lens[rng.random(B) < 0.2] = 0
+        p = oracle.plan(lens, T, C, 1 << 20, lib=lib)
+        check_plan_invariants(p, list(lens), T, C, 1 << 20)
+        if B * C < 20000:
+            _, _, segs = brute_force_plan(list(lens), T, C, 1 << 20)
+            got = list(zip(p["seg_req"], p["seg_cta"], p["seg_tile_begin"], p["seg_tile_end"]))
+            assert got == [tuple(s) for s in segs]
+
+
+def pin_plan_bad_lengths(lib=None):
+    p = oracle.plan([5, -3, 7, 99, 2], 2, 3, 10, lib=lib)
+    assert p["status"] == oracle.ERR_BAD_SEQLEN and p["bad_index"] == 1
+    check_plan_invariants(p, [5, 0, 7, 0, 2], 2, 3, 10)
+    p = oracle.plan([5, 3], 2, 3, 10, lib=lib)
+    assert p["status"] == oracle.OK and p["bad_index"] == -1
+
+
+def brute_force_static(seq_lens, T, S, capacity):
+    n = [(-(-L // T) if 0 <= L <= capacity else 0) for L in seq_lens]
+    maxT = max(n, default=0)
+    chunk = -(-maxT // S)
+    # split s of request b takes the tiles t < n_b with t // chunk == s
+    segs = []
+    for b, nb in enumerate(n):
+        for s in range(S):
+            tiles = [t for t in range(nb) if chunk and t // chunk == s]
+            lo = tiles[0] if tiles else min(s * chunk, nb)
+            hi = tiles[-1] + 1 if tiles else lo
+            segs.append((b, b * S + s, lo, hi))
+    return n, segs
+
+
+def pin_static_brute_force(lib=None):
+    import itertools
+    for B in range(0, 4):
+        for lens in itertools.product([0, 1, 3, 8, 17], repeat=B):
+            for T in (1, 4):
+                for S in (1, 2, 3, 5):
+                    p = oracle.static_plan(list(lens), T, S, 1 << 20, lib=lib)
+                    n, segs = brute_force_static(list(lens), T, S, 1 << 20)
+                    got = list(zip(p["seg_req"], p["seg_cta"], p["seg_tile_begin"], p["seg_tile_end"]))
+                    assert got == segs, (lens, T, S)
+                    assert p["num_units"] == sum(n)
+                    assert list(p["req_seg_begin"]) == [b * S for b in range(B + 1)]
+                    assert list(p["cta_seg_begin"]) == list(range(B * S + 1))
+                    # the longest request's splits are non-empty up to ceil(maxT / chunk) of them
+                    if n and max(n):
+                        chunk = -(-max(n) // S)
+                        assert sum(1 for s in segs if s[3] > s[2]) == sum(-(-x // chunk) for x in n)
+
+
+PLAN_PINS = [pin_golden_plans, pin_plan_brute_force, pin_plan_random, pin_plan_bad_lengths, pin_static_brute_force]
