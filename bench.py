@@ -1,0 +1,436 @@
+#!/usr/bin/env python
+"""Benchmark: one decode step of dynamic split-KV attention over a paged KV cache.
+
+A step is the whole hot path on one batch: on-device plan -> decode kernel ->
+log-sum-exp combine, through the C ABI (libda.so).  The default workload is the
+mixed-length batch (32 requests, lengths uniform in [1000, 16000], 64 query /
+8 KV heads, head_dim 128, page 64): 1.11 GB of K/V per step, far larger than
+the 126 MB L2, so consecutive steps cannot hit in L2.
+
+Printed (rank 0, one JSON line): KV-read GB/s of the whole step (value), the
+step time, the decode kernel's own achieved bandwidth against the measured HBM
+peak, the same step under the static split-k schedule (default and best split
+count), an end-to-end number with host<->device copies, the CPU oracle's rate
+on this machine's cores, and the SM clocks seen during the measurement.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference] [--config mixed]
+
+With N > 1 (torchrun) every rank runs its own, differently seeded batch of the
+same shape (weak scaling: requests are independent, so there is no data-path
+collective); the step time is the max over ranks and the value is the KV bytes
+of all ranks over that time.  `--impl reference` times the CPU oracle instead.
+"""
+
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "µs/decode step and KV-read HBM GB/s (% of B200 peak) vs static split-k"
+FALLBACK_HBM_GBS = 6650.0
+DATASHEET_HBM_GBS = 8000.0
+KERNEL_SOURCES = ["variable_length_paged_b200/csrc/decode.cu", "variable_length_paged_b200/csrc/da_internal.cuh"]
+TRAFFIC_FILE = os.path.join(ROOT, "profiles", "decode_kernel_traffic.json")
+
+
+def parse_args():
+    ap = argparse.ArgumentParser(description=__doc__.splitlines()[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--config", default="mixed", choices=["mixed", "skewed", "low_conc", "uniform", "tiny"])
+    ap.add_argument("--tile", type=int, default=64)
+    ap.add_argument("--width", type=int, default=0, help="CTAs per KV head (0 = 2 per SM / Hkv)")
+    ap.add_argument("--no-static", action="store_true", help="skip the static split-k comparison")
+    ap.add_argument("--no-cpu", action="store_true", help="skip the CPU oracle baseline")
+    ap.add_argument("--cpu-seconds", type=float, default=10.0)
+    return ap.parse_args()
+
+
+# ------------------------------------------------------------------------------------------------
+# plumbing
+
+
+def dist_setup(args):
+    import torch
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        backend = "nccl" if torch.cuda.is_available() else "gloo"
+        if backend == "nccl":
+            torch.cuda.set_device(local)
+        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=120))
+    elif torch.cuda.is_available():
+        torch.cuda.set_device(0)
+    return world, rank, local
+
+
+def reduce_max_sum(values_max, values_sum, world):
+    """Max over ranks of `values_max`, sum over ranks of `values_sum` (host floats)."""
+    if world == 1:
+        return list(values_max), list(values_sum)
+    import torch
+    import torch.distributed as dist
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    a = torch.tensor(values_max, dtype=torch.float64, device=dev)
+    b = torch.tensor(values_sum, dtype=torch.float64, device=dev)
+    dist.all_reduce(a, op=dist.ReduceOp.MAX)
+    dist.all_reduce(b, op=dist.ReduceOp.SUM)
+    return a.cpu().tolist(), b.cpu().tolist()
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def measured_peak():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            j = json.load(f)
+        return float(j["hbm_gbs"]), "MEASURED_PEAKS.json hbm_gbs (copy test on this pool; of measured)"
+    except Exception:
+        return FALLBACK_HBM_GBS, "profiling-recipe fallback 6.65 TB/s (of fallback)"
+
+
+def kernel_source_hash():
+    h = hashlib.sha256()
+    for rel in KERNEL_SOURCES:
+        with open(os.path.join(ROOT, rel), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def recorded_traffic(workload_name):
+    """DRAM bytes per decode launch from the committed ncu summary, if it matches this kernel source."""
+    try:
+        with open(TRAFFIC_FILE) as f:
+            j = json.load(f)
+    except Exception:
+        return None, "no ncu capture recorded"
+    if j.get("kernel_source_sha") != kernel_source_hash():
+        return None, "kernel changed since the ncu capture"
+    if j.get("workload") != workload_name:
+        return None, f"ncu capture was on {j.get('workload')}"
+    return int(j["dram_bytes_per_launch"]), j.get("command", "")
+
+
+class ClockSampler:
+    """nvidia-smi clocks/throttle reasons sampled every 200 ms while active."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index: int):
+        import torch
+        self.proc = None
+        self.file = tempfile.NamedTemporaryFile("w+", suffix=".csv", delete=False)
+        sel = []
+        try:
+            pr = torch.cuda.get_device_properties(device_index)
+            sel = ["-i", f"{pr.pci_domain_id:08X}:{pr.pci_bus_id:02X}:{pr.pci_device_id:02X}.0"]
+        except Exception:
+            vis = os.environ.get("CUDA_VISIBLE_DEVICES", "")
+            if vis:
+                sel = ["-i", vis.split(",")[device_index]]
+        self.cmd = ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits", "-lms", "200", *sel]
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(self.cmd, stdout=self.file, stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+        time.sleep(0.3)
+        return self
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+
+    def summary(self):
+        self.file.flush()
+        self.file.seek(0)
+        rows = [ln.strip().split(", ") for ln in self.file.read().splitlines() if ln.strip()]
+        rows = [r for r in rows if len(r) >= 9]
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no nvidia-smi samples"], "samples": 0}
+
+        def num(x):
+            try:
+                return float(x)
+            except ValueError:
+                return None
+        sm = [num(r[1]) for r in rows if num(r[1]) is not None]
+        smax = [num(r[2]) for r in rows if num(r[2]) is not None]
+        power = [num(r[3]) for r in rows if num(r[3]) is not None]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4) if r[5 + i].strip().lower() == "active"})
+        # median over samples taken while the GPU was clocked up (under load)
+        hi = [s for s in sm if smax and s >= 0.5 * max(smax)] or sm
+        return {"sm_mhz": statistics.median(hi) if hi else None, "sm_max_mhz": max(smax) if smax else None,
+                "reasons": reasons, "samples": len(rows), "power_w_max": max(power) if power else None}
+
+
+# ------------------------------------------------------------------------------------------------
+# our arm
+
+
+def time_region(stream, fn, steps):
+    """Device time of `steps` calls of fn() on `stream`, bracketed by CUDA events (ms)."""
+    import torch
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    e0.record(stream)
+    for _ in range(steps):
+        fn()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    return e0.elapsed_time(e1)
+
+
+def run_ours(args, world, rank, local):
+    import numpy as np
+    import torch
+
+    from variable_length_paged_b200 import da
+    from variable_length_paged_b200 import workloads as W
+
+    da.lib()  # fail loudly if the CUDA library is missing
+    seed_shift = 1000 * rank
+    gen = W.CONFIGS[args.config]
+    w = gen(seed=gen.__defaults__[0] + seed_shift) if rank else gen()
+    dw = w.to("cuda")
+    prob = da.problem_from(dw.problem)
+    desc = da.da_plan_desc_init(prob, da.PLAN_DYNAMIC, args.tile, args.width)
+    bufs = da.Buffers(prob, desc, "cuda")
+    kv_bytes = w.kv_bytes
+    stream = torch.cuda.Stream()
+    steps, warm = max(1, args.steps), max(3, args.warmup)
+
+    def step(d=desc, b=bufs):
+        da.decode_step(prob, d, dw.q, dw.k_cache, dw.v_cache, dw.block_table, dw.seq_lens, b, stream=stream)
+
+    result = {}
+    clocks = ClockSampler(local)
+    with clocks:
+        with torch.cuda.stream(stream):
+            for _ in range(warm):
+                step()
+            torch.cuda.synchronize()
+            status = da.da_read_status(bufs.ws, stream=stream)
+            # headline: the step captured in a CUDA graph (plan, decode, combine), replayed K times
+            graph = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(graph, stream=stream):
+                step()
+            for _ in range(warm):
+                graph.replay()
+            barrier(world)
+            ms_graph = time_region(stream, graph.replay, steps)
+            barrier(world)
+            ms_eager = time_region(stream, step, steps)
+            # decode kernel alone, per launch, inside a run of eager steps
+            ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
+            torch.cuda.synchronize()
+            for a, b in ev:
+                da.da_plan(prob, desc, dw.seq_lens, bufs.ws, stream=stream)
+                a.record(stream)
+                da.da_decode_attention(prob, desc, dw.q, dw.k_cache, dw.v_cache, dw.block_table, dw.seq_lens,
+                                       bufs.ws, bufs.partial_o, bufs.partial_lse, bufs.out, bufs.lse, stream=stream)
+                b.record(stream)
+                da.da_combine(prob, desc, bufs.ws, bufs.partial_o, bufs.partial_lse, bufs.out, bufs.lse,
+                              stream=stream)
+            torch.cuda.synchronize()
+            dec_ms = [a.elapsed_time(b) for a, b in ev]
+            # static split-k comparator: default split count, then a sweep
+            static = {}
+            if not args.no_static:
+                sdef = da.da_plan_desc_init(prob, da.PLAN_STATIC, args.tile, 0)
+                for S in [sdef.splits] + [s for s in (1, 2, 4, 8, 16, 32, 64) if s != sdef.splits]:
+                    sd = da.da_plan_desc_init(prob, da.PLAN_STATIC, args.tile, S)
+                    sb = da.Buffers(prob, sd, "cuda")
+                    for _ in range(warm):
+                        step(sd, sb)
+                    g2 = torch.cuda.CUDAGraph()
+                    with torch.cuda.graph(g2, stream=stream):
+                        step(sd, sb)
+                    ks = max(3, steps // 4)
+                    static[S] = time_region(stream, g2.replay, ks) / ks
+                    del g2, sb
+                static_default = static[sdef.splits]
+                best_S = min(static, key=static.get)
+            # end to end: host inputs -> device, step, outputs -> host, every step
+            q_h = w.q.pin_memory()
+            sl_h = torch.from_numpy(w.seq_lens).pin_memory()
+            bt_h = torch.from_numpy(w.block_table).pin_memory()
+            out_h = torch.empty(bufs.out.shape, dtype=bufs.out.dtype).pin_memory()
+            lse_h = torch.empty(bufs.lse.shape, dtype=bufs.lse.dtype).pin_memory()
+
+            def e2e_step():
+                dw.q.copy_(q_h, non_blocking=True)
+                dw.seq_lens.copy_(sl_h, non_blocking=True)
+                dw.block_table.copy_(bt_h, non_blocking=True)
+                step()
+                out_h.copy_(bufs.out, non_blocking=True)
+                lse_h.copy_(bufs.lse, non_blocking=True)
+
+            for _ in range(warm):
+                e2e_step()
+            barrier(world)
+            ms_e2e = time_region(stream, e2e_step, steps)
+    h2d = q_h.numel() * q_h.element_size() + sl_h.numel() * 4 + bt_h.numel() * 4
+    d2h = out_h.numel() * out_h.element_size() + lse_h.numel() * 4
+
+    dec_avg_ms = statistics.mean(dec_ms)
+    maxes, sums = reduce_max_sum([ms_graph, ms_eager, ms_e2e, dec_avg_ms], [float(kv_bytes)], world)
+    ms_graph, ms_eager, ms_e2e, dec_avg_ms = maxes
+    total_bytes = sums[0]
+    step_s = ms_graph / 1e3 / steps
+    value = total_bytes / step_s / 1e9
+    peak, peak_src = measured_peak()
+    dec_gbs = kv_bytes / (dec_avg_ms / 1e3) / 1e9
+    traffic, traffic_note = recorded_traffic(args.config)
+    result.update(
+        metric=METRIC, value=round(value, 2), unit="GB/s", n_gpus=world, steps=steps, warmup=warm,
+        ms_per_step=round(ms_graph / steps, 5), us_per_step=round(ms_graph / steps * 1e3, 2),
+        higher_is_better=True, scaling="weak", vs_baseline=None, dtype="bf16", data="synthetic",
+        config={"workload": f"{args.config}: {w.recipe}", "batch": w.problem.batch,
+                "kv_bytes_per_step_per_gpu": kv_bytes, "tile_tokens": desc.tile_tokens,
+                "ctas_per_kv_head": desc.num_ctas, "graph": True,
+                "l2": "inputs larger than L2 (K/V read per step >> 126 MB), no flush"},
+        frac_of_peak=round(value / world / peak, 4), frac_of_datasheet_8tbs=round(value / world / DATASHEET_HBM_GBS, 4),
+        eager_us_per_step=round(ms_eager / steps * 1e3, 2),
+        roofline={"bound": "hbm", "achieved": round(dec_gbs, 2), "peak": peak, "unit": "GB/s",
+                  "frac": round(dec_gbs / peak, 4), "traffic": traffic,
+                  "kernel": f"decode_kernel<{w.problem.head_dim}>", "algorithmic_bytes_per_launch": kv_bytes,
+                  "launch_us": round(dec_avg_ms * 1e3, 2), "peak_source": peak_src, "traffic_source": traffic_note},
+        e2e={"value": round(total_bytes / (ms_e2e / 1e3 / steps) / 1e9, 2), "unit": "GB/s",
+             "us_per_step": round(ms_e2e / steps * 1e3, 2), "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+        gpu_launches=3 * steps,
+        device_status=status[0],
+    )
+    if static:
+        result["static_split_k"] = {"default_splits": sdef.splits,
+                                    "default_us_per_step": round(static_default * 1e3, 2),
+                                    "best_splits": best_S, "best_us_per_step": round(static[best_S] * 1e3, 2),
+                                    "sweep_us": {str(k): round(v * 1e3, 2) for k, v in sorted(static.items())}}
+        result["speedup_vs_static_default"] = round(static_default / (ms_graph / steps), 3)
+        result["speedup_vs_static_best"] = round(static[best_S] / (ms_graph / steps), 3)
+    result["clocks"] = clocks.summary()
+    if rank == 0 and world == 1 and not args.no_cpu:
+        result["cpu_baseline"] = cpu_baseline(w, args.cpu_seconds)
+    return result
+
+
+def cpu_baseline(w, seconds):
+    """The CPU oracle (fp64) on this host's cores, repeated over the full batch for a bounded time."""
+    import oracle
+    oracle.build()
+    t0 = time.perf_counter()
+    passes = 0
+    while True:
+        oracle.attention(w.q, w.k_cache, w.v_cache, w.block_table, w.seq_lens, scale=w.problem.scale)
+        passes += 1
+        if time.perf_counter() - t0 >= seconds or passes >= 50:
+            break
+    dt = time.perf_counter() - t0
+    return {"value": round(passes * w.kv_bytes / dt / 1e9, 4), "unit": "GB/s", "cores": oracle.num_threads(),
+            "kind": "oracle", "sample": f"{passes} pass(es) of the fp64 oracle over the full batch "
+                                        f"({w.problem.batch} requests x {w.problem.num_q_heads} heads), {dt:.1f} s"}
+
+
+# ------------------------------------------------------------------------------------------------
+# reference arm: the CPU oracle, timed on bounded samples of the same workload
+
+
+def run_reference(args, rank):
+    import numpy as np
+
+    import oracle
+    from variable_length_paged_b200 import workloads as W
+
+    oracle.build()
+    w = W.CONFIGS[args.config]()
+    B, Hq = w.problem.batch, w.problem.num_q_heads
+    order = np.argsort(-w.seq_lens, kind="stable")
+    # calibrate: aim for about one second of oracle work per step, and at most ~150 s in total
+    t0 = time.perf_counter()
+    oracle.attention(w.q, w.k_cache, w.v_cache, w.block_table, w.seq_lens, scale=w.problem.scale,
+                     pairs=(np.full(Hq, order[-1], np.int32), np.arange(Hq, dtype=np.int32)))
+    rate = max(int(w.seq_lens[order[-1]]), 1) / max(time.perf_counter() - t0, 1e-6)  # tokens/s over all heads
+    steps, warm = max(1, args.steps), max(3, args.warmup)
+    budget_tokens = rate * min(1.0, 150.0 / (steps + warm))
+    picks, acc = [], 0
+    for b in np.random.default_rng(0).permutation(B):
+        if picks and acc + w.seq_lens[b] > budget_tokens:
+            continue
+        picks.append(int(b))
+        acc += int(w.seq_lens[b])
+    pb = np.repeat(np.array(picks, np.int32), Hq)
+    ph = np.tile(np.arange(Hq, dtype=np.int32), len(picks))
+    sample_bytes = acc * w.problem.num_kv_heads * w.problem.head_dim * 4
+
+    def one():
+        oracle.attention(w.q, w.k_cache, w.v_cache, w.block_table, w.seq_lens, scale=w.problem.scale, pairs=(pb, ph))
+
+    for _ in range(warm):
+        one()
+    t0 = time.perf_counter()
+    for _ in range(steps):
+        one()
+    dt = time.perf_counter() - t0
+    value = steps * sample_bytes / dt / 1e9
+    cpu = {"value": round(value, 4), "unit": "GB/s", "cores": oracle.num_threads(), "kind": "oracle",
+           "sample": f"{len(picks)} of {B} requests (all {Hq} heads, {acc} tokens) per step"}
+    return {"impl": "reference", "metric": METRIC, "value": round(value, 4), "unit": "GB/s", "n_gpus": 1,
+            "steps": steps, "warmup": warm, "ms_per_step": round(dt / steps * 1e3, 3), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": f"{args.config}: {w.recipe}", "batch": B,
+                       "kv_bytes_per_step_sample": sample_bytes},
+            "cpu_baseline": cpu,
+            "e2e": {"value": round(value, 4), "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+
+
+def main():
+    args = parse_args()
+    if args.impl == "reference":
+        if int(os.environ.get("RANK", "0")) != 0:
+            return 0
+        print(json.dumps(run_reference(args, 0)), flush=True)
+        return 0
+    world, rank, local = dist_setup(args)
+    try:
+        res = run_ours(args, world, rank, local)
+        if rank == 0:
+            print(json.dumps(res), flush=True)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.barrier()
+            dist.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

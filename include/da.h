@@ -1,0 +1,236 @@
+/*
+ * da.h -- C ABI of libda.so: split-KV decode attention over a paged,
+ * variable-length KV cache, load-balanced by an on-device tile planner
+ * ("Dynamic Attention"), for NVIDIA B200 (sm_100a).
+ *
+ * Source of the operation: "Tencent HPC lands in SGLang, challenging default
+ * inference kernels", section "Why Tencent HPC matters for online model
+ * serving": in a continuous batch one request may hold a 16,000-token context
+ * while another has just started with 1,000, so a static attention schedule
+ * leaves one block with far more work than another; the KV-cache work is cut
+ * into smaller uniform tiles and a scheduler hands the tiles to CTAs according
+ * to the current workload, rebuilding that mapping as request lengths change
+ * during decoding.  The same section names the baseline: a static split-k
+ * policy, which either idles units or launches empty chunks for short
+ * requests.  The article gives no API; the calls below are this library's.
+ *
+ * One decode step is three asynchronous calls on one stream:
+ *   da_plan              (or da_static_plan)  seq_lens -> work list in `ws`
+ *   da_decode_attention  work list -> out/lse (single-segment requests) and
+ *                        per-segment partials (split requests)
+ *   da_combine           partials -> out/lse by log-sum-exp merge
+ * The host never reads seq_lens: every launch's grid is fixed by the problem
+ * and the plan descriptor, so requests can join, grow, finish or be cancelled
+ * between steps without a host round trip, and the three calls can be
+ * captured in a CUDA graph.
+ *
+ * Conventions for every call:
+ *   - Return 0 (DA_OK) or a negative DA_ERR_* code.  Host-side argument
+ *     checks happen before anything is enqueued; a call that returns an error
+ *     has enqueued nothing.  DA_ERR_CUDA means a CUDA runtime call failed; its
+ *     cudaError_t value is available from da_last_cuda_error() (per thread).
+ *   - "dev" pointers are device memory (or managed memory) on the current
+ *     device; "host" pointers are ordinary host memory.  The caller allocates
+ *     and owns every buffer; the library allocates, frees and synchronises
+ *     nothing, except da_read_status, which synchronises its stream.
+ *   - `stream` is a cudaStream_t passed as void* (NULL = legacy default
+ *     stream).  Work is asynchronous; buffers must stay alive until it ends.
+ *   - Data errors found on the device (a length out of range, a page id out
+ *     of range, a wait that timed out) are not faults: the kernels skip the
+ *     bad work, record a DA_DEV_* code and the first offending index in the
+ *     workspace header, and keep going.  da_read_status reads them back.
+ */
+#ifndef DA_H
+#define DA_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define DA_API __attribute__((visibility("default")))
+#else
+#define DA_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* ---- return codes ------------------------------------------------------------------- */
+#define DA_OK 0
+#define DA_ERR_INVALID_ARG (-1) /* null pointer, negative size, inconsistent shapes */
+#define DA_ERR_UNSUPPORTED (-2) /* valid but not built: head_dim, group size, page size, tile size */
+#define DA_ERR_CUDA (-3)        /* a CUDA runtime call failed; see da_last_cuda_error() */
+#define DA_ERR_WORKSPACE (-4)   /* workspace smaller than da_workspace_size() asks for */
+
+/* ---- device status codes (workspace header, read with da_read_status) --------------- */
+#define DA_DEV_OK 0
+#define DA_DEV_BAD_SEQLEN 1 /* seq_lens[b] < 0 or > max_pages_per_req*page_size; request b treated as empty */
+#define DA_DEV_BAD_PAGE 2   /* a block-table entry outside [0, num_pages); that chunk is skipped */
+#define DA_DEV_TIMEOUT 3    /* a pipeline wait gave up after its time limit; results are incomplete */
+#define DA_DEV_BAD_PLAN 4   /* the workspace holds no plan matching this descriptor */
+
+/* ---- plan kinds ---------------------------------------------------------------------- */
+#define DA_PLAN_DYNAMIC 0 /* load-balanced: U tiles over C CTAs per KV head, contiguous ranges */
+#define DA_PLAN_STATIC 1  /* comparator: S equal splits per request, B*S CTAs per KV head */
+
+/*
+ * The problem: one decode step of a continuous batch.
+ *
+ *   q            bf16 [batch][num_q_heads][head_dim]            (one query token per request)
+ *   k/v cache    bf16 [num_pages][num_kv_heads][page_size][head_dim]
+ *                token t of request b lives in page block_table[b][t / page_size],
+ *                slot t % page_size; each (page, KV head) is one contiguous
+ *                page_size*head_dim*2-byte block.  Slots past a request's length
+ *                may hold anything (they are never used).
+ *   block_table  int32 [batch][max_pages_per_req]; only the first
+ *                ceil(seq_lens[b]/page_size) entries of row b are read, and several
+ *                requests may name the same page (shared prefixes).
+ *   seq_lens     int32 [batch], the number of cached tokens of each request,
+ *                0 for a finished or cancelled slot.
+ *   out          bf16 [batch][num_q_heads][head_dim];  lse fp32 [batch][num_q_heads]
+ *
+ * Query head h reads KV head h / (num_q_heads / num_kv_heads) (consecutive
+ * grouping).  out = softmax(scale * q . K^T) . V over the request's tokens and
+ * lse = ln sum_t exp(scale * q . k_t) (natural log of the scaled scores); an
+ * empty request gives out = 0, lse = -inf.
+ *
+ * Supported: head_dim 64 or 128; num_q_heads / num_kv_heads in 1..8;
+ * page_size a positive multiple of 16; num_pages * num_kv_heads * page_size
+ * below 2^31.
+ */
+typedef struct da_problem {
+  int32_t batch;
+  int32_t num_q_heads;
+  int32_t num_kv_heads;
+  int32_t head_dim;
+  int32_t page_size;
+  int32_t max_pages_per_req;
+  int32_t num_pages;
+  float scale;
+} da_problem;
+
+/*
+ * Host-side description of a plan, filled by da_plan_desc_init from host
+ * arguments only.  Pass the same descriptor to every call of a step.
+ */
+typedef struct da_plan_desc {
+  int32_t kind;         /* DA_PLAN_DYNAMIC or DA_PLAN_STATIC */
+  int32_t batch;        /* B, copied from the problem */
+  int32_t tile_tokens;  /* T: tokens per tile (the planner's unit of work) */
+  int32_t num_ctas;     /* grid width per KV head: C (dynamic) or B*S (static) */
+  int32_t splits;       /* S for a static plan, 0 for a dynamic one */
+  int32_t max_segments; /* capacity of the segment list: C+B-1 (dynamic) or B*S (static) */
+} da_plan_desc;
+
+/*
+ * da_plan_desc_init -- validate a problem and fix the plan geometry.
+ *   kind         DA_PLAN_DYNAMIC or DA_PLAN_STATIC.
+ *   tile_tokens  T > 0, a multiple of 16; 0 = default (64).
+ *   width        dynamic: C, CTAs per KV head; 0 = default
+ *                  max(1, floor(num_SMs * 2 / num_kv_heads)) on the current device.
+ *                static: S, splits per request; 0 = default
+ *                  clamp(ceil(num_SMs * 2 / (batch * num_kv_heads)), 1, 64).
+ *   desc         host, out.
+ * Tile size and C change only how work is spread; the result is the same up
+ * to fp32 rounding.  Queries the current device only when a default is asked.
+ */
+DA_API int da_plan_desc_init(const da_problem* prob, int32_t kind, int32_t tile_tokens, int32_t width,
+                             da_plan_desc* desc);
+
+/*
+ * da_workspace_size -- bytes the caller must allocate on the device:
+ *   ws_bytes           the plan (int32 header and work list), 16-byte aligned
+ *   partial_o_bytes    fp32 [max_segments][num_q_heads][head_dim]
+ *   partial_lse_bytes  fp32 [max_segments][num_q_heads]
+ * Any output pointer may be NULL.
+ */
+DA_API int da_workspace_size(const da_problem* prob, const da_plan_desc* desc, size_t* ws_bytes,
+                             size_t* partial_o_bytes, size_t* partial_lse_bytes);
+
+/*
+ * da_workspace_offsets -- word (int32) offsets of the arrays inside `ws`, for
+ * callers that inspect a plan (tests, tools):
+ *   off[0] header (16 words: units U, segments S, C, T, status, bad index,
+ *          kind, B, max_segments, splits, 6 spare)
+ *   off[1] segments, int32x4 [max_segments] = {request, cta, tile_begin, tile_end}
+ *          (tiles relative to the request; tile_begin == tile_end is an empty
+ *          static split)
+ *   off[2] req_tile_prefix [B+1]   off[3] req_seg_begin [B+1]
+ *   off[4] cta_seg_begin [num_ctas+1]
+ *   off[5] total words
+ * Segments of request b are [req_seg_begin[b], req_seg_begin[b+1]); segments
+ * of CTA c are [cta_seg_begin[c], cta_seg_begin[c+1]); both in tile order.
+ */
+DA_API int da_workspace_offsets(const da_plan_desc* desc, int64_t off[6]);
+
+/*
+ * da_plan -- dynamic (load-balanced) plan, one 1-CTA kernel.
+ *   seq_lens  dev int32 [batch].
+ *   ws        dev, >= ws_bytes, 16-byte aligned; overwritten (header status reset).
+ * n_b = ceil(L_b / T) tiles per request, U = sum n_b; KV head by KV head, CTA c
+ * gets the contiguous global tile range [floor(c*U/C), floor((c+1)*U/C)), cut
+ * at request boundaries into segments.  Requests with a bad length get 0
+ * tiles and DA_DEV_BAD_SEQLEN (first bad index = the lowest such b).
+ */
+DA_API int da_plan(const da_problem* prob, const da_plan_desc* desc, const int32_t* seq_lens, void* ws,
+                   size_t ws_bytes, void* stream);
+
+/*
+ * da_static_plan -- static split-k plan (the comparator), same work-list format.
+ * With maxT = ceil(max_b L_b / T) and chunk = ceil(maxT / S) tiles, split s of
+ * request b is CTA b*S+s and covers tiles [min(s*chunk, n_b), min((s+1)*chunk, n_b)),
+ * empty when s*chunk >= n_b (the CTA is launched and finds nothing to do).
+ */
+DA_API int da_static_plan(const da_problem* prob, const da_plan_desc* desc, const int32_t* seq_lens, void* ws,
+                          size_t ws_bytes, void* stream);
+
+/*
+ * da_decode_attention -- the split-KV decode kernel, grid (num_ctas, num_kv_heads).
+ *   q, k_cache, v_cache, block_table, seq_lens: dev, layouts as in da_problem;
+ *     k_cache and v_cache must be 16-byte aligned.
+ *   ws: dev, a plan made by da_plan / da_static_plan with the same descriptor
+ *     and the same seq_lens contents.
+ *   partial_o, partial_lse: dev scratch, sizes from da_workspace_size.
+ *   out, lse: dev outputs.  Requests with exactly one segment are written
+ *     here directly; the others are written by da_combine.
+ * Each CTA streams its tiles' K and V rows (bf16, TMA, multi-stage shared
+ * memory ring) and keeps, per query head of its KV group, the running max,
+ * running sum and fp32 accumulator of the online softmax.
+ */
+DA_API int da_decode_attention(const da_problem* prob, const da_plan_desc* desc, const void* q,
+                               const void* k_cache, const void* v_cache, const int32_t* block_table,
+                               const int32_t* seq_lens, const void* ws, float* partial_o, float* partial_lse,
+                               void* out, float* lse, void* stream);
+
+/*
+ * da_combine -- merge the partials of requests with two or more segments:
+ *   LSE = M + ln sum_i exp(lse_i - M),  M = max_i lse_i,
+ *   out = sum_i exp(lse_i - LSE) o_i    (fp32, segment order, then bf16),
+ * and write out = 0, lse = -inf for requests with no segment.
+ */
+DA_API int da_combine(const da_problem* prob, const da_plan_desc* desc, const void* ws, const float* partial_o,
+                      const float* partial_lse, void* out, float* lse, void* stream);
+
+/*
+ * da_read_status -- copy the device status word and first bad index out of
+ * `ws` (host outputs; either may be NULL).  Synchronises `stream`.
+ */
+DA_API int da_read_status(const void* ws, int32_t* dev_status, int32_t* bad_index, void* stream);
+
+/* Static text for a DA_OK / DA_ERR_* return code. */
+DA_API const char* da_status_string(int32_t code);
+
+/* Static text for a DA_DEV_* device status code. */
+DA_API const char* da_dev_status_string(int32_t code);
+
+/* cudaError_t of the last failing CUDA call made by this library on this thread (0 if none). */
+DA_API int32_t da_last_cuda_error(void);
+
+/* Number of SMs of the current device (host out). */
+DA_API int da_device_num_sms(int32_t* num_sms);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* DA_H */

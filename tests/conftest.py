@@ -18,3 +18,17 @@ def oracle_lib():
     import oracle
     oracle.build()
     return oracle
+
+
+@pytest.fixture(scope="session")
+def da_lib():
+    """The CUDA library, built in-tree if missing (nvcc cross-compiles without a GPU)."""
+    from variable_length_paged_b200 import build, da
+    build.build()
+    da.lib()
+    return da
+
+
+def cuda_available() -> bool:
+    import torch
+    return torch.cuda.is_available()

@@ -1,0 +1,118 @@
+"""The C ABI seen from the host, without a GPU: exports, sizes, layout and argument checks.
+
+Every call here returns before any CUDA call is made (argument checks come
+first), so nothing is launched.
+"""
+
+import re
+import subprocess
+
+import pytest
+
+from conftest import ROOT, cuda_available
+
+HEADER = f"{ROOT}/include/da.h"
+
+
+def header_functions():
+    text = open(HEADER).read()
+    return sorted(set(re.findall(r"DA_API\s+[\w\s\*]+?\b(da_\w+)\s*\(", text)))
+
+
+def test_every_declared_symbol_is_exported(da_lib):
+    declared = header_functions()
+    assert len(declared) >= 10
+    out = subprocess.run(["nm", "-D", "--defined-only", da_lib.LIB_PATH], capture_output=True, text=True).stdout
+    exported = set(re.findall(r" T (da_\w+)", out))
+    assert set(declared) <= exported, set(declared) - exported
+    assert exported <= set(declared), f"undeclared exports: {exported - set(declared)}"
+    assert sorted(da_lib.EXPORTS) == declared
+    for name in declared:
+        getattr(da_lib.lib(), name)
+
+
+def prob(da, **kw):
+    base = dict(batch=32, num_q_heads=64, num_kv_heads=8, head_dim=128, page_size=64, max_pages_per_req=250,
+                num_pages=8400, scale=0.08838834764831845)
+    base.update(kw)
+    return da.problem(**base)
+
+
+def test_plan_descriptor_and_sizes(da_lib):
+    da = da_lib
+    p = prob(da)
+    d = da.da_plan_desc_init(p, da.PLAN_DYNAMIC, 64, 37)
+    assert (d.kind, d.batch, d.tile_tokens, d.num_ctas, d.splits, d.max_segments) == (0, 32, 64, 37, 0, 37 + 32 - 1)
+    ws, po, pl = da.da_workspace_size(p, d)
+    off = da.da_workspace_offsets(d)
+    assert off[0] == 0 and off[1] == 16 and off[2] == 16 + 4 * d.max_segments
+    assert off[3] == off[2] + 33 and off[4] == off[3] + 33 and off[5] >= off[4] + 38 and off[5] % 4 == 0
+    assert ws == off[5] * 4 and ws % 16 == 0
+    assert po == d.max_segments * 64 * 128 * 4 and pl == d.max_segments * 64 * 4
+    s = da.da_plan_desc_init(p, da.PLAN_STATIC, 32, 3)
+    assert (s.kind, s.num_ctas, s.splits, s.max_segments, s.tile_tokens) == (1, 96, 3, 96, 32)
+    d0 = da.da_plan_desc_init(p, da.PLAN_DYNAMIC, 0, 5)
+    assert d0.tile_tokens == 64
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(num_q_heads=60), -1),          # Hq % Hkv != 0
+    (dict(head_dim=96), -2),             # only 64 / 128 are built
+    (dict(page_size=8), -2),             # pages must be multiples of 16 rows
+    (dict(num_q_heads=128, num_kv_heads=8), -2),  # group of 16 not built
+    (dict(batch=-1), -1),
+    (dict(num_pages=0), -1),
+    (dict(num_pages=1 << 30), -2),       # row index would overflow int32
+])
+def test_problem_checks(da_lib, kw, code):
+    da = da_lib
+    with pytest.raises(da.DaError) as e:
+        da.da_plan_desc_init(prob(da, **kw), da.PLAN_DYNAMIC, 64, 37)
+    assert e.value.code == code
+
+
+def test_descriptor_checks(da_lib):
+    da = da_lib
+    p = prob(da)
+    for kind, T, w, code in [(0, 24, 37, -2), (0, -16, 37, -1), (0, 64, -1, -1), (7, 64, 37, -1)]:
+        with pytest.raises(da.DaError) as e:
+            da.da_plan_desc_init(p, kind, T, w)
+        assert e.value.code == code
+    lib = da.lib()
+    import ctypes
+    d = da.da_plan_desc_init(p, da.PLAN_DYNAMIC, 64, 37)
+    bad = da.DaPlanDesc(d.kind, d.batch, d.tile_tokens, d.num_ctas, d.splits, d.max_segments - 1)
+    assert lib.da_workspace_size(ctypes.byref(p), ctypes.byref(bad), None, None, None) == -1
+    # a dynamic call given a static descriptor, and a workspace that is too small
+    s = da.da_plan_desc_init(p, da.PLAN_STATIC, 64, 2)
+    assert lib.da_plan(ctypes.byref(p), ctypes.byref(s), 16, 256, 1 << 20, None) == -1
+    assert lib.da_plan(ctypes.byref(p), ctypes.byref(d), 16, 256, 64, None) == -4
+    assert lib.da_plan(ctypes.byref(p), ctypes.byref(d), None, 256, 1 << 20, None) == -1
+    assert lib.da_plan(ctypes.byref(p), ctypes.byref(d), 16, 8, 1 << 20, None) == -1  # misaligned workspace
+    assert lib.da_decode_attention(ctypes.byref(p), ctypes.byref(d), *([None] * 10), None) == -1
+    assert lib.da_combine(None, ctypes.byref(d), *([None] * 5), None) == -1
+    assert lib.da_read_status(None, None, None, None) == -1
+    assert lib.da_workspace_offsets(None, None) == -1
+
+
+def test_status_strings(da_lib):
+    da = da_lib
+    assert da.status_string(0) == "ok" and "workspace" in da.status_string(-4)
+    assert "length" in da.dev_status_string(1) and "page" in da.dev_status_string(2)
+    assert "timed out" in da.dev_status_string(3) and "plan" in da.dev_status_string(4)
+
+
+@pytest.mark.skipif(cuda_available(), reason="checks the no-device error path")
+def test_default_width_needs_a_device(da_lib):
+    da = da_lib
+    with pytest.raises(da.DaError) as e:
+        da.da_plan_desc_init(prob(da), da.PLAN_DYNAMIC, 64, 0)
+    assert e.value.code == da.ERR_CUDA and e.value.cuda_error != 0
+
+
+def test_binding_fails_loudly_without_library(tmp_path, monkeypatch):
+    from variable_length_paged_b200 import da
+    monkeypatch.setattr(da, "_lib", None)
+    monkeypatch.setattr(da, "LIB_PATH", str(tmp_path / "missing.so"))
+    with pytest.raises(RuntimeError, match="libda.so not found"):
+        da.lib()

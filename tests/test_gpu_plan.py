@@ -1,0 +1,87 @@
+"""The on-device planners against the oracle's plans: bit-exact work lists."""
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from gpu_helpers import assert_plan_equal
+from variable_length_paged_b200 import da
+
+pytestmark = pytest.mark.gpu
+
+
+def plan_on_device(lens, T, width, kind, cap_pages=2048, P=64):
+    lens = np.asarray(lens, np.int32)
+    B = len(lens)
+    prob = da.problem(B, 8, 1, 128, P, cap_pages, 16, 0.1)
+    desc = da.da_plan_desc_init(prob, kind, T, width)
+    ws_bytes, _, _ = da.da_workspace_size(prob, desc)
+    ws = torch.full((ws_bytes // 4,), -7, dtype=torch.int32, device="cuda")
+    sl = torch.from_numpy(lens).cuda()
+    if kind == da.PLAN_DYNAMIC:
+        da.da_plan(prob, desc, sl, ws)
+    else:
+        da.da_static_plan(prob, desc, sl, ws)
+    torch.cuda.synchronize()
+    return da.read_plan(desc, ws), cap_pages * P
+
+
+CASES = [
+    [],
+    [0],
+    [0, 0, 0],
+    [1],
+    [1, 7, 64, 300],
+    [131072, 1000],
+    [4096] * 64,
+    [5, 0, 2],
+]
+
+
+def random_lens(seed):
+    rng = np.random.default_rng(seed)
+    B = int(rng.choice([1, 3, 32, 128, 256, 1500, 3000]))
+    lens = rng.integers(0, 20000, size=B)
+    lens[rng.random(B) < 0.15] = 0
+    short = rng.random(B) < 0.1
+    lens[short] = rng.integers(1, 70, size=int(short.sum()))
+    return lens
+
+
+@pytest.mark.parametrize("T", [16, 64, 256])
+@pytest.mark.parametrize("C", [1, 7, 37, 148, 1000])
+def test_dynamic_plan_fixed_cases(da_lib, oracle_lib, T, C):
+    for lens in CASES:
+        if not lens:
+            continue
+        got, cap = plan_on_device(lens, T, C, da.PLAN_DYNAMIC)
+        assert_plan_equal(got, oracle.plan(lens, T, C, cap))
+        assert got["status"] == 0
+
+
+@pytest.mark.parametrize("seed", range(12))
+def test_dynamic_plan_random(da_lib, oracle_lib, seed):
+    rng = np.random.default_rng(100 + seed)
+    lens = random_lens(seed)
+    T = int(rng.choice([16, 32, 64, 128]))
+    C = int(rng.choice([1, 5, 37, 74, 296, 999]))
+    got, cap = plan_on_device(lens, T, C, da.PLAN_DYNAMIC)
+    assert_plan_equal(got, oracle.plan(lens, T, C, cap))
+
+
+def test_dynamic_plan_bad_lengths(da_lib, oracle_lib):
+    lens = [100, -5, 7000, 2048 * 64 + 1, 3, -1]
+    got, cap = plan_on_device(lens, 64, 37, da.PLAN_DYNAMIC)
+    ref = oracle.plan(lens, 64, 37, cap)
+    assert ref["bad_index"] == 1
+    assert_plan_equal(got, ref)
+    assert got["status"] == da.DEV_BAD_SEQLEN
+
+
+@pytest.mark.parametrize("S", [1, 2, 3, 8, 64])
+def test_static_plan(da_lib, oracle_lib, S):
+    for lens in CASES[1:] + [list(random_lens(7)), list(random_lens(8))]:
+        got, cap = plan_on_device(lens, 64, S, da.PLAN_STATIC)
+        assert_plan_equal(got, oracle.static_plan(lens, 64, S, cap))
+        assert got["splits"] == S and got["kind"] == da.PLAN_STATIC

@@ -1,0 +1,321 @@
+// api.cu -- host side of libda.so: argument checks, plan geometry, TMA
+// descriptors and launches.  Nothing here allocates, frees or synchronises
+// (except da_read_status, documented to synchronise its stream).
+#include <cudaTypedefs.h>
+
+#include <climits>
+#include <cstring>
+#include <mutex>
+
+#include "da_internal.cuh"
+
+namespace {
+
+thread_local int32_t g_last_cuda_error = 0;
+
+constexpr int kDefaultTile = 64;
+constexpr int kCtasPerSm = 2;  // decode kernel residency (shared memory sized for two)
+constexpr int kMaxGroup = 8;
+
+int cuda_fail(cudaError_t e) {
+  g_last_cuda_error = (int32_t)e;
+  return DA_ERR_CUDA;
+}
+
+int check_problem(const da_problem* p) {
+  if (!p) return DA_ERR_INVALID_ARG;
+  if (p->batch < 0 || p->num_q_heads <= 0 || p->num_kv_heads <= 0 || p->head_dim <= 0 || p->page_size <= 0 ||
+      p->max_pages_per_req <= 0 || p->num_pages <= 0)
+    return DA_ERR_INVALID_ARG;
+  if (p->num_q_heads % p->num_kv_heads != 0) return DA_ERR_INVALID_ARG;
+  if (!(p->scale == p->scale)) return DA_ERR_INVALID_ARG;  // NaN scale
+  if (p->head_dim != 64 && p->head_dim != 128) return DA_ERR_UNSUPPORTED;
+  if (p->num_q_heads / p->num_kv_heads > kMaxGroup) return DA_ERR_UNSUPPORTED;
+  if (p->page_size % 16 != 0) return DA_ERR_UNSUPPORTED;
+  if ((int64_t)p->num_pages * p->num_kv_heads * p->page_size >= (int64_t)INT_MAX) return DA_ERR_UNSUPPORTED;
+  if ((int64_t)p->max_pages_per_req * p->page_size >= (int64_t)INT_MAX) return DA_ERR_UNSUPPORTED;
+  return DA_OK;
+}
+
+int check_desc(const da_problem* p, const da_plan_desc* d) {
+  if (!d) return DA_ERR_INVALID_ARG;
+  if (d->batch != p->batch || d->tile_tokens <= 0 || d->tile_tokens % 16 != 0 || d->num_ctas <= 0)
+    return DA_ERR_INVALID_ARG;
+  if (d->kind == DA_PLAN_DYNAMIC) {
+    if (d->splits != 0 || (int64_t)d->max_segments != (int64_t)d->num_ctas + (p->batch > 0 ? p->batch : 1) - 1)
+      return DA_ERR_INVALID_ARG;
+  } else if (d->kind == DA_PLAN_STATIC) {
+    if (d->splits <= 0 || (int64_t)d->num_ctas != (int64_t)p->batch * d->splits || d->max_segments != d->num_ctas)
+      return DA_ERR_INVALID_ARG;
+  } else {
+    return DA_ERR_INVALID_ARG;
+  }
+  // every tile index and unit count stays inside int32
+  const int64_t cap = (int64_t)p->max_pages_per_req * p->page_size;
+  if ((int64_t)p->batch * ((cap + d->tile_tokens - 1) / d->tile_tokens) >= (int64_t)INT_MAX) return DA_ERR_UNSUPPORTED;
+  if ((int64_t)d->num_ctas * ((int64_t)p->batch * ((cap + d->tile_tokens - 1) / d->tile_tokens) + 1) >=
+      ((int64_t)1 << 62))
+    return DA_ERR_UNSUPPORTED;
+  return DA_OK;
+}
+
+size_t ws_words(const da_plan_desc* d) {
+  return (size_t)da::ws_layout(d->batch, d->num_ctas, d->max_segments).total;
+}
+
+// cuTensorMapEncodeTiled, looked up once through the runtime (no link-time libcuda dependency).
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  });
+  return fn;
+}
+
+// 2-D bf16 view of a cache: x = head_dim (inner), y = (page, kv head, slot) rows.
+// Box = 64 columns (128 bytes, the 128-byte swizzle span) x box_rows rows.
+bool make_cache_map(CUtensorMap* map, const void* base, const da_problem* p, int box_rows) {
+  PFN_cuTensorMapEncodeTiled_v12000 enc = encode_fn();
+  if (!enc) return false;
+  cuuint64_t dims[2] = {(cuuint64_t)p->head_dim,
+                        (cuuint64_t)p->num_pages * (cuuint64_t)p->num_kv_heads * (cuuint64_t)p->page_size};
+  cuuint64_t strides[1] = {(cuuint64_t)p->head_dim * 2};
+  cuuint32_t box[2] = {64u, (cuuint32_t)box_rows};
+  cuuint32_t estr[2] = {1u, 1u};
+  CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+}  // namespace
+
+extern "C" {
+
+DA_API int32_t da_last_cuda_error(void) { return g_last_cuda_error; }
+
+DA_API int da_device_num_sms(int32_t* num_sms) {
+  if (!num_sms) return DA_ERR_INVALID_ARG;
+  int dev = 0, n = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e);
+  e = cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+  if (e != cudaSuccess) return cuda_fail(e);
+  *num_sms = n;
+  return DA_OK;
+}
+
+DA_API int da_plan_desc_init(const da_problem* prob, int32_t kind, int32_t tile_tokens, int32_t width,
+                             da_plan_desc* desc) {
+  int rc = check_problem(prob);
+  if (rc != DA_OK) return rc;
+  if (!desc || width < 0 || tile_tokens < 0) return DA_ERR_INVALID_ARG;
+  if (kind != DA_PLAN_DYNAMIC && kind != DA_PLAN_STATIC) return DA_ERR_INVALID_ARG;
+  const int T = tile_tokens == 0 ? kDefaultTile : tile_tokens;
+  if (T % 16 != 0) return DA_ERR_UNSUPPORTED;
+  int w = width;
+  if (w == 0) {
+    int32_t sms = 0;
+    rc = da_device_num_sms(&sms);
+    if (rc != DA_OK) return rc;
+    const int slots = sms * kCtasPerSm;
+    if (kind == DA_PLAN_DYNAMIC) {
+      w = slots / prob->num_kv_heads;
+      if (w < 1) w = 1;
+    } else {
+      const int64_t per = (int64_t)(prob->batch > 0 ? prob->batch : 1) * prob->num_kv_heads;
+      int64_t s = (slots + per - 1) / per;
+      w = (int)(s < 1 ? 1 : s > 64 ? 64 : s);
+    }
+  }
+  da_plan_desc d;
+  d.kind = kind;
+  d.batch = prob->batch;
+  d.tile_tokens = T;
+  if (kind == DA_PLAN_DYNAMIC) {
+    d.num_ctas = w;
+    d.splits = 0;
+    const int64_t ms = (int64_t)w + (prob->batch > 0 ? prob->batch : 1) - 1;
+    if (ms >= INT_MAX) return DA_ERR_UNSUPPORTED;
+    d.max_segments = (int32_t)ms;
+  } else {
+    const int64_t n = (int64_t)prob->batch * w;
+    if (n >= INT_MAX / 4) return DA_ERR_UNSUPPORTED;
+    if (n == 0) return DA_ERR_INVALID_ARG;  // a static grid needs at least one request
+    d.num_ctas = (int32_t)n;
+    d.splits = w;
+    d.max_segments = (int32_t)n;
+  }
+  rc = check_desc(prob, &d);
+  if (rc != DA_OK) return rc;
+  *desc = d;
+  return DA_OK;
+}
+
+DA_API int da_workspace_size(const da_problem* prob, const da_plan_desc* desc, size_t* ws_bytes,
+                             size_t* partial_o_bytes, size_t* partial_lse_bytes) {
+  int rc = check_problem(prob);
+  if (rc != DA_OK) return rc;
+  rc = check_desc(prob, desc);
+  if (rc != DA_OK) return rc;
+  if (ws_bytes) *ws_bytes = ws_words(desc) * 4;
+  if (partial_o_bytes) *partial_o_bytes = (size_t)desc->max_segments * prob->num_q_heads * prob->head_dim * 4;
+  if (partial_lse_bytes) *partial_lse_bytes = (size_t)desc->max_segments * prob->num_q_heads * 4;
+  return DA_OK;
+}
+
+DA_API int da_workspace_offsets(const da_plan_desc* desc, int64_t off[6]) {
+  if (!desc || !off || desc->batch < 0 || desc->num_ctas <= 0 || desc->max_segments <= 0) return DA_ERR_INVALID_ARG;
+  const da::WsLayout L = da::ws_layout(desc->batch, desc->num_ctas, desc->max_segments);
+  off[0] = L.hdr;
+  off[1] = L.segs;
+  off[2] = L.req_tile_prefix;
+  off[3] = L.req_seg_begin;
+  off[4] = L.cta_seg_begin;
+  off[5] = L.total;
+  return DA_OK;
+}
+
+static int plan_common(const da_problem* prob, const da_plan_desc* desc, const int32_t* seq_lens, void* ws,
+                       size_t ws_bytes, void* stream, int kind) {
+  int rc = check_problem(prob);
+  if (rc != DA_OK) return rc;
+  rc = check_desc(prob, desc);
+  if (rc != DA_OK) return rc;
+  if (desc->kind != kind) return DA_ERR_INVALID_ARG;
+  if (!ws || (prob->batch > 0 && !seq_lens)) return DA_ERR_INVALID_ARG;
+  if (reinterpret_cast<uintptr_t>(ws) % 16 != 0) return DA_ERR_INVALID_ARG;
+  if (ws_bytes < ws_words(desc) * 4) return DA_ERR_WORKSPACE;
+  da::PlanParams p;
+  p.seq_lens = seq_lens;
+  p.ws = static_cast<int32_t*>(ws);
+  p.batch = prob->batch;
+  p.tile_tokens = desc->tile_tokens;
+  p.width = kind == DA_PLAN_DYNAMIC ? desc->num_ctas : desc->splits;
+  p.max_segments = desc->max_segments;
+  p.num_ctas = desc->num_ctas;
+  p.capacity_tokens = (int64_t)prob->max_pages_per_req * prob->page_size;
+  cudaError_t e = kind == DA_PLAN_DYNAMIC ? da::launch_plan_dynamic(p, static_cast<cudaStream_t>(stream))
+                                          : da::launch_plan_static(p, static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? DA_OK : cuda_fail(e);
+}
+
+DA_API int da_plan(const da_problem* prob, const da_plan_desc* desc, const int32_t* seq_lens, void* ws,
+                   size_t ws_bytes, void* stream) {
+  return plan_common(prob, desc, seq_lens, ws, ws_bytes, stream, DA_PLAN_DYNAMIC);
+}
+
+DA_API int da_static_plan(const da_problem* prob, const da_plan_desc* desc, const int32_t* seq_lens, void* ws,
+                          size_t ws_bytes, void* stream) {
+  return plan_common(prob, desc, seq_lens, ws, ws_bytes, stream, DA_PLAN_STATIC);
+}
+
+DA_API int da_decode_attention(const da_problem* prob, const da_plan_desc* desc, const void* q,
+                               const void* k_cache, const void* v_cache, const int32_t* block_table,
+                               const int32_t* seq_lens, const void* ws, float* partial_o, float* partial_lse,
+                               void* out, float* lse, void* stream) {
+  int rc = check_problem(prob);
+  if (rc != DA_OK) return rc;
+  rc = check_desc(prob, desc);
+  if (rc != DA_OK) return rc;
+  if (prob->batch == 0) return DA_OK;
+  if (!q || !k_cache || !v_cache || !block_table || !seq_lens || !ws || !partial_o || !partial_lse || !out || !lse)
+    return DA_ERR_INVALID_ARG;
+  if (reinterpret_cast<uintptr_t>(k_cache) % 16 != 0 || reinterpret_cast<uintptr_t>(v_cache) % 16 != 0 ||
+      reinterpret_cast<uintptr_t>(q) % 4 != 0 || reinterpret_cast<uintptr_t>(out) % 4 != 0 ||
+      reinterpret_cast<uintptr_t>(partial_o) % 16 != 0 || reinterpret_cast<uintptr_t>(ws) % 16 != 0)
+    return DA_ERR_INVALID_ARG;
+  CUtensorMap maps[4];
+  if (!make_cache_map(&maps[0], k_cache, prob, 64) || !make_cache_map(&maps[1], v_cache, prob, 64) ||
+      !make_cache_map(&maps[2], k_cache, prob, 16) || !make_cache_map(&maps[3], v_cache, prob, 16))
+    return cuda_fail(cudaErrorInvalidValue);
+  da::DecodeParams p;
+  p.q = static_cast<const __nv_bfloat16*>(q);
+  p.block_table = block_table;
+  p.seq_lens = seq_lens;
+  p.ws = static_cast<const int32_t*>(ws);
+  p.partial_o = partial_o;
+  p.partial_lse = partial_lse;
+  p.out = static_cast<__nv_bfloat16*>(out);
+  p.lse = lse;
+  p.batch = prob->batch;
+  p.num_q_heads = prob->num_q_heads;
+  p.num_kv_heads = prob->num_kv_heads;
+  p.group = prob->num_q_heads / prob->num_kv_heads;
+  p.page_size = prob->page_size;
+  p.max_pages_per_req = prob->max_pages_per_req;
+  p.num_pages = prob->num_pages;
+  p.tile_tokens = desc->tile_tokens;
+  p.num_ctas = desc->num_ctas;
+  p.max_segments = desc->max_segments;
+  p.kind = desc->kind;
+  p.capacity_tokens = (int64_t)prob->max_pages_per_req * prob->page_size;
+  p.scale_log2 = prob->scale * 1.4426950408889634f;
+  cudaError_t e = da::launch_decode(p, prob->head_dim, maps, static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? DA_OK : cuda_fail(e);
+}
+
+DA_API int da_combine(const da_problem* prob, const da_plan_desc* desc, const void* ws, const float* partial_o,
+                      const float* partial_lse, void* out, float* lse, void* stream) {
+  int rc = check_problem(prob);
+  if (rc != DA_OK) return rc;
+  rc = check_desc(prob, desc);
+  if (rc != DA_OK) return rc;
+  if (prob->batch == 0) return DA_OK;
+  if (!ws || !partial_o || !partial_lse || !out || !lse) return DA_ERR_INVALID_ARG;
+  if (reinterpret_cast<uintptr_t>(partial_o) % 16 != 0 || reinterpret_cast<uintptr_t>(out) % 8 != 0)
+    return DA_ERR_INVALID_ARG;
+  da::CombineParams p;
+  p.ws = static_cast<const int32_t*>(ws);
+  p.partial_o = partial_o;
+  p.partial_lse = partial_lse;
+  p.out = static_cast<__nv_bfloat16*>(out);
+  p.lse = lse;
+  p.batch = prob->batch;
+  p.num_q_heads = prob->num_q_heads;
+  p.num_ctas = desc->num_ctas;
+  p.max_segments = desc->max_segments;
+  cudaError_t e = da::launch_combine(p, prob->head_dim, static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? DA_OK : cuda_fail(e);
+}
+
+DA_API int da_read_status(const void* ws, int32_t* dev_status, int32_t* bad_index, void* stream) {
+  if (!ws) return DA_ERR_INVALID_ARG;
+  int32_t h[da::kHdrWords];
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  cudaError_t e = cudaMemcpyAsync(h, ws, sizeof h, cudaMemcpyDeviceToHost, s);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(s);
+  if (e != cudaSuccess) return cuda_fail(e);
+  if (dev_status) *dev_status = h[da::kHdrStatus];
+  if (bad_index) *bad_index = h[da::kHdrBadIndex];
+  return DA_OK;
+}
+
+DA_API const char* da_status_string(int32_t code) {
+  switch (code) {
+    case DA_OK: return "ok";
+    case DA_ERR_INVALID_ARG: return "invalid argument";
+    case DA_ERR_UNSUPPORTED: return "unsupported problem shape";
+    case DA_ERR_CUDA: return "CUDA runtime error";
+    case DA_ERR_WORKSPACE: return "workspace too small";
+    default: return "unknown return code";
+  }
+}
+
+DA_API const char* da_dev_status_string(int32_t code) {
+  switch (code) {
+    case DA_DEV_OK: return "ok";
+    case DA_DEV_BAD_SEQLEN: return "sequence length out of range";
+    case DA_DEV_BAD_PAGE: return "block-table page id out of range";
+    case DA_DEV_TIMEOUT: return "pipeline wait timed out";
+    case DA_DEV_BAD_PLAN: return "workspace plan does not match the descriptor";
+    default: return "unknown device status";
+  }
+}
+
+}  // extern "C"

@@ -1,0 +1,219 @@
+// da_internal.cuh -- shared pieces of libda.so: workspace layout, kernel
+// parameter blocks, and thin inline-PTX wrappers for the sm_100a features the
+// kernels use (mbarrier, TMA tensor loads, ldmatrix, bf16 mma).
+#pragma once
+
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "da.h"
+
+namespace da {
+
+// ---- workspace layout (int32 words) ------------------------------------------------------
+enum HeaderWord {
+  kHdrUnits = 0,
+  kHdrSegments = 1,
+  kHdrCtas = 2,
+  kHdrTile = 3,
+  kHdrStatus = 4,
+  kHdrBadIndex = 5,
+  kHdrKind = 6,
+  kHdrBatch = 7,
+  kHdrMaxSegments = 8,
+  kHdrSplits = 9,
+  kHdrWords = 16,
+};
+
+struct WsLayout {
+  int64_t hdr, segs, req_tile_prefix, req_seg_begin, cta_seg_begin, total;
+};
+
+__host__ __device__ inline WsLayout ws_layout(int64_t batch, int64_t num_ctas, int64_t max_segments) {
+  WsLayout L;
+  L.hdr = 0;
+  L.segs = kHdrWords;                       // int4 per segment, 64-byte aligned start
+  L.req_tile_prefix = L.segs + 4 * max_segments;
+  L.req_seg_begin = L.req_tile_prefix + batch + 1;
+  L.cta_seg_begin = L.req_seg_begin + batch + 1;
+  L.total = (L.cta_seg_begin + num_ctas + 1 + 3) / 4 * 4;
+  return L;
+}
+
+// Record the first device-side data error (status word, then the offending index).
+__device__ inline void record_status(int32_t* hdr, int32_t code, int32_t index) {
+  if (atomicCAS(&hdr[kHdrStatus], DA_DEV_OK, code) == DA_DEV_OK) atomicExch(&hdr[kHdrBadIndex], index);
+}
+
+// ---- kernel parameter blocks -------------------------------------------------------------
+struct PlanParams {
+  const int32_t* seq_lens;
+  int32_t* ws;
+  int32_t batch, tile_tokens, width, max_segments, num_ctas;
+  int64_t capacity_tokens;
+};
+
+struct DecodeParams {
+  const __nv_bfloat16* q;
+  const int32_t* block_table;
+  const int32_t* seq_lens;
+  const int32_t* ws;
+  float* partial_o;
+  float* partial_lse;
+  __nv_bfloat16* out;
+  float* lse;
+  int32_t batch, num_q_heads, num_kv_heads, group, page_size, max_pages_per_req, num_pages;
+  int32_t tile_tokens, num_ctas, max_segments, kind;
+  int64_t capacity_tokens;
+  float scale_log2;  // scale * log2(e): scores are kept in base-2 units
+};
+
+struct CombineParams {
+  const int32_t* ws;
+  const float* partial_o;
+  const float* partial_lse;
+  __nv_bfloat16* out;
+  float* lse;
+  int32_t batch, num_q_heads, num_ctas, max_segments;
+};
+
+// Host launchers (defined next to their kernels).
+cudaError_t launch_plan_dynamic(const PlanParams& p, cudaStream_t stream);
+cudaError_t launch_plan_static(const PlanParams& p, cudaStream_t stream);
+cudaError_t launch_decode(const DecodeParams& p, int head_dim, const CUtensorMap maps[4], cudaStream_t stream);
+cudaError_t launch_combine(const CombineParams& p, int head_dim, cudaStream_t stream);
+
+// ---- inline PTX ----------------------------------------------------------------------------
+__device__ __forceinline__ uint32_t smem_u32(const void* p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+__device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count) : "memory");
+}
+
+__device__ __forceinline__ void fence_mbar_init() {
+  asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive(uint32_t bar) {
+  asm volatile("mbarrier.arrive.release.cta.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint32_t bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.release.cta.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes)
+               : "memory");
+}
+
+__device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
+  uint32_t done;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.acquire.cta.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(done)
+      : "r"(bar), "r"(parity)
+      : "memory");
+  return done != 0;
+}
+
+__device__ __forceinline__ uint64_t global_timer_ns() {
+  uint64_t t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
+
+// Bounded wait on an mbarrier phase.  Gives up (returns false) when *abort is
+// set by another warp or after `limit_ns` of wall time, so no wait can spin
+// forever.
+__device__ __forceinline__ bool mbar_wait_bounded(uint32_t bar, uint32_t parity, volatile int* abort,
+                                                  uint64_t limit_ns) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = global_timer_ns();
+  for (uint32_t it = 1;; ++it) {
+    if (mbar_try_wait(bar, parity)) return true;
+    if ((it & 63) == 0) {
+      if (*abort) return false;
+      if (global_timer_ns() - t0 > limit_ns) return false;
+    }
+  }
+}
+
+__device__ __forceinline__ void fence_proxy_async_smem() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+__device__ __forceinline__ void prefetch_tensormap(const CUtensorMap* m) {
+  asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(m)) : "memory");
+}
+
+// 2-D tiled TMA load global -> shared, completion counted on `bar` in bytes.
+__device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map, int32_t x, int32_t y,
+                                            uint32_t bar, uint64_t policy) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes.L2::cache_hint"
+      " [%0], [%1, {%2, %3}], [%4], %5;" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(bar), "l"(policy)
+      : "memory");
+}
+
+__device__ __forceinline__ uint64_t policy_evict_first() {
+  uint64_t p;
+  asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(p));
+  return p;
+}
+
+__device__ __forceinline__ void ldmatrix_x4(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2, uint32_t& r3) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0, %1, %2, %3}, [%4];"
+               : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
+               : "r"(addr));
+}
+
+__device__ __forceinline__ void ldmatrix_x4_trans(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2,
+                                                  uint32_t& r3) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0, %1, %2, %3}, [%4];"
+               : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
+               : "r"(addr));
+}
+
+// D = A(16x16 bf16, row) * B(16x8 bf16, col) + C, fp32 accumulate.  Only the
+// upper 8 rows of A are used here (a1 = a3 = 0), so only d0, d1 are kept.
+__device__ __forceinline__ void mma_bf16_upper(float& d0, float& d1, uint32_t a0, uint32_t a2, uint32_t b0,
+                                               uint32_t b1) {
+  float d2 = 0.f, d3 = 0.f;  // rows 8..15 of the tile: A is zero there
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, "
+      "{%0, %1, %2, %3};"
+      : "+f"(d0), "+f"(d1), "+f"(d2), "+f"(d3)
+      : "r"(a0), "r"(0u), "r"(a2), "r"(0u), "r"(b0), "r"(b1));
+}
+
+__device__ __forceinline__ float fast_exp2(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
+__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
+  uint32_t r;
+  asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
+  return r;
+}
+
+__device__ __forceinline__ float bf16_lo_to_f32(uint32_t v) { return __uint_as_float(v << 16); }
+__device__ __forceinline__ float bf16_hi_to_f32(uint32_t v) { return __uint_as_float(v & 0xFFFF0000u); }
+
+__device__ __forceinline__ void named_barrier_sync(int id, int threads) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(threads) : "memory");
+}
+
+// Programmatic dependent launch: wait for the previous kernel in the stream
+// (no-op when the launch did not opt in).
+__device__ __forceinline__ void grid_dependency_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void grid_dependents_launch() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
+}  // namespace da

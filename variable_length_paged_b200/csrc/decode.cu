@@ -1,0 +1,442 @@
+// decode.cu -- split-KV decode attention over a paged KV cache, sm_100a.
+//
+// "Tencent HPC lands in SGLang, challenging default inference kernels",
+// section "Why Tencent HPC matters for online model serving": attention over
+// each request's KV cache, with the cache work cut into uniform tiles that
+// CTAs take from a plan rebuilt every step; a longer history means more
+// cached data to read, so this kernel is bound by HBM reads of K and V.
+//
+// Grid (C, Hkv): CTA (c, g) walks the segments the plan gave CTA c, for KV
+// head g.  Block = 4 consumer warps + 1 producer warp.
+//
+//   producer  One lane issues TMA tensor loads (128-byte swizzle) of 64-token
+//             K and V chunks into a ring of shared-memory stages, each stage
+//             guarded by a "full" mbarrier (transaction bytes) and an "empty"
+//             mbarrier (one arrival per consumer warp).  Page ids come from the
+//             block table 32 at a time, one per lane.
+//   consumers Warp w owns tokens [16w, 16w+16) of each chunk and keeps its own
+//             online-softmax state for all G query heads of the group:
+//               S^T block: S = Q . K^T with mma.m16n8k16 (rows = heads, the
+//               upper 8 of the 16 MMA rows; n = tokens; k = head_dim), K read
+//               with ldmatrix from the swizzled tile;
+//               running max m, running sum l, fp32 accumulator O += P . V with
+//               P rounded to bf16 in registers and V read with ldmatrix.trans.
+//             At the end of a segment the four warp states are merged by
+//             log-sum-exp through shared memory; the result goes to out/lse
+//             (request with one segment) or to the segment's partial slot.
+//
+// Scores are kept in base-2 units (scale * log2 e), so exp is one ex2 and the
+// natural-log lse is (m + log2 l) * ln 2.  Tokens past the end of a request
+// inside a loaded chunk are masked to -inf; their V rows are zeroed in shared
+// memory first, since unused cache slots may hold anything (NaN included).
+#include <cfloat>
+
+#include "da_internal.cuh"
+
+namespace da {
+namespace {
+
+constexpr int kChunk = 64;            // tokens per pipeline stage
+constexpr int kConsumerWarps = 4;
+constexpr int kThreads = (kConsumerWarps + 1) * 32;
+constexpr uint64_t kWaitLimitNs = 2000000000ull;  // 2 s: far beyond any legitimate wait
+
+template <int D>
+struct Cfg {
+  static constexpr int kHalves = D / 64;                 // 128-byte column blocks per row
+  static constexpr int kTileBytes = kHalves * kChunk * 128;  // one K (or V) chunk
+  static constexpr int kStageBytes = 2 * kTileBytes;
+  static constexpr int kStages = D == 128 ? 3 : 6;
+  static constexpr int kSlotStride = D + 8;              // floats per head row in a merge slot
+  static constexpr int kSlotFloats = 8 * kSlotStride;
+  // shared memory map (offsets from a 1024-byte aligned base)
+  static constexpr int kOffStages = 0;
+  static constexpr int kOffSlots = kStages * kStageBytes;
+  static constexpr int kOffML = kOffSlots + 3 * kSlotFloats * 4;        // [3][2][8] floats
+  static constexpr int kOffBars = kOffML + 3 * 2 * 8 * 4;                // full[kStages], empty[kStages]
+  static constexpr int kOffMeta = kOffBars + 2 * kStages * 8;            // int per stage
+  static constexpr int kOffAbort = kOffMeta + kStages * 4;
+  static constexpr int kBytes = kOffAbort + 16;
+  static constexpr int kSmemRequest = kBytes + 1024;                     // slack for manual alignment
+};
+
+// Byte offset of (row, 16-byte column chunk) inside a TMA tile written with
+// 128-byte swizzle: the chunk index is XORed with row % 8 inside each 128-byte row.
+__device__ __forceinline__ uint32_t swz(int row, int chunk) {
+  return (uint32_t)((chunk >> 3) * (kChunk * 128) + row * 128 + (((chunk & 7) ^ (row & 7)) << 4));
+}
+
+struct SegmentInfo {
+  int b, tok0, tok1;
+  bool valid;
+};
+
+// Same decoding of a segment on the producer and consumer side, so both walk
+// the same chunks.
+__device__ __forceinline__ SegmentInfo load_segment(const DecodeParams& p, const int4* segs, int s) {
+  const int4 sg = segs[s];
+  SegmentInfo r;
+  r.b = sg.x;
+  r.valid = sg.x >= 0 && sg.x < p.batch && sg.z >= 0 && sg.w >= sg.z;
+  int L = r.valid ? p.seq_lens[sg.x] : 0;
+  if (L < 0 || (int64_t)L > p.capacity_tokens) L = 0;
+  const int64_t t0 = (int64_t)sg.z * p.tile_tokens, t1 = min((int64_t)sg.w * p.tile_tokens, (int64_t)L);
+  r.tok0 = (int)min(t0, (int64_t)L);
+  r.tok1 = (int)t1;
+  return r;
+}
+
+template <int D>
+__global__ void __launch_bounds__(kThreads, 2)
+    decode_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap k64,
+                  const __grid_constant__ CUtensorMap v64, const __grid_constant__ CUtensorMap k16,
+                  const __grid_constant__ CUtensorMap v16) {
+  using C = Cfg<D>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const uint32_t sbase = smem_u32(smem);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int cta = blockIdx.x, g = blockIdx.y;
+
+  grid_dependency_wait();  // the plan is written by the previous kernel in the stream
+
+  const WsLayout WL = ws_layout(p.batch, p.num_ctas, p.max_segments);
+  const int32_t* hdr = p.ws + WL.hdr;
+  const int4* segs = reinterpret_cast<const int4*>(p.ws + WL.segs);
+  const int32_t* rsb = p.ws + WL.req_seg_begin;
+  const int32_t* csb = p.ws + WL.cta_seg_begin;
+  int32_t* hdr_w = const_cast<int32_t*>(hdr);
+
+  // The plan must match the descriptor this launch was given.
+  if (hdr[kHdrCtas] != p.num_ctas || hdr[kHdrBatch] != p.batch || hdr[kHdrMaxSegments] != p.max_segments ||
+      hdr[kHdrKind] != p.kind) {
+    if (threadIdx.x == 0 && cta == 0 && g == 0) record_status(hdr_w, DA_DEV_BAD_PLAN, 0);
+    return;
+  }
+  const int nseg_total = min(hdr[kHdrSegments], p.max_segments);
+  const int seg_lo = csb[cta], seg_hi = min(csb[cta + 1], nseg_total);
+  if (seg_lo < 0 || seg_lo >= seg_hi) return;  // nothing planned for this CTA (uniform over the block)
+
+  uint32_t* bars = reinterpret_cast<uint32_t*>(smem + C::kOffBars);
+  const uint32_t full0 = sbase + C::kOffBars, empty0 = full0 + C::kStages * 8;
+  volatile int* meta = reinterpret_cast<volatile int*>(smem + C::kOffMeta);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::kOffAbort);
+  (void)bars;
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < C::kStages; ++s) {
+      mbar_init(full0 + 8 * s, 1);
+      mbar_init(empty0 + 8 * s, kConsumerWarps);
+    }
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  __syncthreads();
+
+  if (warp == kConsumerWarps) {
+    // ------------------------------------------------------------------ producer warp
+    if (lane == 0) {
+      prefetch_tensormap(&k64);
+      prefetch_tensormap(&v64);
+      prefetch_tensormap(&k16);
+      prefetch_tensormap(&v16);
+    }
+    const uint64_t policy = policy_evict_first();
+    const int P = p.page_size;
+    int stage = 0;
+    uint32_t phase = 0;
+    int fills = 0;
+    bool aborted = false;
+    for (int s = seg_lo; s < seg_hi && !aborted; ++s) {
+      const SegmentInfo si = load_segment(p, segs, s);
+      if (!si.valid) continue;
+      const int32_t* bt_row = p.block_table + (int64_t)si.b * p.max_pages_per_req;
+      int win_base = INT_MIN / 2, win_val = -1;
+      for (int c0 = si.tok0; c0 < si.tok1; c0 += kChunk) {
+        const int n = min(kChunk, si.tok1 - c0);
+        const int lp_first = c0 / P, lp_last = (c0 + n - 1) / P;
+        if (lp_first < win_base || lp_last >= win_base + 32) {
+          win_base = lp_first;
+          const int lp = win_base + lane;
+          win_val = lp < p.max_pages_per_req ? __ldg(bt_row + lp) : -1;
+        }
+        const bool fast = (c0 % P) + kChunk <= P;  // the whole chunk sits in one page
+        const int pieces = fast ? 1 : (n + 15) >> 4;
+        int pid[4];
+        bool ok = true;
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const int lp = (c0 + 16 * i) / P;
+          pid[i] = __shfl_sync(0xffffffffu, win_val, (lp - win_base) & 31);
+          if (i < pieces) ok = ok && pid[i] >= 0 && pid[i] < p.num_pages;
+        }
+        // wait until the consumers have released this stage
+        bool got = true;
+        if (lane == 0) got = mbar_wait_bounded(empty0 + 8 * stage, phase ^ 1, abort_flag, kWaitLimitNs);
+        got = __shfl_sync(0xffffffffu, got, 0);
+        if (!got) {
+          if (lane == 0) {
+            if (!*abort_flag) record_status(hdr_w, DA_DEV_TIMEOUT, s);
+            *abort_flag = 1;
+          }
+          aborted = true;
+          break;
+        }
+        if (lane == 0) {
+          if (!ok) record_status(hdr_w, DA_DEV_BAD_PAGE, si.b);
+          meta[stage] = ok ? n : 0;
+          const uint32_t bytes = !ok ? 0u : fast ? (uint32_t)C::kStageBytes : (uint32_t)(pieces * C::kHalves * 2048 * 2);
+          const uint32_t full = full0 + 8 * stage;
+          mbar_arrive_expect_tx(full, bytes);
+          if (ok) {
+            const uint32_t sk = sbase + C::kOffStages + stage * C::kStageBytes, sv = sk + C::kTileBytes;
+            if (fast) {
+              const int row = (pid[0] * p.num_kv_heads + g) * P + c0 % P;
+#pragma unroll
+              for (int h = 0; h < C::kHalves; ++h) {
+                tma_load_2d(sk + h * kChunk * 128, &k64, h * 64, row, full, policy);
+                tma_load_2d(sv + h * kChunk * 128, &v64, h * 64, row, full, policy);
+              }
+            } else {
+#pragma unroll
+              for (int i = 0; i < 4; ++i) {
+                if (i >= pieces) break;
+                const int row = (pid[i] * p.num_kv_heads + g) * P + (c0 + 16 * i) % P;
+#pragma unroll
+                for (int h = 0; h < C::kHalves; ++h) {
+                  tma_load_2d(sk + h * kChunk * 128 + i * 2048, &k16, h * 64, row, full, policy);
+                  tma_load_2d(sv + h * kChunk * 128 + i * 2048, &v16, h * 64, row, full, policy);
+                }
+              }
+            }
+          }
+        }
+        __syncwarp();
+        ++fills;
+        if (++stage == C::kStages) {
+          stage = 0;
+          phase ^= 1;
+        }
+      }
+    }
+    // Drain: every stage's last fill must have landed before the CTA may exit.
+    if (lane == 0) {
+      for (int k = max(0, fills - C::kStages); k < fills; ++k)
+        mbar_wait_bounded(full0 + 8 * (k % C::kStages), (k / C::kStages) & 1, abort_flag, kWaitLimitNs);
+    }
+    return;
+  }
+
+  // -------------------------------------------------------------------- consumer warps
+  const int w = warp;
+  const int r = lane >> 2;   // query head within the group (MMA row)
+  const int tq = lane & 3;   // thread within the quad
+  const bool row_live = r < p.group;
+  float* slots = reinterpret_cast<float*>(smem + C::kOffSlots);
+  float* ml = reinterpret_cast<float*>(smem + C::kOffML);
+  int stage = 0;
+  uint32_t phase = 0;
+
+  // ldmatrix row addresses that do not depend on the chunk: lane i feeds row i%8
+  // of matrix i/8.
+  const int mat = lane >> 3, mrow = lane & 7;
+  const int k_tok = 16 * w + (mat >> 1) * 8 + mrow;  // S: matrices (tok 0-7, c), (tok 0-7, c+1), (tok 8-15, c), (tok 8-15, c+1)
+  const int k_chk = mat & 1;
+  const int v_tok = 16 * w + (mat & 1) * 8 + mrow;   // PV: matrices (tok 0-7, c), (tok 8-15, c), (tok 0-7, c+1), (tok 8-15, c+1)
+  const int v_chk = mat >> 1;
+
+  for (int s = seg_lo; s < seg_hi; ++s) {
+    const SegmentInfo si = load_segment(p, segs, s);
+    if (!si.valid) continue;
+    const int b = si.b;
+
+    // Q fragments for rows r (upper half of the MMA tile); rows >= G are zero.
+    uint32_t qlo[D / 16], qhi[D / 16];
+    {
+      const uint32_t* qrow = reinterpret_cast<const uint32_t*>(
+          p.q + ((int64_t)b * p.num_q_heads + (int64_t)g * p.group + (row_live ? r : 0)) * D);
+#pragma unroll
+      for (int kk = 0; kk < D / 16; ++kk) {
+        qlo[kk] = row_live ? __ldg(qrow + kk * 8 + tq) : 0u;
+        qhi[kk] = row_live ? __ldg(qrow + kk * 8 + 4 + tq) : 0u;
+      }
+    }
+    float m = -INFINITY, l = 0.f;
+    float o[D / 8][2];
+#pragma unroll
+    for (int i = 0; i < D / 8; ++i) o[i][0] = o[i][1] = 0.f;
+
+    for (int c0 = si.tok0; c0 < si.tok1; c0 += kChunk) {
+      const bool got = mbar_wait_bounded(full0 + 8 * stage, phase, abort_flag, kWaitLimitNs);
+      if (!got && lane == 0) {
+        if (!*abort_flag) record_status(hdr_w, DA_DEV_TIMEOUT, s);
+        *abort_flag = 1;
+      }
+      const int n = got ? meta[stage] : 0;
+      const int nw = min(max(n - 16 * w, 0), 16);  // valid tokens in this warp's 16 rows
+      const uint32_t sk = sbase + C::kOffStages + stage * C::kStageBytes, sv = sk + C::kTileBytes;
+      if (nw > 0) {
+        if (nw < 16) {
+          // zero V rows [nw, 16) of this warp's piece: stale or unused slots must not reach P.V
+          uint8_t* vrows = smem + C::kOffStages + stage * C::kStageBytes + C::kTileBytes;
+          for (int i = lane; i < (16 - nw) * C::kHalves * 8; i += 32) {
+            const int row = 16 * w + nw + i / (C::kHalves * 8);
+            const int rem = i % (C::kHalves * 8);
+            const int half = rem >> 3, chunk16 = rem & 7;
+            *reinterpret_cast<uint4*>(vrows + half * kChunk * 128 + row * 128 + chunk16 * 16) = make_uint4(0, 0, 0, 0);
+          }
+          fence_proxy_async_smem();
+          __syncwarp();
+        }
+        // S = Q . K^T for this warp's 16 tokens (two n-tiles of 8)
+        float sc[2][2] = {{0.f, 0.f}, {0.f, 0.f}};
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          uint32_t b0, b1, b2, b3;
+          ldmatrix_x4(sk + swz(k_tok, 2 * kk + k_chk), b0, b1, b2, b3);
+          mma_bf16_upper(sc[0][0], sc[0][1], qlo[kk], qhi[kk], b0, b1);
+          mma_bf16_upper(sc[1][0], sc[1][1], qlo[kk], qhi[kk], b2, b3);
+        }
+        // mask, scale to base 2, online softmax update
+        float x[2][2];
+        float mx = -INFINITY;
+#pragma unroll
+        for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+          for (int e = 0; e < 2; ++e) {
+            const int tok = 8 * nt + 2 * tq + e;
+            x[nt][e] = tok < nw ? sc[nt][e] * p.scale_log2 : -INFINITY;
+            mx = fmaxf(mx, x[nt][e]);
+          }
+        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
+        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
+        const float m_new = fmaxf(m, mx);
+        const float m_use = m_new == -INFINITY ? 0.f : m_new;
+        const float corr = fast_exp2(m - m_use);
+        const uint32_t pa0 = pack_bf16x2(fast_exp2(x[0][0] - m_use), fast_exp2(x[0][1] - m_use));
+        const uint32_t pa1 = pack_bf16x2(fast_exp2(x[1][0] - m_use), fast_exp2(x[1][1] - m_use));
+        l = l * corr + (bf16_lo_to_f32(pa0) + bf16_hi_to_f32(pa0)) + (bf16_lo_to_f32(pa1) + bf16_hi_to_f32(pa1));
+        m = m_new;
+#pragma unroll
+        for (int i = 0; i < D / 8; ++i) {
+          o[i][0] *= corr;
+          o[i][1] *= corr;
+        }
+        // O += P . V
+#pragma unroll
+        for (int np = 0; np < D / 16; ++np) {
+          uint32_t v0, v1, v2, v3;
+          ldmatrix_x4_trans(sv + swz(v_tok, 2 * np + v_chk), v0, v1, v2, v3);
+          mma_bf16_upper(o[2 * np][0], o[2 * np][1], pa0, pa1, v0, v1);
+          mma_bf16_upper(o[2 * np + 1][0], o[2 * np + 1][1], pa0, pa1, v2, v3);
+        }
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(empty0 + 8 * stage);
+      if (++stage == C::kStages) {
+        stage = 0;
+        phase ^= 1;
+      }
+    }
+
+    // ---- merge the four warp states of this segment
+    l += __shfl_xor_sync(0xffffffffu, l, 1);
+    l += __shfl_xor_sync(0xffffffffu, l, 2);
+    if (w > 0) {
+      float* slot = slots + (w - 1) * C::kSlotFloats + r * C::kSlotStride + 2 * tq;
+#pragma unroll
+      for (int i = 0; i < D / 8; ++i) *reinterpret_cast<float2*>(slot + 8 * i) = make_float2(o[i][0], o[i][1]);
+      if (tq == 0) {
+        ml[(w - 1) * 16 + r] = m;
+        ml[(w - 1) * 16 + 8 + r] = l;
+      }
+    }
+    named_barrier_sync(1, kConsumerWarps * 32);
+    if (w == 0) {
+      float mw[3], lw[3];
+      float M = m;
+#pragma unroll
+      for (int j = 0; j < 3; ++j) {
+        mw[j] = ml[j * 16 + r];
+        lw[j] = ml[j * 16 + 8 + r];
+        M = fmaxf(M, mw[j]);
+      }
+      const bool empty = M == -INFINITY;
+      const float f0 = empty ? 0.f : fast_exp2(m - M);
+      float fw[3];
+      float Lsum = f0 * l;
+#pragma unroll
+      for (int j = 0; j < 3; ++j) {
+        fw[j] = empty ? 0.f : fast_exp2(mw[j] - M);
+        Lsum += fw[j] * lw[j];
+      }
+      const float inv = Lsum > 0.f ? 1.f / Lsum : 0.f;
+      const float lse_nat = Lsum > 0.f ? (M + log2f(Lsum)) * 0.69314718055994530942f : -INFINITY;
+      const int h = g * p.group + r;
+      const int nseg_b = rsb[b + 1] - rsb[b];
+      const bool direct = nseg_b == 1;
+#pragma unroll
+      for (int i = 0; i < D / 8; ++i) {
+        float a0 = f0 * o[i][0], a1 = f0 * o[i][1];
+#pragma unroll
+        for (int j = 0; j < 3; ++j) {
+          const float2 v = *reinterpret_cast<const float2*>(slots + j * C::kSlotFloats + r * C::kSlotStride + 8 * i + 2 * tq);
+          a0 += fw[j] * v.x;
+          a1 += fw[j] * v.y;
+        }
+        o[i][0] = a0 * inv;
+        o[i][1] = a1 * inv;
+      }
+      if (row_live) {
+        if (direct) {
+          uint32_t* dst = reinterpret_cast<uint32_t*>(p.out + ((int64_t)b * p.num_q_heads + h) * D + 2 * tq);
+#pragma unroll
+          for (int i = 0; i < D / 8; ++i) dst[4 * i] = pack_bf16x2(o[i][0], o[i][1]);
+          if (tq == 0) p.lse[(int64_t)b * p.num_q_heads + h] = lse_nat;
+        } else {
+          float* dst = p.partial_o + ((int64_t)s * p.num_q_heads + h) * D + 2 * tq;
+#pragma unroll
+          for (int i = 0; i < D / 8; ++i) *reinterpret_cast<float2*>(dst + 8 * i) = make_float2(o[i][0], o[i][1]);
+          if (tq == 0) p.partial_lse[(int64_t)s * p.num_q_heads + h] = lse_nat;
+        }
+      }
+    }
+    named_barrier_sync(1, kConsumerWarps * 32);  // slots are free again
+  }
+}
+
+template <int D>
+cudaError_t launch_decode_d(const DecodeParams& p, const CUtensorMap maps[4], cudaStream_t stream) {
+  using C = Cfg<D>;
+  static_assert(C::kSmemRequest * 2 <= 227 * 1024, "two CTAs per SM must fit");
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  static bool configured[64] = {false};
+  if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+  if (!configured[dev]) {
+    e = cudaFuncSetAttribute(decode_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemRequest);
+    if (e != cudaSuccess) return e;
+    configured[dev] = true;
+  }
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)p.num_ctas, (unsigned)p.num_kv_heads, 1);
+  cfg.blockDim = dim3(kThreads, 1, 1);
+  cfg.dynamicSmemBytes = C::kSmemRequest;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, decode_kernel<D>, p, maps[0], maps[1], maps[2], maps[3]);
+}
+
+}  // namespace
+
+cudaError_t launch_decode(const DecodeParams& p, int head_dim, const CUtensorMap maps[4], cudaStream_t stream) {
+  if (head_dim == 128) return launch_decode_d<128>(p, maps, stream);
+  if (head_dim == 64) return launch_decode_d<64>(p, maps, stream);
+  return cudaErrorInvalidValue;
+}
+
+}  // namespace da

@@ -1,0 +1,214 @@
+// plan.cu -- on-device work planners, rebuilt every decode step from seq_lens.
+//
+// "Tencent HPC lands in SGLang, challenging default inference kernels",
+// section "Why Tencent HPC matters for online model serving": the KV-cache
+// work is cut into uniform tiles and handed to CTAs by the current workload,
+// and the mapping is rebuilt as request lengths change; the comparator is a
+// static split-k schedule that idles units or launches empty chunks.
+//
+// Both planners run as one 1024-thread CTA and write the same work list:
+// segments {request, cta, tile_begin, tile_end} in global tile order, the
+// per-request and per-CTA segment ranges, and a header.  Everything is integer
+// arithmetic, so the result is bit-exact and independent of thread timing.
+#include <climits>
+
+#include "da_internal.cuh"
+
+namespace da {
+namespace {
+
+constexpr int kPlanThreads = 1024;
+
+// Exclusive block-wide scan of one value per thread; also returns the total.
+__device__ int block_exclusive_scan(int v, int* total, int* warp_buf) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  int x = v;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int y = __shfl_up_sync(0xffffffffu, x, o);
+    if (lane >= o) x += y;
+  }
+  if (lane == 31) warp_buf[warp] = x;
+  __syncthreads();
+  if (warp == 0) {
+    int w = warp_buf[lane];
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, w, o);
+      if (lane >= o) w += y;
+    }
+    warp_buf[lane] = w;  // inclusive warp totals
+  }
+  __syncthreads();
+  const int before = warp == 0 ? 0 : warp_buf[warp - 1];
+  *total = warp_buf[31];
+  __syncthreads();  // warp_buf may be reused by the next call
+  return before + x - v;
+}
+
+// Tile count of one request; an out-of-range length counts as 0 and is reported.
+__device__ int request_tiles(const PlanParams& p, int b, int* s_bad) {
+  const int L = p.seq_lens[b];
+  if (L < 0 || (int64_t)L > p.capacity_tokens) {
+    atomicMin(s_bad, b);
+    return 0;
+  }
+  return (int)(((int64_t)L + p.tile_tokens - 1) / p.tile_tokens);
+}
+
+// Phase shared by both planners: req_tile_prefix and U (and the largest n_b).
+__device__ void tile_prefix(const PlanParams& p, int32_t* rtp, int* warp_buf, int* s_bad, int* U, int* max_tiles) {
+  int carry = 0, mx = 0;
+  for (int base = 0; base < p.batch; base += kPlanThreads) {
+    const int b = base + threadIdx.x;
+    const int n = b < p.batch ? request_tiles(p, b, s_bad) : 0;
+    int total;
+    const int excl = block_exclusive_scan(n, &total, warp_buf);
+    if (b < p.batch) rtp[b + 1] = carry + excl + n;
+    carry += total;
+    mx = max(mx, n);
+  }
+  if (threadIdx.x == 0) rtp[0] = 0;
+  // block max of n
+  for (int o = 16; o > 0; o >>= 1) mx = max(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+  if ((threadIdx.x & 31) == 0) warp_buf[threadIdx.x >> 5] = mx;
+  __syncthreads();
+  if (threadIdx.x < 32) {
+    int w = warp_buf[threadIdx.x];
+    for (int o = 16; o > 0; o >>= 1) w = max(w, __shfl_xor_sync(0xffffffffu, w, o));
+    if (threadIdx.x == 0) warp_buf[0] = w;
+  }
+  __syncthreads();
+  *max_tiles = warp_buf[0];
+  *U = carry;
+  __syncthreads();
+}
+
+__device__ void write_header(const PlanParams& p, int32_t* hdr, int U, int S, int kind, int splits, int bad) {
+  hdr[kHdrUnits] = U;
+  hdr[kHdrSegments] = S;
+  hdr[kHdrCtas] = p.num_ctas;
+  hdr[kHdrTile] = p.tile_tokens;
+  hdr[kHdrStatus] = bad == INT_MAX ? DA_DEV_OK : DA_DEV_BAD_SEQLEN;
+  hdr[kHdrBadIndex] = bad == INT_MAX ? -1 : bad;
+  hdr[kHdrKind] = kind;
+  hdr[kHdrBatch] = p.batch;
+  hdr[kHdrMaxSegments] = p.max_segments;
+  hdr[kHdrSplits] = splits;
+  for (int i = kHdrSplits + 1; i < kHdrWords; ++i) hdr[i] = 0;
+}
+
+// CTA that owns global tile u: the unique c with floor(c*U/C) <= u < floor((c+1)*U/C).
+__device__ __forceinline__ int owner_cta(int64_t u, int64_t U, int64_t C) { return (int)(((u + 1) * C - 1) / U); }
+__device__ __forceinline__ int64_t cta_first_unit(int64_t c, int64_t U, int64_t C) { return c * U / C; }
+
+__global__ void __launch_bounds__(kPlanThreads) plan_dynamic_kernel(const PlanParams p) {
+  __shared__ int warp_buf[32];
+  __shared__ int s_bad;
+  if (threadIdx.x == 0) s_bad = INT_MAX;
+  __syncthreads();
+
+  const WsLayout L = ws_layout(p.batch, p.num_ctas, p.max_segments);
+  int32_t* hdr = p.ws + L.hdr;
+  int4* segs = reinterpret_cast<int4*>(p.ws + L.segs);
+  int32_t* rtp = p.ws + L.req_tile_prefix;
+  int32_t* rsb = p.ws + L.req_seg_begin;
+  int32_t* csb = p.ws + L.cta_seg_begin;
+  const int64_t C = p.num_ctas;
+
+  int U, max_tiles;
+  tile_prefix(p, rtp, warp_buf, &s_bad, &U, &max_tiles);
+
+  // Segments per request.  With U >= C every CTA owns at least one tile, so a
+  // request spanning CTAs [cf, cl] has cl - cf + 1 segments.  With U < C each
+  // non-empty CTA owns exactly one tile, so every tile is its own segment.
+  const bool sparse = (int64_t)U < C;
+  int carry = 0;
+  for (int base = 0; base < p.batch; base += kPlanThreads) {
+    const int b = base + threadIdx.x;
+    int ns = 0;
+    if (b < p.batch) {
+      const int p0 = rtp[b], n = rtp[b + 1] - p0;
+      if (n > 0) ns = sparse ? n : owner_cta(p0 + n - 1, U, C) - owner_cta(p0, U, C) + 1;
+    }
+    int total;
+    const int excl = block_exclusive_scan(ns, &total, warp_buf);
+    if (b < p.batch) rsb[b + 1] = carry + excl + ns;
+    carry += total;
+  }
+  if (threadIdx.x == 0) rsb[0] = 0;
+  const int S = carry;
+  __syncthreads();
+
+  // Segments and the per-CTA segment ranges.
+  for (int b = threadIdx.x; b < p.batch; b += kPlanThreads) {
+    const int p0 = rtp[b], n = rtp[b + 1] - p0;
+    if (n == 0) continue;
+    const int s0 = rsb[b];
+    if (sparse) {
+      for (int j = 0; j < n; ++j) segs[s0 + j] = make_int4(b, owner_cta(p0 + j, U, C), j, j + 1);
+      continue;
+    }
+    const int cf = owner_cta(p0, U, C), cl = owner_cta(p0 + n - 1, U, C);
+    const int prev = p0 > 0 ? owner_cta(p0 - 1, U, C) : -1;
+    for (int c = prev + 1; c <= cf; ++c) csb[c] = s0;  // this segment opens CTA cf
+    for (int c = cf; c <= cl; ++c) {
+      const int64_t lo = max((int64_t)p0, cta_first_unit(c, U, C));
+      const int64_t hi = min((int64_t)p0 + n, cta_first_unit(c + 1, U, C));
+      const int s = s0 + (c - cf);
+      segs[s] = make_int4(b, c, (int)(lo - p0), (int)(hi - p0));
+      if (c > cf) csb[c] = s;
+    }
+  }
+  if (sparse) {
+    // every tile is a segment, so CTA c starts at segment floor(c*U/C)
+    for (int c = threadIdx.x; c <= p.num_ctas; c += kPlanThreads) csb[c] = (int)cta_first_unit(c, U, C);
+  } else {
+    const int last = owner_cta((int64_t)U - 1, U, C);
+    for (int c = last + 1 + threadIdx.x; c <= p.num_ctas; c += kPlanThreads) csb[c] = S;
+  }
+  if (threadIdx.x == 0) write_header(p, hdr, U, S, DA_PLAN_DYNAMIC, 0, s_bad);
+}
+
+__global__ void __launch_bounds__(kPlanThreads) plan_static_kernel(const PlanParams p) {
+  __shared__ int warp_buf[32];
+  __shared__ int s_bad;
+  if (threadIdx.x == 0) s_bad = INT_MAX;
+  __syncthreads();
+
+  const WsLayout L = ws_layout(p.batch, p.num_ctas, p.max_segments);
+  int32_t* hdr = p.ws + L.hdr;
+  int4* segs = reinterpret_cast<int4*>(p.ws + L.segs);
+  int32_t* rtp = p.ws + L.req_tile_prefix;
+  int32_t* rsb = p.ws + L.req_seg_begin;
+  int32_t* csb = p.ws + L.cta_seg_begin;
+  const int S = p.width;
+
+  int U, max_tiles;
+  tile_prefix(p, rtp, warp_buf, &s_bad, &U, &max_tiles);
+  const int chunk = (max_tiles + S - 1) / S;
+  const int total = p.batch * S;
+  for (int i = threadIdx.x; i < total; i += kPlanThreads) {
+    const int b = i / S, s = i - b * S;
+    const int n = rtp[b + 1] - rtp[b];
+    const int64_t lo = min((int64_t)s * chunk, (int64_t)n), hi = min((int64_t)(s + 1) * chunk, (int64_t)n);
+    segs[i] = make_int4(b, i, (int)lo, (int)hi);
+  }
+  for (int b = threadIdx.x; b <= p.batch; b += kPlanThreads) rsb[b] = b * S;
+  for (int c = threadIdx.x; c <= total; c += kPlanThreads) csb[c] = c;
+  if (threadIdx.x == 0) write_header(p, hdr, U, total, DA_PLAN_STATIC, S, s_bad);
+}
+
+}  // namespace
+
+cudaError_t launch_plan_dynamic(const PlanParams& p, cudaStream_t stream) {
+  plan_dynamic_kernel<<<1, kPlanThreads, 0, stream>>>(p);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_plan_static(const PlanParams& p, cudaStream_t stream) {
+  plan_static_kernel<<<1, kPlanThreads, 0, stream>>>(p);
+  return cudaGetLastError();
+}
+
+}  // namespace da

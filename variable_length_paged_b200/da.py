@@ -1,0 +1,224 @@
+"""Thin ctypes binding of libda.so (C ABI in include/da.h).
+
+Functions keep the C names and only marshal arguments: torch tensors (device
+memory) become raw pointers, the current torch CUDA stream becomes the
+cudaStream_t.  Every step of the computation runs in the library's kernels;
+there is no Python or CPU fallback, and a missing library raises.
+"""
+
+from __future__ import annotations
+
+import ctypes
+import os
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(HERE, "libda.so")
+
+OK, ERR_INVALID_ARG, ERR_UNSUPPORTED, ERR_CUDA, ERR_WORKSPACE = 0, -1, -2, -3, -4
+DEV_OK, DEV_BAD_SEQLEN, DEV_BAD_PAGE, DEV_TIMEOUT, DEV_BAD_PLAN = 0, 1, 2, 3, 4
+PLAN_DYNAMIC, PLAN_STATIC = 0, 1
+
+# Every symbol include/da.h declares.
+EXPORTS = ("da_plan_desc_init", "da_workspace_size", "da_workspace_offsets", "da_plan", "da_static_plan",
+           "da_decode_attention", "da_combine", "da_read_status", "da_status_string", "da_dev_status_string",
+           "da_last_cuda_error", "da_device_num_sms")
+
+
+class DaProblem(ctypes.Structure):
+    _fields_ = [("batch", ctypes.c_int32), ("num_q_heads", ctypes.c_int32), ("num_kv_heads", ctypes.c_int32),
+                ("head_dim", ctypes.c_int32), ("page_size", ctypes.c_int32), ("max_pages_per_req", ctypes.c_int32),
+                ("num_pages", ctypes.c_int32), ("scale", ctypes.c_float)]
+
+
+class DaPlanDesc(ctypes.Structure):
+    _fields_ = [("kind", ctypes.c_int32), ("batch", ctypes.c_int32), ("tile_tokens", ctypes.c_int32),
+                ("num_ctas", ctypes.c_int32), ("splits", ctypes.c_int32), ("max_segments", ctypes.c_int32)]
+
+
+class DaError(RuntimeError):
+    def __init__(self, fn: str, code: int, cuda_error: int = 0):
+        self.code = code
+        self.cuda_error = cuda_error
+        msg = f"{fn} returned {code} ({status_string(code)})"
+        if code == ERR_CUDA:
+            msg += f", cudaError {cuda_error}"
+        super().__init__(msg)
+
+
+_lib = None
+_vp = ctypes.c_void_p
+_sz = ctypes.c_size_t
+
+
+def lib():
+    """Load libda.so (raises if it has not been built)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(f"libda.so not found at {LIB_PATH}; build it with "
+                               "`python -m variable_length_paged_b200.build`")
+        L = ctypes.CDLL(LIB_PATH)
+        P, D = ctypes.POINTER(DaProblem), ctypes.POINTER(DaPlanDesc)
+        sig = {
+            "da_plan_desc_init": [P, ctypes.c_int32, ctypes.c_int32, ctypes.c_int32, D],
+            "da_workspace_size": [P, D, ctypes.POINTER(_sz), ctypes.POINTER(_sz), ctypes.POINTER(_sz)],
+            "da_workspace_offsets": [D, ctypes.POINTER(ctypes.c_int64)],
+            "da_plan": [P, D, _vp, _vp, _sz, _vp],
+            "da_static_plan": [P, D, _vp, _vp, _sz, _vp],
+            "da_decode_attention": [P, D, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp],
+            "da_combine": [P, D, _vp, _vp, _vp, _vp, _vp, _vp],
+            "da_read_status": [_vp, ctypes.POINTER(ctypes.c_int32), ctypes.POINTER(ctypes.c_int32), _vp],
+            "da_last_cuda_error": [],
+            "da_device_num_sms": [ctypes.POINTER(ctypes.c_int32)],
+        }
+        for name, args in sig.items():
+            fn = getattr(L, name)
+            fn.argtypes = args
+            fn.restype = ctypes.c_int32
+        for name in ("da_status_string", "da_dev_status_string"):
+            fn = getattr(L, name)
+            fn.argtypes = [ctypes.c_int32]
+            fn.restype = ctypes.c_char_p
+        _lib = L
+    return _lib
+
+
+def status_string(code: int) -> str:
+    return lib().da_status_string(int(code)).decode()
+
+
+def dev_status_string(code: int) -> str:
+    return lib().da_dev_status_string(int(code)).decode()
+
+
+def _check(fn: str, rc: int):
+    if rc != OK:
+        raise DaError(fn, rc, lib().da_last_cuda_error() if rc == ERR_CUDA else 0)
+
+
+def problem(batch, num_q_heads, num_kv_heads, head_dim, page_size, max_pages_per_req, num_pages, scale) -> DaProblem:
+    return DaProblem(int(batch), int(num_q_heads), int(num_kv_heads), int(head_dim), int(page_size),
+                     int(max_pages_per_req), int(num_pages), float(scale))
+
+
+def problem_from(p) -> DaProblem:
+    """From any object with the da_problem field names (e.g. workloads.Problem)."""
+    return problem(p.batch, p.num_q_heads, p.num_kv_heads, p.head_dim, p.page_size, p.max_pages_per_req,
+                   p.num_pages, p.scale)
+
+
+def _ptr(t) -> int | None:
+    if t is None:
+        return None
+    if isinstance(t, int):
+        return t
+    return t.data_ptr()
+
+
+def _stream(stream) -> int | None:
+    if stream is None:
+        import torch
+        return torch.cuda.current_stream().cuda_stream
+    return stream if isinstance(stream, int) else stream.cuda_stream
+
+
+# ---- the C calls -------------------------------------------------------------------------------
+
+def da_plan_desc_init(prob: DaProblem, kind: int, tile_tokens: int = 0, width: int = 0) -> DaPlanDesc:
+    d = DaPlanDesc()
+    _check("da_plan_desc_init", lib().da_plan_desc_init(ctypes.byref(prob), int(kind), int(tile_tokens), int(width),
+                                                         ctypes.byref(d)))
+    return d
+
+
+def da_workspace_size(prob: DaProblem, desc: DaPlanDesc) -> tuple[int, int, int]:
+    a, b, c = _sz(), _sz(), _sz()
+    _check("da_workspace_size", lib().da_workspace_size(ctypes.byref(prob), ctypes.byref(desc), ctypes.byref(a),
+                                                         ctypes.byref(b), ctypes.byref(c)))
+    return a.value, b.value, c.value
+
+
+def da_workspace_offsets(desc: DaPlanDesc) -> list[int]:
+    off = (ctypes.c_int64 * 6)()
+    _check("da_workspace_offsets", lib().da_workspace_offsets(ctypes.byref(desc), off))
+    return list(off)
+
+
+def da_plan(prob, desc, seq_lens, ws, ws_bytes: int | None = None, stream=None):
+    nbytes = ws.numel() * ws.element_size() if ws_bytes is None else ws_bytes
+    _check("da_plan", lib().da_plan(ctypes.byref(prob), ctypes.byref(desc), _ptr(seq_lens), _ptr(ws), nbytes,
+                                    _stream(stream)))
+
+
+def da_static_plan(prob, desc, seq_lens, ws, ws_bytes: int | None = None, stream=None):
+    nbytes = ws.numel() * ws.element_size() if ws_bytes is None else ws_bytes
+    _check("da_static_plan", lib().da_static_plan(ctypes.byref(prob), ctypes.byref(desc), _ptr(seq_lens), _ptr(ws),
+                                                  nbytes, _stream(stream)))
+
+
+def da_decode_attention(prob, desc, q, k_cache, v_cache, block_table, seq_lens, ws, partial_o, partial_lse, out, lse,
+                        stream=None):
+    _check("da_decode_attention", lib().da_decode_attention(
+        ctypes.byref(prob), ctypes.byref(desc), _ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(block_table),
+        _ptr(seq_lens), _ptr(ws), _ptr(partial_o), _ptr(partial_lse), _ptr(out), _ptr(lse), _stream(stream)))
+
+
+def da_combine(prob, desc, ws, partial_o, partial_lse, out, lse, stream=None):
+    _check("da_combine", lib().da_combine(ctypes.byref(prob), ctypes.byref(desc), _ptr(ws), _ptr(partial_o),
+                                          _ptr(partial_lse), _ptr(out), _ptr(lse), _stream(stream)))
+
+
+def da_read_status(ws, stream=None) -> tuple[int, int]:
+    st, bad = ctypes.c_int32(), ctypes.c_int32()
+    _check("da_read_status", lib().da_read_status(_ptr(ws), ctypes.byref(st), ctypes.byref(bad), _stream(stream)))
+    return st.value, bad.value
+
+
+def da_device_num_sms() -> int:
+    n = ctypes.c_int32()
+    _check("da_device_num_sms", lib().da_device_num_sms(ctypes.byref(n)))
+    return n.value
+
+
+# ---- buffers and one whole step --------------------------------------------------------------------
+
+class Buffers:
+    """Device buffers for one plan descriptor: workspace, partials, outputs (allocated with torch)."""
+
+    def __init__(self, prob: DaProblem, desc: DaPlanDesc, device):
+        import torch
+        ws, po, pl = da_workspace_size(prob, desc)
+        self.ws = torch.zeros(max(ws // 4, 4), dtype=torch.int32, device=device)
+        self.partial_o = torch.empty(max(po // 4, 4), dtype=torch.float32, device=device)
+        self.partial_lse = torch.empty(max(pl // 4, 1), dtype=torch.float32, device=device)
+        self.out = torch.empty((prob.batch, prob.num_q_heads, prob.head_dim), dtype=torch.bfloat16, device=device)
+        self.lse = torch.empty((prob.batch, prob.num_q_heads), dtype=torch.float32, device=device)
+
+
+def decode_step(prob, desc, q, k_cache, v_cache, block_table, seq_lens, bufs: Buffers, stream=None):
+    """Plan (dynamic or static, per `desc.kind`) + decode + combine, asynchronously on `stream`."""
+    if desc.kind == PLAN_DYNAMIC:
+        da_plan(prob, desc, seq_lens, bufs.ws, stream=stream)
+    else:
+        da_static_plan(prob, desc, seq_lens, bufs.ws, stream=stream)
+    da_decode_attention(prob, desc, q, k_cache, v_cache, block_table, seq_lens, bufs.ws, bufs.partial_o,
+                        bufs.partial_lse, bufs.out, bufs.lse, stream=stream)
+    da_combine(prob, desc, bufs.ws, bufs.partial_o, bufs.partial_lse, bufs.out, bufs.lse, stream=stream)
+    return bufs.out, bufs.lse
+
+
+def read_plan(desc: DaPlanDesc, ws) -> dict:
+    """Copy a plan out of the workspace into numpy arrays (same keys as the oracle's plan)."""
+    import numpy as np
+    off = da_workspace_offsets(desc)
+    w = ws.detach().cpu().numpy().astype(np.int32)
+    hdr = w[off[0]:off[0] + 16]
+    S = int(hdr[1])
+    segs = w[off[1]:off[1] + 4 * desc.max_segments].reshape(-1, 4)[:S]
+    B, C = desc.batch, desc.num_ctas
+    return dict(num_units=int(hdr[0]), num_segments=S, num_ctas=int(hdr[2]), tile_tokens=int(hdr[3]),
+                status=int(hdr[4]), bad_index=int(hdr[5]), kind=int(hdr[6]), batch=int(hdr[7]),
+                max_segments=int(hdr[8]), splits=int(hdr[9]),
+                seg_req=segs[:, 0].copy(), seg_cta=segs[:, 1].copy(), seg_tile_begin=segs[:, 2].copy(),
+                seg_tile_end=segs[:, 3].copy(), req_tile_prefix=w[off[2]:off[2] + B + 1].copy(),
+                req_seg_begin=w[off[3]:off[3] + B + 1].copy(), cta_seg_begin=w[off[4]:off[4] + C + 1].copy())
