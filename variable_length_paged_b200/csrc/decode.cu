@@ -52,8 +52,8 @@ struct Cfg {
   // shared memory map (offsets from a 1024-byte aligned base)
   static constexpr int kOffStages = 0;
   static constexpr int kOffSlots = kStages * kStageBytes;
-  static constexpr int kOffML = kOffSlots + 3 * kSlotFloats * 4;        // [3][2][8] floats
-  static constexpr int kOffBars = kOffML + 3 * 2 * 8 * 4;                // full[kStages], empty[kStages]
+  static constexpr int kOffML = kOffSlots + 3 * kSlotFloats * 4;        // [3][m, l_r, l_e][8] floats
+  static constexpr int kOffBars = kOffML + 3 * 3 * 8 * 4;                // full[kStages], empty[kStages]
   static constexpr int kOffMeta = kOffBars + 2 * kStages * 8;            // int per stage
   static constexpr int kOffAbort = kOffMeta + kStages * 4;
   static constexpr int kBytes = kOffAbort + 16;
@@ -260,7 +260,9 @@ __global__ void __launch_bounds__(kThreads, 2)
         qhi[kk] = row_live ? __ldg(qrow + kk * 8 + 4 + tq) : 0u;
       }
     }
-    float m = -INFINITY, l = 0.f;
+    // l_r: sum of the bf16-rounded weights that enter P.V (normalises O);
+    // l_e: sum of the unrounded fp32 weights (gives the log-sum-exp)
+    float m = -INFINITY, l_r = 0.f, l_e = 0.f;
     float o[D / 8][2];
 #pragma unroll
     for (int i = 0; i < D / 8; ++i) o[i][0] = o[i][1] = 0.f;
@@ -312,9 +314,12 @@ __global__ void __launch_bounds__(kThreads, 2)
         const float m_new = fmaxf(m, mx);
         const float m_use = m_new == -INFINITY ? 0.f : m_new;
         const float corr = fast_exp2(m - m_use);
-        const uint32_t pa0 = pack_bf16x2(fast_exp2(x[0][0] - m_use), fast_exp2(x[0][1] - m_use));
-        const uint32_t pa1 = pack_bf16x2(fast_exp2(x[1][0] - m_use), fast_exp2(x[1][1] - m_use));
-        l = l * corr + (bf16_lo_to_f32(pa0) + bf16_hi_to_f32(pa0)) + (bf16_lo_to_f32(pa1) + bf16_hi_to_f32(pa1));
+        const float p00 = fast_exp2(x[0][0] - m_use), p01 = fast_exp2(x[0][1] - m_use);
+        const float p10 = fast_exp2(x[1][0] - m_use), p11 = fast_exp2(x[1][1] - m_use);
+        const uint32_t pa0 = pack_bf16x2(p00, p01);
+        const uint32_t pa1 = pack_bf16x2(p10, p11);
+        l_r = l_r * corr + (bf16_lo_to_f32(pa0) + bf16_hi_to_f32(pa0)) + (bf16_lo_to_f32(pa1) + bf16_hi_to_f32(pa1));
+        l_e = l_e * corr + ((p00 + p01) + (p10 + p11));
         m = m_new;
 #pragma unroll
         for (int i = 0; i < D / 8; ++i) {
@@ -339,38 +344,43 @@ __global__ void __launch_bounds__(kThreads, 2)
     }
 
     // ---- merge the four warp states of this segment
-    l += __shfl_xor_sync(0xffffffffu, l, 1);
-    l += __shfl_xor_sync(0xffffffffu, l, 2);
+    l_r += __shfl_xor_sync(0xffffffffu, l_r, 1);
+    l_r += __shfl_xor_sync(0xffffffffu, l_r, 2);
+    l_e += __shfl_xor_sync(0xffffffffu, l_e, 1);
+    l_e += __shfl_xor_sync(0xffffffffu, l_e, 2);
     if (w > 0) {
       float* slot = slots + (w - 1) * C::kSlotFloats + r * C::kSlotStride + 2 * tq;
 #pragma unroll
       for (int i = 0; i < D / 8; ++i) *reinterpret_cast<float2*>(slot + 8 * i) = make_float2(o[i][0], o[i][1]);
       if (tq == 0) {
-        ml[(w - 1) * 16 + r] = m;
-        ml[(w - 1) * 16 + 8 + r] = l;
+        ml[(w - 1) * 24 + r] = m;
+        ml[(w - 1) * 24 + 8 + r] = l_r;
+        ml[(w - 1) * 24 + 16 + r] = l_e;
       }
     }
     named_barrier_sync(1, kConsumerWarps * 32);
     if (w == 0) {
-      float mw[3], lw[3];
+      float mw[3], lrw[3], lew[3];
       float M = m;
 #pragma unroll
       for (int j = 0; j < 3; ++j) {
-        mw[j] = ml[j * 16 + r];
-        lw[j] = ml[j * 16 + 8 + r];
+        mw[j] = ml[j * 24 + r];
+        lrw[j] = ml[j * 24 + 8 + r];
+        lew[j] = ml[j * 24 + 16 + r];
         M = fmaxf(M, mw[j]);
       }
       const bool empty = M == -INFINITY;
       const float f0 = empty ? 0.f : fast_exp2(m - M);
       float fw[3];
-      float Lsum = f0 * l;
+      float Lr = f0 * l_r, Le = f0 * l_e;
 #pragma unroll
       for (int j = 0; j < 3; ++j) {
         fw[j] = empty ? 0.f : fast_exp2(mw[j] - M);
-        Lsum += fw[j] * lw[j];
+        Lr += fw[j] * lrw[j];
+        Le += fw[j] * lew[j];
       }
-      const float inv = Lsum > 0.f ? 1.f / Lsum : 0.f;
-      const float lse_nat = Lsum > 0.f ? (M + log2f(Lsum)) * 0.69314718055994530942f : -INFINITY;
+      const float inv = Lr > 0.f ? 1.f / Lr : 0.f;
+      const float lse_nat = Le > 0.f ? (M + log2f(Le)) * 0.69314718055994530942f : -INFINITY;
       const int h = g * p.group + r;
       const int nseg_b = rsb[b + 1] - rsb[b];
       const bool direct = nseg_b == 1;
