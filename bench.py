@@ -41,7 +41,7 @@ METRIC = "µs/decode step and KV-read HBM GB/s (% of B200 peak) vs static split-
 FALLBACK_HBM_GBS = 6650.0
 DATASHEET_HBM_GBS = 8000.0
 KERNEL_SOURCES = ["variable_length_paged_b200/csrc/decode.cu", "variable_length_paged_b200/csrc/da_internal.cuh"]
-TRAFFIC_FILE = os.path.join(ROOT, "profiles", "decode_kernel_traffic.json")
+TRAFFIC_FILE = os.path.join(ROOT, "profiles", "decode_kernel_traffic.txt")
 
 
 def parse_args():
@@ -122,14 +122,14 @@ def recorded_traffic(workload_name):
     """DRAM bytes per decode launch from the committed ncu summary, if it matches this kernel source."""
     try:
         with open(TRAFFIC_FILE) as f:
-            j = json.load(f)
+            j = dict(ln.split(": ", 1) for ln in f.read().splitlines() if ln and not ln.startswith("#"))
     except Exception:
         return None, "no ncu capture recorded"
     if j.get("kernel_source_sha") != kernel_source_hash():
         return None, "kernel changed since the ncu capture"
     if j.get("workload") != workload_name:
         return None, f"ncu capture was on {j.get('workload')}"
-    return int(j["dram_bytes_per_launch"]), j.get("command", "")
+    return int(j["dram_bytes_read_per_launch"]) + int(j["dram_bytes_write_per_launch"]), j.get("command", "")
 
 
 class ClockSampler:
