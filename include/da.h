@@ -230,6 +230,38 @@ DA_API int32_t da_last_cuda_error(void);
 /* Number of SMs of the current device (host out). */
 DA_API int da_device_num_sms(int32_t* num_sms);
 
+/* Size of the library-owned device scratch used by da_decode_step_noalloc. */
+#define DA_NOALLOC_SCRATCH_BYTES (16u << 20)
+
+/*
+ * da_decode_step_noalloc -- one whole decode step (dynamic plan, decode,
+ * combine) that allocates nothing and takes no workspace from the caller.
+ * The article has no counterpart to this call.  It is for callers that cannot
+ * allocate device memory where they run a step: an op inside a host framework
+ * whose per-call hook must not allocate, an engine that has given nearly all
+ * device memory to its KV-cache pool, or a latency-critical path where a
+ * cudaMalloc (which may synchronise the device) is not acceptable.
+ *   tile_tokens, num_ctas  as for da_plan_desc_init with DA_PLAN_DYNAMIC (0 = defaults).
+ *   q, k_cache, v_cache, block_table, seq_lens, out, lse  dev, as for
+ *     da_decode_attention; the caller still allocates inputs and outputs.
+ * Scratch: a static device array of DA_NOALLOC_SCRATCH_BYTES (16 MiB) inside
+ * the library, reserved on every GPU that loads the library's device code and
+ * held until the process exits.  A problem fits when the three sizes from
+ * da_workspace_size, each rounded up to 256 bytes, sum to at most 16 MiB
+ * (e.g. 64 query heads, head_dim 128, C = 37: C + B - 1 <= 507 segments, so
+ * batches up to 471 requests); otherwise
+ * the call returns DA_ERR_WORKSPACE and enqueues nothing.
+ * The first call on each device looks up the array's device address
+ * (cudaGetSymbolAddress) with that device current; make that first call
+ * before any stream capture.  All calls share the one array and each call
+ * overwrites it, so calls that can overlap on the GPU (other streams, other
+ * threads) race and must be serialised by the caller.  Errors as for
+ * da_decode_attention.
+ */
+DA_API int da_decode_step_noalloc(const da_problem* prob, int32_t tile_tokens, int32_t num_ctas, const void* q,
+                                  const void* k_cache, const void* v_cache, const int32_t* block_table,
+                                  const int32_t* seq_lens, void* out, float* lse, void* stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -95,6 +95,10 @@ bool make_cache_map(CUtensorMap* map, const void* base, const da_problem* p, int
 
 }  // namespace
 
+namespace da {
+void set_last_cuda_error(cudaError_t e) { g_last_cuda_error = (int32_t)e; }
+}  // namespace da
+
 extern "C" {
 
 DA_API int32_t da_last_cuda_error(void) { return g_last_cuda_error; }

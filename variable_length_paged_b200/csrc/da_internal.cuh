@@ -85,6 +85,9 @@ cudaError_t launch_plan_static(const PlanParams& p, cudaStream_t stream);
 cudaError_t launch_decode(const DecodeParams& p, int head_dim, const CUtensorMap maps[4], cudaStream_t stream);
 cudaError_t launch_combine(const CombineParams& p, int head_dim, cudaStream_t stream);
 
+// Record a CUDA error for da_last_cuda_error() from code outside api.cu.
+void set_last_cuda_error(cudaError_t e);
+
 // ---- inline PTX ----------------------------------------------------------------------------
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));

@@ -21,7 +21,9 @@ PLAN_DYNAMIC, PLAN_STATIC = 0, 1
 # Every symbol include/da.h declares.
 EXPORTS = ("da_plan_desc_init", "da_workspace_size", "da_workspace_offsets", "da_plan", "da_static_plan",
            "da_decode_attention", "da_combine", "da_read_status", "da_status_string", "da_dev_status_string",
-           "da_last_cuda_error", "da_device_num_sms")
+           "da_last_cuda_error", "da_device_num_sms", "da_decode_step_noalloc")
+
+NOALLOC_SCRATCH_BYTES = 16 << 20  # DA_NOALLOC_SCRATCH_BYTES
 
 
 class DaProblem(ctypes.Structure):
@@ -70,6 +72,7 @@ def lib():
             "da_read_status": [_vp, ctypes.POINTER(ctypes.c_int32), ctypes.POINTER(ctypes.c_int32), _vp],
             "da_last_cuda_error": [],
             "da_device_num_sms": [ctypes.POINTER(ctypes.c_int32)],
+            "da_decode_step_noalloc": [P, ctypes.c_int32, ctypes.c_int32, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp],
         }
         for name, args in sig.items():
             fn = getattr(L, name)
@@ -178,6 +181,14 @@ def da_device_num_sms() -> int:
     n = ctypes.c_int32()
     _check("da_device_num_sms", lib().da_device_num_sms(ctypes.byref(n)))
     return n.value
+
+
+def da_decode_step_noalloc(prob, q, k_cache, v_cache, block_table, seq_lens, out, lse, tile_tokens: int = 0,
+                           num_ctas: int = 0, stream=None):
+    """Whole step on the library's static scratch (for callers that cannot allocate; see include/da.h)."""
+    _check("da_decode_step_noalloc", lib().da_decode_step_noalloc(
+        ctypes.byref(prob), int(tile_tokens), int(num_ctas), _ptr(q), _ptr(k_cache), _ptr(v_cache),
+        _ptr(block_table), _ptr(seq_lens), _ptr(out), _ptr(lse), _stream(stream)))
 
 
 # ---- buffers and one whole step --------------------------------------------------------------------
