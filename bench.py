@@ -50,7 +50,7 @@ def parse_args():
     ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--config", default="mixed", choices=["mixed", "skewed", "low_conc", "uniform", "tiny"])
+    ap.add_argument("--config", default="mixed", choices=["mixed", "skewed", "low_conc", "uniform", "tiny", "trace"])
     ap.add_argument("--tile", type=int, default=64)
     ap.add_argument("--width", type=int, default=0, help="CTAs per KV head (0 = 2 per SM / Hkv)")
     ap.add_argument("--no-static", action="store_true", help="skip the static split-k comparison")
@@ -343,6 +343,81 @@ def run_ours(args, world, rank, local):
     return result
 
 
+def run_trace(args, world, rank, local):
+    """The 256-step decode trace: per step, untimed host updates + KV append, then the timed step."""
+    import numpy as np
+    import torch
+
+    from variable_length_paged_b200 import da
+    from variable_length_paged_b200 import workloads as W
+    from variable_length_paged_b200.trace import DeviceTrace
+
+    da.lib()
+    tr = W.DecodeTrace(seed=4 + 1000 * rank)
+    dt = DeviceTrace(tr)
+    prob = dt.prob
+    stream = torch.cuda.Stream()
+    desc = da.da_plan_desc_init(prob, da.PLAN_DYNAMIC, args.tile, args.width)
+    sdesc = da.da_plan_desc_init(prob, da.PLAN_STATIC, args.tile, 0)
+    bufs, sbufs = da.Buffers(prob, desc, "cuda"), da.Buffers(prob, sdesc, "cuda")
+    steps, warm = min(max(1, args.steps), tr.steps), max(3, args.warmup)
+
+    def step(d, b):
+        da.decode_step(prob, d, dt.q, dt.k_cache, dt.v_cache, dt.block_table, dt.seq_lens, b, stream=stream)
+
+    graphs = {}
+    with torch.cuda.stream(stream):
+        for key, d, b in (("dynamic", desc, bufs), ("static", sdesc, sbufs)):
+            for _ in range(warm):
+                step(d, b)
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g, stream=stream):
+                step(d, b)
+            graphs[key] = g
+        torch.cuda.synchronize()
+    times = {"dynamic": [], "static": []}
+    kv = []
+    clocks = ClockSampler(local)
+    with clocks:
+        barrier(world)
+        for t in range(steps):
+            if t > 0:
+                with torch.cuda.stream(stream):
+                    dt.advance(stream=stream)
+                torch.cuda.synchronize()
+            kv.append(tr.kv_bytes())
+            for key in ("dynamic", "static"):
+                e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                e0.record(stream)
+                graphs[key].replay()
+                e1.record(stream)
+                torch.cuda.synchronize()
+                times[key].append(e0.elapsed_time(e1))
+        status = da.da_read_status(bufs.ws, stream=stream)
+    tot_ms = {k: sum(v) for k, v in times.items()}
+    maxes, sums = reduce_max_sum([tot_ms["dynamic"], tot_ms["static"]], [float(sum(kv))], world)
+    dyn_ms, st_ms = maxes
+    value = sums[0] / (dyn_ms / 1e3) / 1e9
+    peak, peak_src = measured_peak()
+    d = np.array(times["dynamic"])
+    return dict(
+        metric=METRIC, value=round(value, 2), unit="GB/s", n_gpus=world, steps=steps, warmup=warm,
+        ms_per_step=round(dyn_ms / steps, 5), us_per_step=round(dyn_ms / steps * 1e3, 2),
+        us_per_step_median=round(float(np.median(d)) * 1e3, 2),
+        us_per_step_p10_p90=[round(float(np.percentile(d, 10)) * 1e3, 2), round(float(np.percentile(d, 90)) * 1e3, 2)],
+        higher_is_better=True, scaling="weak", vs_baseline=None, dtype="bf16", data="synthetic",
+        config={"workload": f"trace: {tr.recipe}", "batch": prob.batch, "steps_timed": steps,
+                "kv_bytes_first_last_step": [kv[0], kv[-1]], "tile_tokens": desc.tile_tokens,
+                "ctas_per_kv_head": desc.num_ctas, "graph": True,
+                "untimed": "host trace update, page copies of restarted requests, KV append kernel",
+                "l2": "inputs larger than L2 (>3 GB K/V per step), no flush"},
+        frac_of_peak=round(value / world / peak, 4), peak=peak, peak_source=peak_src,
+        static_split_k={"default_splits": sdesc.splits, "us_per_step": round(st_ms / steps * 1e3, 2)},
+        speedup_vs_static_default=round(st_ms / dyn_ms, 3),
+        gpu_launches=3 * steps * 2 + (steps - 1), device_status=status[0],
+        append_status=dt.status.tolist(), clocks=clocks.summary())
+
+
 def cpu_baseline(w, seconds):
     """The CPU oracle (fp64) on this host's cores, repeated over the full batch for a bounded time."""
     import oracle
@@ -371,7 +446,7 @@ def run_reference(args, rank):
     from variable_length_paged_b200 import workloads as W
 
     oracle.build()
-    w = W.CONFIGS[args.config]()
+    w = W.DecodeTrace().workload() if args.config == "trace" else W.CONFIGS[args.config]()
     B, Hq = w.problem.batch, w.problem.num_q_heads
     order = np.argsort(-w.seq_lens, kind="stable")
     # calibrate: aim for about one second of oracle work per step, and at most ~150 s in total
@@ -421,7 +496,7 @@ def main():
         return 0
     world, rank, local = dist_setup(args)
     try:
-        res = run_ours(args, world, rank, local)
+        res = run_trace(args, world, rank, local) if args.config == "trace" else run_ours(args, world, rank, local)
         if rank == 0:
             print(json.dumps(res), flush=True)
     finally:

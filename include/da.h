@@ -206,11 +206,31 @@ DA_API int da_decode_attention(const da_problem* prob, const da_plan_desc* desc,
 /*
  * da_combine -- merge the partials of requests with two or more segments:
  *   LSE = M + ln sum_i exp(lse_i - M),  M = max_i lse_i,
- *   out = sum_i exp(lse_i - LSE) o_i    (fp32, segment order, then bf16),
+ *   out = sum_i exp(lse_i - LSE) o_i    (fp32 sums in a fixed order, then bf16),
  * and write out = 0, lse = -inf for requests with no segment.
  */
 DA_API int da_combine(const da_problem* prob, const da_plan_desc* desc, const void* ws, const float* partial_o,
                       const float* partial_lse, void* out, float* lse, void* stream);
+
+/*
+ * da_append_kv -- write each request's newest token into the paged cache
+ * (the step before attention in every decode step: lengths grow by one).
+ *   new_k, new_v  dev bf16 [batch][num_kv_heads][head_dim], 16-byte aligned.
+ *   seq_lens      dev int32 [batch], lengths that already count the new token:
+ *                 request b's rows go to position seq_lens[b]-1, i.e. page
+ *                 block_table[b][(seq_lens[b]-1)/page_size], slot
+ *                 (seq_lens[b]-1) % page_size.  Requests with length 0 are skipped.
+ *   k_cache, v_cache  dev, written in place (16-byte aligned).
+ *   status        optional dev int32 [2], or NULL: the first bad request is
+ *                 recorded as {DA_DEV_BAD_SEQLEN or DA_DEV_BAD_PAGE, b} and its
+ *                 row skipped; the caller clears it.
+ * The engine allocates pages: the block-table entry for a new page must be set
+ * before the call.  Source: "Tencent HPC lands in SGLang, challenging default
+ * inference kernels", section "Why Tencent HPC matters for online model
+ * serving" (request lengths change during decoding).
+ */
+DA_API int da_append_kv(const da_problem* prob, const void* new_k, const void* new_v, const int32_t* block_table,
+                        const int32_t* seq_lens, void* k_cache, void* v_cache, int32_t* status, void* stream);
 
 /*
  * da_read_status -- copy the device status word and first bad index out of

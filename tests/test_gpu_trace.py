@@ -1,0 +1,90 @@
+"""The decode trace (256 steps, batch 256, lengths changing every step) and the append kernel.
+
+The plan is rebuilt on the device every step and checked bit-exactly against
+the oracle's plan at every step; attention outputs are checked against the
+fp64 oracle on every (request, head) at steps 0, 1, 127 and 255; at the end the
+device cache, written step by step by da_append_kv, must equal the host cache
+bit for bit at every live token.
+"""
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from gpu_helpers import assert_plan_equal, check_against_oracle
+from variable_length_paged_b200 import da
+from variable_length_paged_b200 import workloads as W
+from variable_length_paged_b200.trace import DeviceTrace
+
+pytestmark = pytest.mark.gpu
+
+
+def test_append_kv_rows_land_in_their_pages(da_lib):
+    w = W.make_workload("a", [63, 64, 1, 0, 200], num_q_heads=8, num_kv_heads=2, head_dim=128, page_size=64,
+                        seed=3, max_pages_per_req=5, extra_pages=4)
+    dw = w.to("cuda")
+    prob = da.problem_from(w.problem)
+    lens = w.seq_lens.copy()
+    bt = w.block_table.copy()
+    spare = sorted(set(range(w.problem.num_pages)) - set(bt[bt >= 0].tolist()))
+    for b in range(len(lens)):  # grow every live request by one token (new page when full)
+        if lens[b] == 0:
+            continue
+        if lens[b] % 64 == 0:
+            bt[b, lens[b] // 64] = spare.pop()
+        lens[b] += 1
+    dw.block_table.copy_(torch.from_numpy(bt))
+    dw.seq_lens.copy_(torch.from_numpy(lens))
+    g = torch.Generator().manual_seed(5)
+    nk = torch.randn(5, 2, 128, generator=g).to(torch.bfloat16)
+    nv = torch.randn(5, 2, 128, generator=g).to(torch.bfloat16)
+    status = torch.zeros(2, dtype=torch.int32, device="cuda")
+    k0, v0 = dw.k_cache.clone(), dw.v_cache.clone()
+    da.da_append_kv(prob, nk.cuda(), nv.cuda(), dw.block_table, dw.seq_lens, dw.k_cache, dw.v_cache, status)
+    torch.cuda.synchronize()
+    assert status.tolist() == [0, 0]
+    ek, ev = k0.clone(), v0.clone()
+    for b in range(5):
+        if lens[b] == 0:
+            continue
+        pos = lens[b] - 1
+        page, slot = bt[b, pos // 64], pos % 64
+        ek[page, :, slot] = nk[b].cuda()
+        ev[page, :, slot] = nv[b].cuda()
+    same = lambda a, b: torch.equal(a.view(torch.int16), b.view(torch.int16))
+    assert same(dw.k_cache, ek) and same(dw.v_cache, ev)
+    # a bad page id is reported and its row skipped
+    dw.block_table[4, (lens[4] - 1) // 64] = w.problem.num_pages + 3
+    da.da_append_kv(prob, nk.cuda(), nv.cuda(), dw.block_table, dw.seq_lens, dw.k_cache, dw.v_cache, status)
+    torch.cuda.synchronize()
+    assert status.tolist() == [da.DEV_BAD_PAGE, 4]
+
+
+def test_decode_trace_256_steps(da_lib, oracle_lib):
+    tr = W.DecodeTrace()
+    dt = DeviceTrace(tr)
+    prob = dt.prob
+    desc = da.da_plan_desc_init(prob, da.PLAN_DYNAMIC, 64, 0)
+    bufs = da.Buffers(prob, desc, "cuda")
+    cap = prob.max_pages_per_req * prob.page_size
+    for t in range(tr.steps):
+        if t > 0:
+            dt.advance()
+        da.decode_step(prob, desc, dt.q, dt.k_cache, dt.v_cache, dt.block_table, dt.seq_lens, bufs)
+        torch.cuda.synchronize()
+        assert_plan_equal(da.read_plan(desc, bufs.ws), oracle.plan(tr.seq_lens, 64, desc.num_ctas, cap))
+        if t in (0, 1, 127, 255):
+            check_against_oracle(tr.workload(), bufs.out, bufs.lse)
+    assert dt.status.tolist() == [0, 0]
+    assert da.da_read_status(bufs.ws) == (0, -1)
+    # the device cache, built step by step by the append kernel, equals the host cache at live tokens
+    live = np.zeros((prob.num_pages, prob.page_size), dtype=bool)
+    for b in range(prob.batch):
+        t = np.arange(int(tr.lens[b]))
+        live[tr.block_table[b, t // prob.page_size], t % prob.page_size] = True
+    m = torch.from_numpy(live)
+    for dev_c, host_c in ((dt.k_cache, tr.k_cache), (dt.v_cache, tr.v_cache)):
+        d = dev_c.cpu().permute(0, 2, 1, 3)[m]
+        h = host_c.permute(0, 2, 1, 3)[m]
+        assert torch.equal(d.view(torch.int16), h.view(torch.int16))

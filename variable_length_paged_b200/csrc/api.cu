@@ -288,6 +288,35 @@ DA_API int da_combine(const da_problem* prob, const da_plan_desc* desc, const vo
   return e == cudaSuccess ? DA_OK : cuda_fail(e);
 }
 
+DA_API int da_append_kv(const da_problem* prob, const void* new_k, const void* new_v, const int32_t* block_table,
+                        const int32_t* seq_lens, void* k_cache, void* v_cache, int32_t* status, void* stream) {
+  int rc = check_problem(prob);
+  if (rc != DA_OK) return rc;
+  if (prob->batch == 0) return DA_OK;
+  if (!new_k || !new_v || !block_table || !seq_lens || !k_cache || !v_cache) return DA_ERR_INVALID_ARG;
+  if (reinterpret_cast<uintptr_t>(new_k) % 16 != 0 || reinterpret_cast<uintptr_t>(new_v) % 16 != 0 ||
+      reinterpret_cast<uintptr_t>(k_cache) % 16 != 0 || reinterpret_cast<uintptr_t>(v_cache) % 16 != 0 ||
+      reinterpret_cast<uintptr_t>(status) % 4 != 0)
+    return DA_ERR_INVALID_ARG;
+  da::AppendParams p;
+  p.new_k = static_cast<const __nv_bfloat16*>(new_k);
+  p.new_v = static_cast<const __nv_bfloat16*>(new_v);
+  p.block_table = block_table;
+  p.seq_lens = seq_lens;
+  p.k_cache = static_cast<__nv_bfloat16*>(k_cache);
+  p.v_cache = static_cast<__nv_bfloat16*>(v_cache);
+  p.status = status;
+  p.batch = prob->batch;
+  p.num_kv_heads = prob->num_kv_heads;
+  p.head_dim = prob->head_dim;
+  p.page_size = prob->page_size;
+  p.max_pages_per_req = prob->max_pages_per_req;
+  p.num_pages = prob->num_pages;
+  p.capacity_tokens = (int64_t)prob->max_pages_per_req * prob->page_size;
+  cudaError_t e = da::launch_append(p, static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? DA_OK : cuda_fail(e);
+}
+
 DA_API int da_read_status(const void* ws, int32_t* dev_status, int32_t* bad_index, void* stream) {
   if (!ws) return DA_ERR_INVALID_ARG;
   int32_t h[da::kHdrWords];

@@ -79,11 +79,24 @@ struct CombineParams {
   int32_t batch, num_q_heads, num_ctas, max_segments;
 };
 
+struct AppendParams {
+  const __nv_bfloat16* new_k;
+  const __nv_bfloat16* new_v;
+  const int32_t* block_table;
+  const int32_t* seq_lens;
+  __nv_bfloat16* k_cache;
+  __nv_bfloat16* v_cache;
+  int32_t* status;  // optional {code, index}
+  int32_t batch, num_kv_heads, head_dim, page_size, max_pages_per_req, num_pages;
+  int64_t capacity_tokens;
+};
+
 // Host launchers (defined next to their kernels).
 cudaError_t launch_plan_dynamic(const PlanParams& p, cudaStream_t stream);
 cudaError_t launch_plan_static(const PlanParams& p, cudaStream_t stream);
 cudaError_t launch_decode(const DecodeParams& p, int head_dim, const CUtensorMap maps[4], cudaStream_t stream);
 cudaError_t launch_combine(const CombineParams& p, int head_dim, cudaStream_t stream);
+cudaError_t launch_append(const AppendParams& p, cudaStream_t stream);
 
 // Record a CUDA error for da_last_cuda_error() from code outside api.cu.
 void set_last_cuda_error(cudaError_t e);

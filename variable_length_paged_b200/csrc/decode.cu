@@ -98,7 +98,29 @@ __global__ void __launch_bounds__(kThreads, 2)
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int cta = blockIdx.x, g = blockIdx.y;
 
-  grid_dependency_wait();  // the plan is written by the previous kernel in the stream
+  // Prologue that does not depend on the plan: barriers and descriptor
+  // prefetch overlap the planner kernel (programmatic dependent launch).
+  const uint32_t full0 = sbase + C::kOffBars, empty0 = full0 + C::kStages * 8;
+  volatile int* meta = reinterpret_cast<volatile int*>(smem + C::kOffMeta);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::kOffAbort);
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < C::kStages; ++s) {
+      mbar_init(full0 + 8 * s, 1);
+      mbar_init(empty0 + 8 * s, kConsumerWarps);
+    }
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == kConsumerWarps && lane == 0) {
+    prefetch_tensormap(&k64);
+    prefetch_tensormap(&v64);
+    prefetch_tensormap(&k16);
+    prefetch_tensormap(&v16);
+  }
+  __syncthreads();
+
+  grid_dependency_wait();    // the plan is written by the previous kernel in the stream
+  grid_dependents_launch();  // the combine kernel may be scheduled; it waits for this grid to finish
 
   const WsLayout WL = ws_layout(p.batch, p.num_ctas, p.max_segments);
   const int32_t* hdr = p.ws + WL.hdr;
@@ -108,38 +130,17 @@ __global__ void __launch_bounds__(kThreads, 2)
   int32_t* hdr_w = const_cast<int32_t*>(hdr);
 
   // The plan must match the descriptor this launch was given.
-  if (hdr[kHdrCtas] != p.num_ctas || hdr[kHdrBatch] != p.batch || hdr[kHdrMaxSegments] != p.max_segments ||
-      hdr[kHdrKind] != p.kind) {
+  const int h_ctas = hdr[kHdrCtas], h_batch = hdr[kHdrBatch], h_ms = hdr[kHdrMaxSegments], h_kind = hdr[kHdrKind];
+  const int h_segs = hdr[kHdrSegments], seg_lo = csb[cta], seg_next = csb[cta + 1];
+  if (h_ctas != p.num_ctas || h_batch != p.batch || h_ms != p.max_segments || h_kind != p.kind) {
     if (threadIdx.x == 0 && cta == 0 && g == 0) record_status(hdr_w, DA_DEV_BAD_PLAN, 0);
     return;
   }
-  const int nseg_total = min(hdr[kHdrSegments], p.max_segments);
-  const int seg_lo = csb[cta], seg_hi = min(csb[cta + 1], nseg_total);
+  const int seg_hi = min(seg_next, min(h_segs, p.max_segments));
   if (seg_lo < 0 || seg_lo >= seg_hi) return;  // nothing planned for this CTA (uniform over the block)
-
-  uint32_t* bars = reinterpret_cast<uint32_t*>(smem + C::kOffBars);
-  const uint32_t full0 = sbase + C::kOffBars, empty0 = full0 + C::kStages * 8;
-  volatile int* meta = reinterpret_cast<volatile int*>(smem + C::kOffMeta);
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::kOffAbort);
-  (void)bars;
-  if (threadIdx.x == 0) {
-    for (int s = 0; s < C::kStages; ++s) {
-      mbar_init(full0 + 8 * s, 1);
-      mbar_init(empty0 + 8 * s, kConsumerWarps);
-    }
-    *abort_flag = 0;
-    fence_mbar_init();
-  }
-  __syncthreads();
 
   if (warp == kConsumerWarps) {
     // ------------------------------------------------------------------ producer warp
-    if (lane == 0) {
-      prefetch_tensormap(&k64);
-      prefetch_tensormap(&v64);
-      prefetch_tensormap(&k16);
-      prefetch_tensormap(&v16);
-    }
     const uint64_t policy = policy_evict_first();
     const int P = p.page_size;
     int stage = 0;
@@ -147,10 +148,17 @@ __global__ void __launch_bounds__(kThreads, 2)
     int fills = 0;
     bool aborted = false;
     for (int s = seg_lo; s < seg_hi && !aborted; ++s) {
+      // first window of page ids, issued before (and independent of) the length load
+      const int4 sg = segs[s];
+      int win_base = INT_MIN / 2, win_val = -1;
+      if (sg.x >= 0 && sg.x < p.batch && sg.z >= 0) {
+        win_base = (int)((int64_t)sg.z * p.tile_tokens / P);
+        const int lp = win_base + lane;
+        win_val = lp < p.max_pages_per_req ? __ldg(p.block_table + (int64_t)sg.x * p.max_pages_per_req + lp) : -1;
+      }
       const SegmentInfo si = load_segment(p, segs, s);
       if (!si.valid) continue;
       const int32_t* bt_row = p.block_table + (int64_t)si.b * p.max_pages_per_req;
-      int win_base = INT_MIN / 2, win_val = -1;
       for (int c0 = si.tok0; c0 < si.tok1; c0 += kChunk) {
         const int n = min(kChunk, si.tok1 - c0);
         const int lp_first = c0 / P, lp_last = (c0 + n - 1) / P;

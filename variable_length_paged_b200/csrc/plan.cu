@@ -56,19 +56,30 @@ __device__ int request_tiles(const PlanParams& p, int b, int* s_bad) {
   return (int)(((int64_t)L + p.tile_tokens - 1) / p.tile_tokens);
 }
 
+// Prefix arrays are kept in shared memory when the batch fits, else read back
+// from global memory (written by this block and visible after __syncthreads).
+constexpr int kSmemBatch = 4096;
+
 // Phase shared by both planners: req_tile_prefix and U (and the largest n_b).
-__device__ void tile_prefix(const PlanParams& p, int32_t* rtp, int* warp_buf, int* s_bad, int* U, int* max_tiles) {
+__device__ void tile_prefix(const PlanParams& p, int32_t* rtp, int32_t* s_rtp, int* warp_buf, int* s_bad, int* U,
+                            int* max_tiles) {
   int carry = 0, mx = 0;
   for (int base = 0; base < p.batch; base += kPlanThreads) {
     const int b = base + threadIdx.x;
     const int n = b < p.batch ? request_tiles(p, b, s_bad) : 0;
     int total;
     const int excl = block_exclusive_scan(n, &total, warp_buf);
-    if (b < p.batch) rtp[b + 1] = carry + excl + n;
+    if (b < p.batch) {
+      rtp[b + 1] = carry + excl + n;
+      if (s_rtp) s_rtp[b + 1] = carry + excl + n;
+    }
     carry += total;
     mx = max(mx, n);
   }
-  if (threadIdx.x == 0) rtp[0] = 0;
+  if (threadIdx.x == 0) {
+    rtp[0] = 0;
+    if (s_rtp) s_rtp[0] = 0;
+  }
   // block max of n
   for (int o = 16; o > 0; o >>= 1) mx = max(mx, __shfl_xor_sync(0xffffffffu, mx, o));
   if ((threadIdx.x & 31) == 0) warp_buf[threadIdx.x >> 5] = mx;
@@ -102,9 +113,22 @@ __device__ void write_header(const PlanParams& p, int32_t* hdr, int U, int S, in
 __device__ __forceinline__ int owner_cta(int64_t u, int64_t U, int64_t C) { return (int)(((u + 1) * C - 1) / U); }
 __device__ __forceinline__ int64_t cta_first_unit(int64_t c, int64_t U, int64_t C) { return c * U / C; }
 
+// Largest i in [0, n] with a[i] <= x, for a non-decreasing a[0..n] with a[0] <= x.
+__device__ __forceinline__ int last_not_above(const int32_t* a, int n, int64_t x) {
+  int lo = 0, hi = n;
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) >> 1;
+    if (a[mid] <= x) lo = mid; else hi = mid - 1;
+  }
+  return lo;
+}
+
 __global__ void __launch_bounds__(kPlanThreads) plan_dynamic_kernel(const PlanParams p) {
   __shared__ int warp_buf[32];
   __shared__ int s_bad;
+  __shared__ int32_t s_rtp[kSmemBatch + 1], s_rsb[kSmemBatch + 1];
+  grid_dependency_wait();     // seq_lens may come from the previous kernel in the stream
+  grid_dependents_launch();   // let the decode kernel start its prologue
   if (threadIdx.x == 0) s_bad = INT_MAX;
   __syncthreads();
 
@@ -114,10 +138,13 @@ __global__ void __launch_bounds__(kPlanThreads) plan_dynamic_kernel(const PlanPa
   int32_t* rtp = p.ws + L.req_tile_prefix;
   int32_t* rsb = p.ws + L.req_seg_begin;
   int32_t* csb = p.ws + L.cta_seg_begin;
+  const bool small = p.batch <= kSmemBatch;
+  const int32_t* rtp_r = small ? s_rtp : rtp;
+  const int32_t* rsb_r = small ? s_rsb : rsb;
   const int64_t C = p.num_ctas;
 
   int U, max_tiles;
-  tile_prefix(p, rtp, warp_buf, &s_bad, &U, &max_tiles);
+  tile_prefix(p, rtp, small ? s_rtp : nullptr, warp_buf, &s_bad, &U, &max_tiles);
 
   // Segments per request.  With U >= C every CTA owns at least one tile, so a
   // request spanning CTAs [cf, cl] has cl - cf + 1 segments.  With U < C each
@@ -128,44 +155,52 @@ __global__ void __launch_bounds__(kPlanThreads) plan_dynamic_kernel(const PlanPa
     const int b = base + threadIdx.x;
     int ns = 0;
     if (b < p.batch) {
-      const int p0 = rtp[b], n = rtp[b + 1] - p0;
+      const int p0 = rtp_r[b], n = rtp_r[b + 1] - p0;
       if (n > 0) ns = sparse ? n : owner_cta(p0 + n - 1, U, C) - owner_cta(p0, U, C) + 1;
     }
     int total;
     const int excl = block_exclusive_scan(ns, &total, warp_buf);
-    if (b < p.batch) rsb[b + 1] = carry + excl + ns;
+    if (b < p.batch) {
+      rsb[b + 1] = carry + excl + ns;
+      if (small) s_rsb[b + 1] = carry + excl + ns;
+    }
     carry += total;
   }
-  if (threadIdx.x == 0) rsb[0] = 0;
+  if (threadIdx.x == 0) {
+    rsb[0] = 0;
+    if (small) s_rsb[0] = 0;
+  }
   const int S = carry;
   __syncthreads();
 
-  // Segments and the per-CTA segment ranges.
-  for (int b = threadIdx.x; b < p.batch; b += kPlanThreads) {
-    const int p0 = rtp[b], n = rtp[b + 1] - p0;
-    if (n == 0) continue;
-    const int s0 = rsb[b];
+  // One thread per segment: find its request, then its CTA and tile range.
+  for (int s = threadIdx.x; s < S; s += kPlanThreads) {
+    const int b = last_not_above(rsb_r, p.batch, s);  // rsb[b] <= s < rsb[b+1]
+    const int j = s - rsb_r[b];
+    const int p0 = rtp_r[b], n = rtp_r[b + 1] - p0;
     if (sparse) {
-      for (int j = 0; j < n; ++j) segs[s0 + j] = make_int4(b, owner_cta(p0 + j, U, C), j, j + 1);
-      continue;
-    }
-    const int cf = owner_cta(p0, U, C), cl = owner_cta(p0 + n - 1, U, C);
-    const int prev = p0 > 0 ? owner_cta(p0 - 1, U, C) : -1;
-    for (int c = prev + 1; c <= cf; ++c) csb[c] = s0;  // this segment opens CTA cf
-    for (int c = cf; c <= cl; ++c) {
+      segs[s] = make_int4(b, owner_cta((int64_t)p0 + j, U, C), j, j + 1);
+    } else {
+      const int c = owner_cta(p0, U, C) + j;
       const int64_t lo = max((int64_t)p0, cta_first_unit(c, U, C));
       const int64_t hi = min((int64_t)p0 + n, cta_first_unit(c + 1, U, C));
-      const int s = s0 + (c - cf);
       segs[s] = make_int4(b, c, (int)(lo - p0), (int)(hi - p0));
-      if (c > cf) csb[c] = s;
     }
   }
-  if (sparse) {
-    // every tile is a segment, so CTA c starts at segment floor(c*U/C)
-    for (int c = threadIdx.x; c <= p.num_ctas; c += kPlanThreads) csb[c] = (int)cta_first_unit(c, U, C);
-  } else {
-    const int last = owner_cta((int64_t)U - 1, U, C);
-    for (int c = last + 1 + threadIdx.x; c <= p.num_ctas; c += kPlanThreads) csb[c] = S;
+  // One thread per CTA: its first segment.
+  for (int c = threadIdx.x; c <= p.num_ctas; c += kPlanThreads) {
+    int first;
+    if (sparse) {
+      first = (int)cta_first_unit(c, U, C);  // every tile is a segment
+    } else if (c == p.num_ctas) {
+      first = S;
+    } else {
+      // the request holding CTA c's first tile opens CTA c
+      const int64_t u0 = cta_first_unit(c, U, C);
+      const int r = last_not_above(rtp_r, p.batch, u0);
+      first = rsb_r[r] + (c - owner_cta(rtp_r[r], U, C));
+    }
+    csb[c] = first;
   }
   if (threadIdx.x == 0) write_header(p, hdr, U, S, DA_PLAN_DYNAMIC, 0, s_bad);
 }
@@ -173,6 +208,9 @@ __global__ void __launch_bounds__(kPlanThreads) plan_dynamic_kernel(const PlanPa
 __global__ void __launch_bounds__(kPlanThreads) plan_static_kernel(const PlanParams p) {
   __shared__ int warp_buf[32];
   __shared__ int s_bad;
+  __shared__ int32_t s_rtp[kSmemBatch + 1];
+  grid_dependency_wait();
+  grid_dependents_launch();
   if (threadIdx.x == 0) s_bad = INT_MAX;
   __syncthreads();
 
@@ -182,15 +220,17 @@ __global__ void __launch_bounds__(kPlanThreads) plan_static_kernel(const PlanPar
   int32_t* rtp = p.ws + L.req_tile_prefix;
   int32_t* rsb = p.ws + L.req_seg_begin;
   int32_t* csb = p.ws + L.cta_seg_begin;
+  const bool small = p.batch <= kSmemBatch;
+  const int32_t* rtp_r = small ? s_rtp : rtp;
   const int S = p.width;
 
   int U, max_tiles;
-  tile_prefix(p, rtp, warp_buf, &s_bad, &U, &max_tiles);
+  tile_prefix(p, rtp, small ? s_rtp : nullptr, warp_buf, &s_bad, &U, &max_tiles);
   const int chunk = (max_tiles + S - 1) / S;
   const int total = p.batch * S;
   for (int i = threadIdx.x; i < total; i += kPlanThreads) {
     const int b = i / S, s = i - b * S;
-    const int n = rtp[b + 1] - rtp[b];
+    const int n = rtp_r[b + 1] - rtp_r[b];
     const int64_t lo = min((int64_t)s * chunk, (int64_t)n), hi = min((int64_t)(s + 1) * chunk, (int64_t)n);
     segs[i] = make_int4(b, i, (int)lo, (int)hi);
   }
@@ -201,14 +241,28 @@ __global__ void __launch_bounds__(kPlanThreads) plan_static_kernel(const PlanPar
 
 }  // namespace
 
+namespace {
+template <typename K>
+cudaError_t launch_planner(K kernel, const PlanParams& p, cudaStream_t stream) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(1, 1, 1);
+  cfg.blockDim = dim3(kPlanThreads, 1, 1);
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, p);
+}
+}  // namespace
+
 cudaError_t launch_plan_dynamic(const PlanParams& p, cudaStream_t stream) {
-  plan_dynamic_kernel<<<1, kPlanThreads, 0, stream>>>(p);
-  return cudaGetLastError();
+  return launch_planner(plan_dynamic_kernel, p, stream);
 }
 
 cudaError_t launch_plan_static(const PlanParams& p, cudaStream_t stream) {
-  plan_static_kernel<<<1, kPlanThreads, 0, stream>>>(p);
-  return cudaGetLastError();
+  return launch_planner(plan_static_kernel, p, stream);
 }
 
 }  // namespace da

@@ -21,7 +21,7 @@ PLAN_DYNAMIC, PLAN_STATIC = 0, 1
 # Every symbol include/da.h declares.
 EXPORTS = ("da_plan_desc_init", "da_workspace_size", "da_workspace_offsets", "da_plan", "da_static_plan",
            "da_decode_attention", "da_combine", "da_read_status", "da_status_string", "da_dev_status_string",
-           "da_last_cuda_error", "da_device_num_sms", "da_decode_step_noalloc")
+           "da_last_cuda_error", "da_device_num_sms", "da_decode_step_noalloc", "da_append_kv")
 
 NOALLOC_SCRATCH_BYTES = 16 << 20  # DA_NOALLOC_SCRATCH_BYTES
 
@@ -73,6 +73,7 @@ def lib():
             "da_last_cuda_error": [],
             "da_device_num_sms": [ctypes.POINTER(ctypes.c_int32)],
             "da_decode_step_noalloc": [P, ctypes.c_int32, ctypes.c_int32, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp],
+            "da_append_kv": [P, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp],
         }
         for name, args in sig.items():
             fn = getattr(L, name)
@@ -169,6 +170,12 @@ def da_decode_attention(prob, desc, q, k_cache, v_cache, block_table, seq_lens, 
 def da_combine(prob, desc, ws, partial_o, partial_lse, out, lse, stream=None):
     _check("da_combine", lib().da_combine(ctypes.byref(prob), ctypes.byref(desc), _ptr(ws), _ptr(partial_o),
                                           _ptr(partial_lse), _ptr(out), _ptr(lse), _stream(stream)))
+
+
+def da_append_kv(prob, new_k, new_v, block_table, seq_lens, k_cache, v_cache, status=None, stream=None):
+    _check("da_append_kv", lib().da_append_kv(ctypes.byref(prob), _ptr(new_k), _ptr(new_v), _ptr(block_table),
+                                              _ptr(seq_lens), _ptr(k_cache), _ptr(v_cache), _ptr(status),
+                                              _stream(stream)))
 
 
 def da_read_status(ws, stream=None) -> tuple[int, int]:

@@ -1,0 +1,45 @@
+"""Run a DecodeTrace on the device.
+
+The host trace (workloads.DecodeTrace) owns the lengths, the page free list
+and the reference copy of the cache; this class keeps a device copy in step:
+restarted requests' pages are copied from the host, the block table and
+lengths are copied whole, and each step's new K/V rows are written into their
+pages by the library's append kernel (da_append_kv).
+"""
+
+from __future__ import annotations
+
+import torch
+
+from . import da
+from .workloads import DecodeTrace
+
+
+class DeviceTrace:
+    def __init__(self, trace: DecodeTrace, device="cuda"):
+        self.trace = trace
+        self.device = torch.device(device)
+        self.prob = da.problem_from(trace.problem)
+        self.k_cache = trace.k_cache.to(self.device)
+        self.v_cache = trace.v_cache.to(self.device)
+        self.seq_lens = torch.from_numpy(trace.seq_lens).to(self.device)
+        self.block_table = torch.from_numpy(trace.block_table).to(self.device)
+        self.q = trace.q.to(self.device)
+        self.status = torch.zeros(2, dtype=torch.int32, device=self.device)
+
+    def advance(self, stream=None) -> dict:
+        """Advance the host trace one step and bring the device copy along (asynchronous)."""
+        upd = self.trace.advance()
+        if upd["restarted_pages"]:
+            idx = torch.tensor(upd["restarted_pages"], dtype=torch.long)
+            didx = idx.to(self.device)
+            self.k_cache[didx] = self.trace.k_cache[idx].to(self.device)
+            self.v_cache[didx] = self.trace.v_cache[idx].to(self.device)
+        self.block_table.copy_(torch.from_numpy(self.trace.block_table))
+        self.seq_lens.copy_(torch.from_numpy(self.trace.seq_lens))
+        self.q.copy_(upd["q"])
+        new_k = upd["new_k"].to(self.device)
+        new_v = upd["new_v"].to(self.device)
+        da.da_append_kv(self.prob, new_k, new_v, self.block_table, self.seq_lens, self.k_cache, self.v_cache,
+                        self.status, stream=stream)
+        return upd

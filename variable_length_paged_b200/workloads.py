@@ -223,3 +223,121 @@ def uniform(seed: int = 5, batch: int = 64, length: int = 4096, **kw) -> Workloa
 
 
 CONFIGS = {"tiny": tiny, "mixed": mixed, "skewed": skewed, "low_conc": low_conc, "uniform": uniform}
+
+
+# ---------------------------------------------------------------------------------------------
+# The decode trace: a continuous batch evolving over many steps.
+
+
+class DecodeTrace:
+    """Continuous-batch decode trace: B request slots stepping together.
+
+    Start: lengths lognormal(ln median, sigma) rounded and clipped to
+    [1, max_len]; pages as in the module recipe, from a host free list (LIFO)
+    of a pool with room to grow.  Step 0 decodes the starting batch.  Before
+    each later step, in this order: every slot finishes with probability
+    p_finish (its pages go back to the free list and a new request of length
+    uniform in new_len takes the slot, with fresh N(0,1) K/V); then every slot
+    grows by one token (a fresh N(0,1) K/V row at position L, a new page when
+    L % P == 0); then a fresh q ~ N(0,1) is drawn.  The host keeps the whole
+    cache (the CPU oracle reads it); `advance()` returns what the device copy
+    needs to follow.
+    """
+
+    def __init__(self, seed: int = 4, batch: int = 256, steps: int = 256, num_q_heads: int = 32,
+                 num_kv_heads: int = 4, head_dim: int = 128, page_size: int = 64, median: float = 4096.0,
+                 sigma: float = 1.0, max_len: int = 32768, p_finish: float = 0.01, new_len=(500, 2000),
+                 spare_pages: int | None = None):
+        self.rng = np.random.default_rng(seed)
+        self.gen = torch.Generator().manual_seed(seed)
+        self.seed, self.steps, self.p_finish, self.new_len = seed, steps, p_finish, new_len
+        P = page_size
+        lens = np.clip(np.round(self.rng.lognormal(math.log(median), sigma, batch)), 1, max_len).astype(np.int64)
+        self.max_pages = -(-(max_len + steps) // P)
+        used = int(sum(-(-int(l) // P) for l in lens))
+        spare = spare_pages if spare_pages is not None else batch * (-(-steps // P) + 2) + used // 4
+        num_pages = used + spare
+        self.problem = Problem(batch=batch, num_q_heads=num_q_heads, num_kv_heads=num_kv_heads,
+                               head_dim=head_dim, page_size=P, max_pages_per_req=self.max_pages,
+                               num_pages=num_pages, scale=_fp32(1.0 / math.sqrt(head_dim)))
+        # free list: a random permutation of the pool, taken from the end
+        self.free = list(self.rng.permutation(num_pages).astype(np.int64))
+        self.block_table = np.full((batch, self.max_pages), -1, dtype=np.int32)
+        self.lens = np.zeros(batch, dtype=np.int64)
+        shape = (num_pages, num_kv_heads, P, head_dim)
+        self.k_cache = torch.full(shape, float("nan"), dtype=torch.bfloat16)  # unused pages stay NaN
+        self.v_cache = torch.full(shape, float("nan"), dtype=torch.bfloat16)
+        for b in range(batch):
+            self._start_request(b, int(lens[b]))
+        self.q = _randn_bf16(self.gen, (batch, num_q_heads, head_dim))
+        self.step = 0
+        self.recipe = (f"B={batch}, L0~lognormal(ln {median:g}, {sigma:g}) clipped [1,{max_len}], {steps} steps: "
+                       f"+1 token/step, finish p={p_finish} -> new U[{new_len[0]},{new_len[1]}]; "
+                       f"{num_q_heads}q/{num_kv_heads}kv; d{head_dim}; P{P}")
+
+    # -- host-side state changes
+    def _take_page(self) -> int:
+        if not self.free:
+            raise RuntimeError("trace page pool exhausted")
+        return int(self.free.pop())
+
+    def _start_request(self, b: int, L: int) -> list[int]:
+        P = self.problem.page_size
+        n = -(-L // P)
+        pages = [self._take_page() for _ in range(n)]
+        self.block_table[b, :] = -1
+        self.block_table[b, :n] = pages
+        self.lens[b] = L
+        idx = torch.tensor(pages, dtype=torch.long)
+        sub = (n, self.problem.num_kv_heads, P, self.problem.head_dim)
+        self.k_cache[idx] = _randn_bf16(self.gen, sub)
+        self.v_cache[idx] = _randn_bf16(self.gen, sub)
+        return pages
+
+    def _finish_request(self, b: int):
+        n = -(-int(self.lens[b]) // self.problem.page_size)
+        self.free.extend(int(x) for x in self.block_table[b, :n][::-1])
+        self.block_table[b, :] = -1
+        self.lens[b] = 0
+
+    def advance(self) -> dict:
+        """Move to the next step; returns the changes: restarted slots and their pages, the
+        appended K/V rows ([B, Hkv, d] bf16, at position lens-1), the new q."""
+        p = self.problem
+        B, P = p.batch, p.page_size
+        finish = self.rng.random(B) < self.p_finish
+        restarted, new_pages = [], []
+        for b in np.nonzero(finish)[0]:
+            self._finish_request(int(b))
+            L = int(self.rng.integers(self.new_len[0], self.new_len[1] + 1))
+            new_pages += self._start_request(int(b), L)
+            restarted.append(int(b))
+        new_k = _randn_bf16(self.gen, (B, p.num_kv_heads, p.head_dim))
+        new_v = _randn_bf16(self.gen, (B, p.num_kv_heads, p.head_dim))
+        for b in range(B):
+            L = int(self.lens[b])
+            if L % P == 0:
+                self.block_table[b, L // P] = self._take_page()
+            page = int(self.block_table[b, L // P])
+            self.k_cache[page, :, L % P, :] = new_k[b]
+            self.v_cache[page, :, L % P, :] = new_v[b]
+            self.lens[b] = L + 1
+        self.q = _randn_bf16(self.gen, (B, p.num_q_heads, p.head_dim))
+        self.step += 1
+        return dict(restarted=restarted, restarted_pages=new_pages, new_k=new_k, new_v=new_v, q=self.q)
+
+    # -- views
+    @property
+    def seq_lens(self) -> np.ndarray:
+        return self.lens.astype(np.int32)
+
+    def workload(self) -> Workload:
+        """The current state as a Workload (host tensors shared, not copied)."""
+        prob = dataclasses.replace(self.problem)
+        return Workload(name=f"trace@{self.step}", problem=prob, seq_lens=self.seq_lens,
+                        block_table=self.block_table.copy(), q=self.q, k_cache=self.k_cache,
+                        v_cache=self.v_cache, seed=self.seed, recipe=self.recipe)
+
+    def kv_bytes(self) -> int:
+        p = self.problem
+        return int(self.lens.sum()) * p.num_kv_heads * p.head_dim * 4
