@@ -378,12 +378,11 @@ def run_trace(args, world, rank, local):
     times = {"dynamic": [], "static": []}
     kv = []
     clocks = ClockSampler(local)
-    with clocks:
+    with clocks, torch.cuda.stream(stream):  # replay() launches on the current stream
         barrier(world)
         for t in range(steps):
             if t > 0:
-                with torch.cuda.stream(stream):
-                    dt.advance(stream=stream)
+                dt.advance(stream=stream)
                 torch.cuda.synchronize()
             kv.append(tr.kv_bytes())
             for key in ("dynamic", "static"):
