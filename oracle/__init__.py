@@ -38,6 +38,7 @@ ERR_CAPACITY = -4
 
 _i32p = ctypes.POINTER(ctypes.c_int32)
 _u16p = ctypes.POINTER(ctypes.c_uint16)
+_u8p = ctypes.POINTER(ctypes.c_uint8)
 _f64p = ctypes.POINTER(ctypes.c_double)
 
 
@@ -71,6 +72,13 @@ def _bind(path: str):
     lib.dao_static_plan.argtypes = plan_args
     lib.dao_num_threads.restype = ctypes.c_int
     lib.dao_num_threads.argtypes = []
+    lib.dao_attention_fp8.restype = ctypes.c_int
+    lib.dao_attention_fp8.argtypes = [
+        ctypes.c_int32, ctypes.c_int32, ctypes.c_int32, ctypes.c_int32, ctypes.c_int32,
+        ctypes.c_int32, ctypes.c_int64, ctypes.c_double, _u16p, _u8p, _u8p, _f64p, _f64p, _i32p, _i32p,
+        ctypes.c_int64, _i32p, _i32p, _f64p, _f64p, ctypes.c_int32]
+    lib.dao_e4m3_value.restype = ctypes.c_double
+    lib.dao_e4m3_value.argtypes = [ctypes.c_uint8]
     return lib
 
 
@@ -153,6 +161,58 @@ def attention(q, k_cache, v_cache, block_table, seq_lens, *, scale: float, num_p
                            None if pb is None else _ptr(pb, ctypes.c_int32),
                            None if ph is None else _ptr(ph, ctypes.c_int32),
                            _ptr(out, ctypes.c_double), _ptr(lse, ctypes.c_double), int(threads))
+    if pairs is None:
+        out = out.reshape(B, Hq, d)
+        lse = lse.reshape(B, Hq)
+    return out, lse, int(st)
+
+
+def _u8(a) -> np.ndarray:
+    """FP8 codes as raw bytes (numpy uint8, C-contiguous)."""
+    if hasattr(a, "dtype") and str(a.dtype).startswith("torch."):
+        import torch  # only for the dtype reinterpretation of CPU tensors
+        a = a.contiguous().view(torch.uint8).numpy()
+    a = np.ascontiguousarray(a)
+    if a.dtype != np.uint8:
+        raise TypeError("fp8 caches must be torch.float8_e4m3fn / uint8 CPU tensors or uint8 arrays")
+    return a
+
+
+def e4m3_value(code: int, lib=None) -> float:
+    """The real number an FP8 E4M3 code stands for (NaN for the NaN codes)."""
+    return float((lib or _load()).dao_e4m3_value(int(code)))
+
+
+def attention_fp8(q, k_code, v_code, k_scale, v_scale, block_table, seq_lens, *, scale: float, pairs=None,
+                  threads: int = 0, lib=None):
+    """fp64 decode attention over an FP8 E4M3 cache with per-KV-head scales (k = k_scale[g] * e4m3(code)).
+
+    Same shapes and results as ``attention``; k_code, v_code are [num_pages, Hkv, P, d] bytes and
+    k_scale, v_scale fp64 [Hkv].
+    """
+    lib = lib or _load()
+    q16, k8, v8 = _u16(q), _u8(k_code), _u8(v_code)
+    ks = np.ascontiguousarray(k_scale, dtype=np.float64)
+    vs = np.ascontiguousarray(v_scale, dtype=np.float64)
+    bt = np.ascontiguousarray(block_table, dtype=np.int32)
+    sl = np.ascontiguousarray(seq_lens, dtype=np.int32)
+    B, Hq, d = q16.shape
+    n_pages, Hkv, P, d2 = k8.shape
+    assert d2 == d and v8.shape == k8.shape and ks.shape == (Hkv,) and vs.shape == (Hkv,)
+    if pairs is None:
+        n, pb, ph = B * Hq, None, None
+    else:
+        pb = np.ascontiguousarray(pairs[0], dtype=np.int32)
+        ph = np.ascontiguousarray(pairs[1], dtype=np.int32)
+        n = pb.shape[0]
+    out = np.empty((n, d), dtype=np.float64)
+    lse = np.empty((n,), dtype=np.float64)
+    st = lib.dao_attention_fp8(B, Hq, Hkv, d, P, bt.shape[1], n_pages, float(scale), _ptr(q16, ctypes.c_uint16),
+                               _ptr(k8, ctypes.c_uint8), _ptr(v8, ctypes.c_uint8), _ptr(ks, ctypes.c_double),
+                               _ptr(vs, ctypes.c_double), _ptr(bt, ctypes.c_int32), _ptr(sl, ctypes.c_int32), n,
+                               None if pb is None else _ptr(pb, ctypes.c_int32),
+                               None if ph is None else _ptr(ph, ctypes.c_int32),
+                               _ptr(out, ctypes.c_double), _ptr(lse, ctypes.c_double), int(threads))
     if pairs is None:
         out = out.reshape(B, Hq, d)
         lse = lse.reshape(B, Hq)

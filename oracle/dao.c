@@ -66,6 +66,22 @@ static double bf16_bits_to_double(uint16_t bits) {
   return (double)f;
 }
 
+/*
+ * An FP8 E4M3 code (OCP 8-bit floating point, "E4M3FN"): 1 sign bit, 4 exponent
+ * bits with bias 7, 3 mantissa bits; exponent 0 is subnormal (m/8 * 2^-6); the
+ * code S.1111.111 is NaN; there are no infinities.  Every code is exact in fp64.
+ */
+static double e4m3_to_double(uint8_t x) {
+  const int sign = x >> 7, e = (x >> 3) & 15, m = x & 7;
+  double mag;
+  if (e == 15 && m == 7) return NAN;
+  if (e == 0) mag = ldexp((double)m, -9);
+  else mag = ldexp((double)(8 + m), e - 10);
+  return sign ? -mag : mag;
+}
+
+double dao_e4m3_value(uint8_t x) { return e4m3_to_double(x); }
+
 /* Length of request b as the method sees it: out-of-range lengths count as 0. */
 static int64_t effective_length(int32_t len, int64_t capacity) {
   if (len < 0 || (int64_t)len > capacity) return 0;
@@ -81,10 +97,28 @@ int dao_num_threads(void) {
 }
 
 /*
+ * K/V element access for the two cache formats: bf16 codes, or FP8 E4M3 codes
+ * times a per-KV-head scale (the value stored for head g is x / scale[g]).
+ */
+typedef struct {
+  int fp8;
+  const void* k;
+  const void* v;
+  const double* k_scale;
+  const double* v_scale;
+} kv_view;
+
+static double kv_elem(const kv_view* kv, int is_v, int64_t index, int32_t g) {
+  if (!kv->fp8) return bf16_bits_to_double(((const uint16_t*)(is_v ? kv->v : kv->k))[index]);
+  const double sc = is_v ? kv->v_scale[g] : kv->k_scale[g];
+  return sc * e4m3_to_double(((const uint8_t*)(is_v ? kv->v : kv->k))[index]);
+}
+
+/*
  * Attention for a list of (request, query head) pairs.
  *
  * q       bf16 bits [batch][num_q_heads][head_dim]
- * k, v    bf16 bits [num_pages][num_kv_heads][page_size][head_dim]
+ * kv      the cache, [num_pages][num_kv_heads][page_size][head_dim] elements
  * out     fp64 [n_pairs][head_dim];  lse fp64 [n_pairs]
  * pair_b, pair_h: the pairs; when pair_b is NULL every (b, h) pair is taken
  * in row-major order (n_pairs must then be batch * num_q_heads).
@@ -93,12 +127,11 @@ int dao_num_threads(void) {
  * out of range).  On a bad length or page the pair's outputs are still
  * written (length treated as 0 / the pair set to NaN respectively).
  */
-int dao_attention(int32_t batch, int32_t num_q_heads, int32_t num_kv_heads, int32_t head_dim,
-                  int32_t page_size, int32_t max_pages_per_req, int64_t num_pages, double scale,
-                  const uint16_t* q, const uint16_t* k, const uint16_t* v,
-                  const int32_t* block_table, const int32_t* seq_lens, int64_t n_pairs,
-                  const int32_t* pair_b, const int32_t* pair_h, double* out, double* lse,
-                  int32_t num_threads) {
+static int attention_impl(int32_t batch, int32_t num_q_heads, int32_t num_kv_heads, int32_t head_dim,
+                          int32_t page_size, int32_t max_pages_per_req, int64_t num_pages, double scale,
+                          const uint16_t* q, const kv_view* kv, const int32_t* block_table,
+                          const int32_t* seq_lens, int64_t n_pairs, const int32_t* pair_b, const int32_t* pair_h,
+                          double* out, double* lse, int32_t num_threads) {
   if (batch < 0 || num_q_heads <= 0 || num_kv_heads <= 0 || head_dim <= 0 || page_size <= 0 ||
       max_pages_per_req < 0 || num_pages < 0 || num_q_heads % num_kv_heads != 0)
     return DAO_ERR_ARG;
@@ -141,9 +174,9 @@ int dao_attention(int32_t batch, int32_t num_q_heads, int32_t num_kv_heads, int3
     for (int64_t t = 0; t < len; ++t) {
       const int32_t page = block_table[(int64_t)b * max_pages_per_req + t / page_size];
       if (page < 0 || (int64_t)page >= num_pages) { bad_page = 1; break; }
-      const uint16_t* kt = k + (((int64_t)page * num_kv_heads + g) * page_size + t % page_size) * head_dim;
+      const int64_t kt = (((int64_t)page * num_kv_heads + g) * page_size + t % page_size) * head_dim;
       double dot = 0.0;
-      for (int32_t j = 0; j < head_dim; ++j) dot += bf16_bits_to_double(qh[j]) * bf16_bits_to_double(kt[j]);
+      for (int32_t j = 0; j < head_dim; ++j) dot += bf16_bits_to_double(qh[j]) * kv_elem(kv, 0, kt + j, g);
       s[t] = scale * dot;
     }
     if (bad_page) {
@@ -162,14 +195,40 @@ int dao_attention(int32_t batch, int32_t num_q_heads, int32_t num_kv_heads, int3
     /* Pass 3: out = sum_t exp(s_t - M) v_t / l. */
     for (int64_t t = 0; t < len; ++t) {
       const int32_t page = block_table[(int64_t)b * max_pages_per_req + t / page_size];
-      const uint16_t* vt = v + (((int64_t)page * num_kv_heads + g) * page_size + t % page_size) * head_dim;
+      const int64_t vt = (((int64_t)page * num_kv_heads + g) * page_size + t % page_size) * head_dim;
       const double w = exp(s[t] - m) / l;
-      for (int32_t j = 0; j < head_dim; ++j) o[j] += w * bf16_bits_to_double(vt[j]);
+      for (int32_t j = 0; j < head_dim; ++j) o[j] += w * kv_elem(kv, 1, vt + j, g);
     }
     lse[i] = m + log(l);
     free(s);
   }
   return status;
+}
+
+int dao_attention(int32_t batch, int32_t num_q_heads, int32_t num_kv_heads, int32_t head_dim,
+                  int32_t page_size, int32_t max_pages_per_req, int64_t num_pages, double scale,
+                  const uint16_t* q, const uint16_t* k, const uint16_t* v,
+                  const int32_t* block_table, const int32_t* seq_lens, int64_t n_pairs,
+                  const int32_t* pair_b, const int32_t* pair_h, double* out, double* lse,
+                  int32_t num_threads) {
+  const kv_view kv = {0, k, v, NULL, NULL};
+  return attention_impl(batch, num_q_heads, num_kv_heads, head_dim, page_size, max_pages_per_req, num_pages,
+                        scale, q, &kv, block_table, seq_lens, n_pairs, pair_b, pair_h, out, lse, num_threads);
+}
+
+/*
+ * Same, for an FP8 E4M3 cache: k_code, v_code [num_pages][Hkv][P][d] one byte
+ * each, dequantised as k = k_scale[g] * e4m3(k_code) (per KV head g).
+ */
+int dao_attention_fp8(int32_t batch, int32_t num_q_heads, int32_t num_kv_heads, int32_t head_dim,
+                      int32_t page_size, int32_t max_pages_per_req, int64_t num_pages, double scale,
+                      const uint16_t* q, const uint8_t* k_code, const uint8_t* v_code, const double* k_scale,
+                      const double* v_scale, const int32_t* block_table, const int32_t* seq_lens,
+                      int64_t n_pairs, const int32_t* pair_b, const int32_t* pair_h, double* out, double* lse,
+                      int32_t num_threads) {
+  const kv_view kv = {1, k_code, v_code, k_scale, v_scale};
+  return attention_impl(batch, num_q_heads, num_kv_heads, head_dim, page_size, max_pages_per_req, num_pages,
+                        scale, q, &kv, block_table, seq_lens, n_pairs, pair_b, pair_h, out, lse, num_threads);
 }
 
 /*

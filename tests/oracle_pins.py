@@ -278,9 +278,82 @@ def pin_pairs_match_full(lib=None):
     assert np.array_equal(sub, full[pb, ph]) and np.array_equal(sub_lse, full_lse[pb, ph])
 
 
+# ---------------------------------------------------------------------------------------------
+# FP8 (E4M3) cache pins.
+
+
+def random_fp8_case(rng, B, Hq, Hkv, d, P, lens, k_scale, v_scale):
+    """Random E4M3 codes (NaN codes excluded) laid out in shuffled pages, plus the dequantised dense K/V."""
+    n_pages = sum(-(-L // P) for L in lens) + 2
+    codes = rng.integers(0, 256, size=(2, n_pages, Hkv, P, d), dtype=np.uint8)
+    codes[(codes & 0x7F) == 0x7F] = 0x3C  # avoid the NaN codes
+    perm = rng.permutation(n_pages)
+    mp = max(1, max(-(-L // P) for L in lens))
+    bt = np.full((B, mp), -1, np.int32)
+    o = 0
+    for b, L in enumerate(lens):
+        n = -(-L // P)
+        bt[b, :n] = perm[o:o + n]
+        o += n
+    deq = torch.from_numpy(codes).view(torch.float8_e4m3fn).to(torch.float64)
+    deq[0] *= torch.tensor(k_scale, dtype=torch.float64)[None, :, None, None]
+    deq[1] *= torch.tensor(v_scale, dtype=torch.float64)[None, :, None, None]
+    dense = []
+    for b, L in enumerate(lens):
+        t = np.arange(L)
+        pages, slots = bt[b, t // P], t % P
+        dense.append((deq[0][pages, :, slots, :], deq[1][pages, :, slots, :]))  # [L, Hkv, d]
+    q = bf16(rng.standard_normal((B, Hq, d)))
+    return q, codes[0], codes[1], bt, np.array(lens, np.int32), dense
+
+
+def pin_e4m3_decoding(lib=None):
+    """All 256 E4M3 codes against torch's float8_e4m3fn conversion."""
+    ref = torch.arange(256, dtype=torch.uint8).view(torch.float8_e4m3fn).to(torch.float64)
+    for c in range(256):
+        v = oracle.e4m3_value(c, lib=lib)
+        r = float(ref[c])
+        assert (math.isnan(v) and math.isnan(r)) or v == r, (c, v, r)
+
+
+def pin_fp8_matches_sdpa(lib=None):
+    rng = np.random.default_rng(22)
+    B, Hq, Hkv, d, P, lens = 3, 8, 2, 64, 16, [1, 40, 97]
+    ks, vs = [0.013, 0.002], [0.5, 0.07]
+    q, kc, vc, bt, sl, dense = random_fp8_case(rng, B, Hq, Hkv, d, P, lens, ks, vs)
+    scale = 0.125
+    out, lse, st = oracle.attention_fp8(q, kc, vc, ks, vs, bt, sl, scale=scale, lib=lib)
+    assert st == oracle.OK
+    for b in range(B):
+        kb = dense[b][0].permute(1, 0, 2).unsqueeze(0)
+        vb = dense[b][1].permute(1, 0, 2).unsqueeze(0)
+        qb = q[b].double().unsqueeze(0).unsqueeze(2)
+        ref = torch.nn.functional.scaled_dot_product_attention(qb, kb, vb, scale=scale, enable_gqa=True)
+        np.testing.assert_allclose(out[b], ref[0, :, 0].numpy(), rtol=1e-11, atol=1e-12)
+        s = torch.einsum("hd,htd->ht", qb[0, :, 0], kb.repeat_interleave(Hq // Hkv, dim=1)[0]) * scale
+        np.testing.assert_allclose(lse[b], torch.logsumexp(s, dim=1).numpy(), rtol=1e-12, atol=1e-12)
+
+
+def pin_fp8_equals_bf16_when_exact(lib=None):
+    """With power-of-two scales every dequantised value is exact in bf16: both formats give the same bits."""
+    rng = np.random.default_rng(23)
+    B, Hq, Hkv, d, P, lens = 2, 4, 2, 32, 8, [9, 30]
+    ks, vs = [0.125, 4.0], [2.0 ** -6, 1.0]
+    q, kc, vc, bt, sl, _ = random_fp8_case(rng, B, Hq, Hkv, d, P, lens, ks, vs)
+    deq = lambda c, sc: (torch.from_numpy(c).view(torch.float8_e4m3fn).to(torch.float64)
+                         * torch.tensor(sc, dtype=torch.float64)[None, :, None, None])
+    kb, vb = deq(kc, ks).to(torch.bfloat16), deq(vc, vs).to(torch.bfloat16)
+    assert torch.equal(kb.double(), deq(kc, ks)) and torch.equal(vb.double(), deq(vc, vs))
+    a = oracle.attention_fp8(q, kc, vc, ks, vs, bt, sl, scale=0.3, lib=lib)
+    b = oracle.attention(q, kb, vb, bt, sl, scale=0.3, lib=lib)
+    assert a[2] == b[2] == oracle.OK
+    assert np.array_equal(a[0], b[0]) and np.array_equal(a[1], b[1])
+
+
 ATTENTION_PINS = [pin_golden_attention, pin_length_one, pin_constant_v, pin_uniform_scores, pin_dominant_key,
                   pin_page_order_invariance, pin_prefix_sharing, pin_matches_sdpa, pin_split_merge_identity,
-                  pin_degenerate_lengths, pin_pairs_match_full]
+                  pin_degenerate_lengths, pin_pairs_match_full, pin_e4m3_decoding, pin_fp8_matches_sdpa,
+                  pin_fp8_equals_bf16_when_exact]
 
 
 # ---------------------------------------------------------------------------------------------

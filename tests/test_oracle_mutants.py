@@ -16,11 +16,16 @@ MUTANTS = [
     ("gqa head mapping", "const int32_t g = h / group;", "const int32_t g = h % num_kv_heads;"),
     ("score without scale", "s[t] = scale * dot;", "s[t] = dot;"),
     ("query head index", "q + ((int64_t)b * num_q_heads + h) * head_dim", "q + ((int64_t)b * num_q_heads + 0) * head_dim"),
-    ("page slot of K", "(((int64_t)page * num_kv_heads + g) * page_size + t % page_size) * head_dim;\n      double dot",
-     "(((int64_t)page * num_kv_heads + g) * page_size + (t + 1) % page_size) * head_dim;\n      double dot"),
-    ("kv head stride of V", "const uint16_t* vt = v + (((int64_t)page * num_kv_heads + g)",
-     "const uint16_t* vt = v + (((int64_t)page * num_kv_heads + 0)"),
-    ("V read from K", "const uint16_t* vt = v +", "const uint16_t* vt = k +"),
+    ("page slot of K", "const int64_t kt = (((int64_t)page * num_kv_heads + g) * page_size + t % page_size)",
+     "const int64_t kt = (((int64_t)page * num_kv_heads + g) * page_size + (t + 1) % page_size)"),
+    ("kv head stride of V", "const int64_t vt = (((int64_t)page * num_kv_heads + g)",
+     "const int64_t vt = (((int64_t)page * num_kv_heads + 0)"),
+    ("V read from K", "o[j] += w * kv_elem(kv, 1, vt + j, g);", "o[j] += w * kv_elem(kv, 0, vt + j, g);"),
+    ("fp8 exponent bias", "else mag = ldexp((double)(8 + m), e - 10);", "else mag = ldexp((double)(8 + m), e - 11);"),
+    ("fp8 subnormal step", "if (e == 0) mag = ldexp((double)m, -9);", "if (e == 0) mag = ldexp((double)m, -10);"),
+    ("fp8 V scaled by K's scale", "const double sc = is_v ? kv->v_scale[g] : kv->k_scale[g];",
+     "const double sc = kv->k_scale[g];"),
+    ("fp8 scale ignored", "return sc * e4m3_to_double(", "return e4m3_to_double("),
     ("block table row", "block_table[(int64_t)b * max_pages_per_req + t / page_size];\n      if",
      "block_table[(int64_t)b + t / page_size];\n      if"),
     ("lse without max", "lse[i] = m + log(l);", "lse[i] = log(l);"),
