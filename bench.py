@@ -51,6 +51,7 @@ def parse_args():
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--config", default="mixed", choices=["mixed", "skewed", "low_conc", "uniform", "tiny", "trace"])
+    ap.add_argument("--kv", choices=["bf16", "fp8"], default="bf16", help="KV cache format")
     ap.add_argument("--tile", type=int, default=64)
     ap.add_argument("--width", type=int, default=0, help="CTAs per KV head (0 = 2 per SM / Hkv)")
     ap.add_argument("--no-static", action="store_true", help="skip the static split-k comparison")
@@ -221,16 +222,27 @@ def run_ours(args, world, rank, local):
     seed_shift = 1000 * rank
     gen = W.CONFIGS[args.config]
     w = gen(seed=gen.__defaults__[0] + seed_shift) if rank else gen()
-    dw = w.to("cuda")
+    w8 = W.quantize_fp8(w) if args.kv == "fp8" else None
+    dw = w8.to("cuda") if w8 is not None else w.to("cuda")
     prob = da.problem_from(dw.problem)
     desc = da.da_plan_desc_init(prob, da.PLAN_DYNAMIC, args.tile, args.width)
     bufs = da.Buffers(prob, desc, "cuda")
-    kv_bytes = w.kv_bytes
+    kv_bytes = w8.kv_bytes if w8 is not None else w.kv_bytes
     stream = torch.cuda.Stream()
     steps, warm = max(1, args.steps), max(3, args.warmup)
 
     def step(d=desc, b=bufs):
-        da.decode_step(prob, d, dw.q, dw.k_cache, dw.v_cache, dw.block_table, dw.seq_lens, b, stream=stream)
+        da.decode_step(prob, d, dw.q, dw.k_cache, dw.v_cache, dw.block_table, dw.seq_lens, b, stream=stream,
+                       k_scale=dw.k_scale, v_scale=dw.v_scale)
+
+    def decode_only(d=desc, b=bufs):
+        if w8 is None:
+            da.da_decode_attention(prob, d, dw.q, dw.k_cache, dw.v_cache, dw.block_table, dw.seq_lens, b.ws,
+                                   b.partial_o, b.partial_lse, b.out, b.lse, stream=stream)
+        else:
+            da.da_decode_attention_fp8(prob, d, dw.q, dw.k_cache, dw.v_cache, dw.k_scale, dw.v_scale,
+                                       dw.block_table, dw.seq_lens, b.ws, b.partial_o, b.partial_lse, b.out, b.lse,
+                                       stream=stream)
 
     result = {}
     clocks = ClockSampler(local)
@@ -256,8 +268,7 @@ def run_ours(args, world, rank, local):
             for a, b in ev:
                 da.da_plan(prob, desc, dw.seq_lens, bufs.ws, stream=stream)
                 a.record(stream)
-                da.da_decode_attention(prob, desc, dw.q, dw.k_cache, dw.v_cache, dw.block_table, dw.seq_lens,
-                                       bufs.ws, bufs.partial_o, bufs.partial_lse, bufs.out, bufs.lse, stream=stream)
+                decode_only()
                 b.record(stream)
                 da.da_combine(prob, desc, bufs.ws, bufs.partial_o, bufs.partial_lse, bufs.out, bufs.lse,
                               stream=stream)
@@ -310,12 +321,13 @@ def run_ours(args, world, rank, local):
     value = total_bytes / step_s / 1e9
     peak, peak_src = measured_peak()
     dec_gbs = kv_bytes / (dec_avg_ms / 1e3) / 1e9
-    traffic, traffic_note = recorded_traffic(args.config)
+    traffic, traffic_note = recorded_traffic(args.config) if args.kv == "bf16" else (None, "no ncu capture for fp8")
     result.update(
         metric=METRIC, value=round(value, 2), unit="GB/s", n_gpus=world, steps=steps, warmup=warm,
         ms_per_step=round(ms_graph / steps, 5), us_per_step=round(ms_graph / steps * 1e3, 2),
         higher_is_better=True, scaling="weak", vs_baseline=None, dtype="bf16", data="synthetic",
-        config={"workload": f"{args.config}: {w.recipe}", "batch": w.problem.batch,
+        config={"workload": f"{args.config}: {w.recipe}" + ("; FP8 E4M3 KV, per-head scales" if w8 else ""),
+                "batch": w.problem.batch, "kv_format": args.kv,
                 "kv_bytes_per_step_per_gpu": kv_bytes, "tile_tokens": desc.tile_tokens,
                 "ctas_per_kv_head": desc.num_ctas, "graph": True,
                 "l2": "inputs larger than L2 (K/V read per step >> 126 MB), no flush"},
@@ -323,7 +335,8 @@ def run_ours(args, world, rank, local):
         eager_us_per_step=round(ms_eager / steps * 1e3, 2),
         roofline={"bound": "hbm", "achieved": round(dec_gbs, 2), "peak": peak, "unit": "GB/s",
                   "frac": round(dec_gbs / peak, 4), "traffic": traffic,
-                  "kernel": f"decode_kernel<{w.problem.head_dim}>", "algorithmic_bytes_per_launch": kv_bytes,
+                  "kernel": f"decode_kernel<{w.problem.head_dim},{'fp8' if w8 else 'bf16'}>",
+                  "algorithmic_bytes_per_launch": kv_bytes,
                   "launch_us": round(dec_avg_ms * 1e3, 2), "peak_source": peak_src, "traffic_source": traffic_note},
         e2e={"value": round(total_bytes / (ms_e2e / 1e3 / steps) / 1e9, 2), "unit": "GB/s",
              "us_per_step": round(ms_e2e / steps * 1e3, 2), "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
@@ -339,7 +352,7 @@ def run_ours(args, world, rank, local):
         result["speedup_vs_static_best"] = round(static[best_S] / (ms_graph / steps), 3)
     result["clocks"] = clocks.summary()
     if rank == 0 and world == 1 and not args.no_cpu:
-        result["cpu_baseline"] = cpu_baseline(w, args.cpu_seconds)
+        result["cpu_baseline"] = cpu_baseline(w, args.cpu_seconds, w8)
     return result
 
 
@@ -417,19 +430,26 @@ def run_trace(args, world, rank, local):
         append_status=dt.status.tolist(), clocks=clocks.summary())
 
 
-def cpu_baseline(w, seconds):
+def cpu_baseline(w, seconds, w8=None):
     """The CPU oracle (fp64) on this host's cores, repeated over the full batch for a bounded time."""
+    import numpy as np
+
     import oracle
     oracle.build()
     t0 = time.perf_counter()
     passes = 0
     while True:
-        oracle.attention(w.q, w.k_cache, w.v_cache, w.block_table, w.seq_lens, scale=w.problem.scale)
+        if w8 is None:
+            oracle.attention(w.q, w.k_cache, w.v_cache, w.block_table, w.seq_lens, scale=w.problem.scale)
+        else:
+            oracle.attention_fp8(w.q, w8.k_code, w8.v_code, w8.k_scale.astype(np.float64),
+                                 w8.v_scale.astype(np.float64), w.block_table, w.seq_lens, scale=w.problem.scale)
         passes += 1
         if time.perf_counter() - t0 >= seconds or passes >= 50:
             break
     dt = time.perf_counter() - t0
-    return {"value": round(passes * w.kv_bytes / dt / 1e9, 4), "unit": "GB/s", "cores": oracle.num_threads(),
+    kv = w8.kv_bytes if w8 is not None else w.kv_bytes
+    return {"value": round(passes * kv / dt / 1e9, 4), "unit": "GB/s", "cores": oracle.num_threads(),
             "kind": "oracle", "sample": f"{passes} pass(es) of the fp64 oracle over the full batch "
                                         f"({w.problem.batch} requests x {w.problem.num_q_heads} heads), {dt:.1f} s"}
 

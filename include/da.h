@@ -204,6 +204,28 @@ DA_API int da_decode_attention(const da_problem* prob, const da_plan_desc* desc,
                                void* out, float* lse, void* stream);
 
 /*
+ * da_decode_attention_fp8 -- the same step over an FP8 KV cache.
+ *   k_cache, v_cache  dev, FP8 E4M3 codes (OCP "E4M3FN", one byte each),
+ *                     [num_pages][num_kv_heads][page_size][head_dim]; head_dim must be 128.
+ *   k_scale, v_scale  dev fp32 [num_kv_heads]: the cached value of KV head g is
+ *                     k_scale[g] * e4m3(code) (and likewise for V).
+ * Everything else, including the plan, workspace, partials, combine and the
+ * bf16 q/out and fp32 lse, is as for da_decode_attention.  K/V bytes per token
+ * are halved.  Codes are widened to f16 (exact), q is converted to f16 (exact
+ * for normal-range values), and P is rounded to f16 for the P.V product.
+ * Source: "Tencent HPC lands in SGLang, challenging default inference
+ * kernels", sections "Why Tencent HPC matters for online model serving" (a
+ * longer history means more cached data to read) and "What the 48.8% TPOT
+ * claim does not prove" (cache precision is one of the settings a benchmark
+ * must state).
+ */
+DA_API int da_decode_attention_fp8(const da_problem* prob, const da_plan_desc* desc, const void* q,
+                                   const void* k_cache, const void* v_cache, const float* k_scale,
+                                   const float* v_scale, const int32_t* block_table, const int32_t* seq_lens,
+                                   const void* ws, float* partial_o, float* partial_lse, void* out, float* lse,
+                                   void* stream);
+
+/*
  * da_combine -- merge the partials of requests with two or more segments:
  *   LSE = M + ln sum_i exp(lse_i - M),  M = max_i lse_i,
  *   out = sum_i exp(lse_i - LSE) o_i    (fp32 sums in a fixed order, then bf16),

@@ -71,3 +71,38 @@ def assert_plan_equal(gpu: dict, ref: dict):
                 "seg_tile_end"):
         assert np.array_equal(np.asarray(gpu[key]), np.asarray(ref[key])), key
     assert gpu["bad_index"] == ref["bad_index"]
+
+
+def run_step_fp8(w8: W.Fp8Workload, kind=da.PLAN_DYNAMIC, tile=64, width=0, dw=None):
+    """FP8-cache step on cuda:0 (same contract as run_step)."""
+    dw = dw if dw is not None else w8.to("cuda")
+    prob = da.problem_from(dw.problem)
+    desc = da.da_plan_desc_init(prob, kind, tile, width)
+    bufs = da.Buffers(prob, desc, "cuda")
+    for t in (bufs.partial_o, bufs.partial_lse, bufs.out, bufs.lse):
+        t.fill_(float("nan"))
+    da.decode_step(prob, desc, dw.q, dw.k_cache, dw.v_cache, dw.block_table, dw.seq_lens, bufs,
+                   k_scale=dw.k_scale, v_scale=dw.v_scale)
+    torch.cuda.synchronize()
+    return bufs.out, bufs.lse, desc, bufs, dw
+
+
+def check_against_oracle_fp8(w8: W.Fp8Workload, out, lse, pairs=None):
+    b = w8.base
+    ref, ref_lse, st = oracle.attention_fp8(b.q, w8.k_code, w8.v_code, w8.k_scale.astype(np.float64),
+                                            w8.v_scale.astype(np.float64), b.block_table, b.seq_lens,
+                                            scale=b.problem.scale, pairs=pairs)
+    o = out.float().cpu().double().numpy()
+    l = lse.cpu().double().numpy()
+    if pairs is not None:
+        o, l = o[pairs[0], pairs[1]], l[pairs[0], pairs[1]]
+    assert np.all(np.isfinite(o)), "non-finite output"
+    err = np.abs(o - ref)
+    bound = OUT_ATOL + OUT_RTOL * np.abs(ref)
+    worst = np.unravel_index(np.argmax(err - bound), err.shape)
+    assert np.all(err <= bound), f"out mismatch at {worst}: gpu {o[worst]} ref {ref[worst]}"
+    both_inf = np.isneginf(l) & np.isneginf(ref_lse)
+    with np.errstate(invalid="ignore"):
+        lerr = np.where(both_inf, 0.0, np.abs(l - ref_lse))
+    assert np.all(lerr <= LSE_ATOL), f"lse mismatch: max err {np.nanmax(lerr)}"
+    return float(err.max()), float(lerr.max())

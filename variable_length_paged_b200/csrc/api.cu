@@ -77,19 +77,20 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
   return fn;
 }
 
-// 2-D bf16 view of a cache: x = head_dim (inner), y = (page, kv head, slot) rows.
-// Box = 64 columns (128 bytes, the 128-byte swizzle span) x box_rows rows.
-bool make_cache_map(CUtensorMap* map, const void* base, const da_problem* p, int box_rows) {
+// 2-D view of a cache: x = head_dim (inner), y = (page, kv head, slot) rows.
+// Box = 128 bytes of columns (the 128-byte swizzle span) x box_rows rows;
+// elements are bf16 (2 bytes) or FP8 codes (1 byte).
+bool make_cache_map(CUtensorMap* map, const void* base, const da_problem* p, int box_rows, int elem_bytes) {
   PFN_cuTensorMapEncodeTiled_v12000 enc = encode_fn();
   if (!enc) return false;
   cuuint64_t dims[2] = {(cuuint64_t)p->head_dim,
                         (cuuint64_t)p->num_pages * (cuuint64_t)p->num_kv_heads * (cuuint64_t)p->page_size};
-  cuuint64_t strides[1] = {(cuuint64_t)p->head_dim * 2};
-  cuuint32_t box[2] = {64u, (cuuint32_t)box_rows};
+  cuuint64_t strides[1] = {(cuuint64_t)p->head_dim * (cuuint64_t)elem_bytes};
+  cuuint32_t box[2] = {(cuuint32_t)(128 / elem_bytes), (cuuint32_t)box_rows};
   cuuint32_t estr[2] = {1u, 1u};
-  CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
-                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  CUresult r = enc(map, elem_bytes == 2 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_UINT8, 2,
+                   const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                   CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;
 }
 
@@ -219,26 +220,31 @@ DA_API int da_static_plan(const da_problem* prob, const da_plan_desc* desc, cons
   return plan_common(prob, desc, seq_lens, ws, ws_bytes, stream, DA_PLAN_STATIC);
 }
 
-DA_API int da_decode_attention(const da_problem* prob, const da_plan_desc* desc, const void* q,
-                               const void* k_cache, const void* v_cache, const int32_t* block_table,
-                               const int32_t* seq_lens, const void* ws, float* partial_o, float* partial_lse,
-                               void* out, float* lse, void* stream) {
+static int decode_common(const da_problem* prob, const da_plan_desc* desc, const void* q, const void* k_cache,
+                         const void* v_cache, const float* k_scale, const float* v_scale,
+                         const int32_t* block_table, const int32_t* seq_lens, const void* ws, float* partial_o,
+                         float* partial_lse, void* out, float* lse, void* stream, bool fp8) {
   int rc = check_problem(prob);
   if (rc != DA_OK) return rc;
   rc = check_desc(prob, desc);
   if (rc != DA_OK) return rc;
+  if (fp8 && prob->head_dim != 128) return DA_ERR_UNSUPPORTED;
   if (prob->batch == 0) return DA_OK;
   if (!q || !k_cache || !v_cache || !block_table || !seq_lens || !ws || !partial_o || !partial_lse || !out || !lse)
     return DA_ERR_INVALID_ARG;
+  if (fp8 && (!k_scale || !v_scale)) return DA_ERR_INVALID_ARG;
   if (reinterpret_cast<uintptr_t>(k_cache) % 16 != 0 || reinterpret_cast<uintptr_t>(v_cache) % 16 != 0 ||
-      reinterpret_cast<uintptr_t>(q) % 4 != 0 || reinterpret_cast<uintptr_t>(out) % 4 != 0 ||
+      reinterpret_cast<uintptr_t>(q) % (fp8 ? 8 : 4) != 0 || reinterpret_cast<uintptr_t>(out) % 8 != 0 ||
       reinterpret_cast<uintptr_t>(partial_o) % 16 != 0 || reinterpret_cast<uintptr_t>(ws) % 16 != 0)
     return DA_ERR_INVALID_ARG;
+  const int eb = fp8 ? 1 : 2;
   CUtensorMap maps[4];
-  if (!make_cache_map(&maps[0], k_cache, prob, 64) || !make_cache_map(&maps[1], v_cache, prob, 64) ||
-      !make_cache_map(&maps[2], k_cache, prob, 16) || !make_cache_map(&maps[3], v_cache, prob, 16))
+  if (!make_cache_map(&maps[0], k_cache, prob, 64, eb) || !make_cache_map(&maps[1], v_cache, prob, 64, eb) ||
+      !make_cache_map(&maps[2], k_cache, prob, 16, eb) || !make_cache_map(&maps[3], v_cache, prob, 16, eb))
     return cuda_fail(cudaErrorInvalidValue);
   da::DecodeParams p;
+  p.k_scale = k_scale;
+  p.v_scale = v_scale;
   p.q = static_cast<const __nv_bfloat16*>(q);
   p.block_table = block_table;
   p.seq_lens = seq_lens;
@@ -260,8 +266,26 @@ DA_API int da_decode_attention(const da_problem* prob, const da_plan_desc* desc,
   p.kind = desc->kind;
   p.capacity_tokens = (int64_t)prob->max_pages_per_req * prob->page_size;
   p.scale_log2 = prob->scale * 1.4426950408889634f;
-  cudaError_t e = da::launch_decode(p, prob->head_dim, maps, static_cast<cudaStream_t>(stream));
+  cudaError_t e = fp8 ? da::launch_decode_fp8(p, prob->head_dim, maps, static_cast<cudaStream_t>(stream))
+                      : da::launch_decode(p, prob->head_dim, maps, static_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? DA_OK : cuda_fail(e);
+}
+
+DA_API int da_decode_attention(const da_problem* prob, const da_plan_desc* desc, const void* q,
+                               const void* k_cache, const void* v_cache, const int32_t* block_table,
+                               const int32_t* seq_lens, const void* ws, float* partial_o, float* partial_lse,
+                               void* out, float* lse, void* stream) {
+  return decode_common(prob, desc, q, k_cache, v_cache, nullptr, nullptr, block_table, seq_lens, ws, partial_o,
+                       partial_lse, out, lse, stream, false);
+}
+
+DA_API int da_decode_attention_fp8(const da_problem* prob, const da_plan_desc* desc, const void* q,
+                                   const void* k_cache, const void* v_cache, const float* k_scale,
+                                   const float* v_scale, const int32_t* block_table, const int32_t* seq_lens,
+                                   const void* ws, float* partial_o, float* partial_lse, void* out, float* lse,
+                                   void* stream) {
+  return decode_common(prob, desc, q, k_cache, v_cache, k_scale, v_scale, block_table, seq_lens, ws, partial_o,
+                       partial_lse, out, lse, stream, true);
 }
 
 DA_API int da_combine(const da_problem* prob, const da_plan_desc* desc, const void* ws, const float* partial_o,

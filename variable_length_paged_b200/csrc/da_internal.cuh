@@ -68,6 +68,8 @@ struct DecodeParams {
   int32_t tile_tokens, num_ctas, max_segments, kind;
   int64_t capacity_tokens;
   float scale_log2;  // scale * log2(e): scores are kept in base-2 units
+  const float* k_scale;  // FP8 caches: per-KV-head dequantisation scales (else null)
+  const float* v_scale;
 };
 
 struct CombineParams {
@@ -95,6 +97,7 @@ struct AppendParams {
 cudaError_t launch_plan_dynamic(const PlanParams& p, cudaStream_t stream);
 cudaError_t launch_plan_static(const PlanParams& p, cudaStream_t stream);
 cudaError_t launch_decode(const DecodeParams& p, int head_dim, const CUtensorMap maps[4], cudaStream_t stream);
+cudaError_t launch_decode_fp8(const DecodeParams& p, int head_dim, const CUtensorMap maps[4], cudaStream_t stream);
 cudaError_t launch_combine(const CombineParams& p, int head_dim, cudaStream_t stream);
 cudaError_t launch_append(const AppendParams& p, cudaStream_t stream);
 
@@ -201,6 +204,17 @@ __device__ __forceinline__ void mma_bf16_upper(float& d0, float& d1, uint32_t a0
   float d2 = 0.f, d3 = 0.f;  // rows 8..15 of the tile: A is zero there
   asm volatile(
       "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, "
+      "{%0, %1, %2, %3};"
+      : "+f"(d0), "+f"(d1), "+f"(d2), "+f"(d3)
+      : "r"(a0), "r"(0u), "r"(a2), "r"(0u), "r"(b0), "r"(b1));
+}
+
+// Same with f16 operands (FP8 caches are widened to f16, exactly).
+__device__ __forceinline__ void mma_f16_upper(float& d0, float& d1, uint32_t a0, uint32_t a2, uint32_t b0,
+                                              uint32_t b1) {
+  float d2 = 0.f, d3 = 0.f;
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, "
       "{%0, %1, %2, %3};"
       : "+f"(d0), "+f"(d1), "+f"(d2), "+f"(d3)
       : "r"(a0), "r"(0u), "r"(a2), "r"(0u), "r"(b0), "r"(b1));

@@ -25,10 +25,21 @@
 //             log-sum-exp through shared memory; the result goes to out/lse
 //             (request with one segment) or to the segment's partial slot.
 //
+// Two cache formats share the kernel.  bf16: K/V rows feed a bf16 MMA directly.
+// FP8 (E4M3 codes with one scale per KV head for K and for V): rows are half as
+// wide (one 128-byte swizzle span at head_dim 128); K and V bytes are widened
+// to f16 in registers (exact for every E4M3 value), q is converted bf16 -> f16
+// (exact for normal-range values), P is rounded to f16, the MMA is f16 with
+// fp32 accumulation, and the K scale is folded into the score scale and the V
+// scale into the final normalisation.
+//
 // Scores are kept in base-2 units (scale * log2 e), so exp is one ex2 and the
 // natural-log lse is (m + log2 l) * ln 2.  Tokens past the end of a request
 // inside a loaded chunk are masked to -inf; their V rows are zeroed in shared
 // memory first, since unused cache slots may hold anything (NaN included).
+#include <cuda_fp16.h>
+#include <cuda_fp8.h>
+
 #include <cfloat>
 
 #include "da_internal.cuh"
@@ -41,13 +52,20 @@ constexpr int kConsumerWarps = 4;
 constexpr int kThreads = (kConsumerWarps + 1) * 32;
 constexpr uint64_t kWaitLimitNs = 2000000000ull;  // 2 s: far beyond any legitimate wait
 
-template <int D>
+template <int D, bool FP8>
 struct Cfg {
-  static constexpr int kHalves = D / 64;                 // 128-byte column blocks per row
+  static constexpr int kElemBytes = FP8 ? 1 : 2;
+  static constexpr int kRowBytes = D * kElemBytes;
+  static_assert(kRowBytes % 128 == 0, "a row must be whole 128-byte swizzle spans");
+  static constexpr int kHalves = kRowBytes / 128;            // 128-byte column blocks per row
+  static constexpr int kBoxCols = 128 / kElemBytes;          // elements per TMA box row
   static constexpr int kTileBytes = kHalves * kChunk * 128;  // one K (or V) chunk
   static constexpr int kStageBytes = 2 * kTileBytes;
-  static constexpr int kStages = D == 128 ? 3 : 6;
-  static constexpr int kSlotStride = D + 8;              // floats per head row in a merge slot
+  static constexpr int kStages = (96 * 1024) / kStageBytes;  // a 96 KB ring per CTA
+  // per-thread output columns: NG groups of GW consecutive columns, group gi at gi*4*GW + GW*tq
+  static constexpr int kGW = FP8 ? 4 : 2;
+  static constexpr int kNG = D / (4 * kGW);
+  static constexpr int kSlotStride = D + (FP8 ? 16 : 8);     // floats per head row (bank-conflict free)
   static constexpr int kSlotFloats = 8 * kSlotStride;
   // shared memory map (offsets from a 1024-byte aligned base)
   static constexpr int kOffStages = 0;
@@ -65,6 +83,21 @@ struct Cfg {
 __device__ __forceinline__ uint32_t swz(int row, int chunk) {
   return (uint32_t)((chunk >> 3) * (kChunk * 128) + row * 128 + (((chunk & 7) ^ (row & 7)) << 4));
 }
+
+// Two E4M3 codes (low byte first) -> f16x2 (low half first); exact.
+__device__ __forceinline__ uint32_t e4m3x2_to_f16x2(uint32_t two_codes) {
+  const __half2_raw h = __nv_cvt_fp8x2_to_halfraw2(static_cast<__nv_fp8x2_storage_t>(two_codes & 0xFFFFu), __NV_E4M3);
+  return static_cast<uint32_t>(h.x) | (static_cast<uint32_t>(h.y) << 16);
+}
+
+__device__ __forceinline__ uint32_t pack_f16x2(float lo, float hi) {
+  uint32_t r;
+  asm("cvt.rn.f16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
+  return r;
+}
+
+__device__ __forceinline__ float f16_lo_to_f32(uint32_t v) { return __half2float(__ushort_as_half((unsigned short)(v & 0xFFFFu))); }
+__device__ __forceinline__ float f16_hi_to_f32(uint32_t v) { return __half2float(__ushort_as_half((unsigned short)(v >> 16))); }
 
 struct SegmentInfo {
   int b, tok0, tok1;
@@ -86,12 +119,12 @@ __device__ __forceinline__ SegmentInfo load_segment(const DecodeParams& p, const
   return r;
 }
 
-template <int D>
+template <int D, bool FP8>
 __global__ void __launch_bounds__(kThreads, 2)
     decode_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap k64,
                   const __grid_constant__ CUtensorMap v64, const __grid_constant__ CUtensorMap k16,
                   const __grid_constant__ CUtensorMap v16) {
-  using C = Cfg<D>;
+  using C = Cfg<D, FP8>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const uint32_t sbase = smem_u32(smem);
@@ -201,8 +234,8 @@ __global__ void __launch_bounds__(kThreads, 2)
               const int row = (pid[0] * p.num_kv_heads + g) * P + c0 % P;
 #pragma unroll
               for (int h = 0; h < C::kHalves; ++h) {
-                tma_load_2d(sk + h * kChunk * 128, &k64, h * 64, row, full, policy);
-                tma_load_2d(sv + h * kChunk * 128, &v64, h * 64, row, full, policy);
+                tma_load_2d(sk + h * kChunk * 128, &k64, h * C::kBoxCols, row, full, policy);
+                tma_load_2d(sv + h * kChunk * 128, &v64, h * C::kBoxCols, row, full, policy);
               }
             } else {
 #pragma unroll
@@ -211,8 +244,8 @@ __global__ void __launch_bounds__(kThreads, 2)
                 const int row = (pid[i] * p.num_kv_heads + g) * P + (c0 + 16 * i) % P;
 #pragma unroll
                 for (int h = 0; h < C::kHalves; ++h) {
-                  tma_load_2d(sk + h * kChunk * 128 + i * 2048, &k16, h * 64, row, full, policy);
-                  tma_load_2d(sv + h * kChunk * 128 + i * 2048, &v16, h * 64, row, full, policy);
+                  tma_load_2d(sk + h * kChunk * 128 + i * 2048, &k16, h * C::kBoxCols, row, full, policy);
+                  tma_load_2d(sv + h * kChunk * 128 + i * 2048, &v16, h * C::kBoxCols, row, full, policy);
                 }
               }
             }
@@ -245,12 +278,17 @@ __global__ void __launch_bounds__(kThreads, 2)
   uint32_t phase = 0;
 
   // ldmatrix row addresses that do not depend on the chunk: lane i feeds row i%8
-  // of matrix i/8.
+  // of matrix i/8.  Matrix order (tokens, 16-byte chunk):
+  //   bf16 K  (0-7, c) (0-7, c+1) (8-15, c) (8-15, c+1)
+  //   others  (0-7, c) (8-15, c) (0-7, c+1) (8-15, c+1)
   const int mat = lane >> 3, mrow = lane & 7;
-  const int k_tok = 16 * w + (mat >> 1) * 8 + mrow;  // S: matrices (tok 0-7, c), (tok 0-7, c+1), (tok 8-15, c), (tok 8-15, c+1)
-  const int k_chk = mat & 1;
-  const int v_tok = 16 * w + (mat & 1) * 8 + mrow;   // PV: matrices (tok 0-7, c), (tok 8-15, c), (tok 0-7, c+1), (tok 8-15, c+1)
+  const int k_tok = FP8 ? 16 * w + (mat & 1) * 8 + mrow : 16 * w + (mat >> 1) * 8 + mrow;
+  const int k_chk = FP8 ? mat >> 1 : mat & 1;
+  const int v_tok = 16 * w + (mat & 1) * 8 + mrow;
   const int v_chk = mat >> 1;
+  const float k_scale = FP8 ? __ldg(p.k_scale + g) : 1.f;
+  const float v_scale = FP8 ? __ldg(p.v_scale + g) : 1.f;
+  const float score_scale = p.scale_log2 * k_scale;
 
   for (int s = seg_lo; s < seg_hi; ++s) {
     const SegmentInfo si = load_segment(p, segs, s);
@@ -258,17 +296,26 @@ __global__ void __launch_bounds__(kThreads, 2)
     const int b = si.b;
 
     // Q fragments for rows r (upper half of the MMA tile); rows >= G are zero.
+    // bf16: k-block kk holds columns 16kk + 2tq + {0,1} and + 8.
+    // FP8:  k-block kk holds columns 16kk + 4tq + {0,1} and {2,3}, as f16 (the
+    //       order in which ldmatrix hands out the bytes of a K row).
     uint32_t qlo[D / 16], qhi[D / 16];
     {
-      const uint32_t* qrow = reinterpret_cast<const uint32_t*>(
-          p.q + ((int64_t)b * p.num_q_heads + (int64_t)g * p.group + (row_live ? r : 0)) * D);
+      const __nv_bfloat16* qh = p.q + ((int64_t)b * p.num_q_heads + (int64_t)g * p.group + (row_live ? r : 0)) * D;
 #pragma unroll
       for (int kk = 0; kk < D / 16; ++kk) {
-        qlo[kk] = row_live ? __ldg(qrow + kk * 8 + tq) : 0u;
-        qhi[kk] = row_live ? __ldg(qrow + kk * 8 + 4 + tq) : 0u;
+        if constexpr (FP8) {
+          const uint2 raw = row_live ? __ldg(reinterpret_cast<const uint2*>(qh) + 4 * kk + tq) : make_uint2(0, 0);
+          qlo[kk] = pack_f16x2(bf16_lo_to_f32(raw.x), bf16_hi_to_f32(raw.x));
+          qhi[kk] = pack_f16x2(bf16_lo_to_f32(raw.y), bf16_hi_to_f32(raw.y));
+        } else {
+          const uint32_t* q32 = reinterpret_cast<const uint32_t*>(qh);
+          qlo[kk] = row_live ? __ldg(q32 + kk * 8 + tq) : 0u;
+          qhi[kk] = row_live ? __ldg(q32 + kk * 8 + 4 + tq) : 0u;
+        }
       }
     }
-    // l_r: sum of the bf16-rounded weights that enter P.V (normalises O);
+    // l_r: sum of the rounded weights that enter P.V (normalises O);
     // l_e: sum of the unrounded fp32 weights (gives the log-sum-exp)
     float m = -INFINITY, l_r = 0.f, l_e = 0.f;
     float o[D / 8][2];
@@ -299,12 +346,24 @@ __global__ void __launch_bounds__(kThreads, 2)
         }
         // S = Q . K^T for this warp's 16 tokens (two n-tiles of 8)
         float sc[2][2] = {{0.f, 0.f}, {0.f, 0.f}};
+        if constexpr (FP8) {
 #pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
-          uint32_t b0, b1, b2, b3;
-          ldmatrix_x4(sk + swz(k_tok, 2 * kk + k_chk), b0, b1, b2, b3);
-          mma_bf16_upper(sc[0][0], sc[0][1], qlo[kk], qhi[kk], b0, b1);
-          mma_bf16_upper(sc[1][0], sc[1][1], qlo[kk], qhi[kk], b2, b3);
+          for (int kk = 0; kk < D / 16; kk += 2) {
+            uint32_t r0, r1, r2, r3;  // (tile 0, kk) (tile 1, kk) (tile 0, kk+1) (tile 1, kk+1): 4 codes each
+            ldmatrix_x4(sk + swz(k_tok, kk + k_chk), r0, r1, r2, r3);
+            mma_f16_upper(sc[0][0], sc[0][1], qlo[kk], qhi[kk], e4m3x2_to_f16x2(r0), e4m3x2_to_f16x2(r0 >> 16));
+            mma_f16_upper(sc[1][0], sc[1][1], qlo[kk], qhi[kk], e4m3x2_to_f16x2(r1), e4m3x2_to_f16x2(r1 >> 16));
+            mma_f16_upper(sc[0][0], sc[0][1], qlo[kk + 1], qhi[kk + 1], e4m3x2_to_f16x2(r2), e4m3x2_to_f16x2(r2 >> 16));
+            mma_f16_upper(sc[1][0], sc[1][1], qlo[kk + 1], qhi[kk + 1], e4m3x2_to_f16x2(r3), e4m3x2_to_f16x2(r3 >> 16));
+          }
+        } else {
+#pragma unroll
+          for (int kk = 0; kk < D / 16; ++kk) {
+            uint32_t b0, b1, b2, b3;
+            ldmatrix_x4(sk + swz(k_tok, 2 * kk + k_chk), b0, b1, b2, b3);
+            mma_bf16_upper(sc[0][0], sc[0][1], qlo[kk], qhi[kk], b0, b1);
+            mma_bf16_upper(sc[1][0], sc[1][1], qlo[kk], qhi[kk], b2, b3);
+          }
         }
         // mask, scale to base 2, online softmax update
         float x[2][2];
@@ -314,7 +373,7 @@ __global__ void __launch_bounds__(kThreads, 2)
 #pragma unroll
           for (int e = 0; e < 2; ++e) {
             const int tok = 8 * nt + 2 * tq + e;
-            x[nt][e] = tok < nw ? sc[nt][e] * p.scale_log2 : -INFINITY;
+            x[nt][e] = tok < nw ? sc[nt][e] * score_scale : -INFINITY;
             mx = fmaxf(mx, x[nt][e]);
           }
         mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
@@ -324,9 +383,18 @@ __global__ void __launch_bounds__(kThreads, 2)
         const float corr = fast_exp2(m - m_use);
         const float p00 = fast_exp2(x[0][0] - m_use), p01 = fast_exp2(x[0][1] - m_use);
         const float p10 = fast_exp2(x[1][0] - m_use), p11 = fast_exp2(x[1][1] - m_use);
-        const uint32_t pa0 = pack_bf16x2(p00, p01);
-        const uint32_t pa1 = pack_bf16x2(p10, p11);
-        l_r = l_r * corr + (bf16_lo_to_f32(pa0) + bf16_hi_to_f32(pa0)) + (bf16_lo_to_f32(pa1) + bf16_hi_to_f32(pa1));
+        uint32_t pa0, pa1;
+        float rounded;
+        if constexpr (FP8) {
+          pa0 = pack_f16x2(p00, p01);
+          pa1 = pack_f16x2(p10, p11);
+          rounded = (f16_lo_to_f32(pa0) + f16_hi_to_f32(pa0)) + (f16_lo_to_f32(pa1) + f16_hi_to_f32(pa1));
+        } else {
+          pa0 = pack_bf16x2(p00, p01);
+          pa1 = pack_bf16x2(p10, p11);
+          rounded = (bf16_lo_to_f32(pa0) + bf16_hi_to_f32(pa0)) + (bf16_lo_to_f32(pa1) + bf16_hi_to_f32(pa1));
+        }
+        l_r = l_r * corr + rounded;
         l_e = l_e * corr + ((p00 + p01) + (p10 + p11));
         m = m_new;
 #pragma unroll
@@ -335,12 +403,31 @@ __global__ void __launch_bounds__(kThreads, 2)
           o[i][1] *= corr;
         }
         // O += P . V
+        if constexpr (FP8) {
+          // ldmatrix.trans hands each thread, per matrix, the code pairs (t0: d, d+1)
+          // and (t1: d, d+1); bytes {0,2} are column d, bytes {1,3} column d+1.
+          // Tile 2c + e holds columns 16c + 2j + e.
 #pragma unroll
-        for (int np = 0; np < D / 16; ++np) {
-          uint32_t v0, v1, v2, v3;
-          ldmatrix_x4_trans(sv + swz(v_tok, 2 * np + v_chk), v0, v1, v2, v3);
-          mma_bf16_upper(o[2 * np][0], o[2 * np][1], pa0, pa1, v0, v1);
-          mma_bf16_upper(o[2 * np + 1][0], o[2 * np + 1][1], pa0, pa1, v2, v3);
+          for (int c = 0; c < D / 16; c += 2) {
+            uint32_t r0, r1, r2, r3;  // (tok 0-7, c) (tok 8-15, c) (tok 0-7, c+1) (tok 8-15, c+1)
+            ldmatrix_x4_trans(sv + swz(v_tok, c + v_chk), r0, r1, r2, r3);
+            mma_f16_upper(o[2 * c][0], o[2 * c][1], pa0, pa1, e4m3x2_to_f16x2(__byte_perm(r0, 0, 0x0020)),
+                          e4m3x2_to_f16x2(__byte_perm(r1, 0, 0x0020)));
+            mma_f16_upper(o[2 * c + 1][0], o[2 * c + 1][1], pa0, pa1, e4m3x2_to_f16x2(__byte_perm(r0, 0, 0x0031)),
+                          e4m3x2_to_f16x2(__byte_perm(r1, 0, 0x0031)));
+            mma_f16_upper(o[2 * c + 2][0], o[2 * c + 2][1], pa0, pa1, e4m3x2_to_f16x2(__byte_perm(r2, 0, 0x0020)),
+                          e4m3x2_to_f16x2(__byte_perm(r3, 0, 0x0020)));
+            mma_f16_upper(o[2 * c + 3][0], o[2 * c + 3][1], pa0, pa1, e4m3x2_to_f16x2(__byte_perm(r2, 0, 0x0031)),
+                          e4m3x2_to_f16x2(__byte_perm(r3, 0, 0x0031)));
+          }
+        } else {
+#pragma unroll
+          for (int np = 0; np < D / 16; ++np) {
+            uint32_t v0, v1, v2, v3;
+            ldmatrix_x4_trans(sv + swz(v_tok, 2 * np + v_chk), v0, v1, v2, v3);
+            mma_bf16_upper(o[2 * np][0], o[2 * np][1], pa0, pa1, v0, v1);
+            mma_bf16_upper(o[2 * np + 1][0], o[2 * np + 1][1], pa0, pa1, v2, v3);
+          }
         }
       }
       __syncwarp();
@@ -351,15 +438,36 @@ __global__ void __launch_bounds__(kThreads, 2)
       }
     }
 
+    // ---- regroup this thread's columns: og[gi][j] is column gi*4*GW + GW*tq + j
+    constexpr int GW = C::kGW, NG = C::kNG;
+    float og[NG][GW];
+#pragma unroll
+    for (int gi = 0; gi < NG; ++gi) {
+      if constexpr (FP8) {  // tiles 2gi (even columns) and 2gi+1 (odd columns) of chunk gi
+        og[gi][0] = o[2 * gi][0];
+        og[gi][1] = o[2 * gi + 1][0];
+        og[gi][2] = o[2 * gi][1];
+        og[gi][3] = o[2 * gi + 1][1];
+      } else {
+        og[gi][0] = o[gi][0];
+        og[gi][1] = o[gi][1];
+      }
+    }
+
     // ---- merge the four warp states of this segment
     l_r += __shfl_xor_sync(0xffffffffu, l_r, 1);
     l_r += __shfl_xor_sync(0xffffffffu, l_r, 2);
     l_e += __shfl_xor_sync(0xffffffffu, l_e, 1);
     l_e += __shfl_xor_sync(0xffffffffu, l_e, 2);
     if (w > 0) {
-      float* slot = slots + (w - 1) * C::kSlotFloats + r * C::kSlotStride + 2 * tq;
+      float* slot = slots + (w - 1) * C::kSlotFloats + r * C::kSlotStride + GW * tq;
 #pragma unroll
-      for (int i = 0; i < D / 8; ++i) *reinterpret_cast<float2*>(slot + 8 * i) = make_float2(o[i][0], o[i][1]);
+      for (int gi = 0; gi < NG; ++gi) {
+        if constexpr (GW == 4)
+          *reinterpret_cast<float4*>(slot + 16 * gi) = make_float4(og[gi][0], og[gi][1], og[gi][2], og[gi][3]);
+        else
+          *reinterpret_cast<float2*>(slot + 8 * gi) = make_float2(og[gi][0], og[gi][1]);
+      }
       if (tq == 0) {
         ml[(w - 1) * 24 + r] = m;
         ml[(w - 1) * 24 + 8 + r] = l_r;
@@ -387,33 +495,46 @@ __global__ void __launch_bounds__(kThreads, 2)
         Lr += fw[j] * lrw[j];
         Le += fw[j] * lew[j];
       }
-      const float inv = Lr > 0.f ? 1.f / Lr : 0.f;
+      const float inv = Lr > 0.f ? v_scale / Lr : 0.f;
       const float lse_nat = Le > 0.f ? (M + log2f(Le)) * 0.69314718055994530942f : -INFINITY;
       const int h = g * p.group + r;
       const int nseg_b = rsb[b + 1] - rsb[b];
       const bool direct = nseg_b == 1;
 #pragma unroll
-      for (int i = 0; i < D / 8; ++i) {
-        float a0 = f0 * o[i][0], a1 = f0 * o[i][1];
+      for (int gi = 0; gi < NG; ++gi) {
+        float a[GW];
+#pragma unroll
+        for (int e = 0; e < GW; ++e) a[e] = f0 * og[gi][e];
 #pragma unroll
         for (int j = 0; j < 3; ++j) {
-          const float2 v = *reinterpret_cast<const float2*>(slots + j * C::kSlotFloats + r * C::kSlotStride + 8 * i + 2 * tq);
-          a0 += fw[j] * v.x;
-          a1 += fw[j] * v.y;
+          const float* src = slots + j * C::kSlotFloats + r * C::kSlotStride + gi * 4 * GW + GW * tq;
+#pragma unroll
+          for (int e = 0; e < GW; ++e) a[e] += fw[j] * src[e];
         }
-        o[i][0] = a0 * inv;
-        o[i][1] = a1 * inv;
+#pragma unroll
+        for (int e = 0; e < GW; ++e) og[gi][e] = a[e] * inv;
       }
       if (row_live) {
         if (direct) {
-          uint32_t* dst = reinterpret_cast<uint32_t*>(p.out + ((int64_t)b * p.num_q_heads + h) * D + 2 * tq);
+          __nv_bfloat16* dst = p.out + ((int64_t)b * p.num_q_heads + h) * D + GW * tq;
 #pragma unroll
-          for (int i = 0; i < D / 8; ++i) dst[4 * i] = pack_bf16x2(o[i][0], o[i][1]);
+          for (int gi = 0; gi < NG; ++gi) {
+            if constexpr (GW == 4)
+              *reinterpret_cast<uint2*>(dst + 16 * gi) =
+                  make_uint2(pack_bf16x2(og[gi][0], og[gi][1]), pack_bf16x2(og[gi][2], og[gi][3]));
+            else
+              *reinterpret_cast<uint32_t*>(dst + 8 * gi) = pack_bf16x2(og[gi][0], og[gi][1]);
+          }
           if (tq == 0) p.lse[(int64_t)b * p.num_q_heads + h] = lse_nat;
         } else {
-          float* dst = p.partial_o + ((int64_t)s * p.num_q_heads + h) * D + 2 * tq;
+          float* dst = p.partial_o + ((int64_t)s * p.num_q_heads + h) * D + GW * tq;
 #pragma unroll
-          for (int i = 0; i < D / 8; ++i) *reinterpret_cast<float2*>(dst + 8 * i) = make_float2(o[i][0], o[i][1]);
+          for (int gi = 0; gi < NG; ++gi) {
+            if constexpr (GW == 4)
+              *reinterpret_cast<float4*>(dst + 16 * gi) = make_float4(og[gi][0], og[gi][1], og[gi][2], og[gi][3]);
+            else
+              *reinterpret_cast<float2*>(dst + 8 * gi) = make_float2(og[gi][0], og[gi][1]);
+          }
           if (tq == 0) p.partial_lse[(int64_t)s * p.num_q_heads + h] = lse_nat;
         }
       }
@@ -422,9 +543,9 @@ __global__ void __launch_bounds__(kThreads, 2)
   }
 }
 
-template <int D>
+template <int D, bool FP8>
 cudaError_t launch_decode_d(const DecodeParams& p, const CUtensorMap maps[4], cudaStream_t stream) {
-  using C = Cfg<D>;
+  using C = Cfg<D, FP8>;
   static_assert(C::kSmemRequest * 2 <= 227 * 1024, "two CTAs per SM must fit");
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
@@ -432,7 +553,7 @@ cudaError_t launch_decode_d(const DecodeParams& p, const CUtensorMap maps[4], cu
   static bool configured[64] = {false};
   if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
   if (!configured[dev]) {
-    e = cudaFuncSetAttribute(decode_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemRequest);
+    e = cudaFuncSetAttribute(decode_kernel<D, FP8>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemRequest);
     if (e != cudaSuccess) return e;
     configured[dev] = true;
   }
@@ -446,14 +567,19 @@ cudaError_t launch_decode_d(const DecodeParams& p, const CUtensorMap maps[4], cu
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, decode_kernel<D>, p, maps[0], maps[1], maps[2], maps[3]);
+  return cudaLaunchKernelEx(&cfg, decode_kernel<D, FP8>, p, maps[0], maps[1], maps[2], maps[3]);
 }
 
 }  // namespace
 
 cudaError_t launch_decode(const DecodeParams& p, int head_dim, const CUtensorMap maps[4], cudaStream_t stream) {
-  if (head_dim == 128) return launch_decode_d<128>(p, maps, stream);
-  if (head_dim == 64) return launch_decode_d<64>(p, maps, stream);
+  if (head_dim == 128) return launch_decode_d<128, false>(p, maps, stream);
+  if (head_dim == 64) return launch_decode_d<64, false>(p, maps, stream);
+  return cudaErrorInvalidValue;
+}
+
+cudaError_t launch_decode_fp8(const DecodeParams& p, int head_dim, const CUtensorMap maps[4], cudaStream_t stream) {
+  if (head_dim == 128) return launch_decode_d<128, true>(p, maps, stream);
   return cudaErrorInvalidValue;
 }
 

@@ -21,7 +21,8 @@ PLAN_DYNAMIC, PLAN_STATIC = 0, 1
 # Every symbol include/da.h declares.
 EXPORTS = ("da_plan_desc_init", "da_workspace_size", "da_workspace_offsets", "da_plan", "da_static_plan",
            "da_decode_attention", "da_combine", "da_read_status", "da_status_string", "da_dev_status_string",
-           "da_last_cuda_error", "da_device_num_sms", "da_decode_step_noalloc", "da_append_kv")
+           "da_last_cuda_error", "da_device_num_sms", "da_decode_step_noalloc", "da_append_kv",
+           "da_decode_attention_fp8")
 
 NOALLOC_SCRATCH_BYTES = 16 << 20  # DA_NOALLOC_SCRATCH_BYTES
 
@@ -74,6 +75,7 @@ def lib():
             "da_device_num_sms": [ctypes.POINTER(ctypes.c_int32)],
             "da_decode_step_noalloc": [P, ctypes.c_int32, ctypes.c_int32, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp],
             "da_append_kv": [P, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp],
+            "da_decode_attention_fp8": [P, D, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp],
         }
         for name, args in sig.items():
             fn = getattr(L, name)
@@ -167,6 +169,14 @@ def da_decode_attention(prob, desc, q, k_cache, v_cache, block_table, seq_lens, 
         _ptr(seq_lens), _ptr(ws), _ptr(partial_o), _ptr(partial_lse), _ptr(out), _ptr(lse), _stream(stream)))
 
 
+def da_decode_attention_fp8(prob, desc, q, k_cache, v_cache, k_scale, v_scale, block_table, seq_lens, ws, partial_o,
+                            partial_lse, out, lse, stream=None):
+    _check("da_decode_attention_fp8", lib().da_decode_attention_fp8(
+        ctypes.byref(prob), ctypes.byref(desc), _ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(k_scale), _ptr(v_scale),
+        _ptr(block_table), _ptr(seq_lens), _ptr(ws), _ptr(partial_o), _ptr(partial_lse), _ptr(out), _ptr(lse),
+        _stream(stream)))
+
+
 def da_combine(prob, desc, ws, partial_o, partial_lse, out, lse, stream=None):
     _check("da_combine", lib().da_combine(ctypes.byref(prob), ctypes.byref(desc), _ptr(ws), _ptr(partial_o),
                                           _ptr(partial_lse), _ptr(out), _ptr(lse), _stream(stream)))
@@ -213,14 +223,21 @@ class Buffers:
         self.lse = torch.empty((prob.batch, prob.num_q_heads), dtype=torch.float32, device=device)
 
 
-def decode_step(prob, desc, q, k_cache, v_cache, block_table, seq_lens, bufs: Buffers, stream=None):
-    """Plan (dynamic or static, per `desc.kind`) + decode + combine, asynchronously on `stream`."""
+def decode_step(prob, desc, q, k_cache, v_cache, block_table, seq_lens, bufs: Buffers, stream=None, k_scale=None,
+                v_scale=None):
+    """Plan (dynamic or static, per `desc.kind`) + decode + combine, asynchronously on `stream`.
+
+    With k_scale/v_scale given, the caches are FP8 E4M3 codes (da_decode_attention_fp8)."""
     if desc.kind == PLAN_DYNAMIC:
         da_plan(prob, desc, seq_lens, bufs.ws, stream=stream)
     else:
         da_static_plan(prob, desc, seq_lens, bufs.ws, stream=stream)
-    da_decode_attention(prob, desc, q, k_cache, v_cache, block_table, seq_lens, bufs.ws, bufs.partial_o,
-                        bufs.partial_lse, bufs.out, bufs.lse, stream=stream)
+    if k_scale is None:
+        da_decode_attention(prob, desc, q, k_cache, v_cache, block_table, seq_lens, bufs.ws, bufs.partial_o,
+                            bufs.partial_lse, bufs.out, bufs.lse, stream=stream)
+    else:
+        da_decode_attention_fp8(prob, desc, q, k_cache, v_cache, k_scale, v_scale, block_table, seq_lens, bufs.ws,
+                                bufs.partial_o, bufs.partial_lse, bufs.out, bufs.lse, stream=stream)
     da_combine(prob, desc, bufs.ws, bufs.partial_o, bufs.partial_lse, bufs.out, bufs.lse, stream=stream)
     return bufs.out, bufs.lse
 

@@ -91,6 +91,8 @@ class DeviceWorkload:
     q: torch.Tensor
     k_cache: torch.Tensor
     v_cache: torch.Tensor
+    k_scale: torch.Tensor | None = None  # FP8 caches only
+    v_scale: torch.Tensor | None = None
 
 
 def _fp32(x: float) -> float:
@@ -172,6 +174,66 @@ def make_workload(name: str, seq_lens, *, num_q_heads: int, num_kv_heads: int, h
                       page_size=P, max_pages_per_req=max_pages_per_req, num_pages=num_pages, scale=scale)
     return Workload(name=name, problem=problem, seq_lens=lens.astype(np.int32), block_table=block_table,
                     q=q, k_cache=k, v_cache=v, seed=seed, recipe=recipe)
+
+
+# ---------------------------------------------------------------------------------------------
+# FP8 (E4M3) caches.
+
+
+@dataclasses.dataclass
+class Fp8Workload:
+    """A workload whose K/V caches are FP8 E4M3 codes with one scale per KV head.
+
+    The cached value of KV head g is k_scale[g] * e4m3(k_code) (and likewise V).
+    Quantisation recipe: scale = fp32(max |x| over the live tokens of that head /
+    448), code = E4M3 rounding (torch, round-to-nearest-even) of x / scale; unused
+    slots stay NaN codes.
+    """
+    base: Workload
+    k_code: torch.Tensor  # uint8 [num_pages, Hkv, P, d]
+    v_code: torch.Tensor
+    k_scale: np.ndarray  # float32 [Hkv]
+    v_scale: np.ndarray
+
+    @property
+    def problem(self) -> Problem:
+        return self.base.problem
+
+    @property
+    def kv_bytes(self) -> int:
+        """Bytes of K and V one decode step reads: sum_b L_b * Hkv * d * 2 (K,V) * 1 B."""
+        p = self.problem
+        return int(np.clip(self.base.seq_lens, 0, None).astype(np.int64).sum()) * p.num_kv_heads * p.head_dim * 2
+
+    def to(self, device) -> "DeviceWorkload":
+        b = self.base
+        return DeviceWorkload(problem=b.problem, seq_lens=torch.from_numpy(b.seq_lens).to(device),
+                              block_table=torch.from_numpy(b.block_table).to(device), q=b.q.to(device),
+                              k_cache=self.k_code.to(device), v_cache=self.v_code.to(device),
+                              k_scale=torch.from_numpy(self.k_scale).to(device),
+                              v_scale=torch.from_numpy(self.v_scale).to(device))
+
+
+def _quantize_cache(cache: torch.Tensor, chunk_pages: int = 2048):
+    Hkv = cache.shape[1]
+    amax = torch.zeros(Hkv, dtype=torch.float32)
+    for p0 in range(0, cache.shape[0], chunk_pages):
+        x = cache[p0:p0 + chunk_pages].float().abs().nan_to_num(0.0)
+        amax = torch.maximum(amax, x.amax(dim=(0, 2, 3)))
+    scale = (amax / 448.0).clamp_min(torch.finfo(torch.float32).tiny).numpy().astype(np.float32)
+    sc = torch.from_numpy(scale)[None, :, None, None]
+    code = torch.empty(cache.shape, dtype=torch.uint8)
+    for p0 in range(0, cache.shape[0], chunk_pages):
+        x = cache[p0:p0 + chunk_pages].float() / sc
+        code[p0:p0 + chunk_pages] = x.to(torch.float8_e4m3fn).view(torch.uint8)
+    return code, scale
+
+
+def quantize_fp8(w: Workload) -> Fp8Workload:
+    """FP8 E4M3 copy of a workload's caches (q, lengths and block table unchanged)."""
+    kc, ks = _quantize_cache(w.k_cache)
+    vc, vs = _quantize_cache(w.v_cache)
+    return Fp8Workload(base=w, k_code=kc, v_code=vc, k_scale=ks, v_scale=vs)
 
 
 # ---------------------------------------------------------------------------------------------
