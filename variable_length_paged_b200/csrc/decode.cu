@@ -9,18 +9,22 @@
 // Grid (C, Hkv): CTA (c, g) walks the segments the plan gave CTA c, for KV
 // head g.  Block = 4 consumer warps + 1 producer warp.
 //
-//   producer  One lane issues TMA tensor loads (128-byte swizzle) of 64-token
-//             K and V chunks into a ring of shared-memory stages, each stage
-//             guarded by a "full" mbarrier (transaction bytes) and an "empty"
-//             mbarrier (one arrival per consumer warp).  Page ids come from the
-//             block table 32 at a time, one per lane.
-//   consumers Warp w owns tokens [16w, 16w+16) of each chunk and keeps its own
-//             online-softmax state for all G query heads of the group:
-//               S^T block: S = Q . K^T with mma.m16n8k16 (rows = heads, the
-//               upper 8 of the 16 MMA rows; n = tokens; k = head_dim), K read
-//               with ldmatrix from the swizzled tile;
-//               running max m, running sum l, fp32 accumulator O += P . V with
-//               P rounded to bf16 in registers and V read with ldmatrix.trans.
+//   producer  One lane issues TMA tensor loads (128-byte swizzle) of K and V
+//             chunks into a ring of shared-memory stages, each stage guarded
+//             by a "full" mbarrier (transaction bytes) and an "empty" mbarrier
+//             (one arrival per consumer warp).  A chunk is loaded as 64-row
+//             boxes when a 64-token run sits inside one page, else as 16-row
+//             boxes.  Page ids come from the block table 32 at a time.
+//   consumers Warp w owns TPW consecutive tokens of each chunk (16 or 32) and
+//             keeps its own online-softmax state for all G query heads of
+//             the group:
+//               S = Q . K^T with mma.m16n8k16 (rows = heads, the upper 8 of
+//               the 16 MMA rows; n = tokens; k = head_dim), K read with
+//               ldmatrix from the swizzled tile, two accumulator chains per
+//               n-tile for instruction-level parallelism;
+//               running max m, running sums, fp32 accumulator O += P . V with
+//               P rounded to the MMA input type in registers and V read with
+//               ldmatrix.trans; O is rescaled only when some row's max moved.
 //             At the end of a segment the four warp states are merged by
 //             log-sum-exp through shared memory; the result goes to out/lse
 //             (request with one segment) or to the segment's partial slot.
@@ -33,12 +37,15 @@
 // fp32 accumulation, and the K scale is folded into the score scale and the V
 // scale into the final normalisation.
 //
+// Every stage is 32 KB (K + V): 64 tokens of 256-byte rows (bf16, d 128) or
+// 128 tokens of 128-byte rows (FP8 d 128, bf16 d 64); three stages per CTA and
+// two CTAs per SM keep 192 KB of loads in flight per SM.
+//
 // Scores are kept in base-2 units (scale * log2 e), so exp is one ex2 and the
 // natural-log lse is (m + log2 l) * ln 2.  Tokens past the end of a request
 // inside a loaded chunk are masked to -inf; their V rows are zeroed in shared
 // memory first, since unused cache slots may hold anything (NaN included).
 #include <cuda_fp16.h>
-#include <cuda_fp8.h>
 
 #include <cfloat>
 
@@ -47,7 +54,6 @@
 namespace da {
 namespace {
 
-constexpr int kChunk = 64;            // tokens per pipeline stage
 constexpr int kConsumerWarps = 4;
 constexpr int kThreads = (kConsumerWarps + 1) * 32;
 constexpr uint64_t kWaitLimitNs = 2000000000ull;  // 2 s: far beyond any legitimate wait
@@ -59,9 +65,13 @@ struct Cfg {
   static_assert(kRowBytes % 128 == 0, "a row must be whole 128-byte swizzle spans");
   static constexpr int kHalves = kRowBytes / 128;            // 128-byte column blocks per row
   static constexpr int kBoxCols = 128 / kElemBytes;          // elements per TMA box row
-  static constexpr int kTileBytes = kHalves * kChunk * 128;  // one K (or V) chunk
+  static constexpr int kTPW = kRowBytes == 128 ? 32 : 16;    // tokens per consumer warp per chunk
+  static constexpr int kChunk = kConsumerWarps * kTPW;       // tokens per stage
+  static constexpr int kSub = kTPW / 16;                     // 16-token MMA pieces per warp
+  static constexpr int kHalfStride = kChunk * 128;           // bytes of one 128-byte column block of a tile
+  static constexpr int kTileBytes = kHalves * kHalfStride;   // one K (or V) chunk
   static constexpr int kStageBytes = 2 * kTileBytes;
-  static constexpr int kStages = (96 * 1024) / kStageBytes;  // a 96 KB ring per CTA
+  static constexpr int kStages = 3;
   // per-thread output columns: NG groups of GW consecutive columns, group gi at gi*4*GW + GW*tq
   static constexpr int kGW = FP8 ? 4 : 2;
   static constexpr int kNG = D / (4 * kGW);
@@ -79,15 +89,22 @@ struct Cfg {
 };
 
 // Byte offset of (row, 16-byte column chunk) inside a TMA tile written with
-// 128-byte swizzle: the chunk index is XORed with row % 8 inside each 128-byte row.
+// 128-byte swizzle: the chunk index is XORed with row % 8 inside each 128-byte
+// row; column blocks of 128 bytes are stored one after the other.
+template <int kHalfStride>
 __device__ __forceinline__ uint32_t swz(int row, int chunk) {
-  return (uint32_t)((chunk >> 3) * (kChunk * 128) + row * 128 + (((chunk & 7) ^ (row & 7)) << 4));
+  return (uint32_t)((chunk >> 3) * kHalfStride + row * 128 + (((chunk & 7) ^ (row & 7)) << 4));
 }
 
-// Two E4M3 codes (low byte first) -> f16x2 (low half first); exact.
-__device__ __forceinline__ uint32_t e4m3x2_to_f16x2(uint32_t two_codes) {
-  const __half2_raw h = __nv_cvt_fp8x2_to_halfraw2(static_cast<__nv_fp8x2_storage_t>(two_codes & 0xFFFFu), __NV_E4M3);
-  return static_cast<uint32_t>(h.x) | (static_cast<uint32_t>(h.y) << 16);
+// Four E4M3 codes c0..c3 (c0 in the low byte) -> two f16x2: lo = (c0, c1),
+// hi = (c2, c3), low half first.  Exact: every E4M3 value is an f16 value.
+__device__ __forceinline__ void e4m3x4_to_f16x2x2(uint32_t codes, uint32_t& lo, uint32_t& hi) {
+  asm("{\n\t.reg .b16 l, h;\n\t"
+      "mov.b32 {l, h}, %2;\n\t"
+      "cvt.rn.f16x2.e4m3x2 %0, l;\n\t"
+      "cvt.rn.f16x2.e4m3x2 %1, h;\n\t}"
+      : "=r"(lo), "=r"(hi)
+      : "r"(codes));
 }
 
 __device__ __forceinline__ uint32_t pack_f16x2(float lo, float hi) {
@@ -125,6 +142,7 @@ __global__ void __launch_bounds__(kThreads, 2)
                   const __grid_constant__ CUtensorMap v64, const __grid_constant__ CUtensorMap k16,
                   const __grid_constant__ CUtensorMap v16) {
   using C = Cfg<D, FP8>;
+  constexpr int kChunk = C::kChunk;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const uint32_t sbase = smem_u32(smem);
@@ -200,15 +218,15 @@ __global__ void __launch_bounds__(kThreads, 2)
           const int lp = win_base + lane;
           win_val = lp < p.max_pages_per_req ? __ldg(bt_row + lp) : -1;
         }
-        const bool fast = (c0 % P) + kChunk <= P;  // the whole chunk sits in one page
-        const int pieces = fast ? 1 : (n + 15) >> 4;
-        int pid[4];
+        // page of every 16-row piece of the chunk (pieces past n are not loaded)
+        constexpr int kPieces = kChunk / 16;
+        int pid[kPieces];
         bool ok = true;
 #pragma unroll
-        for (int i = 0; i < 4; ++i) {
+        for (int i = 0; i < kPieces; ++i) {
           const int lp = (c0 + 16 * i) / P;
           pid[i] = __shfl_sync(0xffffffffu, win_val, (lp - win_base) & 31);
-          if (i < pieces) ok = ok && pid[i] >= 0 && pid[i] < p.num_pages;
+          if (16 * i < n) ok = ok && pid[i] >= 0 && pid[i] < p.num_pages;
         }
         // wait until the consumers have released this stage
         bool got = true;
@@ -225,27 +243,44 @@ __global__ void __launch_bounds__(kThreads, 2)
         if (lane == 0) {
           if (!ok) record_status(hdr_w, DA_DEV_BAD_PAGE, si.b);
           meta[stage] = ok ? n : 0;
-          const uint32_t bytes = !ok ? 0u : fast ? (uint32_t)C::kStageBytes : (uint32_t)(pieces * C::kHalves * 2048 * 2);
+          // bytes: per 64-row sub-chunk, one 64-row box per column block when it sits in
+          // one page, else one 16-row box per column block for each piece that holds tokens
+          uint32_t bytes = 0;
+          if (ok) {
+#pragma unroll
+            for (int j = 0; j < kChunk / 64; ++j) {
+              if (64 * j >= n) break;
+              const bool fast = ((c0 + 64 * j) % P) + 64 <= P;
+              const int pieces = fast ? 4 : min(4, (n - 64 * j + 15) >> 4);
+              bytes += (uint32_t)(pieces * 16 * 128 * C::kHalves * 2);
+            }
+          }
           const uint32_t full = full0 + 8 * stage;
           mbar_arrive_expect_tx(full, bytes);
           if (ok) {
             const uint32_t sk = sbase + C::kOffStages + stage * C::kStageBytes, sv = sk + C::kTileBytes;
-            if (fast) {
-              const int row = (pid[0] * p.num_kv_heads + g) * P + c0 % P;
 #pragma unroll
-              for (int h = 0; h < C::kHalves; ++h) {
-                tma_load_2d(sk + h * kChunk * 128, &k64, h * C::kBoxCols, row, full, policy);
-                tma_load_2d(sv + h * kChunk * 128, &v64, h * C::kBoxCols, row, full, policy);
-              }
-            } else {
-#pragma unroll
-              for (int i = 0; i < 4; ++i) {
-                if (i >= pieces) break;
-                const int row = (pid[i] * p.num_kv_heads + g) * P + (c0 + 16 * i) % P;
+            for (int j = 0; j < kChunk / 64; ++j) {
+              if (64 * j >= n) break;
+              const int tok = c0 + 64 * j;
+              if ((tok % P) + 64 <= P) {
+                const int row = (pid[4 * j] * p.num_kv_heads + g) * P + tok % P;
 #pragma unroll
                 for (int h = 0; h < C::kHalves; ++h) {
-                  tma_load_2d(sk + h * kChunk * 128 + i * 2048, &k16, h * C::kBoxCols, row, full, policy);
-                  tma_load_2d(sv + h * kChunk * 128 + i * 2048, &v16, h * C::kBoxCols, row, full, policy);
+                  tma_load_2d(sk + h * C::kHalfStride + j * 64 * 128, &k64, h * C::kBoxCols, row, full, policy);
+                  tma_load_2d(sv + h * C::kHalfStride + j * 64 * 128, &v64, h * C::kBoxCols, row, full, policy);
+                }
+              } else {
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                  if (64 * j + 16 * i >= n) break;
+                  const int row = (pid[4 * j + i] * p.num_kv_heads + g) * P + (tok + 16 * i) % P;
+#pragma unroll
+                  for (int h = 0; h < C::kHalves; ++h) {
+                    const uint32_t off = h * C::kHalfStride + (64 * j + 16 * i) * 128;
+                    tma_load_2d(sk + off, &k16, h * C::kBoxCols, row, full, policy);
+                    tma_load_2d(sv + off, &v16, h * C::kBoxCols, row, full, policy);
+                  }
                 }
               }
             }
@@ -268,6 +303,7 @@ __global__ void __launch_bounds__(kThreads, 2)
   }
 
   // -------------------------------------------------------------------- consumer warps
+  constexpr int TPW = C::kTPW, SUB = C::kSub, HS = C::kHalfStride;
   const int w = warp;
   const int r = lane >> 2;   // query head within the group (MMA row)
   const int tq = lane & 3;   // thread within the quad
@@ -278,13 +314,13 @@ __global__ void __launch_bounds__(kThreads, 2)
   uint32_t phase = 0;
 
   // ldmatrix row addresses that do not depend on the chunk: lane i feeds row i%8
-  // of matrix i/8.  Matrix order (tokens, 16-byte chunk):
+  // of matrix i/8.  Matrix order (tokens of a 16-token piece, 16-byte chunk):
   //   bf16 K  (0-7, c) (0-7, c+1) (8-15, c) (8-15, c+1)
   //   others  (0-7, c) (8-15, c) (0-7, c+1) (8-15, c+1)
   const int mat = lane >> 3, mrow = lane & 7;
-  const int k_tok = FP8 ? 16 * w + (mat & 1) * 8 + mrow : 16 * w + (mat >> 1) * 8 + mrow;
+  const int k_tok = TPW * w + (FP8 ? (mat & 1) * 8 : (mat >> 1) * 8) + mrow;
   const int k_chk = FP8 ? mat >> 1 : mat & 1;
-  const int v_tok = 16 * w + (mat & 1) * 8 + mrow;
+  const int v_tok = TPW * w + (mat & 1) * 8 + mrow;
   const int v_chk = mat >> 1;
   const float k_scale = FP8 ? __ldg(p.k_scale + g) : 1.f;
   const float v_scale = FP8 ? __ldg(p.v_scale + g) : 1.f;
@@ -329,51 +365,67 @@ __global__ void __launch_bounds__(kThreads, 2)
         *abort_flag = 1;
       }
       const int n = got ? meta[stage] : 0;
-      const int nw = min(max(n - 16 * w, 0), 16);  // valid tokens in this warp's 16 rows
+      const int nw = min(max(n - TPW * w, 0), TPW);  // valid tokens in this warp's rows
       const uint32_t sk = sbase + C::kOffStages + stage * C::kStageBytes, sv = sk + C::kTileBytes;
       if (nw > 0) {
-        if (nw < 16) {
-          // zero V rows [nw, 16) of this warp's piece: stale or unused slots must not reach P.V
+        if (nw < TPW) {
+          // zero V rows [nw, TPW) of this warp: stale or unused slots must not reach P.V
           uint8_t* vrows = smem + C::kOffStages + stage * C::kStageBytes + C::kTileBytes;
-          for (int i = lane; i < (16 - nw) * C::kHalves * 8; i += 32) {
-            const int row = 16 * w + nw + i / (C::kHalves * 8);
+          for (int i = lane; i < (TPW - nw) * C::kHalves * 8; i += 32) {
+            const int row = TPW * w + nw + i / (C::kHalves * 8);
             const int rem = i % (C::kHalves * 8);
             const int half = rem >> 3, chunk16 = rem & 7;
-            *reinterpret_cast<uint4*>(vrows + half * kChunk * 128 + row * 128 + chunk16 * 16) = make_uint4(0, 0, 0, 0);
+            *reinterpret_cast<uint4*>(vrows + half * HS + row * 128 + chunk16 * 16) = make_uint4(0, 0, 0, 0);
           }
           fence_proxy_async_smem();
           __syncwarp();
         }
-        // S = Q . K^T for this warp's 16 tokens (two n-tiles of 8)
-        float sc[2][2] = {{0.f, 0.f}, {0.f, 0.f}};
-        if constexpr (FP8) {
+        // S = Q . K^T for this warp's tokens: n-tile nt = tokens [8nt, 8nt+8) of the
+        // warp; two accumulator chains (even / odd k-blocks) per n-tile.
+        float sc[2 * SUB][2][2];
 #pragma unroll
-          for (int kk = 0; kk < D / 16; kk += 2) {
-            uint32_t r0, r1, r2, r3;  // (tile 0, kk) (tile 1, kk) (tile 0, kk+1) (tile 1, kk+1): 4 codes each
-            ldmatrix_x4(sk + swz(k_tok, kk + k_chk), r0, r1, r2, r3);
-            mma_f16_upper(sc[0][0], sc[0][1], qlo[kk], qhi[kk], e4m3x2_to_f16x2(r0), e4m3x2_to_f16x2(r0 >> 16));
-            mma_f16_upper(sc[1][0], sc[1][1], qlo[kk], qhi[kk], e4m3x2_to_f16x2(r1), e4m3x2_to_f16x2(r1 >> 16));
-            mma_f16_upper(sc[0][0], sc[0][1], qlo[kk + 1], qhi[kk + 1], e4m3x2_to_f16x2(r2), e4m3x2_to_f16x2(r2 >> 16));
-            mma_f16_upper(sc[1][0], sc[1][1], qlo[kk + 1], qhi[kk + 1], e4m3x2_to_f16x2(r3), e4m3x2_to_f16x2(r3 >> 16));
-          }
-        } else {
+        for (int nt = 0; nt < 2 * SUB; ++nt) sc[nt][0][0] = sc[nt][0][1] = sc[nt][1][0] = sc[nt][1][1] = 0.f;
 #pragma unroll
-          for (int kk = 0; kk < D / 16; ++kk) {
-            uint32_t b0, b1, b2, b3;
-            ldmatrix_x4(sk + swz(k_tok, 2 * kk + k_chk), b0, b1, b2, b3);
-            mma_bf16_upper(sc[0][0], sc[0][1], qlo[kk], qhi[kk], b0, b1);
-            mma_bf16_upper(sc[1][0], sc[1][1], qlo[kk], qhi[kk], b2, b3);
+        for (int sp = 0; sp < SUB; ++sp) {
+          const int ktok = k_tok + 16 * sp;
+          if constexpr (FP8) {
+#pragma unroll
+            for (int kk = 0; kk < D / 16; kk += 2) {
+              uint32_t r0, r1, r2, r3;  // (tile 0, kk) (tile 1, kk) (tile 0, kk+1) (tile 1, kk+1): 4 codes each
+              ldmatrix_x4(sk + swz<HS>(ktok, kk + k_chk), r0, r1, r2, r3);
+              uint32_t b00, b01, b10, b11, b20, b21, b30, b31;
+              e4m3x4_to_f16x2x2(r0, b00, b01);
+              e4m3x4_to_f16x2x2(r1, b10, b11);
+              e4m3x4_to_f16x2x2(r2, b20, b21);
+              e4m3x4_to_f16x2x2(r3, b30, b31);
+              float(&a)[2][2] = sc[2 * sp];
+              float(&c)[2][2] = sc[2 * sp + 1];
+              mma_f16_upper(a[0][0], a[0][1], qlo[kk], qhi[kk], b00, b01);
+              mma_f16_upper(c[0][0], c[0][1], qlo[kk], qhi[kk], b10, b11);
+              mma_f16_upper(a[1][0], a[1][1], qlo[kk + 1], qhi[kk + 1], b20, b21);
+              mma_f16_upper(c[1][0], c[1][1], qlo[kk + 1], qhi[kk + 1], b30, b31);
+            }
+          } else {
+#pragma unroll
+            for (int kk = 0; kk < D / 16; ++kk) {
+              uint32_t b0, b1, b2, b3;
+              ldmatrix_x4(sk + swz<HS>(ktok, 2 * kk + k_chk), b0, b1, b2, b3);
+              float(&a)[2] = sc[2 * sp][kk & 1];
+              float(&c)[2] = sc[2 * sp + 1][kk & 1];
+              mma_bf16_upper(a[0], a[1], qlo[kk], qhi[kk], b0, b1);
+              mma_bf16_upper(c[0], c[1], qlo[kk], qhi[kk], b2, b3);
+            }
           }
         }
         // mask, scale to base 2, online softmax update
-        float x[2][2];
+        float x[2 * SUB][2];
         float mx = -INFINITY;
 #pragma unroll
-        for (int nt = 0; nt < 2; ++nt)
+        for (int nt = 0; nt < 2 * SUB; ++nt)
 #pragma unroll
           for (int e = 0; e < 2; ++e) {
             const int tok = 8 * nt + 2 * tq + e;
-            x[nt][e] = tok < nw ? sc[nt][e] * score_scale : -INFINITY;
+            x[nt][e] = tok < nw ? (sc[nt][0][e] + sc[nt][1][e]) * score_scale : -INFINITY;
             mx = fmaxf(mx, x[nt][e]);
           }
         mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
@@ -381,52 +433,66 @@ __global__ void __launch_bounds__(kThreads, 2)
         const float m_new = fmaxf(m, mx);
         const float m_use = m_new == -INFINITY ? 0.f : m_new;
         const float corr = fast_exp2(m - m_use);
-        const float p00 = fast_exp2(x[0][0] - m_use), p01 = fast_exp2(x[0][1] - m_use);
-        const float p10 = fast_exp2(x[1][0] - m_use), p11 = fast_exp2(x[1][1] - m_use);
-        uint32_t pa0, pa1;
-        float rounded;
-        if constexpr (FP8) {
-          pa0 = pack_f16x2(p00, p01);
-          pa1 = pack_f16x2(p10, p11);
-          rounded = (f16_lo_to_f32(pa0) + f16_hi_to_f32(pa0)) + (f16_lo_to_f32(pa1) + f16_hi_to_f32(pa1));
-        } else {
-          pa0 = pack_bf16x2(p00, p01);
-          pa1 = pack_bf16x2(p10, p11);
-          rounded = (bf16_lo_to_f32(pa0) + bf16_hi_to_f32(pa0)) + (bf16_lo_to_f32(pa1) + bf16_hi_to_f32(pa1));
+        uint32_t pa[SUB][2];
+        float rounded = 0.f, exact = 0.f;
+#pragma unroll
+        for (int sp = 0; sp < SUB; ++sp) {
+          const float p00 = fast_exp2(x[2 * sp][0] - m_use), p01 = fast_exp2(x[2 * sp][1] - m_use);
+          const float p10 = fast_exp2(x[2 * sp + 1][0] - m_use), p11 = fast_exp2(x[2 * sp + 1][1] - m_use);
+          if constexpr (FP8) {
+            pa[sp][0] = pack_f16x2(p00, p01);
+            pa[sp][1] = pack_f16x2(p10, p11);
+            rounded += (f16_lo_to_f32(pa[sp][0]) + f16_hi_to_f32(pa[sp][0])) +
+                       (f16_lo_to_f32(pa[sp][1]) + f16_hi_to_f32(pa[sp][1]));
+          } else {
+            pa[sp][0] = pack_bf16x2(p00, p01);
+            pa[sp][1] = pack_bf16x2(p10, p11);
+            rounded += (bf16_lo_to_f32(pa[sp][0]) + bf16_hi_to_f32(pa[sp][0])) +
+                       (bf16_lo_to_f32(pa[sp][1]) + bf16_hi_to_f32(pa[sp][1]));
+          }
+          exact += (p00 + p01) + (p10 + p11);
         }
         l_r = l_r * corr + rounded;
-        l_e = l_e * corr + ((p00 + p01) + (p10 + p11));
+        l_e = l_e * corr + exact;
         m = m_new;
+        if (!__all_sync(0xffffffffu, corr == 1.f)) {  // some row's running max moved
 #pragma unroll
-        for (int i = 0; i < D / 8; ++i) {
-          o[i][0] *= corr;
-          o[i][1] *= corr;
-        }
-        // O += P . V
-        if constexpr (FP8) {
-          // ldmatrix.trans hands each thread, per matrix, the code pairs (t0: d, d+1)
-          // and (t1: d, d+1); bytes {0,2} are column d, bytes {1,3} column d+1.
-          // Tile 2c + e holds columns 16c + 2j + e.
-#pragma unroll
-          for (int c = 0; c < D / 16; c += 2) {
-            uint32_t r0, r1, r2, r3;  // (tok 0-7, c) (tok 8-15, c) (tok 0-7, c+1) (tok 8-15, c+1)
-            ldmatrix_x4_trans(sv + swz(v_tok, c + v_chk), r0, r1, r2, r3);
-            mma_f16_upper(o[2 * c][0], o[2 * c][1], pa0, pa1, e4m3x2_to_f16x2(__byte_perm(r0, 0, 0x0020)),
-                          e4m3x2_to_f16x2(__byte_perm(r1, 0, 0x0020)));
-            mma_f16_upper(o[2 * c + 1][0], o[2 * c + 1][1], pa0, pa1, e4m3x2_to_f16x2(__byte_perm(r0, 0, 0x0031)),
-                          e4m3x2_to_f16x2(__byte_perm(r1, 0, 0x0031)));
-            mma_f16_upper(o[2 * c + 2][0], o[2 * c + 2][1], pa0, pa1, e4m3x2_to_f16x2(__byte_perm(r2, 0, 0x0020)),
-                          e4m3x2_to_f16x2(__byte_perm(r3, 0, 0x0020)));
-            mma_f16_upper(o[2 * c + 3][0], o[2 * c + 3][1], pa0, pa1, e4m3x2_to_f16x2(__byte_perm(r2, 0, 0x0031)),
-                          e4m3x2_to_f16x2(__byte_perm(r3, 0, 0x0031)));
+          for (int i = 0; i < D / 8; ++i) {
+            o[i][0] *= corr;
+            o[i][1] *= corr;
           }
-        } else {
+        }
+        // O += P . V, one k-step of 16 tokens per piece
 #pragma unroll
-          for (int np = 0; np < D / 16; ++np) {
-            uint32_t v0, v1, v2, v3;
-            ldmatrix_x4_trans(sv + swz(v_tok, 2 * np + v_chk), v0, v1, v2, v3);
-            mma_bf16_upper(o[2 * np][0], o[2 * np][1], pa0, pa1, v0, v1);
-            mma_bf16_upper(o[2 * np + 1][0], o[2 * np + 1][1], pa0, pa1, v2, v3);
+        for (int sp = 0; sp < SUB; ++sp) {
+          const int vtok = v_tok + 16 * sp;
+          if constexpr (FP8) {
+            // ldmatrix.trans hands each thread, per matrix, the code pairs (t0: d, d+1)
+            // and (t1: d, d+1) as bytes 0..3; one byte permute to (0, 2, 1, 3) gives
+            // column d's pair (t0, t1) and column d+1's pair.  Tile 2c + e holds
+            // columns 16c + 2j + e.
+#pragma unroll
+            for (int c = 0; c < D / 16; c += 2) {
+              uint32_t r0, r1, r2, r3;  // (tok 0-7, c) (tok 8-15, c) (tok 0-7, c+1) (tok 8-15, c+1)
+              ldmatrix_x4_trans(sv + swz<HS>(vtok, c + v_chk), r0, r1, r2, r3);
+              uint32_t e0, o0, e1, o1, e2, o2, e3, o3;
+              e4m3x4_to_f16x2x2(__byte_perm(r0, 0, 0x3120), e0, o0);
+              e4m3x4_to_f16x2x2(__byte_perm(r1, 0, 0x3120), e1, o1);
+              e4m3x4_to_f16x2x2(__byte_perm(r2, 0, 0x3120), e2, o2);
+              e4m3x4_to_f16x2x2(__byte_perm(r3, 0, 0x3120), e3, o3);
+              mma_f16_upper(o[2 * c][0], o[2 * c][1], pa[sp][0], pa[sp][1], e0, e1);
+              mma_f16_upper(o[2 * c + 1][0], o[2 * c + 1][1], pa[sp][0], pa[sp][1], o0, o1);
+              mma_f16_upper(o[2 * c + 2][0], o[2 * c + 2][1], pa[sp][0], pa[sp][1], e2, e3);
+              mma_f16_upper(o[2 * c + 3][0], o[2 * c + 3][1], pa[sp][0], pa[sp][1], o2, o3);
+            }
+          } else {
+#pragma unroll
+            for (int np = 0; np < D / 16; ++np) {
+              uint32_t v0, v1, v2, v3;
+              ldmatrix_x4_trans(sv + swz<HS>(vtok, 2 * np + v_chk), v0, v1, v2, v3);
+              mma_bf16_upper(o[2 * np][0], o[2 * np][1], pa[sp][0], pa[sp][1], v0, v1);
+              mma_bf16_upper(o[2 * np + 1][0], o[2 * np + 1][1], pa[sp][0], pa[sp][1], v2, v3);
+            }
           }
         }
       }
