@@ -24,7 +24,9 @@
 //               n-tile for instruction-level parallelism;
 //               running max m, running sums, fp32 accumulator O += P . V with
 //               P rounded to the MMA input type in registers and V read with
-//               ldmatrix.trans; O is rescaled only when some row's max moved.
+//               ldmatrix.trans; the sum of the rounded P comes from one more
+//               MMA against a tile of ones; O is rescaled only when some row's
+//               max moved.
 //             At the end of a segment the four warp states are merged by
 //             log-sum-exp through shared memory; the result goes to out/lse
 //             (request with one segment) or to the segment's partial slot.
@@ -113,8 +115,6 @@ __device__ __forceinline__ uint32_t pack_f16x2(float lo, float hi) {
   return r;
 }
 
-__device__ __forceinline__ float f16_lo_to_f32(uint32_t v) { return __half2float(__ushort_as_half((unsigned short)(v & 0xFFFFu))); }
-__device__ __forceinline__ float f16_hi_to_f32(uint32_t v) { return __half2float(__ushort_as_half((unsigned short)(v >> 16))); }
 
 struct SegmentInfo {
   int b, tok0, tok1;
@@ -351,9 +351,11 @@ __global__ void __launch_bounds__(kThreads, 2)
         }
       }
     }
-    // l_r: sum of the rounded weights that enter P.V (normalises O);
-    // l_e: sum of the unrounded fp32 weights (gives the log-sum-exp)
-    float m = -INFINITY, l_r = 0.f, l_e = 0.f;
+    // lr: sum of the rounded weights that enter P.V (normalises O), kept as an
+    //     MMA accumulator tile of P times ones (both entries hold the row sum);
+    // l_e: per-thread sum of the unrounded fp32 weights (gives the log-sum-exp)
+    float m = -INFINITY, l_e = 0.f;
+    float lr[2] = {0.f, 0.f};
     float o[D / 8][2];
 #pragma unroll
     for (int i = 0; i < D / 8; ++i) o[i][0] = o[i][1] = 0.f;
@@ -417,24 +419,29 @@ __global__ void __launch_bounds__(kThreads, 2)
             }
           }
         }
-        // mask, scale to base 2, online softmax update
+        // scale to base 2, mask the tail (only in a partial chunk), online softmax update
         float x[2 * SUB][2];
-        float mx = -INFINITY;
 #pragma unroll
         for (int nt = 0; nt < 2 * SUB; ++nt)
 #pragma unroll
-          for (int e = 0; e < 2; ++e) {
-            const int tok = 8 * nt + 2 * tq + e;
-            x[nt][e] = tok < nw ? (sc[nt][0][e] + sc[nt][1][e]) * score_scale : -INFINITY;
-            mx = fmaxf(mx, x[nt][e]);
-          }
+          for (int e = 0; e < 2; ++e) x[nt][e] = (sc[nt][0][e] + sc[nt][1][e]) * score_scale;
+        if (nw < TPW) {
+#pragma unroll
+          for (int nt = 0; nt < 2 * SUB; ++nt)
+#pragma unroll
+            for (int e = 0; e < 2; ++e)
+              if (8 * nt + 2 * tq + e >= nw) x[nt][e] = -INFINITY;
+        }
+        float mx = -INFINITY;
+#pragma unroll
+        for (int nt = 0; nt < 2 * SUB; ++nt) mx = fmaxf(mx, fmaxf(x[nt][0], x[nt][1]));
         mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
         mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
         const float m_new = fmaxf(m, mx);
         const float m_use = m_new == -INFINITY ? 0.f : m_new;
         const float corr = fast_exp2(m - m_use);
         uint32_t pa[SUB][2];
-        float rounded = 0.f, exact = 0.f;
+        float exact = 0.f;
 #pragma unroll
         for (int sp = 0; sp < SUB; ++sp) {
           const float p00 = fast_exp2(x[2 * sp][0] - m_use), p01 = fast_exp2(x[2 * sp][1] - m_use);
@@ -442,17 +449,12 @@ __global__ void __launch_bounds__(kThreads, 2)
           if constexpr (FP8) {
             pa[sp][0] = pack_f16x2(p00, p01);
             pa[sp][1] = pack_f16x2(p10, p11);
-            rounded += (f16_lo_to_f32(pa[sp][0]) + f16_hi_to_f32(pa[sp][0])) +
-                       (f16_lo_to_f32(pa[sp][1]) + f16_hi_to_f32(pa[sp][1]));
           } else {
             pa[sp][0] = pack_bf16x2(p00, p01);
             pa[sp][1] = pack_bf16x2(p10, p11);
-            rounded += (bf16_lo_to_f32(pa[sp][0]) + bf16_hi_to_f32(pa[sp][0])) +
-                       (bf16_lo_to_f32(pa[sp][1]) + bf16_hi_to_f32(pa[sp][1]));
           }
           exact += (p00 + p01) + (p10 + p11);
         }
-        l_r = l_r * corr + rounded;
         l_e = l_e * corr + exact;
         m = m_new;
         if (!__all_sync(0xffffffffu, corr == 1.f)) {  // some row's running max moved
@@ -461,6 +463,17 @@ __global__ void __launch_bounds__(kThreads, 2)
             o[i][0] *= corr;
             o[i][1] *= corr;
           }
+          lr[0] *= corr;
+          lr[1] *= corr;
+        }
+        // the sum of the rounded weights, as the tensor core sees them: P times a
+        // column block of ones (every column of the tile holds the row sum)
+#pragma unroll
+        for (int sp = 0; sp < SUB; ++sp) {
+          if constexpr (FP8)
+            mma_f16_upper(lr[0], lr[1], pa[sp][0], pa[sp][1], 0x3C003C00u, 0x3C003C00u);
+          else
+            mma_bf16_upper(lr[0], lr[1], pa[sp][0], pa[sp][1], 0x3F803F80u, 0x3F803F80u);
         }
         // O += P . V, one k-step of 16 tokens per piece
 #pragma unroll
@@ -521,8 +534,7 @@ __global__ void __launch_bounds__(kThreads, 2)
     }
 
     // ---- merge the four warp states of this segment
-    l_r += __shfl_xor_sync(0xffffffffu, l_r, 1);
-    l_r += __shfl_xor_sync(0xffffffffu, l_r, 2);
+    const float l_r = lr[0];  // already the full row sum over the warp's tokens
     l_e += __shfl_xor_sync(0xffffffffu, l_e, 1);
     l_e += __shfl_xor_sync(0xffffffffu, l_e, 2);
     if (w > 0) {
