@@ -77,6 +77,11 @@ def _bind(path: str):
         ctypes.c_int32, ctypes.c_int32, ctypes.c_int32, ctypes.c_int32, ctypes.c_int32,
         ctypes.c_int32, ctypes.c_int64, ctypes.c_double, _u16p, _u8p, _u8p, _f64p, _f64p, _i32p, _i32p,
         ctypes.c_int64, _i32p, _i32p, _f64p, _f64p, ctypes.c_int32]
+    lib.dao_attention_mq.restype = ctypes.c_int
+    lib.dao_attention_mq.argtypes = [
+        ctypes.c_int32, ctypes.c_int32, ctypes.c_int32, ctypes.c_int32, ctypes.c_int32, ctypes.c_int32,
+        ctypes.c_int32, ctypes.c_int64, ctypes.c_double, _u16p, _u16p, _u16p, _i32p, _i32p, _f64p, _f64p,
+        ctypes.c_int32]
     lib.dao_e4m3_value.restype = ctypes.c_double
     lib.dao_e4m3_value.argtypes = [ctypes.c_uint8]
     return lib
@@ -164,6 +169,25 @@ def attention(q, k_cache, v_cache, block_table, seq_lens, *, scale: float, num_p
     if pairs is None:
         out = out.reshape(B, Hq, d)
         lse = lse.reshape(B, Hq)
+    return out, lse, int(st)
+
+
+def attention_mq(q, k_cache, v_cache, block_table, seq_lens, *, scale: float, threads: int = 0, lib=None):
+    """fp64 multi-query decode: q bf16 [B, Q, Hq, d], the Q queries being the last Q cached tokens;
+    query i attends causally to tokens [0, L_b - Q + i].  Returns (out [B, Q, Hq, d], lse [B, Q, Hq], status)."""
+    lib = lib or _load()
+    q16, k16, v16 = _u16(q), _u16(k_cache), _u16(v_cache)
+    bt = np.ascontiguousarray(block_table, dtype=np.int32)
+    sl = np.ascontiguousarray(seq_lens, dtype=np.int32)
+    B, Q, Hq, d = q16.shape
+    n_pages, Hkv, P, d2 = k16.shape
+    assert d2 == d and v16.shape == k16.shape and bt.shape[0] == B and sl.shape == (B,)
+    out = np.empty((B, Q, Hq, d), dtype=np.float64)
+    lse = np.empty((B, Q, Hq), dtype=np.float64)
+    st = lib.dao_attention_mq(B, Q, Hq, Hkv, d, P, bt.shape[1], n_pages, float(scale), _ptr(q16, ctypes.c_uint16),
+                              _ptr(k16, ctypes.c_uint16), _ptr(v16, ctypes.c_uint16), _ptr(bt, ctypes.c_int32),
+                              _ptr(sl, ctypes.c_int32), _ptr(out, ctypes.c_double), _ptr(lse, ctypes.c_double),
+                              int(threads))
     return out, lse, int(st)
 
 

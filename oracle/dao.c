@@ -205,6 +205,49 @@ static int attention_impl(int32_t batch, int32_t num_q_heads, int32_t num_kv_hea
   return status;
 }
 
+/*
+ * Multi-query decode: q_len new tokens per request, the last q_len positions of
+ * its cache.  Query i (0 <= i < q_len) sits at position L_b - q_len + i and
+ * attends causally to tokens [0, L_b - q_len + i]; it is therefore plain
+ * attention over the first L_b - q_len + i + 1 tokens (empty when that is <= 0).
+ *   q    bf16 [batch][q_len][num_q_heads][head_dim]
+ *   out  fp64 [batch][q_len][num_q_heads][head_dim];  lse fp64 [batch][q_len][num_q_heads]
+ * Lengths out of range are reported as for dao_attention and count as 0.
+ */
+int dao_attention_mq(int32_t batch, int32_t q_len, int32_t num_q_heads, int32_t num_kv_heads, int32_t head_dim,
+                     int32_t page_size, int32_t max_pages_per_req, int64_t num_pages, double scale,
+                     const uint16_t* q, const uint16_t* k, const uint16_t* v, const int32_t* block_table,
+                     const int32_t* seq_lens, double* out, double* lse, int32_t num_threads) {
+  if (batch < 0 || q_len <= 0 || max_pages_per_req < 0 || page_size <= 0) return DAO_ERR_ARG;
+  const int64_t capacity = (int64_t)max_pages_per_req * page_size;
+  const int64_t rows = (int64_t)batch * q_len;
+  /* Every (request, query) becomes one single-query request with its own length. */
+  int32_t* lens = (int32_t*)malloc((size_t)(rows > 0 ? rows : 1) * sizeof(int32_t));
+  int32_t* bt = (int32_t*)malloc((size_t)(rows > 0 ? rows : 1) * (size_t)(max_pages_per_req > 0 ? max_pages_per_req : 1) *
+                                 sizeof(int32_t));
+  int status = DAO_OK;
+  for (int32_t b = 0; b < batch; ++b) {
+    int64_t L = seq_lens[b];
+    if (L < 0 || L > capacity) {
+      status = DAO_ERR_BAD_SEQLEN;
+      L = 0;
+    }
+    for (int32_t i = 0; i < q_len; ++i) {
+      const int64_t li = L - q_len + i + 1;
+      lens[(int64_t)b * q_len + i] = (int32_t)(li > 0 ? li : 0);
+      memcpy(bt + ((int64_t)b * q_len + i) * max_pages_per_req, block_table + (int64_t)b * max_pages_per_req,
+             (size_t)max_pages_per_req * sizeof(int32_t));
+    }
+  }
+  const kv_view kv = {0, k, v, NULL, NULL};
+  const int st = attention_impl((int32_t)rows, num_q_heads, num_kv_heads, head_dim, page_size, max_pages_per_req,
+                                num_pages, scale, q, &kv, bt, lens, rows * num_q_heads, NULL, NULL, out, lse,
+                                num_threads);
+  free(lens);
+  free(bt);
+  return st != DAO_OK ? st : status;
+}
+
 int dao_attention(int32_t batch, int32_t num_q_heads, int32_t num_kv_heads, int32_t head_dim,
                   int32_t page_size, int32_t max_pages_per_req, int64_t num_pages, double scale,
                   const uint16_t* q, const uint16_t* k, const uint16_t* v,

@@ -350,10 +350,53 @@ def pin_fp8_equals_bf16_when_exact(lib=None):
     assert np.array_equal(a[0], b[0]) and np.array_equal(a[1], b[1])
 
 
+# ---------------------------------------------------------------------------------------------
+# Multi-query decode pins.
+
+
+def pin_mq_matches_sdpa_with_causal_mask(lib=None):
+    """Q new tokens at the end of each cache; torch SDPA (float64) with an explicit position mask."""
+    rng = np.random.default_rng(24)
+    for (B, Q, Hq, Hkv, d, P, lens) in [(3, 2, 8, 2, 16, 4, [2, 9, 30]), (2, 4, 4, 1, 8, 3, [1, 13]),
+                                        (1, 3, 6, 3, 32, 8, [5])]:
+        _, dk, dv, kc, vc, bt, sl, scale = random_case(rng, B, Hq, Hkv, d, P, lens)
+        q = bf16(rng.standard_normal((B, Q, Hq, d)))
+        out, lse, st = oracle.attention_mq(q, kc, vc, bt, sl, scale=scale, lib=lib)
+        assert st == oracle.OK
+        for b, L in enumerate(lens):
+            pos = torch.arange(L)
+            for i in range(Q):
+                qpos = L - Q + i
+                if qpos < 0:
+                    assert not out[b, i].any() and np.all(lse[b, i] == -np.inf)
+                    continue
+                mask = (pos <= qpos).view(1, 1, 1, L)
+                qb = q[b, i].double().unsqueeze(0).unsqueeze(2)
+                kb = dk[b].double().permute(1, 0, 2).unsqueeze(0)
+                vb = dv[b].double().permute(1, 0, 2).unsqueeze(0)
+                ref = torch.nn.functional.scaled_dot_product_attention(qb, kb, vb, attn_mask=mask, scale=scale,
+                                                                       enable_gqa=True)
+                np.testing.assert_allclose(out[b, i], ref[0, :, 0].numpy(), rtol=1e-11, atol=1e-12)
+                s_ = torch.einsum("hd,htd->ht", qb[0, :, 0], kb.repeat_interleave(Hq // Hkv, dim=1)[0]) * scale
+                s_ = s_.masked_fill(~mask.view(1, L), float("-inf"))
+                np.testing.assert_allclose(lse[b, i], torch.logsumexp(s_, dim=1).numpy(), rtol=1e-12, atol=1e-12)
+
+
+def pin_mq_single_query_is_decode(lib=None):
+    """With one query per request, multi-query decode is plain decode, bit for bit."""
+    rng = np.random.default_rng(25)
+    q, dk, dv, kc, vc, bt, sl, scale = random_case(rng, 3, 8, 2, 16, 4, [1, 7, 33])
+    a = oracle.attention(q, kc, vc, bt, sl, scale=scale, lib=lib)
+    b = oracle.attention_mq(q.unsqueeze(1).contiguous(), kc, vc, bt, sl, scale=scale, lib=lib)
+    assert a[2] == b[2] == oracle.OK
+    assert np.array_equal(a[0], b[0][:, 0]) and np.array_equal(a[1], b[1][:, 0])
+
+
 ATTENTION_PINS = [pin_golden_attention, pin_length_one, pin_constant_v, pin_uniform_scores, pin_dominant_key,
                   pin_page_order_invariance, pin_prefix_sharing, pin_matches_sdpa, pin_split_merge_identity,
                   pin_degenerate_lengths, pin_pairs_match_full, pin_e4m3_decoding, pin_fp8_matches_sdpa,
-                  pin_fp8_equals_bf16_when_exact]
+                  pin_fp8_equals_bf16_when_exact, pin_mq_matches_sdpa_with_causal_mask,
+                  pin_mq_single_query_is_decode]
 
 
 # ---------------------------------------------------------------------------------------------

@@ -26,6 +26,9 @@ MUTANTS = [
     ("fp8 V scaled by K's scale", "const double sc = is_v ? kv->v_scale[g] : kv->k_scale[g];",
      "const double sc = kv->k_scale[g];"),
     ("fp8 scale ignored", "return sc * e4m3_to_double(", "return e4m3_to_double("),
+    ("multi-query causal offset", "const int64_t li = L - q_len + i + 1;", "const int64_t li = L - q_len + i;"),
+    ("multi-query wrong block-table row", "block_table + (int64_t)b * max_pages_per_req,\n",
+     "block_table + (int64_t)0 * max_pages_per_req,\n"),
     ("block table row", "block_table[(int64_t)b * max_pages_per_req + t / page_size];\n      if",
      "block_table[(int64_t)b + t / page_size];\n      if"),
     ("lse without max", "lse[i] = m + log(l);", "lse[i] = log(l);"),
