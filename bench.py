@@ -52,6 +52,7 @@ def parse_args():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--config", default="mixed", choices=["mixed", "skewed", "low_conc", "uniform", "tiny", "trace"])
     ap.add_argument("--kv", choices=["bf16", "fp8"], default="bf16", help="KV cache format")
+    ap.add_argument("--q-len", type=int, default=1, help="queries per request (multi-query decode)")
     ap.add_argument("--tile", type=int, default=64)
     ap.add_argument("--width", type=int, default=0, help="CTAs per KV head (0 = 2 per SM / Hkv)")
     ap.add_argument("--no-static", action="store_true", help="skip the static split-k comparison")
@@ -221,7 +222,8 @@ def run_ours(args, world, rank, local):
     da.lib()  # fail loudly if the CUDA library is missing
     seed_shift = 1000 * rank
     gen = W.CONFIGS[args.config]
-    w = gen(seed=gen.__defaults__[0] + seed_shift) if rank else gen()
+    qkw = {"q_len": args.q_len} if args.q_len > 1 else {}
+    w = gen(seed=gen.__defaults__[0] + seed_shift, **qkw) if rank else gen(**qkw)
     w8 = W.quantize_fp8(w) if args.kv == "fp8" else None
     dw = w8.to("cuda") if w8 is not None else w.to("cuda")
     prob = da.problem_from(dw.problem)
@@ -326,8 +328,9 @@ def run_ours(args, world, rank, local):
         metric=METRIC, value=round(value, 2), unit="GB/s", n_gpus=world, steps=steps, warmup=warm,
         ms_per_step=round(ms_graph / steps, 5), us_per_step=round(ms_graph / steps * 1e3, 2),
         higher_is_better=True, scaling="weak", vs_baseline=None, dtype="bf16", data="synthetic",
-        config={"workload": f"{args.config}: {w.recipe}" + ("; FP8 E4M3 KV, per-head scales" if w8 else ""),
-                "batch": w.problem.batch, "kv_format": args.kv,
+        config={"workload": f"{args.config}: {w.recipe}" + ("; FP8 E4M3 KV, per-head scales" if w8 else "")
+                + (f"; {args.q_len} queries per request" if args.q_len > 1 else ""),
+                "batch": w.problem.batch, "kv_format": args.kv, "q_len": args.q_len,
                 "kv_bytes_per_step_per_gpu": kv_bytes, "tile_tokens": desc.tile_tokens,
                 "ctas_per_kv_head": desc.num_ctas, "graph": True,
                 "l2": "inputs larger than L2 (K/V read per step >> 126 MB), no flush"},
@@ -439,7 +442,9 @@ def cpu_baseline(w, seconds, w8=None):
     t0 = time.perf_counter()
     passes = 0
     while True:
-        if w8 is None:
+        if w8 is None and w.q.dim() == 4:
+            oracle.attention_mq(w.q, w.k_cache, w.v_cache, w.block_table, w.seq_lens, scale=w.problem.scale)
+        elif w8 is None:
             oracle.attention(w.q, w.k_cache, w.v_cache, w.block_table, w.seq_lens, scale=w.problem.scale)
         else:
             oracle.attention_fp8(w.q, w8.k_code, w8.v_code, w8.k_scale.astype(np.float64),

@@ -95,9 +95,17 @@ extern "C" {
  * lse = ln sum_t exp(scale * q . k_t) (natural log of the scaled scores); an
  * empty request gives out = 0, lse = -inf.
  *
- * Supported: head_dim 64 or 128; num_q_heads / num_kv_heads in 1..8;
- * page_size a positive multiple of 16; num_pages * num_kv_heads * page_size
- * below 2^31.
+ * Multi-query decode (q_len > 1: several new tokens per request, e.g. draft
+ * tokens of speculative decoding): the q_len queries are the last q_len tokens
+ * already in the cache; query i of request b sits at position
+ * seq_lens[b] - q_len + i and attends causally to tokens [0, seq_lens[b] - q_len + i]
+ * (none when that range is empty).  Then q, out are [batch][q_len][num_q_heads][head_dim]
+ * and lse is [batch][q_len][num_q_heads]; the K/V of each request are read once for
+ * all its queries.
+ *
+ * Supported: head_dim 64 or 128; G = num_q_heads / num_kv_heads with
+ * G * q_len <= 16; page_size a positive multiple of
+ * 16; num_pages * num_kv_heads * page_size below 2^31.
  */
 typedef struct da_problem {
   int32_t batch;
@@ -108,6 +116,7 @@ typedef struct da_problem {
   int32_t max_pages_per_req;
   int32_t num_pages;
   float scale;
+  int32_t q_len; /* queries per request; 0 or 1 = plain single-token decode */
 } da_problem;
 
 /*
@@ -141,8 +150,8 @@ DA_API int da_plan_desc_init(const da_problem* prob, int32_t kind, int32_t tile_
 /*
  * da_workspace_size -- bytes the caller must allocate on the device:
  *   ws_bytes           the plan (int32 header and work list), 16-byte aligned
- *   partial_o_bytes    fp32 [max_segments][num_q_heads][head_dim]
- *   partial_lse_bytes  fp32 [max_segments][num_q_heads]
+ *   partial_o_bytes    fp32 [max_segments][q_len][num_q_heads][head_dim]
+ *   partial_lse_bytes  fp32 [max_segments][q_len][num_q_heads]
  * Any output pointer may be NULL.
  */
 DA_API int da_workspace_size(const da_problem* prob, const da_plan_desc* desc, size_t* ws_bytes,

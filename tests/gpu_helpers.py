@@ -106,3 +106,38 @@ def check_against_oracle_fp8(w8: W.Fp8Workload, out, lse, pairs=None):
         lerr = np.where(both_inf, 0.0, np.abs(l - ref_lse))
     assert np.all(lerr <= LSE_ATOL), f"lse mismatch: max err {np.nanmax(lerr)}"
     return float(err.max()), float(lerr.max())
+
+
+def check_mq_against_oracle(w: W.Workload, out, lse):
+    """Multi-query outputs [B, Q, Hq, d] against the fp64 multi-query oracle."""
+    ref, ref_lse, st = oracle.attention_mq(w.q, w.k_cache, w.v_cache, w.block_table, w.seq_lens,
+                                           scale=w.problem.scale)
+    return _compare(out, lse, ref, ref_lse)
+
+
+def check_mq_fp8_against_oracle(w8: W.Fp8Workload, out, lse):
+    """FP8 multi-query: each (request, query i) is a single-query request over its first
+    L - Q + i + 1 tokens (the multi-query definition, pinned in the oracle pins)."""
+    b = w8.base
+    B, Q = b.q.shape[0], b.q.shape[1]
+    lens = np.array([max(int(b.seq_lens[r]) - Q + i + 1, 0) for r in range(B) for i in range(Q)], np.int32)
+    bt = np.repeat(b.block_table, Q, axis=0)
+    q = b.q.reshape(B * Q, b.q.shape[2], b.q.shape[3])
+    ref, ref_lse, st = oracle.attention_fp8(q, w8.k_code, w8.v_code, w8.k_scale.astype(np.float64),
+                                            w8.v_scale.astype(np.float64), bt, lens, scale=b.problem.scale)
+    return _compare(out, lse, ref.reshape(B, Q, *ref.shape[1:]), ref_lse.reshape(B, Q, -1))
+
+
+def _compare(out, lse, ref, ref_lse):
+    o = out.float().cpu().double().numpy()
+    l = lse.cpu().double().numpy()
+    assert np.all(np.isfinite(o)), "non-finite output"
+    err = np.abs(o - ref)
+    bound = OUT_ATOL + OUT_RTOL * np.abs(ref)
+    worst = np.unravel_index(np.argmax(err - bound), err.shape)
+    assert np.all(err <= bound), f"out mismatch at {worst}: gpu {o[worst]} ref {ref[worst]}"
+    both_inf = np.isneginf(l) & np.isneginf(ref_lse)
+    with np.errstate(invalid="ignore"):
+        lerr = np.where(both_inf, 0.0, np.abs(l - ref_lse))
+    assert np.all(lerr <= LSE_ATOL), f"lse mismatch: max err {np.nanmax(lerr)}"
+    return float(err.max()), float(lerr.max())

@@ -59,7 +59,9 @@ def test_plan_descriptor_and_sizes(da_lib):
     (dict(num_q_heads=60), -1),          # Hq % Hkv != 0
     (dict(head_dim=96), -2),             # only 64 / 128 are built
     (dict(page_size=8), -2),             # pages must be multiples of 16 rows
-    (dict(num_q_heads=128, num_kv_heads=8), -2),  # group of 16 not built
+    (dict(num_q_heads=256, num_kv_heads=8), -2),  # 32 query heads per KV head do not fit one MMA tile
+    (dict(q_len=3), -2),                 # 8 heads x 3 queries > 16 rows
+    (dict(q_len=-1), -1),
     (dict(batch=-1), -1),
     (dict(num_pages=0), -1),
     (dict(num_pages=1 << 30), -2),       # row index would overflow int32

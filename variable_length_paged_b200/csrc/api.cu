@@ -15,7 +15,9 @@ thread_local int32_t g_last_cuda_error = 0;
 
 constexpr int kDefaultTile = 64;
 constexpr int kCtasPerSm = 2;  // decode kernel residency (shared memory sized for two)
-constexpr int kMaxGroup = 8;
+constexpr int kMaxRows = 16;  // query heads x queries per request packed on one MMA tile
+
+int q_len_of(const da_problem* p) { return p->q_len > 1 ? p->q_len : 1; }
 
 int cuda_fail(cudaError_t e) {
   g_last_cuda_error = (int32_t)e;
@@ -30,7 +32,8 @@ int check_problem(const da_problem* p) {
   if (p->num_q_heads % p->num_kv_heads != 0) return DA_ERR_INVALID_ARG;
   if (!(p->scale == p->scale)) return DA_ERR_INVALID_ARG;  // NaN scale
   if (p->head_dim != 64 && p->head_dim != 128) return DA_ERR_UNSUPPORTED;
-  if (p->num_q_heads / p->num_kv_heads > kMaxGroup) return DA_ERR_UNSUPPORTED;
+  if (p->q_len < 0) return DA_ERR_INVALID_ARG;
+  if ((int64_t)(p->num_q_heads / p->num_kv_heads) * q_len_of(p) > kMaxRows) return DA_ERR_UNSUPPORTED;
   if (p->page_size % 16 != 0) return DA_ERR_UNSUPPORTED;
   if ((int64_t)p->num_pages * p->num_kv_heads * p->page_size >= (int64_t)INT_MAX) return DA_ERR_UNSUPPORTED;
   if ((int64_t)p->max_pages_per_req * p->page_size >= (int64_t)INT_MAX) return DA_ERR_UNSUPPORTED;
@@ -169,8 +172,9 @@ DA_API int da_workspace_size(const da_problem* prob, const da_plan_desc* desc, s
   rc = check_desc(prob, desc);
   if (rc != DA_OK) return rc;
   if (ws_bytes) *ws_bytes = ws_words(desc) * 4;
-  if (partial_o_bytes) *partial_o_bytes = (size_t)desc->max_segments * prob->num_q_heads * prob->head_dim * 4;
-  if (partial_lse_bytes) *partial_lse_bytes = (size_t)desc->max_segments * prob->num_q_heads * 4;
+  const size_t rows = (size_t)q_len_of(prob) * prob->num_q_heads;
+  if (partial_o_bytes) *partial_o_bytes = (size_t)desc->max_segments * rows * prob->head_dim * 4;
+  if (partial_lse_bytes) *partial_lse_bytes = (size_t)desc->max_segments * rows * 4;
   return DA_OK;
 }
 
@@ -266,6 +270,9 @@ static int decode_common(const da_problem* prob, const da_plan_desc* desc, const
   p.kind = desc->kind;
   p.capacity_tokens = (int64_t)prob->max_pages_per_req * prob->page_size;
   p.scale_log2 = prob->scale * 1.4426950408889634f;
+  p.q_len = q_len_of(prob);
+  // more than 8 rows (G > 8, or several queries) take the kernel that uses all 16 MMA rows
+  p.full_rows = p.group * p.q_len > 8 ? 1 : 0;
   cudaError_t e = fp8 ? da::launch_decode_fp8(p, prob->head_dim, maps, static_cast<cudaStream_t>(stream))
                       : da::launch_decode(p, prob->head_dim, maps, static_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? DA_OK : cuda_fail(e);
@@ -305,7 +312,7 @@ DA_API int da_combine(const da_problem* prob, const da_plan_desc* desc, const vo
   p.out = static_cast<__nv_bfloat16*>(out);
   p.lse = lse;
   p.batch = prob->batch;
-  p.num_q_heads = prob->num_q_heads;
+  p.num_q_heads = prob->num_q_heads * q_len_of(prob);  // every (query, head) row merges the same way
   p.num_ctas = desc->num_ctas;
   p.max_segments = desc->max_segments;
   cudaError_t e = da::launch_combine(p, prob->head_dim, static_cast<cudaStream_t>(stream));

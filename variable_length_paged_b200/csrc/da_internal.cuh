@@ -70,6 +70,8 @@ struct DecodeParams {
   float scale_log2;  // scale * log2(e): scores are kept in base-2 units
   const float* k_scale;  // FP8 caches: per-KV-head dequantisation scales (else null)
   const float* v_scale;
+  int32_t q_len;  // queries per request (1 = plain decode)
+  int32_t full_rows;  // 1: G * q_len > 8, all 16 MMA rows carry (query, head) rows
 };
 
 struct CombineParams {
@@ -207,6 +209,25 @@ __device__ __forceinline__ void mma_bf16_upper(float& d0, float& d1, uint32_t a0
       "{%0, %1, %2, %3};"
       : "+f"(d0), "+f"(d1), "+f"(d2), "+f"(d3)
       : "r"(a0), "r"(0u), "r"(a2), "r"(0u), "r"(b0), "r"(b1));
+}
+
+// All 16 rows of A used (rows r: a0, a2; rows r + 8: a1, a3): d[0..1] row r, d[2..3] row r + 8.
+__device__ __forceinline__ void mma_bf16_full(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
+                                              uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, "
+      "{%0, %1, %2, %3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+__device__ __forceinline__ void mma_f16_full(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
+                                             uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, "
+      "{%0, %1, %2, %3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
 }
 
 // Same with f16 operands (FP8 caches are widened to f16, exactly).

@@ -60,20 +60,21 @@ constexpr int kConsumerWarps = 4;
 constexpr int kThreads = (kConsumerWarps + 1) * 32;
 constexpr uint64_t kWaitLimitNs = 2000000000ull;  // 2 s: far beyond any legitimate wait
 
-template <int D, bool FP8>
+template <int D, bool FP8, bool MQ>
 struct Cfg {
   static constexpr int kElemBytes = FP8 ? 1 : 2;
   static constexpr int kRowBytes = D * kElemBytes;
   static_assert(kRowBytes % 128 == 0, "a row must be whole 128-byte swizzle spans");
   static constexpr int kHalves = kRowBytes / 128;            // 128-byte column blocks per row
   static constexpr int kBoxCols = 128 / kElemBytes;          // elements per TMA box row
-  static constexpr int kTPW = kRowBytes == 128 ? 32 : 16;    // tokens per consumer warp per chunk
+  static constexpr int kNR = MQ ? 2 : 1;                     // MMA row halves used (upper 8 rows, or all 16)
+  static constexpr int kTPW = (kRowBytes == 128 && !MQ) ? 32 : 16;  // tokens per consumer warp per chunk
   static constexpr int kChunk = kConsumerWarps * kTPW;       // tokens per stage
   static constexpr int kSub = kTPW / 16;                     // 16-token MMA pieces per warp
   static constexpr int kHalfStride = kChunk * 128;           // bytes of one 128-byte column block of a tile
   static constexpr int kTileBytes = kHalves * kHalfStride;   // one K (or V) chunk
   static constexpr int kStageBytes = 2 * kTileBytes;
-  static constexpr int kStages = 3;
+  static constexpr int kStages = (96 * 1024) / kStageBytes;  // a 96 KB ring per CTA
   // per-thread output columns: NG groups of GW consecutive columns, group gi at gi*4*GW + GW*tq
   static constexpr int kGW = FP8 ? 4 : 2;
   static constexpr int kNG = D / (4 * kGW);
@@ -117,7 +118,7 @@ __device__ __forceinline__ uint32_t pack_f16x2(float lo, float hi) {
 
 
 struct SegmentInfo {
-  int b, tok0, tok1;
+  int b, tok0, tok1, len;
   bool valid;
 };
 
@@ -133,15 +134,16 @@ __device__ __forceinline__ SegmentInfo load_segment(const DecodeParams& p, const
   const int64_t t0 = (int64_t)sg.z * p.tile_tokens, t1 = min((int64_t)sg.w * p.tile_tokens, (int64_t)L);
   r.tok0 = (int)min(t0, (int64_t)L);
   r.tok1 = (int)t1;
+  r.len = L;
   return r;
 }
 
-template <int D, bool FP8>
+template <int D, bool FP8, bool MQ>
 __global__ void __launch_bounds__(kThreads, 2)
     decode_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap k64,
                   const __grid_constant__ CUtensorMap v64, const __grid_constant__ CUtensorMap k16,
                   const __grid_constant__ CUtensorMap v16) {
-  using C = Cfg<D, FP8>;
+  using C = Cfg<D, FP8, MQ>;
   constexpr int kChunk = C::kChunk;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -303,11 +305,29 @@ __global__ void __launch_bounds__(kThreads, 2)
   }
 
   // -------------------------------------------------------------------- consumer warps
-  constexpr int TPW = C::kTPW, SUB = C::kSub, HS = C::kHalfStride;
+  constexpr int TPW = C::kTPW, SUB = C::kSub, HS = C::kHalfStride, NR = C::kNR;
   const int w = warp;
-  const int r = lane >> 2;   // query head within the group (MMA row)
+  const int r = lane >> 2;   // MMA row within a row half
   const int tq = lane & 3;   // thread within the quad
-  const bool row_live = r < p.group;
+  // MMA row R = r + 8*hh (hh < NR) holds query qi = R / G of head hj = R % G of the group;
+  // when G * q_len <= 8 only the upper 8 rows are used (then q_len = 1 and R = r, the head).
+  const int qlen = MQ ? p.q_len : 1;
+  const int hq_rows = qlen * p.num_q_heads;  // output "heads" per request: q_len * Hq
+  int qi[NR], hj[NR];
+  bool live[NR];
+#pragma unroll
+  for (int hh = 0; hh < NR; ++hh) {
+    if constexpr (MQ) {
+      const int R = r + 8 * hh;
+      qi[hh] = R / p.group;
+      hj[hh] = R - qi[hh] * p.group;
+      live[hh] = qi[hh] < qlen;
+    } else {
+      qi[hh] = 0;
+      hj[hh] = r;
+      live[hh] = r < p.group;
+    }
+  }
   float* slots = reinterpret_cast<float*>(smem + C::kOffSlots);
   float* ml = reinterpret_cast<float*>(smem + C::kOffML);
   int stage = 0;
@@ -326,39 +346,66 @@ __global__ void __launch_bounds__(kThreads, 2)
   const float v_scale = FP8 ? __ldg(p.v_scale + g) : 1.f;
   const float score_scale = p.scale_log2 * k_scale;
 
+  // D += A * B for one m16n8k16 tile; A rows r (a0, a2) and r + 8 (a1, a3).
+  auto mma = [](float (&d)[2 * NR], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3, uint32_t b0, uint32_t b1) {
+    if constexpr (NR == 1) {
+      if constexpr (FP8) mma_f16_upper(d[0], d[1], a0, a2, b0, b1);
+      else mma_bf16_upper(d[0], d[1], a0, a2, b0, b1);
+    } else {
+      if constexpr (FP8) mma_f16_full(d, a0, a1, a2, a3, b0, b1);
+      else mma_bf16_full(d, a0, a1, a2, a3, b0, b1);
+    }
+  };
+
   for (int s = seg_lo; s < seg_hi; ++s) {
     const SegmentInfo si = load_segment(p, segs, s);
     if (!si.valid) continue;
     const int b = si.b;
+    // tokens row hh may see: all L for plain decode; L - q_len + qi + 1 for query qi
+    [[maybe_unused]] int vis[NR];
+#pragma unroll
+    for (int hh = 0; hh < NR; ++hh) vis[hh] = si.len - qlen + qi[hh] + 1;  // = len for plain decode
 
-    // Q fragments for rows r (upper half of the MMA tile); rows >= G are zero.
+    // Q fragments, per row half; rows past the queries are zero.
     // bf16: k-block kk holds columns 16kk + 2tq + {0,1} and + 8.
     // FP8:  k-block kk holds columns 16kk + 4tq + {0,1} and {2,3}, as f16 (the
     //       order in which ldmatrix hands out the bytes of a K row).
-    uint32_t qlo[D / 16], qhi[D / 16];
-    {
-      const __nv_bfloat16* qh = p.q + ((int64_t)b * p.num_q_heads + (int64_t)g * p.group + (row_live ? r : 0)) * D;
+    uint32_t qa[D / 16][NR][2];
+#pragma unroll
+    for (int hh = 0; hh < NR; ++hh) {
+      const __nv_bfloat16* qh =
+          p.q + (((int64_t)b * qlen + (live[hh] ? qi[hh] : 0)) * p.num_q_heads + (int64_t)g * p.group +
+                 (live[hh] ? hj[hh] : 0)) * D;
 #pragma unroll
       for (int kk = 0; kk < D / 16; ++kk) {
         if constexpr (FP8) {
-          const uint2 raw = row_live ? __ldg(reinterpret_cast<const uint2*>(qh) + 4 * kk + tq) : make_uint2(0, 0);
-          qlo[kk] = pack_f16x2(bf16_lo_to_f32(raw.x), bf16_hi_to_f32(raw.x));
-          qhi[kk] = pack_f16x2(bf16_lo_to_f32(raw.y), bf16_hi_to_f32(raw.y));
+          const uint2 raw = live[hh] ? __ldg(reinterpret_cast<const uint2*>(qh) + 4 * kk + tq) : make_uint2(0, 0);
+          qa[kk][hh][0] = pack_f16x2(bf16_lo_to_f32(raw.x), bf16_hi_to_f32(raw.x));
+          qa[kk][hh][1] = pack_f16x2(bf16_lo_to_f32(raw.y), bf16_hi_to_f32(raw.y));
         } else {
           const uint32_t* q32 = reinterpret_cast<const uint32_t*>(qh);
-          qlo[kk] = row_live ? __ldg(q32 + kk * 8 + tq) : 0u;
-          qhi[kk] = row_live ? __ldg(q32 + kk * 8 + 4 + tq) : 0u;
+          qa[kk][hh][0] = live[hh] ? __ldg(q32 + kk * 8 + tq) : 0u;
+          qa[kk][hh][1] = live[hh] ? __ldg(q32 + kk * 8 + 4 + tq) : 0u;
         }
       }
     }
+    auto qA = [&](int kk, int part, int hh) -> uint32_t { return hh < NR ? qa[kk][hh < NR ? hh : 0][part] : 0u; };
     // lr: sum of the rounded weights that enter P.V (normalises O), kept as an
-    //     MMA accumulator tile of P times ones (both entries hold the row sum);
+    //     MMA accumulator tile of P times ones (entries 2hh, 2hh+1 hold row half hh's sum);
     // l_e: per-thread sum of the unrounded fp32 weights (gives the log-sum-exp)
-    float m = -INFINITY, l_e = 0.f;
-    float lr[2] = {0.f, 0.f};
-    float o[D / 8][2];
+    float m[NR], l_e[NR];
+    float lr[2 * NR];
 #pragma unroll
-    for (int i = 0; i < D / 8; ++i) o[i][0] = o[i][1] = 0.f;
+    for (int hh = 0; hh < NR; ++hh) {
+      m[hh] = -INFINITY;
+      l_e[hh] = 0.f;
+      lr[2 * hh] = lr[2 * hh + 1] = 0.f;
+    }
+    float o[D / 8][2 * NR];
+#pragma unroll
+    for (int i = 0; i < D / 8; ++i)
+#pragma unroll
+      for (int e = 0; e < 2 * NR; ++e) o[i][e] = 0.f;
 
     for (int c0 = si.tok0; c0 < si.tok1; c0 += kChunk) {
       const bool got = mbar_wait_bounded(full0 + 8 * stage, phase, abort_flag, kWaitLimitNs);
@@ -367,7 +414,7 @@ __global__ void __launch_bounds__(kThreads, 2)
         *abort_flag = 1;
       }
       const int n = got ? meta[stage] : 0;
-      const int nw = min(max(n - TPW * w, 0), TPW);  // valid tokens in this warp's rows
+      const int nw = min(max(n - TPW * w, 0), TPW);  // loaded tokens in this warp's rows
       const uint32_t sk = sbase + C::kOffStages + stage * C::kStageBytes, sv = sk + C::kTileBytes;
       if (nw > 0) {
         if (nw < TPW) {
@@ -382,11 +429,20 @@ __global__ void __launch_bounds__(kThreads, 2)
           fence_proxy_async_smem();
           __syncwarp();
         }
+        // tokens of this warp's rows that row half hh may see
+        int lim[NR];
+#pragma unroll
+        for (int hh = 0; hh < NR; ++hh) {
+          if constexpr (MQ) lim[hh] = min(nw, max(vis[hh] - c0 - TPW * w, 0));
+          else lim[hh] = nw;  // a plain decode row sees every loaded token
+        }
         // S = Q . K^T for this warp's tokens: n-tile nt = tokens [8nt, 8nt+8) of the
         // warp; two accumulator chains (even / odd k-blocks) per n-tile.
-        float sc[2 * SUB][2][2];
+        float sc[2 * SUB][2][2 * NR];
 #pragma unroll
-        for (int nt = 0; nt < 2 * SUB; ++nt) sc[nt][0][0] = sc[nt][0][1] = sc[nt][1][0] = sc[nt][1][1] = 0.f;
+        for (int nt = 0; nt < 2 * SUB; ++nt)
+#pragma unroll
+          for (int e = 0; e < 2 * NR; ++e) sc[nt][0][e] = sc[nt][1][e] = 0.f;
 #pragma unroll
         for (int sp = 0; sp < SUB; ++sp) {
           const int ktok = k_tok + 16 * sp;
@@ -400,81 +456,99 @@ __global__ void __launch_bounds__(kThreads, 2)
               e4m3x4_to_f16x2x2(r1, b10, b11);
               e4m3x4_to_f16x2x2(r2, b20, b21);
               e4m3x4_to_f16x2x2(r3, b30, b31);
-              float(&a)[2][2] = sc[2 * sp];
-              float(&c)[2][2] = sc[2 * sp + 1];
-              mma_f16_upper(a[0][0], a[0][1], qlo[kk], qhi[kk], b00, b01);
-              mma_f16_upper(c[0][0], c[0][1], qlo[kk], qhi[kk], b10, b11);
-              mma_f16_upper(a[1][0], a[1][1], qlo[kk + 1], qhi[kk + 1], b20, b21);
-              mma_f16_upper(c[1][0], c[1][1], qlo[kk + 1], qhi[kk + 1], b30, b31);
+              mma(sc[2 * sp][0], qA(kk, 0, 0), qA(kk, 0, 1), qA(kk, 1, 0), qA(kk, 1, 1), b00, b01);
+              mma(sc[2 * sp + 1][0], qA(kk, 0, 0), qA(kk, 0, 1), qA(kk, 1, 0), qA(kk, 1, 1), b10, b11);
+              mma(sc[2 * sp][1], qA(kk + 1, 0, 0), qA(kk + 1, 0, 1), qA(kk + 1, 1, 0), qA(kk + 1, 1, 1), b20, b21);
+              mma(sc[2 * sp + 1][1], qA(kk + 1, 0, 0), qA(kk + 1, 0, 1), qA(kk + 1, 1, 0), qA(kk + 1, 1, 1), b30,
+                  b31);
             }
           } else {
 #pragma unroll
             for (int kk = 0; kk < D / 16; ++kk) {
               uint32_t b0, b1, b2, b3;
               ldmatrix_x4(sk + swz<HS>(ktok, 2 * kk + k_chk), b0, b1, b2, b3);
-              float(&a)[2] = sc[2 * sp][kk & 1];
-              float(&c)[2] = sc[2 * sp + 1][kk & 1];
-              mma_bf16_upper(a[0], a[1], qlo[kk], qhi[kk], b0, b1);
-              mma_bf16_upper(c[0], c[1], qlo[kk], qhi[kk], b2, b3);
+              mma(sc[2 * sp][kk & 1], qA(kk, 0, 0), qA(kk, 0, 1), qA(kk, 1, 0), qA(kk, 1, 1), b0, b1);
+              mma(sc[2 * sp + 1][kk & 1], qA(kk, 0, 0), qA(kk, 0, 1), qA(kk, 1, 0), qA(kk, 1, 1), b2, b3);
             }
           }
         }
-        // scale to base 2, mask the tail (only in a partial chunk), online softmax update
-        float x[2 * SUB][2];
+        // scale to base 2, mask what a row may not see (only in a partial chunk or at
+        // a query's causal edge), online softmax update per row half
+        float x[2 * SUB][NR][2];
 #pragma unroll
         for (int nt = 0; nt < 2 * SUB; ++nt)
 #pragma unroll
-          for (int e = 0; e < 2; ++e) x[nt][e] = (sc[nt][0][e] + sc[nt][1][e]) * score_scale;
-        if (nw < TPW) {
+          for (int hh = 0; hh < NR; ++hh)
+#pragma unroll
+            for (int e = 0; e < 2; ++e) x[nt][hh][e] = (sc[nt][0][2 * hh + e] + sc[nt][1][2 * hh + e]) * score_scale;
+        bool partial = lim[0] < TPW;
+        if constexpr (NR == 2) partial = partial || lim[1] < TPW;
+        if (__any_sync(0xffffffffu, partial)) {
 #pragma unroll
           for (int nt = 0; nt < 2 * SUB; ++nt)
 #pragma unroll
-            for (int e = 0; e < 2; ++e)
-              if (8 * nt + 2 * tq + e >= nw) x[nt][e] = -INFINITY;
-        }
-        float mx = -INFINITY;
+            for (int hh = 0; hh < NR; ++hh)
 #pragma unroll
-        for (int nt = 0; nt < 2 * SUB; ++nt) mx = fmaxf(mx, fmaxf(x[nt][0], x[nt][1]));
-        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
-        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
-        const float m_new = fmaxf(m, mx);
-        const float m_use = m_new == -INFINITY ? 0.f : m_new;
-        const float corr = fast_exp2(m - m_use);
-        uint32_t pa[SUB][2];
-        float exact = 0.f;
+              for (int e = 0; e < 2; ++e)
+                if (8 * nt + 2 * tq + e >= lim[hh]) x[nt][hh][e] = -INFINITY;
+        }
+        float corr[NR], m_use[NR];
+        bool moved = false;
+#pragma unroll
+        for (int hh = 0; hh < NR; ++hh) {
+          float mx = -INFINITY;
+#pragma unroll
+          for (int nt = 0; nt < 2 * SUB; ++nt) mx = fmaxf(mx, fmaxf(x[nt][hh][0], x[nt][hh][1]));
+          mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
+          mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
+          const float m_new = fmaxf(m[hh], mx);
+          m_use[hh] = m_new == -INFINITY ? 0.f : m_new;
+          corr[hh] = fast_exp2(m[hh] - m_use[hh]);
+          moved = moved || corr[hh] != 1.f;
+          m[hh] = m_new;
+        }
+        // P fragments (A operand of P.V): rows r (a0, a2) and r + 8 (a1, a3),
+        // tokens 0-7 of the piece in a0/a1 and 8-15 in a2/a3
+        uint32_t pa[SUB][4];
 #pragma unroll
         for (int sp = 0; sp < SUB; ++sp) {
-          const float p00 = fast_exp2(x[2 * sp][0] - m_use), p01 = fast_exp2(x[2 * sp][1] - m_use);
-          const float p10 = fast_exp2(x[2 * sp + 1][0] - m_use), p11 = fast_exp2(x[2 * sp + 1][1] - m_use);
-          if constexpr (FP8) {
-            pa[sp][0] = pack_f16x2(p00, p01);
-            pa[sp][1] = pack_f16x2(p10, p11);
-          } else {
-            pa[sp][0] = pack_bf16x2(p00, p01);
-            pa[sp][1] = pack_bf16x2(p10, p11);
-          }
-          exact += (p00 + p01) + (p10 + p11);
-        }
-        l_e = l_e * corr + exact;
-        m = m_new;
-        if (!__all_sync(0xffffffffu, corr == 1.f)) {  // some row's running max moved
 #pragma unroll
-          for (int i = 0; i < D / 8; ++i) {
-            o[i][0] *= corr;
-            o[i][1] *= corr;
+          for (int hh = 0; hh < 2; ++hh) {
+            if (hh >= NR) {
+              pa[sp][hh] = pa[sp][2 + hh] = 0u;
+              continue;
+            }
+            const int h2 = hh < NR ? hh : 0;
+            const float p00 = fast_exp2(x[2 * sp][h2][0] - m_use[h2]), p01 = fast_exp2(x[2 * sp][h2][1] - m_use[h2]);
+            const float p10 = fast_exp2(x[2 * sp + 1][h2][0] - m_use[h2]);
+            const float p11 = fast_exp2(x[2 * sp + 1][h2][1] - m_use[h2]);
+            if constexpr (FP8) {
+              pa[sp][hh] = pack_f16x2(p00, p01);
+              pa[sp][2 + hh] = pack_f16x2(p10, p11);
+            } else {
+              pa[sp][hh] = pack_bf16x2(p00, p01);
+              pa[sp][2 + hh] = pack_bf16x2(p10, p11);
+            }
+            l_e[h2] = (sp == 0 ? l_e[h2] * corr[h2] : l_e[h2]) + ((p00 + p01) + (p10 + p11));
           }
-          lr[0] *= corr;
-          lr[1] *= corr;
+        }
+        if (__any_sync(0xffffffffu, moved)) {  // some row's running max moved
+#pragma unroll
+          for (int hh = 0; hh < NR; ++hh) {
+#pragma unroll
+            for (int i = 0; i < D / 8; ++i) {
+              o[i][2 * hh] *= corr[hh];
+              o[i][2 * hh + 1] *= corr[hh];
+            }
+            lr[2 * hh] *= corr[hh];
+            lr[2 * hh + 1] *= corr[hh];
+          }
         }
         // the sum of the rounded weights, as the tensor core sees them: P times a
         // column block of ones (every column of the tile holds the row sum)
+        constexpr uint32_t kOnes = FP8 ? 0x3C003C00u : 0x3F803F80u;
 #pragma unroll
-        for (int sp = 0; sp < SUB; ++sp) {
-          if constexpr (FP8)
-            mma_f16_upper(lr[0], lr[1], pa[sp][0], pa[sp][1], 0x3C003C00u, 0x3C003C00u);
-          else
-            mma_bf16_upper(lr[0], lr[1], pa[sp][0], pa[sp][1], 0x3F803F80u, 0x3F803F80u);
-        }
+        for (int sp = 0; sp < SUB; ++sp) mma(lr, pa[sp][0], pa[sp][1], pa[sp][2], pa[sp][3], kOnes, kOnes);
         // O += P . V, one k-step of 16 tokens per piece
 #pragma unroll
         for (int sp = 0; sp < SUB; ++sp) {
@@ -493,18 +567,18 @@ __global__ void __launch_bounds__(kThreads, 2)
               e4m3x4_to_f16x2x2(__byte_perm(r1, 0, 0x3120), e1, o1);
               e4m3x4_to_f16x2x2(__byte_perm(r2, 0, 0x3120), e2, o2);
               e4m3x4_to_f16x2x2(__byte_perm(r3, 0, 0x3120), e3, o3);
-              mma_f16_upper(o[2 * c][0], o[2 * c][1], pa[sp][0], pa[sp][1], e0, e1);
-              mma_f16_upper(o[2 * c + 1][0], o[2 * c + 1][1], pa[sp][0], pa[sp][1], o0, o1);
-              mma_f16_upper(o[2 * c + 2][0], o[2 * c + 2][1], pa[sp][0], pa[sp][1], e2, e3);
-              mma_f16_upper(o[2 * c + 3][0], o[2 * c + 3][1], pa[sp][0], pa[sp][1], o2, o3);
+              mma(o[2 * c], pa[sp][0], pa[sp][1], pa[sp][2], pa[sp][3], e0, e1);
+              mma(o[2 * c + 1], pa[sp][0], pa[sp][1], pa[sp][2], pa[sp][3], o0, o1);
+              mma(o[2 * c + 2], pa[sp][0], pa[sp][1], pa[sp][2], pa[sp][3], e2, e3);
+              mma(o[2 * c + 3], pa[sp][0], pa[sp][1], pa[sp][2], pa[sp][3], o2, o3);
             }
           } else {
 #pragma unroll
             for (int np = 0; np < D / 16; ++np) {
               uint32_t v0, v1, v2, v3;
               ldmatrix_x4_trans(sv + swz<HS>(vtok, 2 * np + v_chk), v0, v1, v2, v3);
-              mma_bf16_upper(o[2 * np][0], o[2 * np][1], pa[sp][0], pa[sp][1], v0, v1);
-              mma_bf16_upper(o[2 * np + 1][0], o[2 * np + 1][1], pa[sp][0], pa[sp][1], v2, v3);
+              mma(o[2 * np], pa[sp][0], pa[sp][1], pa[sp][2], pa[sp][3], v0, v1);
+              mma(o[2 * np + 1], pa[sp][0], pa[sp][1], pa[sp][2], pa[sp][3], v2, v3);
             }
           }
         }
@@ -517,113 +591,117 @@ __global__ void __launch_bounds__(kThreads, 2)
       }
     }
 
-    // ---- regroup this thread's columns: og[gi][j] is column gi*4*GW + GW*tq + j
-    constexpr int GW = C::kGW, NG = C::kNG;
-    float og[NG][GW];
+    // ---- merge the four warp states of this segment, one row half at a time
+    const int nseg_b = rsb[b + 1] - rsb[b];
+    const bool direct = nseg_b == 1;
 #pragma unroll
-    for (int gi = 0; gi < NG; ++gi) {
-      if constexpr (FP8) {  // tiles 2gi (even columns) and 2gi+1 (odd columns) of chunk gi
-        og[gi][0] = o[2 * gi][0];
-        og[gi][1] = o[2 * gi + 1][0];
-        og[gi][2] = o[2 * gi][1];
-        og[gi][3] = o[2 * gi + 1][1];
-      } else {
-        og[gi][0] = o[gi][0];
-        og[gi][1] = o[gi][1];
-      }
-    }
-
-    // ---- merge the four warp states of this segment
-    const float l_r = lr[0];  // already the full row sum over the warp's tokens
-    l_e += __shfl_xor_sync(0xffffffffu, l_e, 1);
-    l_e += __shfl_xor_sync(0xffffffffu, l_e, 2);
-    if (w > 0) {
-      float* slot = slots + (w - 1) * C::kSlotFloats + r * C::kSlotStride + GW * tq;
+    for (int hh = 0; hh < NR; ++hh) {
+      // regroup this thread's columns: og[gi][j] is column gi*4*GW + GW*tq + j
+      constexpr int GW = C::kGW, NG = C::kNG;
+      float og[NG][GW];
 #pragma unroll
       for (int gi = 0; gi < NG; ++gi) {
-        if constexpr (GW == 4)
-          *reinterpret_cast<float4*>(slot + 16 * gi) = make_float4(og[gi][0], og[gi][1], og[gi][2], og[gi][3]);
-        else
-          *reinterpret_cast<float2*>(slot + 8 * gi) = make_float2(og[gi][0], og[gi][1]);
+        if constexpr (FP8) {  // tiles 2gi (even columns) and 2gi+1 (odd columns) of chunk gi
+          og[gi][0] = o[2 * gi][2 * hh];
+          og[gi][1] = o[2 * gi + 1][2 * hh];
+          og[gi][2] = o[2 * gi][2 * hh + 1];
+          og[gi][3] = o[2 * gi + 1][2 * hh + 1];
+        } else {
+          og[gi][0] = o[gi][2 * hh];
+          og[gi][1] = o[gi][2 * hh + 1];
+        }
       }
-      if (tq == 0) {
-        ml[(w - 1) * 24 + r] = m;
-        ml[(w - 1) * 24 + 8 + r] = l_r;
-        ml[(w - 1) * 24 + 16 + r] = l_e;
+      const float l_r = lr[2 * hh];  // already the full row sum over the warp's tokens
+      float le = l_e[hh];
+      le += __shfl_xor_sync(0xffffffffu, le, 1);
+      le += __shfl_xor_sync(0xffffffffu, le, 2);
+      if (w > 0) {
+        float* slot = slots + (w - 1) * C::kSlotFloats + r * C::kSlotStride + GW * tq;
+#pragma unroll
+        for (int gi = 0; gi < NG; ++gi) {
+          if constexpr (GW == 4)
+            *reinterpret_cast<float4*>(slot + 16 * gi) = make_float4(og[gi][0], og[gi][1], og[gi][2], og[gi][3]);
+          else
+            *reinterpret_cast<float2*>(slot + 8 * gi) = make_float2(og[gi][0], og[gi][1]);
+        }
+        if (tq == 0) {
+          ml[(w - 1) * 24 + r] = m[hh];
+          ml[(w - 1) * 24 + 8 + r] = l_r;
+          ml[(w - 1) * 24 + 16 + r] = le;
+        }
       }
-    }
-    named_barrier_sync(1, kConsumerWarps * 32);
-    if (w == 0) {
-      float mw[3], lrw[3], lew[3];
-      float M = m;
-#pragma unroll
-      for (int j = 0; j < 3; ++j) {
-        mw[j] = ml[j * 24 + r];
-        lrw[j] = ml[j * 24 + 8 + r];
-        lew[j] = ml[j * 24 + 16 + r];
-        M = fmaxf(M, mw[j]);
-      }
-      const bool empty = M == -INFINITY;
-      const float f0 = empty ? 0.f : fast_exp2(m - M);
-      float fw[3];
-      float Lr = f0 * l_r, Le = f0 * l_e;
-#pragma unroll
-      for (int j = 0; j < 3; ++j) {
-        fw[j] = empty ? 0.f : fast_exp2(mw[j] - M);
-        Lr += fw[j] * lrw[j];
-        Le += fw[j] * lew[j];
-      }
-      const float inv = Lr > 0.f ? v_scale / Lr : 0.f;
-      const float lse_nat = Le > 0.f ? (M + log2f(Le)) * 0.69314718055994530942f : -INFINITY;
-      const int h = g * p.group + r;
-      const int nseg_b = rsb[b + 1] - rsb[b];
-      const bool direct = nseg_b == 1;
-#pragma unroll
-      for (int gi = 0; gi < NG; ++gi) {
-        float a[GW];
-#pragma unroll
-        for (int e = 0; e < GW; ++e) a[e] = f0 * og[gi][e];
+      named_barrier_sync(1, kConsumerWarps * 32);
+      if (w == 0) {
+        float mw[3], lrw[3], lew[3];
+        float M = m[hh];
 #pragma unroll
         for (int j = 0; j < 3; ++j) {
-          const float* src = slots + j * C::kSlotFloats + r * C::kSlotStride + gi * 4 * GW + GW * tq;
-#pragma unroll
-          for (int e = 0; e < GW; ++e) a[e] += fw[j] * src[e];
+          mw[j] = ml[j * 24 + r];
+          lrw[j] = ml[j * 24 + 8 + r];
+          lew[j] = ml[j * 24 + 16 + r];
+          M = fmaxf(M, mw[j]);
         }
+        const bool empty = M == -INFINITY;
+        const float f0 = empty ? 0.f : fast_exp2(m[hh] - M);
+        float fw[3];
+        float Lr = f0 * l_r, Le = f0 * le;
 #pragma unroll
-        for (int e = 0; e < GW; ++e) og[gi][e] = a[e] * inv;
-      }
-      if (row_live) {
-        if (direct) {
-          __nv_bfloat16* dst = p.out + ((int64_t)b * p.num_q_heads + h) * D + GW * tq;
+        for (int j = 0; j < 3; ++j) {
+          fw[j] = empty ? 0.f : fast_exp2(mw[j] - M);
+          Lr += fw[j] * lrw[j];
+          Le += fw[j] * lew[j];
+        }
+        const float inv = Lr > 0.f ? v_scale / Lr : 0.f;
+        const float lse_nat = Le > 0.f ? (M + log2f(Le)) * 0.69314718055994530942f : -INFINITY;
 #pragma unroll
-          for (int gi = 0; gi < NG; ++gi) {
-            if constexpr (GW == 4)
-              *reinterpret_cast<uint2*>(dst + 16 * gi) =
-                  make_uint2(pack_bf16x2(og[gi][0], og[gi][1]), pack_bf16x2(og[gi][2], og[gi][3]));
-            else
-              *reinterpret_cast<uint32_t*>(dst + 8 * gi) = pack_bf16x2(og[gi][0], og[gi][1]);
+        for (int gi = 0; gi < NG; ++gi) {
+          float a[GW];
+#pragma unroll
+          for (int e = 0; e < GW; ++e) a[e] = f0 * og[gi][e];
+#pragma unroll
+          for (int j = 0; j < 3; ++j) {
+            const float* src = slots + j * C::kSlotFloats + r * C::kSlotStride + gi * 4 * GW + GW * tq;
+#pragma unroll
+            for (int e = 0; e < GW; ++e) a[e] += fw[j] * src[e];
           }
-          if (tq == 0) p.lse[(int64_t)b * p.num_q_heads + h] = lse_nat;
-        } else {
-          float* dst = p.partial_o + ((int64_t)s * p.num_q_heads + h) * D + GW * tq;
 #pragma unroll
-          for (int gi = 0; gi < NG; ++gi) {
-            if constexpr (GW == 4)
-              *reinterpret_cast<float4*>(dst + 16 * gi) = make_float4(og[gi][0], og[gi][1], og[gi][2], og[gi][3]);
-            else
-              *reinterpret_cast<float2*>(dst + 8 * gi) = make_float2(og[gi][0], og[gi][1]);
+          for (int e = 0; e < GW; ++e) og[gi][e] = a[e] * inv;
+        }
+        if (live[hh]) {
+          // output row: query qi, head g*G + hj, i.e. "head" qi*Hq + g*G + hj of q_len*Hq
+          const int hrow = qi[hh] * p.num_q_heads + g * p.group + hj[hh];
+          if (direct) {
+            __nv_bfloat16* dst = p.out + ((int64_t)b * hq_rows + hrow) * D + GW * tq;
+#pragma unroll
+            for (int gi = 0; gi < NG; ++gi) {
+              if constexpr (GW == 4)
+                *reinterpret_cast<uint2*>(dst + 16 * gi) =
+                    make_uint2(pack_bf16x2(og[gi][0], og[gi][1]), pack_bf16x2(og[gi][2], og[gi][3]));
+              else
+                *reinterpret_cast<uint32_t*>(dst + 8 * gi) = pack_bf16x2(og[gi][0], og[gi][1]);
+            }
+            if (tq == 0) p.lse[(int64_t)b * hq_rows + hrow] = lse_nat;
+          } else {
+            float* dst = p.partial_o + ((int64_t)s * hq_rows + hrow) * D + GW * tq;
+#pragma unroll
+            for (int gi = 0; gi < NG; ++gi) {
+              if constexpr (GW == 4)
+                *reinterpret_cast<float4*>(dst + 16 * gi) = make_float4(og[gi][0], og[gi][1], og[gi][2], og[gi][3]);
+              else
+                *reinterpret_cast<float2*>(dst + 8 * gi) = make_float2(og[gi][0], og[gi][1]);
+            }
+            if (tq == 0) p.partial_lse[(int64_t)s * hq_rows + hrow] = lse_nat;
           }
-          if (tq == 0) p.partial_lse[(int64_t)s * p.num_q_heads + h] = lse_nat;
         }
       }
+      named_barrier_sync(1, kConsumerWarps * 32);  // slots are free again
     }
-    named_barrier_sync(1, kConsumerWarps * 32);  // slots are free again
   }
 }
 
-template <int D, bool FP8>
+template <int D, bool FP8, bool MQ>
 cudaError_t launch_decode_d(const DecodeParams& p, const CUtensorMap maps[4], cudaStream_t stream) {
-  using C = Cfg<D, FP8>;
+  using C = Cfg<D, FP8, MQ>;
   static_assert(C::kSmemRequest * 2 <= 227 * 1024, "two CTAs per SM must fit");
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
@@ -631,7 +709,8 @@ cudaError_t launch_decode_d(const DecodeParams& p, const CUtensorMap maps[4], cu
   static bool configured[64] = {false};
   if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
   if (!configured[dev]) {
-    e = cudaFuncSetAttribute(decode_kernel<D, FP8>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemRequest);
+    e = cudaFuncSetAttribute(decode_kernel<D, FP8, MQ>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             C::kSmemRequest);
     if (e != cudaSuccess) return e;
     configured[dev] = true;
   }
@@ -645,19 +724,24 @@ cudaError_t launch_decode_d(const DecodeParams& p, const CUtensorMap maps[4], cu
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, decode_kernel<D, FP8>, p, maps[0], maps[1], maps[2], maps[3]);
+  return cudaLaunchKernelEx(&cfg, decode_kernel<D, FP8, MQ>, p, maps[0], maps[1], maps[2], maps[3]);
 }
 
 }  // namespace
 
 cudaError_t launch_decode(const DecodeParams& p, int head_dim, const CUtensorMap maps[4], cudaStream_t stream) {
-  if (head_dim == 128) return launch_decode_d<128, false>(p, maps, stream);
-  if (head_dim == 64) return launch_decode_d<64, false>(p, maps, stream);
+  const bool mq = p.full_rows != 0;
+  if (head_dim == 128) return mq ? launch_decode_d<128, false, true>(p, maps, stream)
+                                 : launch_decode_d<128, false, false>(p, maps, stream);
+  if (head_dim == 64) return mq ? launch_decode_d<64, false, true>(p, maps, stream)
+                                : launch_decode_d<64, false, false>(p, maps, stream);
   return cudaErrorInvalidValue;
 }
 
 cudaError_t launch_decode_fp8(const DecodeParams& p, int head_dim, const CUtensorMap maps[4], cudaStream_t stream) {
-  if (head_dim == 128) return launch_decode_d<128, true>(p, maps, stream);
+  const bool mq = p.full_rows != 0;
+  if (head_dim == 128) return mq ? launch_decode_d<128, true, true>(p, maps, stream)
+                                 : launch_decode_d<128, true, false>(p, maps, stream);
   return cudaErrorInvalidValue;
 }
 

@@ -30,7 +30,7 @@ NOALLOC_SCRATCH_BYTES = 16 << 20  # DA_NOALLOC_SCRATCH_BYTES
 class DaProblem(ctypes.Structure):
     _fields_ = [("batch", ctypes.c_int32), ("num_q_heads", ctypes.c_int32), ("num_kv_heads", ctypes.c_int32),
                 ("head_dim", ctypes.c_int32), ("page_size", ctypes.c_int32), ("max_pages_per_req", ctypes.c_int32),
-                ("num_pages", ctypes.c_int32), ("scale", ctypes.c_float)]
+                ("num_pages", ctypes.c_int32), ("scale", ctypes.c_float), ("q_len", ctypes.c_int32)]
 
 
 class DaPlanDesc(ctypes.Structure):
@@ -102,15 +102,16 @@ def _check(fn: str, rc: int):
         raise DaError(fn, rc, lib().da_last_cuda_error() if rc == ERR_CUDA else 0)
 
 
-def problem(batch, num_q_heads, num_kv_heads, head_dim, page_size, max_pages_per_req, num_pages, scale) -> DaProblem:
+def problem(batch, num_q_heads, num_kv_heads, head_dim, page_size, max_pages_per_req, num_pages, scale,
+            q_len: int = 1) -> DaProblem:
     return DaProblem(int(batch), int(num_q_heads), int(num_kv_heads), int(head_dim), int(page_size),
-                     int(max_pages_per_req), int(num_pages), float(scale))
+                     int(max_pages_per_req), int(num_pages), float(scale), int(q_len))
 
 
 def problem_from(p) -> DaProblem:
     """From any object with the da_problem field names (e.g. workloads.Problem)."""
     return problem(p.batch, p.num_q_heads, p.num_kv_heads, p.head_dim, p.page_size, p.max_pages_per_req,
-                   p.num_pages, p.scale)
+                   p.num_pages, p.scale, getattr(p, "q_len", 1))
 
 
 def _ptr(t) -> int | None:
@@ -219,8 +220,9 @@ class Buffers:
         self.ws = torch.zeros(max(ws // 4, 4), dtype=torch.int32, device=device)
         self.partial_o = torch.empty(max(po // 4, 4), dtype=torch.float32, device=device)
         self.partial_lse = torch.empty(max(pl // 4, 1), dtype=torch.float32, device=device)
-        self.out = torch.empty((prob.batch, prob.num_q_heads, prob.head_dim), dtype=torch.bfloat16, device=device)
-        self.lse = torch.empty((prob.batch, prob.num_q_heads), dtype=torch.float32, device=device)
+        lead = (prob.batch,) if prob.q_len <= 1 else (prob.batch, prob.q_len)
+        self.out = torch.empty(lead + (prob.num_q_heads, prob.head_dim), dtype=torch.bfloat16, device=device)
+        self.lse = torch.empty(lead + (prob.num_q_heads,), dtype=torch.float32, device=device)
 
 
 def decode_step(prob, desc, q, k_cache, v_cache, block_table, seq_lens, bufs: Buffers, stream=None, k_scale=None,

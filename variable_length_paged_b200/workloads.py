@@ -17,7 +17,8 @@ integers and ``torch.Generator().manual_seed(seed)`` for values):
      the requests in order; unused block-table entries hold -1;
   3. K rows picked as outliers (Bernoulli per token row, shared by all KV
      heads of that row), when the config asks for them;
-  4. q ~ N(0,1), then K ~ N(0,1) (outlier rows multiplied before rounding),
+  4. q ~ N(0,1) ([B, Hq, d], or [B, q_len, Hq, d] for multi-query decode),
+     then K ~ N(0,1) (outlier rows multiplied before rounding),
      then V ~ N(0,1), each rounded to bf16 (round-to-nearest-even);
   5. slots past the end of each request and the spare pages are filled with
      NaN ("poison"), so that any read outside the valid tokens shows up.
@@ -44,6 +45,7 @@ class Problem:
     max_pages_per_req: int
     num_pages: int
     scale: float  # an fp32 value; both sides use exactly this number
+    q_len: int = 1  # queries per request (the last q_len cached tokens)
 
     @property
     def group(self) -> int:
@@ -120,7 +122,7 @@ def make_workload(name: str, seq_lens, *, num_q_heads: int, num_kv_heads: int, h
                   seed: int, scale: float | None = None, rng: np.random.Generator | None = None,
                   outlier_frac: float = 0.0, outlier_mult: float = 8.0, spare_frac: float = 0.05,
                   shuffle_pages: bool = True, poison: bool = True, max_pages_per_req: int | None = None,
-                  extra_pages: int = 0, recipe: str = "") -> Workload:
+                  extra_pages: int = 0, recipe: str = "", q_len: int = 1) -> Workload:
     """Build a paged workload for given lengths (steps 2-5 of the module recipe)."""
     rng = rng if rng is not None else np.random.default_rng(seed)
     gen = torch.Generator().manual_seed(seed)
@@ -152,7 +154,7 @@ def make_workload(name: str, seq_lens, *, num_q_heads: int, num_kv_heads: int, h
             row_scale[block_table[b, t // P], t % P] = outlier_mult
 
     scale = _fp32(1.0 / math.sqrt(head_dim)) if scale is None else _fp32(scale)
-    q = _randn_bf16(gen, (B, num_q_heads, head_dim))
+    q = _randn_bf16(gen, (B, num_q_heads, head_dim) if q_len == 1 else (B, q_len, num_q_heads, head_dim))
     shape = (num_pages, num_kv_heads, P, head_dim)
     k = _randn_bf16(gen, shape, row_scale)
     v = _randn_bf16(gen, shape)
@@ -171,7 +173,8 @@ def make_workload(name: str, seq_lens, *, num_q_heads: int, num_kv_heads: int, h
             cache.permute(0, 2, 1, 3)[dead] = nan
 
     problem = Problem(batch=B, num_q_heads=num_q_heads, num_kv_heads=num_kv_heads, head_dim=head_dim,
-                      page_size=P, max_pages_per_req=max_pages_per_req, num_pages=num_pages, scale=scale)
+                      page_size=P, max_pages_per_req=max_pages_per_req, num_pages=num_pages, scale=scale,
+                      q_len=q_len)
     return Workload(name=name, problem=problem, seq_lens=lens.astype(np.int32), block_table=block_table,
                     q=q, k_cache=k, v_cache=v, seed=seed, recipe=recipe)
 
