@@ -271,8 +271,9 @@ static int decode_common(const da_problem* prob, const da_plan_desc* desc, const
   p.capacity_tokens = (int64_t)prob->max_pages_per_req * prob->page_size;
   p.scale_log2 = prob->scale * 1.4426950408889634f;
   p.q_len = q_len_of(prob);
-  // more than 8 rows (G > 8, or several queries) take the kernel that uses all 16 MMA rows
-  p.full_rows = p.group * p.q_len > 8 ? 1 : 0;
+  // several queries per request, or more than 8 heads per group, take the kernel that maps
+  // (query, head) rows over all 16 MMA rows; plain decode with G <= 8 uses the upper 8
+  p.full_rows = (p.q_len > 1 || p.group > 8) ? 1 : 0;
   cudaError_t e = fp8 ? da::launch_decode_fp8(p, prob->head_dim, maps, static_cast<cudaStream_t>(stream))
                       : da::launch_decode(p, prob->head_dim, maps, static_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? DA_OK : cuda_fail(e);

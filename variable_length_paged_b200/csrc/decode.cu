@@ -310,7 +310,7 @@ __global__ void __launch_bounds__(kThreads, 2)
   const int r = lane >> 2;   // MMA row within a row half
   const int tq = lane & 3;   // thread within the quad
   // MMA row R = r + 8*hh (hh < NR) holds query qi = R / G of head hj = R % G of the group;
-  // when G * q_len <= 8 only the upper 8 rows are used (then q_len = 1 and R = r, the head).
+  // plain decode with G <= 8 uses only the upper 8 rows (R = r, the head).
   const int qlen = MQ ? p.q_len : 1;
   const int hq_rows = qlen * p.num_q_heads;  // output "heads" per request: q_len * Hq
   int qi[NR], hj[NR];
