@@ -71,7 +71,7 @@ struct DecodeParams {
   const float* k_scale;  // FP8 caches: per-KV-head dequantisation scales (else null)
   const float* v_scale;
   int32_t q_len;  // queries per request (1 = plain decode)
-  int32_t full_rows;  // 1: G * q_len > 8, all 16 MMA rows carry (query, head) rows
+  int32_t full_rows;  // 1: q_len > 1 or G > 8: all 16 MMA rows carry (query, head) rows
 };
 
 struct CombineParams {
