@@ -264,6 +264,23 @@ DA_API int da_append_kv(const da_problem* prob, const void* new_k, const void* n
                         const int32_t* seq_lens, void* k_cache, void* v_cache, int32_t* status, void* stream);
 
 /*
+ * da_merge_partials -- merge results computed over disjoint token slices of
+ * the same requests (e.g. one slice per GPU when a long request's KV cache is
+ * spread over several GPUs and each GPU runs the decode step on its slice):
+ *   LSE = M + ln sum_j exp(lse_j - M),  M = max_j lse_j,
+ *   out = sum_j exp(lse_j - LSE) * out_j   (fp32 sums in part order, then bf16);
+ * parts with lse = -inf (empty slices) carry no weight; all empty gives 0, -inf.
+ *   part_out  dev bf16 [num_parts][rows][head_dim] (each part's `out`, 8-byte aligned)
+ *   part_lse  dev fp32 [num_parts][rows]
+ *   out, lse  dev bf16 [rows][head_dim], fp32 [rows]; rows = batch * q_len * num_q_heads.
+ * Source: "Tencent HPC lands in SGLang, challenging default inference
+ * kernels", section "Why Tencent HPC matters for online model serving"
+ * (longer histories mean more cached data to read).
+ */
+DA_API int da_merge_partials(int32_t num_parts, int64_t rows, int32_t head_dim, const void* part_out,
+                             const float* part_lse, void* out, float* lse, void* stream);
+
+/*
  * da_read_status -- copy the device status word and first bad index out of
  * `ws` (host outputs; either may be NULL).  Synchronises `stream`.
  */

@@ -349,6 +349,25 @@ DA_API int da_append_kv(const da_problem* prob, const void* new_k, const void* n
   return e == cudaSuccess ? DA_OK : cuda_fail(e);
 }
 
+DA_API int da_merge_partials(int32_t num_parts, int64_t rows, int32_t head_dim, const void* part_out,
+                             const float* part_lse, void* out, float* lse, void* stream) {
+  if (num_parts <= 0 || rows < 0) return DA_ERR_INVALID_ARG;
+  if (head_dim != 64 && head_dim != 128) return DA_ERR_UNSUPPORTED;
+  if (rows == 0) return DA_OK;
+  if (!part_out || !part_lse || !out || !lse) return DA_ERR_INVALID_ARG;
+  if (reinterpret_cast<uintptr_t>(part_out) % 8 != 0 || reinterpret_cast<uintptr_t>(out) % 8 != 0)
+    return DA_ERR_INVALID_ARG;
+  da::MergeParams p;
+  p.part_out = static_cast<const __nv_bfloat16*>(part_out);
+  p.part_lse = part_lse;
+  p.out = static_cast<__nv_bfloat16*>(out);
+  p.lse = lse;
+  p.num_parts = num_parts;
+  p.rows = rows;
+  cudaError_t e = da::launch_merge(p, head_dim, static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? DA_OK : cuda_fail(e);
+}
+
 DA_API int da_read_status(const void* ws, int32_t* dev_status, int32_t* bad_index, void* stream) {
   if (!ws) return DA_ERR_INVALID_ARG;
   int32_t h[da::kHdrWords];

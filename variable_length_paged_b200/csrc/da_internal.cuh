@@ -95,6 +95,15 @@ struct AppendParams {
   int64_t capacity_tokens;
 };
 
+struct MergeParams {
+  const __nv_bfloat16* part_out;  // [num_parts][rows][head_dim]
+  const float* part_lse;          // [num_parts][rows]
+  __nv_bfloat16* out;             // [rows][head_dim]
+  float* lse;                     // [rows]
+  int32_t num_parts;
+  int64_t rows;
+};
+
 // Host launchers (defined next to their kernels).
 cudaError_t launch_plan_dynamic(const PlanParams& p, cudaStream_t stream);
 cudaError_t launch_plan_static(const PlanParams& p, cudaStream_t stream);
@@ -102,6 +111,7 @@ cudaError_t launch_decode(const DecodeParams& p, int head_dim, const CUtensorMap
 cudaError_t launch_decode_fp8(const DecodeParams& p, int head_dim, const CUtensorMap maps[4], cudaStream_t stream);
 cudaError_t launch_combine(const CombineParams& p, int head_dim, cudaStream_t stream);
 cudaError_t launch_append(const AppendParams& p, cudaStream_t stream);
+cudaError_t launch_merge(const MergeParams& p, int head_dim, cudaStream_t stream);
 
 // Record a CUDA error for da_last_cuda_error() from code outside api.cu.
 void set_last_cuda_error(cudaError_t e);

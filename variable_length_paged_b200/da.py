@@ -22,7 +22,7 @@ PLAN_DYNAMIC, PLAN_STATIC = 0, 1
 EXPORTS = ("da_plan_desc_init", "da_workspace_size", "da_workspace_offsets", "da_plan", "da_static_plan",
            "da_decode_attention", "da_combine", "da_read_status", "da_status_string", "da_dev_status_string",
            "da_last_cuda_error", "da_device_num_sms", "da_decode_step_noalloc", "da_append_kv",
-           "da_decode_attention_fp8")
+           "da_decode_attention_fp8", "da_merge_partials")
 
 NOALLOC_SCRATCH_BYTES = 16 << 20  # DA_NOALLOC_SCRATCH_BYTES
 
@@ -75,6 +75,7 @@ def lib():
             "da_device_num_sms": [ctypes.POINTER(ctypes.c_int32)],
             "da_decode_step_noalloc": [P, ctypes.c_int32, ctypes.c_int32, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp],
             "da_append_kv": [P, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp],
+            "da_merge_partials": [ctypes.c_int32, ctypes.c_int64, ctypes.c_int32, _vp, _vp, _vp, _vp, _vp],
             "da_decode_attention_fp8": [P, D, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp],
         }
         for name, args in sig.items():
@@ -187,6 +188,14 @@ def da_append_kv(prob, new_k, new_v, block_table, seq_lens, k_cache, v_cache, st
     _check("da_append_kv", lib().da_append_kv(ctypes.byref(prob), _ptr(new_k), _ptr(new_v), _ptr(block_table),
                                               _ptr(seq_lens), _ptr(k_cache), _ptr(v_cache), _ptr(status),
                                               _stream(stream)))
+
+
+def da_merge_partials(part_out, part_lse, out, lse, stream=None):
+    """part_out [n, ..., d] bf16 and part_lse [n, ...] fp32 -> out [..., d], lse [...]."""
+    n = part_out.shape[0]
+    rows = lse.numel()
+    _check("da_merge_partials", lib().da_merge_partials(int(n), int(rows), int(part_out.shape[-1]), _ptr(part_out),
+                                                        _ptr(part_lse), _ptr(out), _ptr(lse), _stream(stream)))
 
 
 def da_read_status(ws, stream=None) -> tuple[int, int]:
