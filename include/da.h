@@ -16,9 +16,12 @@
  *
  * One decode step is three asynchronous calls on one stream:
  *   da_plan              (or da_static_plan)  seq_lens -> work list in `ws`
- *   da_decode_attention  work list -> out/lse (single-segment requests) and
- *                        per-segment partials (split requests)
- *   da_combine           partials -> out/lse by log-sum-exp merge
+ *   da_decode_attention  work list -> out/lse; a request split over several
+ *                        CTAs leaves one partial per segment, and the CTA that
+ *                        finishes its last segment merges them by log-sum-exp
+ *   da_combine           the same merge as a separate kernel, used when the
+ *                        descriptor asks for it (merge_in_decode = 0); with
+ *                        the default descriptor it enqueues nothing
  * The host never reads seq_lens: every launch's grid is fixed by the problem
  * and the plan descriptor, so requests can join, grow, finish or be cancelled
  * between steps without a host round trip, and the three calls can be
@@ -124,12 +127,15 @@ typedef struct da_problem {
  * arguments only.  Pass the same descriptor to every call of a step.
  */
 typedef struct da_plan_desc {
-  int32_t kind;         /* DA_PLAN_DYNAMIC or DA_PLAN_STATIC */
-  int32_t batch;        /* B, copied from the problem */
-  int32_t tile_tokens;  /* T: tokens per tile (the planner's unit of work) */
-  int32_t num_ctas;     /* grid width per KV head: C (dynamic) or B*S (static) */
-  int32_t splits;       /* S for a static plan, 0 for a dynamic one */
-  int32_t max_segments; /* capacity of the segment list: C+B-1 (dynamic) or B*S (static) */
+  int32_t kind;            /* DA_PLAN_DYNAMIC or DA_PLAN_STATIC */
+  int32_t batch;           /* B, copied from the problem */
+  int32_t tile_tokens;     /* T: tokens per tile (the planner's unit of work) */
+  int32_t num_ctas;        /* grid width per KV head: C (dynamic) or B*S (static) */
+  int32_t splits;          /* S for a static plan, 0 for a dynamic one */
+  int32_t max_segments;    /* capacity of the segment list: C+B-1 (dynamic) or B*S (static) */
+  int32_t num_kv_heads;    /* Hkv, copied from the problem */
+  int32_t merge_in_decode; /* 1 (default): split requests are merged by the decode kernel's last
+                              CTA for them; 0: by da_combine's separate kernel */
 } da_plan_desc;
 
 /*
@@ -167,11 +173,12 @@ DA_API int da_workspace_size(const da_problem* prob, const da_plan_desc* desc, s
  *          static split)
  *   off[2] req_tile_prefix [B+1]   off[3] req_seg_begin [B+1]
  *   off[4] cta_seg_begin [num_ctas+1]
- *   off[5] total words
+ *   off[5] req_done [B][num_kv_heads]: segments finished this step (reset by the planner)
+ *   off[6] total words
  * Segments of request b are [req_seg_begin[b], req_seg_begin[b+1]); segments
  * of CTA c are [cta_seg_begin[c], cta_seg_begin[c+1]); both in tile order.
  */
-DA_API int da_workspace_offsets(const da_plan_desc* desc, int64_t off[6]);
+DA_API int da_workspace_offsets(const da_plan_desc* desc, int64_t off[7]);
 
 /*
  * da_plan -- dynamic (load-balanced) plan, one 1-CTA kernel.
@@ -201,8 +208,11 @@ DA_API int da_static_plan(const da_problem* prob, const da_plan_desc* desc, cons
  *   ws: dev, a plan made by da_plan / da_static_plan with the same descriptor
  *     and the same seq_lens contents.
  *   partial_o, partial_lse: dev scratch, sizes from da_workspace_size.
- *   out, lse: dev outputs.  Requests with exactly one segment are written
- *     here directly; the others are written by da_combine.
+ *   out, lse: dev outputs.  Requests with one segment are written directly;
+ *     with merge_in_decode (the default) so are split requests (by the last
+ *     CTA to finish one of their segments: counters in `ws`, release/acquire
+ *     fences, partials read back from L2) and requests with no segment;
+ *     otherwise da_combine writes those.
  * Each CTA streams its tiles' K and V rows (bf16, TMA, multi-stage shared
  * memory ring) and keeps, per query head of its KV group, the running max,
  * running sum and fp32 accumulator of the online softmax.
@@ -235,7 +245,9 @@ DA_API int da_decode_attention_fp8(const da_problem* prob, const da_plan_desc* d
                                    void* stream);
 
 /*
- * da_combine -- merge the partials of requests with two or more segments:
+ * da_combine -- when desc->merge_in_decode is 0, merge the partials of
+ * requests with two or more segments (with the default descriptor the decode
+ * kernel has done it and this call enqueues nothing):
  *   LSE = M + ln sum_i exp(lse_i - M),  M = max_i lse_i,
  *   out = sum_i exp(lse_i - LSE) o_i    (fp32 sums in a fixed order, then bf16),
  * and write out = 0, lse = -inf for requests with no segment.

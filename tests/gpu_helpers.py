@@ -14,11 +14,12 @@ from variable_length_paged_b200 import workloads as W
 OUT_ATOL, OUT_RTOL, LSE_ATOL = 1e-2, 1e-2, 1e-3
 
 
-def run_step(w: W.Workload | W.DeviceWorkload, kind=da.PLAN_DYNAMIC, tile=64, width=0, dw=None, bufs=None):
+def run_step(w: W.Workload | W.DeviceWorkload, kind=da.PLAN_DYNAMIC, tile=64, width=0, dw=None, bufs=None,
+             merge_in_decode=True):
     """Plan + decode + combine on cuda:0. Returns (out bf16 [B,Hq,d], lse [B,Hq], desc, bufs, dw)."""
     dw = dw if dw is not None else (w.to("cuda") if isinstance(w, W.Workload) else w)
     prob = da.problem_from(dw.problem)
-    desc = da.da_plan_desc_init(prob, kind, tile, width)
+    desc = da.da_plan_desc_init(prob, kind, tile, width, merge_in_decode=merge_in_decode)
     bufs = bufs if bufs is not None else da.Buffers(prob, desc, "cuda")
     # poison the partials and outputs so that an unwritten value cannot pass
     bufs.partial_o.fill_(float("nan"))

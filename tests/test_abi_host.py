@@ -43,11 +43,13 @@ def test_plan_descriptor_and_sizes(da_lib):
     p = prob(da)
     d = da.da_plan_desc_init(p, da.PLAN_DYNAMIC, 64, 37)
     assert (d.kind, d.batch, d.tile_tokens, d.num_ctas, d.splits, d.max_segments) == (0, 32, 64, 37, 0, 37 + 32 - 1)
+    assert (d.num_kv_heads, d.merge_in_decode) == (8, 1)
     ws, po, pl = da.da_workspace_size(p, d)
     off = da.da_workspace_offsets(d)
     assert off[0] == 0 and off[1] == 16 and off[2] == 16 + 4 * d.max_segments
-    assert off[3] == off[2] + 33 and off[4] == off[3] + 33 and off[5] >= off[4] + 38 and off[5] % 4 == 0
-    assert ws == off[5] * 4 and ws % 16 == 0
+    assert off[3] == off[2] + 33 and off[4] == off[3] + 33 and off[5] == off[4] + 38
+    assert off[6] >= off[5] + 32 * 8 and off[6] % 4 == 0
+    assert ws == off[6] * 4 and ws % 16 == 0
     assert po == d.max_segments * 64 * 128 * 4 and pl == d.max_segments * 64 * 4
     s = da.da_plan_desc_init(p, da.PLAN_STATIC, 32, 3)
     assert (s.kind, s.num_ctas, s.splits, s.max_segments, s.tile_tokens) == (1, 96, 3, 96, 32)
@@ -83,7 +85,7 @@ def test_descriptor_checks(da_lib):
     lib = da.lib()
     import ctypes
     d = da.da_plan_desc_init(p, da.PLAN_DYNAMIC, 64, 37)
-    bad = da.DaPlanDesc(d.kind, d.batch, d.tile_tokens, d.num_ctas, d.splits, d.max_segments - 1)
+    bad = da.DaPlanDesc(d.kind, d.batch, d.tile_tokens, d.num_ctas, d.splits, d.max_segments - 1, 8, 1)
     assert lib.da_workspace_size(ctypes.byref(p), ctypes.byref(bad), None, None, None) == -1
     # a dynamic call given a static descriptor, and a workspace that is too small
     s = da.da_plan_desc_init(p, da.PLAN_STATIC, 64, 2)

@@ -42,6 +42,25 @@ def test_tile_and_cta_count_do_not_change_the_result(da_lib, oracle_lib, T, C):
     check_against_oracle(w, out, lse)
 
 
+@pytest.mark.parametrize("kind,width", [(da.PLAN_DYNAMIC, 1), (da.PLAN_DYNAMIC, 37), (da.PLAN_DYNAMIC, 1000),
+                                        (da.PLAN_STATIC, 1), (da.PLAN_STATIC, 7)])
+def test_standalone_combine_kernel(da_lib, oracle_lib, kind, width):
+    """merge_in_decode = 0: split requests and empty ones are finished by the separate combine kernel."""
+    w = small([3000, 70, 1, 512, 2049, 0, 33], Hq=16, Hkv=2, seed=13)
+    out, lse, desc, *_ = run_step(w, kind=kind, width=width, merge_in_decode=False)
+    assert desc.merge_in_decode == 0
+    check_against_oracle(w, out, lse)
+
+
+def test_merge_in_decode_counts_reset_every_step(da_lib, oracle_lib):
+    """The per-request segment counters live in the workspace and are reset by each plan."""
+    w = small([3000, 70, 1, 512, 2049, 0, 33], Hq=16, Hkv=2, seed=14)
+    out, lse, desc, bufs, dw = run_step(w, width=37)
+    for _ in range(3):
+        out, lse, *_ = run_step(None, dw=dw, bufs=bufs, width=37)
+        check_against_oracle(w, out, lse)
+
+
 @pytest.mark.parametrize("S", [1, 2, 4, 7, 16, 64])
 def test_static_split_k(da_lib, oracle_lib, S):
     w = small([3000, 70, 1, 512, 2049, 0, 33], Hq=16, Hkv=2, seed=3)

@@ -44,6 +44,8 @@ int check_desc(const da_problem* p, const da_plan_desc* d) {
   if (!d) return DA_ERR_INVALID_ARG;
   if (d->batch != p->batch || d->tile_tokens <= 0 || d->tile_tokens % 16 != 0 || d->num_ctas <= 0)
     return DA_ERR_INVALID_ARG;
+  if (d->num_kv_heads != p->num_kv_heads || (d->merge_in_decode != 0 && d->merge_in_decode != 1))
+    return DA_ERR_INVALID_ARG;
   if (d->kind == DA_PLAN_DYNAMIC) {
     if (d->splits != 0 || (int64_t)d->max_segments != (int64_t)d->num_ctas + (p->batch > 0 ? p->batch : 1) - 1)
       return DA_ERR_INVALID_ARG;
@@ -63,7 +65,7 @@ int check_desc(const da_problem* p, const da_plan_desc* d) {
 }
 
 size_t ws_words(const da_plan_desc* d) {
-  return (size_t)da::ws_layout(d->batch, d->num_ctas, d->max_segments).total;
+  return (size_t)da::ws_layout(d->batch, d->num_ctas, d->max_segments, d->num_kv_heads).total;
 }
 
 // cuTensorMapEncodeTiled, looked up once through the runtime (no link-time libcuda dependency).
@@ -145,6 +147,8 @@ DA_API int da_plan_desc_init(const da_problem* prob, int32_t kind, int32_t tile_
   d.kind = kind;
   d.batch = prob->batch;
   d.tile_tokens = T;
+  d.num_kv_heads = prob->num_kv_heads;
+  d.merge_in_decode = 1;
   if (kind == DA_PLAN_DYNAMIC) {
     d.num_ctas = w;
     d.splits = 0;
@@ -178,15 +182,17 @@ DA_API int da_workspace_size(const da_problem* prob, const da_plan_desc* desc, s
   return DA_OK;
 }
 
-DA_API int da_workspace_offsets(const da_plan_desc* desc, int64_t off[6]) {
-  if (!desc || !off || desc->batch < 0 || desc->num_ctas <= 0 || desc->max_segments <= 0) return DA_ERR_INVALID_ARG;
-  const da::WsLayout L = da::ws_layout(desc->batch, desc->num_ctas, desc->max_segments);
+DA_API int da_workspace_offsets(const da_plan_desc* desc, int64_t off[7]) {
+  if (!desc || !off || desc->batch < 0 || desc->num_ctas <= 0 || desc->max_segments <= 0 || desc->num_kv_heads <= 0)
+    return DA_ERR_INVALID_ARG;
+  const da::WsLayout L = da::ws_layout(desc->batch, desc->num_ctas, desc->max_segments, desc->num_kv_heads);
   off[0] = L.hdr;
   off[1] = L.segs;
   off[2] = L.req_tile_prefix;
   off[3] = L.req_seg_begin;
   off[4] = L.cta_seg_begin;
-  off[5] = L.total;
+  off[5] = L.req_done;
+  off[6] = L.total;
   return DA_OK;
 }
 
@@ -208,6 +214,7 @@ static int plan_common(const da_problem* prob, const da_plan_desc* desc, const i
   p.width = kind == DA_PLAN_DYNAMIC ? desc->num_ctas : desc->splits;
   p.max_segments = desc->max_segments;
   p.num_ctas = desc->num_ctas;
+  p.num_kv_heads = prob->num_kv_heads;
   p.capacity_tokens = (int64_t)prob->max_pages_per_req * prob->page_size;
   cudaError_t e = kind == DA_PLAN_DYNAMIC ? da::launch_plan_dynamic(p, static_cast<cudaStream_t>(stream))
                                           : da::launch_plan_static(p, static_cast<cudaStream_t>(stream));
@@ -274,6 +281,7 @@ static int decode_common(const da_problem* prob, const da_plan_desc* desc, const
   // several queries per request, or more than 8 heads per group, take the kernel that maps
   // (query, head) rows over all 16 MMA rows; plain decode with G <= 8 uses the upper 8
   p.full_rows = (p.q_len > 1 || p.group > 8) ? 1 : 0;
+  p.merge_in_decode = desc->merge_in_decode;
   cudaError_t e = fp8 ? da::launch_decode_fp8(p, prob->head_dim, maps, static_cast<cudaStream_t>(stream))
                       : da::launch_decode(p, prob->head_dim, maps, static_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? DA_OK : cuda_fail(e);
@@ -306,6 +314,7 @@ DA_API int da_combine(const da_problem* prob, const da_plan_desc* desc, const vo
   if (!ws || !partial_o || !partial_lse || !out || !lse) return DA_ERR_INVALID_ARG;
   if (reinterpret_cast<uintptr_t>(partial_o) % 16 != 0 || reinterpret_cast<uintptr_t>(out) % 8 != 0)
     return DA_ERR_INVALID_ARG;
+  if (desc->merge_in_decode) return DA_OK;  // the decode kernel has finished every request
   da::CombineParams p;
   p.ws = static_cast<const int32_t*>(ws);
   p.partial_o = partial_o;
@@ -316,6 +325,7 @@ DA_API int da_combine(const da_problem* prob, const da_plan_desc* desc, const vo
   p.num_q_heads = prob->num_q_heads * q_len_of(prob);  // every (query, head) row merges the same way
   p.num_ctas = desc->num_ctas;
   p.max_segments = desc->max_segments;
+  p.num_kv_heads = prob->num_kv_heads;
   cudaError_t e = da::launch_combine(p, prob->head_dim, static_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? DA_OK : cuda_fail(e);
 }

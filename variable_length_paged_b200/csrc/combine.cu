@@ -40,7 +40,7 @@ __global__ void __launch_bounds__(128) combine_kernel(const CombineParams p) {
   grid_dependency_wait();  // partials come from the decode kernel just before
   const int b = blockIdx.x, h = blockIdx.y;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const WsLayout WL = ws_layout(p.batch, p.num_ctas, p.max_segments);
+  const WsLayout WL = ws_layout(p.batch, p.num_ctas, p.max_segments, p.num_kv_heads);
   const int32_t* rsb = p.ws + WL.req_seg_begin;
   const int s0 = rsb[b], s1 = rsb[b + 1];
   const int n = s1 - s0;

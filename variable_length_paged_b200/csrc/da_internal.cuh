@@ -28,17 +28,19 @@ enum HeaderWord {
 };
 
 struct WsLayout {
-  int64_t hdr, segs, req_tile_prefix, req_seg_begin, cta_seg_begin, total;
+  int64_t hdr, segs, req_tile_prefix, req_seg_begin, cta_seg_begin, req_done, total;
 };
 
-__host__ __device__ inline WsLayout ws_layout(int64_t batch, int64_t num_ctas, int64_t max_segments) {
+__host__ __device__ inline WsLayout ws_layout(int64_t batch, int64_t num_ctas, int64_t max_segments,
+                                              int64_t num_kv_heads) {
   WsLayout L;
   L.hdr = 0;
   L.segs = kHdrWords;                       // int4 per segment, 64-byte aligned start
   L.req_tile_prefix = L.segs + 4 * max_segments;
   L.req_seg_begin = L.req_tile_prefix + batch + 1;
   L.cta_seg_begin = L.req_seg_begin + batch + 1;
-  L.total = (L.cta_seg_begin + num_ctas + 1 + 3) / 4 * 4;
+  L.req_done = L.cta_seg_begin + num_ctas + 1;  // [batch][num_kv_heads] finished segments
+  L.total = (L.req_done + batch * num_kv_heads + 3) / 4 * 4;
   return L;
 }
 
@@ -51,7 +53,7 @@ __device__ inline void record_status(int32_t* hdr, int32_t code, int32_t index) 
 struct PlanParams {
   const int32_t* seq_lens;
   int32_t* ws;
-  int32_t batch, tile_tokens, width, max_segments, num_ctas;
+  int32_t batch, tile_tokens, width, max_segments, num_ctas, num_kv_heads;
   int64_t capacity_tokens;
 };
 
@@ -72,6 +74,7 @@ struct DecodeParams {
   const float* v_scale;
   int32_t q_len;  // queries per request (1 = plain decode)
   int32_t full_rows;  // 1: q_len > 1 or G > 8: all 16 MMA rows carry (query, head) rows
+  int32_t merge_in_decode;  // 1: the last CTA to finish a request's segment merges its partials
 };
 
 struct CombineParams {
@@ -80,7 +83,7 @@ struct CombineParams {
   const float* partial_lse;
   __nv_bfloat16* out;
   float* lse;
-  int32_t batch, num_q_heads, num_ctas, max_segments;
+  int32_t batch, num_q_heads, num_ctas, max_segments, num_kv_heads;
 };
 
 struct AppendParams {

@@ -86,7 +86,7 @@ struct Cfg {
   static constexpr int kOffML = kOffSlots + 3 * kSlotFloats * 4;        // [3][m, l_r, l_e][8] floats
   static constexpr int kOffBars = kOffML + 3 * 3 * 8 * 4;                // full[kStages], empty[kStages]
   static constexpr int kOffMeta = kOffBars + 2 * kStages * 8;            // int per stage
-  static constexpr int kOffAbort = kOffMeta + kStages * 4;
+  static constexpr int kOffAbort = kOffMeta + kStages * 4;  // abort flag, then the "last segment" flag
   static constexpr int kBytes = kOffAbort + 16;
   static constexpr int kSmemRequest = kBytes + 1024;                     // slack for manual alignment
 };
@@ -116,6 +116,61 @@ __device__ __forceinline__ uint32_t pack_f16x2(float lo, float hi) {
   return r;
 }
 
+
+// Merge every segment partial of request b for the rows of KV head g (G heads x
+// q_len queries) into out/lse: LSE = M + ln sum_i exp(lse_i - M), out = sum_i
+// exp(lse_i - LSE) o_i, fp32 in a fixed order.  Run by the four consumer warps of
+// the CTA that finished the request's last segment; the partials of the other
+// CTAs are read from L2 (ld.global.cg) after the acquire fence.
+template <int D>
+__device__ void merge_request_rows(const DecodeParams& p, int b, int g, int s0, int n, int qlen, int hq_rows,
+                                   int warp, int lane) {
+  constexpr int kPer = D / 32;
+  const int rows = p.group * qlen;
+  for (int R = warp; R < rows; R += 4) {
+    const int qi = R / p.group, hj = R - qi * p.group;
+    const int hrow = qi * p.num_q_heads + g * p.group + hj;
+    const float* plse = p.partial_lse + (int64_t)s0 * hq_rows + hrow;
+    float M = -INFINITY;
+    for (int i = lane; i < n; i += 32) M = fmaxf(M, __ldcg(plse + (int64_t)i * hq_rows));
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
+    float total = -INFINITY;
+    float acc[kPer];
+#pragma unroll
+    for (int e = 0; e < kPer; ++e) acc[e] = 0.f;
+    if (M != -INFINITY) {
+      float sum = 0.f;
+      for (int i = lane; i < n; i += 32) sum += expf(__ldcg(plse + (int64_t)i * hq_rows) - M);
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
+      total = M + logf(sum);
+      const float* po = p.partial_o + ((int64_t)s0 * hq_rows + hrow) * D + lane * kPer;
+#pragma unroll 8
+      for (int i = 0; i < n; ++i) {
+        const float wgt = expf(__ldcg(plse + (int64_t)i * hq_rows) - total);
+        const float* src = po + (int64_t)i * hq_rows * D;
+        if constexpr (kPer == 4) {
+          const float4 v = __ldcg(reinterpret_cast<const float4*>(src));
+          acc[0] += wgt * v.x;
+          acc[1] += wgt * v.y;
+          acc[2] += wgt * v.z;
+          acc[3] += wgt * v.w;
+        } else {
+          const float2 v = __ldcg(reinterpret_cast<const float2*>(src));
+          acc[0] += wgt * v.x;
+          acc[1] += wgt * v.y;
+        }
+      }
+    }
+    __nv_bfloat16* dst = p.out + ((int64_t)b * hq_rows + hrow) * D + lane * kPer;
+    if constexpr (kPer == 4)
+      *reinterpret_cast<uint2*>(dst) = make_uint2(pack_bf16x2(acc[0], acc[1]), pack_bf16x2(acc[2], acc[3]));
+    else
+      *reinterpret_cast<uint32_t*>(dst) = pack_bf16x2(acc[0], acc[1]);
+    if (lane == 0) p.lse[(int64_t)b * hq_rows + hrow] = total;
+  }
+}
 
 struct SegmentInfo {
   int b, tok0, tok1, len;
@@ -175,7 +230,7 @@ __global__ void __launch_bounds__(kThreads, 2)
   grid_dependency_wait();    // the plan is written by the previous kernel in the stream
   grid_dependents_launch();  // the combine kernel may be scheduled; it waits for this grid to finish
 
-  const WsLayout WL = ws_layout(p.batch, p.num_ctas, p.max_segments);
+  const WsLayout WL = ws_layout(p.batch, p.num_ctas, p.max_segments, p.num_kv_heads);
   const int32_t* hdr = p.ws + WL.hdr;
   const int4* segs = reinterpret_cast<const int4*>(p.ws + WL.segs);
   const int32_t* rsb = p.ws + WL.req_seg_begin;
@@ -190,6 +245,20 @@ __global__ void __launch_bounds__(kThreads, 2)
     return;
   }
   const int seg_hi = min(seg_next, min(h_segs, p.max_segments));
+  if (p.merge_in_decode && cta == 0) {
+    // requests with no segment (length 0, or refused) get out = 0, lse = -inf here
+    const int qlen0 = p.q_len > 1 ? p.q_len : 1;
+    const int rows = p.group * qlen0, hq_rows0 = qlen0 * p.num_q_heads;
+    for (int b = 0; b < p.batch; ++b) {
+      if (rsb[b + 1] != rsb[b]) continue;
+      for (int i = threadIdx.x; i < rows * (D / 8); i += kThreads) {
+        const int R = i / (D / 8), c8 = i - R * (D / 8);
+        const int hrow = (R / p.group) * p.num_q_heads + g * p.group + R % p.group;
+        *reinterpret_cast<uint4*>(p.out + ((int64_t)b * hq_rows0 + hrow) * D + c8 * 8) = make_uint4(0, 0, 0, 0);
+        if (c8 == 0) p.lse[(int64_t)b * hq_rows0 + hrow] = -INFINITY;
+      }
+    }
+  }
   if (seg_lo < 0 || seg_lo >= seg_hi) return;  // nothing planned for this CTA (uniform over the block)
 
   if (warp == kConsumerWarps) {
@@ -695,6 +764,23 @@ __global__ void __launch_bounds__(kThreads, 2)
         }
       }
       named_barrier_sync(1, kConsumerWarps * 32);  // slots are free again
+    }
+    // ---- the CTA that finishes a split request's last segment merges its partials
+    if (!direct && p.merge_in_decode) {
+      volatile int* last_flag = abort_flag + 1;
+      if (w == 0) {
+        __threadfence();  // this segment's partials are visible before the count moves
+        __syncwarp();
+        if (lane == 0) {
+          const int prev = atomicAdd(const_cast<int32_t*>(p.ws) + WL.req_done + (int64_t)b * p.num_kv_heads + g, 1);
+          *last_flag = prev == nseg_b - 1;
+        }
+      }
+      named_barrier_sync(1, kConsumerWarps * 32);
+      if (*last_flag) {
+        __threadfence();  // acquire: the other CTAs' partials
+        merge_request_rows<D>(p, b, g, rsb[b], nseg_b, qlen, hq_rows, w, lane);
+      }
     }
   }
 }

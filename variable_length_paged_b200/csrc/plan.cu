@@ -17,7 +17,8 @@
 namespace da {
 namespace {
 
-constexpr int kPlanThreads = 1024;
+constexpr int kPlanThreads = 256;  // few warps: the plan is latency-bound, every barrier counts
+constexpr int kPlanWarps = kPlanThreads / 32;
 
 // Exclusive block-wide scan of one value per thread; also returns the total.
 __device__ int block_exclusive_scan(int v, int* total, int* warp_buf) {
@@ -30,18 +31,14 @@ __device__ int block_exclusive_scan(int v, int* total, int* warp_buf) {
   }
   if (lane == 31) warp_buf[warp] = x;
   __syncthreads();
-  if (warp == 0) {
-    int w = warp_buf[lane];
+  int before = 0, all = 0;
 #pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      const int y = __shfl_up_sync(0xffffffffu, w, o);
-      if (lane >= o) w += y;
-    }
-    warp_buf[lane] = w;  // inclusive warp totals
+  for (int i = 0; i < kPlanWarps; ++i) {
+    const int t = warp_buf[i];
+    before += i < warp ? t : 0;
+    all += t;
   }
-  __syncthreads();
-  const int before = warp == 0 ? 0 : warp_buf[warp - 1];
-  *total = warp_buf[31];
+  *total = all;
   __syncthreads();  // warp_buf may be reused by the next call
   return before + x - v;
 }
@@ -80,17 +77,15 @@ __device__ void tile_prefix(const PlanParams& p, int32_t* rtp, int32_t* s_rtp, i
     rtp[0] = 0;
     if (s_rtp) s_rtp[0] = 0;
   }
-  // block max of n
-  for (int o = 16; o > 0; o >>= 1) mx = max(mx, __shfl_xor_sync(0xffffffffu, mx, o));
-  if ((threadIdx.x & 31) == 0) warp_buf[threadIdx.x >> 5] = mx;
-  __syncthreads();
-  if (threadIdx.x < 32) {
-    int w = warp_buf[threadIdx.x];
-    for (int o = 16; o > 0; o >>= 1) w = max(w, __shfl_xor_sync(0xffffffffu, w, o));
-    if (threadIdx.x == 0) warp_buf[0] = w;
+  if (max_tiles) {  // block max of n (static plan only)
+    for (int o = 16; o > 0; o >>= 1) mx = max(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+    if ((threadIdx.x & 31) == 0) warp_buf[threadIdx.x >> 5] = mx;
+    __syncthreads();
+    int all = 0;
+#pragma unroll
+    for (int i = 0; i < kPlanWarps; ++i) all = max(all, warp_buf[i]);
+    *max_tiles = all;
   }
-  __syncthreads();
-  *max_tiles = warp_buf[0];
   *U = carry;
   __syncthreads();
 }
@@ -109,9 +104,22 @@ __device__ void write_header(const PlanParams& p, int32_t* hdr, int U, int S, in
   for (int i = kHdrSplits + 1; i < kHdrWords; ++i) hdr[i] = 0;
 }
 
-// CTA that owns global tile u: the unique c with floor(c*U/C) <= u < floor((c+1)*U/C).
-__device__ __forceinline__ int owner_cta(int64_t u, int64_t U, int64_t C) { return (int)(((u + 1) * C - 1) / U); }
-__device__ __forceinline__ int64_t cta_first_unit(int64_t c, int64_t U, int64_t C) { return c * U / C; }
+// CTA that owns global tile u: the unique c with floor(c*U/C) <= u < floor((c+1)*U/C),
+// and the first tile of CTA c.  Every product is below C*(U+1); when that fits in 32
+// bits (the common case) the divisions are done in 32-bit integers.
+struct Split {
+  int64_t U, C;
+  bool narrow;
+  __device__ Split(int64_t u, int64_t c) : U(u), C(c), narrow(c * (u + 1) < (int64_t(1) << 31)) {}
+  __device__ __forceinline__ int owner(int64_t u) const {
+    if (narrow) return (int)(((uint32_t)(u + 1) * (uint32_t)C - 1u) / (uint32_t)U);
+    return (int)(((u + 1) * C - 1) / U);
+  }
+  __device__ __forceinline__ int64_t first(int64_t c) const {
+    if (narrow) return (int64_t)(((uint32_t)c * (uint32_t)U) / (uint32_t)C);
+    return c * U / C;
+  }
+};
 
 // Largest i in [0, n] with a[i] <= x, for a non-decreasing a[0..n] with a[0] <= x.
 __device__ __forceinline__ int last_not_above(const int32_t* a, int n, int64_t x) {
@@ -132,7 +140,9 @@ __global__ void __launch_bounds__(kPlanThreads) plan_dynamic_kernel(const PlanPa
   if (threadIdx.x == 0) s_bad = INT_MAX;
   __syncthreads();
 
-  const WsLayout L = ws_layout(p.batch, p.num_ctas, p.max_segments);
+  const WsLayout L = ws_layout(p.batch, p.num_ctas, p.max_segments, p.num_kv_heads);
+  int32_t* done = p.ws + L.req_done;
+  for (int64_t i = threadIdx.x; i < (int64_t)p.batch * p.num_kv_heads; i += kPlanThreads) done[i] = 0;
   int32_t* hdr = p.ws + L.hdr;
   int4* segs = reinterpret_cast<int4*>(p.ws + L.segs);
   int32_t* rtp = p.ws + L.req_tile_prefix;
@@ -143,8 +153,9 @@ __global__ void __launch_bounds__(kPlanThreads) plan_dynamic_kernel(const PlanPa
   const int32_t* rsb_r = small ? s_rsb : rsb;
   const int64_t C = p.num_ctas;
 
-  int U, max_tiles;
-  tile_prefix(p, rtp, small ? s_rtp : nullptr, warp_buf, &s_bad, &U, &max_tiles);
+  int U;
+  tile_prefix(p, rtp, small ? s_rtp : nullptr, warp_buf, &s_bad, &U, nullptr);
+  const Split sp(U, C);
 
   // Segments per request.  With U >= C every CTA owns at least one tile, so a
   // request spanning CTAs [cf, cl] has cl - cf + 1 segments.  With U < C each
@@ -156,7 +167,7 @@ __global__ void __launch_bounds__(kPlanThreads) plan_dynamic_kernel(const PlanPa
     int ns = 0;
     if (b < p.batch) {
       const int p0 = rtp_r[b], n = rtp_r[b + 1] - p0;
-      if (n > 0) ns = sparse ? n : owner_cta(p0 + n - 1, U, C) - owner_cta(p0, U, C) + 1;
+      if (n > 0) ns = sparse ? n : sp.owner(p0 + n - 1) - sp.owner(p0) + 1;
     }
     int total;
     const int excl = block_exclusive_scan(ns, &total, warp_buf);
@@ -179,11 +190,11 @@ __global__ void __launch_bounds__(kPlanThreads) plan_dynamic_kernel(const PlanPa
     const int j = s - rsb_r[b];
     const int p0 = rtp_r[b], n = rtp_r[b + 1] - p0;
     if (sparse) {
-      segs[s] = make_int4(b, owner_cta((int64_t)p0 + j, U, C), j, j + 1);
+      segs[s] = make_int4(b, sp.owner((int64_t)p0 + j), j, j + 1);
     } else {
-      const int c = owner_cta(p0, U, C) + j;
-      const int64_t lo = max((int64_t)p0, cta_first_unit(c, U, C));
-      const int64_t hi = min((int64_t)p0 + n, cta_first_unit(c + 1, U, C));
+      const int c = sp.owner(p0) + j;
+      const int64_t lo = max((int64_t)p0, sp.first(c));
+      const int64_t hi = min((int64_t)p0 + n, sp.first(c + 1));
       segs[s] = make_int4(b, c, (int)(lo - p0), (int)(hi - p0));
     }
   }
@@ -191,14 +202,14 @@ __global__ void __launch_bounds__(kPlanThreads) plan_dynamic_kernel(const PlanPa
   for (int c = threadIdx.x; c <= p.num_ctas; c += kPlanThreads) {
     int first;
     if (sparse) {
-      first = (int)cta_first_unit(c, U, C);  // every tile is a segment
+      first = (int)sp.first(c);  // every tile is a segment
     } else if (c == p.num_ctas) {
       first = S;
     } else {
       // the request holding CTA c's first tile opens CTA c
-      const int64_t u0 = cta_first_unit(c, U, C);
+      const int64_t u0 = sp.first(c);
       const int r = last_not_above(rtp_r, p.batch, u0);
-      first = rsb_r[r] + (c - owner_cta(rtp_r[r], U, C));
+      first = rsb_r[r] + (c - sp.owner(rtp_r[r]));
     }
     csb[c] = first;
   }
@@ -214,7 +225,9 @@ __global__ void __launch_bounds__(kPlanThreads) plan_static_kernel(const PlanPar
   if (threadIdx.x == 0) s_bad = INT_MAX;
   __syncthreads();
 
-  const WsLayout L = ws_layout(p.batch, p.num_ctas, p.max_segments);
+  const WsLayout L = ws_layout(p.batch, p.num_ctas, p.max_segments, p.num_kv_heads);
+  int32_t* done = p.ws + L.req_done;
+  for (int64_t i = threadIdx.x; i < (int64_t)p.batch * p.num_kv_heads; i += kPlanThreads) done[i] = 0;
   int32_t* hdr = p.ws + L.hdr;
   int4* segs = reinterpret_cast<int4*>(p.ws + L.segs);
   int32_t* rtp = p.ws + L.req_tile_prefix;

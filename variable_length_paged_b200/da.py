@@ -35,7 +35,8 @@ class DaProblem(ctypes.Structure):
 
 class DaPlanDesc(ctypes.Structure):
     _fields_ = [("kind", ctypes.c_int32), ("batch", ctypes.c_int32), ("tile_tokens", ctypes.c_int32),
-                ("num_ctas", ctypes.c_int32), ("splits", ctypes.c_int32), ("max_segments", ctypes.c_int32)]
+                ("num_ctas", ctypes.c_int32), ("splits", ctypes.c_int32), ("max_segments", ctypes.c_int32),
+                ("num_kv_heads", ctypes.c_int32), ("merge_in_decode", ctypes.c_int32)]
 
 
 class DaError(RuntimeError):
@@ -132,10 +133,12 @@ def _stream(stream) -> int | None:
 
 # ---- the C calls -------------------------------------------------------------------------------
 
-def da_plan_desc_init(prob: DaProblem, kind: int, tile_tokens: int = 0, width: int = 0) -> DaPlanDesc:
+def da_plan_desc_init(prob: DaProblem, kind: int, tile_tokens: int = 0, width: int = 0,
+                      merge_in_decode: bool = True) -> DaPlanDesc:
     d = DaPlanDesc()
     _check("da_plan_desc_init", lib().da_plan_desc_init(ctypes.byref(prob), int(kind), int(tile_tokens), int(width),
                                                          ctypes.byref(d)))
+    d.merge_in_decode = 1 if merge_in_decode else 0
     return d
 
 
@@ -147,7 +150,7 @@ def da_workspace_size(prob: DaProblem, desc: DaPlanDesc) -> tuple[int, int, int]
 
 
 def da_workspace_offsets(desc: DaPlanDesc) -> list[int]:
-    off = (ctypes.c_int64 * 6)()
+    off = (ctypes.c_int64 * 7)()
     _check("da_workspace_offsets", lib().da_workspace_offsets(ctypes.byref(desc), off))
     return list(off)
 
