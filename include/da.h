@@ -16,12 +16,11 @@
  *
  * One decode step is three asynchronous calls on one stream:
  *   da_plan              (or da_static_plan)  seq_lens -> work list in `ws`
- *   da_decode_attention  work list -> out/lse; a request split over several
- *                        CTAs leaves one partial per segment, and the CTA that
- *                        finishes its last segment merges them by log-sum-exp
- *   da_combine           the same merge as a separate kernel, used when the
- *                        descriptor asks for it (merge_in_decode = 0); with
- *                        the default descriptor it enqueues nothing
+ *   da_decode_attention  work list -> out/lse (single-segment requests) and
+ *                        per-segment partials (requests split over CTAs)
+ *   da_combine           partials -> out/lse by log-sum-exp merge
+ * (With merge_in_decode = 1 in the descriptor the decode kernel merges split
+ * requests itself and da_combine enqueues nothing.)
  * The host never reads seq_lens: every launch's grid is fixed by the problem
  * and the plan descriptor, so requests can join, grow, finish or be cancelled
  * between steps without a host round trip, and the three calls can be
@@ -134,8 +133,10 @@ typedef struct da_plan_desc {
   int32_t splits;          /* S for a static plan, 0 for a dynamic one */
   int32_t max_segments;    /* capacity of the segment list: C+B-1 (dynamic) or B*S (static) */
   int32_t num_kv_heads;    /* Hkv, copied from the problem */
-  int32_t merge_in_decode; /* 1 (default): split requests are merged by the decode kernel's last
-                              CTA for them; 0: by da_combine's separate kernel */
+  int32_t merge_in_decode; /* 0 (default): split requests are merged by da_combine's kernel;
+                              1: by the decode kernel's last CTA for each of them (no extra launch;
+                              faster for batches of many long requests, slower when one request
+                              is split over many CTAs) */
 } da_plan_desc;
 
 /*
@@ -209,10 +210,10 @@ DA_API int da_static_plan(const da_problem* prob, const da_plan_desc* desc, cons
  *     and the same seq_lens contents.
  *   partial_o, partial_lse: dev scratch, sizes from da_workspace_size.
  *   out, lse: dev outputs.  Requests with one segment are written directly;
- *     with merge_in_decode (the default) so are split requests (by the last
- *     CTA to finish one of their segments: counters in `ws`, release/acquire
- *     fences, partials read back from L2) and requests with no segment;
- *     otherwise da_combine writes those.
+ *     the others by da_combine, or, with merge_in_decode = 1, by the decode
+ *     kernel: the last CTA to finish a segment of a split request (counters in
+ *     `ws`, release/acquire fences, partials read back from L2) merges it, and
+ *     requests with no segment are written as 0 / -inf.
  * Each CTA streams its tiles' K and V rows (bf16, TMA, multi-stage shared
  * memory ring) and keeps, per query head of its KV group, the running max,
  * running sum and fp32 accumulator of the online softmax.
@@ -245,9 +246,9 @@ DA_API int da_decode_attention_fp8(const da_problem* prob, const da_plan_desc* d
                                    void* stream);
 
 /*
- * da_combine -- when desc->merge_in_decode is 0, merge the partials of
- * requests with two or more segments (with the default descriptor the decode
- * kernel has done it and this call enqueues nothing):
+ * da_combine -- merge the partials of requests with two or more segments
+ * (when desc->merge_in_decode is 1 the decode kernel has done it and this call
+ * enqueues nothing):
  *   LSE = M + ln sum_i exp(lse_i - M),  M = max_i lse_i,
  *   out = sum_i exp(lse_i - LSE) o_i    (fp32 sums in a fixed order, then bf16),
  * and write out = 0, lse = -inf for requests with no segment.

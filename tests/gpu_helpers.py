@@ -15,7 +15,7 @@ OUT_ATOL, OUT_RTOL, LSE_ATOL = 1e-2, 1e-2, 1e-3
 
 
 def run_step(w: W.Workload | W.DeviceWorkload, kind=da.PLAN_DYNAMIC, tile=64, width=0, dw=None, bufs=None,
-             merge_in_decode=True):
+             merge_in_decode=False):
     """Plan + decode + combine on cuda:0. Returns (out bf16 [B,Hq,d], lse [B,Hq], desc, bufs, dw)."""
     dw = dw if dw is not None else (w.to("cuda") if isinstance(w, W.Workload) else w)
     prob = da.problem_from(dw.problem)

@@ -43,7 +43,7 @@ def test_plan_descriptor_and_sizes(da_lib):
     p = prob(da)
     d = da.da_plan_desc_init(p, da.PLAN_DYNAMIC, 64, 37)
     assert (d.kind, d.batch, d.tile_tokens, d.num_ctas, d.splits, d.max_segments) == (0, 32, 64, 37, 0, 37 + 32 - 1)
-    assert (d.num_kv_heads, d.merge_in_decode) == (8, 1)
+    assert (d.num_kv_heads, d.merge_in_decode) == (8, 0)
     ws, po, pl = da.da_workspace_size(p, d)
     off = da.da_workspace_offsets(d)
     assert off[0] == 0 and off[1] == 16 and off[2] == 16 + 4 * d.max_segments

@@ -44,20 +44,28 @@ def test_tile_and_cta_count_do_not_change_the_result(da_lib, oracle_lib, T, C):
 
 @pytest.mark.parametrize("kind,width", [(da.PLAN_DYNAMIC, 1), (da.PLAN_DYNAMIC, 37), (da.PLAN_DYNAMIC, 1000),
                                         (da.PLAN_STATIC, 1), (da.PLAN_STATIC, 7)])
-def test_standalone_combine_kernel(da_lib, oracle_lib, kind, width):
-    """merge_in_decode = 0: split requests and empty ones are finished by the separate combine kernel."""
+def test_merge_in_decode(da_lib, oracle_lib, kind, width):
+    """merge_in_decode = 1: the decode kernel's last CTA per split request merges it, and
+    requests without segments are written by the decode kernel too (no combine launch)."""
     w = small([3000, 70, 1, 512, 2049, 0, 33], Hq=16, Hkv=2, seed=13)
-    out, lse, desc, *_ = run_step(w, kind=kind, width=width, merge_in_decode=False)
-    assert desc.merge_in_decode == 0
+    out, lse, desc, *_ = run_step(w, kind=kind, width=width, merge_in_decode=True)
+    assert desc.merge_in_decode == 1
+    check_against_oracle(w, out, lse)
+
+
+@pytest.mark.parametrize("name", ["mixed", "low_conc"])
+def test_merge_in_decode_full_size(da_lib, oracle_lib, name):
+    w = W.CONFIGS[name]()
+    out, lse, desc, *_ = run_step(w, merge_in_decode=True)
     check_against_oracle(w, out, lse)
 
 
 def test_merge_in_decode_counts_reset_every_step(da_lib, oracle_lib):
     """The per-request segment counters live in the workspace and are reset by each plan."""
     w = small([3000, 70, 1, 512, 2049, 0, 33], Hq=16, Hkv=2, seed=14)
-    out, lse, desc, bufs, dw = run_step(w, width=37)
+    out, lse, desc, bufs, dw = run_step(w, width=37, merge_in_decode=True)
     for _ in range(3):
-        out, lse, *_ = run_step(None, dw=dw, bufs=bufs, width=37)
+        out, lse, *_ = run_step(None, dw=dw, bufs=bufs, width=37, merge_in_decode=True)
         check_against_oracle(w, out, lse)
 
 

@@ -148,7 +148,7 @@ DA_API int da_plan_desc_init(const da_problem* prob, int32_t kind, int32_t tile_
   d.batch = prob->batch;
   d.tile_tokens = T;
   d.num_kv_heads = prob->num_kv_heads;
-  d.merge_in_decode = 1;
+  d.merge_in_decode = 0;
   if (kind == DA_PLAN_DYNAMIC) {
     d.num_ctas = w;
     d.splits = 0;

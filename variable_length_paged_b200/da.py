@@ -134,7 +134,7 @@ def _stream(stream) -> int | None:
 # ---- the C calls -------------------------------------------------------------------------------
 
 def da_plan_desc_init(prob: DaProblem, kind: int, tile_tokens: int = 0, width: int = 0,
-                      merge_in_decode: bool = True) -> DaPlanDesc:
+                      merge_in_decode: bool = False) -> DaPlanDesc:
     d = DaPlanDesc()
     _check("da_plan_desc_init", lib().da_plan_desc_init(ctypes.byref(prob), int(kind), int(tile_tokens), int(width),
                                                          ctypes.byref(d)))
