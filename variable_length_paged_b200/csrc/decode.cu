@@ -193,7 +193,7 @@ __device__ __forceinline__ SegmentInfo load_segment(const DecodeParams& p, const
   return r;
 }
 
-template <int D, bool FP8, bool MQ>
+template <int D, bool FP8, bool MQ, bool MERGE>
 __global__ void __launch_bounds__(kThreads, 2)
     decode_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap k64,
                   const __grid_constant__ CUtensorMap v64, const __grid_constant__ CUtensorMap k16,
@@ -245,7 +245,7 @@ __global__ void __launch_bounds__(kThreads, 2)
     return;
   }
   const int seg_hi = min(seg_next, min(h_segs, p.max_segments));
-  if (p.merge_in_decode && cta == 0) {
+  if (MERGE && cta == 0) {
     // requests with no segment (length 0, or refused) get out = 0, lse = -inf here
     const int qlen0 = p.q_len > 1 ? p.q_len : 1;
     const int rows = p.group * qlen0, hq_rows0 = qlen0 * p.num_q_heads;
@@ -766,7 +766,7 @@ __global__ void __launch_bounds__(kThreads, 2)
       named_barrier_sync(1, kConsumerWarps * 32);  // slots are free again
     }
     // ---- the CTA that finishes a split request's last segment merges its partials
-    if (!direct && p.merge_in_decode) {
+    if (MERGE && !direct) {
       volatile int* last_flag = abort_flag + 1;
       if (w == 0) {
         __threadfence();  // this segment's partials are visible before the count moves
@@ -785,7 +785,7 @@ __global__ void __launch_bounds__(kThreads, 2)
   }
 }
 
-template <int D, bool FP8, bool MQ>
+template <int D, bool FP8, bool MQ, bool MERGE>
 cudaError_t launch_decode_d(const DecodeParams& p, const CUtensorMap maps[4], cudaStream_t stream) {
   using C = Cfg<D, FP8, MQ>;
   static_assert(C::kSmemRequest * 2 <= 227 * 1024, "two CTAs per SM must fit");
@@ -795,7 +795,7 @@ cudaError_t launch_decode_d(const DecodeParams& p, const CUtensorMap maps[4], cu
   static bool configured[64] = {false};
   if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
   if (!configured[dev]) {
-    e = cudaFuncSetAttribute(decode_kernel<D, FP8, MQ>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    e = cudaFuncSetAttribute(decode_kernel<D, FP8, MQ, MERGE>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              C::kSmemRequest);
     if (e != cudaSuccess) return e;
     configured[dev] = true;
@@ -810,24 +810,28 @@ cudaError_t launch_decode_d(const DecodeParams& p, const CUtensorMap maps[4], cu
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, decode_kernel<D, FP8, MQ>, p, maps[0], maps[1], maps[2], maps[3]);
+  return cudaLaunchKernelEx(&cfg, decode_kernel<D, FP8, MQ, MERGE>, p, maps[0], maps[1], maps[2], maps[3]);
+}
+
+template <int D, bool FP8>
+cudaError_t launch_variant(const DecodeParams& p, const CUtensorMap maps[4], cudaStream_t stream) {
+  const bool mq = p.full_rows != 0, merge = p.merge_in_decode != 0;
+  if (mq) return merge ? launch_decode_d<D, FP8, true, true>(p, maps, stream)
+                       : launch_decode_d<D, FP8, true, false>(p, maps, stream);
+  return merge ? launch_decode_d<D, FP8, false, true>(p, maps, stream)
+               : launch_decode_d<D, FP8, false, false>(p, maps, stream);
 }
 
 }  // namespace
 
 cudaError_t launch_decode(const DecodeParams& p, int head_dim, const CUtensorMap maps[4], cudaStream_t stream) {
-  const bool mq = p.full_rows != 0;
-  if (head_dim == 128) return mq ? launch_decode_d<128, false, true>(p, maps, stream)
-                                 : launch_decode_d<128, false, false>(p, maps, stream);
-  if (head_dim == 64) return mq ? launch_decode_d<64, false, true>(p, maps, stream)
-                                : launch_decode_d<64, false, false>(p, maps, stream);
+  if (head_dim == 128) return launch_variant<128, false>(p, maps, stream);
+  if (head_dim == 64) return launch_variant<64, false>(p, maps, stream);
   return cudaErrorInvalidValue;
 }
 
 cudaError_t launch_decode_fp8(const DecodeParams& p, int head_dim, const CUtensorMap maps[4], cudaStream_t stream) {
-  const bool mq = p.full_rows != 0;
-  if (head_dim == 128) return mq ? launch_decode_d<128, true, true>(p, maps, stream)
-                                 : launch_decode_d<128, true, false>(p, maps, stream);
+  if (head_dim == 128) return launch_variant<128, true>(p, maps, stream);
   return cudaErrorInvalidValue;
 }
 
