@@ -10,7 +10,8 @@ the 126 MB L2, so consecutive steps cannot hit in L2.
 Printed (rank 0, one JSON line): KV-read GB/s of the whole step (value), the
 step time, the decode kernel's own achieved bandwidth against the measured HBM
 peak, the same step under the static split-k schedule (default and best split
-count), an end-to-end number with host<->device copies, the CPU oracle's rate
+count), an end-to-end number (one da_decode_step_host call per step: host
+inputs copied in, the step, outputs copied back to host), the CPU oracle's rate
 on this machine's cores, and the SM clocks seen during the measurement.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference] [--config mixed]
@@ -300,13 +301,10 @@ def run_ours(args, world, rank, local):
             out_h = torch.empty(bufs.out.shape, dtype=bufs.out.dtype).pin_memory()
             lse_h = torch.empty(bufs.lse.shape, dtype=bufs.lse.dtype).pin_memory()
 
-            def e2e_step():
-                dw.q.copy_(q_h, non_blocking=True)
-                dw.seq_lens.copy_(sl_h, non_blocking=True)
-                dw.block_table.copy_(bt_h, non_blocking=True)
-                step()
-                out_h.copy_(bufs.out, non_blocking=True)
-                lse_h.copy_(bufs.lse, non_blocking=True)
+            def e2e_step():  # one C call: copies in, plan, decode, combine, copies out
+                da.da_decode_step_host(prob, desc, q_h, bt_h, sl_h, dw.k_cache, dw.v_cache, dw.q, dw.block_table,
+                                       dw.seq_lens, bufs, out_h, lse_h, k_scale=dw.k_scale, v_scale=dw.v_scale,
+                                       stream=stream)
 
             for _ in range(warm):
                 e2e_step()

@@ -257,6 +257,43 @@ DA_API int da_combine(const da_problem* prob, const da_plan_desc* desc, const vo
                       const float* partial_lse, void* out, float* lse, void* stream);
 
 /*
+ * da_decode_step_host -- one whole decode step for a caller whose per-step
+ * inputs and outputs live in host memory, in one call, all enqueued on
+ * `stream` in this order:
+ *   copy seq_lens_host, block_table_host, q_host to their device copies;
+ *   plan (da_plan or da_static_plan, per desc->kind); decode (bf16 cache when
+ *   k_scale and v_scale are NULL, FP8 E4M3 cache with per-KV-head scales when
+ *   both are given); combine;
+ *   copy out_dev, lse_dev to out_host, lse_host.
+ * The step computed is the one the separate calls compute (same plan, kernels
+ * and results).
+ *   q_host, block_table_host, seq_lens_host  host, layouts as in da_problem;
+ *     read by the copies, so they must stay unchanged until the stream passes them.
+ *   k_cache, v_cache, k_scale, v_scale       dev, as for da_decode_attention(_fp8).
+ *   q_dev, block_table_dev, seq_lens_dev     dev, the caller's device copies of
+ *     the three inputs (same sizes and alignment rules as for da_decode_attention).
+ *   ws, ws_bytes, partial_o, partial_lse     dev, as for da_plan / da_decode_attention.
+ *   out_dev, lse_dev                         dev outputs, as for da_decode_attention.
+ *   out_host, lse_host                       host, bf16 / fp32, same layouts as out, lse.
+ * Host buffers should be page-locked (cudaHostAlloc / cudaHostRegister); with
+ * pageable memory the copies are correct but may block the calling thread.
+ * The host outputs are valid once the stream has passed the call (e.g. after
+ * cudaStreamSynchronize); the call itself does not synchronise.  Every argument
+ * check of the plan, decode and combine calls runs before anything is enqueued,
+ * so an error return means nothing was enqueued, except DA_ERR_CUDA from a copy
+ * or launch that the CUDA runtime refused.  Source: "Tencent HPC lands in SGLang,
+ * challenging default inference kernels", section "Why Tencent HPC matters for
+ * online model serving" (each decode step's schedule follows the current
+ * request lengths, which the serving engine owns on the host).
+ */
+DA_API int da_decode_step_host(const da_problem* prob, const da_plan_desc* desc, const void* q_host,
+                               const int32_t* block_table_host, const int32_t* seq_lens_host, const void* k_cache,
+                               const void* v_cache, const float* k_scale, const float* v_scale, void* q_dev,
+                               int32_t* block_table_dev, int32_t* seq_lens_dev, void* ws, size_t ws_bytes,
+                               float* partial_o, float* partial_lse, void* out_dev, float* lse_dev, void* out_host,
+                               float* lse_host, void* stream);
+
+/*
  * da_append_kv -- write each request's newest token into the paged cache
  * (the step before attention in every decode step: lengths grow by one).
  *   new_k, new_v  dev bf16 [batch][num_kv_heads][head_dim], 16-byte aligned.

@@ -99,6 +99,41 @@ def test_descriptor_checks(da_lib):
     assert lib.da_workspace_offsets(None, None) == -1
 
 
+def test_host_step_checks(da_lib):
+    """da_decode_step_host rejects bad arguments before it enqueues a copy (no pointer is dereferenced)."""
+    import ctypes
+    da = da_lib
+    lib = da.lib()
+    p = prob(da)
+    d = da.da_plan_desc_init(p, da.PLAN_DYNAMIC, 64, 37)
+    A = 1 << 12  # a 16-byte-aligned stand-in address, never touched: every case fails a check first
+
+    def call(prob_=p, desc=d, ws_bytes=1 << 24, **kw):
+        a = dict(q_host=A, bt_host=A, sl_host=A, k=A, v=A, ks=None, vs=None, q_dev=A, bt_dev=A, sl_dev=A, ws=A,
+                 po=A, pl=A, out_dev=A, lse_dev=A, out_host=A, lse_host=A)
+        a.update(kw)
+        return lib.da_decode_step_host(ctypes.byref(prob_), ctypes.byref(desc), a["q_host"], a["bt_host"],
+                                       a["sl_host"], a["k"], a["v"], a["ks"], a["vs"], a["q_dev"], a["bt_dev"],
+                                       a["sl_dev"], a["ws"], ws_bytes, a["po"], a["pl"], a["out_dev"], a["lse_dev"],
+                                       a["out_host"], a["lse_host"], None)
+
+    for name in ("q_host", "bt_host", "sl_host", "out_host", "lse_host", "sl_dev", "ws", "q_dev", "bt_dev", "k",
+                 "po", "pl", "out_dev", "lse_dev"):
+        assert call(**{name: None}) == da.ERR_INVALID_ARG, name
+    assert call(ks=A) == da.ERR_INVALID_ARG  # one scale without the other
+    assert call(ws_bytes=64) == da.ERR_WORKSPACE
+    assert call(ws=A + 8) == da.ERR_INVALID_ARG  # misaligned workspace
+    assert call(k=A + 4) == da.ERR_INVALID_ARG  # misaligned cache
+    p64 = prob(da, head_dim=64)
+    d64 = da.da_plan_desc_init(p64, da.PLAN_DYNAMIC, 64, 37)
+    assert call(prob_=p64, desc=d64, ks=A, vs=A) == da.ERR_UNSUPPORTED  # FP8 needs head_dim 128
+    s = da.da_plan_desc_init(p, da.PLAN_STATIC, 64, 2)
+    assert call(desc=s, ws_bytes=64) == da.ERR_WORKSPACE  # the static descriptor is checked the same way
+    p0 = prob(da, batch=0)
+    d0 = da.da_plan_desc_init(p0, da.PLAN_DYNAMIC, 64, 37)
+    assert call(prob_=p0, desc=d0, q_host=None) == da.OK  # an empty batch enqueues nothing
+
+
 def test_status_strings(da_lib):
     da = da_lib
     assert da.status_string(0) == "ok" and "workspace" in da.status_string(-4)

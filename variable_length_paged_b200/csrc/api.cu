@@ -196,8 +196,9 @@ DA_API int da_workspace_offsets(const da_plan_desc* desc, int64_t off[7]) {
   return DA_OK;
 }
 
-static int plan_common(const da_problem* prob, const da_plan_desc* desc, const int32_t* seq_lens, void* ws,
-                       size_t ws_bytes, void* stream, int kind) {
+// Checks a plan call and fills its kernel parameters; enqueues nothing.
+static int plan_prepare(const da_problem* prob, const da_plan_desc* desc, const int32_t* seq_lens, void* ws,
+                        size_t ws_bytes, int kind, da::PlanParams* p) {
   int rc = check_problem(prob);
   if (rc != DA_OK) return rc;
   rc = check_desc(prob, desc);
@@ -206,19 +207,29 @@ static int plan_common(const da_problem* prob, const da_plan_desc* desc, const i
   if (!ws || (prob->batch > 0 && !seq_lens)) return DA_ERR_INVALID_ARG;
   if (reinterpret_cast<uintptr_t>(ws) % 16 != 0) return DA_ERR_INVALID_ARG;
   if (ws_bytes < ws_words(desc) * 4) return DA_ERR_WORKSPACE;
-  da::PlanParams p;
-  p.seq_lens = seq_lens;
-  p.ws = static_cast<int32_t*>(ws);
-  p.batch = prob->batch;
-  p.tile_tokens = desc->tile_tokens;
-  p.width = kind == DA_PLAN_DYNAMIC ? desc->num_ctas : desc->splits;
-  p.max_segments = desc->max_segments;
-  p.num_ctas = desc->num_ctas;
-  p.num_kv_heads = prob->num_kv_heads;
-  p.capacity_tokens = (int64_t)prob->max_pages_per_req * prob->page_size;
+  p->seq_lens = seq_lens;
+  p->ws = static_cast<int32_t*>(ws);
+  p->batch = prob->batch;
+  p->tile_tokens = desc->tile_tokens;
+  p->width = kind == DA_PLAN_DYNAMIC ? desc->num_ctas : desc->splits;
+  p->max_segments = desc->max_segments;
+  p->num_ctas = desc->num_ctas;
+  p->num_kv_heads = prob->num_kv_heads;
+  p->capacity_tokens = (int64_t)prob->max_pages_per_req * prob->page_size;
+  return DA_OK;
+}
+
+static int plan_launch(const da::PlanParams& p, int kind, void* stream) {
   cudaError_t e = kind == DA_PLAN_DYNAMIC ? da::launch_plan_dynamic(p, static_cast<cudaStream_t>(stream))
                                           : da::launch_plan_static(p, static_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? DA_OK : cuda_fail(e);
+}
+
+static int plan_common(const da_problem* prob, const da_plan_desc* desc, const int32_t* seq_lens, void* ws,
+                       size_t ws_bytes, void* stream, int kind) {
+  da::PlanParams p;
+  const int rc = plan_prepare(prob, desc, seq_lens, ws, ws_bytes, kind, &p);
+  return rc != DA_OK ? rc : plan_launch(p, kind, stream);
 }
 
 DA_API int da_plan(const da_problem* prob, const da_plan_desc* desc, const int32_t* seq_lens, void* ws,
@@ -231,16 +242,13 @@ DA_API int da_static_plan(const da_problem* prob, const da_plan_desc* desc, cons
   return plan_common(prob, desc, seq_lens, ws, ws_bytes, stream, DA_PLAN_STATIC);
 }
 
-static int decode_common(const da_problem* prob, const da_plan_desc* desc, const void* q, const void* k_cache,
-                         const void* v_cache, const float* k_scale, const float* v_scale,
-                         const int32_t* block_table, const int32_t* seq_lens, const void* ws, float* partial_o,
-                         float* partial_lse, void* out, float* lse, void* stream, bool fp8) {
-  int rc = check_problem(prob);
-  if (rc != DA_OK) return rc;
-  rc = check_desc(prob, desc);
-  if (rc != DA_OK) return rc;
-  if (fp8 && prob->head_dim != 128) return DA_ERR_UNSUPPORTED;
-  if (prob->batch == 0) return DA_OK;
+// Checks a decode call and fills its kernel parameters and tensor maps; enqueues
+// nothing.  Call only with batch > 0.
+static int decode_prepare(const da_problem* prob, const da_plan_desc* desc, const void* q, const void* k_cache,
+                          const void* v_cache, const float* k_scale, const float* v_scale,
+                          const int32_t* block_table, const int32_t* seq_lens, const void* ws, float* partial_o,
+                          float* partial_lse, void* out, float* lse, bool fp8, da::DecodeParams* pp,
+                          CUtensorMap maps[4]) {
   if (!q || !k_cache || !v_cache || !block_table || !seq_lens || !ws || !partial_o || !partial_lse || !out || !lse)
     return DA_ERR_INVALID_ARG;
   if (fp8 && (!k_scale || !v_scale)) return DA_ERR_INVALID_ARG;
@@ -249,11 +257,10 @@ static int decode_common(const da_problem* prob, const da_plan_desc* desc, const
       reinterpret_cast<uintptr_t>(partial_o) % 16 != 0 || reinterpret_cast<uintptr_t>(ws) % 16 != 0)
     return DA_ERR_INVALID_ARG;
   const int eb = fp8 ? 1 : 2;
-  CUtensorMap maps[4];
   if (!make_cache_map(&maps[0], k_cache, prob, 64, eb) || !make_cache_map(&maps[1], v_cache, prob, 64, eb) ||
       !make_cache_map(&maps[2], k_cache, prob, 16, eb) || !make_cache_map(&maps[3], v_cache, prob, 16, eb))
     return cuda_fail(cudaErrorInvalidValue);
-  da::DecodeParams p;
+  da::DecodeParams& p = *pp;
   p.k_scale = k_scale;
   p.v_scale = v_scale;
   p.q = static_cast<const __nv_bfloat16*>(q);
@@ -282,9 +289,31 @@ static int decode_common(const da_problem* prob, const da_plan_desc* desc, const
   // (query, head) rows over all 16 MMA rows; plain decode with G <= 8 uses the upper 8
   p.full_rows = (p.q_len > 1 || p.group > 8) ? 1 : 0;
   p.merge_in_decode = desc->merge_in_decode;
-  cudaError_t e = fp8 ? da::launch_decode_fp8(p, prob->head_dim, maps, static_cast<cudaStream_t>(stream))
-                      : da::launch_decode(p, prob->head_dim, maps, static_cast<cudaStream_t>(stream));
+  return DA_OK;
+}
+
+static int decode_launch(const da::DecodeParams& p, int head_dim, const CUtensorMap maps[4], bool fp8,
+                         void* stream) {
+  cudaError_t e = fp8 ? da::launch_decode_fp8(p, head_dim, maps, static_cast<cudaStream_t>(stream))
+                      : da::launch_decode(p, head_dim, maps, static_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? DA_OK : cuda_fail(e);
+}
+
+static int decode_common(const da_problem* prob, const da_plan_desc* desc, const void* q, const void* k_cache,
+                         const void* v_cache, const float* k_scale, const float* v_scale,
+                         const int32_t* block_table, const int32_t* seq_lens, const void* ws, float* partial_o,
+                         float* partial_lse, void* out, float* lse, void* stream, bool fp8) {
+  int rc = check_problem(prob);
+  if (rc != DA_OK) return rc;
+  rc = check_desc(prob, desc);
+  if (rc != DA_OK) return rc;
+  if (fp8 && prob->head_dim != 128) return DA_ERR_UNSUPPORTED;
+  if (prob->batch == 0) return DA_OK;
+  da::DecodeParams p;
+  CUtensorMap maps[4];
+  rc = decode_prepare(prob, desc, q, k_cache, v_cache, k_scale, v_scale, block_table, seq_lens, ws, partial_o,
+                      partial_lse, out, lse, fp8, &p, maps);
+  return rc != DA_OK ? rc : decode_launch(p, prob->head_dim, maps, fp8, stream);
 }
 
 DA_API int da_decode_attention(const da_problem* prob, const da_plan_desc* desc, const void* q,
@@ -304,6 +333,33 @@ DA_API int da_decode_attention_fp8(const da_problem* prob, const da_plan_desc* d
                        partial_lse, out, lse, stream, true);
 }
 
+// Checks a combine call and fills its kernel parameters; enqueues nothing.
+// Call only with batch > 0.
+static int combine_prepare(const da_problem* prob, const da_plan_desc* desc, const void* ws,
+                           const float* partial_o, const float* partial_lse, void* out, float* lse,
+                           da::CombineParams* p) {
+  if (!ws || !partial_o || !partial_lse || !out || !lse) return DA_ERR_INVALID_ARG;
+  if (reinterpret_cast<uintptr_t>(partial_o) % 16 != 0 || reinterpret_cast<uintptr_t>(out) % 8 != 0)
+    return DA_ERR_INVALID_ARG;
+  p->ws = static_cast<const int32_t*>(ws);
+  p->partial_o = partial_o;
+  p->partial_lse = partial_lse;
+  p->out = static_cast<__nv_bfloat16*>(out);
+  p->lse = lse;
+  p->batch = prob->batch;
+  p->num_q_heads = prob->num_q_heads * q_len_of(prob);  // every (query, head) row merges the same way
+  p->num_ctas = desc->num_ctas;
+  p->max_segments = desc->max_segments;
+  p->num_kv_heads = prob->num_kv_heads;
+  return DA_OK;
+}
+
+static int combine_launch(const da::CombineParams& p, const da_plan_desc* desc, int head_dim, void* stream) {
+  if (desc->merge_in_decode) return DA_OK;  // the decode kernel has finished every request
+  cudaError_t e = da::launch_combine(p, head_dim, static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? DA_OK : cuda_fail(e);
+}
+
 DA_API int da_combine(const da_problem* prob, const da_plan_desc* desc, const void* ws, const float* partial_o,
                       const float* partial_lse, void* out, float* lse, void* stream) {
   int rc = check_problem(prob);
@@ -311,22 +367,56 @@ DA_API int da_combine(const da_problem* prob, const da_plan_desc* desc, const vo
   rc = check_desc(prob, desc);
   if (rc != DA_OK) return rc;
   if (prob->batch == 0) return DA_OK;
-  if (!ws || !partial_o || !partial_lse || !out || !lse) return DA_ERR_INVALID_ARG;
-  if (reinterpret_cast<uintptr_t>(partial_o) % 16 != 0 || reinterpret_cast<uintptr_t>(out) % 8 != 0)
-    return DA_ERR_INVALID_ARG;
-  if (desc->merge_in_decode) return DA_OK;  // the decode kernel has finished every request
   da::CombineParams p;
-  p.ws = static_cast<const int32_t*>(ws);
-  p.partial_o = partial_o;
-  p.partial_lse = partial_lse;
-  p.out = static_cast<__nv_bfloat16*>(out);
-  p.lse = lse;
-  p.batch = prob->batch;
-  p.num_q_heads = prob->num_q_heads * q_len_of(prob);  // every (query, head) row merges the same way
-  p.num_ctas = desc->num_ctas;
-  p.max_segments = desc->max_segments;
-  p.num_kv_heads = prob->num_kv_heads;
-  cudaError_t e = da::launch_combine(p, prob->head_dim, static_cast<cudaStream_t>(stream));
+  rc = combine_prepare(prob, desc, ws, partial_o, partial_lse, out, lse, &p);
+  return rc != DA_OK ? rc : combine_launch(p, desc, prob->head_dim, stream);
+}
+
+DA_API int da_decode_step_host(const da_problem* prob, const da_plan_desc* desc, const void* q_host,
+                               const int32_t* block_table_host, const int32_t* seq_lens_host, const void* k_cache,
+                               const void* v_cache, const float* k_scale, const float* v_scale, void* q_dev,
+                               int32_t* block_table_dev, int32_t* seq_lens_dev, void* ws, size_t ws_bytes,
+                               float* partial_o, float* partial_lse, void* out_dev, float* lse_dev, void* out_host,
+                               float* lse_host, void* stream) {
+  int rc = check_problem(prob);
+  if (rc != DA_OK) return rc;
+  rc = check_desc(prob, desc);
+  if (rc != DA_OK) return rc;
+  if ((k_scale == nullptr) != (v_scale == nullptr)) return DA_ERR_INVALID_ARG;
+  const bool fp8 = k_scale != nullptr;
+  if (fp8 && prob->head_dim != 128) return DA_ERR_UNSUPPORTED;
+  if (prob->batch == 0) return DA_OK;
+  if (!q_host || !block_table_host || !seq_lens_host || !out_host || !lse_host) return DA_ERR_INVALID_ARG;
+  // every check of the three device calls runs before the first copy is enqueued
+  da::PlanParams pp;
+  rc = plan_prepare(prob, desc, seq_lens_dev, ws, ws_bytes, desc->kind, &pp);
+  if (rc != DA_OK) return rc;
+  da::DecodeParams dp;
+  CUtensorMap maps[4];
+  rc = decode_prepare(prob, desc, q_dev, k_cache, v_cache, k_scale, v_scale, block_table_dev, seq_lens_dev, ws,
+                      partial_o, partial_lse, out_dev, lse_dev, fp8, &dp, maps);
+  if (rc != DA_OK) return rc;
+  da::CombineParams cp;
+  rc = combine_prepare(prob, desc, ws, partial_o, partial_lse, out_dev, lse_dev, &cp);
+  if (rc != DA_OK) return rc;
+
+  const cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const size_t B = (size_t)prob->batch;
+  const size_t rows = B * (size_t)q_len_of(prob) * (size_t)prob->num_q_heads;
+  const size_t q_bytes = rows * (size_t)prob->head_dim * 2;
+  const size_t bt_bytes = B * (size_t)prob->max_pages_per_req * 4;
+  cudaError_t e = cudaMemcpyAsync(seq_lens_dev, seq_lens_host, B * 4, cudaMemcpyHostToDevice, s);
+  if (e == cudaSuccess) e = cudaMemcpyAsync(block_table_dev, block_table_host, bt_bytes, cudaMemcpyHostToDevice, s);
+  if (e == cudaSuccess) e = cudaMemcpyAsync(q_dev, q_host, q_bytes, cudaMemcpyHostToDevice, s);
+  if (e != cudaSuccess) return cuda_fail(e);
+  rc = plan_launch(pp, desc->kind, stream);
+  if (rc != DA_OK) return rc;
+  rc = decode_launch(dp, prob->head_dim, maps, fp8, stream);
+  if (rc != DA_OK) return rc;
+  rc = combine_launch(cp, desc, prob->head_dim, stream);
+  if (rc != DA_OK) return rc;
+  e = cudaMemcpyAsync(out_host, out_dev, q_bytes, cudaMemcpyDeviceToHost, s);
+  if (e == cudaSuccess) e = cudaMemcpyAsync(lse_host, lse_dev, rows * 4, cudaMemcpyDeviceToHost, s);
   return e == cudaSuccess ? DA_OK : cuda_fail(e);
 }
 

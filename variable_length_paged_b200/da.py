@@ -22,7 +22,7 @@ PLAN_DYNAMIC, PLAN_STATIC = 0, 1
 EXPORTS = ("da_plan_desc_init", "da_workspace_size", "da_workspace_offsets", "da_plan", "da_static_plan",
            "da_decode_attention", "da_combine", "da_read_status", "da_status_string", "da_dev_status_string",
            "da_last_cuda_error", "da_device_num_sms", "da_decode_step_noalloc", "da_append_kv",
-           "da_decode_attention_fp8", "da_merge_partials")
+           "da_decode_attention_fp8", "da_merge_partials", "da_decode_step_host")
 
 NOALLOC_SCRATCH_BYTES = 16 << 20  # DA_NOALLOC_SCRATCH_BYTES
 
@@ -78,6 +78,8 @@ def lib():
             "da_append_kv": [P, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp],
             "da_merge_partials": [ctypes.c_int32, ctypes.c_int64, ctypes.c_int32, _vp, _vp, _vp, _vp, _vp],
             "da_decode_attention_fp8": [P, D, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp],
+            "da_decode_step_host": [P, D, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _sz, _vp, _vp, _vp,
+                                    _vp, _vp, _vp, _vp],
         }
         for name, args in sig.items():
             fn = getattr(L, name)
@@ -185,6 +187,19 @@ def da_decode_attention_fp8(prob, desc, q, k_cache, v_cache, k_scale, v_scale, b
 def da_combine(prob, desc, ws, partial_o, partial_lse, out, lse, stream=None):
     _check("da_combine", lib().da_combine(ctypes.byref(prob), ctypes.byref(desc), _ptr(ws), _ptr(partial_o),
                                           _ptr(partial_lse), _ptr(out), _ptr(lse), _stream(stream)))
+
+
+def da_decode_step_host(prob, desc, q_host, block_table_host, seq_lens_host, k_cache, v_cache, q_dev,
+                        block_table_dev, seq_lens_dev, bufs: "Buffers", out_host, lse_host, k_scale=None, v_scale=None,
+                        stream=None):
+    """Whole step from host inputs to host outputs in one C call (copies in, plan, decode, combine, copies out).
+
+    Asynchronous: `out_host` / `lse_host` are valid after the stream is synchronised."""
+    _check("da_decode_step_host", lib().da_decode_step_host(
+        ctypes.byref(prob), ctypes.byref(desc), _ptr(q_host), _ptr(block_table_host), _ptr(seq_lens_host),
+        _ptr(k_cache), _ptr(v_cache), _ptr(k_scale), _ptr(v_scale), _ptr(q_dev), _ptr(block_table_dev),
+        _ptr(seq_lens_dev), _ptr(bufs.ws), bufs.ws.numel() * bufs.ws.element_size(), _ptr(bufs.partial_o),
+        _ptr(bufs.partial_lse), _ptr(bufs.out), _ptr(bufs.lse), _ptr(out_host), _ptr(lse_host), _stream(stream)))
 
 
 def da_append_kv(prob, new_k, new_v, block_table, seq_lens, k_cache, v_cache, status=None, stream=None):
