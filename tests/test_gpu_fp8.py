@@ -6,6 +6,7 @@ path (|out - ref| <= 1e-2 + 1e-2*|ref|, |lse - ref| <= 1e-3).
 
 import numpy as np
 import pytest
+import torch
 
 from gpu_helpers import check_against_oracle_fp8, run_step_fp8
 from variable_length_paged_b200 import da
@@ -55,3 +56,55 @@ def test_fp8_full_size(da_lib, oracle_lib, name):
     out, lse, desc, bufs, _ = run_step_fp8(w8)
     assert da.da_read_status(bufs.ws) == (0, -1)
     check_against_oracle_fp8(w8, out, lse)
+
+
+def _set_key(w, b, t, g, row):
+    """Write K row `row` (float tensor [d]) for token t of request b, KV head g."""
+    P = w.problem.page_size
+    page = int(w.block_table[b, t // P])
+    w.k_cache[page, g, t % P] = row.to(torch.bfloat16)
+
+
+def test_fp8_query_magnitudes(da_lib, oracle_lib):
+    """Query rows from 1e-4 to 30 in size, and a row whose entries span three decades."""
+    w = W.make_workload("small", [700, 33, 2048, 1, 5000], num_q_heads=16, num_kv_heads=2, head_dim=128,
+                        page_size=64, seed=21)
+    f = torch.tensor([1e-4, 1e-2, 0.3, 1.0, 3.0, 10.0, 30.0, 0.05] * 2, dtype=torch.float32)
+    q = w.q.float() * f[None, :, None]
+    q[:, 3, :64] *= 1e-3
+    w.q = q.to(torch.bfloat16)
+    w8 = W.quantize_fp8(w)
+    out, lse, *_ = run_step_fp8(w8, width=7)
+    check_against_oracle_fp8(w8, out, lse)
+
+
+@pytest.mark.parametrize("spike", [12.0, 20.0])
+def test_fp8_spike_over_a_flat_tail(da_lib, oracle_lib, spike):
+    """One key far above thousands of equal ones: the tail's total weight (about 20000 e^-12
+    against 1 at spike 12) must survive the rounding of the small weights."""
+    L = [20000, 5000, 3000]
+    w = W.make_workload("small", L, num_q_heads=16, num_kv_heads=2, head_dim=128, page_size=64, seed=22)
+    d = w.problem.head_dim
+    w.k_cache.zero_()  # every key 0 (score 0), then one spike per (request, KV head)
+    e1 = torch.zeros(d)
+    e1[5] = 1.0
+    a = spike * float(np.sqrt(d))  # score of the spike for a query e1: a * 1/sqrt(d) = spike
+    for b, t0 in [(0, 7777), (1, 100), (2, 2999)]:
+        for g in range(2):
+            _set_key(w, b, t0, g, a * e1)
+    s = torch.tensor([1.0, 0.5, -1.0, 0.9, 1.0, 0.25, 0.75, 1.0] * 2)  # per-head spike strength
+    w.q = (s[None, :, None] * e1[None, None, :]).expand(3, 16, d).contiguous().to(torch.bfloat16)
+    w8 = W.quantize_fp8(w)
+    for T, C in [(64, 37), (64, 3), (128, 1)]:
+        out, lse, *_ = run_step_fp8(w8, tile=T, width=C)
+        check_against_oracle_fp8(w8, out, lse)
+
+
+def test_fp8_zero_query_long_request(da_lib, oracle_lib):
+    """q = 0: every weight equal over 30000 tokens; out is the mean of V, lse = ln L."""
+    w = W.make_workload("small", [30000, 17], num_q_heads=8, num_kv_heads=1, head_dim=128, page_size=64, seed=23)
+    w.q.zero_()
+    w8 = W.quantize_fp8(w)
+    out, lse, *_ = run_step_fp8(w8, width=5)
+    check_against_oracle_fp8(w8, out, lse)
+    assert np.allclose(lse.cpu().numpy(), np.log(np.array([30000, 17], np.float64))[:, None], atol=1e-4)
