@@ -88,3 +88,27 @@ def test_decode_trace_256_steps(da_lib, oracle_lib):
         d = dev_c.cpu().permute(0, 2, 1, 3)[m]
         h = host_c.permute(0, 2, 1, 3)[m]
         assert torch.equal(d.view(torch.int16), h.view(torch.int16))
+
+
+def test_recorded_trace_replays_the_live_trace(da_lib):
+    """record + apply (the bench's device-only replay) leaves the device in the same state, bit for
+    bit, as live advance steps, and the steps give the same outputs."""
+    kw = dict(seed=9, batch=48, steps=40, num_q_heads=16, num_kv_heads=2, median=900.0, max_len=4096,
+              p_finish=0.05)
+    live, rec = DeviceTrace(W.DecodeTrace(**kw)), DeviceTrace(W.DecodeTrace(**kw))
+    prob = live.prob
+    desc = da.da_plan_desc_init(prob, da.PLAN_DYNAMIC, 64, 0)
+    b1, b2 = da.Buffers(prob, desc, "cuda"), da.Buffers(prob, desc, "cuda")
+    ups = rec.record(39)
+    same = lambda a, b: torch.equal(a.view(torch.int16), b.view(torch.int16))
+    for t in range(40):
+        if t > 0:
+            live.advance()
+            rec.apply(ups[t - 1])
+        for dt, b in ((live, b1), (rec, b2)):
+            da.decode_step(prob, desc, dt.q, dt.k_cache, dt.v_cache, dt.block_table, dt.seq_lens, b)
+        torch.cuda.synchronize()
+        assert torch.equal(live.seq_lens, rec.seq_lens) and torch.equal(live.block_table, rec.block_table)
+        assert same(b1.out, b2.out) and torch.equal(b1.lse, b2.lse)
+    assert same(live.k_cache, rec.k_cache) and same(live.v_cache, rec.v_cache)
+    assert live.status.tolist() == rec.status.tolist() == [0, 0]
