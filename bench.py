@@ -121,8 +121,8 @@ def kernel_source_hash():
     return h.hexdigest()[:16]
 
 
-def recorded_traffic(workload_name):
-    """DRAM bytes per decode launch from the committed ncu summary, if it matches this kernel source."""
+def recorded_traffic(workload_name, kv="bf16", q_len=1):
+    """DRAM bytes per decode launch from the committed ncu record, if it matches this kernel source."""
     try:
         with open(TRAFFIC_FILE) as f:
             j = dict(ln.split(": ", 1) for ln in f.read().splitlines() if ln and not ln.startswith("#"))
@@ -130,9 +130,11 @@ def recorded_traffic(workload_name):
         return None, "no ncu capture recorded"
     if j.get("kernel_source_sha") != kernel_source_hash():
         return None, "kernel changed since the ncu capture"
-    if j.get("workload") != workload_name:
-        return None, f"ncu capture was on {j.get('workload')}"
-    return int(j["dram_bytes_read_per_launch"]) + int(j["dram_bytes_write_per_launch"]), j.get("command", "")
+    key = f"{workload_name}.{kv}"
+    if q_len > 1 or f"{key}.dram_bytes_read_per_launch" not in j:
+        return None, f"no ncu capture for {key}" + (f" with {q_len} queries" if q_len > 1 else "")
+    return (int(j[f"{key}.dram_bytes_read_per_launch"]) + int(j[f"{key}.dram_bytes_write_per_launch"]),
+            j.get(f"{key}.command", ""))
 
 
 class ClockSampler:
@@ -321,7 +323,7 @@ def run_ours(args, world, rank, local):
     value = total_bytes / step_s / 1e9
     peak, peak_src = measured_peak()
     dec_gbs = kv_bytes / (dec_avg_ms / 1e3) / 1e9
-    traffic, traffic_note = recorded_traffic(args.config) if args.kv == "bf16" else (None, "no ncu capture for fp8")
+    traffic, traffic_note = recorded_traffic(args.config, args.kv, args.q_len)
     result.update(
         metric=METRIC, value=round(value, 2), unit="GB/s", n_gpus=world, steps=steps, warmup=warm,
         ms_per_step=round(ms_graph / steps, 5), us_per_step=round(ms_graph / steps * 1e3, 2),

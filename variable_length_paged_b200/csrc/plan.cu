@@ -6,7 +6,7 @@
 // and the mapping is rebuilt as request lengths change; the comparator is a
 // static split-k schedule that idles units or launches empty chunks.
 //
-// Both planners run as one 1024-thread CTA and write the same work list:
+// Both planners run as one 256-thread CTA and write the same work list:
 // segments {request, cta, tile_begin, tile_end} in global tile order, the
 // per-request and per-CTA segment ranges, and a header.  Everything is integer
 // arithmetic, so the result is bit-exact and independent of thread timing.
