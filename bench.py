@@ -41,7 +41,8 @@ if ROOT not in sys.path:
 METRIC = "µs/decode step and KV-read HBM GB/s (% of B200 peak) vs static split-k"
 FALLBACK_HBM_GBS = 6650.0
 DATASHEET_HBM_GBS = 8000.0
-KERNEL_SOURCES = ["variable_length_paged_b200/csrc/decode.cu", "variable_length_paged_b200/csrc/da_internal.cuh"]
+KERNEL_SOURCES = ["variable_length_paged_b200/csrc/decode.cu", "variable_length_paged_b200/csrc/decode_tc.cu",
+                  "variable_length_paged_b200/csrc/da_internal.cuh"]
 TRAFFIC_FILE = os.path.join(ROOT, "profiles", "decode_kernel_traffic.txt")
 
 
@@ -119,6 +120,13 @@ def kernel_source_hash():
         with open(os.path.join(ROOT, rel), "rb") as f:
             h.update(f.read())
     return h.hexdigest()[:16]
+
+
+def decode_kernel_name(problem, fp8, q_len):
+    """The decode kernel the library launches for this shape (the one the roofline describes)."""
+    if fp8 and q_len <= 1 and problem.num_q_heads // problem.num_kv_heads <= 8:
+        return f"decode_tc_kernel<{problem.head_dim},fp8> (tcgen05)"
+    return f"decode_kernel<{problem.head_dim},{'fp8' if fp8 else 'bf16'}>"
 
 
 def recorded_traffic(workload_name, kv="bf16", q_len=1):
@@ -338,7 +346,7 @@ def run_ours(args, world, rank, local):
         eager_us_per_step=round(ms_eager / steps * 1e3, 2),
         roofline={"bound": "hbm", "achieved": round(dec_gbs, 2), "peak": peak, "unit": "GB/s",
                   "frac": round(dec_gbs / peak, 4), "traffic": traffic,
-                  "kernel": f"decode_kernel<{w.problem.head_dim},{'fp8' if w8 else 'bf16'}>",
+                  "kernel": decode_kernel_name(w.problem, bool(w8), args.q_len),
                   "algorithmic_bytes_per_launch": kv_bytes,
                   "launch_us": round(dec_avg_ms * 1e3, 2), "peak_source": peak_src, "traffic_source": traffic_note},
         e2e={"value": round(total_bytes / (ms_e2e / 1e3 / steps) / 1e9, 2), "unit": "GB/s",

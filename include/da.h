@@ -231,8 +231,12 @@ DA_API int da_decode_attention(const da_problem* prob, const da_plan_desc* desc,
  *                     k_scale[g] * e4m3(code) (and likewise for V).
  * Everything else, including the plan, workspace, partials, combine and the
  * bf16 q/out and fp32 lse, is as for da_decode_attention.  K/V bytes per token
- * are halved.  Codes are widened to f16 (exact), q is converted to f16 (exact
- * for normal-range values), and P is rounded to f16 for the P.V product.
+ * are halved.  Plain decode (q_len 1, at most 8 query heads per KV head,
+ * merge_in_decode 0) runs on the 5th-generation tensor cores (tcgen05, E4M3
+ * operands, accumulators in tensor memory): q and the softmax weights enter as
+ * two E4M3 terms each (hi + lo, 8 significant bits).  The other shapes widen
+ * the codes to f16 (exact), convert q to f16 and round P to f16 for a
+ * warp-level MMA.
  * Source: "Tencent HPC lands in SGLang, challenging default inference
  * kernels", sections "Why Tencent HPC matters for online model serving" (a
  * longer history means more cached data to read) and "What the 48.8% TPOT

@@ -292,10 +292,18 @@ static int decode_prepare(const da_problem* prob, const da_plan_desc* desc, cons
   return DA_OK;
 }
 
+// FP8 plain decode (one query, at most 8 heads per KV head, merge by da_combine) runs
+// on the tcgen05 kernel; multi-query and in-decode merge use the warp-MMA kernel.
 static int decode_launch(const da::DecodeParams& p, int head_dim, const CUtensorMap maps[4], bool fp8,
                          void* stream) {
-  cudaError_t e = fp8 ? da::launch_decode_fp8(p, head_dim, maps, static_cast<cudaStream_t>(stream))
-                      : da::launch_decode(p, head_dim, maps, static_cast<cudaStream_t>(stream));
+  const cudaStream_t s = static_cast<cudaStream_t>(stream);
+  cudaError_t e;
+  if (!fp8)
+    e = da::launch_decode(p, head_dim, maps, s);
+  else if (head_dim == 128 && p.full_rows == 0 && p.merge_in_decode == 0)
+    e = da::launch_decode_fp8_tc(p, maps, s);
+  else
+    e = da::launch_decode_fp8(p, head_dim, maps, s);
   return e == cudaSuccess ? DA_OK : cuda_fail(e);
 }
 

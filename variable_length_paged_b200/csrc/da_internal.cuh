@@ -107,11 +107,34 @@ struct MergeParams {
   int64_t rows;
 };
 
+// One planned segment as the decode kernels walk it: request, token range [tok0, tok1)
+// clipped to the request's length, and the length (bad lengths count as 0).  Every
+// role of a decode CTA decodes a segment the same way, so all walk the same chunks.
+struct SegmentInfo {
+  int b, tok0, tok1, len;
+  bool valid;
+};
+
+__device__ __forceinline__ SegmentInfo load_segment(const DecodeParams& p, const int4* segs, int s) {
+  const int4 sg = segs[s];
+  SegmentInfo r;
+  r.b = sg.x;
+  r.valid = sg.x >= 0 && sg.x < p.batch && sg.z >= 0 && sg.w >= sg.z;
+  int L = r.valid ? p.seq_lens[sg.x] : 0;
+  if (L < 0 || (int64_t)L > p.capacity_tokens) L = 0;
+  const int64_t t0 = (int64_t)sg.z * p.tile_tokens, t1 = min((int64_t)sg.w * p.tile_tokens, (int64_t)L);
+  r.tok0 = (int)min(t0, (int64_t)L);
+  r.tok1 = (int)t1;
+  r.len = L;
+  return r;
+}
+
 // Host launchers (defined next to their kernels).
 cudaError_t launch_plan_dynamic(const PlanParams& p, cudaStream_t stream);
 cudaError_t launch_plan_static(const PlanParams& p, cudaStream_t stream);
 cudaError_t launch_decode(const DecodeParams& p, int head_dim, const CUtensorMap maps[4], cudaStream_t stream);
 cudaError_t launch_decode_fp8(const DecodeParams& p, int head_dim, const CUtensorMap maps[4], cudaStream_t stream);
+cudaError_t launch_decode_fp8_tc(const DecodeParams& p, const CUtensorMap maps[4], cudaStream_t stream);
 cudaError_t launch_combine(const CombineParams& p, int head_dim, cudaStream_t stream);
 cudaError_t launch_append(const AppendParams& p, cudaStream_t stream);
 cudaError_t launch_merge(const MergeParams& p, int head_dim, cudaStream_t stream);

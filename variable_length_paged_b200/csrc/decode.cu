@@ -172,27 +172,6 @@ __device__ void merge_request_rows(const DecodeParams& p, int b, int g, int s0, 
   }
 }
 
-struct SegmentInfo {
-  int b, tok0, tok1, len;
-  bool valid;
-};
-
-// Same decoding of a segment on the producer and consumer side, so both walk
-// the same chunks.
-__device__ __forceinline__ SegmentInfo load_segment(const DecodeParams& p, const int4* segs, int s) {
-  const int4 sg = segs[s];
-  SegmentInfo r;
-  r.b = sg.x;
-  r.valid = sg.x >= 0 && sg.x < p.batch && sg.z >= 0 && sg.w >= sg.z;
-  int L = r.valid ? p.seq_lens[sg.x] : 0;
-  if (L < 0 || (int64_t)L > p.capacity_tokens) L = 0;
-  const int64_t t0 = (int64_t)sg.z * p.tile_tokens, t1 = min((int64_t)sg.w * p.tile_tokens, (int64_t)L);
-  r.tok0 = (int)min(t0, (int64_t)L);
-  r.tok1 = (int)t1;
-  r.len = L;
-  return r;
-}
-
 template <int D, bool FP8, bool MQ, bool MERGE>
 __global__ void __launch_bounds__(kThreads, 2)
     decode_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap k64,
