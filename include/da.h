@@ -349,6 +349,20 @@ DA_API const char* da_dev_status_string(int32_t code);
 /* cudaError_t of the last failing CUDA call made by this library on this thread (0 if none). */
 DA_API int32_t da_last_cuda_error(void);
 
+/*
+ * da_test_stall_next_decode -- a test of the failure path; the article has no
+ * counterpart.  The next decode launch made on this thread (da_decode_attention,
+ * da_decode_attention_fp8, or the decode inside da_decode_step_host or
+ * da_decode_step_noalloc) runs with its load stage idle: no K/V is requested,
+ * so every wait of the consumers runs out after wait_limit_us microseconds
+ * (1 .. 2,000,000) instead of the usual 2 s.  The kernel then records
+ * DA_DEV_TIMEOUT in the workspace status word, ends every role's loop and
+ * returns; nothing is trapped, the context stays usable, and the next step is
+ * unaffected.  The stalled launch's out/lse are invalid.  Returns
+ * DA_ERR_INVALID_ARG for a limit out of range.
+ */
+DA_API int da_test_stall_next_decode(uint32_t wait_limit_us);
+
 /* Number of SMs of the current device (host out). */
 DA_API int da_device_num_sms(int32_t* num_sms);
 

@@ -134,6 +134,15 @@ def test_host_step_checks(da_lib):
     assert call(prob_=p0, desc=d0, q_host=None) == da.OK  # an empty batch enqueues nothing
 
 
+def test_stall_switch_checks_its_limit(da_lib):
+    """Only the argument check is exercised here: a valid call would arm the next decode launch."""
+    da = da_lib
+    for bad in (0, 2000001):
+        with pytest.raises(da.DaError) as e:
+            da.da_test_stall_next_decode(bad)
+        assert e.value.code == da.ERR_INVALID_ARG
+
+
 def test_status_strings(da_lib):
     da = da_lib
     assert da.status_string(0) == "ok" and "workspace" in da.status_string(-4)

@@ -12,6 +12,9 @@
 namespace {
 
 thread_local int32_t g_last_cuda_error = 0;
+// failure-path test: limit (ns) for the next decode launch on this thread, which then stalls
+thread_local uint64_t g_stall_next_ns = 0;
+constexpr uint64_t kWaitLimitNs = 2000000000ull;  // 2 s: far beyond any legitimate pipeline wait
 
 constexpr int kDefaultTile = 64;
 constexpr int kCtasPerSm = 2;  // decode kernel residency (shared memory sized for two)
@@ -108,6 +111,12 @@ void set_last_cuda_error(cudaError_t e) { g_last_cuda_error = (int32_t)e; }
 extern "C" {
 
 DA_API int32_t da_last_cuda_error(void) { return g_last_cuda_error; }
+
+DA_API int da_test_stall_next_decode(uint32_t wait_limit_us) {
+  if (wait_limit_us == 0 || wait_limit_us > 2000000u) return DA_ERR_INVALID_ARG;
+  g_stall_next_ns = (uint64_t)wait_limit_us * 1000u;
+  return DA_OK;
+}
 
 DA_API int da_device_num_sms(int32_t* num_sms) {
   if (!num_sms) return DA_ERR_INVALID_ARG;
@@ -289,6 +298,9 @@ static int decode_prepare(const da_problem* prob, const da_plan_desc* desc, cons
   // (query, head) rows over all 16 MMA rows; plain decode with G <= 8 uses the upper 8
   p.full_rows = (p.q_len > 1 || p.group > 8) ? 1 : 0;
   p.merge_in_decode = desc->merge_in_decode;
+  p.stall_producer = g_stall_next_ns != 0 ? 1 : 0;
+  p.wait_limit_ns = g_stall_next_ns != 0 ? g_stall_next_ns : kWaitLimitNs;
+  g_stall_next_ns = 0;  // one launch only
   return DA_OK;
 }
 

@@ -75,6 +75,8 @@ struct DecodeParams {
   int32_t q_len;  // queries per request (1 = plain decode)
   int32_t full_rows;  // 1: q_len > 1 or G > 8: all 16 MMA rows carry (query, head) rows
   int32_t merge_in_decode;  // 1: the last CTA to finish a request's segment merges its partials
+  int32_t stall_producer;   // failure-path test: the producer sends nothing, so every wait runs out
+  uint64_t wait_limit_ns;   // limit of every pipeline wait
 };
 
 struct CombineParams {
@@ -188,6 +190,7 @@ __device__ __forceinline__ uint64_t global_timer_ns() {
 __device__ __forceinline__ bool mbar_wait_bounded(uint32_t bar, uint32_t parity, volatile int* abort,
                                                   uint64_t limit_ns) {
   if (mbar_try_wait(bar, parity)) return true;
+  if (*abort) return false;
   const uint64_t t0 = global_timer_ns();
   for (uint32_t it = 1;; ++it) {
     if (mbar_try_wait(bar, parity)) return true;

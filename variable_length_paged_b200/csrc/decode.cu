@@ -58,7 +58,6 @@ namespace {
 
 constexpr int kConsumerWarps = 4;
 constexpr int kThreads = (kConsumerWarps + 1) * 32;
-constexpr uint64_t kWaitLimitNs = 2000000000ull;  // 2 s: far beyond any legitimate wait
 
 template <int D, bool FP8, bool MQ>
 struct Cfg {
@@ -247,7 +246,7 @@ __global__ void __launch_bounds__(kThreads, 2)
     int stage = 0;
     uint32_t phase = 0;
     int fills = 0;
-    bool aborted = false;
+    bool aborted = p.stall_producer != 0;  // failure-path test: send nothing
     for (int s = seg_lo; s < seg_hi && !aborted; ++s) {
       // first window of page ids, issued before (and independent of) the length load
       const int4 sg = segs[s];
@@ -280,7 +279,7 @@ __global__ void __launch_bounds__(kThreads, 2)
         }
         // wait until the consumers have released this stage
         bool got = true;
-        if (lane == 0) got = mbar_wait_bounded(empty0 + 8 * stage, phase ^ 1, abort_flag, kWaitLimitNs);
+        if (lane == 0) got = mbar_wait_bounded(empty0 + 8 * stage, phase ^ 1, abort_flag, p.wait_limit_ns);
         got = __shfl_sync(0xffffffffu, got, 0);
         if (!got) {
           if (lane == 0) {
@@ -347,7 +346,7 @@ __global__ void __launch_bounds__(kThreads, 2)
     // Drain: every stage's last fill must have landed before the CTA may exit.
     if (lane == 0) {
       for (int k = max(0, fills - C::kStages); k < fills; ++k)
-        mbar_wait_bounded(full0 + 8 * (k % C::kStages), (k / C::kStages) & 1, abort_flag, kWaitLimitNs);
+        mbar_wait_bounded(full0 + 8 * (k % C::kStages), (k / C::kStages) & 1, abort_flag, p.wait_limit_ns);
     }
     return;
   }
@@ -456,7 +455,7 @@ __global__ void __launch_bounds__(kThreads, 2)
       for (int e = 0; e < 2 * NR; ++e) o[i][e] = 0.f;
 
     for (int c0 = si.tok0; c0 < si.tok1; c0 += kChunk) {
-      const bool got = mbar_wait_bounded(full0 + 8 * stage, phase, abort_flag, kWaitLimitNs);
+      const bool got = mbar_wait_bounded(full0 + 8 * stage, phase, abort_flag, p.wait_limit_ns);
       if (!got && lane == 0) {
         if (!*abort_flag) record_status(hdr_w, DA_DEV_TIMEOUT, s);
         *abort_flag = 1;

@@ -34,7 +34,8 @@
 // reads TMEM lanes 32w..32w+31), 4 TMA producer, 5 MMA issuer (one thread).
 // TMEM: 64 columns = S[2] and O[2] (16 fp32 columns each), double buffered so
 // the tensor core computes chunk i+1's scores while the softmax warps work on
-// chunk i.  Every wait is bounded; TMEM is freed on every path out.
+// chunk i.  Every wait is bounded (DecodeParams::wait_limit_ns); TMEM is freed on
+// every path out.
 #include <cuda_fp16.h>
 
 #include <cfloat>
@@ -55,7 +56,6 @@ constexpr int kStagesTc = 3;
 constexpr int kTileBytes = kChunk * 128;  // K (or V) of one chunk: 16 KB
 constexpr int kStageBytes = 2 * kTileBytes;
 constexpr uint32_t kTmemCols = 64;    // S[2] at columns 0, 16; O[2] at 32, 48
-constexpr uint64_t kWaitNs = 2000000000ull;  // 2 s: far beyond any legitimate wait
 constexpr float kPShift = 8.f;        // P' = 2^8 P
 constexpr float kFloor = 40.f;        // a chunk's reference stays within 2^40 of the running max
 
@@ -309,7 +309,7 @@ __global__ void __launch_bounds__(kThreadsTc, 2)
     int stage = 0;
     uint32_t phase = 0;
     int fills = 0;
-    bool aborted = false;
+    bool aborted = p.stall_producer != 0;  // failure-path test: send nothing
     for (int s = seg_lo; s < seg_hi && !aborted; ++s) {
       const int4 sg = segs[s];
       int win_base = INT_MIN / 2, win_val = -1;
@@ -339,7 +339,7 @@ __global__ void __launch_bounds__(kThreadsTc, 2)
           if (16 * i < n) ok = ok && pid[i] >= 0 && pid[i] < p.num_pages;
         }
         bool got = true;
-        if (lane == 0) got = mbar_wait_bounded(bar(kBarEmpty + stage), phase ^ 1, abort_flag, kWaitNs);
+        if (lane == 0) got = mbar_wait_bounded(bar(kBarEmpty + stage), phase ^ 1, abort_flag, p.wait_limit_ns);
         got = __shfl_sync(0xffffffffu, got, 0);
         if (!got) {
           if (lane == 0) {
@@ -398,7 +398,7 @@ __global__ void __launch_bounds__(kThreadsTc, 2)
     // every stage's last fill must have landed before the CTA may exit
     if (lane == 0) {
       for (int k = max(0, fills - kStagesTc); k < fills; ++k)
-        mbar_wait_bounded(bar(kBarFull + k % kStagesTc), (k / kStagesTc) & 1, abort_flag, kWaitNs);
+        mbar_wait_bounded(bar(kBarFull + k % kStagesTc), (k / kStagesTc) & 1, abort_flag, p.wait_limit_ns);
     }
   } else if (warp == kMmaWarp) {
     // ------------------------------------------------------------------ MMA issuer
@@ -420,7 +420,7 @@ __global__ void __launch_bounds__(kThreadsTc, 2)
         if (!si.valid) continue;
         const int nch = (si.tok1 - si.tok0 + kChunk - 1) / kChunk;
         if (nch == 0) continue;  // no chunk, no q tile: the softmax warps write 0 / -inf
-        if (!mbar_wait_bounded(bar(kBarQFull), js & 1, abort_flag, kWaitNs)) {
+        if (!mbar_wait_bounded(bar(kBarQFull), js & 1, abort_flag, p.wait_limit_ns)) {
           fail(s);
           break;
         }
@@ -463,7 +463,7 @@ __global__ void __launch_bounds__(kThreadsTc, 2)
           }
           if (progressed) {
             t_last = global_timer_ns();
-          } else if ((it & 63) == 0 && (*abort_flag || global_timer_ns() - t_last > kWaitNs)) {
+          } else if ((it & 63) == 0 && (*abort_flag || global_timer_ns() - t_last > p.wait_limit_ns)) {
             fail(s);
             break;
           }
@@ -472,7 +472,7 @@ __global__ void __launch_bounds__(kThreadsTc, 2)
       }
       // drain: every MMA this thread issued has completed before TMEM is freed
       tc_commit(bar(kBarDone));
-      mbar_wait_timeout(bar(kBarDone), 0, kWaitNs);
+      mbar_wait_timeout(bar(kBarDone), 0, p.wait_limit_ns);
     }
     __syncwarp();
   } else {
@@ -497,7 +497,7 @@ __global__ void __launch_bounds__(kThreadsTc, 2)
     // returns: after a timeout the warps keep walking the plan, skip the tensor-memory
     // reads and write results that the status word marks as invalid.
     auto wait = [&](uint32_t b, uint32_t parity, int s) -> bool {
-      const bool ok = __all_sync(0xffffffffu, mbar_wait_bounded(b, parity, abort_flag, kWaitNs));
+      const bool ok = __all_sync(0xffffffffu, mbar_wait_bounded(b, parity, abort_flag, p.wait_limit_ns));
       if (!ok) fail(s);
       return ok;
     };

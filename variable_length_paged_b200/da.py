@@ -22,7 +22,7 @@ PLAN_DYNAMIC, PLAN_STATIC = 0, 1
 EXPORTS = ("da_plan_desc_init", "da_workspace_size", "da_workspace_offsets", "da_plan", "da_static_plan",
            "da_decode_attention", "da_combine", "da_read_status", "da_status_string", "da_dev_status_string",
            "da_last_cuda_error", "da_device_num_sms", "da_decode_step_noalloc", "da_append_kv",
-           "da_decode_attention_fp8", "da_merge_partials", "da_decode_step_host")
+           "da_decode_attention_fp8", "da_merge_partials", "da_decode_step_host", "da_test_stall_next_decode")
 
 NOALLOC_SCRATCH_BYTES = 16 << 20  # DA_NOALLOC_SCRATCH_BYTES
 
@@ -78,6 +78,7 @@ def lib():
             "da_append_kv": [P, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp],
             "da_merge_partials": [ctypes.c_int32, ctypes.c_int64, ctypes.c_int32, _vp, _vp, _vp, _vp, _vp],
             "da_decode_attention_fp8": [P, D, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp],
+            "da_test_stall_next_decode": [ctypes.c_uint32],
             "da_decode_step_host": [P, D, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _sz, _vp, _vp, _vp,
                                     _vp, _vp, _vp, _vp],
         }
@@ -220,6 +221,12 @@ def da_read_status(ws, stream=None) -> tuple[int, int]:
     st, bad = ctypes.c_int32(), ctypes.c_int32()
     _check("da_read_status", lib().da_read_status(_ptr(ws), ctypes.byref(st), ctypes.byref(bad), _stream(stream)))
     return st.value, bad.value
+
+
+def da_test_stall_next_decode(wait_limit_us: int):
+    """Failure-path test: the next decode launch on this thread waits for K/V that never come
+    and gives up after `wait_limit_us` (status DA_DEV_TIMEOUT); see include/da.h."""
+    _check("da_test_stall_next_decode", lib().da_test_stall_next_decode(int(wait_limit_us)))
 
 
 def da_device_num_sms() -> int:
