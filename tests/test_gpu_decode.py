@@ -173,3 +173,15 @@ def test_full_size_configs(da_lib, oracle_lib, name):
     # the static comparator on the same inputs
     out_s, lse_s, *_ = run_step(w, kind=da.PLAN_STATIC)
     check_against_oracle(w, out_s, lse_s)
+
+
+def test_batch_past_the_planner_shared_memory_copy(da_lib, oracle_lib):
+    """5000 short requests (empty ones included): the planner's global-memory path, a combine
+    grid of 5000 x Hq blocks, and the decode kernel walking thousands of one-tile segments."""
+    rng = np.random.default_rng(77)
+    lens = rng.integers(0, 400, size=5000)
+    lens[rng.random(5000) < 0.1] = 0
+    w = W.make_workload("many", lens, num_q_heads=8, num_kv_heads=2, head_dim=64, page_size=32, seed=77)
+    out, lse, desc, bufs, _ = run_step(w)
+    assert da.da_read_status(bufs.ws) == (0, -1)
+    check_against_oracle(w, out, lse)

@@ -85,3 +85,21 @@ def test_static_plan(da_lib, oracle_lib, S):
         got, cap = plan_on_device(lens, 64, S, da.PLAN_STATIC)
         assert_plan_equal(got, oracle.static_plan(lens, 64, S, cap))
         assert got["splits"] == S and got["kind"] == da.PLAN_STATIC
+
+
+@pytest.mark.parametrize("B,C", [(4097, 37), (6000, 296), (20000, 1000)])
+def test_dynamic_plan_batches_past_the_shared_memory_copy(da_lib, oracle_lib, B, C):
+    """Above 4096 requests the planner reads its prefix arrays back from global memory."""
+    rng = np.random.default_rng(B)
+    lens = rng.integers(0, 3000, size=B)
+    lens[rng.random(B) < 0.2] = 0
+    got, cap = plan_on_device(lens, 64, C, da.PLAN_DYNAMIC)
+    assert_plan_equal(got, oracle.plan(lens, 64, C, cap))
+    assert got["status"] == 0
+
+
+def test_static_plan_large_batch(da_lib, oracle_lib):
+    rng = np.random.default_rng(5)
+    lens = rng.integers(0, 2000, size=5000)
+    got, cap = plan_on_device(lens, 64, 2, da.PLAN_STATIC)
+    assert_plan_equal(got, oracle.static_plan(lens, 64, 2, cap))

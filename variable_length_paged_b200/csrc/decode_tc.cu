@@ -34,7 +34,8 @@
 // reads TMEM lanes 32w..32w+31), 4 TMA producer, 5 MMA issuer (one thread).
 // TMEM: 64 columns = S[2] and O[2] (16 fp32 columns each), double buffered so
 // the tensor core computes chunk i+1's scores while the softmax warps work on
-// chunk i.  Every wait is bounded (DecodeParams::wait_limit_ns); TMEM is freed on
+// chunk i.  The q tile is double buffered too: segment j+1's tile is written when
+// segment j starts, so the MMA thread runs on across segment boundaries.  Every wait is bounded (DecodeParams::wait_limit_ns); TMEM is freed on
 // every path out.
 #include <cuda_fp16.h>
 
@@ -61,14 +62,14 @@ constexpr float kFloor = 40.f;        // a chunk's reference stays within 2^40 o
 
 // shared memory map (offsets from a 1024-byte aligned base)
 constexpr int kOffStages = 0;
-constexpr int kOffQ8 = kStagesTc * kStageBytes;  // 16 rows x 128 B, 128-byte swizzle (1024-aligned)
-constexpr int kOffP = kOffQ8 + 2048;             // [2][128 tokens][16 B]
+constexpr int kOffQ8 = kStagesTc * kStageBytes;  // [2][16 rows x 128 B], 128-byte swizzle (1024-aligned)
+constexpr int kOffP = kOffQ8 + 2 * 2048;         // [2][128 tokens][16 B]
 constexpr int kOffRed = kOffP + 2 * 2048;        // [2][4 warps][8] floats
-constexpr int kOffRowScale = kOffRed + 2 * 32 * 4;  // [8] floats
-constexpr int kOffBars = kOffRowScale + 8 * 4;
-// mbarriers: full[3], empty[3], s_full[2], s_free[2], p_full[2], o_full[2], o_free[2], q_full, done
+constexpr int kOffRowScale = kOffRed + 2 * 32 * 4;  // [2][8] floats
+constexpr int kOffBars = kOffRowScale + 2 * 8 * 4;
+// mbarriers: full[3], empty[3], s_full[2], s_free[2], p_full[2], o_full[2], o_free[2], q_full[2], done
 constexpr int kBarFull = 0, kBarEmpty = 3, kBarSFull = 6, kBarSFree = 8, kBarPFull = 10, kBarOFull = 12,
-              kBarOFree = 14, kBarQFull = 16, kBarDone = 17, kNumBars = 18;
+              kBarOFree = 14, kBarQFull = 16, kBarDone = 18, kNumBars = 19;
 constexpr int kOffMeta = kOffBars + kNumBars * 8;  // loaded tokens per stage
 constexpr int kOffFlags = kOffMeta + kStagesTc * 4;  // abort flag, TMEM base address
 constexpr int kBytesTc = kOffFlags + 16;
@@ -262,6 +263,7 @@ __global__ void __launch_bounds__(kThreadsTc, 2)
       mbar_init(bar(kBarOFree + j), kSoftmaxWarps);
     }
     mbar_init(bar(kBarQFull), kSoftmaxWarps);
+    mbar_init(bar(kBarQFull + 1), kSoftmaxWarps);
     mbar_init(bar(kBarDone), 1);
     *abort_flag = 0;
     fence_mbar_init();
@@ -407,68 +409,75 @@ __global__ void __launch_bounds__(kThreadsTc, 2)
     // producer), S of chunk is as soon as its K/V have landed and its score
     // buffer is free.  Chunk ic sits in stage ic % kStagesTc, S and O buffers ic % 2.
     if (lane == 0) {
-      const uint32_t q8 = sbase + kOffQ8;
-      int i0 = 0, js = 0;  // first chunk of the segment, segment counter (as on every role)
       bool aborted = false;
       auto fail = [&](int s) {
         if (!*abort_flag) record_status(hdr_w, DA_DEV_TIMEOUT, s);
         *abort_flag = 1;
         aborted = true;
       };
-      for (int s = seg_lo; s < seg_hi && !aborted; ++s) {
-        const SegmentInfo si = load_segment(p, segs, s);
-        if (!si.valid) continue;
-        const int nch = (si.tok1 - si.tok0 + kChunk - 1) / kChunk;
-        if (nch == 0) continue;  // no chunk, no q tile: the softmax warps write 0 / -inf
-        if (!mbar_wait_bounded(bar(kBarQFull), js & 1, abort_flag, p.wait_limit_ns)) {
-          fail(s);
+      // S cursor: segment s_seg (the s_js-th with chunks) holds chunks [.., s_end); segments
+      // without chunks are skipped, as on every role
+      int s_seg = seg_lo - 1, s_end = 0, s_js = -1;
+      bool q_ready = false;
+      auto next_segment = [&]() -> bool {
+        for (++s_seg; s_seg < seg_hi; ++s_seg) {
+          const SegmentInfo si = load_segment(p, segs, s_seg);
+          if (!si.valid) continue;
+          const int nch = (si.tok1 - si.tok0 + kChunk - 1) / kChunk;
+          if (nch == 0) continue;
+          s_end += nch;
+          ++s_js;
+          q_ready = false;
+          return true;
+        }
+        return false;
+      };
+      bool more = next_segment();  // chunks left whose S is not issued
+      int is = 0, ip = 0;
+      uint64_t t_last = global_timer_ns();
+      for (uint32_t it = 0; !aborted && (more || ip < is); ++it) {
+        bool progressed = false;
+        if (ip < is) {  // O^T (chunk ic) = V^T . P'^T, then release the stage
+          const int ic = ip, ob = ic & 1, st = ic % kStagesTc;
+          if (mbar_test(bar(kBarPFull + ob), (ic >> 1) & 1) &&
+              (ic < 2 || mbar_test(bar(kBarOFree + ob), ((ic >> 1) - 1) & 1))) {
+            tc_fence_after();
+            const uint32_t vt = sbase + kOffStages + st * kStageBytes + kTileBytes;
+            const uint32_t pt = sbase + kOffP + ob * 2048;
+#pragma unroll
+            for (int j = 0; j < 4; ++j)
+              tc_mma(tmem + 32 + 16 * ob, smem_desc(vt + 4096 * j, 1024, 1024, 2),
+                     smem_desc(pt + 512 * j, 128, 128, 0), kIdescPV, j > 0);
+            tc_commit(bar(kBarOFull + ob));
+            tc_commit(bar(kBarEmpty + st));
+            ++ip;
+            progressed = true;
+          }
+        }
+        if (more) {  // S^T (chunk ic) = K . Q8^T, with the q tile of the chunk's segment
+          if (!q_ready) q_ready = mbar_test(bar(kBarQFull + (s_js & 1)), (s_js >> 1) & 1);
+          const int ic = is, sb = ic & 1, st = ic % kStagesTc;
+          if (q_ready && mbar_test(bar(kBarFull + st), (ic / kStagesTc) & 1) &&
+              (ic < 2 || mbar_test(bar(kBarSFree + sb), ((ic >> 1) - 1) & 1))) {
+            tc_fence_after();
+            const uint32_t kt = sbase + kOffStages + st * kStageBytes;
+            const uint32_t q8 = sbase + kOffQ8 + (s_js & 1) * 2048;
+#pragma unroll
+            for (int j = 0; j < 4; ++j)
+              tc_mma(tmem + 16 * sb, smem_desc(kt + 32 * j, 16, 1024, 2), smem_desc(q8 + 32 * j, 16, 1024, 2),
+                     kIdescS, j > 0);
+            tc_commit(bar(kBarSFull + sb));
+            ++is;
+            progressed = true;
+            if (is == s_end) more = next_segment();
+          }
+        }
+        if (progressed) {
+          t_last = global_timer_ns();
+        } else if ((it & 63) == 0 && (*abort_flag || global_timer_ns() - t_last > p.wait_limit_ns)) {
+          fail(s_seg);
           break;
         }
-        ++js;
-        int is = 0, ip = 0;
-        uint64_t t_last = global_timer_ns();
-        for (uint32_t it = 0; ip < nch; ++it) {
-          bool progressed = false;
-          if (ip < is) {  // O^T (chunk ic) = V^T . P'^T, then release the stage
-            const int ic = i0 + ip, ob = ic & 1, st = ic % kStagesTc;
-            if (mbar_test(bar(kBarPFull + ob), (ic >> 1) & 1) &&
-                (ic < 2 || mbar_test(bar(kBarOFree + ob), ((ic >> 1) - 1) & 1))) {
-              tc_fence_after();
-              const uint32_t vt = sbase + kOffStages + st * kStageBytes + kTileBytes;
-              const uint32_t pt = sbase + kOffP + ob * 2048;
-#pragma unroll
-              for (int j = 0; j < 4; ++j)
-                tc_mma(tmem + 32 + 16 * ob, smem_desc(vt + 4096 * j, 1024, 1024, 2),
-                       smem_desc(pt + 512 * j, 128, 128, 0), kIdescPV, j > 0);
-              tc_commit(bar(kBarOFull + ob));
-              tc_commit(bar(kBarEmpty + st));
-              ++ip;
-              progressed = true;
-            }
-          }
-          if (is < nch) {  // S^T (chunk ic) = K . Q8^T
-            const int ic = i0 + is, sb = ic & 1, st = ic % kStagesTc;
-            if (mbar_test(bar(kBarFull + st), (ic / kStagesTc) & 1) &&
-                (ic < 2 || mbar_test(bar(kBarSFree + sb), ((ic >> 1) - 1) & 1))) {
-              tc_fence_after();
-              const uint32_t kt = sbase + kOffStages + st * kStageBytes;
-#pragma unroll
-              for (int j = 0; j < 4; ++j)
-                tc_mma(tmem + 16 * sb, smem_desc(kt + 32 * j, 16, 1024, 2), smem_desc(q8 + 32 * j, 16, 1024, 2),
-                       kIdescS, j > 0);
-              tc_commit(bar(kBarSFull + sb));
-              ++is;
-              progressed = true;
-            }
-          }
-          if (progressed) {
-            t_last = global_timer_ns();
-          } else if ((it & 63) == 0 && (*abort_flag || global_timer_ns() - t_last > p.wait_limit_ns)) {
-            fail(s);
-            break;
-          }
-        }
-        i0 += nch;
       }
       // drain: every MMA this thread issued has completed before TMEM is freed
       tc_commit(bar(kBarDone));
@@ -501,6 +510,54 @@ __global__ void __launch_bounds__(kThreadsTc, 2)
       if (!ok) fail(s);
       return ok;
     };
+    // q of request b as E4M3 rows of q tile jq & 1: row h = hi terms of head h, row 8 + h =
+    // lo terms (rows of heads >= G stay 0).  Thread t: head t / 16, dims 8 (t % 16) .. + 7;
+    // head h's q is scaled by 2^e_h, e_h putting its largest |q| in [128, 256); 2^-e_h goes
+    // into that head's score scale.  Ends with the named barrier and q_full's arrival.
+    auto write_q = [&](int b, int jq) {
+      const int h = t >> 4, part = t & 15;
+      uint2 r0 = make_uint2(0, 0), r1 = make_uint2(0, 0);  // q is 8-byte aligned (API rule)
+      if (h < G) {
+        const uint2* src =
+            reinterpret_cast<const uint2*>(p.q + ((int64_t)b * p.num_q_heads + (int64_t)g * G + h) * kD + 8 * part);
+        r0 = __ldg(src);
+        r1 = __ldg(src + 1);
+      }
+      const uint32_t w4[4] = {r0.x, r0.y, r1.x, r1.y};
+      float v[8];
+      float amax = 0.f;
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        v[2 * k] = bf16_lo_to_f32(w4[k]);
+        v[2 * k + 1] = bf16_hi_to_f32(w4[k]);
+        amax = fmaxf(amax, fmaxf(fabsf(v[2 * k]), fabsf(v[2 * k + 1])));
+      }
+#pragma unroll
+      for (int o = 1; o < 16; o <<= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+      const int e = amax > 0.f ? min(max(134 - (int)(__float_as_uint(amax) >> 23), -120), 120) : 0;
+      const float up = __uint_as_float((uint32_t)(127 + e) << 23);
+      uint32_t hi[4], lo[4];
+#pragma unroll
+      for (int k = 0; k < 4; ++k) split_e4m3x2(pack_f16x2(v[2 * k] * up, v[2 * k + 1] * up), hi[k], lo[k]);
+      // row r, logical bytes 8 part .. + 7: 16-byte chunk part / 2 (xor r % 8), half part % 2
+      uint8_t* tile = smem + kOffQ8 + (jq & 1) * 2048;
+      auto q_at = [&](int r) -> uint8_t* { return tile + r * 128 + ((((part >> 1) ^ (r & 7))) << 4) + (part & 1) * 8; };
+      *reinterpret_cast<uint2*>(q_at(h)) = make_uint2(hi[0] | (hi[1] << 16), hi[2] | (hi[3] << 16));
+      *reinterpret_cast<uint2*>(q_at(8 + h)) = make_uint2(lo[0] | (lo[1] << 16), lo[2] | (lo[3] << 16));
+      if (part == 0) row_scale[(jq & 1) * 8 + h] = score_scale * __uint_as_float((uint32_t)(127 - e) << 23);
+      fence_proxy_async_smem();  // the tensor core reads the q tile
+      named_barrier_sync(1, kSoftmaxWarps * 32);
+      if (lane == 0) mbar_arrive(bar(kBarQFull + (jq & 1)));
+    };
+    // the next segment after s that has chunks (its request), or -1
+    auto next_with_chunks = [&](int s) -> int {
+      for (int s2 = s + 1; s2 < seg_hi; ++s2) {
+        const SegmentInfo n2 = load_segment(p, segs, s2);
+        if (n2.valid && n2.tok1 > n2.tok0) return n2.b;
+      }
+      return -1;
+    };
+    int js = 0;  // segments with chunks seen so far (same count as the MMA thread's)
     for (int s = seg_lo; s < seg_hi; ++s) {
       const SegmentInfo si = load_segment(p, segs, s);
       if (!si.valid) continue;
@@ -515,49 +572,15 @@ __global__ void __launch_bounds__(kThreadsTc, 2)
         f_prev[h] = 1.f;
       }
       if (nch > 0) {
-        // q of the segment as E4M3 rows of the Q8 tile: row h = hi terms of head h, row
-        // 8 + h = lo terms (rows of heads >= G stay 0).  Thread t: head t / 16, dims
-        // 8 (t % 16) .. + 7; head h's q is scaled by 2^e_h, e_h putting its largest |q|
-        // in [128, 256); 2^-e_h goes into that head's score scale.
-        {
-          const int h = t >> 4, part = t & 15;
-          uint2 r0 = make_uint2(0, 0), r1 = make_uint2(0, 0);  // q is 8-byte aligned (API rule)
-          if (h < G) {
-            const uint2* src = reinterpret_cast<const uint2*>(
-                p.q + ((int64_t)b * p.num_q_heads + (int64_t)g * G + h) * kD + 8 * part);
-            r0 = __ldg(src);
-            r1 = __ldg(src + 1);
-          }
-          const uint32_t w4[4] = {r0.x, r0.y, r1.x, r1.y};
-          float v[8];
-          float amax = 0.f;
-#pragma unroll
-          for (int k = 0; k < 4; ++k) {
-            v[2 * k] = bf16_lo_to_f32(w4[k]);
-            v[2 * k + 1] = bf16_hi_to_f32(w4[k]);
-            amax = fmaxf(amax, fmaxf(fabsf(v[2 * k]), fabsf(v[2 * k + 1])));
-          }
-#pragma unroll
-          for (int o = 1; o < 16; o <<= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
-          const int e = amax > 0.f ? min(max(134 - (int)(__float_as_uint(amax) >> 23), -120), 120) : 0;
-          const float up = __uint_as_float((uint32_t)(127 + e) << 23);
-          uint32_t hi[4], lo[4];
-#pragma unroll
-          for (int k = 0; k < 4; ++k) split_e4m3x2(pack_f16x2(v[2 * k] * up, v[2 * k + 1] * up), hi[k], lo[k]);
-          // row r, logical bytes 8 part .. + 7: 16-byte chunk part / 2 (xor r % 8), half part % 2
-          auto q_at = [&](int r) -> uint8_t* {
-            return smem + kOffQ8 + r * 128 + ((((part >> 1) ^ (r & 7))) << 4) + (part & 1) * 8;
-          };
-          *reinterpret_cast<uint2*>(q_at(h)) = make_uint2(hi[0] | (hi[1] << 16), hi[2] | (hi[3] << 16));
-          *reinterpret_cast<uint2*>(q_at(8 + h)) = make_uint2(lo[0] | (lo[1] << 16), lo[2] | (lo[3] << 16));
-          if (part == 0) row_scale[h] = score_scale * __uint_as_float((uint32_t)(127 - e) << 23);
-        }
-        fence_proxy_async_smem();  // the tensor core reads the Q8 tile
-        named_barrier_sync(1, kSoftmaxWarps * 32);
-        if (lane == 0) mbar_arrive(bar(kBarQFull));
+        // this segment's q tile was written one segment ahead (the first one, now); write the
+        // next segment's into the other buffer, whose last user (segment js - 1) is finished
+        if (js == 0) write_q(b, 0);
+        const int bn = next_with_chunks(s);
+        if (bn >= 0) write_q(bn, js + 1);
+        const int jcur = js++;
         float rsc[8];
 #pragma unroll
-        for (int h = 0; h < 8; ++h) rsc[h] = row_scale[h];
+        for (int h = 0; h < 8; ++h) rsc[h] = row_scale[(jcur & 1) * 8 + h];
 
         // fold chunk ic's O^T (its reference reached by factor f from the previous one)
         auto fold = [&](int ic, const float (&f)[8]) {
