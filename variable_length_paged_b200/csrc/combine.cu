@@ -8,35 +8,23 @@
 // Requests with one segment were written by the decode kernel; requests with
 // none get out = 0, lse = -inf.
 //
-// One 128-thread block per (request, query head).  Every warp reads the
-// segments' lse values with its lanes in parallel (max and sum by warp
-// reductions, in a fixed order); warp w then accumulates segments w, w+4,
-// w+8, ... with each lane owning head_dim/32 columns and the loads unrolled so
-// that several are in flight (a request split over many CTAs has tens of
-// segments); the four warp sums are added in warp order through shared
-// memory.  The order of every sum is fixed, so results are deterministic.
+// One 128-thread block per (request, query head), one pass over the partials:
+// warp w takes segments w, w+4, w+8, ... (lse and the lane's head_dim/32 columns
+// loaded together, unrolled so that several segments are in flight) and keeps
+// its own max m_w, sum l_w = sum exp(lse_i - m_w) and accumulator; the four warp
+// states are then merged in warp order through shared memory.  Every sum has a
+// fixed order, so results are deterministic.
 #include "da_internal.cuh"
 
 namespace da {
 namespace {
 
-__device__ __forceinline__ float warp_max(float v) {
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
-  return v;
-}
-
-__device__ __forceinline__ float warp_sum(float v) {
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
-  return v;
-}
-
 template <int D>
 __global__ void __launch_bounds__(128) combine_kernel(const CombineParams p) {
   constexpr int kPer = D / 32;
   constexpr int kWarps = 4;
-  __shared__ float4 part[kWarps - 1][32 * kPer / 4];
+  __shared__ float4 part[kWarps][32 * kPer / 4];
+  __shared__ float ml[kWarps][2];
   grid_dependency_wait();  // partials come from the decode kernel just before
   const int b = blockIdx.x, h = blockIdx.y;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -48,59 +36,68 @@ __global__ void __launch_bounds__(128) combine_kernel(const CombineParams p) {
   const bool ok = s0 >= 0 && s1 <= p.max_segments && n >= 0;
   const int64_t hq = p.num_q_heads;
   const float* plse = p.partial_lse + (int64_t)s0 * hq + h;
+  const float* po = p.partial_o + ((int64_t)s0 * hq + h) * D + lane * kPer;
 
-  float M = -INFINITY;
-  if (ok)
-    for (int i = lane; i < n; i += 32) M = fmaxf(M, __ldcg(plse + i * hq));
-  M = warp_max(M);
-  float total = -INFINITY;
-  if (ok && M != -INFINITY) {
-    float sum = 0.f;
-    for (int i = lane; i < n; i += 32) sum += expf(__ldcg(plse + i * hq) - M);
-    total = M + logf(warp_sum(sum));
-  }
-
+  // this warp's segments, online: m = running max, l = sum exp(lse - m), acc = sum exp(lse - m) o
+  float m = -INFINITY, l = 0.f;
   float acc[kPer];
 #pragma unroll
-  for (int j = 0; j < kPer; ++j) acc[j] = 0.f;
-  if (total != -INFINITY) {
-    const float* po = p.partial_o + ((int64_t)s0 * hq + h) * D + lane * kPer;
-#pragma unroll 8
+  for (int k = 0; k < kPer; ++k) acc[k] = 0.f;
+  if (ok) {
+#pragma unroll 4
     for (int j = warp; j < n; j += kWarps) {
-      const float wj = expf(__ldcg(plse + j * hq) - total);
-      const float* src = po + (int64_t)j * hq * D;
+      const float x = __ldcg(plse + (int64_t)j * hq);
+      float v[kPer];
       if constexpr (kPer == 4) {
-        const float4 v = __ldcg(reinterpret_cast<const float4*>(src));
-        acc[0] += wj * v.x;
-        acc[1] += wj * v.y;
-        acc[2] += wj * v.z;
-        acc[3] += wj * v.w;
+        const float4 t = __ldcg(reinterpret_cast<const float4*>(po + (int64_t)j * hq * D));
+        v[0] = t.x, v[1] = t.y, v[2] = t.z, v[3] = t.w;
       } else {
-        const float2 v = __ldcg(reinterpret_cast<const float2*>(src));
-        acc[0] += wj * v.x;
-        acc[1] += wj * v.y;
+        const float2 t = __ldcg(reinterpret_cast<const float2*>(po + (int64_t)j * hq * D));
+        v[0] = t.x, v[1] = t.y;
       }
+      if (x == -INFINITY) continue;  // an empty partial carries no weight
+      const float mn = fmaxf(m, x);
+      const float c = expf(m - mn), w = expf(x - mn);  // c = 0 while m is -inf
+      l = l * c + w;
+#pragma unroll
+      for (int k = 0; k < kPer; ++k) acc[k] = acc[k] * c + w * v[k];
+      m = mn;
     }
   }
-  // warps 1..3 hand their sums to warp 0, which adds them in warp order
-  if (warp > 0) {
-    float* dst = reinterpret_cast<float*>(&part[warp - 1][0]) + lane * kPer;
+  float* mine = reinterpret_cast<float*>(&part[warp][0]) + lane * kPer;
 #pragma unroll
-    for (int j = 0; j < kPer; ++j) dst[j] = acc[j];
+  for (int k = 0; k < kPer; ++k) mine[k] = acc[k];
+  if (lane == 0) {
+    ml[warp][0] = m;
+    ml[warp][1] = l;
   }
   __syncthreads();
   if (warp != 0) return;
+  // merge the four warp states in warp order
+  float M = -INFINITY;
 #pragma unroll
-  for (int w = 0; w < kWarps - 1; ++w) {
-    const float* src = reinterpret_cast<const float*>(&part[w][0]) + lane * kPer;
+  for (int w = 0; w < kWarps; ++w) M = fmaxf(M, ml[w][0]);
+  float L = 0.f, o[kPer];
 #pragma unroll
-    for (int j = 0; j < kPer; ++j) acc[j] += src[j];
+  for (int k = 0; k < kPer; ++k) o[k] = 0.f;
+  if (M != -INFINITY) {
+#pragma unroll
+    for (int w = 0; w < kWarps; ++w) {
+      const float f = expf(ml[w][0] - M);  // 0 for a warp that saw nothing
+      L += f * ml[w][1];
+      const float* src = reinterpret_cast<const float*>(&part[w][0]) + lane * kPer;
+#pragma unroll
+      for (int k = 0; k < kPer; ++k) o[k] += f * src[k];
+    }
   }
+  const float inv = L > 0.f ? 1.f / L : 0.f;
+  const float total = L > 0.f ? M + logf(L) : -INFINITY;
   __nv_bfloat16* dst = p.out + ((int64_t)b * hq + h) * D + lane * kPer;
   if constexpr (kPer == 4) {
-    *reinterpret_cast<uint2*>(dst) = make_uint2(pack_bf16x2(acc[0], acc[1]), pack_bf16x2(acc[2], acc[3]));
+    *reinterpret_cast<uint2*>(dst) =
+        make_uint2(pack_bf16x2(o[0] * inv, o[1] * inv), pack_bf16x2(o[2] * inv, o[3] * inv));
   } else {
-    *reinterpret_cast<uint32_t*>(dst) = pack_bf16x2(acc[0], acc[1]);
+    *reinterpret_cast<uint32_t*>(dst) = pack_bf16x2(o[0] * inv, o[1] * inv);
   }
   if (lane == 0) p.lse[(int64_t)b * hq + h] = total;
 }
