@@ -538,4 +538,13 @@ def pin_static_brute_force(lib=None):
                         assert sum(1 for s in segs if s[3] > s[2]) == sum(-(-x // chunk) for x in n)
 
 
-PLAN_PINS = [pin_golden_plans, pin_plan_brute_force, pin_plan_random, pin_plan_bad_lengths, pin_static_brute_force]
+def pin_static_empty_splits(lib=None):
+    """Static split-k sized by the longest request leaves the short ones' later splits empty
+    (counted by hand: chunk = ceil(250 / 8) = 32 tiles; busy splits 1 + 3 + 1 + 8 of 32)."""
+    p = oracle.static_plan([100, 5000, 70, 16000], 64, 8, 2048 * 64, lib=lib)
+    empty = int(np.sum(np.asarray(p["seg_tile_end"]) == np.asarray(p["seg_tile_begin"])))
+    assert p["num_segments"] == 32 and empty == 19
+
+
+PLAN_PINS = [pin_golden_plans, pin_plan_brute_force, pin_plan_random, pin_plan_bad_lengths, pin_static_brute_force,
+             pin_static_empty_splits]

@@ -103,3 +103,19 @@ def test_static_plan_large_batch(da_lib, oracle_lib):
     lens = rng.integers(0, 2000, size=5000)
     got, cap = plan_on_device(lens, 64, 2, da.PLAN_STATIC)
     assert_plan_equal(got, oracle.static_plan(lens, 64, 2, cap))
+
+
+def test_static_plan_launches_empty_splits(da_lib, oracle_lib):
+    """The comparator's weakness the article names: with lengths that differ, a static split
+    count sized by the longest request leaves the short requests' later splits empty (their
+    CTAs are launched and find nothing), while the dynamic plan gives every CTA work."""
+    lens = [100, 5000, 70, 16000]
+    got, cap = plan_on_device(lens, 64, 8, da.PLAN_STATIC)
+    empty = int(np.sum(np.asarray(got["seg_tile_end"]) == np.asarray(got["seg_tile_begin"])))
+    # chunk = ceil(ceil(16000/64)/8) = 32 tiles: 100 -> 1 busy split, 5000 -> 3, 70 -> 1, 16000 -> 8
+    assert empty == 8 * 4 - (1 + 3 + 1 + 8)
+    dyn, _ = plan_on_device(lens, 64, 32, da.PLAN_DYNAMIC)
+    loads = np.bincount(np.asarray(dyn["seg_cta"]),
+                        weights=np.asarray(dyn["seg_tile_end"]) - np.asarray(dyn["seg_tile_begin"]), minlength=32)
+    U = sum(-(-L // 64) for L in lens)
+    assert loads.min() >= U // 32 and loads.max() <= -(-U // 32)
