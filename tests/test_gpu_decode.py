@@ -185,3 +185,15 @@ def test_batch_past_the_planner_shared_memory_copy(da_lib, oracle_lib):
     out, lse, desc, bufs, _ = run_step(w)
     assert da.da_read_status(bufs.ws) == (0, -1)
     check_against_oracle(w, out, lse)
+
+
+def test_two_million_token_request(da_lib, oracle_lib):
+    """One 2^21-token request next to short ones (32768 pages of the first request, 1 GB of
+    K/V): long segments on every CTA; sampled heads against the oracle."""
+    lens = [2 ** 21, 1, 777]
+    w = W.make_workload("long", lens, num_q_heads=8, num_kv_heads=1, head_dim=128, page_size=64, seed=41,
+                        spare_frac=0.0)
+    out, lse, desc, bufs, _ = run_step(w)
+    assert da.da_read_status(bufs.ws) == (0, -1)
+    pairs = (np.array([0, 0, 0, 1, 2], np.int32), np.array([0, 3, 7, 5, 2], np.int32))
+    check_against_oracle(w, out, lse, pairs=pairs)

@@ -119,3 +119,14 @@ def test_static_plan_launches_empty_splits(da_lib, oracle_lib):
                         weights=np.asarray(dyn["seg_tile_end"]) - np.asarray(dyn["seg_tile_begin"]), minlength=32)
     U = sum(-(-L // 64) for L in lens)
     assert loads.min() >= U // 32 and loads.max() <= -(-U // 32)
+
+
+def test_dynamic_plan_wide_division_path(da_lib, oracle_lib):
+    """C * (U + 1) >= 2^31: the planner's owner/first-tile formulas take their 64-bit form."""
+    rng = np.random.default_rng(9)
+    lens = rng.integers(2000, 6000, size=20000)
+    T, C = 16, 1000
+    U = int(sum(-(-int(L) // T) for L in lens))
+    assert C * (U + 1) >= 2 ** 31
+    got, cap = plan_on_device(lens, T, C, da.PLAN_DYNAMIC)
+    assert_plan_equal(got, oracle.plan(lens, T, C, cap))
