@@ -367,6 +367,26 @@ def run_ours(args, world, rank, local):
     return result
 
 
+def warm_apply_path(da, prob, stream):
+    """Run every kernel on a step's change path once on scratch data, so that the first timed step
+    does not pay for loading them (CUDA loads kernels lazily, on first launch)."""
+    import torch
+    with torch.cuda.stream(stream):
+        p1 = da.problem(1, prob.num_q_heads, prob.num_kv_heads, prob.head_dim, prob.page_size, 1, 2, prob.scale)
+        d1 = da.da_plan_desc_init(p1, da.PLAN_DYNAMIC, 64, 0)
+        ws = da.Buffers(p1, d1, "cuda").ws
+        kc = torch.zeros(2, prob.num_kv_heads, prob.page_size, prob.head_dim, dtype=torch.bfloat16, device="cuda")
+        vc = torch.zeros_like(kc)
+        nk = torch.zeros(1, prob.num_kv_heads, prob.head_dim, dtype=torch.bfloat16, device="cuda")
+        sl = torch.ones(1, dtype=torch.int32, device="cuda")
+        bt = torch.zeros(1, 1, dtype=torch.int32, device="cuda")
+        st = torch.zeros(2, dtype=torch.int32, device="cuda")
+        kc.index_copy_(0, torch.ones(1, dtype=torch.long, device="cuda"), vc[:1])
+        da.da_append_kv(p1, nk, nk, bt, sl, kc, vc, st, stream=stream)
+        da.da_plan_append(p1, d1, sl, ws, nk, nk, bt, kc, vc, st, stream=stream)
+    torch.cuda.synchronize()
+
+
 def run_trace(args, world, rank, local):
     """The 256-step decode trace: per step, that step's recorded changes applied on the device (untimed),
     then the timed step."""
@@ -387,33 +407,44 @@ def run_trace(args, world, rank, local):
     bufs, sbufs = da.Buffers(prob, desc, "cuda"), da.Buffers(prob, sdesc, "cuda")
     steps, warm = min(max(1, args.steps), tr.steps), max(3, args.warmup)
 
-    def step(d, b):
-        da.decode_step(prob, d, dt.q, dt.k_cache, dt.v_cache, dt.block_table, dt.seq_lens, b, stream=stream)
+    def step(d, b, planned=False):
+        da.decode_step(prob, d, dt.q, dt.k_cache, dt.v_cache, dt.block_table, dt.seq_lens, b, stream=stream,
+                       planned=planned)
 
     graphs = {}
     with torch.cuda.stream(stream):
-        for key, d, b in (("dynamic", desc, bufs), ("static", sdesc, sbufs)):
+        for key, d, b, planned in (("dynamic", desc, bufs, False), ("static", sdesc, sbufs, False),
+                                   ("after_plan_append", desc, bufs, True)):
             for _ in range(warm):
-                step(d, b)
+                step(d, b, planned)
             g = torch.cuda.CUDAGraph()
             with torch.cuda.graph(g, stream=stream):
-                step(d, b)
+                step(d, b, planned)
             graphs[key] = g
         torch.cuda.synchronize()
     # the host trace runs ahead; its per-step changes wait on the device, so the timed loop below
     # is device work only: apply step t's changes (untimed), then the two timed step variants
+    warm_apply_path(da, prob, stream)
     kv0 = tr.kv_bytes()
     ups = dt.record(steps - 1)
     kv = [kv0] + [u["kv_bytes"] for u in ups]
     ev = {k: [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
-          for k in ("dynamic", "static")}
+          for k in ("dynamic", "static", "append_separate", "append_fused")}
     clocks = ClockSampler(local)
     with clocks, torch.cuda.stream(stream):  # replay() launches on the current stream
         torch.cuda.synchronize()
         barrier(world)
         for t in range(steps):
             if t > 0:
-                dt.apply(ups[t - 1], stream=stream)
+                # the step's changes plus the step, twice: append kernel then the planned step, and the
+                # fused plan + append launch then the step without its plan (both leave the same state,
+                # every change is written at an absolute place)
+                for key, plan in (("append_separate", None), ("append_fused", (desc, bufs.ws))):
+                    e0, e1 = ev[key][t]
+                    e0.record(stream)
+                    dt.apply(ups[t - 1], stream=stream, plan=plan)
+                    graphs["dynamic" if plan is None else "after_plan_append"].replay()
+                    e1.record(stream)
             for key in ("dynamic", "static"):
                 e0, e1 = ev[key][t]
                 e0.record(stream)
@@ -421,7 +452,7 @@ def run_trace(args, world, rank, local):
                 e1.record(stream)
         torch.cuda.synchronize()
         status = da.da_read_status(bufs.ws, stream=stream)
-    times = {k: [a.elapsed_time(b) for a, b in v] for k, v in ev.items()}
+    times = {k: [a.elapsed_time(b) for a, b in (v[1:] if k.startswith("append") else v)] for k, v in ev.items()}
     tot_ms = {k: sum(v) for k, v in times.items()}
     maxes, sums = reduce_max_sum([tot_ms["dynamic"], tot_ms["static"]], [float(sum(kv))], world)
     dyn_ms, st_ms = maxes
@@ -443,7 +474,13 @@ def run_trace(args, world, rank, local):
         frac_of_peak=round(value / world / peak, 4), peak=peak, peak_source=peak_src,
         static_split_k={"default_splits": sdesc.splits, "us_per_step": round(st_ms / steps * 1e3, 2)},
         speedup_vs_static_default=round(st_ms / dyn_ms, 3),
-        gpu_launches=3 * steps * 2 + (steps - 1), device_status=status[0],
+        with_append={"note": "steps 1.. with their changes applied inside the timed region: device copies of "
+                             "block table, lengths, q and restarted pages, then the KV append",
+                     "separate_us_per_step": round(float(np.mean(times["append_separate"])) * 1e3, 2),
+                     "fused_plan_append_us_per_step": round(float(np.mean(times["append_fused"])) * 1e3, 2),
+                     "separate_us_median": round(float(np.median(times["append_separate"])) * 1e3, 2),
+                     "fused_plan_append_us_median": round(float(np.median(times["append_fused"])) * 1e3, 2)},
+        gpu_launches=3 * steps * 2 + 7 * (steps - 1), device_status=status[0],
         append_status=dt.status.tolist(), clocks=clocks.summary())
 
 

@@ -318,6 +318,21 @@ DA_API int da_append_kv(const da_problem* prob, const void* new_k, const void* n
                         const int32_t* seq_lens, void* k_cache, void* v_cache, int32_t* status, void* stream);
 
 /*
+ * da_plan_append -- da_append_kv and da_plan (DA_PLAN_DYNAMIC) in one launch: the
+ * step's bookkeeping before attention.  Block 0 of the grid builds the plan
+ * while the other blocks write every request's new K/V rows, so the appends add
+ * no time to the plan; the decode kernel that follows waits for the whole grid.
+ * Arguments, layouts, checks and results are those of the two calls (seq_lens
+ * counts the new token; `status` receives append errors, the plan's own status
+ * goes to `ws` as usual).  Source: "Tencent HPC lands in SGLang, challenging
+ * default inference kernels", section "Why Tencent HPC matters for online model
+ * serving" (lengths grow every step and the mapping is rebuilt every step).
+ */
+DA_API int da_plan_append(const da_problem* prob, const da_plan_desc* desc, const int32_t* seq_lens, void* ws,
+                          size_t ws_bytes, const void* new_k, const void* new_v, const int32_t* block_table,
+                          void* k_cache, void* v_cache, int32_t* status, void* stream);
+
+/*
  * da_merge_partials -- merge results computed over disjoint token slices of
  * the same requests (e.g. one slice per GPU when a long request's KV cache is
  * spread over several GPUs and each GPU runs the decode step on its slice):

@@ -134,6 +134,31 @@ def test_host_step_checks(da_lib):
     assert call(prob_=p0, desc=d0, q_host=None) == da.OK  # an empty batch enqueues nothing
 
 
+def test_plan_append_checks(da_lib):
+    """da_plan_append checks the plan's arguments and the append's before it launches anything."""
+    import ctypes
+    da = da_lib
+    lib = da.lib()
+    p = prob(da)
+    d = da.da_plan_desc_init(p, da.PLAN_DYNAMIC, 64, 37)
+    A = 1 << 12  # never dereferenced: every case below fails a check first
+
+    def call(prob_=p, desc=d, ws_bytes=1 << 24, **kw):
+        a = dict(sl=A, ws=A, nk=A, nv=A, bt=A, kc=A, vc=A, st=None)
+        a.update(kw)
+        return lib.da_plan_append(ctypes.byref(prob_), ctypes.byref(desc), a["sl"], a["ws"], ws_bytes, a["nk"],
+                                  a["nv"], a["bt"], a["kc"], a["vc"], a["st"], None)
+
+    for name in ("sl", "ws", "nk", "nv", "bt", "kc", "vc"):
+        assert call(**{name: None}) == da.ERR_INVALID_ARG, name
+    assert call(nk=A + 8) == da.ERR_INVALID_ARG  # rows are moved in 16-byte pieces
+    assert call(st=A + 2) == da.ERR_INVALID_ARG
+    assert call(ws_bytes=64) == da.ERR_WORKSPACE
+    s = da.da_plan_desc_init(p, da.PLAN_STATIC, 64, 2)
+    assert call(desc=s) == da.ERR_INVALID_ARG  # the fused launch builds the dynamic plan only
+    assert call(prob_=prob(da, num_q_heads=60)) == da.ERR_INVALID_ARG
+
+
 def test_stall_switch_checks_its_limit(da_lib):
     """Only the argument check is exercised here: a valid call would arm the next decode launch."""
     da = da_lib

@@ -112,3 +112,57 @@ def test_recorded_trace_replays_the_live_trace(da_lib):
         assert same(b1.out, b2.out) and torch.equal(b1.lse, b2.lse)
     assert same(live.k_cache, rec.k_cache) and same(live.v_cache, rec.v_cache)
     assert live.status.tolist() == rec.status.tolist() == [0, 0]
+
+
+def test_fused_plan_append_matches_separate_launches(da_lib, oracle_lib):
+    """da_plan_append (one launch: block 0 plans, the others append) leaves the caches, the plan and
+    the step's outputs bit for bit as da_append_kv followed by da_plan do, step after step; the plan
+    also equals the oracle's, and the outputs the fp64 oracle's at the last step."""
+    kw = dict(seed=17, batch=300, steps=24, num_q_heads=16, num_kv_heads=2, median=700.0, max_len=4096,
+              p_finish=0.08)
+    sep, fus = DeviceTrace(W.DecodeTrace(**kw)), DeviceTrace(W.DecodeTrace(**kw))
+    host = W.DecodeTrace(**kw)
+    prob = sep.prob
+    desc = da.da_plan_desc_init(prob, da.PLAN_DYNAMIC, 64, 0)
+    b1, b2 = da.Buffers(prob, desc, "cuda"), da.Buffers(prob, desc, "cuda")
+    u1, u2 = sep.record(23), fus.record(23)
+    same = lambda a, b: torch.equal(a.view(torch.int16), b.view(torch.int16))
+    cap = prob.max_pages_per_req * prob.page_size
+    for t in range(24):
+        if t > 0:
+            sep.apply(u1[t - 1])
+            fus.apply(u2[t - 1], plan=(desc, b2.ws))
+            host.advance()
+        da.decode_step(prob, desc, sep.q, sep.k_cache, sep.v_cache, sep.block_table, sep.seq_lens, b1)
+        da.decode_step(prob, desc, fus.q, fus.k_cache, fus.v_cache, fus.block_table, fus.seq_lens, b2,
+                       planned=t > 0)
+        torch.cuda.synchronize()
+        assert torch.equal(b1.ws, b2.ws)
+        assert_plan_equal(da.read_plan(desc, b2.ws), oracle.plan(host.seq_lens, 64, desc.num_ctas, cap))
+        assert same(b1.out, b2.out) and torch.equal(b1.lse, b2.lse)
+        assert same(sep.k_cache, fus.k_cache) and same(sep.v_cache, fus.v_cache)
+    check_against_oracle(host.workload(), b2.out, b2.lse)
+    assert sep.status.tolist() == fus.status.tolist() == [0, 0]
+
+
+def test_fused_plan_append_reports_bad_pages_and_lengths(da_lib):
+    """Append errors reach the append status pair, plan errors the workspace, as with the two calls."""
+    w = W.make_workload("a", [63, 64, 1, 0, 200], num_q_heads=8, num_kv_heads=2, head_dim=128, page_size=64,
+                        seed=3, max_pages_per_req=5, extra_pages=4)
+    dw = w.to("cuda")
+    prob = da.problem_from(w.problem)
+    desc = da.da_plan_desc_init(prob, da.PLAN_DYNAMIC, 64, 0)
+    bufs = da.Buffers(prob, desc, "cuda")
+    nk = torch.zeros(5, 2, 128, dtype=torch.bfloat16, device="cuda")
+    status = torch.zeros(2, dtype=torch.int32, device="cuda")
+    dw.block_table[2, 0] = w.problem.num_pages + 1
+    da.da_plan_append(prob, desc, dw.seq_lens, bufs.ws, nk, nk, dw.block_table, dw.k_cache, dw.v_cache, status)
+    torch.cuda.synchronize()
+    assert status.tolist() == [da.DEV_BAD_PAGE, 2]
+    assert da.da_read_status(bufs.ws) == (0, -1)  # the planner reads lengths only
+    status.zero_()
+    dw.seq_lens[3] = -4
+    da.da_plan_append(prob, desc, dw.seq_lens, bufs.ws, nk, nk, dw.block_table, dw.k_cache, dw.v_cache, status)
+    torch.cuda.synchronize()
+    assert status.tolist()[0] != 0
+    assert da.da_read_status(bufs.ws) == (da.DEV_BAD_SEQLEN, 3)

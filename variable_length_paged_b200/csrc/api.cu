@@ -7,6 +7,7 @@
 #include <cstring>
 #include <mutex>
 
+#include "append_rows.cuh"
 #include "da_internal.cuh"
 
 namespace {
@@ -440,32 +441,55 @@ DA_API int da_decode_step_host(const da_problem* prob, const da_plan_desc* desc,
   return e == cudaSuccess ? DA_OK : cuda_fail(e);
 }
 
-DA_API int da_append_kv(const da_problem* prob, const void* new_k, const void* new_v, const int32_t* block_table,
-                        const int32_t* seq_lens, void* k_cache, void* v_cache, int32_t* status, void* stream) {
-  int rc = check_problem(prob);
-  if (rc != DA_OK) return rc;
-  if (prob->batch == 0) return DA_OK;
+// Checks an append and fills its kernel parameters; enqueues nothing.  Call only with batch > 0.
+static int append_prepare(const da_problem* prob, const void* new_k, const void* new_v, const int32_t* block_table,
+                          const int32_t* seq_lens, void* k_cache, void* v_cache, int32_t* status,
+                          da::AppendParams* p) {
   if (!new_k || !new_v || !block_table || !seq_lens || !k_cache || !v_cache) return DA_ERR_INVALID_ARG;
   if (reinterpret_cast<uintptr_t>(new_k) % 16 != 0 || reinterpret_cast<uintptr_t>(new_v) % 16 != 0 ||
       reinterpret_cast<uintptr_t>(k_cache) % 16 != 0 || reinterpret_cast<uintptr_t>(v_cache) % 16 != 0 ||
       reinterpret_cast<uintptr_t>(status) % 4 != 0)
     return DA_ERR_INVALID_ARG;
+  p->new_k = static_cast<const __nv_bfloat16*>(new_k);
+  p->new_v = static_cast<const __nv_bfloat16*>(new_v);
+  p->block_table = block_table;
+  p->seq_lens = seq_lens;
+  p->k_cache = static_cast<__nv_bfloat16*>(k_cache);
+  p->v_cache = static_cast<__nv_bfloat16*>(v_cache);
+  p->status = status;
+  p->batch = prob->batch;
+  p->num_kv_heads = prob->num_kv_heads;
+  p->head_dim = prob->head_dim;
+  p->page_size = prob->page_size;
+  p->max_pages_per_req = prob->max_pages_per_req;
+  p->num_pages = prob->num_pages;
+  p->capacity_tokens = (int64_t)prob->max_pages_per_req * prob->page_size;
+  return DA_OK;
+}
+
+DA_API int da_append_kv(const da_problem* prob, const void* new_k, const void* new_v, const int32_t* block_table,
+                        const int32_t* seq_lens, void* k_cache, void* v_cache, int32_t* status, void* stream) {
+  int rc = check_problem(prob);
+  if (rc != DA_OK) return rc;
+  if (prob->batch == 0) return DA_OK;
   da::AppendParams p;
-  p.new_k = static_cast<const __nv_bfloat16*>(new_k);
-  p.new_v = static_cast<const __nv_bfloat16*>(new_v);
-  p.block_table = block_table;
-  p.seq_lens = seq_lens;
-  p.k_cache = static_cast<__nv_bfloat16*>(k_cache);
-  p.v_cache = static_cast<__nv_bfloat16*>(v_cache);
-  p.status = status;
-  p.batch = prob->batch;
-  p.num_kv_heads = prob->num_kv_heads;
-  p.head_dim = prob->head_dim;
-  p.page_size = prob->page_size;
-  p.max_pages_per_req = prob->max_pages_per_req;
-  p.num_pages = prob->num_pages;
-  p.capacity_tokens = (int64_t)prob->max_pages_per_req * prob->page_size;
+  rc = append_prepare(prob, new_k, new_v, block_table, seq_lens, k_cache, v_cache, status, &p);
+  if (rc != DA_OK) return rc;
   cudaError_t e = da::launch_append(p, static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? DA_OK : cuda_fail(e);
+}
+
+DA_API int da_plan_append(const da_problem* prob, const da_plan_desc* desc, const int32_t* seq_lens, void* ws,
+                          size_t ws_bytes, const void* new_k, const void* new_v, const int32_t* block_table,
+                          void* k_cache, void* v_cache, int32_t* status, void* stream) {
+  da::PlanParams pp;
+  int rc = plan_prepare(prob, desc, seq_lens, ws, ws_bytes, DA_PLAN_DYNAMIC, &pp);
+  if (rc != DA_OK) return rc;
+  if (prob->batch == 0) return plan_launch(pp, DA_PLAN_DYNAMIC, stream);  // nothing to append
+  da::AppendParams ap;
+  rc = append_prepare(prob, new_k, new_v, block_table, seq_lens, k_cache, v_cache, status, &ap);
+  if (rc != DA_OK) return rc;
+  cudaError_t e = da::launch_plan_append(pp, ap, static_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? DA_OK : cuda_fail(e);
 }
 

@@ -12,6 +12,7 @@
 // arithmetic, so the result is bit-exact and independent of thread timing.
 #include <climits>
 
+#include "append_rows.cuh"
 #include "da_internal.cuh"
 
 namespace da {
@@ -131,12 +132,11 @@ __device__ __forceinline__ int last_not_above(const int32_t* a, int n, int64_t x
   return lo;
 }
 
-__global__ void __launch_bounds__(kPlanThreads) plan_dynamic_kernel(const PlanParams p) {
+// The dynamic plan, computed by one block of kPlanThreads threads.
+__device__ void plan_dynamic_body(const PlanParams& p) {
   __shared__ int warp_buf[32];
   __shared__ int s_bad;
   __shared__ int32_t s_rtp[kSmemBatch + 1], s_rsb[kSmemBatch + 1];
-  grid_dependency_wait();     // seq_lens may come from the previous kernel in the stream
-  grid_dependents_launch();   // let the decode kernel start its prologue
   if (threadIdx.x == 0) s_bad = INT_MAX;
   __syncthreads();
 
@@ -216,6 +216,25 @@ __global__ void __launch_bounds__(kPlanThreads) plan_dynamic_kernel(const PlanPa
   if (threadIdx.x == 0) write_header(p, hdr, U, S, DA_PLAN_DYNAMIC, 0, s_bad);
 }
 
+__global__ void __launch_bounds__(kPlanThreads) plan_dynamic_kernel(const PlanParams p) {
+  grid_dependency_wait();    // seq_lens may come from the previous kernel in the stream
+  grid_dependents_launch();  // let the decode kernel start its prologue
+  plan_dynamic_body(p);
+}
+
+// One launch for the step's bookkeeping: block 0 plans while the other blocks write
+// every request's new K/V rows into their pages, so the appends add no time to the
+// plan's critical path.  The decode kernel waits for the whole grid.
+__global__ void __launch_bounds__(kPlanThreads) plan_append_kernel(const PlanParams p, const AppendParams a) {
+  grid_dependency_wait();
+  grid_dependents_launch();
+  if (blockIdx.x == 0) {
+    plan_dynamic_body(p);
+  } else {
+    for (int b = blockIdx.x - 1; b < a.batch; b += gridDim.x - 1) append_request_rows(a, b, threadIdx.x, blockDim.x);
+  }
+}
+
 __global__ void __launch_bounds__(kPlanThreads) plan_static_kernel(const PlanParams p) {
   __shared__ int warp_buf[32];
   __shared__ int s_bad;
@@ -276,6 +295,19 @@ cudaError_t launch_plan_dynamic(const PlanParams& p, cudaStream_t stream) {
 
 cudaError_t launch_plan_static(const PlanParams& p, cudaStream_t stream) {
   return launch_planner(plan_static_kernel, p, stream);
+}
+
+cudaError_t launch_plan_append(const PlanParams& p, const AppendParams& a, cudaStream_t stream) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(1 + (unsigned)min(a.batch, 512), 1, 1);
+  cfg.blockDim = dim3(kPlanThreads, 1, 1);
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, plan_append_kernel, p, a);
 }
 
 }  // namespace da

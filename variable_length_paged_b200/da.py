@@ -22,7 +22,8 @@ PLAN_DYNAMIC, PLAN_STATIC = 0, 1
 EXPORTS = ("da_plan_desc_init", "da_workspace_size", "da_workspace_offsets", "da_plan", "da_static_plan",
            "da_decode_attention", "da_combine", "da_read_status", "da_status_string", "da_dev_status_string",
            "da_last_cuda_error", "da_device_num_sms", "da_decode_step_noalloc", "da_append_kv",
-           "da_decode_attention_fp8", "da_merge_partials", "da_decode_step_host", "da_test_stall_next_decode")
+           "da_decode_attention_fp8", "da_merge_partials", "da_decode_step_host", "da_test_stall_next_decode",
+           "da_plan_append")
 
 NOALLOC_SCRATCH_BYTES = 16 << 20  # DA_NOALLOC_SCRATCH_BYTES
 
@@ -79,6 +80,7 @@ def lib():
             "da_merge_partials": [ctypes.c_int32, ctypes.c_int64, ctypes.c_int32, _vp, _vp, _vp, _vp, _vp],
             "da_decode_attention_fp8": [P, D, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp],
             "da_test_stall_next_decode": [ctypes.c_uint32],
+            "da_plan_append": [P, D, _vp, _vp, _sz, _vp, _vp, _vp, _vp, _vp, _vp, _vp],
             "da_decode_step_host": [P, D, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _sz, _vp, _vp, _vp,
                                     _vp, _vp, _vp, _vp],
         }
@@ -209,6 +211,15 @@ def da_append_kv(prob, new_k, new_v, block_table, seq_lens, k_cache, v_cache, st
                                               _stream(stream)))
 
 
+def da_plan_append(prob, desc, seq_lens, ws, new_k, new_v, block_table, k_cache, v_cache, status=None,
+                   ws_bytes: int | None = None, stream=None):
+    """da_append_kv + da_plan in one launch (block 0 plans, the other blocks append)."""
+    nbytes = ws.numel() * ws.element_size() if ws_bytes is None else ws_bytes
+    _check("da_plan_append", lib().da_plan_append(
+        ctypes.byref(prob), ctypes.byref(desc), _ptr(seq_lens), _ptr(ws), nbytes, _ptr(new_k), _ptr(new_v),
+        _ptr(block_table), _ptr(k_cache), _ptr(v_cache), _ptr(status), _stream(stream)))
+
+
 def da_merge_partials(part_out, part_lse, out, lse, stream=None):
     """part_out [n, ..., d] bf16 and part_lse [n, ...] fp32 -> out [..., d], lse [...]."""
     n = part_out.shape[0]
@@ -260,11 +271,14 @@ class Buffers:
 
 
 def decode_step(prob, desc, q, k_cache, v_cache, block_table, seq_lens, bufs: Buffers, stream=None, k_scale=None,
-                v_scale=None):
+                v_scale=None, planned: bool = False):
     """Plan (dynamic or static, per `desc.kind`) + decode + combine, asynchronously on `stream`.
 
-    With k_scale/v_scale given, the caches are FP8 E4M3 codes (da_decode_attention_fp8)."""
-    if desc.kind == PLAN_DYNAMIC:
+    With k_scale/v_scale given, the caches are FP8 E4M3 codes (da_decode_attention_fp8).
+    planned=True skips the plan: da_plan_append has already written it into bufs.ws."""
+    if planned:
+        pass
+    elif desc.kind == PLAN_DYNAMIC:
         da_plan(prob, desc, seq_lens, bufs.ws, stream=stream)
     else:
         da_static_plan(prob, desc, seq_lens, bufs.ws, stream=stream)

@@ -66,9 +66,12 @@ class DeviceTrace:
             ups.append(d)
         return ups
 
-    def apply(self, upd: dict, stream=None):
+    def apply(self, upd: dict, stream=None, plan=None):
         """Enqueue one recorded step's changes on `stream`: page copies of restarted requests,
-        block table, lengths and q (device to device), then the append kernel."""
+        block table, lengths and q (device to device), then the append kernel.
+
+        With plan=(desc, ws) the append is fused with the step's dynamic plan into `ws`
+        (da_plan_append), and the decode that follows skips its own planning."""
         s = stream if stream is not None else torch.cuda.current_stream()
         with torch.cuda.stream(s):
             if "pages" in upd:
@@ -77,5 +80,10 @@ class DeviceTrace:
             self.block_table.copy_(upd["block_table"])
             self.seq_lens.copy_(upd["seq_lens"])
             self.q.copy_(upd["q"])
-        da.da_append_kv(self.prob, upd["new_k"], upd["new_v"], self.block_table, self.seq_lens, self.k_cache,
-                        self.v_cache, self.status, stream=s)
+        if plan is None:
+            da.da_append_kv(self.prob, upd["new_k"], upd["new_v"], self.block_table, self.seq_lens, self.k_cache,
+                            self.v_cache, self.status, stream=s)
+        else:
+            desc, ws = plan
+            da.da_plan_append(self.prob, desc, self.seq_lens, ws, upd["new_k"], upd["new_v"], self.block_table,
+                              self.k_cache, self.v_cache, self.status, stream=s)
