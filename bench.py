@@ -10,8 +10,9 @@ the 126 MB L2, so consecutive steps cannot hit in L2.
 Printed (rank 0, one JSON line): KV-read GB/s of the whole step (value), the
 step time, the decode kernel's own achieved bandwidth against the measured HBM
 peak, the same step under the static split-k schedule (default and best split
-count), an end-to-end number (one da_decode_step_host call per step: host
-inputs copied in, the step, outputs copied back to host), the CPU oracle's rate
+count), an end-to-end number (one da_decode_step_host call per step from pinned
+host buffers: the plan launch reads lengths, block table and q over PCIe, and
+out/lse are written in place into host memory), the CPU oracle's rate
 on this machine's cores, and the SM clocks seen during the measurement.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference] [--config mixed]
@@ -311,7 +312,8 @@ def run_ours(args, world, rank, local):
             out_h = torch.empty(bufs.out.shape, dtype=bufs.out.dtype).pin_memory()
             lse_h = torch.empty(bufs.lse.shape, dtype=bufs.lse.dtype).pin_memory()
 
-            def e2e_step():  # one C call: copies in, plan, decode, combine, copies out
+            def e2e_step():  # one C call: the plan launch reads lengths, block table and q from the pinned
+                # host buffers; decode and combine write out / lse in place in pinned host memory
                 da.da_decode_step_host(prob, desc, q_h, bt_h, sl_h, dw.k_cache, dw.v_cache, dw.q, dw.block_table,
                                        dw.seq_lens, bufs, out_h, lse_h, k_scale=dw.k_scale, v_scale=dw.v_scale,
                                        stream=stream)
@@ -350,7 +352,9 @@ def run_ours(args, world, rank, local):
                   "algorithmic_bytes_per_launch": kv_bytes,
                   "launch_us": round(dec_avg_ms * 1e3, 2), "peak_source": peak_src, "traffic_source": traffic_note},
         e2e={"value": round(total_bytes / (ms_e2e / 1e3 / steps) / 1e9, 2), "unit": "GB/s",
-             "us_per_step": round(ms_e2e / steps * 1e3, 2), "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+             "us_per_step": round(ms_e2e / steps * 1e3, 2), "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+             "transfer": "da_decode_step_host with pinned host buffers: the plan launch reads seq_lens, block "
+                         "table and q over PCIe; decode and combine write out/lse in place over PCIe"},
         gpu_launches=3 * steps,
         device_status=status[0],
     )

@@ -269,15 +269,28 @@ DA_API int da_combine(const da_problem* prob, const da_plan_desc* desc, const vo
  *   k_scale and v_scale are NULL, FP8 E4M3 cache with per-KV-head scales when
  *   both are given); combine;
  *   copy out_dev, lse_dev to out_host, lse_host.
+ * Host buffers in page-locked memory mapped into the device's address space
+ * (every cudaHostAlloc / cudaMallocHost allocation under unified addressing,
+ * cudaHostRegister with cudaHostRegisterMapped) need no copy call:
+ *   - when seq_lens_host, block_table_host and q_host all are, the plan launch
+ *     brings them in itself: its first block reads the lengths over the bus,
+ *     writes seq_lens_dev and plans, while its other blocks copy the block
+ *     table into block_table_dev and, when q is at most 1 MiB, q into q_dev;
+ *     a larger q is read in place by the decode kernel (q_dev stays untouched),
+ *     which spreads its bus traffic over the K/V stream;
+ *   - out_host and lse_host, when mapped and 16-byte aligned, are written in
+ *     place by the decode and combine kernels (out_dev, lse_dev stay untouched).
  * The step computed is the one the separate calls compute (same plan, kernels
  * and results).
  *   q_host, block_table_host, seq_lens_host  host, layouts as in da_problem;
  *     read by the copies, so they must stay unchanged until the stream passes them.
  *   k_cache, v_cache, k_scale, v_scale       dev, as for da_decode_attention(_fp8).
  *   q_dev, block_table_dev, seq_lens_dev     dev, the caller's device copies of
- *     the three inputs (same sizes and alignment rules as for da_decode_attention).
+ *     the three inputs (same sizes and alignment rules as for da_decode_attention);
+ *     always written, whichever way the inputs move.
  *   ws, ws_bytes, partial_o, partial_lse     dev, as for da_plan / da_decode_attention.
- *   out_dev, lse_dev                         dev outputs, as for da_decode_attention.
+ *   out_dev, lse_dev                         dev outputs, as for da_decode_attention
+ *     (required; used when out_host / lse_host are not used in place).
  *   out_host, lse_host                       host, bf16 / fp32, same layouts as out, lse.
  * Host buffers should be page-locked (cudaHostAlloc / cudaHostRegister); with
  * pageable memory the copies are correct but may block the calling thread.

@@ -105,3 +105,84 @@ def test_host_step_multi_query():
     out_h, lse_h, _ = host_step(w)
     assert out_h.shape == (len(RAGGED), 2, 16, 128)
     check_mq_against_oracle(w, out_h, lse_h)
+
+
+def test_mapped_host_buffers_skip_the_copies():
+    """With pinned (mapped) host buffers the plan launch itself brings lengths, block table and q in,
+    and out / lse are written in place: the device outputs stay untouched, and the results equal the
+    copy path's (pageable buffers) bit for bit."""
+    w = ragged(seed=16)
+    out_p, lse_p, st = host_step(w, pinned=True)
+    dw, bufs = st["dw"], st["bufs"]
+    assert torch.equal(dw.q.cpu().view(torch.int16), w.q.view(torch.int16))  # copied by the plan launch
+    assert torch.equal(dw.seq_lens.cpu(), torch.from_numpy(w.seq_lens))
+    assert torch.equal(dw.block_table.cpu(), torch.from_numpy(w.block_table))
+    assert torch.isnan(bufs.out.float()).all() and torch.isnan(bufs.lse).all()  # never written
+    check_against_oracle(w, out_p, lse_p)
+    out_c, lse_c, st_c = host_step(w, pinned=False)
+    assert not torch.isnan(st_c["bufs"].lse).all()  # the copy path wrote the device outputs
+    assert torch.equal(out_p.view(torch.int16), out_c.view(torch.int16)) and torch.equal(lse_p, lse_c)
+
+
+def test_unaligned_pinned_views():
+    """q 8 bytes past a 16-byte boundary is brought in by 4-byte pieces; lse 4 bytes past one is not
+    written in place but copied back.  Same results."""
+    w = ragged(seed=17)
+    out_h, lse_h, st = host_step(w)
+    ref_out, ref_lse = out_h.clone(), lse_h.clone()
+    s = st
+    q_big = torch.empty(w.q.numel() + 8, dtype=torch.bfloat16).pin_memory()
+    q_off = q_big[4:4 + w.q.numel()].view(w.q.shape)
+    q_off.copy_(w.q)
+    lse_big = torch.full((s["lse_h"].numel() + 2,), float("nan")).pin_memory()
+    lse_off = lse_big[1:1 + s["lse_h"].numel()].view(s["lse_h"].shape)
+    s["q_h"], s["lse_h"] = q_off, lse_off
+    s["dw"].q.zero_()
+    s["bufs"].lse.fill_(float("nan"))
+    out2, lse2, _ = host_step(w, state=s)
+    assert torch.equal(s["dw"].q.cpu().view(torch.int16), w.q.view(torch.int16))
+    assert not torch.isnan(s["bufs"].lse).all()  # lse went through its device copy
+    assert torch.equal(out2.view(torch.int16), ref_out.view(torch.int16)) and torch.equal(lse2, ref_lse)
+
+
+@pytest.mark.parametrize("kind", [da.PLAN_DYNAMIC, da.PLAN_STATIC])
+def test_host_inputs_plan_matches_the_oracle_plan(kind, oracle_lib):
+    """The plan built from host lengths inside the input launch is the oracle's plan, for a batch
+    larger than one block's pass (600 requests) and with lengths changing between calls."""
+    import oracle
+    from gpu_helpers import assert_plan_equal
+    lens = np.random.default_rng(5).integers(0, 3000, 600).astype(np.int32)
+    w = W.make_workload("wide", lens.tolist(), num_q_heads=8, num_kv_heads=1, head_dim=64, page_size=64, seed=18,
+                        recipe="host-step plan test")
+    _, _, st = host_step(w, kind=kind)
+    cap = w.problem.max_pages_per_req * w.problem.page_size
+    for t in range(3):
+        cur = np.maximum(lens - 100 * t, 0).astype(np.int32)
+        out_h, lse_h, st = host_step(w, kind=kind, seq_lens=cur, state=st)
+        d = st["desc"]
+        got = da.read_plan(d, st["bufs"].ws)
+        want = (oracle.plan(cur, 64, d.num_ctas, cap) if kind == da.PLAN_DYNAMIC
+                else oracle.static_plan(cur, 64, d.splits, cap))
+        assert_plan_equal(got, want)
+        assert torch.equal(st["dw"].seq_lens.cpu(), torch.from_numpy(cur))
+    check_against_oracle(w, out_h, lse_h, seq_lens=cur)
+
+
+def test_large_q_is_read_in_place():
+    """A q above 1 MiB in mapped memory is read by the decode kernel over the bus (q_dev untouched);
+    lengths and block table still come in through the plan launch.  Same bits as the copy path."""
+    lens = np.random.default_rng(6).integers(0, 700, 160).astype(np.int32)
+    w = W.make_workload("big-q", lens.tolist(), num_q_heads=32, num_kv_heads=4, head_dim=128, page_size=64,
+                        seed=19, recipe="host-step large q")
+    assert w.q.numel() * 2 > (1 << 20)
+    for w8 in (None, W.quantize_fp8(w)):
+        base = w if w8 is None else w8.base
+        out_p, lse_p, st = host_step(base, w8=w8)
+        assert torch.count_nonzero(st["dw"].q) == 0  # never copied in
+        assert torch.equal(st["dw"].seq_lens.cpu(), torch.from_numpy(w.seq_lens))
+        if w8 is None:
+            check_against_oracle(w, out_p, lse_p)
+        else:
+            check_against_oracle_fp8(w8, out_p, lse_p)
+        out_c, lse_c, _ = host_step(base, w8=w8, pinned=False)
+        assert torch.equal(out_p.view(torch.int16), out_c.view(torch.int16)) and torch.equal(lse_p, lse_c)

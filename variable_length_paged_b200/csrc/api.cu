@@ -9,6 +9,7 @@
 
 #include "append_rows.cuh"
 #include "da_internal.cuh"
+#include "host_inputs.cuh"
 
 namespace {
 
@@ -393,6 +394,19 @@ DA_API int da_combine(const da_problem* prob, const da_plan_desc* desc, const vo
   return rc != DA_OK ? rc : combine_launch(p, desc, prob->head_dim, stream);
 }
 
+// The device address of host memory that kernels may use in place (page-locked and mapped
+// into this device's address space), aligned to `align` bytes; nullptr for any other memory.
+static void* mapped_host(const void* ptr, size_t align) {
+  cudaPointerAttributes a;
+  if (cudaPointerGetAttributes(&a, ptr) != cudaSuccess) {
+    (void)cudaGetLastError();  // not a pointer the runtime knows: plain host memory
+    return nullptr;
+  }
+  if (a.type != cudaMemoryTypeHost || a.devicePointer == nullptr) return nullptr;
+  if (reinterpret_cast<uintptr_t>(a.devicePointer) % align != 0) return nullptr;
+  return a.devicePointer;
+}
+
 DA_API int da_decode_step_host(const da_problem* prob, const da_plan_desc* desc, const void* q_host,
                                const int32_t* block_table_host, const int32_t* seq_lens_host, const void* k_cache,
                                const void* v_cache, const float* k_scale, const float* v_scale, void* q_dev,
@@ -408,36 +422,74 @@ DA_API int da_decode_step_host(const da_problem* prob, const da_plan_desc* desc,
   if (fp8 && prob->head_dim != 128) return DA_ERR_UNSUPPORTED;
   if (prob->batch == 0) return DA_OK;
   if (!q_host || !block_table_host || !seq_lens_host || !out_host || !lse_host) return DA_ERR_INVALID_ARG;
+  if (!q_dev || !out_dev || !lse_dev) return DA_ERR_INVALID_ARG;  // required whichever way q, out, lse move
+  const size_t B = (size_t)prob->batch;
+  const size_t rows = B * (size_t)q_len_of(prob) * (size_t)prob->num_q_heads;
+  const size_t q_bytes = rows * (size_t)prob->head_dim * 2;
+  const size_t bt_bytes = B * (size_t)prob->max_pages_per_req * 4;
+  // Inputs in mapped page-locked memory need no copy call.  The plan launch brings them in:
+  // block 0 reads the lengths and plans, the other blocks copy the block table and a small q
+  // (up to kQInLaunch bytes: the bus moves it within the launch).  A larger q is read in place
+  // by the decode kernel, which spreads the bus traffic over the K/V stream.  out and lse in
+  // mapped memory are written in place by the decode and combine kernels.  Anything else goes
+  // through copies on the stream.
+  constexpr size_t kQInLaunch = size_t(1) << 20;
+  const int32_t* sl_map = static_cast<const int32_t*>(mapped_host(seq_lens_host, 4));
+  const void* bt_map = mapped_host(block_table_host, 4);
+  const void* q_map = mapped_host(q_host, fp8 ? 8 : 4);
+  const bool in_launch = sl_map && bt_map && q_map;
+  const bool q_in_place = in_launch && q_bytes > kQInLaunch;
+  void* out_map = mapped_host(out_host, 16);
+  float* lse_map = static_cast<float*>(mapped_host(lse_host, 16));
+  void* out_use = out_map ? out_map : out_dev;
+  float* lse_use = lse_map ? lse_map : lse_dev;
   // every check of the three device calls runs before the first copy is enqueued
   da::PlanParams pp;
   rc = plan_prepare(prob, desc, seq_lens_dev, ws, ws_bytes, desc->kind, &pp);
   if (rc != DA_OK) return rc;
   da::DecodeParams dp;
   CUtensorMap maps[4];
-  rc = decode_prepare(prob, desc, q_dev, k_cache, v_cache, k_scale, v_scale, block_table_dev, seq_lens_dev, ws,
-                      partial_o, partial_lse, out_dev, lse_dev, fp8, &dp, maps);
+  rc = decode_prepare(prob, desc, q_in_place ? q_map : q_dev, k_cache, v_cache, k_scale, v_scale, block_table_dev,
+                      seq_lens_dev, ws, partial_o, partial_lse, out_use, lse_use, fp8, &dp, maps);
   if (rc != DA_OK) return rc;
   da::CombineParams cp;
-  rc = combine_prepare(prob, desc, ws, partial_o, partial_lse, out_dev, lse_dev, &cp);
+  rc = combine_prepare(prob, desc, ws, partial_o, partial_lse, out_use, lse_use, &cp);
   if (rc != DA_OK) return rc;
 
   const cudaStream_t s = static_cast<cudaStream_t>(stream);
-  const size_t B = (size_t)prob->batch;
-  const size_t rows = B * (size_t)q_len_of(prob) * (size_t)prob->num_q_heads;
-  const size_t q_bytes = rows * (size_t)prob->head_dim * 2;
-  const size_t bt_bytes = B * (size_t)prob->max_pages_per_req * 4;
-  cudaError_t e = cudaMemcpyAsync(seq_lens_dev, seq_lens_host, B * 4, cudaMemcpyHostToDevice, s);
-  if (e == cudaSuccess) e = cudaMemcpyAsync(block_table_dev, block_table_host, bt_bytes, cudaMemcpyHostToDevice, s);
-  if (e == cudaSuccess) e = cudaMemcpyAsync(q_dev, q_host, q_bytes, cudaMemcpyHostToDevice, s);
-  if (e != cudaSuccess) return cuda_fail(e);
-  rc = plan_launch(pp, desc->kind, stream);
-  if (rc != DA_OK) return rc;
+  cudaError_t e = cudaSuccess;
+  if (in_launch) {
+    da::HostInputs hi{};
+    hi.seq_lens_dev = seq_lens_dev;
+    const void* src[2] = {bt_map, q_map};
+    void* dst[2] = {block_table_dev, q_dev};
+    const size_t bytes[2] = {bt_bytes, q_bytes};
+    for (int k = 0; k < 2; ++k) {
+      const bool wide = (reinterpret_cast<uintptr_t>(src[k]) | reinterpret_cast<uintptr_t>(dst[k])) % 16 == 0;
+      hi.copies[k].src = src[k];
+      hi.copies[k].dst = dst[k];
+      hi.copies[k].n16 = wide ? (int64_t)(bytes[k] / 16) : 0;
+      hi.copies[k].n4 = (int64_t)((bytes[k] - 16 * (size_t)hi.copies[k].n16) / 4);
+    }
+    hi.num_copies = q_in_place ? 1 : 2;
+    pp.seq_lens = sl_map;  // the planner reads the host lengths; the device copy is for the decode
+    e = da::launch_plan_host(pp, desc->kind, hi, s);
+    if (e != cudaSuccess) return cuda_fail(e);
+  } else {
+    e = cudaMemcpyAsync(seq_lens_dev, seq_lens_host, B * 4, cudaMemcpyHostToDevice, s);
+    if (e == cudaSuccess) e = cudaMemcpyAsync(block_table_dev, block_table_host, bt_bytes, cudaMemcpyHostToDevice, s);
+    if (e == cudaSuccess) e = cudaMemcpyAsync(q_dev, q_host, q_bytes, cudaMemcpyHostToDevice, s);
+    if (e != cudaSuccess) return cuda_fail(e);
+    rc = plan_launch(pp, desc->kind, stream);
+    if (rc != DA_OK) return rc;
+  }
   rc = decode_launch(dp, prob->head_dim, maps, fp8, stream);
   if (rc != DA_OK) return rc;
   rc = combine_launch(cp, desc, prob->head_dim, stream);
   if (rc != DA_OK) return rc;
-  e = cudaMemcpyAsync(out_host, out_dev, q_bytes, cudaMemcpyDeviceToHost, s);
-  if (e == cudaSuccess) e = cudaMemcpyAsync(lse_host, lse_dev, rows * 4, cudaMemcpyDeviceToHost, s);
+  e = cudaSuccess;
+  if (!out_map) e = cudaMemcpyAsync(out_host, out_dev, q_bytes, cudaMemcpyDeviceToHost, s);
+  if (e == cudaSuccess && !lse_map) e = cudaMemcpyAsync(lse_host, lse_dev, rows * 4, cudaMemcpyDeviceToHost, s);
   return e == cudaSuccess ? DA_OK : cuda_fail(e);
 }
 

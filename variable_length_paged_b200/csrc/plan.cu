@@ -10,10 +10,12 @@
 // segments {request, cta, tile_begin, tile_end} in global tile order, the
 // per-request and per-CTA segment ranges, and a header.  Everything is integer
 // arithmetic, so the result is bit-exact and independent of thread timing.
+#include <algorithm>
 #include <climits>
 
 #include "append_rows.cuh"
 #include "da_internal.cuh"
+#include "host_inputs.cuh"
 
 namespace da {
 namespace {
@@ -45,8 +47,10 @@ __device__ int block_exclusive_scan(int v, int* total, int* warp_buf) {
 }
 
 // Tile count of one request; an out-of-range length counts as 0 and is reported.
-__device__ int request_tiles(const PlanParams& p, int b, int* s_bad) {
+// With `sl_copy`, the length read is also written there (lengths read from host memory).
+__device__ int request_tiles(const PlanParams& p, int b, int* s_bad, int32_t* sl_copy) {
   const int L = p.seq_lens[b];
+  if (sl_copy) sl_copy[b] = L;
   if (L < 0 || (int64_t)L > p.capacity_tokens) {
     atomicMin(s_bad, b);
     return 0;
@@ -60,11 +64,11 @@ constexpr int kSmemBatch = 4096;
 
 // Phase shared by both planners: req_tile_prefix and U (and the largest n_b).
 __device__ void tile_prefix(const PlanParams& p, int32_t* rtp, int32_t* s_rtp, int* warp_buf, int* s_bad, int* U,
-                            int* max_tiles) {
+                            int* max_tiles, int32_t* sl_copy) {
   int carry = 0, mx = 0;
   for (int base = 0; base < p.batch; base += kPlanThreads) {
     const int b = base + threadIdx.x;
-    const int n = b < p.batch ? request_tiles(p, b, s_bad) : 0;
+    const int n = b < p.batch ? request_tiles(p, b, s_bad, sl_copy) : 0;
     int total;
     const int excl = block_exclusive_scan(n, &total, warp_buf);
     if (b < p.batch) {
@@ -133,7 +137,7 @@ __device__ __forceinline__ int last_not_above(const int32_t* a, int n, int64_t x
 }
 
 // The dynamic plan, computed by one block of kPlanThreads threads.
-__device__ void plan_dynamic_body(const PlanParams& p) {
+__device__ void plan_dynamic_body(const PlanParams& p, int32_t* sl_copy = nullptr) {
   __shared__ int warp_buf[32];
   __shared__ int s_bad;
   __shared__ int32_t s_rtp[kSmemBatch + 1], s_rsb[kSmemBatch + 1];
@@ -154,7 +158,7 @@ __device__ void plan_dynamic_body(const PlanParams& p) {
   const int64_t C = p.num_ctas;
 
   int U;
-  tile_prefix(p, rtp, small ? s_rtp : nullptr, warp_buf, &s_bad, &U, nullptr);
+  tile_prefix(p, rtp, small ? s_rtp : nullptr, warp_buf, &s_bad, &U, nullptr, sl_copy);
   const Split sp(U, C);
 
   // Segments per request.  With U >= C every CTA owns at least one tile, so a
@@ -235,12 +239,11 @@ __global__ void __launch_bounds__(kPlanThreads) plan_append_kernel(const PlanPar
   }
 }
 
-__global__ void __launch_bounds__(kPlanThreads) plan_static_kernel(const PlanParams p) {
+// The static split-k plan, computed by one block of kPlanThreads threads.
+__device__ void plan_static_body(const PlanParams& p, int32_t* sl_copy = nullptr) {
   __shared__ int warp_buf[32];
   __shared__ int s_bad;
   __shared__ int32_t s_rtp[kSmemBatch + 1];
-  grid_dependency_wait();
-  grid_dependents_launch();
   if (threadIdx.x == 0) s_bad = INT_MAX;
   __syncthreads();
 
@@ -257,7 +260,7 @@ __global__ void __launch_bounds__(kPlanThreads) plan_static_kernel(const PlanPar
   const int S = p.width;
 
   int U, max_tiles;
-  tile_prefix(p, rtp, small ? s_rtp : nullptr, warp_buf, &s_bad, &U, &max_tiles);
+  tile_prefix(p, rtp, small ? s_rtp : nullptr, warp_buf, &s_bad, &U, &max_tiles, sl_copy);
   const int chunk = (max_tiles + S - 1) / S;
   const int total = p.batch * S;
   for (int i = threadIdx.x; i < total; i += kPlanThreads) {
@@ -269,6 +272,53 @@ __global__ void __launch_bounds__(kPlanThreads) plan_static_kernel(const PlanPar
   for (int b = threadIdx.x; b <= p.batch; b += kPlanThreads) rsb[b] = b * S;
   for (int c = threadIdx.x; c <= total; c += kPlanThreads) csb[c] = c;
   if (threadIdx.x == 0) write_header(p, hdr, U, total, DA_PLAN_STATIC, S, s_bad);
+}
+
+__global__ void __launch_bounds__(kPlanThreads) plan_static_kernel(const PlanParams p) {
+  grid_dependency_wait();
+  grid_dependents_launch();
+  plan_static_body(p);
+}
+
+// Copy units [first, n) with stride `stride`, four loads in flight per thread (host
+// memory is a bus round trip away).
+template <typename T>
+__device__ __forceinline__ void strided_copy(const T* src, T* dst, int64_t n, int64_t first, int64_t stride) {
+  int64_t i = first;
+  for (; i + 3 * stride < n; i += 4 * stride) {
+    const T a = src[i], b = src[i + stride], c = src[i + 2 * stride], d = src[i + 3 * stride];
+    dst[i] = a;
+    dst[i + stride] = b;
+    dst[i + 2 * stride] = c;
+    dst[i + 3 * stride] = d;
+  }
+  for (; i < n; i += stride) dst[i] = src[i];
+}
+
+// One launch brings the step's inputs in from mapped host memory and plans: block 0
+// reads the lengths from the host, writes their device copy and plans; the other
+// blocks copy the block table and q.  The decode kernel waits for the whole grid.
+template <int kKind>
+__global__ void __launch_bounds__(kPlanThreads) plan_host_kernel(const PlanParams p, const HostInputs h) {
+  grid_dependency_wait();  // the previous step's kernels may still read the device copies
+  grid_dependents_launch();
+  if (blockIdx.x == 0) {
+    if constexpr (kKind == DA_PLAN_DYNAMIC)
+      plan_dynamic_body(p, h.seq_lens_dev);
+    else
+      plan_static_body(p, h.seq_lens_dev);
+    return;
+  }
+  const int64_t first = (int64_t)(blockIdx.x - 1) * kPlanThreads + threadIdx.x;
+  const int64_t stride = (int64_t)(gridDim.x - 1) * kPlanThreads;
+#pragma unroll
+  for (int k = 0; k < 2; ++k) {
+    if (k >= h.num_copies) break;
+    const HostCopy& c = h.copies[k];
+    strided_copy(static_cast<const int4*>(c.src), static_cast<int4*>(c.dst), c.n16, first, stride);
+    strided_copy(reinterpret_cast<const int32_t*>(static_cast<const int4*>(c.src) + c.n16),
+                 reinterpret_cast<int32_t*>(static_cast<int4*>(c.dst) + c.n16), c.n4, first, stride);
+  }
 }
 
 }  // namespace
@@ -295,6 +345,24 @@ cudaError_t launch_plan_dynamic(const PlanParams& p, cudaStream_t stream) {
 
 cudaError_t launch_plan_static(const PlanParams& p, cudaStream_t stream) {
   return launch_planner(plan_static_kernel, p, stream);
+}
+
+cudaError_t launch_plan_host(const PlanParams& p, int kind, const HostInputs& h, cudaStream_t stream) {
+  int64_t units = 0;
+  for (int k = 0; k < h.num_copies; ++k) units = max(units, h.copies[k].n16 + h.copies[k].n4);
+  const int64_t per_pass = 4 * kPlanThreads;  // units one block moves with four loads in flight
+  const int blocks = (int)std::min<int64_t>(147, (units + per_pass - 1) / per_pass);
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(1 + (unsigned)std::max(blocks, 1), 1, 1);
+  cfg.blockDim = dim3(kPlanThreads, 1, 1);
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  if (kind == DA_PLAN_DYNAMIC) return cudaLaunchKernelEx(&cfg, plan_host_kernel<DA_PLAN_DYNAMIC>, p, h);
+  return cudaLaunchKernelEx(&cfg, plan_host_kernel<DA_PLAN_STATIC>, p, h);
 }
 
 cudaError_t launch_plan_append(const PlanParams& p, const AppendParams& a, cudaStream_t stream) {
