@@ -31,7 +31,9 @@
 // fp32 state (O and the weight sums) is rescaled to each chunk's reference.
 //
 // Warps: 0-3 softmax (thread t = token t of a chunk for S, dim t for O; warp w
-// reads TMEM lanes 32w..32w+31), 4 TMA producer, 5 MMA issuer (one thread).
+// reads TMEM lanes 32w..32w+31; thread 0 issues each chunk's P.V as soon as the
+// four warps have written its weights), 4 TMA producer, 5 score-MMA issuer (one
+// thread).
 // TMEM: 64 columns = S[2] and O[2] (16 fp32 columns each), double buffered so
 // the tensor core computes chunk i+1's scores while the softmax warps work on
 // chunk i.  The q tile is double buffered too: segment j+1's tile is written when
@@ -67,9 +69,10 @@ constexpr int kOffP = kOffQ8 + 2 * 2048;         // [2][128 tokens][16 B]
 constexpr int kOffRed = kOffP + 2 * 2048;        // [2][4 warps][8] floats
 constexpr int kOffRowScale = kOffRed + 2 * 32 * 4;  // [2][8] floats
 constexpr int kOffBars = kOffRowScale + 2 * 8 * 4;
-// mbarriers: full[3], empty[3], s_full[2], s_free[2], p_full[2], o_full[2], o_free[2], q_full[2], done
-constexpr int kBarFull = 0, kBarEmpty = 3, kBarSFull = 6, kBarSFree = 8, kBarPFull = 10, kBarOFull = 12,
-              kBarOFree = 14, kBarQFull = 16, kBarDone = 18, kNumBars = 19;
+// mbarriers: full[3], empty[3], s_full[2], s_free[2], o_full[2], q_full[2], done (MMA thread), done_pv
+// (softmax thread 0, which issues P.V)
+constexpr int kBarFull = 0, kBarEmpty = 3, kBarSFull = 6, kBarSFree = 8, kBarOFull = 10, kBarQFull = 12,
+              kBarDone = 14, kBarDonePV = 15, kNumBars = 16;
 constexpr int kOffMeta = kOffBars + kNumBars * 8;  // loaded tokens per stage
 constexpr int kOffFlags = kOffMeta + kStagesTc * 4;  // abort flag, TMEM base address
 constexpr int kBytesTc = kOffFlags + 16;
@@ -258,13 +261,12 @@ __global__ void __launch_bounds__(kThreadsTc, 2)
     for (int j = 0; j < 2; ++j) {
       mbar_init(bar(kBarSFull + j), 1);
       mbar_init(bar(kBarSFree + j), kSoftmaxWarps);
-      mbar_init(bar(kBarPFull + j), kSoftmaxWarps);
       mbar_init(bar(kBarOFull + j), 1);
-      mbar_init(bar(kBarOFree + j), kSoftmaxWarps);
     }
     mbar_init(bar(kBarQFull), kSoftmaxWarps);
     mbar_init(bar(kBarQFull + 1), kSoftmaxWarps);
     mbar_init(bar(kBarDone), 1);
+    mbar_init(bar(kBarDonePV), 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -404,10 +406,10 @@ __global__ void __launch_bounds__(kThreadsTc, 2)
     }
   } else if (warp == kMmaWarp) {
     // ------------------------------------------------------------------ MMA issuer
-    // One thread issues, in whatever order the inputs become ready: P.V of chunk
-    // ip as soon as its weights are written (it frees the chunk's stage for the
-    // producer), S of chunk is as soon as its K/V have landed and its score
-    // buffer is free.  Chunk ic sits in stage ic % kStagesTc, S and O buffers ic % 2.
+    // One thread issues the score MMAs: S of chunk is as soon as its K/V have landed, the
+    // q tile of its segment is written and its score buffer is free.  (P.V is issued by the
+    // softmax warps themselves, the moment their weights are written.)  Chunk ic sits in
+    // stage ic % kStagesTc, S buffer ic % 2.
     if (lane == 0) {
       bool aborted = false;
       auto fail = [&](int s) {
@@ -433,44 +435,26 @@ __global__ void __launch_bounds__(kThreadsTc, 2)
         return false;
       };
       bool more = next_segment();  // chunks left whose S is not issued
-      int is = 0, ip = 0;
+      int is = 0;
       uint64_t t_last = global_timer_ns();
-      for (uint32_t it = 0; !aborted && (more || ip < is); ++it) {
+      for (uint32_t it = 0; !aborted && more; ++it) {
         bool progressed = false;
-        if (ip < is) {  // O^T (chunk ic) = V^T . P'^T, then release the stage
-          const int ic = ip, ob = ic & 1, st = ic % kStagesTc;
-          if (mbar_test(bar(kBarPFull + ob), (ic >> 1) & 1) &&
-              (ic < 2 || mbar_test(bar(kBarOFree + ob), ((ic >> 1) - 1) & 1))) {
-            tc_fence_after();
-            const uint32_t vt = sbase + kOffStages + st * kStageBytes + kTileBytes;
-            const uint32_t pt = sbase + kOffP + ob * 2048;
+        // S^T (chunk ic) = K . Q8^T, with the q tile of the chunk's segment
+        if (!q_ready) q_ready = mbar_test(bar(kBarQFull + (s_js & 1)), (s_js >> 1) & 1);
+        const int ic = is, sb = ic & 1, st = ic % kStagesTc;
+        if (q_ready && mbar_test(bar(kBarFull + st), (ic / kStagesTc) & 1) &&
+            (ic < 2 || mbar_test(bar(kBarSFree + sb), ((ic >> 1) - 1) & 1))) {
+          tc_fence_after();
+          const uint32_t kt = sbase + kOffStages + st * kStageBytes;
+          const uint32_t q8 = sbase + kOffQ8 + (s_js & 1) * 2048;
 #pragma unroll
-            for (int j = 0; j < 4; ++j)
-              tc_mma(tmem + 32 + 16 * ob, smem_desc(vt + 4096 * j, 1024, 1024, 2),
-                     smem_desc(pt + 512 * j, 128, 128, 0), kIdescPV, j > 0);
-            tc_commit(bar(kBarOFull + ob));
-            tc_commit(bar(kBarEmpty + st));
-            ++ip;
-            progressed = true;
-          }
-        }
-        if (more) {  // S^T (chunk ic) = K . Q8^T, with the q tile of the chunk's segment
-          if (!q_ready) q_ready = mbar_test(bar(kBarQFull + (s_js & 1)), (s_js >> 1) & 1);
-          const int ic = is, sb = ic & 1, st = ic % kStagesTc;
-          if (q_ready && mbar_test(bar(kBarFull + st), (ic / kStagesTc) & 1) &&
-              (ic < 2 || mbar_test(bar(kBarSFree + sb), ((ic >> 1) - 1) & 1))) {
-            tc_fence_after();
-            const uint32_t kt = sbase + kOffStages + st * kStageBytes;
-            const uint32_t q8 = sbase + kOffQ8 + (s_js & 1) * 2048;
-#pragma unroll
-            for (int j = 0; j < 4; ++j)
-              tc_mma(tmem + 16 * sb, smem_desc(kt + 32 * j, 16, 1024, 2), smem_desc(q8 + 32 * j, 16, 1024, 2),
-                     kIdescS, j > 0);
-            tc_commit(bar(kBarSFull + sb));
-            ++is;
-            progressed = true;
-            if (is == s_end) more = next_segment();
-          }
+          for (int j = 0; j < 4; ++j)
+            tc_mma(tmem + 16 * sb, smem_desc(kt + 32 * j, 16, 1024, 2), smem_desc(q8 + 32 * j, 16, 1024, 2),
+                   kIdescS, j > 0);
+          tc_commit(bar(kBarSFull + sb));
+          ++is;
+          progressed = true;
+          if (is == s_end) more = next_segment();
         }
         if (progressed) {
           t_last = global_timer_ns();
@@ -558,6 +542,7 @@ __global__ void __launch_bounds__(kThreadsTc, 2)
       return -1;
     };
     int js = 0;  // segments with chunks seen so far (same count as the MMA thread's)
+    bool pv_issued = false;  // thread 0 has issued P.V MMAs (to drain before TMEM is freed)
     for (int s = seg_lo; s < seg_hi; ++s) {
       const SegmentInfo si = load_segment(p, segs, s);
       if (!si.valid) continue;
@@ -594,8 +579,6 @@ __global__ void __launch_bounds__(kThreadsTc, 2)
 #pragma unroll
             for (int j = 0; j < 16; ++j) o[j] = 0u;
           }
-          __syncwarp();
-          if (lane == 0) mbar_arrive(bar(kBarOFree + ob));
 #pragma unroll
           for (int h = 0; h < 8; ++h)
             o_acc[h] = o_acc[h] * f[h] + (__uint_as_float(o[h]) + __uint_as_float(o[8 + h]));
@@ -611,7 +594,9 @@ __global__ void __launch_bounds__(kThreadsTc, 2)
             for (int c = 0; c < 8; ++c) vrow[c] = make_uint4(0, 0, 0, 0);
           }
           uint32_t sr[16];
-          if (wait(bar(kBarSFull + sb), (i >> 1) & 1, s)) {
+          const bool s_ok = wait(bar(kBarSFull + sb), (i >> 1) & 1, s);
+          const bool pv_ok = landed && s_ok;  // thread 0's view decides whether P.V is issued
+          if (s_ok) {
             tc_fence_after();
             tc_ld16(lane_base + 16 * sb, sr);
             tc_fence_before();
@@ -644,8 +629,23 @@ __global__ void __launch_bounds__(kThreadsTc, 2)
           *reinterpret_cast<uint4*>(smem + kOffP + sb * 2048 + 16 * t) =
               make_uint4(ph[0] | (ph[1] << 16), ph[2] | (ph[3] << 16), pl[0] | (pl[1] << 16), pl[2] | (pl[3] << 16));
           fence_proxy_async_smem();  // P' and the zeroed V rows are read by the tensor core
-          __syncwarp();
-          if (lane == 0) mbar_arrive(bar(kBarPFull + sb));
+          // O^T (chunk i) = V^T . P'^T, issued by thread 0 once all four warps have written their
+          // weights; O buffer sb was last read by the fold of chunk i - 2, which every softmax
+          // thread finished (tcgen05.wait::ld, fence) before this barrier.  The commits hand O to
+          // the fold and the stage back to the producer.
+          named_barrier_sync(1, kSoftmaxWarps * 32);
+          if (t == 0 && pv_ok) {
+            tc_fence_after();
+            const uint32_t vt = sbase + kOffStages + stage * kStageBytes + kTileBytes;
+            const uint32_t pt = sbase + kOffP + sb * 2048;
+#pragma unroll
+            for (int j = 0; j < 4; ++j)
+              tc_mma(tmem + 32 + 16 * sb, smem_desc(vt + 4096 * j, 1024, 1024, 2), smem_desc(pt + 512 * j, 128, 128, 0),
+                     kIdescPV, j > 0);
+            tc_commit(bar(kBarOFull + sb));
+            tc_commit(bar(kBarEmpty + stage));
+            pv_issued = true;
+          }
           if (k > 0) fold(i - 1, f_prev);
 #pragma unroll
           for (int h = 0; h < 8; ++h) f_prev[h] = f[h];
@@ -678,6 +678,11 @@ __global__ void __launch_bounds__(kThreadsTc, 2)
             p.partial_lse[(int64_t)s * p.num_q_heads + row] = lse;
         }
       }
+    }
+    // drain: thread 0's P.V MMAs have completed before TMEM is freed and the stages' barriers die
+    if (t == 0 && pv_issued) {
+      tc_commit(bar(kBarDonePV));
+      mbar_wait_timeout(bar(kBarDonePV), 0, p.wait_limit_ns);
     }
   }
 
