@@ -460,6 +460,7 @@ DA_API int da_decode_step_host(const da_problem* prob, const da_plan_desc* desc,
   cudaError_t e = cudaSuccess;
   if (in_launch) {
     da::HostInputs hi{};
+    hi.seq_lens_host = sl_map;
     hi.seq_lens_dev = seq_lens_dev;
     const void* src[2] = {bt_map, q_map};
     void* dst[2] = {block_table_dev, q_dev};
@@ -472,7 +473,6 @@ DA_API int da_decode_step_host(const da_problem* prob, const da_plan_desc* desc,
       hi.copies[k].n4 = (int64_t)((bytes[k] - 16 * (size_t)hi.copies[k].n16) / 4);
     }
     hi.num_copies = q_in_place ? 1 : 2;
-    pp.seq_lens = sl_map;  // the planner reads the host lengths; the device copy is for the decode
     e = da::launch_plan_host(pp, desc->kind, hi, s);
     if (e != cudaSuccess) return cuda_fail(e);
   } else {

@@ -16,10 +16,11 @@ struct HostCopy {
   int64_t n4;
 };
 
-// The plan reads the lengths from PlanParams::seq_lens (host) and writes them
-// to seq_lens_dev for the kernels that follow; the other blocks of the launch
-// run `copies` (block table, q).
+// The plan's block copies the lengths from seq_lens_host (the device address of
+// mapped host memory) to seq_lens_dev and plans from that copy; the other blocks
+// of the launch run `copies` (block table, q).
 struct HostInputs {
+  const int32_t* seq_lens_host;
   int32_t* seq_lens_dev;
   HostCopy copies[2];
   int num_copies;

@@ -47,10 +47,8 @@ __device__ int block_exclusive_scan(int v, int* total, int* warp_buf) {
 }
 
 // Tile count of one request; an out-of-range length counts as 0 and is reported.
-// With `sl_copy`, the length read is also written there (lengths read from host memory).
-__device__ int request_tiles(const PlanParams& p, int b, int* s_bad, int32_t* sl_copy) {
+__device__ int request_tiles(const PlanParams& p, int b, int* s_bad) {
   const int L = p.seq_lens[b];
-  if (sl_copy) sl_copy[b] = L;
   if (L < 0 || (int64_t)L > p.capacity_tokens) {
     atomicMin(s_bad, b);
     return 0;
@@ -64,11 +62,11 @@ constexpr int kSmemBatch = 4096;
 
 // Phase shared by both planners: req_tile_prefix and U (and the largest n_b).
 __device__ void tile_prefix(const PlanParams& p, int32_t* rtp, int32_t* s_rtp, int* warp_buf, int* s_bad, int* U,
-                            int* max_tiles, int32_t* sl_copy) {
+                            int* max_tiles) {
   int carry = 0, mx = 0;
   for (int base = 0; base < p.batch; base += kPlanThreads) {
     const int b = base + threadIdx.x;
-    const int n = b < p.batch ? request_tiles(p, b, s_bad, sl_copy) : 0;
+    const int n = b < p.batch ? request_tiles(p, b, s_bad) : 0;
     int total;
     const int excl = block_exclusive_scan(n, &total, warp_buf);
     if (b < p.batch) {
@@ -137,7 +135,7 @@ __device__ __forceinline__ int last_not_above(const int32_t* a, int n, int64_t x
 }
 
 // The dynamic plan, computed by one block of kPlanThreads threads.
-__device__ void plan_dynamic_body(const PlanParams& p, int32_t* sl_copy = nullptr) {
+__device__ void plan_dynamic_body(const PlanParams& p) {
   __shared__ int warp_buf[32];
   __shared__ int s_bad;
   __shared__ int32_t s_rtp[kSmemBatch + 1], s_rsb[kSmemBatch + 1];
@@ -158,7 +156,7 @@ __device__ void plan_dynamic_body(const PlanParams& p, int32_t* sl_copy = nullpt
   const int64_t C = p.num_ctas;
 
   int U;
-  tile_prefix(p, rtp, small ? s_rtp : nullptr, warp_buf, &s_bad, &U, nullptr, sl_copy);
+  tile_prefix(p, rtp, small ? s_rtp : nullptr, warp_buf, &s_bad, &U, nullptr);
   const Split sp(U, C);
 
   // Segments per request.  With U >= C every CTA owns at least one tile, so a
@@ -240,7 +238,7 @@ __global__ void __launch_bounds__(kPlanThreads) plan_append_kernel(const PlanPar
 }
 
 // The static split-k plan, computed by one block of kPlanThreads threads.
-__device__ void plan_static_body(const PlanParams& p, int32_t* sl_copy = nullptr) {
+__device__ void plan_static_body(const PlanParams& p) {
   __shared__ int warp_buf[32];
   __shared__ int s_bad;
   __shared__ int32_t s_rtp[kSmemBatch + 1];
@@ -260,7 +258,7 @@ __device__ void plan_static_body(const PlanParams& p, int32_t* sl_copy = nullptr
   const int S = p.width;
 
   int U, max_tiles;
-  tile_prefix(p, rtp, small ? s_rtp : nullptr, warp_buf, &s_bad, &U, &max_tiles, sl_copy);
+  tile_prefix(p, rtp, small ? s_rtp : nullptr, warp_buf, &s_bad, &U, &max_tiles);
   const int chunk = (max_tiles + S - 1) / S;
   const int total = p.batch * S;
   for (int i = threadIdx.x; i < total; i += kPlanThreads) {
@@ -296,17 +294,22 @@ __device__ __forceinline__ void strided_copy(const T* src, T* dst, int64_t n, in
 }
 
 // One launch brings the step's inputs in from mapped host memory and plans: block 0
-// reads the lengths from the host, writes their device copy and plans; the other
-// blocks copy the block table and q.  The decode kernel waits for the whole grid.
+// copies the lengths to the device (all its loads in flight at once) and plans from
+// that copy; the other blocks copy the block table and q.  The decode kernel waits for
+// the whole grid.
 template <int kKind>
 __global__ void __launch_bounds__(kPlanThreads) plan_host_kernel(const PlanParams p, const HostInputs h) {
   grid_dependency_wait();  // the previous step's kernels may still read the device copies
   grid_dependents_launch();
   if (blockIdx.x == 0) {
+    strided_copy(h.seq_lens_host, h.seq_lens_dev, (int64_t)p.batch, (int64_t)threadIdx.x, (int64_t)kPlanThreads);
+    __syncthreads();  // the block's own global writes are visible to it after the barrier
+    PlanParams pd = p;
+    pd.seq_lens = h.seq_lens_dev;
     if constexpr (kKind == DA_PLAN_DYNAMIC)
-      plan_dynamic_body(p, h.seq_lens_dev);
+      plan_dynamic_body(pd);
     else
-      plan_static_body(p, h.seq_lens_dev);
+      plan_static_body(pd);
     return;
   }
   const int64_t first = (int64_t)(blockIdx.x - 1) * kPlanThreads + threadIdx.x;
