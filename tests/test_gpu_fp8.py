@@ -108,3 +108,45 @@ def test_fp8_zero_query_long_request(da_lib, oracle_lib):
     out, lse, *_ = run_step_fp8(w8, width=5)
     check_against_oracle_fp8(w8, out, lse)
     assert np.allclose(lse.cpu().numpy(), np.log(np.array([30000, 17], np.float64))[:, None], atol=1e-4)
+
+
+def test_fp8_shared_prefix_pages(da_lib, oracle_lib):
+    """Two requests whose block tables name the same pages (a shared prefix) on the tensor-core path."""
+    w = W.make_workload("small", [900, 900, 300], num_q_heads=8, num_kv_heads=1, head_dim=128, page_size=64,
+                        seed=8)
+    bt = w.block_table.copy()
+    bt[1, :10] = bt[0, :10]  # request 1 shares the first 640 tokens of request 0
+    w.block_table = bt
+    w8 = W.quantize_fp8(w)
+    out, lse, *_ = run_step_fp8(w8, width=7)
+    check_against_oracle_fp8(w8, out, lse)
+
+
+def test_fp8_lengths_change_inside_one_graph(da_lib, oracle_lib):
+    """One captured FP8 step serves requests that grow, finish and restart (lengths edited in device
+    memory only); every replay matches the oracle at its lengths."""
+    import dataclasses
+    w = W.make_workload("small", [3800, 3800, 3800, 3800], num_q_heads=16, num_kv_heads=2, head_dim=128,
+                        page_size=64, seed=21, max_pages_per_req=60)
+    w8 = W.quantize_fp8(w)
+    dw = w8.to("cuda")
+    prob = da.problem_from(dw.problem)
+    desc = da.da_plan_desc_init(prob, da.PLAN_DYNAMIC, 64, 37)
+    bufs = da.Buffers(prob, desc, "cuda")
+    step = lambda: da.decode_step(prob, desc, dw.q, dw.k_cache, dw.v_cache, dw.block_table, dw.seq_lens, bufs,
+                                  k_scale=dw.k_scale, v_scale=dw.v_scale)
+    dw.seq_lens.copy_(torch.tensor([2000, 10, 3000, 640], dtype=torch.int32))
+    s = torch.cuda.Stream()
+    with torch.cuda.stream(s):
+        step()  # warm up
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=s):
+        step()
+    for lens in [[2000, 10, 3000, 640], [2001, 0, 3001, 1], [0, 0, 0, 0], [17, 3800, 128, 129], [1, 2, 3, 3799]]:
+        dw.seq_lens.copy_(torch.tensor(lens, dtype=torch.int32))
+        g.replay()
+        torch.cuda.synchronize()
+        cur = dataclasses.replace(w8, base=dataclasses.replace(w, seq_lens=np.array(lens, np.int32)))
+        check_against_oracle_fp8(cur, bufs.out, bufs.lse)
+    assert da.da_read_status(bufs.ws) == (0, -1)
