@@ -58,6 +58,8 @@ def parse_args():
     ap.add_argument("--q-len", type=int, default=1, help="queries per request (multi-query decode)")
     ap.add_argument("--tile", type=int, default=64)
     ap.add_argument("--width", type=int, default=0, help="CTAs per KV head (0 = 2 per SM / Hkv)")
+    ap.add_argument("--merge-in-decode", action="store_true",
+                    help="dynamic plan: merge split requests in the decode kernel instead of a combine launch")
     ap.add_argument("--no-static", action="store_true", help="skip the static split-k comparison")
     ap.add_argument("--no-cpu", action="store_true", help="skip the CPU oracle baseline")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
@@ -239,7 +241,7 @@ def run_ours(args, world, rank, local):
     w8 = W.quantize_fp8(w) if args.kv == "fp8" else None
     dw = w8.to("cuda") if w8 is not None else w.to("cuda")
     prob = da.problem_from(dw.problem)
-    desc = da.da_plan_desc_init(prob, da.PLAN_DYNAMIC, args.tile, args.width)
+    desc = da.da_plan_desc_init(prob, da.PLAN_DYNAMIC, args.tile, args.width, merge_in_decode=args.merge_in_decode)
     bufs = da.Buffers(prob, desc, "cuda")
     kv_bytes = w8.kv_bytes if w8 is not None else w.kv_bytes
     stream = torch.cuda.Stream()
@@ -342,7 +344,7 @@ def run_ours(args, world, rank, local):
                 + (f"; {args.q_len} queries per request" if args.q_len > 1 else ""),
                 "batch": w.problem.batch, "kv_format": args.kv, "q_len": args.q_len,
                 "kv_bytes_per_step_per_gpu": kv_bytes, "tile_tokens": desc.tile_tokens,
-                "ctas_per_kv_head": desc.num_ctas, "graph": True,
+                "ctas_per_kv_head": desc.num_ctas, "merge_in_decode": bool(desc.merge_in_decode), "graph": True,
                 "l2": "inputs larger than L2 (K/V read per step >> 126 MB), no flush"},
         frac_of_peak=round(value / world / peak, 4), frac_of_datasheet_8tbs=round(value / world / DATASHEET_HBM_GBS, 4),
         eager_us_per_step=round(ms_eager / steps * 1e3, 2),
@@ -355,7 +357,7 @@ def run_ours(args, world, rank, local):
              "us_per_step": round(ms_e2e / steps * 1e3, 2), "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
              "transfer": "da_decode_step_host with pinned host buffers: the plan launch reads seq_lens, block "
                          "table and q over PCIe; decode and combine write out/lse in place over PCIe"},
-        gpu_launches=3 * steps,
+        gpu_launches=(3 - desc.merge_in_decode) * steps,  # plan, decode (+ combine unless merged in decode)
         device_status=status[0],
     )
     if static:
@@ -406,7 +408,7 @@ def run_trace(args, world, rank, local):
     dt = DeviceTrace(tr)
     prob = dt.prob
     stream = torch.cuda.Stream()
-    desc = da.da_plan_desc_init(prob, da.PLAN_DYNAMIC, args.tile, args.width)
+    desc = da.da_plan_desc_init(prob, da.PLAN_DYNAMIC, args.tile, args.width, merge_in_decode=args.merge_in_decode)
     sdesc = da.da_plan_desc_init(prob, da.PLAN_STATIC, args.tile, 0)
     bufs, sbufs = da.Buffers(prob, desc, "cuda"), da.Buffers(prob, sdesc, "cuda")
     steps, warm = min(max(1, args.steps), tr.steps), max(3, args.warmup)
@@ -471,7 +473,7 @@ def run_trace(args, world, rank, local):
         higher_is_better=True, scaling="weak", vs_baseline=None, dtype="bf16", data="synthetic",
         config={"workload": f"trace: {tr.recipe}", "batch": prob.batch, "steps_timed": steps,
                 "kv_bytes_first_last_step": [kv[0], kv[-1]], "tile_tokens": desc.tile_tokens,
-                "ctas_per_kv_head": desc.num_ctas, "graph": True,
+                "ctas_per_kv_head": desc.num_ctas, "merge_in_decode": bool(desc.merge_in_decode), "graph": True,
                 "untimed": "device copies of each step's changes (restarted pages, block table, lengths, q) "
                            "and the KV append kernel, enqueued between the timed steps",
                 "l2": f"inputs larger than L2 ({min(kv) / 1e9:.1f}-{max(kv) / 1e9:.1f} GB K/V per step), no flush"},
@@ -484,7 +486,10 @@ def run_trace(args, world, rank, local):
                      "fused_plan_append_us_per_step": round(float(np.mean(times["append_fused"])) * 1e3, 2),
                      "separate_us_median": round(float(np.median(times["append_separate"])) * 1e3, 2),
                      "fused_plan_append_us_median": round(float(np.median(times["append_fused"])) * 1e3, 2)},
-        gpu_launches=3 * steps * 2 + 7 * (steps - 1), device_status=status[0],
+        # per step: dynamic (plan, decode, combine unless merged) + static (3); steps 1..: append + dynamic step,
+        # plan_append + decode (+ combine)
+        gpu_launches=(6 - desc.merge_in_decode) * steps + (7 - 2 * desc.merge_in_decode) * (steps - 1),
+        device_status=status[0],
         append_status=dt.status.tolist(), clocks=clocks.summary())
 
 
