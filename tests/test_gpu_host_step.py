@@ -186,3 +186,17 @@ def test_large_q_is_read_in_place():
             check_against_oracle_fp8(w8, out_p, lse_p)
         out_c, lse_c, _ = host_step(base, w8=w8, pinned=False)
         assert torch.equal(out_p.view(torch.int16), out_c.view(torch.int16)) and torch.equal(lse_p, lse_c)
+
+
+def test_large_multi_query_q_is_read_in_place():
+    """Multi-query decode with a q above 1 MiB in mapped memory: the multi-query kernel reads it over
+    the bus; causal limits and results as on the copy path."""
+    lens = np.random.default_rng(7).integers(2, 600, 160).astype(np.int32)
+    w = W.make_workload("big-q-mq", lens.tolist(), num_q_heads=32, num_kv_heads=4, head_dim=128, page_size=64,
+                        seed=20, q_len=2, recipe="host-step large multi-query q")
+    assert w.q.numel() * 2 > (1 << 20)
+    out_p, lse_p, st = host_step(w)
+    assert torch.count_nonzero(st["dw"].q) == 0  # never copied in
+    check_mq_against_oracle(w, out_p, lse_p)
+    out_c, lse_c, _ = host_step(w, pinned=False)
+    assert torch.equal(out_p.view(torch.int16), out_c.view(torch.int16)) and torch.equal(lse_p, lse_c)
