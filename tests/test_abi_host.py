@@ -159,6 +159,62 @@ def test_plan_append_checks(da_lib):
     assert call(prob_=prob(da, num_q_heads=60)) == da.ERR_INVALID_ARG
 
 
+def test_every_launching_call_checks_before_it_enqueues(da_lib):
+    """Null and misaligned arguments of each launching entry point come back as DA_ERR_INVALID_ARG
+    (shapes it does not build as DA_ERR_UNSUPPORTED) before any CUDA call; an empty batch is a no-op."""
+    import ctypes
+    da = da_lib
+    lib = da.lib()
+    p = prob(da)
+    d = da.da_plan_desc_init(p, da.PLAN_DYNAMIC, 64, 37)
+    A = 1 << 12  # a 16-byte-aligned stand-in address that no check dereferences
+    P, D = ctypes.byref(p), ctypes.byref(d)
+
+    def decode(fp8=False, **kw):
+        a = dict(q=A, k=A, v=A, ks=A, vs=A, bt=A, sl=A, ws=A, po=A, pl=A, out=A, lse=A)
+        a.update(kw)
+        if fp8:
+            return lib.da_decode_attention_fp8(P, D, a["q"], a["k"], a["v"], a["ks"], a["vs"], a["bt"], a["sl"],
+                                               a["ws"], a["po"], a["pl"], a["out"], a["lse"], None)
+        return lib.da_decode_attention(P, D, a["q"], a["k"], a["v"], a["bt"], a["sl"], a["ws"], a["po"], a["pl"],
+                                       a["out"], a["lse"], None)
+
+    for name in ("q", "k", "v", "bt", "sl", "ws", "po", "pl", "out", "lse"):
+        assert decode(**{name: None}) == da.ERR_INVALID_ARG, name
+    for name, off in (("k", 8), ("v", 8), ("q", 2), ("out", 4), ("po", 8), ("ws", 8)):
+        assert decode(**{name: A + off}) == da.ERR_INVALID_ARG, name
+    assert decode(fp8=True, ks=None) == da.ERR_INVALID_ARG and decode(fp8=True, vs=None) == da.ERR_INVALID_ARG
+    assert decode(fp8=True, q=A + 4) == da.ERR_INVALID_ARG  # the FP8 kernels read q in 8-byte pieces
+    s = da.da_plan_desc_init(p, da.PLAN_STATIC, 64, 2)
+    assert lib.da_static_plan(P, D, A, A, 1 << 24, None) == da.ERR_INVALID_ARG  # a dynamic descriptor
+    assert lib.da_static_plan(P, ctypes.byref(s), A, A, 64, None) == da.ERR_WORKSPACE
+    # append
+    assert lib.da_append_kv(P, None, A, A, A, A, A, None, None) == da.ERR_INVALID_ARG
+    assert lib.da_append_kv(P, A + 8, A, A, A, A, A, None, None) == da.ERR_INVALID_ARG
+    assert lib.da_append_kv(P, A, A, A, A, A + 8, A, None, None) == da.ERR_INVALID_ARG
+    p0 = prob(da, batch=0)
+    assert lib.da_append_kv(ctypes.byref(p0), None, None, None, None, None, None, None, None) == da.OK
+    # cross-GPU merge
+    assert lib.da_merge_partials(0, 10, 128, A, A, A, A, None) == da.ERR_INVALID_ARG
+    assert lib.da_merge_partials(2, -1, 128, A, A, A, A, None) == da.ERR_INVALID_ARG
+    assert lib.da_merge_partials(2, 10, 96, A, A, A, A, None) == da.ERR_UNSUPPORTED
+    assert lib.da_merge_partials(2, 0, 128, None, None, None, None, None) == da.OK
+    assert lib.da_merge_partials(2, 10, 128, A, A, None, A, None) == da.ERR_INVALID_ARG
+    assert lib.da_merge_partials(2, 10, 128, A + 4, A, A, A, None) == da.ERR_INVALID_ARG
+    # the no-allocation step: shape, scratch size, pointers and alignment, all before the plan is enqueued
+    def noalloc(prob_=p, width=37, **kw):
+        a = dict(q=A, k=A, v=A, bt=A, sl=A, out=A, lse=A)
+        a.update(kw)
+        return lib.da_decode_step_noalloc(ctypes.byref(prob_), 64, width, a["q"], a["k"], a["v"], a["bt"], a["sl"],
+                                          a["out"], a["lse"], None)
+    assert noalloc(prob_=prob(da, head_dim=96)) == da.ERR_UNSUPPORTED
+    assert noalloc(prob_=prob(da, batch=2000, num_pages=60000)) == da.ERR_WORKSPACE  # past the 16 MiB scratch
+    for name in ("q", "k", "v", "bt", "sl", "out", "lse"):
+        assert noalloc(**{name: None}) == da.ERR_INVALID_ARG, name
+    for name, off in (("k", 8), ("v", 8), ("q", 2), ("out", 4)):
+        assert noalloc(**{name: A + off}) == da.ERR_INVALID_ARG, name
+
+
 def test_stall_switch_checks_its_limit(da_lib):
     """Only the argument check is exercised here: a valid call would arm the next decode launch."""
     da = da_lib

@@ -62,6 +62,11 @@ extern "C" DA_API int da_decode_step_noalloc(const da_problem* prob, int32_t til
   if (ws_r + po_r + pl_r > (size_t)DA_NOALLOC_SCRATCH_BYTES) return DA_ERR_WORKSPACE;
   if (prob->batch > 0 && (!q || !k_cache || !v_cache || !block_table || !seq_lens || !out || !lse))
     return DA_ERR_INVALID_ARG;
+  // the decode call's alignment rules, checked here so that an error enqueues nothing (not even the plan)
+  if (prob->batch > 0 &&
+      (reinterpret_cast<uintptr_t>(k_cache) % 16 != 0 || reinterpret_cast<uintptr_t>(v_cache) % 16 != 0 ||
+       reinterpret_cast<uintptr_t>(q) % 4 != 0 || reinterpret_cast<uintptr_t>(out) % 8 != 0))
+    return DA_ERR_INVALID_ARG;
   void* base = nullptr;
   cudaError_t e = scratch_address(&base);
   if (e != cudaSuccess) {
