@@ -65,6 +65,14 @@ def test_cp_decode_step_single_rank_group(da_lib, oracle_lib):
         cp_decode_step(prob, desc, dw.q, dw.k_cache, dw.v_cache, dw.block_table, dw.seq_lens, bufs, out, lse)
         torch.cuda.synchronize()
         check_against_oracle(w, out, lse)
+        # on a side stream: the gather and the merge follow that stream's decode
+        side = torch.cuda.Stream()
+        out.fill_(float("nan"))
+        lse.fill_(float("nan"))
+        cp_decode_step(prob, desc, dw.q, dw.k_cache, dw.v_cache, dw.block_table, dw.seq_lens, bufs, out, lse,
+                       stream=side)
+        torch.cuda.synchronize()
+        check_against_oracle(w, out, lse)
     finally:
         if created:
             dist.destroy_process_group()

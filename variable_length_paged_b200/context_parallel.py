@@ -48,15 +48,21 @@ def cp_decode_step(prob, desc, q, k_cache, v_cache, local_block_table, local_seq
 
     `out` [B, Hq, d] bf16 and `lse` [B, Hq] fp32 receive the merged result on every rank.
     """
+    import contextlib
+
     import torch.distributed as dist
 
     if prob.q_len > 1:
         raise ValueError("context-parallel decode handles one query per request")
-    da.decode_step(prob, desc, q, k_cache, v_cache, local_block_table, local_seq_lens, bufs, stream=stream)
-    world = dist.get_world_size(group)
-    parts_out = torch.empty((world,) + tuple(bufs.out.shape), dtype=bufs.out.dtype, device=bufs.out.device)
-    parts_lse = torch.empty((world,) + tuple(bufs.lse.shape), dtype=bufs.lse.dtype, device=bufs.lse.device)
-    dist.all_gather_into_tensor(parts_out, bufs.out, group=group)
-    dist.all_gather_into_tensor(parts_lse, bufs.lse, group=group)
-    da.da_merge_partials(parts_out, parts_lse, out, lse, stream=stream)
+    # the collectives order themselves after the current stream's work: make `stream` current so that
+    # the all-gather follows this rank's decode and the merge follows the all-gather
+    on_stream = torch.cuda.stream(stream) if stream is not None else contextlib.nullcontext()
+    with on_stream:
+        da.decode_step(prob, desc, q, k_cache, v_cache, local_block_table, local_seq_lens, bufs, stream=stream)
+        world = dist.get_world_size(group)
+        parts_out = torch.empty((world,) + tuple(bufs.out.shape), dtype=bufs.out.dtype, device=bufs.out.device)
+        parts_lse = torch.empty((world,) + tuple(bufs.lse.shape), dtype=bufs.lse.dtype, device=bufs.lse.device)
+        dist.all_gather_into_tensor(parts_out, bufs.out, group=group)
+        dist.all_gather_into_tensor(parts_lse, bufs.lse, group=group)
+        da.da_merge_partials(parts_out, parts_lse, out, lse, stream=stream)
     return out, lse
