@@ -20,7 +20,11 @@
  *                        per-segment partials (requests split over CTAs)
  *   da_combine           partials -> out/lse by log-sum-exp merge
  * (With merge_in_decode = 1 in the descriptor the decode kernel merges split
- * requests itself and da_combine enqueues nothing.)
+ * requests itself and da_combine enqueues nothing.)  Before the step, the new
+ * token's K/V rows go into their pages with da_append_kv, or with
+ * da_plan_append, which also builds the dynamic plan in the same launch and
+ * then stands in for da_plan.  da_decode_step_host runs a whole step from host
+ * buffers in one call.
  * The host never reads seq_lens: every launch's grid is fixed by the problem
  * and the plan descriptor, so requests can join, grow, finish or be cancelled
  * between steps without a host round trip, and the three calls can be
