@@ -110,3 +110,29 @@ def test_trace_steps_grow_finish_and_restart():
         assert live + len(tr.free) == tr.problem.num_pages  # no page lost or handed out twice
     assert restarts > 0
     check_layout(tr.workload(), poisoned=False)
+
+
+def test_fp8_quantiser_recipe():
+    """scale = max |x| / 448 per KV head; every live value comes back within half an E4M3 step of its
+    exponent (3 mantissa bits: |x/scale - e4m3| <= 2^-4 |x/scale|, or an absolute 2^-10 in the
+    subnormal range); the largest |x| of each head maps to the largest finite code 448."""
+    w = W.make_workload("q8", [1, 17, 300, 64], num_q_heads=4, num_kv_heads=2, head_dim=128, page_size=16, seed=4)
+    w8 = W.quantize_fp8(w)
+    P = w.problem.page_size
+    for cache, code, scale in ((w.k_cache, w8.k_code, w8.k_scale), (w.v_cache, w8.v_code, w8.v_scale)):
+        assert code.dtype == torch.uint8 and code.shape == cache.shape and scale.dtype == np.float32
+        vals, decs = [], []
+        for b in range(w.problem.batch):
+            t = np.arange(int(w.seq_lens[b]))
+            pages = torch.from_numpy(w.block_table[b, t // P].astype(np.int64))
+            slots = torch.from_numpy(t % P)
+            vals.append(cache[pages, :, slots].float())  # [L, Hkv, d]
+            decs.append(code[pages, :, slots].view(torch.float8_e4m3fn).float())
+        x, c = torch.cat(vals), torch.cat(decs)
+        for g in range(w.problem.num_kv_heads):
+            amax = float(x[:, g].abs().max())
+            assert scale[g] == np.float32(amax / 448.0)
+            y = x[:, g] / float(scale[g])
+            err = (y - c[:, g]).abs()
+            assert torch.all(err <= torch.maximum(y.abs() * 2.0 ** -4, torch.full_like(y, 2.0 ** -10)))
+            assert float(c[:, g].abs().max()) == 448.0
