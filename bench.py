@@ -3,19 +3,23 @@
 
 A step is the whole hot path on one batch: on-device plan -> decode kernel ->
 log-sum-exp combine, through the C ABI (libda.so).  The default workload is the
-mixed-length batch (32 requests, lengths uniform in [1000, 16000], 64 query /
-8 KV heads, head_dim 128, page 64): 1.11 GB of K/V per step, far larger than
-the 126 MB L2, so consecutive steps cannot hit in L2.
+skewed continuous batch (128 requests: 115 with lengths uniform in [256, 2048],
+13 with lengths uniform in [16384, 65536]; 1 % of K rows scaled by 8; 64 query /
+8 KV heads, head_dim 128, page 64): 2.72 GB of K/V per step, the largest
+single-step workload, far larger than the 126 MB L2, so consecutive steps cannot
+hit in L2.
 
 Printed (rank 0, one JSON line): KV-read GB/s of the whole step (value), the
-step time, the decode kernel's own achieved bandwidth against the measured HBM
+step time (mean over the timed region, and median / p10 / p90 of the per-step
+times), the decode kernel's own achieved bandwidth against the measured HBM
 peak, the same step under the static split-k schedule (default and best split
 count), an end-to-end number (one da_decode_step_host call per step from pinned
 host buffers: the plan launch reads lengths, block table and q over PCIe, and
 out/lse are written in place into host memory), the CPU oracle's rate
-on this machine's cores, and the SM clocks seen during the measurement.
+on this machine's cores (all of them, and one thread), and the SM clocks seen
+during the measurement.
 
-    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference] [--config mixed]
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference] [--config skewed]
 
 With N > 1 (torchrun) every rank runs its own, differently seeded batch of the
 same shape (weak scaling: requests are independent, so there is no data-path
@@ -42,8 +46,12 @@ if ROOT not in sys.path:
 METRIC = "µs/decode step and KV-read HBM GB/s (% of B200 peak) vs static split-k"
 FALLBACK_HBM_GBS = 6650.0
 DATASHEET_HBM_GBS = 8000.0
-KERNEL_SOURCES = ["variable_length_paged_b200/csrc/decode.cu", "variable_length_paged_b200/csrc/decode_tc.cu",
-                  "variable_length_paged_b200/csrc/da_internal.cuh"]
+L2_BYTES = 126 * 2**20
+# the sources each cache format's decode kernel is built from (the ncu traffic record is keyed to them)
+KERNEL_SOURCES = {
+    "bf16": ["variable_length_paged_b200/csrc/decode.cu", "variable_length_paged_b200/csrc/da_internal.cuh"],
+    "fp8": ["variable_length_paged_b200/csrc/decode_tc.cu", "variable_length_paged_b200/csrc/da_internal.cuh"],
+}
 TRAFFIC_FILE = os.path.join(ROOT, "profiles", "decode_kernel_traffic.txt")
 
 
@@ -53,7 +61,7 @@ def parse_args():
     ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--config", default="mixed", choices=["mixed", "skewed", "low_conc", "uniform", "tiny", "trace"])
+    ap.add_argument("--config", default="skewed", choices=["mixed", "skewed", "low_conc", "uniform", "tiny", "trace"])
     ap.add_argument("--kv", choices=["bf16", "fp8"], default="bf16", help="KV cache format")
     ap.add_argument("--q-len", type=int, default=1, help="queries per request (multi-query decode)")
     ap.add_argument("--tile", type=int, default=64)
@@ -117,9 +125,9 @@ def measured_peak():
         return FALLBACK_HBM_GBS, "profiling-recipe fallback 6.65 TB/s (of fallback)"
 
 
-def kernel_source_hash():
+def kernel_source_hash(kv="bf16"):
     h = hashlib.sha256()
-    for rel in KERNEL_SOURCES:
+    for rel in KERNEL_SOURCES[kv]:
         with open(os.path.join(ROOT, rel), "rb") as f:
             h.update(f.read())
     return h.hexdigest()[:16]
@@ -133,19 +141,22 @@ def decode_kernel_name(problem, fp8, q_len):
 
 
 def recorded_traffic(workload_name, kv="bf16", q_len=1):
-    """DRAM bytes per decode launch from the committed ncu record, if it matches this kernel source."""
+    """DRAM bytes per decode launch from the committed ncu record, if it matches this kernel source.
+
+    Returns (bytes or None, where they come from or why there are none)."""
+    rel = os.path.relpath(TRAFFIC_FILE, ROOT)
     try:
         with open(TRAFFIC_FILE) as f:
             j = dict(ln.split(": ", 1) for ln in f.read().splitlines() if ln and not ln.startswith("#"))
     except Exception:
-        return None, "no ncu capture recorded"
-    if j.get("kernel_source_sha") != kernel_source_hash():
-        return None, "kernel changed since the ncu capture"
+        return None, f"no ncu capture recorded ({rel} missing)"
+    if j.get(f"kernel_source_sha.{kv}") != kernel_source_hash(kv):
+        return None, f"{kv} decode kernel changed since the ncu capture in {rel}"
     key = f"{workload_name}.{kv}"
     if q_len > 1 or f"{key}.dram_bytes_read_per_launch" not in j:
-        return None, f"no ncu capture for {key}" + (f" with {q_len} queries" if q_len > 1 else "")
+        return None, f"no ncu capture for {key}" + (f" with {q_len} queries" if q_len > 1 else "") + f" in {rel}"
     return (int(j[f"{key}.dram_bytes_read_per_launch"]) + int(j[f"{key}.dram_bytes_write_per_launch"]),
-            j.get(f"{key}.command", ""))
+            f"{rel} ({key}; captured with: {j.get(f'{key}.command', '')})")
 
 
 class ClockSampler:
@@ -213,17 +224,45 @@ class ClockSampler:
 # our arm
 
 
-def time_region(stream, fn, steps):
-    """Device time of `steps` calls of fn() on `stream`, bracketed by CUDA events (ms)."""
+def time_region(stream, fn, steps, per_step=False):
+    """Device time of `steps` calls of fn() on `stream`, bracketed by CUDA events (ms).
+
+    With per_step, an event is also recorded between consecutive calls, and the list of
+    per-call times (ms) is returned as well; their sum is the bracketed time."""
     import torch
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(steps + 1 if per_step else 2)]
     torch.cuda.synchronize()
-    e0.record(stream)
-    for _ in range(steps):
+    ev[0].record(stream)
+    for i in range(steps):
         fn()
-    e1.record(stream)
+        if per_step:
+            ev[i + 1].record(stream)
+    if not per_step:
+        ev[1].record(stream)
     torch.cuda.synchronize()
-    return e0.elapsed_time(e1)
+    total = ev[0].elapsed_time(ev[-1])
+    if not per_step:
+        return total
+    return total, [ev[i].elapsed_time(ev[i + 1]) for i in range(steps)]
+
+
+def step_stats(ms_list):
+    """Median, p10 and p90 of per-step times, in µs."""
+    import numpy as np
+    a = np.asarray(ms_list, dtype=np.float64) * 1e3
+    return {"median": round(float(np.median(a)), 2), "p10": round(float(np.percentile(a, 10)), 2),
+            "p90": round(float(np.percentile(a, 90)), 2)}
+
+
+def workload_config(name, w, w8=None, q_len=1):
+    """The `config` object of the JSON line: the workload alone, identical for both arms."""
+    kv = w8.kv_bytes if w8 is not None else w.kv_bytes
+    return {"workload": f"{name}: {w.recipe}" + ("; FP8 E4M3 KV, per-head scales" if w8 is not None else "")
+            + (f"; {q_len} queries per request" if q_len > 1 else ""),
+            "batch": w.problem.batch, "kv_format": "fp8" if w8 is not None else "bf16", "q_len": q_len,
+            "kv_bytes_per_step_per_gpu": int(kv),
+            "l2": "inputs larger than L2 (K/V read per step >> 126 MB), no flush" if kv > L2_BYTES else
+                  f"inputs fit in L2 ({kv} B of K/V per step): a latency case, not an HBM figure"}
 
 
 def run_ours(args, world, rank, local):
@@ -275,7 +314,7 @@ def run_ours(args, world, rank, local):
             for _ in range(warm):
                 graph.replay()
             barrier(world)
-            ms_graph = time_region(stream, graph.replay, steps)
+            ms_graph, per_step_ms = time_region(stream, graph.replay, steps, per_step=True)
             barrier(world)
             ms_eager = time_region(stream, step, steps)
             # decode kernel alone, per launch, inside a run of eager steps
@@ -328,8 +367,11 @@ def run_ours(args, world, rank, local):
     d2h = out_h.numel() * out_h.element_size() + lse_h.numel() * 4
 
     dec_avg_ms = statistics.mean(dec_ms)
-    maxes, sums = reduce_max_sum([ms_graph, ms_eager, ms_e2e, dec_avg_ms], [float(kv_bytes)], world)
-    ms_graph, ms_eager, ms_e2e, dec_avg_ms = maxes
+    st = step_stats(per_step_ms)
+    maxes, sums = reduce_max_sum([ms_graph, ms_eager, ms_e2e, dec_avg_ms, st["median"], st["p10"], st["p90"]],
+                                 [float(kv_bytes)], world)
+    ms_graph, ms_eager, ms_e2e, dec_avg_ms = maxes[:4]
+    st = {"median": round(maxes[4], 2), "p10": round(maxes[5], 2), "p90": round(maxes[6], 2)}
     total_bytes = sums[0]
     step_s = ms_graph / 1e3 / steps
     value = total_bytes / step_s / 1e9
@@ -339,13 +381,13 @@ def run_ours(args, world, rank, local):
     result.update(
         metric=METRIC, value=round(value, 2), unit="GB/s", n_gpus=world, steps=steps, warmup=warm,
         ms_per_step=round(ms_graph / steps, 5), us_per_step=round(ms_graph / steps * 1e3, 2),
+        us_per_step_median_p10_p90=[st["median"], st["p10"], st["p90"]],
         higher_is_better=True, scaling="weak", vs_baseline=None, dtype="bf16", data="synthetic",
-        config={"workload": f"{args.config}: {w.recipe}" + ("; FP8 E4M3 KV, per-head scales" if w8 else "")
-                + (f"; {args.q_len} queries per request" if args.q_len > 1 else ""),
-                "batch": w.problem.batch, "kv_format": args.kv, "q_len": args.q_len,
-                "kv_bytes_per_step_per_gpu": kv_bytes, "tile_tokens": desc.tile_tokens,
-                "ctas_per_kv_head": desc.num_ctas, "merge_in_decode": bool(desc.merge_in_decode), "graph": True,
-                "l2": "inputs larger than L2 (K/V read per step >> 126 MB), no flush"},
+        config=workload_config(args.config, w, w8, args.q_len),
+        launch={"tile_tokens": desc.tile_tokens, "ctas_per_kv_head": desc.num_ctas,
+                "merge_in_decode": bool(desc.merge_in_decode), "graph": True,
+                "timing": "one CUDA graph per step (plan, decode, combine), K replays between CUDA events on "
+                          "the launching stream, an event between replays for the per-step times"},
         frac_of_peak=round(value / world / peak, 4), frac_of_datasheet_8tbs=round(value / world / DATASHEET_HBM_GBS, 4),
         eager_us_per_step=round(ms_eager / steps * 1e3, 2),
         roofline={"bound": "hbm", "achieved": round(dec_gbs, 2), "peak": peak, "unit": "GB/s",
@@ -493,30 +535,75 @@ def run_trace(args, world, rank, local):
         append_status=dt.status.tolist(), clocks=clocks.summary())
 
 
-def cpu_baseline(w, seconds, w8=None):
-    """The CPU oracle (fp64) on this host's cores, repeated over the full batch for a bounded time."""
+def _oracle_run(w, w8, pairs=None, threads=0):
+    """One oracle call over the (request, head) pairs (all of them when None)."""
     import numpy as np
 
     import oracle
+    if w8 is None and w.q.dim() == 4:  # multi-query: whole batch only
+        oracle.attention_mq(w.q, w.k_cache, w.v_cache, w.block_table, w.seq_lens, scale=w.problem.scale,
+                            threads=threads)
+    elif w8 is None:
+        oracle.attention(w.q, w.k_cache, w.v_cache, w.block_table, w.seq_lens, scale=w.problem.scale, pairs=pairs,
+                         threads=threads)
+    else:
+        oracle.attention_fp8(w.q, w8.k_code, w8.v_code, w8.k_scale.astype(np.float64), w8.v_scale.astype(np.float64),
+                             w.block_table, w.seq_lens, scale=w.problem.scale, pairs=pairs, threads=threads)
+
+
+def request_sample(w, w8, seconds, threads):
+    """A seeded sample of whole requests (all heads) that the oracle runs in about `seconds` with
+    `threads` threads (at least one request), from a calibration run on the shortest request.
+    Returns (pairs, requests, tokens)."""
+    import numpy as np
+    B, Hq = w.problem.batch, w.problem.num_q_heads
+    live = [b for b in range(B) if w.seq_lens[b] > 0] or [0]
+    short = min(live, key=lambda b: w.seq_lens[b])
+    t0 = time.perf_counter()
+    _oracle_run(w, w8, (np.full(Hq, short, np.int32), np.arange(Hq, dtype=np.int32)), threads)
+    rate = max(int(w.seq_lens[short]), 1) / max(time.perf_counter() - t0, 1e-6)  # tokens/s, all heads
+    budget = rate * seconds
+    picks, acc = [], 0
+    for b in np.random.default_rng(0).permutation(B):
+        if picks and acc + w.seq_lens[b] > budget:
+            continue
+        picks.append(int(b))
+        acc += int(w.seq_lens[b])
+    pairs = (np.repeat(np.array(picks, np.int32), Hq), np.tile(np.arange(Hq, dtype=np.int32), len(picks)))
+    return pairs, picks, acc
+
+
+def cpu_baseline(w, seconds, w8=None):
+    """The CPU oracle (fp64) on this host: all cores over whole batches, repeated for about `seconds`;
+    then one thread over a seeded sample of requests sized to about `seconds`."""
+    import oracle
     oracle.build()
+    kv = w8.kv_bytes if w8 is not None else w.kv_bytes
+    per_token = kv / max(int(w.seq_lens.sum()), 1)  # K/V bytes per cached token (all KV heads)
     t0 = time.perf_counter()
     passes = 0
     while True:
-        if w8 is None and w.q.dim() == 4:
-            oracle.attention_mq(w.q, w.k_cache, w.v_cache, w.block_table, w.seq_lens, scale=w.problem.scale)
-        elif w8 is None:
-            oracle.attention(w.q, w.k_cache, w.v_cache, w.block_table, w.seq_lens, scale=w.problem.scale)
-        else:
-            oracle.attention_fp8(w.q, w8.k_code, w8.v_code, w8.k_scale.astype(np.float64),
-                                 w8.v_scale.astype(np.float64), w.block_table, w.seq_lens, scale=w.problem.scale)
+        _oracle_run(w, w8)
         passes += 1
         if time.perf_counter() - t0 >= seconds or passes >= 50:
             break
     dt = time.perf_counter() - t0
-    kv = w8.kv_bytes if w8 is not None else w.kv_bytes
-    return {"value": round(passes * kv / dt / 1e9, 4), "unit": "GB/s", "cores": oracle.num_threads(),
-            "kind": "oracle", "sample": f"{passes} pass(es) of the fp64 oracle over the full batch "
-                                        f"({w.problem.batch} requests x {w.problem.num_q_heads} heads), {dt:.1f} s"}
+    res = {"value": round(passes * kv / dt / 1e9, 4), "unit": "GB/s", "cores": oracle.num_threads(),
+           "kind": "oracle", "sample": f"{passes} pass(es) of the fp64 oracle over the full batch "
+                                       f"({w.problem.batch} requests x {w.problem.num_q_heads} heads), {dt:.1f} s"}
+    if w.q.dim() == 4 and w8 is None:
+        t0 = time.perf_counter()
+        _oracle_run(w, w8, threads=1)
+        dt1, tok, desc = time.perf_counter() - t0, int(w.seq_lens.sum()), "the full batch"
+    else:
+        pairs, picks, tok = request_sample(w, w8, seconds, 1)
+        t0 = time.perf_counter()
+        _oracle_run(w, w8, pairs, threads=1)
+        dt1 = time.perf_counter() - t0
+        desc = f"{len(picks)} of {w.problem.batch} requests (all {w.problem.num_q_heads} heads, {tok} tokens)"
+    res["one_thread"] = {"value": round(tok * per_token / dt1 / 1e9, 4), "unit": "GB/s", "cores": 1,
+                         "sample": f"{desc}, {dt1:.1f} s"}
+    return res
 
 
 # ------------------------------------------------------------------------------------------------
@@ -524,49 +611,32 @@ def cpu_baseline(w, seconds, w8=None):
 
 
 def run_reference(args, rank):
-    import numpy as np
-
     import oracle
     from variable_length_paged_b200 import workloads as W
 
     oracle.build()
     w = W.DecodeTrace().workload() if args.config == "trace" else W.CONFIGS[args.config]()
-    B, Hq = w.problem.batch, w.problem.num_q_heads
-    order = np.argsort(-w.seq_lens, kind="stable")
-    # calibrate: aim for about one second of oracle work per step, and at most ~150 s in total
-    t0 = time.perf_counter()
-    oracle.attention(w.q, w.k_cache, w.v_cache, w.block_table, w.seq_lens, scale=w.problem.scale,
-                     pairs=(np.full(Hq, order[-1], np.int32), np.arange(Hq, dtype=np.int32)))
-    rate = max(int(w.seq_lens[order[-1]]), 1) / max(time.perf_counter() - t0, 1e-6)  # tokens/s over all heads
+    w8 = W.quantize_fp8(w) if args.kv == "fp8" else None
     steps, warm = max(1, args.steps), max(3, args.warmup)
-    budget_tokens = rate * min(1.0, 150.0 / (steps + warm))
-    picks, acc = [], 0
-    for b in np.random.default_rng(0).permutation(B):
-        if picks and acc + w.seq_lens[b] > budget_tokens:
-            continue
-        picks.append(int(b))
-        acc += int(w.seq_lens[b])
-    pb = np.repeat(np.array(picks, np.int32), Hq)
-    ph = np.tile(np.arange(Hq, dtype=np.int32), len(picks))
-    sample_bytes = acc * w.problem.num_kv_heads * w.problem.head_dim * 4
-
-    def one():
-        oracle.attention(w.q, w.k_cache, w.v_cache, w.block_table, w.seq_lens, scale=w.problem.scale, pairs=(pb, ph))
-
+    # about one second of oracle work per step, and at most ~150 s in total
+    pairs, picks, tok = request_sample(w, w8, min(1.0, 150.0 / (steps + warm)), 0)
+    per_token = (w8.kv_bytes if w8 is not None else w.kv_bytes) / max(int(w.seq_lens.sum()), 1)
+    sample_bytes = int(round(tok * per_token))
     for _ in range(warm):
-        one()
+        _oracle_run(w, w8, pairs)
     t0 = time.perf_counter()
     for _ in range(steps):
-        one()
+        _oracle_run(w, w8, pairs)
     dt = time.perf_counter() - t0
     value = steps * sample_bytes / dt / 1e9
+    B, Hq = w.problem.batch, w.problem.num_q_heads
     cpu = {"value": round(value, 4), "unit": "GB/s", "cores": oracle.num_threads(), "kind": "oracle",
-           "sample": f"{len(picks)} of {B} requests (all {Hq} heads, {acc} tokens) per step"}
+           "sample": f"{len(picks)} of {B} requests (all {Hq} heads, {tok} tokens, {sample_bytes} K/V bytes) "
+                     f"per step"}
     return {"impl": "reference", "metric": METRIC, "value": round(value, 4), "unit": "GB/s", "n_gpus": 1,
             "steps": steps, "warmup": warm, "ms_per_step": round(dt / steps * 1e3, 3), "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-            "config": {"workload": f"{args.config}: {w.recipe}", "batch": B,
-                       "kv_bytes_per_step_sample": sample_bytes},
+            "config": workload_config(args.config if args.config != "trace" else "trace", w, w8),
             "cpu_baseline": cpu,
             "e2e": {"value": round(value, 4), "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
 

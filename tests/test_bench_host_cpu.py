@@ -20,18 +20,43 @@ def bench(monkeypatch):
 def test_traffic_record_follows_the_kernel_source(bench, monkeypatch):
     rec = dict(ln.split(": ", 1) for ln in open(bench.TRAFFIC_FILE).read().splitlines()
                if ln and not ln.startswith("#"))
-    monkeypatch.setattr(bench, "kernel_source_hash", lambda: rec["kernel_source_sha"])  # the captured kernels
-    t, cmd = bench.recorded_traffic("mixed", "bf16")
-    assert t == int(rec["mixed.bf16.dram_bytes_read_per_launch"]) + int(rec["mixed.bf16.dram_bytes_write_per_launch"])
-    assert "ncu" in cmd and "--clock-control none" in cmd and "bench.py" in cmd
-    # traffic must be a little above the algorithmic bytes (no re-reads), never below
-    alg = int(rec["mixed.bf16.algorithmic_bytes_per_launch"])
-    assert alg <= int(rec["mixed.bf16.dram_bytes_read_per_launch"]) <= 1.02 * alg
+    # the captured kernels, per cache format
+    monkeypatch.setattr(bench, "kernel_source_hash", lambda kv="bf16": rec[f"kernel_source_sha.{kv}"])
+    for kv in ("bf16", "fp8"):
+        t, src = bench.recorded_traffic("mixed", kv)
+        assert t == (int(rec[f"mixed.{kv}.dram_bytes_read_per_launch"]) +
+                     int(rec[f"mixed.{kv}.dram_bytes_write_per_launch"]))
+        # the source names the committed record and the command that made it
+        assert src.startswith("profiles/decode_kernel_traffic.txt") and "gpurun_out" not in src.split("(")[0]
+        assert "ncu" in src and "--clock-control none" in src and "bench.py" in src
+        # traffic must be a little above the algorithmic bytes (no re-reads), never below
+        alg = int(rec[f"mixed.{kv}.algorithmic_bytes_per_launch"])
+        assert alg <= int(rec[f"mixed.{kv}.dram_bytes_read_per_launch"]) <= 1.02 * alg
     assert bench.recorded_traffic("mixed", "bf16", q_len=2)[0] is None  # no capture for multi-query
     assert bench.recorded_traffic("no_such_workload", "bf16")[0] is None
-    monkeypatch.setattr(bench, "kernel_source_hash", lambda: "0" * 16)  # any other kernel source
-    t, why = bench.recorded_traffic("mixed", "bf16")
+    # a change to one format's kernel voids that format's record only
+    monkeypatch.setattr(bench, "kernel_source_hash",
+                        lambda kv="bf16": "0" * 16 if kv == "fp8" else rec["kernel_source_sha.bf16"])
+    t, why = bench.recorded_traffic("mixed", "fp8")
     assert t is None and "changed" in why
+    assert bench.recorded_traffic("mixed", "bf16")[0] is not None
+
+
+def test_kernel_source_hash_covers_each_format_sources(bench):
+    import hashlib
+    import os
+    for kv in ("bf16", "fp8"):
+        h = hashlib.sha256()
+        for rel in bench.KERNEL_SOURCES[kv]:
+            h.update(open(os.path.join(bench.ROOT, rel), "rb").read())
+        assert bench.kernel_source_hash(kv) == h.hexdigest()[:16]
+    assert any("decode_tc.cu" in f for f in bench.KERNEL_SOURCES["fp8"])
+    assert not any("decode_tc.cu" in f for f in bench.KERNEL_SOURCES["bf16"])
+
+
+def test_step_statistics(bench):
+    s = bench.step_stats([0.1, 0.2, 0.3, 0.4, 0.5])
+    assert s == {"median": 300.0, "p10": 140.0, "p90": 460.0}
 
 
 def test_clock_record_summary(bench, tmp_path):

@@ -33,6 +33,12 @@ def test_reference_arm_line(oracle_lib):
     assert d["value"] > 0 and d["unit"] == "GB/s" and d["higher_is_better"] is True
     assert d["data"] == "synthetic" and d["vs_baseline"] is None
     assert d["config"]["workload"].startswith("tiny")
+    # the reference arm's config is the GPU arm's (both come from one function of the workload)
+    sys.argv = ["bench.py"]
+    sys.path.insert(0, ROOT)
+    import bench
+    from variable_length_paged_b200 import workloads as W
+    assert d["config"] == bench.workload_config("tiny", W.tiny())
     cpu = d["cpu_baseline"]
     assert cpu["kind"] == "oracle" and cpu["cores"] >= 1 and cpu["value"] == d["value"] and cpu["sample"]
     assert d["e2e"] == {"value": d["value"], "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}
