@@ -19,6 +19,8 @@
  *   da_decode_attention  work list -> out/lse (single-segment requests) and
  *                        per-segment partials (requests split over CTAs)
  *   da_combine           partials -> out/lse by log-sum-exp merge
+ * or one call, da_decode_step, which enqueues the same three launches and lets the
+ * decode kernel request its first K/V chunks before the plan has landed.
  * (With merge_in_decode = 1 in the descriptor the decode kernel merges split
  * requests itself and da_combine enqueues nothing.)  Before the step, the new
  * token's K/V rows go into their pages with da_append_kv, or with
@@ -80,6 +82,10 @@ extern "C" {
 #define DA_PLAN_DYNAMIC 0 /* load-balanced: U tiles over C CTAs per KV head, contiguous ranges */
 #define DA_PLAN_STATIC 1  /* comparator: S equal splits per request, B*S CTAs per KV head */
 
+/* ---- output formats (da_plan_desc.out_format) ----------------------------------------- */
+#define DA_OUT_BF16 0 /* out is bf16; single-segment requests are written by the decode kernel */
+#define DA_OUT_F32 1  /* out is fp32; every request's result goes through the partials and da_combine */
+
 /*
  * The problem: one decode step of a continuous batch.
  *
@@ -94,7 +100,8 @@ extern "C" {
  *                requests may name the same page (shared prefixes).
  *   seq_lens     int32 [batch], the number of cached tokens of each request,
  *                0 for a finished or cancelled slot.
- *   out          bf16 [batch][num_q_heads][head_dim];  lse fp32 [batch][num_q_heads]
+ *   out          bf16 [batch][num_q_heads][head_dim] (fp32 with out_format DA_OUT_F32);
+ *                lse fp32 [batch][num_q_heads]
  *
  * Query head h reads KV head h / (num_q_heads / num_kv_heads) (consecutive
  * grouping).  out = softmax(scale * q . K^T) . V over the request's tokens and
@@ -141,6 +148,12 @@ typedef struct da_plan_desc {
                               1: by the decode kernel's last CTA for each of them (no extra launch;
                               faster for batches of many long requests, slower when one request
                               is split over many CTAs) */
+  int32_t out_format;      /* DA_OUT_BF16 (default) or DA_OUT_F32: `out` holds fp32 values, for a
+                              caller that merges this step's result with others (one slice of a
+                              request's cache per GPU) and wants no bf16 rounding before that
+                              merge.  Every segment's result then goes to the partials and
+                              da_combine writes `out` for every request (also those with one
+                              segment); merge_in_decode must be 0 */
 } da_plan_desc;
 
 /*
@@ -154,6 +167,12 @@ typedef struct da_plan_desc {
  *   desc         host, out.
  * Tile size and C change only how work is spread; the result is the same up
  * to fp32 rounding.  Queries the current device only when a default is asked.
+ * Errors: DA_ERR_INVALID_ARG for a bad problem or kind, DA_ERR_UNSUPPORTED for
+ * a shape the kernels are not built for, DA_ERR_CUDA if a default needs a device
+ * query that fails.  Source: "Tencent HPC lands in SGLang, challenging default
+ * inference kernels", section "Why Tencent HPC matters for online model serving"
+ * (the KV-cache work is cut into uniform tiles that a scheduler hands to CTAs):
+ * T is the tile, C the number of CTAs per KV head that share the tiles.
  */
 DA_API int da_plan_desc_init(const da_problem* prob, int32_t kind, int32_t tile_tokens, int32_t width,
                              da_plan_desc* desc);
@@ -163,10 +182,27 @@ DA_API int da_plan_desc_init(const da_problem* prob, int32_t kind, int32_t tile_
  *   ws_bytes           the plan (int32 header and work list), 16-byte aligned
  *   partial_o_bytes    fp32 [max_segments][q_len][num_q_heads][head_dim]
  *   partial_lse_bytes  fp32 [max_segments][q_len][num_q_heads]
- * Any output pointer may be NULL.
+ * Any output pointer may be NULL.  Host only; enqueues nothing.  Errors as for
+ * da_plan_desc_init (a descriptor that does not match the problem is
+ * DA_ERR_INVALID_ARG).  Source: as for da_plan below (the work list) and
+ * da_combine (the split partials).
  */
 DA_API int da_workspace_size(const da_problem* prob, const da_plan_desc* desc, size_t* ws_bytes,
                              size_t* partial_o_bytes, size_t* partial_lse_bytes);
+
+/*
+ * da_plan_workspace_size -- the same three sizes for a dynamic plan of tile
+ * size tile_tokens and num_ctas CTAs per KV head (0 = the defaults of
+ * da_plan_desc_init), without building a descriptor first: it is
+ * da_plan_desc_init(prob, DA_PLAN_DYNAMIC, tile_tokens, num_ctas) followed by
+ * da_workspace_size.  Host only; any output pointer may be NULL; errors as for
+ * those two calls.  The descriptor exists because every call of a step must
+ * agree on the plan geometry (T, C, the segment capacity C + B - 1, the plan
+ * kind); this call is for callers that size buffers before they build one.
+ * Source: as for da_plan.
+ */
+DA_API int da_plan_workspace_size(const da_problem* prob, int32_t tile_tokens, int32_t num_ctas, size_t* ws_bytes,
+                                  size_t* partial_o_bytes, size_t* partial_lse_bytes);
 
 /*
  * da_workspace_offsets -- word (int32) offsets of the arrays inside `ws`, for
@@ -193,6 +229,13 @@ DA_API int da_workspace_offsets(const da_plan_desc* desc, int64_t off[7]);
  * gets the contiguous global tile range [floor(c*U/C), floor((c+1)*U/C)), cut
  * at request boundaries into segments.  Requests with a bad length get 0
  * tiles and DA_DEV_BAD_SEQLEN (first bad index = the lowest such b).
+ * The host never reads seq_lens: the plan is rebuilt on the device every step.
+ * Errors: DA_ERR_INVALID_ARG (null or unaligned pointer, a static descriptor),
+ * DA_ERR_WORKSPACE (ws_bytes too small), DA_ERR_CUDA (launch refused).
+ * Source: "Tencent HPC lands in SGLang, challenging default inference kernels",
+ * section "Why Tencent HPC matters for online model serving": the KV-cache work
+ * is cut into smaller uniform tiles and assigned by the current workload, and
+ * the mapping is rebuilt as request lengths change during decoding.
  */
 DA_API int da_plan(const da_problem* prob, const da_plan_desc* desc, const int32_t* seq_lens, void* ws,
                    size_t ws_bytes, void* stream);
@@ -202,6 +245,11 @@ DA_API int da_plan(const da_problem* prob, const da_plan_desc* desc, const int32
  * With maxT = ceil(max_b L_b / T) and chunk = ceil(maxT / S) tiles, split s of
  * request b is CTA b*S+s and covers tiles [min(s*chunk, n_b), min((s+1)*chunk, n_b)),
  * empty when s*chunk >= n_b (the CTA is launched and finds nothing to do).
+ * Errors as for da_plan (a dynamic descriptor is DA_ERR_INVALID_ARG).
+ * Source: "Tencent HPC lands in SGLang, challenging default inference kernels",
+ * section "Why Tencent HPC matters for online model serving": the library's own
+ * static split-k baseline, a fixed split policy that either leaves units idle or
+ * launches empty chunks for short requests.
  */
 DA_API int da_static_plan(const da_problem* prob, const da_plan_desc* desc, const int32_t* seq_lens, void* ws,
                           size_t ws_bytes, void* stream);
@@ -213,7 +261,8 @@ DA_API int da_static_plan(const da_problem* prob, const da_plan_desc* desc, cons
  *   ws: dev, a plan made by da_plan / da_static_plan with the same descriptor
  *     and the same seq_lens contents.
  *   partial_o, partial_lse: dev scratch, sizes from da_workspace_size.
- *   out, lse: dev outputs.  Requests with one segment are written directly;
+ *   out, lse: dev outputs.  Requests with one segment are written directly
+ *     (with out_format DA_OUT_F32 they too go through the partials and da_combine);
  *     the others by da_combine, or, with merge_in_decode = 1, by the decode
  *     kernel: the last CTA to finish a segment of a split request (counters in
  *     `ws`, release/acquire fences, partials read back from L2) merges it, and
@@ -221,6 +270,17 @@ DA_API int da_static_plan(const da_problem* prob, const da_plan_desc* desc, cons
  * Each CTA streams its tiles' K and V rows (bf16, TMA, multi-stage shared
  * memory ring) and keeps, per query head of its KV group, the running max,
  * running sum and fp32 accumulator of the online softmax.
+ * Errors: DA_ERR_INVALID_ARG (null pointer; k_cache, v_cache, partial_o or ws
+ * not 16-byte aligned, q not 4-byte or out not 8-byte aligned; a descriptor
+ * that does not match the problem), DA_ERR_UNSUPPORTED (shape), DA_ERR_CUDA
+ * (tensor-map encoding or launch refused).  Data errors go to the status word
+ * in `ws` (DA_DEV_BAD_PAGE, DA_DEV_TIMEOUT, DA_DEV_BAD_PLAN when `ws` holds no
+ * plan for this descriptor).
+ * Source: "Tencent HPC lands in SGLang, challenging default inference kernels",
+ * section "Why Tencent HPC matters for online model serving": decode attention
+ * over each request's cached history, whose work is uneven because one request
+ * may hold a far longer context than another, and a longer history means more
+ * cached data to read; the CTAs take the uniform tiles the plan gives them.
  */
 DA_API int da_decode_attention(const da_problem* prob, const da_plan_desc* desc, const void* q,
                                const void* k_cache, const void* v_cache, const int32_t* block_table,
@@ -260,9 +320,41 @@ DA_API int da_decode_attention_fp8(const da_problem* prob, const da_plan_desc* d
  *   LSE = M + ln sum_i exp(lse_i - M),  M = max_i lse_i,
  *   out = sum_i exp(lse_i - LSE) o_i    (fp32 sums in a fixed order, then bf16),
  * and write out = 0, lse = -inf for requests with no segment.
+ *   ws, partial_o, partial_lse: dev, as written by da_plan / da_decode_attention
+ *     with the same descriptor; out, lse: dev outputs (out 8-byte aligned; 16-byte
+ *     aligned and fp32 with out_format DA_OUT_F32, in which case every request is
+ *     written here, those with one segment included).
+ * Errors: DA_ERR_INVALID_ARG (null or unaligned pointer, descriptor mismatch),
+ * DA_ERR_CUDA (launch refused).
+ * Source: "Tencent HPC lands in SGLang, challenging default inference kernels",
+ * section "Why Tencent HPC matters for online model serving": when one request's
+ * tiles go to several CTAs, each CTA holds a softmax over part of the history;
+ * the log-sum-exp merge that joins them is the exact re-association of one
+ * softmax (a fact of the arithmetic; the article names no merge).
  */
 DA_API int da_combine(const da_problem* prob, const da_plan_desc* desc, const void* ws, const float* partial_o,
                       const float* partial_lse, void* out, float* lse, void* stream);
+
+/*
+ * da_decode_step -- one whole decode step in one call: da_plan (or da_static_plan,
+ * per desc->kind), the decode (bf16 cache when k_scale and v_scale are NULL, FP8
+ * E4M3 cache with per-KV-head scales when both are given) and da_combine, enqueued
+ * on `stream` in that order.  Arguments, layouts, results and errors are those of
+ * the three calls; every check runs before the first launch.  Because the launch
+ * before the decode is then the planner, which writes only `ws`, each decode CTA
+ * (for batches up to 1024 requests) works out its first segment from seq_lens with
+ * the planner's formulas and requests that segment's first K/V chunks while the
+ * planner is still running, then checks the plan against it (a mismatch, which
+ * only a changed seq_lens could cause, is DA_DEV_BAD_PLAN).  The separate calls
+ * cannot do this, since they do not know what the caller enqueues between them.
+ * Source: "Tencent HPC lands in SGLang, challenging default inference kernels",
+ * section "Why Tencent HPC matters for online model serving" (the tile-to-CTA
+ * mapping is rebuilt every decode step; the step's work then runs on it).
+ */
+DA_API int da_decode_step(const da_problem* prob, const da_plan_desc* desc, const void* q, const void* k_cache,
+                          const void* v_cache, const float* k_scale, const float* v_scale,
+                          const int32_t* block_table, const int32_t* seq_lens, void* ws, size_t ws_bytes,
+                          float* partial_o, float* partial_lse, void* out, float* lse, void* stream);
 
 /*
  * da_decode_step_host -- one whole decode step for a caller whose per-step
@@ -367,8 +459,24 @@ DA_API int da_merge_partials(int32_t num_parts, int64_t rows, int32_t head_dim, 
                              const float* part_lse, void* out, float* lse, void* stream);
 
 /*
+ * da_merge_partials_f32 -- da_merge_partials over fp32 parts: part_out is dev fp32
+ * [num_parts][rows][head_dim] (16-byte aligned), each part being the `out` of a step
+ * run with out_format DA_OUT_F32, so that no part is rounded to bf16 before the
+ * merge; out is bf16 as for da_merge_partials.  Same formula, order, checks and
+ * errors.  Source: as for da_merge_partials.
+ */
+DA_API int da_merge_partials_f32(int32_t num_parts, int64_t rows, int32_t head_dim, const float* part_out,
+                                 const float* part_lse, void* out, float* lse, void* stream);
+
+/*
  * da_read_status -- copy the device status word and first bad index out of
- * `ws` (host outputs; either may be NULL).  Synchronises `stream`.
+ * `ws` (host outputs; either may be NULL).  Synchronises `stream`; the only
+ * call here that does.  Errors: DA_ERR_INVALID_ARG (ws NULL), DA_ERR_CUDA (the
+ * copy or the synchronisation failed).
+ * Source: "Tencent HPC lands in SGLang, challenging default inference kernels",
+ * section "What the 48.8% TPOT claim does not prove": serving kernels must cope
+ * with boundary shapes, cancellation and changing lengths, so bad lengths and
+ * page ids are skipped and reported here instead of faulting the device.
  */
 DA_API int da_read_status(const void* ws, int32_t* dev_status, int32_t* bad_index, void* stream);
 
@@ -411,24 +519,43 @@ DA_API int da_device_num_sms(int32_t* num_sms);
  * cudaMalloc (which may synchronise the device) is not acceptable.
  *   tile_tokens, num_ctas  as for da_plan_desc_init with DA_PLAN_DYNAMIC (0 = defaults).
  *   q, k_cache, v_cache, block_table, seq_lens, out, lse  dev, as for
- *     da_decode_attention; the caller still allocates inputs and outputs.
+ *     da_decode_attention (bf16 cache); the caller still allocates inputs and outputs.
  * Scratch: a static device array of DA_NOALLOC_SCRATCH_BYTES (16 MiB) inside
  * the library, reserved on every GPU that loads the library's device code and
  * held until the process exits.  A problem fits when the three sizes from
  * da_workspace_size, each rounded up to 256 bytes, sum to at most 16 MiB
  * (e.g. 64 query heads, head_dim 128, C = 37: C + B - 1 <= 507 segments, so
- * batches up to 471 requests); otherwise
- * the call returns DA_ERR_WORKSPACE and enqueues nothing.
+ * batches up to 471 requests); otherwise the call returns DA_ERR_WORKSPACE.
  * The first call on each device looks up the array's device address
  * (cudaGetSymbolAddress) with that device current; make that first call
- * before any stream capture.  All calls share the one array and each call
- * overwrites it, so calls that can overlap on the GPU (other streams, other
- * threads) race and must be serialised by the caller.  Errors as for
- * da_decode_attention.
+ * before any stream capture.  The lookup is made again when the device's
+ * context is no longer the one it was made in (after a cudaDeviceReset).
+ * All calls share the one array and each call overwrites it, so calls that
+ * can overlap on the GPU (other streams, other threads) race and must be
+ * serialised by the caller.
+ * Errors: every argument check, alignment rule and tensor map of the three
+ * launches is done before the first enqueue, so an error return has enqueued
+ * nothing, except DA_ERR_CUDA from a launch the CUDA runtime refused.  Codes
+ * as for da_plan and da_decode_attention, plus DA_ERR_WORKSPACE for a problem
+ * that does not fit the scratch.  Data errors found on the device (a bad
+ * length or page id, a wait that timed out) go to the status word inside the
+ * scratch: read them with da_noalloc_read_status before the next call.
  */
 DA_API int da_decode_step_noalloc(const da_problem* prob, int32_t tile_tokens, int32_t num_ctas, const void* q,
                                   const void* k_cache, const void* v_cache, const int32_t* block_table,
                                   const int32_t* seq_lens, void* out, float* lse, void* stream);
+
+/*
+ * da_noalloc_read_status -- da_read_status for the last da_decode_step_noalloc
+ * on the current device: the device status word and first bad index of that
+ * step (host outputs; either may be NULL).  Synchronises `stream`, which must
+ * be the step's stream (or one ordered after it).  The next call of
+ * da_decode_step_noalloc on the device overwrites the word (its plan resets
+ * it).  No counterpart in the article; it exists because the step's workspace
+ * is the library's own scratch, which the caller has no pointer to.
+ * Errors as for da_read_status.
+ */
+DA_API int da_noalloc_read_status(int32_t* dev_status, int32_t* bad_index, void* stream);
 
 #ifdef __cplusplus
 }

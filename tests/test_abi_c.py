@@ -30,6 +30,9 @@ int main(void) {
   CHECK(da_plan_desc_init(&p, DA_PLAN_DYNAMIC, 64, 37, &d) == DA_OK);
   CHECK(d.kind == DA_PLAN_DYNAMIC && d.batch == 32 && d.tile_tokens == 64 && d.num_ctas == 37);
   CHECK(d.splits == 0 && d.max_segments == 37 + 32 - 1 && d.num_kv_heads == 8 && d.merge_in_decode == 0);
+  CHECK(d.out_format == DA_OUT_BF16);
+  CHECK(da_plan_workspace_size(&p, 64, 37, &ws, &po, &pl) == DA_OK);
+  CHECK(po == (size_t)d.max_segments * 64 * 128 * 4);
   CHECK(da_workspace_size(&p, &d, &ws, &po, &pl) == DA_OK);
   CHECK(po == (size_t)d.max_segments * 64 * 128 * 4 && pl == (size_t)d.max_segments * 64 * 4);
   CHECK(ws % 16 == 0 && ws > 0);
@@ -38,6 +41,15 @@ int main(void) {
 
   CHECK(da_plan_desc_init(&p, DA_PLAN_STATIC, 32, 3, &s) == DA_OK);
   CHECK(s.kind == DA_PLAN_STATIC && s.num_ctas == 96 && s.splits == 3 && s.max_segments == 96);
+
+  /* fp32 output: every request goes through the combine, which cannot run inside the decode */
+  d.out_format = DA_OUT_F32;
+  CHECK(da_workspace_size(&p, &d, &ws, &po, &pl) == DA_OK);
+  d.merge_in_decode = 1;
+  CHECK(da_workspace_size(&p, &d, &ws, &po, &pl) == DA_ERR_INVALID_ARG);
+  d.merge_in_decode = 0; d.out_format = 2;
+  CHECK(da_workspace_size(&p, &d, &ws, &po, &pl) == DA_ERR_INVALID_ARG);
+  d.out_format = DA_OUT_BF16;
 
   /* argument checks: nothing is enqueued */
   CHECK(da_plan(&p, &s, (const int32_t*)16, (void*)256, 1 << 20, NULL) == DA_ERR_INVALID_ARG);

@@ -55,6 +55,29 @@ def test_plan_descriptor_and_sizes(da_lib):
     assert (s.kind, s.num_ctas, s.splits, s.max_segments, s.tile_tokens) == (1, 96, 3, 96, 32)
     d0 = da.da_plan_desc_init(p, da.PLAN_DYNAMIC, 0, 5)
     assert d0.tile_tokens == 64
+    # the one-call size query is the descriptor's sizes
+    assert da.da_plan_workspace_size(p, 64, 37) == (ws, po, pl)
+    assert da.da_plan_workspace_size(p, 32, 5) == da.da_workspace_size(p, da.da_plan_desc_init(p, da.PLAN_DYNAMIC,
+                                                                                                 32, 5))
+    with pytest.raises(da.DaError) as e:
+        da.da_plan_workspace_size(prob(da, head_dim=96), 64, 37)
+    assert e.value.code == da.ERR_UNSUPPORTED
+
+
+def test_noalloc_scratch_limit_boundary(da_lib):
+    """The documented limit of the no-allocation step at 64 query heads, d 128, C = 37: 471 requests
+    fit the 16 MiB scratch, 472 do not.  With null buffers the first passes the size check and stops
+    at the pointer check; the second is refused for size first."""
+    import ctypes
+    da = da_lib
+    sizes = {}
+    for B in (471, 472):
+        p = prob(da, batch=B)
+        ws, po, pl = da.da_plan_workspace_size(p, 64, 37)
+        sizes[B] = sum((x + 255) // 256 * 256 for x in (ws, po, pl))
+        rc = da.lib().da_decode_step_noalloc(ctypes.byref(p), 64, 37, *([None] * 7), None)
+        assert rc == (da.ERR_INVALID_ARG if B == 471 else da.ERR_WORKSPACE), (B, rc)
+    assert sizes[471] <= da.NOALLOC_SCRATCH_BYTES < sizes[472]
 
 
 @pytest.mark.parametrize("kw,code", [
@@ -97,6 +120,21 @@ def test_descriptor_checks(da_lib):
     assert lib.da_combine(None, ctypes.byref(d), *([None] * 5), None) == -1
     assert lib.da_read_status(None, None, None, None) == -1
     assert lib.da_workspace_offsets(None, None) == -1
+    # output format: bf16 by default; fp32 is allowed with the combine kernel only
+    assert d.out_format == da.OUT_BF16
+    f = da.da_plan_desc_init(p, da.PLAN_DYNAMIC, 64, 37, out_f32=True)
+    assert da.da_workspace_size(p, f) == da.da_workspace_size(p, d)
+    for merge, fmt in ((1, da.OUT_F32), (0, 2), (0, -1)):
+        bad = da.da_plan_desc_init(p, da.PLAN_DYNAMIC, 64, 37)
+        bad.merge_in_decode, bad.out_format = merge, fmt
+        assert lib.da_workspace_size(ctypes.byref(p), ctypes.byref(bad), None, None, None) == -1
+    # fp32 output must be 16-byte aligned (the combine stores four floats at a time)
+    A = 1 << 12
+    assert lib.da_combine(ctypes.byref(p), ctypes.byref(f), A, A, A, A + 8, A, None) == -1
+    assert lib.da_decode_attention(ctypes.byref(p), ctypes.byref(f), A, A, A, A, A, A, A, A, A + 8, A, None) == -1
+    assert lib.da_merge_partials_f32(2, 10, 128, A + 8, A, A, A, None) == -1
+    assert lib.da_merge_partials_f32(2, 10, 96, A, A, A, A, None) == -2
+    assert lib.da_merge_partials_f32(2, 0, 128, None, None, None, None, None) == 0
 
 
 def test_host_step_checks(da_lib):

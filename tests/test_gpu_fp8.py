@@ -50,7 +50,7 @@ def test_fp8_head_dim_64_is_refused(da_lib):
     assert e.value.code == da.ERR_UNSUPPORTED
 
 
-@pytest.mark.parametrize("name", ["mixed", "skewed"])
+@pytest.mark.parametrize("name", ["mixed", "skewed", "low_conc", "uniform"])
 def test_fp8_full_size(da_lib, oracle_lib, name):
     w8 = W.quantize_fp8(W.CONFIGS[name]())
     out, lse, desc, bufs, _ = run_step_fp8(w8)

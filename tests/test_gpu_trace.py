@@ -2,9 +2,11 @@
 
 The plan is rebuilt on the device every step and checked bit-exactly against
 the oracle's plan at every step; attention outputs are checked against the
-fp64 oracle on every (request, head) at steps 0, 1, 127 and 255; at the end the
-device cache, written step by step by da_append_kv, must equal the host cache
-bit for bit at every live token.
+fp64 oracle on every (request, head) at steps 0, 1, 127 and 255, and the same
+two ends of the trace (steps 0 and 255) run once more over an FP8 E4M3 copy of
+the cache (the tensor-core kernel) against the FP8 oracle; at the end the device
+cache, written step by step by da_append_kv, must equal the host cache bit for
+bit at every live token.
 """
 
 import numpy as np
@@ -12,7 +14,7 @@ import pytest
 import torch
 
 import oracle
-from gpu_helpers import assert_plan_equal, check_against_oracle
+from gpu_helpers import assert_plan_equal, check_against_oracle, check_against_oracle_fp8, run_step_fp8
 from variable_length_paged_b200 import da
 from variable_length_paged_b200 import workloads as W
 from variable_length_paged_b200.trace import DeviceTrace
@@ -76,6 +78,12 @@ def test_decode_trace_256_steps(da_lib, oracle_lib):
         assert_plan_equal(da.read_plan(desc, bufs.ws), oracle.plan(tr.seq_lens, 64, desc.num_ctas, cap))
         if t in (0, 1, 127, 255):
             check_against_oracle(tr.workload(), bufs.out, bufs.lse)
+        if t in (0, tr.steps - 1):  # the trace's batch at both ends, over an FP8 copy of its cache
+            w8 = W.quantize_fp8(tr.workload())
+            out8, lse8, _, bufs8, _ = run_step_fp8(w8)
+            assert da.da_read_status(bufs8.ws) == (0, -1)
+            check_against_oracle_fp8(w8, out8, lse8)
+            del out8, lse8, bufs8, w8
     assert dt.status.tolist() == [0, 0]
     assert da.da_read_status(bufs.ws) == (0, -1)
     # the device cache, built step by step by the append kernel, equals the host cache at live tokens

@@ -3,11 +3,12 @@
 Rank r of W holds a contiguous, page-aligned slice of every request's pages:
 pages [floor(r*n/W), floor((r+1)*n/W)) of the request's n = ceil(L/P) pages.
 Each rank runs the ordinary decode step (plan, decode, combine) on its slice,
-producing (out_r, lse_r); softmax over disjoint token sets merges exactly by
-log-sum-exp, so after an all-gather of the partial results every rank merges
-them with da_merge_partials.  The exchange is B * Hq * (d * 2 + 4) bytes per
-rank and step.  Plain decode only (q_len = 1): the query is the last token and
-sees every slice whole.
+producing (out_r, lse_r) in fp32 (the step runs with fp32 output, so no rank's
+result is rounded to bf16 before the merge); softmax over disjoint token sets
+merges exactly by log-sum-exp, so after an all-gather of the partial results
+every rank merges them with da_merge_partials_f32, which rounds once, at the
+end.  The exchange is B * Hq * (d + 1) * 4 bytes per rank and step.  Plain
+decode only (q_len = 1): the query is the last token and sees every slice whole.
 
 Source of the method: "Tencent HPC lands in SGLang, challenging default
 inference kernels", section "Why Tencent HPC matters for online model serving"
@@ -46,6 +47,7 @@ def cp_decode_step(prob, desc, q, k_cache, v_cache, local_block_table, local_seq
                    out: torch.Tensor, lse: torch.Tensor, group=None, stream=None):
     """Decode step on this rank's slice, all-gather of the partial results, log-sum-exp merge.
 
+    `desc` must ask for fp32 output (da_plan_desc_init(..., out_f32=True)), and `bufs` be made for it;
     `out` [B, Hq, d] bf16 and `lse` [B, Hq] fp32 receive the merged result on every rank.
     """
     import contextlib
@@ -54,6 +56,8 @@ def cp_decode_step(prob, desc, q, k_cache, v_cache, local_block_table, local_seq
 
     if prob.q_len > 1:
         raise ValueError("context-parallel decode handles one query per request")
+    if desc.out_format != da.OUT_F32 or bufs.out.dtype != torch.float32:
+        raise ValueError("context-parallel decode exchanges fp32 results: build desc with out_f32=True")
     # the collectives order themselves after the current stream's work: make `stream` current so that
     # the all-gather follows this rank's decode and the merge follows the all-gather
     on_stream = torch.cuda.stream(stream) if stream is not None else contextlib.nullcontext()
@@ -64,5 +68,5 @@ def cp_decode_step(prob, desc, q, k_cache, v_cache, local_block_table, local_seq
         parts_lse = torch.empty((world,) + tuple(bufs.lse.shape), dtype=bufs.lse.dtype, device=bufs.lse.device)
         dist.all_gather_into_tensor(parts_out, bufs.out, group=group)
         dist.all_gather_into_tensor(parts_lse, bufs.lse, group=group)
-        da.da_merge_partials(parts_out, parts_lse, out, lse, stream=stream)
+        da.da_merge_partials_f32(parts_out, parts_lse, out, lse, stream=stream)
     return out, lse

@@ -9,7 +9,9 @@
 
 #include "append_rows.cuh"
 #include "da_internal.cuh"
+#include "early_start.cuh"
 #include "host_inputs.cuh"
+#include "prepared_step.cuh"
 
 namespace {
 
@@ -51,6 +53,8 @@ int check_desc(const da_problem* p, const da_plan_desc* d) {
     return DA_ERR_INVALID_ARG;
   if (d->num_kv_heads != p->num_kv_heads || (d->merge_in_decode != 0 && d->merge_in_decode != 1))
     return DA_ERR_INVALID_ARG;
+  if (d->out_format != DA_OUT_BF16 && d->out_format != DA_OUT_F32) return DA_ERR_INVALID_ARG;
+  if (d->out_format == DA_OUT_F32 && d->merge_in_decode) return DA_ERR_INVALID_ARG;  // the combine writes fp32 out
   if (d->kind == DA_PLAN_DYNAMIC) {
     if (d->splits != 0 || (int64_t)d->max_segments != (int64_t)d->num_ctas + (p->batch > 0 ? p->batch : 1) - 1)
       return DA_ERR_INVALID_ARG;
@@ -160,6 +164,7 @@ DA_API int da_plan_desc_init(const da_problem* prob, int32_t kind, int32_t tile_
   d.tile_tokens = T;
   d.num_kv_heads = prob->num_kv_heads;
   d.merge_in_decode = 0;
+  d.out_format = DA_OUT_BF16;
   if (kind == DA_PLAN_DYNAMIC) {
     d.num_ctas = w;
     d.splits = 0;
@@ -191,6 +196,13 @@ DA_API int da_workspace_size(const da_problem* prob, const da_plan_desc* desc, s
   if (partial_o_bytes) *partial_o_bytes = (size_t)desc->max_segments * rows * prob->head_dim * 4;
   if (partial_lse_bytes) *partial_lse_bytes = (size_t)desc->max_segments * rows * 4;
   return DA_OK;
+}
+
+DA_API int da_plan_workspace_size(const da_problem* prob, int32_t tile_tokens, int32_t num_ctas, size_t* ws_bytes,
+                                  size_t* partial_o_bytes, size_t* partial_lse_bytes) {
+  da_plan_desc d;
+  const int rc = da_plan_desc_init(prob, DA_PLAN_DYNAMIC, tile_tokens, num_ctas, &d);
+  return rc != DA_OK ? rc : da_workspace_size(prob, &d, ws_bytes, partial_o_bytes, partial_lse_bytes);
 }
 
 DA_API int da_workspace_offsets(const da_plan_desc* desc, int64_t off[7]) {
@@ -263,8 +275,9 @@ static int decode_prepare(const da_problem* prob, const da_plan_desc* desc, cons
   if (!q || !k_cache || !v_cache || !block_table || !seq_lens || !ws || !partial_o || !partial_lse || !out || !lse)
     return DA_ERR_INVALID_ARG;
   if (fp8 && (!k_scale || !v_scale)) return DA_ERR_INVALID_ARG;
+  const bool out_f32 = desc->out_format == DA_OUT_F32;
   if (reinterpret_cast<uintptr_t>(k_cache) % 16 != 0 || reinterpret_cast<uintptr_t>(v_cache) % 16 != 0 ||
-      reinterpret_cast<uintptr_t>(q) % (fp8 ? 8 : 4) != 0 || reinterpret_cast<uintptr_t>(out) % 8 != 0 ||
+      reinterpret_cast<uintptr_t>(q) % (fp8 ? 8 : 4) != 0 || reinterpret_cast<uintptr_t>(out) % (out_f32 ? 16 : 8) != 0 ||
       reinterpret_cast<uintptr_t>(partial_o) % 16 != 0 || reinterpret_cast<uintptr_t>(ws) % 16 != 0)
     return DA_ERR_INVALID_ARG;
   const int eb = fp8 ? 1 : 2;
@@ -300,6 +313,8 @@ static int decode_prepare(const da_problem* prob, const da_plan_desc* desc, cons
   // (query, head) rows over all 16 MMA rows; plain decode with G <= 8 uses the upper 8
   p.full_rows = (p.q_len > 1 || p.group > 8) ? 1 : 0;
   p.merge_in_decode = desc->merge_in_decode;
+  p.out_f32 = out_f32 ? 1 : 0;
+  p.early = 0;  // set by the callers that launch the planner just before
   p.stall_producer = g_stall_next_ns != 0 ? 1 : 0;
   p.wait_limit_ns = g_stall_next_ns != 0 ? g_stall_next_ns : kWaitLimitNs;
   g_stall_next_ns = 0;  // one launch only
@@ -355,14 +370,21 @@ DA_API int da_decode_attention_fp8(const da_problem* prob, const da_plan_desc* d
                        partial_lse, out, lse, stream, true);
 }
 
+DA_API int da_decode_step(const da_problem* prob, const da_plan_desc* desc, const void* q, const void* k_cache,
+                          const void* v_cache, const float* k_scale, const float* v_scale,
+                          const int32_t* block_table, const int32_t* seq_lens, void* ws, size_t ws_bytes,
+                          float* partial_o, float* partial_lse, void* out, float* lse, void* stream);
+
 // Checks a combine call and fills its kernel parameters; enqueues nothing.
 // Call only with batch > 0.
 static int combine_prepare(const da_problem* prob, const da_plan_desc* desc, const void* ws,
                            const float* partial_o, const float* partial_lse, void* out, float* lse,
                            da::CombineParams* p) {
   if (!ws || !partial_o || !partial_lse || !out || !lse) return DA_ERR_INVALID_ARG;
-  if (reinterpret_cast<uintptr_t>(partial_o) % 16 != 0 || reinterpret_cast<uintptr_t>(out) % 8 != 0)
+  const bool out_f32 = desc->out_format == DA_OUT_F32;
+  if (reinterpret_cast<uintptr_t>(partial_o) % 16 != 0 || reinterpret_cast<uintptr_t>(out) % (out_f32 ? 16 : 8) != 0)
     return DA_ERR_INVALID_ARG;
+  p->out_f32 = out_f32 ? 1 : 0;
   p->ws = static_cast<const int32_t*>(ws);
   p->partial_o = partial_o;
   p->partial_lse = partial_lse;
@@ -392,6 +414,37 @@ DA_API int da_combine(const da_problem* prob, const da_plan_desc* desc, const vo
   da::CombineParams p;
   rc = combine_prepare(prob, desc, ws, partial_o, partial_lse, out, lse, &p);
   return rc != DA_OK ? rc : combine_launch(p, desc, prob->head_dim, stream);
+}
+
+DA_API int da_decode_step(const da_problem* prob, const da_plan_desc* desc, const void* q, const void* k_cache,
+                          const void* v_cache, const float* k_scale, const float* v_scale,
+                          const int32_t* block_table, const int32_t* seq_lens, void* ws, size_t ws_bytes,
+                          float* partial_o, float* partial_lse, void* out, float* lse, void* stream) {
+  int rc = check_problem(prob);
+  if (rc != DA_OK) return rc;
+  rc = check_desc(prob, desc);
+  if (rc != DA_OK) return rc;
+  if ((k_scale == nullptr) != (v_scale == nullptr)) return DA_ERR_INVALID_ARG;
+  const bool fp8 = k_scale != nullptr;
+  if (fp8 && prob->head_dim != 128) return DA_ERR_UNSUPPORTED;
+  da::PlanParams pp;
+  rc = plan_prepare(prob, desc, seq_lens, ws, ws_bytes, desc->kind, &pp);
+  if (rc != DA_OK) return rc;
+  if (prob->batch == 0) return plan_launch(pp, desc->kind, stream);
+  da::DecodeParams dp;
+  CUtensorMap maps[4];
+  rc = decode_prepare(prob, desc, q, k_cache, v_cache, k_scale, v_scale, block_table, seq_lens, ws, partial_o,
+                      partial_lse, out, lse, fp8, &dp, maps);
+  if (rc != DA_OK) return rc;
+  dp.early = prob->batch <= da::kEarlyMaxBatch ? 1 : 0;  // the planner is the launch just before
+  da::CombineParams cp;
+  rc = combine_prepare(prob, desc, ws, partial_o, partial_lse, out, lse, &cp);
+  if (rc != DA_OK) return rc;
+  rc = plan_launch(pp, desc->kind, stream);
+  if (rc != DA_OK) return rc;
+  rc = decode_launch(dp, prob->head_dim, maps, fp8, stream);
+  if (rc != DA_OK) return rc;
+  return combine_launch(cp, desc, prob->head_dim, stream);
 }
 
 // The device address of host memory that kernels may use in place (page-locked and mapped
@@ -426,6 +479,7 @@ DA_API int da_decode_step_host(const da_problem* prob, const da_plan_desc* desc,
   const size_t B = (size_t)prob->batch;
   const size_t rows = B * (size_t)q_len_of(prob) * (size_t)prob->num_q_heads;
   const size_t q_bytes = rows * (size_t)prob->head_dim * 2;
+  const size_t out_bytes = rows * (size_t)prob->head_dim * (desc->out_format == DA_OUT_F32 ? 4 : 2);
   const size_t bt_bytes = B * (size_t)prob->max_pages_per_req * 4;
   // Inputs in mapped page-locked memory need no copy call.  The plan launch brings them in:
   // block 0 reads the lengths and plans, the other blocks copy the block table and a small q
@@ -482,13 +536,15 @@ DA_API int da_decode_step_host(const da_problem* prob, const da_plan_desc* desc,
     if (e != cudaSuccess) return cuda_fail(e);
     rc = plan_launch(pp, desc->kind, stream);
     if (rc != DA_OK) return rc;
+    // the copies are complete before the planner starts, and the planner writes only `ws`
+    dp.early = prob->batch <= da::kEarlyMaxBatch ? 1 : 0;
   }
   rc = decode_launch(dp, prob->head_dim, maps, fp8, stream);
   if (rc != DA_OK) return rc;
   rc = combine_launch(cp, desc, prob->head_dim, stream);
   if (rc != DA_OK) return rc;
   e = cudaSuccess;
-  if (!out_map) e = cudaMemcpyAsync(out_host, out_dev, q_bytes, cudaMemcpyDeviceToHost, s);
+  if (!out_map) e = cudaMemcpyAsync(out_host, out_dev, out_bytes, cudaMemcpyDeviceToHost, s);
   if (e == cudaSuccess && !lse_map) e = cudaMemcpyAsync(lse_host, lse_dev, rows * 4, cudaMemcpyDeviceToHost, s);
   return e == cudaSuccess ? DA_OK : cuda_fail(e);
 }
@@ -545,16 +601,17 @@ DA_API int da_plan_append(const da_problem* prob, const da_plan_desc* desc, cons
   return e == cudaSuccess ? DA_OK : cuda_fail(e);
 }
 
-DA_API int da_merge_partials(int32_t num_parts, int64_t rows, int32_t head_dim, const void* part_out,
-                             const float* part_lse, void* out, float* lse, void* stream) {
+static int merge_common(int32_t num_parts, int64_t rows, int32_t head_dim, const void* part_out, bool f32,
+                        const float* part_lse, void* out, float* lse, void* stream) {
   if (num_parts <= 0 || rows < 0) return DA_ERR_INVALID_ARG;
   if (head_dim != 64 && head_dim != 128) return DA_ERR_UNSUPPORTED;
   if (rows == 0) return DA_OK;
   if (!part_out || !part_lse || !out || !lse) return DA_ERR_INVALID_ARG;
-  if (reinterpret_cast<uintptr_t>(part_out) % 8 != 0 || reinterpret_cast<uintptr_t>(out) % 8 != 0)
+  if (reinterpret_cast<uintptr_t>(part_out) % (f32 ? 16 : 8) != 0 || reinterpret_cast<uintptr_t>(out) % 8 != 0)
     return DA_ERR_INVALID_ARG;
   da::MergeParams p;
-  p.part_out = static_cast<const __nv_bfloat16*>(part_out);
+  p.part_out = f32 ? nullptr : static_cast<const __nv_bfloat16*>(part_out);
+  p.part_out_f32 = f32 ? static_cast<const float*>(part_out) : nullptr;
   p.part_lse = part_lse;
   p.out = static_cast<__nv_bfloat16*>(out);
   p.lse = lse;
@@ -562,6 +619,16 @@ DA_API int da_merge_partials(int32_t num_parts, int64_t rows, int32_t head_dim, 
   p.rows = rows;
   cudaError_t e = da::launch_merge(p, head_dim, static_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? DA_OK : cuda_fail(e);
+}
+
+DA_API int da_merge_partials(int32_t num_parts, int64_t rows, int32_t head_dim, const void* part_out,
+                             const float* part_lse, void* out, float* lse, void* stream) {
+  return merge_common(num_parts, rows, head_dim, part_out, false, part_lse, out, lse, stream);
+}
+
+DA_API int da_merge_partials_f32(int32_t num_parts, int64_t rows, int32_t head_dim, const float* part_out,
+                                 const float* part_lse, void* out, float* lse, void* stream) {
+  return merge_common(num_parts, rows, head_dim, part_out, true, part_lse, out, lse, stream);
 }
 
 DA_API int da_read_status(const void* ws, int32_t* dev_status, int32_t* bad_index, void* stream) {
@@ -599,3 +666,37 @@ DA_API const char* da_dev_status_string(int32_t code) {
 }
 
 }  // extern "C"
+
+namespace da {
+
+// Every check and parameter block of a dynamic step (plan, bf16 decode, combine) on device
+// buffers, before anything is enqueued; launch_prepared_step then only enqueues.
+int prepare_dynamic_step(const da_problem* prob, const da_plan_desc* desc, const void* q, const void* k_cache,
+                         const void* v_cache, const int32_t* block_table, const int32_t* seq_lens, void* ws,
+                         size_t ws_bytes, float* partial_o, float* partial_lse, void* out, float* lse,
+                         PreparedStep* st) {
+  int rc = check_problem(prob);
+  if (rc != DA_OK) return rc;
+  rc = check_desc(prob, desc);
+  if (rc != DA_OK) return rc;
+  st->batch = prob->batch;
+  st->head_dim = prob->head_dim;
+  st->desc = *desc;
+  rc = plan_prepare(prob, desc, seq_lens, ws, ws_bytes, DA_PLAN_DYNAMIC, &st->plan);
+  if (rc != DA_OK || prob->batch == 0) return rc;
+  rc = decode_prepare(prob, desc, q, k_cache, v_cache, nullptr, nullptr, block_table, seq_lens, ws, partial_o,
+                      partial_lse, out, lse, false, &st->decode, st->maps);
+  if (rc != DA_OK) return rc;
+  st->decode.early = prob->batch <= kEarlyMaxBatch ? 1 : 0;  // launch_prepared_step plans just before
+  return combine_prepare(prob, desc, ws, partial_o, partial_lse, out, lse, &st->combine);
+}
+
+int launch_prepared_step(const PreparedStep& st, void* stream) {
+  int rc = plan_launch(st.plan, DA_PLAN_DYNAMIC, stream);
+  if (rc != DA_OK || st.batch == 0) return rc;
+  rc = decode_launch(st.decode, st.head_dim, st.maps, false, stream);
+  if (rc != DA_OK) return rc;
+  return combine_launch(st.combine, &st.desc, st.head_dim, stream);
+}
+
+}  // namespace da

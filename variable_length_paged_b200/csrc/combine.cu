@@ -5,8 +5,9 @@
 // so the full result is
 //   LSE = M + ln sum_i exp(lse_i - M),   M = max_i lse_i
 //   out = sum_i exp(lse_i - LSE) * o_i
-// Requests with one segment were written by the decode kernel; requests with
-// none get out = 0, lse = -inf.
+// Requests with one segment were written by the decode kernel (with fp32
+// output they are merged here too, from their one partial); requests with none
+// get out = 0, lse = -inf.
 //
 // One 128-thread block per (request, query head), one pass over the partials:
 // warp w takes segments w, w+4, w+8, ... (lse and the lane's head_dim/32 columns
@@ -32,7 +33,7 @@ __global__ void __launch_bounds__(128) combine_kernel(const CombineParams p) {
   const int32_t* rsb = p.ws + WL.req_seg_begin;
   const int s0 = rsb[b], s1 = rsb[b + 1];
   const int n = s1 - s0;
-  if (n == 1) return;  // written by the decode kernel (uniform over the block)
+  if (n == 1 && !p.out_f32) return;  // written by the decode kernel (uniform over the block)
   const bool ok = s0 >= 0 && s1 <= p.max_segments && n >= 0;
   const int64_t hq = p.num_q_heads;
   const float* plse = p.partial_lse + (int64_t)s0 * hq + h;
@@ -92,12 +93,20 @@ __global__ void __launch_bounds__(128) combine_kernel(const CombineParams p) {
   }
   const float inv = L > 0.f ? 1.f / L : 0.f;
   const float total = L > 0.f ? M + logf(L) : -INFINITY;
-  __nv_bfloat16* dst = p.out + ((int64_t)b * hq + h) * D + lane * kPer;
-  if constexpr (kPer == 4) {
-    *reinterpret_cast<uint2*>(dst) =
-        make_uint2(pack_bf16x2(o[0] * inv, o[1] * inv), pack_bf16x2(o[2] * inv, o[3] * inv));
+  if (p.out_f32) {
+    float* dst = reinterpret_cast<float*>(p.out) + ((int64_t)b * hq + h) * D + lane * kPer;
+    if constexpr (kPer == 4)
+      *reinterpret_cast<float4*>(dst) = make_float4(o[0] * inv, o[1] * inv, o[2] * inv, o[3] * inv);
+    else
+      *reinterpret_cast<float2*>(dst) = make_float2(o[0] * inv, o[1] * inv);
   } else {
-    *reinterpret_cast<uint32_t*>(dst) = pack_bf16x2(o[0] * inv, o[1] * inv);
+    __nv_bfloat16* dst = p.out + ((int64_t)b * hq + h) * D + lane * kPer;
+    if constexpr (kPer == 4) {
+      *reinterpret_cast<uint2*>(dst) =
+          make_uint2(pack_bf16x2(o[0] * inv, o[1] * inv), pack_bf16x2(o[2] * inv, o[3] * inv));
+    } else {
+      *reinterpret_cast<uint32_t*>(dst) = pack_bf16x2(o[0] * inv, o[1] * inv);
+    }
   }
   if (lane == 0) p.lse[(int64_t)b * hq + h] = total;
 }

@@ -77,6 +77,9 @@ struct DecodeParams {
   int32_t merge_in_decode;  // 1: the last CTA to finish a request's segment merges its partials
   int32_t stall_producer;   // failure-path test: the producer sends nothing, so every wait runs out
   uint64_t wait_limit_ns;   // limit of every pipeline wait
+  int32_t out_f32;          // 1: every segment's result goes to the partials (the combine writes fp32 out)
+  int32_t early;            // 1: the launch before is the planner alone, so the CTA may request its
+                            //    first chunks (derived from seq_lens) before the plan has landed
 };
 
 struct CombineParams {
@@ -86,6 +89,7 @@ struct CombineParams {
   __nv_bfloat16* out;
   float* lse;
   int32_t batch, num_q_heads, num_ctas, max_segments, num_kv_heads;
+  int32_t out_f32;  // 1: out is fp32 and every request is written (one segment too)
 };
 
 struct AppendParams {
@@ -101,7 +105,8 @@ struct AppendParams {
 };
 
 struct MergeParams {
-  const __nv_bfloat16* part_out;  // [num_parts][rows][head_dim]
+  const __nv_bfloat16* part_out;  // [num_parts][rows][head_dim] (bf16 parts)
+  const float* part_out_f32;      // or fp32 parts (exactly one of the two is set)
   const float* part_lse;          // [num_parts][rows]
   __nv_bfloat16* out;             // [rows][head_dim]
   float* lse;                     // [rows]

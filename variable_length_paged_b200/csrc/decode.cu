@@ -52,6 +52,7 @@
 #include <cfloat>
 
 #include "da_internal.cuh"
+#include "early_start.cuh"
 
 namespace da {
 namespace {
@@ -171,6 +172,166 @@ __device__ void merge_request_rows(const DecodeParams& p, int b, int g, int s0, 
   }
 }
 
+#if DA_BF16_FFMA
+// CUDA-core (FFMA) consumer for plain bf16 decode at head_dim 128, built only with
+// -DDA_BF16_FFMA=1: the comparison point for the warp-level MMA consumer (same grid,
+// producer, ring, plan and outputs).  Lane (h, qd) = (lane / 4, lane % 4) owns head h of
+// the group and dims 32 qd .. 32 qd + 31.  Per token of its warp's 16 rows it dots q with
+// the K row over its dims in fp32 (two shuffles finish the dot product), keeps head h's
+// online softmax, and accumulates P.V over its 32 dims; P is not rounded.  The four warp
+// states merge at segment end as in the MMA consumer.
+template <typename C>
+__device__ void ffma_consumer(const DecodeParams& p, uint8_t* smem, const int4* segs, const int32_t* rsb,
+                              int32_t* hdr_w, uint32_t full0, uint32_t empty0, volatile int* meta,
+                              volatile int* abort_flag, int seg_lo, int seg_hi, int g, int w, int lane) {
+  constexpr int D = 128, TPW = C::kTPW, HS = C::kHalfStride;
+  static_assert(C::kElemBytes == 2 && C::kRowBytes == 256 && TPW == 16, "bf16, head_dim 128");
+  const int h = lane >> 2, qd = lane & 3;
+  const bool live = h < p.group;
+  float* slots = reinterpret_cast<float*>(smem + C::kOffSlots);
+  float* ml = reinterpret_cast<float*>(smem + C::kOffML);
+  int stage = 0;
+  uint32_t phase = 0;
+  for (int s = seg_lo; s < seg_hi; ++s) {
+    const SegmentInfo si = load_segment(p, segs, s);
+    if (!si.valid) continue;
+    const int b = si.b;
+    float qf[32];  // q of head h, dims 32 qd .., scaled to base-2 scores
+    {
+      const uint32_t* src = reinterpret_cast<const uint32_t*>(
+          p.q + ((int64_t)b * p.num_q_heads + (int64_t)g * p.group + (live ? h : 0)) * D + 32 * qd);
+#pragma unroll
+      for (int j = 0; j < 16; ++j) {
+        const uint32_t u = live ? __ldg(src + j) : 0u;
+        qf[2 * j] = bf16_lo_to_f32(u) * p.scale_log2;
+        qf[2 * j + 1] = bf16_hi_to_f32(u) * p.scale_log2;
+      }
+    }
+    float m = -INFINITY, l = 0.f, acc[32];
+#pragma unroll
+    for (int e = 0; e < 32; ++e) acc[e] = 0.f;
+    for (int c0 = si.tok0; c0 < si.tok1; c0 += C::kChunk) {
+      const bool got = mbar_wait_bounded(full0 + 8 * stage, phase, abort_flag, p.wait_limit_ns);
+      if (!got && lane == 0) {
+        if (!*abort_flag) record_status(hdr_w, DA_DEV_TIMEOUT, s);
+        *abort_flag = 1;
+      }
+      const int n = got ? meta[stage] : 0;
+      const int nw = min(max(n - TPW * w, 0), TPW);
+      const uint8_t* kt = smem + C::kOffStages + stage * C::kStageBytes;
+      const uint8_t* vt = kt + C::kTileBytes;
+      if (nw > 0) {
+        float sc[TPW];
+#pragma unroll
+        for (int tt = 0; tt < TPW; ++tt) {
+          const int row = TPW * w + tt;
+          float a = 0.f;
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            const uint4 u = *reinterpret_cast<const uint4*>(kt + swz<HS>(row, 4 * qd + j));
+            const uint32_t uw[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+              a = fmaf(qf[8 * j + 2 * k], bf16_lo_to_f32(uw[k]), a);
+              a = fmaf(qf[8 * j + 2 * k + 1], bf16_hi_to_f32(uw[k]), a);
+            }
+          }
+          a += __shfl_xor_sync(0xffffffffu, a, 1);
+          a += __shfl_xor_sync(0xffffffffu, a, 2);
+          sc[tt] = tt < nw ? a : -INFINITY;  // rows past the loaded tokens may hold anything
+        }
+        float mx = sc[0];
+#pragma unroll
+        for (int tt = 1; tt < TPW; ++tt) mx = fmaxf(mx, sc[tt]);
+        const float m_new = fmaxf(m, mx);
+        const float m_use = m_new == -INFINITY ? 0.f : m_new;
+        const float corr = fast_exp2(m - m_use);
+        l *= corr;
+#pragma unroll
+        for (int e = 0; e < 32; ++e) acc[e] *= corr;
+#pragma unroll
+        for (int tt = 0; tt < TPW; ++tt) {
+          if (tt >= nw) break;
+          const float pt = fast_exp2(sc[tt] - m_use);
+          l += pt;
+          const int row = TPW * w + tt;
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            const uint4 u = *reinterpret_cast<const uint4*>(vt + swz<HS>(row, 4 * qd + j));
+            const uint32_t uw[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+              acc[8 * j + 2 * k] = fmaf(pt, bf16_lo_to_f32(uw[k]), acc[8 * j + 2 * k]);
+              acc[8 * j + 2 * k + 1] = fmaf(pt, bf16_hi_to_f32(uw[k]), acc[8 * j + 2 * k + 1]);
+            }
+          }
+        }
+        m = m_new;
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(empty0 + 8 * stage);
+      if (++stage == C::kStages) {
+        stage = 0;
+        phase ^= 1;
+      }
+    }
+    // ---- merge the four warp states of this segment (head h, dims 32 qd ..)
+    const bool direct = rsb[b + 1] - rsb[b] == 1 && !p.out_f32;
+    if (w > 0) {
+      float* slot = slots + (w - 1) * C::kSlotFloats + h * C::kSlotStride + 32 * qd;
+#pragma unroll
+      for (int e = 0; e < 32; e += 4) *reinterpret_cast<float4*>(slot + e) = make_float4(acc[e], acc[e + 1], acc[e + 2], acc[e + 3]);
+      if (qd == 0) {
+        ml[(w - 1) * 24 + h] = m;
+        ml[(w - 1) * 24 + 8 + h] = l;
+      }
+    }
+    named_barrier_sync(1, kConsumerWarps * 32);
+    if (w == 0) {
+      float M = m, mw[3], lw[3];
+#pragma unroll
+      for (int j = 0; j < 3; ++j) {
+        mw[j] = ml[j * 24 + h];
+        lw[j] = ml[j * 24 + 8 + h];
+        M = fmaxf(M, mw[j]);
+      }
+      const bool empty = M == -INFINITY;
+      const float f0 = empty ? 0.f : fast_exp2(m - M);
+      float L = f0 * l, fw[3];
+#pragma unroll
+      for (int j = 0; j < 3; ++j) {
+        fw[j] = empty ? 0.f : fast_exp2(mw[j] - M);
+        L += fw[j] * lw[j];
+      }
+      const float inv = L > 0.f ? 1.f / L : 0.f;
+      const float lse_nat = L > 0.f ? (M + log2f(L)) * 0.69314718055994530942f : -INFINITY;
+#pragma unroll
+      for (int e = 0; e < 32; ++e) {
+        float a = f0 * acc[e];
+#pragma unroll
+        for (int j = 0; j < 3; ++j) a += fw[j] * slots[j * C::kSlotFloats + h * C::kSlotStride + 32 * qd + e];
+        acc[e] = a * inv;
+      }
+      if (live) {
+        const int hrow = g * p.group + h;
+        if (direct) {
+          __nv_bfloat16* dst = p.out + ((int64_t)b * p.num_q_heads + hrow) * D + 32 * qd;
+#pragma unroll
+          for (int e = 0; e < 32; e += 2) *reinterpret_cast<uint32_t*>(dst + e) = pack_bf16x2(acc[e], acc[e + 1]);
+          if (qd == 0) p.lse[(int64_t)b * p.num_q_heads + hrow] = lse_nat;
+        } else {
+          float* dst = p.partial_o + ((int64_t)s * p.num_q_heads + hrow) * D + 32 * qd;
+#pragma unroll
+          for (int e = 0; e < 32; e += 4) *reinterpret_cast<float4*>(dst + e) = make_float4(acc[e], acc[e + 1], acc[e + 2], acc[e + 3]);
+          if (qd == 0) p.partial_lse[(int64_t)s * p.num_q_heads + hrow] = lse_nat;
+        }
+      }
+    }
+    named_barrier_sync(1, kConsumerWarps * 32);  // slots are free again
+  }
+}
+#endif  // DA_BF16_FFMA
+
 template <int D, bool FP8, bool MQ, bool MERGE>
 __global__ void __launch_bounds__(kThreads, 2)
     decode_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap k64,
@@ -205,6 +366,99 @@ __global__ void __launch_bounds__(kThreads, 2)
   }
   __syncthreads();
 
+  // Stage `stage` <- K and V of tokens [c0, c0 + n) of one request, whose 16-token pieces sit
+  // in pages pid[]; the stage's "full" barrier expects the bytes.  Lane 0 of the producer.
+  constexpr int kPieces = kChunk / 16;
+  auto issue_chunk = [&](int stage, int c0, int n, const int (&pid)[kPieces], bool ok, uint64_t policy) {
+    const int P = p.page_size;
+    meta[stage] = ok ? n : 0;
+    // bytes: per 64-row sub-chunk, one 64-row box per column block when it sits in
+    // one page, else one 16-row box per column block for each piece that holds tokens
+    uint32_t bytes = 0;
+    if (ok) {
+#pragma unroll
+      for (int j = 0; j < kChunk / 64; ++j) {
+        if (64 * j >= n) break;
+        const bool fast = ((c0 + 64 * j) % P) + 64 <= P;
+        const int pieces = fast ? 4 : min(4, (n - 64 * j + 15) >> 4);
+        bytes += (uint32_t)(pieces * 16 * 128 * C::kHalves * 2);
+      }
+    }
+    const uint32_t full = full0 + 8 * stage;
+    mbar_arrive_expect_tx(full, bytes);
+    if (ok) {
+      const uint32_t sk = sbase + C::kOffStages + stage * C::kStageBytes, sv = sk + C::kTileBytes;
+#pragma unroll
+      for (int j = 0; j < kChunk / 64; ++j) {
+        if (64 * j >= n) break;
+        const int tok = c0 + 64 * j;
+        if ((tok % P) + 64 <= P) {
+          const int row = (pid[4 * j] * p.num_kv_heads + g) * P + tok % P;
+#pragma unroll
+          for (int h = 0; h < C::kHalves; ++h) {
+            tma_load_2d(sk + h * C::kHalfStride + j * 64 * 128, &k64, h * C::kBoxCols, row, full, policy);
+            tma_load_2d(sv + h * C::kHalfStride + j * 64 * 128, &v64, h * C::kBoxCols, row, full, policy);
+          }
+        } else {
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            if (64 * j + 16 * i >= n) break;
+            const int row = (pid[4 * j + i] * p.num_kv_heads + g) * P + (tok + 16 * i) % P;
+#pragma unroll
+            for (int h = 0; h < C::kHalves; ++h) {
+              const uint32_t off = h * C::kHalfStride + (64 * j + 16 * i) * 128;
+              tma_load_2d(sk + off, &k16, h * C::kBoxCols, row, full, policy);
+              tma_load_2d(sv + off, &v16, h * C::kBoxCols, row, full, policy);
+            }
+          }
+        }
+      }
+    }
+  };
+
+  // Early start (launch sequences built by the library only): before the plan has landed,
+  // derive this CTA's first segment from seq_lens and request its first chunks, one per
+  // stage; the producer checks the plan against it below and skips those chunks.
+  FirstSegment early{-1, 0, 0};
+  int prefetched = 0;
+  if (p.early) {
+    early = derive_first_segment(p, cta, reinterpret_cast<int*>(smem + C::kOffSlots));
+    if (warp == kConsumerWarps && early.b >= 0 && !p.stall_producer) {
+      if (lane == 0) {
+        const int L = p.seq_lens[early.b];
+        const int tok0 = (int)min((int64_t)early.tile0 * p.tile_tokens, (int64_t)L);
+        const int tok1 = (int)min((int64_t)early.tile1 * p.tile_tokens, (int64_t)L);
+        const int32_t* bt_row = p.block_table + (int64_t)early.b * p.max_pages_per_req;
+        const uint64_t policy = policy_evict_first();
+        for (int k = 0; k < C::kStages; ++k) {
+          const int c0 = tok0 + k * kChunk;
+          if (c0 >= tok1) break;
+          const int n = min(kChunk, tok1 - c0);
+          int pid[kPieces];
+          bool ok = true;
+#pragma unroll
+          for (int i = 0; i < kPieces; ++i) {
+            const int lp = (c0 + 16 * i) / p.page_size;
+            pid[i] = 0;
+            if (16 * i < n) {
+              pid[i] = lp < p.max_pages_per_req ? __ldg(bt_row + lp) : -1;
+              ok = ok && pid[i] >= 0 && pid[i] < p.num_pages;
+            }
+          }
+          if (!ok) break;  // the main loop requests it and reports the page
+          issue_chunk(k, c0, n, pid, true, policy);  // a fresh stage: no "empty" wait
+          ++prefetched;
+        }
+      }
+      prefetched = __shfl_sync(0xffffffffu, prefetched, 0);
+    }
+  }
+  // the producer's lane 0 waits (bounded) for the early requests before the CTA may exit
+  auto drain_prefetch = [&]() {
+    if (warp == kConsumerWarps && lane == 0)
+      for (int k = 0; k < prefetched; ++k) mbar_wait_drain(full0 + 8 * k, 0, p.wait_limit_ns);
+  };
+
   grid_dependency_wait();    // the plan is written by the previous kernel in the stream
   grid_dependents_launch();  // the combine kernel may be scheduled; it waits for this grid to finish
 
@@ -220,6 +474,7 @@ __global__ void __launch_bounds__(kThreads, 2)
   const int h_segs = hdr[kHdrSegments], seg_lo = csb[cta], seg_next = csb[cta + 1];
   if (h_ctas != p.num_ctas || h_batch != p.batch || h_ms != p.max_segments || h_kind != p.kind) {
     if (threadIdx.x == 0 && cta == 0 && g == 0) record_status(hdr_w, DA_DEV_BAD_PLAN, 0);
+    drain_prefetch();
     return;
   }
   const int seg_hi = min(seg_next, min(h_segs, p.max_segments));
@@ -237,7 +492,11 @@ __global__ void __launch_bounds__(kThreads, 2)
       }
     }
   }
-  if (seg_lo < 0 || seg_lo >= seg_hi) return;  // nothing planned for this CTA (uniform over the block)
+  if (seg_lo < 0 || seg_lo >= seg_hi) {  // nothing planned for this CTA (uniform over the block)
+    if (early.b >= 0 && threadIdx.x == 0) record_status(hdr_w, DA_DEV_BAD_PLAN, cta);  // the plan disagrees
+    drain_prefetch();
+    return;
+  }
 
   if (warp == kConsumerWarps) {
     // ------------------------------------------------------------------ producer warp
@@ -247,6 +506,22 @@ __global__ void __launch_bounds__(kThreads, 2)
     uint32_t phase = 0;
     int fills = 0;
     bool aborted = p.stall_producer != 0;  // failure-path test: send nothing
+    int skip = 0;  // chunks of the first segment already requested by the early start
+    if (prefetched > 0) {
+      const int4 sg = segs[seg_lo];
+      if (sg.x == early.b && sg.z == early.tile0 && sg.w == early.tile1) {
+        skip = prefetched;
+      } else {  // cannot happen when the plan was made from the same lengths: stop, drain, report
+        if (lane == 0) {
+          record_status(hdr_w, DA_DEV_BAD_PLAN, cta);
+          *abort_flag = 1;
+        }
+        aborted = true;
+      }
+      fills = prefetched;
+      stage = prefetched % C::kStages;
+      phase = (prefetched / C::kStages) & 1;
+    }
     for (int s = seg_lo; s < seg_hi && !aborted; ++s) {
       // first window of page ids, issued before (and independent of) the length load
       const int4 sg = segs[s];
@@ -259,7 +534,9 @@ __global__ void __launch_bounds__(kThreads, 2)
       const SegmentInfo si = load_segment(p, segs, s);
       if (!si.valid) continue;
       const int32_t* bt_row = p.block_table + (int64_t)si.b * p.max_pages_per_req;
-      for (int c0 = si.tok0; c0 < si.tok1; c0 += kChunk) {
+      const int c_first = si.tok0 + skip * kChunk;  // the early requests: this (first) segment's first chunks
+      skip = 0;
+      for (int c0 = c_first; c0 < si.tok1; c0 += kChunk) {
         const int n = min(kChunk, si.tok1 - c0);
         const int lp_first = c0 / P, lp_last = (c0 + n - 1) / P;
         if (lp_first < win_base || lp_last >= win_base + 32) {
@@ -268,7 +545,6 @@ __global__ void __launch_bounds__(kThreads, 2)
           win_val = lp < p.max_pages_per_req ? __ldg(bt_row + lp) : -1;
         }
         // page of every 16-row piece of the chunk (pieces past n are not loaded)
-        constexpr int kPieces = kChunk / 16;
         int pid[kPieces];
         bool ok = true;
 #pragma unroll
@@ -291,49 +567,7 @@ __global__ void __launch_bounds__(kThreads, 2)
         }
         if (lane == 0) {
           if (!ok) record_status(hdr_w, DA_DEV_BAD_PAGE, si.b);
-          meta[stage] = ok ? n : 0;
-          // bytes: per 64-row sub-chunk, one 64-row box per column block when it sits in
-          // one page, else one 16-row box per column block for each piece that holds tokens
-          uint32_t bytes = 0;
-          if (ok) {
-#pragma unroll
-            for (int j = 0; j < kChunk / 64; ++j) {
-              if (64 * j >= n) break;
-              const bool fast = ((c0 + 64 * j) % P) + 64 <= P;
-              const int pieces = fast ? 4 : min(4, (n - 64 * j + 15) >> 4);
-              bytes += (uint32_t)(pieces * 16 * 128 * C::kHalves * 2);
-            }
-          }
-          const uint32_t full = full0 + 8 * stage;
-          mbar_arrive_expect_tx(full, bytes);
-          if (ok) {
-            const uint32_t sk = sbase + C::kOffStages + stage * C::kStageBytes, sv = sk + C::kTileBytes;
-#pragma unroll
-            for (int j = 0; j < kChunk / 64; ++j) {
-              if (64 * j >= n) break;
-              const int tok = c0 + 64 * j;
-              if ((tok % P) + 64 <= P) {
-                const int row = (pid[4 * j] * p.num_kv_heads + g) * P + tok % P;
-#pragma unroll
-                for (int h = 0; h < C::kHalves; ++h) {
-                  tma_load_2d(sk + h * C::kHalfStride + j * 64 * 128, &k64, h * C::kBoxCols, row, full, policy);
-                  tma_load_2d(sv + h * C::kHalfStride + j * 64 * 128, &v64, h * C::kBoxCols, row, full, policy);
-                }
-              } else {
-#pragma unroll
-                for (int i = 0; i < 4; ++i) {
-                  if (64 * j + 16 * i >= n) break;
-                  const int row = (pid[4 * j + i] * p.num_kv_heads + g) * P + (tok + 16 * i) % P;
-#pragma unroll
-                  for (int h = 0; h < C::kHalves; ++h) {
-                    const uint32_t off = h * C::kHalfStride + (64 * j + 16 * i) * 128;
-                    tma_load_2d(sk + off, &k16, h * C::kBoxCols, row, full, policy);
-                    tma_load_2d(sv + off, &v16, h * C::kBoxCols, row, full, policy);
-                  }
-                }
-              }
-            }
-          }
+          issue_chunk(stage, c0, n, pid, ok, policy);
         }
         __syncwarp();
         ++fills;
@@ -343,15 +577,22 @@ __global__ void __launch_bounds__(kThreads, 2)
         }
       }
     }
-    // Drain: every stage's last fill must have landed before the CTA may exit.
+    // Drain: every stage's last fill must have landed before the CTA may exit (also after
+    // an abort: the copies were requested, so they are waited for, within the limit).
     if (lane == 0) {
       for (int k = max(0, fills - C::kStages); k < fills; ++k)
-        mbar_wait_bounded(full0 + 8 * (k % C::kStages), (k / C::kStages) & 1, abort_flag, p.wait_limit_ns);
+        mbar_wait_drain(full0 + 8 * (k % C::kStages), (k / C::kStages) & 1, p.wait_limit_ns);
     }
     return;
   }
 
   // -------------------------------------------------------------------- consumer warps
+#if DA_BF16_FFMA
+  if constexpr (!FP8 && !MQ && !MERGE && D == 128) {
+    ffma_consumer<C>(p, smem, segs, rsb, hdr_w, full0, empty0, meta, abort_flag, seg_lo, seg_hi, g, warp, lane);
+    return;
+  }
+#endif
   constexpr int TPW = C::kTPW, SUB = C::kSub, HS = C::kHalfStride, NR = C::kNR;
   const int w = warp;
   const int r = lane >> 2;   // MMA row within a row half
@@ -640,7 +881,7 @@ __global__ void __launch_bounds__(kThreads, 2)
 
     // ---- merge the four warp states of this segment, one row half at a time
     const int nseg_b = rsb[b + 1] - rsb[b];
-    const bool direct = nseg_b == 1;
+    const bool direct = nseg_b == 1 && !p.out_f32;  // fp32 output: the combine writes every request
 #pragma unroll
     for (int hh = 0; hh < NR; ++hh) {
       // regroup this thread's columns: og[gi][j] is column gi*4*GW + GW*tq + j

@@ -45,6 +45,7 @@
 #include <climits>
 
 #include "da_internal.cuh"
+#include "early_start.cuh"
 
 namespace da {
 namespace {
@@ -278,6 +279,93 @@ __global__ void __launch_bounds__(kThreadsTc, 2)
   }
   __syncthreads();
 
+  // Stage `stage` <- K and V codes of tokens [c0, c0 + n) of one request, whose 16-token
+  // pieces sit in pages pid[]; the stage's "full" barrier expects the bytes.  Lane 0 of the
+  // producer.
+  constexpr int kPieces = kChunk / 16;
+  auto issue_chunk = [&](int stage, int c0, int n, const int (&pid)[kPieces], bool ok, uint64_t policy) {
+    const int P = p.page_size;
+    meta[stage] = ok ? n : 0;
+    uint32_t bytes = 0;
+    if (ok) {
+#pragma unroll
+      for (int j = 0; j < kChunk / 64; ++j) {
+        if (64 * j >= n) break;
+        const bool fast = ((c0 + 64 * j) % P) + 64 <= P;
+        const int pieces = fast ? 4 : min(4, (n - 64 * j + 15) >> 4);
+        bytes += (uint32_t)(pieces * 16 * 128 * 2);
+      }
+    }
+    const uint32_t full = bar(kBarFull + stage);
+    mbar_arrive_expect_tx(full, bytes);
+    if (ok) {
+      const uint32_t sk = sbase + kOffStages + stage * kStageBytes, sv = sk + kTileBytes;
+#pragma unroll
+      for (int j = 0; j < kChunk / 64; ++j) {
+        if (64 * j >= n) break;
+        const int tok = c0 + 64 * j;
+        if ((tok % P) + 64 <= P) {
+          const int row = (pid[4 * j] * p.num_kv_heads + g) * P + tok % P;
+          tma_load_2d(sk + j * 64 * 128, &k64, 0, row, full, policy);
+          tma_load_2d(sv + j * 64 * 128, &v64, 0, row, full, policy);
+        } else {
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            if (64 * j + 16 * i >= n) break;
+            const int row = (pid[4 * j + i] * p.num_kv_heads + g) * P + (tok + 16 * i) % P;
+            const uint32_t off = (64 * j + 16 * i) * 128;
+            tma_load_2d(sk + off, &k16, 0, row, full, policy);
+            tma_load_2d(sv + off, &v16, 0, row, full, policy);
+          }
+        }
+      }
+    }
+  };
+
+  // Early start (launch sequences built by the library only): before the plan has landed,
+  // and before tensor memory is allocated and the q tiles are built, derive this CTA's first
+  // segment from seq_lens and request its first chunks, one per stage; the producer checks
+  // the plan against it below and skips those chunks.
+  FirstSegment early{-1, 0, 0};
+  int prefetched = 0;
+  if (p.early) {
+    early = derive_first_segment(p, cta, reinterpret_cast<int*>(smem + kOffP));
+    if (warp == kProducerWarp && early.b >= 0 && !p.stall_producer) {
+      if (lane == 0) {
+        const int L = p.seq_lens[early.b];
+        const int tok0 = (int)min((int64_t)early.tile0 * p.tile_tokens, (int64_t)L);
+        const int tok1 = (int)min((int64_t)early.tile1 * p.tile_tokens, (int64_t)L);
+        const int32_t* bt_row = p.block_table + (int64_t)early.b * p.max_pages_per_req;
+        const uint64_t policy = policy_evict_first();
+        for (int k = 0; k < kStagesTc; ++k) {
+          const int c0 = tok0 + k * kChunk;
+          if (c0 >= tok1) break;
+          const int n = min(kChunk, tok1 - c0);
+          int pid[kPieces];
+          bool ok = true;
+#pragma unroll
+          for (int i = 0; i < kPieces; ++i) {
+            const int lp = (c0 + 16 * i) / p.page_size;
+            pid[i] = 0;
+            if (16 * i < n) {
+              pid[i] = lp < p.max_pages_per_req ? __ldg(bt_row + lp) : -1;
+              ok = ok && pid[i] >= 0 && pid[i] < p.num_pages;
+            }
+          }
+          if (!ok) break;  // the main loop requests it and reports the page
+          issue_chunk(k, c0, n, pid, true, policy);  // a fresh stage: no "empty" wait
+          ++prefetched;
+        }
+      }
+      prefetched = __shfl_sync(0xffffffffu, prefetched, 0);
+    }
+  }
+  // the producer's lane 0 waits (bounded) for the early requests before the CTA may exit
+  auto drain_prefetch = [&]() {
+    if (warp == kProducerWarp && lane == 0)
+      for (int k = 0; k < prefetched; ++k) mbar_wait_drain(bar(kBarFull + k), 0, p.wait_limit_ns);
+  };
+
   grid_dependency_wait();    // the plan is written by the previous kernel in the stream
   grid_dependents_launch();  // the combine kernel may be scheduled; it waits for this grid to finish
 
@@ -291,10 +379,15 @@ __global__ void __launch_bounds__(kThreadsTc, 2)
   const int h_segs = hdr[kHdrSegments], seg_lo = csb[cta], seg_next = csb[cta + 1];
   if (h_ctas != p.num_ctas || h_batch != p.batch || h_ms != p.max_segments || h_kind != p.kind) {
     if (threadIdx.x == 0 && cta == 0 && g == 0) record_status(hdr_w, DA_DEV_BAD_PLAN, 0);
+    drain_prefetch();
     return;  // before TMEM is allocated
   }
   const int seg_hi = min(seg_next, min(h_segs, p.max_segments));
-  if (seg_lo < 0 || seg_lo >= seg_hi) return;  // nothing planned for this CTA (uniform over the block)
+  if (seg_lo < 0 || seg_lo >= seg_hi) {  // nothing planned for this CTA (uniform over the block)
+    if (early.b >= 0 && threadIdx.x == 0) record_status(hdr_w, DA_DEV_BAD_PLAN, cta);  // the plan disagrees
+    drain_prefetch();
+    return;
+  }
 
   // TMEM for this CTA (64 of the SM's 512 columns; two CTAs per SM)
   if (warp == kMmaWarp) {
@@ -314,6 +407,22 @@ __global__ void __launch_bounds__(kThreadsTc, 2)
     uint32_t phase = 0;
     int fills = 0;
     bool aborted = p.stall_producer != 0;  // failure-path test: send nothing
+    int skip = 0;  // chunks of the first segment already requested by the early start
+    if (prefetched > 0) {
+      const int4 sg = segs[seg_lo];
+      if (sg.x == early.b && sg.z == early.tile0 && sg.w == early.tile1) {
+        skip = prefetched;
+      } else {  // cannot happen when the plan was made from the same lengths: stop, drain, report
+        if (lane == 0) {
+          record_status(hdr_w, DA_DEV_BAD_PLAN, cta);
+          *abort_flag = 1;
+        }
+        aborted = true;
+      }
+      fills = prefetched;
+      stage = prefetched % kStagesTc;
+      phase = (prefetched / kStagesTc) & 1;
+    }
     for (int s = seg_lo; s < seg_hi && !aborted; ++s) {
       const int4 sg = segs[s];
       int win_base = INT_MIN / 2, win_val = -1;
@@ -325,7 +434,9 @@ __global__ void __launch_bounds__(kThreadsTc, 2)
       const SegmentInfo si = load_segment(p, segs, s);
       if (!si.valid) continue;
       const int32_t* bt_row = p.block_table + (int64_t)si.b * p.max_pages_per_req;
-      for (int c0 = si.tok0; c0 < si.tok1; c0 += kChunk) {
+      const int c_first = si.tok0 + skip * kChunk;  // the early requests: this (first) segment's first chunks
+      skip = 0;
+      for (int c0 = c_first; c0 < si.tok1; c0 += kChunk) {
         const int n = min(kChunk, si.tok1 - c0);
         const int lp_first = c0 / P, lp_last = (c0 + n - 1) / P;
         if (lp_first < win_base || lp_last >= win_base + 32) {
@@ -333,7 +444,6 @@ __global__ void __launch_bounds__(kThreadsTc, 2)
           const int lp = win_base + lane;
           win_val = lp < p.max_pages_per_req ? __ldg(bt_row + lp) : -1;
         }
-        constexpr int kPieces = kChunk / 16;
         int pid[kPieces];
         bool ok = true;
 #pragma unroll
@@ -355,41 +465,7 @@ __global__ void __launch_bounds__(kThreadsTc, 2)
         }
         if (lane == 0) {
           if (!ok) record_status(hdr_w, DA_DEV_BAD_PAGE, si.b);
-          meta[stage] = ok ? n : 0;
-          uint32_t bytes = 0;
-          if (ok) {
-#pragma unroll
-            for (int j = 0; j < kChunk / 64; ++j) {
-              if (64 * j >= n) break;
-              const bool fast = ((c0 + 64 * j) % P) + 64 <= P;
-              const int pieces = fast ? 4 : min(4, (n - 64 * j + 15) >> 4);
-              bytes += (uint32_t)(pieces * 16 * 128 * 2);
-            }
-          }
-          const uint32_t full = bar(kBarFull + stage);
-          mbar_arrive_expect_tx(full, bytes);
-          if (ok) {
-            const uint32_t sk = sbase + kOffStages + stage * kStageBytes, sv = sk + kTileBytes;
-#pragma unroll
-            for (int j = 0; j < kChunk / 64; ++j) {
-              if (64 * j >= n) break;
-              const int tok = c0 + 64 * j;
-              if ((tok % P) + 64 <= P) {
-                const int row = (pid[4 * j] * p.num_kv_heads + g) * P + tok % P;
-                tma_load_2d(sk + j * 64 * 128, &k64, 0, row, full, policy);
-                tma_load_2d(sv + j * 64 * 128, &v64, 0, row, full, policy);
-              } else {
-#pragma unroll
-                for (int i = 0; i < 4; ++i) {
-                  if (64 * j + 16 * i >= n) break;
-                  const int row = (pid[4 * j + i] * p.num_kv_heads + g) * P + (tok + 16 * i) % P;
-                  const uint32_t off = (64 * j + 16 * i) * 128;
-                  tma_load_2d(sk + off, &k16, 0, row, full, policy);
-                  tma_load_2d(sv + off, &v16, 0, row, full, policy);
-                }
-              }
-            }
-          }
+          issue_chunk(stage, c0, n, pid, ok, policy);
         }
         __syncwarp();
         ++fills;
@@ -399,10 +475,11 @@ __global__ void __launch_bounds__(kThreadsTc, 2)
         }
       }
     }
-    // every stage's last fill must have landed before the CTA may exit
+    // every stage's last fill must have landed before the CTA may exit (also after an abort:
+    // the copies were requested, so they are waited for, within the limit)
     if (lane == 0) {
       for (int k = max(0, fills - kStagesTc); k < fills; ++k)
-        mbar_wait_bounded(bar(kBarFull + k % kStagesTc), (k / kStagesTc) & 1, abort_flag, p.wait_limit_ns);
+        mbar_wait_drain(bar(kBarFull + k % kStagesTc), (k / kStagesTc) & 1, p.wait_limit_ns);
     }
   } else if (warp == kMmaWarp) {
     // ------------------------------------------------------------------ MMA issuer
@@ -660,7 +737,7 @@ __global__ void __launch_bounds__(kThreadsTc, 2)
       // ---- the segment's result: per head, O / (sum of weights) and the log-sum-exp
       float lt[8];
       reduce8<false>(l_part, lt, red + 32 * (calls++ & 1), warp, lane);
-      const bool direct = rsb[b + 1] - rsb[b] == 1;
+      const bool direct = rsb[b + 1] - rsb[b] == 1 && !p.out_f32;  // fp32 output: the combine writes it
 #pragma unroll
       for (int h = 0; h < 8; ++h) {
         if (h >= G) break;

@@ -11,6 +11,8 @@
 //
 // One warp per output row (request x query x head); lanes own head_dim/32
 // columns; parts are summed in part order (fp32), so results are deterministic.
+// Parts are bf16 (each GPU's ordinary `out`) or fp32 (steps run with fp32
+// output, so that nothing is rounded to bf16 before the merge).
 #include "da_internal.cuh"
 
 namespace da {
@@ -35,18 +37,26 @@ __global__ void __launch_bounds__(128) merge_parts_kernel(const MergeParams p) {
     total = M + logf(sum);
     for (int j = 0; j < p.num_parts; ++j) {
       const float wgt = expf(__ldg(p.part_lse + (int64_t)j * p.rows + row) - total);
-      const __nv_bfloat16* src = p.part_out + ((int64_t)j * p.rows + row) * D + lane * kPer;
-      if constexpr (kPer == 4) {
-        const uint2 v = __ldg(reinterpret_cast<const uint2*>(src));
-        acc[0] += wgt * bf16_lo_to_f32(v.x);
-        acc[1] += wgt * bf16_hi_to_f32(v.x);
-        acc[2] += wgt * bf16_lo_to_f32(v.y);
-        acc[3] += wgt * bf16_hi_to_f32(v.y);
+      const int64_t at = ((int64_t)j * p.rows + row) * D + lane * kPer;
+      float v[kPer];
+      if (p.part_out_f32) {
+        if constexpr (kPer == 4) {
+          const float4 t = __ldg(reinterpret_cast<const float4*>(p.part_out_f32 + at));
+          v[0] = t.x, v[1] = t.y, v[2] = t.z, v[3] = t.w;
+        } else {
+          const float2 t = __ldg(reinterpret_cast<const float2*>(p.part_out_f32 + at));
+          v[0] = t.x, v[1] = t.y;
+        }
+      } else if constexpr (kPer == 4) {
+        const uint2 t = __ldg(reinterpret_cast<const uint2*>(p.part_out + at));
+        v[0] = bf16_lo_to_f32(t.x), v[1] = bf16_hi_to_f32(t.x), v[2] = bf16_lo_to_f32(t.y);
+        v[3] = bf16_hi_to_f32(t.y);
       } else {
-        const uint32_t v = __ldg(reinterpret_cast<const uint32_t*>(src));
-        acc[0] += wgt * bf16_lo_to_f32(v);
-        acc[1] += wgt * bf16_hi_to_f32(v);
+        const uint32_t t = __ldg(reinterpret_cast<const uint32_t*>(p.part_out + at));
+        v[0] = bf16_lo_to_f32(t), v[1] = bf16_hi_to_f32(t);
       }
+#pragma unroll
+      for (int e = 0; e < kPer; ++e) acc[e] += wgt * v[e];
     }
   }
   __nv_bfloat16* dst = p.out + row * D + lane * kPer;

@@ -15,9 +15,11 @@
 // device address (on the host it names a stand-in object), so the address is
 // looked up once per device with cudaGetSymbolAddress and passed to the
 // kernels.
+#include <cudaTypedefs.h>
+
 #include <mutex>
 
-#include "da_internal.cuh"
+#include "prepared_step.cuh"
 
 namespace {
 
@@ -25,24 +27,71 @@ static __device__ __align__(256) unsigned char g_step_scratch[DA_NOALLOC_SCRATCH
 
 constexpr int kMaxDevices = 64;
 std::mutex g_scratch_mutex;
-void* g_scratch_addr[kMaxDevices] = {};
+
+// The array's address as resolved on one device, and the id of the context it was resolved
+// in.  Context ids are never reused within a process, so a context made after a device reset
+// (whose copy of the array may sit elsewhere) never matches an old entry.
+struct ScratchEntry {
+  void* addr;
+  unsigned long long ctx_id;
+  bool have_id;
+};
+ScratchEntry g_scratch[kMaxDevices] = {};
+
+// Driver entry points for the current context's id, looked up once through the runtime.
+struct CtxFns {
+  PFN_cuCtxGetCurrent_v4000 get_current = nullptr;
+  PFN_cuCtxGetId_v12000 get_id = nullptr;
+};
+const CtxFns& ctx_fns() {
+  static CtxFns f;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      f.get_current = reinterpret_cast<PFN_cuCtxGetCurrent_v4000>(p);
+    p = nullptr;
+    if (cudaGetDriverEntryPoint("cuCtxGetId", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      f.get_id = reinterpret_cast<PFN_cuCtxGetId_v12000>(p);
+  });
+  return f;
+}
+
+// Id of the calling thread's current context; false when there is none or it cannot be read.
+bool current_ctx_id(unsigned long long* id) {
+  const CtxFns& f = ctx_fns();
+  CUcontext ctx = nullptr;
+  if (!f.get_current || !f.get_id || f.get_current(&ctx) != CUDA_SUCCESS || !ctx) return false;
+  return f.get_id(ctx, id) == CUDA_SUCCESS;
+}
 
 size_t round_up_256(size_t n) { return (n + 255) / 256 * 256; }
 
-// Device address of g_step_scratch on the current device (looked up on first use).
+// Device address of g_step_scratch on the current device.  Looked up with cudaGetSymbolAddress
+// (which loads the module into the device's context if needed) the first time on each device,
+// and again whenever the device's context is not the one of the last lookup.
 cudaError_t scratch_address(void** addr) {
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
   if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
   std::lock_guard<std::mutex> lock(g_scratch_mutex);
-  if (!g_scratch_addr[dev]) {
-    void* p = nullptr;
-    e = cudaGetSymbolAddress(&p, g_step_scratch);
-    if (e != cudaSuccess) return e;
-    g_scratch_addr[dev] = p;
+  ScratchEntry& ent = g_scratch[dev];
+  unsigned long long id = 0;
+  const bool have_id = current_ctx_id(&id);
+  if (ent.addr && ent.have_id && have_id && ent.ctx_id == id) {
+    *addr = ent.addr;
+    return cudaSuccess;
   }
-  *addr = g_scratch_addr[dev];
+  void* p = nullptr;
+  e = cudaGetSymbolAddress(&p, g_step_scratch);
+  if (e != cudaSuccess) return e;
+  ent.addr = p;
+  ent.have_id = current_ctx_id(&ent.ctx_id);  // the lookup made the primary context current if it was not
+  *addr = p;
   return cudaSuccess;
 }
 
@@ -62,7 +111,7 @@ extern "C" DA_API int da_decode_step_noalloc(const da_problem* prob, int32_t til
   if (ws_r + po_r + pl_r > (size_t)DA_NOALLOC_SCRATCH_BYTES) return DA_ERR_WORKSPACE;
   if (prob->batch > 0 && (!q || !k_cache || !v_cache || !block_table || !seq_lens || !out || !lse))
     return DA_ERR_INVALID_ARG;
-  // the decode call's alignment rules, checked here so that an error enqueues nothing (not even the plan)
+  // the decode call's alignment rules, checked before the first CUDA call (the scratch lookup)
   if (prob->batch > 0 &&
       (reinterpret_cast<uintptr_t>(k_cache) % 16 != 0 || reinterpret_cast<uintptr_t>(v_cache) % 16 != 0 ||
        reinterpret_cast<uintptr_t>(q) % 4 != 0 || reinterpret_cast<uintptr_t>(out) % 8 != 0))
@@ -80,10 +129,21 @@ extern "C" DA_API int da_decode_step_noalloc(const da_problem* prob, int32_t til
   // The plan kernel rewrites every scratch word that decode and combine read
   // (header, status, segment list, prefixes), and decode writes every partial
   // that combine reads, so nothing left by an earlier call needs clearing.
-  rc = da_plan(prob, &desc, seq_lens, ws, ws_r, stream);
+  // Every check of the three launches (alignment, tensor maps) runs first, so an
+  // error return enqueues nothing unless the CUDA runtime refuses a launch.
+  da::PreparedStep st;
+  rc = da::prepare_dynamic_step(prob, &desc, q, k_cache, v_cache, block_table, seq_lens, ws, ws_r, partial_o,
+                                partial_lse, out, lse, &st);
   if (rc != DA_OK) return rc;
-  rc = da_decode_attention(prob, &desc, q, k_cache, v_cache, block_table, seq_lens, ws, partial_o, partial_lse, out,
-                           lse, stream);
-  if (rc != DA_OK) return rc;
-  return da_combine(prob, &desc, ws, partial_o, partial_lse, out, lse, stream);
+  return da::launch_prepared_step(st, stream);
+}
+
+extern "C" DA_API int da_noalloc_read_status(int32_t* dev_status, int32_t* bad_index, void* stream) {
+  void* base = nullptr;
+  cudaError_t e = scratch_address(&base);
+  if (e != cudaSuccess) {
+    da::set_last_cuda_error(e);
+    return DA_ERR_CUDA;
+  }
+  return da_read_status(base, dev_status, bad_index, stream);
 }

@@ -17,13 +17,15 @@ LIB_PATH = os.path.join(HERE, "libda.so")
 OK, ERR_INVALID_ARG, ERR_UNSUPPORTED, ERR_CUDA, ERR_WORKSPACE = 0, -1, -2, -3, -4
 DEV_OK, DEV_BAD_SEQLEN, DEV_BAD_PAGE, DEV_TIMEOUT, DEV_BAD_PLAN = 0, 1, 2, 3, 4
 PLAN_DYNAMIC, PLAN_STATIC = 0, 1
+OUT_BF16, OUT_F32 = 0, 1
 
 # Every symbol include/da.h declares.
 EXPORTS = ("da_plan_desc_init", "da_workspace_size", "da_workspace_offsets", "da_plan", "da_static_plan",
            "da_decode_attention", "da_combine", "da_read_status", "da_status_string", "da_dev_status_string",
            "da_last_cuda_error", "da_device_num_sms", "da_decode_step_noalloc", "da_append_kv",
            "da_decode_attention_fp8", "da_merge_partials", "da_decode_step_host", "da_test_stall_next_decode",
-           "da_plan_append")
+           "da_plan_append", "da_plan_workspace_size", "da_noalloc_read_status",
+           "da_merge_partials_f32", "da_decode_step")
 
 NOALLOC_SCRATCH_BYTES = 16 << 20  # DA_NOALLOC_SCRATCH_BYTES
 
@@ -37,7 +39,8 @@ class DaProblem(ctypes.Structure):
 class DaPlanDesc(ctypes.Structure):
     _fields_ = [("kind", ctypes.c_int32), ("batch", ctypes.c_int32), ("tile_tokens", ctypes.c_int32),
                 ("num_ctas", ctypes.c_int32), ("splits", ctypes.c_int32), ("max_segments", ctypes.c_int32),
-                ("num_kv_heads", ctypes.c_int32), ("merge_in_decode", ctypes.c_int32)]
+                ("num_kv_heads", ctypes.c_int32), ("merge_in_decode", ctypes.c_int32),
+                ("out_format", ctypes.c_int32)]
 
 
 class DaError(RuntimeError):
@@ -68,6 +71,9 @@ def lib():
             "da_plan_desc_init": [P, ctypes.c_int32, ctypes.c_int32, ctypes.c_int32, D],
             "da_workspace_size": [P, D, ctypes.POINTER(_sz), ctypes.POINTER(_sz), ctypes.POINTER(_sz)],
             "da_workspace_offsets": [D, ctypes.POINTER(ctypes.c_int64)],
+            "da_plan_workspace_size": [P, ctypes.c_int32, ctypes.c_int32, ctypes.POINTER(_sz), ctypes.POINTER(_sz),
+                                       ctypes.POINTER(_sz)],
+            "da_noalloc_read_status": [ctypes.POINTER(ctypes.c_int32), ctypes.POINTER(ctypes.c_int32), _vp],
             "da_plan": [P, D, _vp, _vp, _sz, _vp],
             "da_static_plan": [P, D, _vp, _vp, _sz, _vp],
             "da_decode_attention": [P, D, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp],
@@ -78,7 +84,9 @@ def lib():
             "da_decode_step_noalloc": [P, ctypes.c_int32, ctypes.c_int32, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp],
             "da_append_kv": [P, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp],
             "da_merge_partials": [ctypes.c_int32, ctypes.c_int64, ctypes.c_int32, _vp, _vp, _vp, _vp, _vp],
+            "da_merge_partials_f32": [ctypes.c_int32, ctypes.c_int64, ctypes.c_int32, _vp, _vp, _vp, _vp, _vp],
             "da_decode_attention_fp8": [P, D, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp],
+            "da_decode_step": [P, D, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _sz, _vp, _vp, _vp, _vp, _vp],
             "da_test_stall_next_decode": [ctypes.c_uint32],
             "da_plan_append": [P, D, _vp, _vp, _sz, _vp, _vp, _vp, _vp, _vp, _vp, _vp],
             "da_decode_step_host": [P, D, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _sz, _vp, _vp, _vp,
@@ -139,11 +147,13 @@ def _stream(stream) -> int | None:
 # ---- the C calls -------------------------------------------------------------------------------
 
 def da_plan_desc_init(prob: DaProblem, kind: int, tile_tokens: int = 0, width: int = 0,
-                      merge_in_decode: bool = False) -> DaPlanDesc:
+                      merge_in_decode: bool = False, out_f32: bool = False) -> DaPlanDesc:
+    """The C call, then the descriptor's two switches (in-decode merge, fp32 output) set as asked."""
     d = DaPlanDesc()
     _check("da_plan_desc_init", lib().da_plan_desc_init(ctypes.byref(prob), int(kind), int(tile_tokens), int(width),
                                                          ctypes.byref(d)))
     d.merge_in_decode = 1 if merge_in_decode else 0
+    d.out_format = OUT_F32 if out_f32 else OUT_BF16
     return d
 
 
@@ -151,6 +161,13 @@ def da_workspace_size(prob: DaProblem, desc: DaPlanDesc) -> tuple[int, int, int]
     a, b, c = _sz(), _sz(), _sz()
     _check("da_workspace_size", lib().da_workspace_size(ctypes.byref(prob), ctypes.byref(desc), ctypes.byref(a),
                                                          ctypes.byref(b), ctypes.byref(c)))
+    return a.value, b.value, c.value
+
+
+def da_plan_workspace_size(prob: DaProblem, tile_tokens: int = 0, num_ctas: int = 0) -> tuple[int, int, int]:
+    a, b, c = _sz(), _sz(), _sz()
+    _check("da_plan_workspace_size", lib().da_plan_workspace_size(
+        ctypes.byref(prob), int(tile_tokens), int(num_ctas), ctypes.byref(a), ctypes.byref(b), ctypes.byref(c)))
     return a.value, b.value, c.value
 
 
@@ -185,6 +202,15 @@ def da_decode_attention_fp8(prob, desc, q, k_cache, v_cache, k_scale, v_scale, b
         ctypes.byref(prob), ctypes.byref(desc), _ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(k_scale), _ptr(v_scale),
         _ptr(block_table), _ptr(seq_lens), _ptr(ws), _ptr(partial_o), _ptr(partial_lse), _ptr(out), _ptr(lse),
         _stream(stream)))
+
+
+def da_decode_step(prob, desc, q, k_cache, v_cache, block_table, seq_lens, bufs: "Buffers", k_scale=None, v_scale=None,
+                   stream=None):
+    """Plan + decode + combine in one C call (the decode may start on its first chunks before the plan lands)."""
+    _check("da_decode_step", lib().da_decode_step(
+        ctypes.byref(prob), ctypes.byref(desc), _ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(k_scale), _ptr(v_scale),
+        _ptr(block_table), _ptr(seq_lens), _ptr(bufs.ws), bufs.ws.numel() * bufs.ws.element_size(),
+        _ptr(bufs.partial_o), _ptr(bufs.partial_lse), _ptr(bufs.out), _ptr(bufs.lse), _stream(stream)))
 
 
 def da_combine(prob, desc, ws, partial_o, partial_lse, out, lse, stream=None):
@@ -228,6 +254,15 @@ def da_merge_partials(part_out, part_lse, out, lse, stream=None):
                                                         _ptr(part_lse), _ptr(out), _ptr(lse), _stream(stream)))
 
 
+def da_merge_partials_f32(part_out, part_lse, out, lse, stream=None):
+    """part_out [n, ..., d] fp32 (steps run with fp32 output) and part_lse [n, ...] -> out bf16, lse."""
+    n = part_out.shape[0]
+    rows = lse.numel()
+    _check("da_merge_partials_f32", lib().da_merge_partials_f32(int(n), int(rows), int(part_out.shape[-1]),
+                                                                _ptr(part_out), _ptr(part_lse), _ptr(out), _ptr(lse),
+                                                                _stream(stream)))
+
+
 def da_read_status(ws, stream=None) -> tuple[int, int]:
     st, bad = ctypes.c_int32(), ctypes.c_int32()
     _check("da_read_status", lib().da_read_status(_ptr(ws), ctypes.byref(st), ctypes.byref(bad), _stream(stream)))
@@ -254,6 +289,14 @@ def da_decode_step_noalloc(prob, q, k_cache, v_cache, block_table, seq_lens, out
         _ptr(block_table), _ptr(seq_lens), _ptr(out), _ptr(lse), _stream(stream)))
 
 
+def da_noalloc_read_status(stream=None) -> tuple[int, int]:
+    """Status word and first bad index of the last da_decode_step_noalloc on this device (syncs `stream`)."""
+    st, bad = ctypes.c_int32(), ctypes.c_int32()
+    _check("da_noalloc_read_status", lib().da_noalloc_read_status(ctypes.byref(st), ctypes.byref(bad),
+                                                                   _stream(stream)))
+    return st.value, bad.value
+
+
 # ---- buffers and one whole step --------------------------------------------------------------------
 
 class Buffers:
@@ -266,16 +309,22 @@ class Buffers:
         self.partial_o = torch.empty(max(po // 4, 4), dtype=torch.float32, device=device)
         self.partial_lse = torch.empty(max(pl // 4, 1), dtype=torch.float32, device=device)
         lead = (prob.batch,) if prob.q_len <= 1 else (prob.batch, prob.q_len)
-        self.out = torch.empty(lead + (prob.num_q_heads, prob.head_dim), dtype=torch.bfloat16, device=device)
+        out_dtype = torch.float32 if desc.out_format == OUT_F32 else torch.bfloat16
+        self.out = torch.empty(lead + (prob.num_q_heads, prob.head_dim), dtype=out_dtype, device=device)
         self.lse = torch.empty(lead + (prob.num_q_heads,), dtype=torch.float32, device=device)
 
 
 def decode_step(prob, desc, q, k_cache, v_cache, block_table, seq_lens, bufs: Buffers, stream=None, k_scale=None,
-                v_scale=None, planned: bool = False):
+                v_scale=None, planned: bool = False, separate: bool = False):
     """Plan (dynamic or static, per `desc.kind`) + decode + combine, asynchronously on `stream`.
 
-    With k_scale/v_scale given, the caches are FP8 E4M3 codes (da_decode_attention_fp8).
-    planned=True skips the plan: da_plan_append has already written it into bufs.ws."""
+    One da_decode_step call, or, with separate=True, the three calls one by one.  With
+    k_scale/v_scale given, the caches are FP8 E4M3 codes.  planned=True skips the plan
+    (da_plan_append has already written it into bufs.ws): decode and combine only."""
+    if not planned and not separate:
+        da_decode_step(prob, desc, q, k_cache, v_cache, block_table, seq_lens, bufs, k_scale=k_scale, v_scale=v_scale,
+                       stream=stream)
+        return bufs.out, bufs.lse
     if planned:
         pass
     elif desc.kind == PLAN_DYNAMIC:
