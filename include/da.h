@@ -19,8 +19,7 @@
  *   da_decode_attention  work list -> out/lse (single-segment requests) and
  *                        per-segment partials (requests split over CTAs)
  *   da_combine           partials -> out/lse by log-sum-exp merge
- * or one call, da_decode_step, which enqueues the same three launches and lets the
- * decode kernel request its first K/V chunks before the plan has landed.
+ * or one call, da_decode_step, which enqueues the same three launches.
  * (With merge_in_decode = 1 in the descriptor the decode kernel merges split
  * requests itself and da_combine enqueues nothing.)  Before the step, the new
  * token's K/V rows go into their pages with da_append_kv, or with
@@ -340,13 +339,9 @@ DA_API int da_combine(const da_problem* prob, const da_plan_desc* desc, const vo
  * per desc->kind), the decode (bf16 cache when k_scale and v_scale are NULL, FP8
  * E4M3 cache with per-KV-head scales when both are given) and da_combine, enqueued
  * on `stream` in that order.  Arguments, layouts, results and errors are those of
- * the three calls; every check runs before the first launch.  Because the launch
- * before the decode is then the planner, which writes only `ws`, each decode CTA
- * (for batches up to 1024 requests) works out its first segment from seq_lens with
- * the planner's formulas and requests that segment's first K/V chunks while the
- * planner is still running, then checks the plan against it (a mismatch, which
- * only a changed seq_lens could cause, is DA_DEV_BAD_PLAN).  The separate calls
- * cannot do this, since they do not know what the caller enqueues between them.
+ * the three calls, and every check of all three runs before the first launch, so
+ * an error return has enqueued nothing (except DA_ERR_CUDA from a launch the CUDA
+ * runtime refused).  Results are those of the separate calls, bit for bit.
  * Source: "Tencent HPC lands in SGLang, challenging default inference kernels",
  * section "Why Tencent HPC matters for online model serving" (the tile-to-CTA
  * mapping is rebuilt every decode step; the step's work then runs on it).

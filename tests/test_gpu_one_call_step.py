@@ -1,13 +1,11 @@
 """The one-call step (da_decode_step) against the three separate calls.
 
-In da_decode_step each decode CTA works out its first segment from seq_lens and
-requests that segment's first K/V chunks before the plan has landed, then checks the
-plan against it.  The arithmetic is unchanged, so its results must equal the separate
-calls' (da_plan / da_static_plan, da_decode_attention(_fp8), da_combine) bit for bit,
-with the same plan in the workspace and a clean status word, on batches that reach
-every case of the derivation: CTAs with no tile (fewer tiles than CTAs), first
-segments shorter than the ring, empty static splits, bad lengths, and a batch above
-the early-start limit (1024 requests), where the decode waits for the plan first.
+da_decode_step enqueues da_plan (or da_static_plan), the decode and da_combine in one
+call, with every check of the three made before the first launch.  Its results must
+equal the separate calls' bit for bit, with the same plan in the workspace and the
+same status word, on batches with CTAs that have no tile (fewer tiles than CTAs),
+segments shorter than the stage ring, empty static splits, bad lengths and a large
+batch, for both cache formats.
 """
 
 import numpy as np
@@ -49,7 +47,7 @@ def _both(w, kind, tile, width, fp8=False):
                                              (da.PLAN_STATIC, 64, 3), (da.PLAN_STATIC, 32, 16)])
 @pytest.mark.parametrize("fp8", [False, True])
 def test_one_call_step_equals_separate_calls(da_lib, oracle_lib, kind, tile, width, fp8):
-    w = W.make_workload("early", [1, 0, 17, 64, 65, 200, 1000, 4097, 33, 20000, 0, 129], num_q_heads=16,
+    w = W.make_workload("one_call", [1, 0, 17, 64, 65, 200, 1000, 4097, 33, 20000, 0, 129], num_q_heads=16,
                         num_kv_heads=2, head_dim=128, page_size=64, seed=41)
     out, lse, st = _both(w, kind, tile, width, fp8)
     assert st == (da.DEV_OK, -1)
@@ -58,17 +56,17 @@ def test_one_call_step_equals_separate_calls(da_lib, oracle_lib, kind, tile, wid
 
 
 def test_one_call_step_with_bad_lengths(da_lib, oracle_lib):
-    w = W.make_workload("early_bad", [300, 5000, 70], num_q_heads=8, num_kv_heads=1, head_dim=128, page_size=64,
+    w = W.make_workload("one_call_bad", [300, 5000, 70], num_q_heads=8, num_kv_heads=1, head_dim=128, page_size=64,
                         seed=42)
     w.seq_lens = w.seq_lens.copy()
-    w.seq_lens[1] = -5  # a bad length: 0 tiles for the planner and for the derivation alike
+    w.seq_lens[1] = -5  # a bad length: the request gets 0 tiles and is reported
     out, lse, st = _both(w, da.PLAN_DYNAMIC, 64, 5)
     assert st == (da.DEV_BAD_SEQLEN, 1)
 
 
-def test_one_call_step_above_the_early_limit(da_lib, oracle_lib):
+def test_one_call_step_large_batch(da_lib, oracle_lib):
     lens = np.random.default_rng(43).integers(0, 200, 1100)
-    w = W.make_workload("early_big", lens, num_q_heads=8, num_kv_heads=1, head_dim=64, page_size=16, seed=43)
+    w = W.make_workload("one_call_big", lens, num_q_heads=8, num_kv_heads=1, head_dim=64, page_size=16, seed=43)
     out, lse, st = _both(w, da.PLAN_DYNAMIC, 64, 0)
     assert st == (da.DEV_OK, -1)
     check_against_oracle(w, out, lse)

@@ -9,7 +9,6 @@
 
 #include "append_rows.cuh"
 #include "da_internal.cuh"
-#include "early_start.cuh"
 #include "host_inputs.cuh"
 #include "prepared_step.cuh"
 
@@ -314,7 +313,6 @@ static int decode_prepare(const da_problem* prob, const da_plan_desc* desc, cons
   p.full_rows = (p.q_len > 1 || p.group > 8) ? 1 : 0;
   p.merge_in_decode = desc->merge_in_decode;
   p.out_f32 = out_f32 ? 1 : 0;
-  p.early = 0;  // set by the callers that launch the planner just before
   p.stall_producer = g_stall_next_ns != 0 ? 1 : 0;
   p.wait_limit_ns = g_stall_next_ns != 0 ? g_stall_next_ns : kWaitLimitNs;
   g_stall_next_ns = 0;  // one launch only
@@ -436,7 +434,6 @@ DA_API int da_decode_step(const da_problem* prob, const da_plan_desc* desc, cons
   rc = decode_prepare(prob, desc, q, k_cache, v_cache, k_scale, v_scale, block_table, seq_lens, ws, partial_o,
                       partial_lse, out, lse, fp8, &dp, maps);
   if (rc != DA_OK) return rc;
-  dp.early = prob->batch <= da::kEarlyMaxBatch ? 1 : 0;  // the planner is the launch just before
   da::CombineParams cp;
   rc = combine_prepare(prob, desc, ws, partial_o, partial_lse, out, lse, &cp);
   if (rc != DA_OK) return rc;
@@ -536,8 +533,6 @@ DA_API int da_decode_step_host(const da_problem* prob, const da_plan_desc* desc,
     if (e != cudaSuccess) return cuda_fail(e);
     rc = plan_launch(pp, desc->kind, stream);
     if (rc != DA_OK) return rc;
-    // the copies are complete before the planner starts, and the planner writes only `ws`
-    dp.early = prob->batch <= da::kEarlyMaxBatch ? 1 : 0;
   }
   rc = decode_launch(dp, prob->head_dim, maps, fp8, stream);
   if (rc != DA_OK) return rc;
@@ -687,7 +682,6 @@ int prepare_dynamic_step(const da_problem* prob, const da_plan_desc* desc, const
   rc = decode_prepare(prob, desc, q, k_cache, v_cache, nullptr, nullptr, block_table, seq_lens, ws, partial_o,
                       partial_lse, out, lse, false, &st->decode, st->maps);
   if (rc != DA_OK) return rc;
-  st->decode.early = prob->batch <= kEarlyMaxBatch ? 1 : 0;  // launch_prepared_step plans just before
   return combine_prepare(prob, desc, ws, partial_o, partial_lse, out, lse, &st->combine);
 }
 

@@ -78,8 +78,6 @@ struct DecodeParams {
   int32_t stall_producer;   // failure-path test: the producer sends nothing, so every wait runs out
   uint64_t wait_limit_ns;   // limit of every pipeline wait
   int32_t out_f32;          // 1: every segment's result goes to the partials (the combine writes fp32 out)
-  int32_t early;            // 1: the launch before is the planner alone, so the CTA may request its
-                            //    first chunks (derived from seq_lens) before the plan has landed
 };
 
 struct CombineParams {
@@ -203,6 +201,17 @@ __device__ __forceinline__ bool mbar_wait_bounded(uint32_t bar, uint32_t parity,
       if (*abort) return false;
       if (global_timer_ns() - t0 > limit_ns) return false;
     }
+  }
+}
+
+// Wait (at most limit_ns) for an mbarrier phase whatever the abort flag says: used to let
+// the TMA copies a CTA requested land before the CTA exits, also after an abort.
+__device__ __forceinline__ bool mbar_wait_drain(uint32_t bar, uint32_t parity, uint64_t limit_ns) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = global_timer_ns();
+  for (uint32_t it = 1;; ++it) {
+    if (mbar_try_wait(bar, parity)) return true;
+    if ((it & 63) == 0 && global_timer_ns() - t0 > limit_ns) return false;
   }
 }
 

@@ -52,7 +52,6 @@
 #include <cfloat>
 
 #include "da_internal.cuh"
-#include "early_start.cuh"
 
 namespace da {
 namespace {
@@ -416,49 +415,6 @@ __global__ void __launch_bounds__(kThreads, 2)
     }
   };
 
-  // Early start (launch sequences built by the library only): before the plan has landed,
-  // derive this CTA's first segment from seq_lens and request its first chunks, one per
-  // stage; the producer checks the plan against it below and skips those chunks.
-  FirstSegment early{-1, 0, 0};
-  int prefetched = 0;
-  if (p.early) {
-    early = derive_first_segment(p, cta, reinterpret_cast<int*>(smem + C::kOffSlots));
-    if (warp == kConsumerWarps && early.b >= 0 && !p.stall_producer) {
-      if (lane == 0) {
-        const int L = p.seq_lens[early.b];
-        const int tok0 = (int)min((int64_t)early.tile0 * p.tile_tokens, (int64_t)L);
-        const int tok1 = (int)min((int64_t)early.tile1 * p.tile_tokens, (int64_t)L);
-        const int32_t* bt_row = p.block_table + (int64_t)early.b * p.max_pages_per_req;
-        const uint64_t policy = policy_evict_first();
-        for (int k = 0; k < C::kStages; ++k) {
-          const int c0 = tok0 + k * kChunk;
-          if (c0 >= tok1) break;
-          const int n = min(kChunk, tok1 - c0);
-          int pid[kPieces];
-          bool ok = true;
-#pragma unroll
-          for (int i = 0; i < kPieces; ++i) {
-            const int lp = (c0 + 16 * i) / p.page_size;
-            pid[i] = 0;
-            if (16 * i < n) {
-              pid[i] = lp < p.max_pages_per_req ? __ldg(bt_row + lp) : -1;
-              ok = ok && pid[i] >= 0 && pid[i] < p.num_pages;
-            }
-          }
-          if (!ok) break;  // the main loop requests it and reports the page
-          issue_chunk(k, c0, n, pid, true, policy);  // a fresh stage: no "empty" wait
-          ++prefetched;
-        }
-      }
-      prefetched = __shfl_sync(0xffffffffu, prefetched, 0);
-    }
-  }
-  // the producer's lane 0 waits (bounded) for the early requests before the CTA may exit
-  auto drain_prefetch = [&]() {
-    if (warp == kConsumerWarps && lane == 0)
-      for (int k = 0; k < prefetched; ++k) mbar_wait_drain(full0 + 8 * k, 0, p.wait_limit_ns);
-  };
-
   grid_dependency_wait();    // the plan is written by the previous kernel in the stream
   grid_dependents_launch();  // the combine kernel may be scheduled; it waits for this grid to finish
 
@@ -474,7 +430,6 @@ __global__ void __launch_bounds__(kThreads, 2)
   const int h_segs = hdr[kHdrSegments], seg_lo = csb[cta], seg_next = csb[cta + 1];
   if (h_ctas != p.num_ctas || h_batch != p.batch || h_ms != p.max_segments || h_kind != p.kind) {
     if (threadIdx.x == 0 && cta == 0 && g == 0) record_status(hdr_w, DA_DEV_BAD_PLAN, 0);
-    drain_prefetch();
     return;
   }
   const int seg_hi = min(seg_next, min(h_segs, p.max_segments));
@@ -492,11 +447,7 @@ __global__ void __launch_bounds__(kThreads, 2)
       }
     }
   }
-  if (seg_lo < 0 || seg_lo >= seg_hi) {  // nothing planned for this CTA (uniform over the block)
-    if (early.b >= 0 && threadIdx.x == 0) record_status(hdr_w, DA_DEV_BAD_PLAN, cta);  // the plan disagrees
-    drain_prefetch();
-    return;
-  }
+  if (seg_lo < 0 || seg_lo >= seg_hi) return;  // nothing planned for this CTA (uniform over the block)
 
   if (warp == kConsumerWarps) {
     // ------------------------------------------------------------------ producer warp
@@ -506,22 +457,6 @@ __global__ void __launch_bounds__(kThreads, 2)
     uint32_t phase = 0;
     int fills = 0;
     bool aborted = p.stall_producer != 0;  // failure-path test: send nothing
-    int skip = 0;  // chunks of the first segment already requested by the early start
-    if (prefetched > 0) {
-      const int4 sg = segs[seg_lo];
-      if (sg.x == early.b && sg.z == early.tile0 && sg.w == early.tile1) {
-        skip = prefetched;
-      } else {  // cannot happen when the plan was made from the same lengths: stop, drain, report
-        if (lane == 0) {
-          record_status(hdr_w, DA_DEV_BAD_PLAN, cta);
-          *abort_flag = 1;
-        }
-        aborted = true;
-      }
-      fills = prefetched;
-      stage = prefetched % C::kStages;
-      phase = (prefetched / C::kStages) & 1;
-    }
     for (int s = seg_lo; s < seg_hi && !aborted; ++s) {
       // first window of page ids, issued before (and independent of) the length load
       const int4 sg = segs[s];
@@ -534,9 +469,7 @@ __global__ void __launch_bounds__(kThreads, 2)
       const SegmentInfo si = load_segment(p, segs, s);
       if (!si.valid) continue;
       const int32_t* bt_row = p.block_table + (int64_t)si.b * p.max_pages_per_req;
-      const int c_first = si.tok0 + skip * kChunk;  // the early requests: this (first) segment's first chunks
-      skip = 0;
-      for (int c0 = c_first; c0 < si.tok1; c0 += kChunk) {
+      for (int c0 = si.tok0; c0 < si.tok1; c0 += kChunk) {
         const int n = min(kChunk, si.tok1 - c0);
         const int lp_first = c0 / P, lp_last = (c0 + n - 1) / P;
         if (lp_first < win_base || lp_last >= win_base + 32) {
