@@ -31,9 +31,9 @@
 // fp32 state (O and the weight sums) is rescaled to each chunk's reference.
 //
 // Warps: 0-3 softmax (thread t = token t of a chunk for S, dim t for O; warp w
-// reads TMEM lanes 32w..32w+31; thread 0 issues each chunk's P.V as soon as the
-// four warps have written its weights), 4 TMA producer, 5 score-MMA issuer (one
-// thread).
+// reads TMEM lanes 32w..32w+31; each warp announces its weights of a chunk on an
+// mbarrier), 4 TMA producer, 5 MMA issuer (one thread: the score MMA of a chunk as
+// soon as its K/V have landed, its P.V as soon as all four warps' weights are in).
 // TMEM: 64 columns = S[2] and O[2] (16 fp32 columns each), double buffered so
 // the tensor core computes chunk i+1's scores while the softmax warps work on
 // chunk i.  The q tile is double buffered too: segment j+1's tile is written when
@@ -69,10 +69,10 @@ constexpr int kOffP = kOffQ8 + 2 * 2048;         // [2][128 tokens][16 B]
 constexpr int kOffRed = kOffP + 2 * 2048;        // [2][4 warps][8] floats
 constexpr int kOffRowScale = kOffRed + 2 * 32 * 4;  // [2][8] floats
 constexpr int kOffBars = kOffRowScale + 2 * 8 * 4;
-// mbarriers: full[3], empty[3], s_full[2], s_free[2], o_full[2], q_full[2], done (MMA thread), done_pv
-// (softmax thread 0, which issues P.V)
+// mbarriers: full[3], empty[3], s_full[2], s_free[2], o_full[2], q_full[2], done (MMA thread),
+// p_full[2] (the four softmax warps' weights of a chunk are written)
 constexpr int kBarFull = 0, kBarEmpty = 3, kBarSFull = 6, kBarSFree = 8, kBarOFull = 10, kBarQFull = 12,
-              kBarDone = 14, kBarDonePV = 15, kNumBars = 16;
+              kBarDone = 14, kBarPFull = 15, kNumBars = 17;
 constexpr int kOffMeta = kOffBars + kNumBars * 8;  // loaded tokens per stage
 constexpr int kOffFlags = kOffMeta + kStagesTc * 4;  // abort flag, TMEM base address
 constexpr int kBytesTc = kOffFlags + 16;
@@ -266,7 +266,8 @@ __global__ void __launch_bounds__(kThreadsTc, 2)
     mbar_init(bar(kBarQFull), kSoftmaxWarps);
     mbar_init(bar(kBarQFull + 1), kSoftmaxWarps);
     mbar_init(bar(kBarDone), 1);
-    mbar_init(bar(kBarDonePV), 1);
+    mbar_init(bar(kBarPFull), kSoftmaxWarps);
+    mbar_init(bar(kBarPFull + 1), kSoftmaxWarps);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -415,10 +416,10 @@ __global__ void __launch_bounds__(kThreadsTc, 2)
     }
   } else if (warp == kMmaWarp) {
     // ------------------------------------------------------------------ MMA issuer
-    // One thread issues the score MMAs: S of chunk is as soon as its K/V have landed, the
-    // q tile of its segment is written and its score buffer is free.  (P.V is issued by the
-    // softmax warps themselves, the moment their weights are written.)  Chunk ic sits in
-    // stage ic % kStagesTc, S buffer ic % 2.
+    // One thread issues every MMA: S of chunk is as soon as its K/V have landed, the q tile
+    // of its segment is written and its score buffer is free; O of chunk ip (ip < is) as
+    // soon as the four softmax warps have written its weights.  Chunk ic sits in stage
+    // ic % kStagesTc, S, P and O buffers ic % 2.
     if (lane == 0) {
       bool aborted = false;
       auto fail = [&](int s) {
@@ -444,14 +445,31 @@ __global__ void __launch_bounds__(kThreadsTc, 2)
         return false;
       };
       bool more = next_segment();  // chunks left whose S is not issued
-      int is = 0;
+      int is = 0, ip = 0;
       uint64_t t_last = global_timer_ns();
-      for (uint32_t it = 0; !aborted && more; ++it) {
+      for (uint32_t it = 0; !aborted && (more || ip < is); ++it) {
         bool progressed = false;
+        // O^T (chunk ip) = V^T . P'^T, first (it hands the stage back to the producer).  The
+        // softmax warps announce the weights after their fold of chunk ip - 2 (the last reader
+        // of O buffer ip % 2) and after zeroing the V rows past the loaded tokens.
+        if (ip < is && mbar_test(bar(kBarPFull + (ip & 1)), (ip >> 1) & 1)) {
+          tc_fence_after();
+          const int pb = ip & 1, pst = ip % kStagesTc;
+          const uint32_t vt = sbase + kOffStages + pst * kStageBytes + kTileBytes;
+          const uint32_t pt = sbase + kOffP + pb * 2048;
+#pragma unroll
+          for (int j = 0; j < 4; ++j)
+            tc_mma(tmem + 32 + 16 * pb, smem_desc(vt + 4096 * j, 1024, 1024, 2), smem_desc(pt + 512 * j, 128, 128, 0),
+                   kIdescPV, j > 0);
+          tc_commit(bar(kBarOFull + pb));
+          tc_commit(bar(kBarEmpty + pst));
+          ++ip;
+          progressed = true;
+        }
         // S^T (chunk ic) = K . Q8^T, with the q tile of the chunk's segment
-        if (!q_ready) q_ready = mbar_test(bar(kBarQFull + (s_js & 1)), (s_js >> 1) & 1);
+        if (more && !q_ready) q_ready = mbar_test(bar(kBarQFull + (s_js & 1)), (s_js >> 1) & 1);
         const int ic = is, sb = ic & 1, st = ic % kStagesTc;
-        if (q_ready && mbar_test(bar(kBarFull + st), (ic / kStagesTc) & 1) &&
+        if (more && q_ready && mbar_test(bar(kBarFull + st), (ic / kStagesTc) & 1) &&
             (ic < 2 || mbar_test(bar(kBarSFree + sb), ((ic >> 1) - 1) & 1))) {
           tc_fence_after();
           const uint32_t kt = sbase + kOffStages + st * kStageBytes;
@@ -551,7 +569,6 @@ __global__ void __launch_bounds__(kThreadsTc, 2)
       return -1;
     };
     int js = 0;  // segments with chunks seen so far (same count as the MMA thread's)
-    bool pv_issued = false;  // thread 0 has issued P.V MMAs (to drain before TMEM is freed)
     for (int s = seg_lo; s < seg_hi; ++s) {
       const SegmentInfo si = load_segment(p, segs, s);
       if (!si.valid) continue;
@@ -604,7 +621,6 @@ __global__ void __launch_bounds__(kThreadsTc, 2)
           }
           uint32_t sr[16];
           const bool s_ok = wait(bar(kBarSFull + sb), (i >> 1) & 1, s);
-          const bool pv_ok = landed && s_ok;  // thread 0's view decides whether P.V is issued
           if (s_ok) {
             tc_fence_after();
             tc_ld16(lane_base + 16 * sb, sr);
@@ -638,23 +654,10 @@ __global__ void __launch_bounds__(kThreadsTc, 2)
           *reinterpret_cast<uint4*>(smem + kOffP + sb * 2048 + 16 * t) =
               make_uint4(ph[0] | (ph[1] << 16), ph[2] | (ph[3] << 16), pl[0] | (pl[1] << 16), pl[2] | (pl[3] << 16));
           fence_proxy_async_smem();  // P' and the zeroed V rows are read by the tensor core
-          // O^T (chunk i) = V^T . P'^T, issued by thread 0 once all four warps have written their
-          // weights; O buffer sb was last read by the fold of chunk i - 2, which every softmax
-          // thread finished (tcgen05.wait::ld, fence) before this barrier.  The commits hand O to
-          // the fold and the stage back to the producer.
-          named_barrier_sync(1, kSoftmaxWarps * 32);
-          if (t == 0 && pv_ok) {
-            tc_fence_after();
-            const uint32_t vt = sbase + kOffStages + stage * kStageBytes + kTileBytes;
-            const uint32_t pt = sbase + kOffP + sb * 2048;
-#pragma unroll
-            for (int j = 0; j < 4; ++j)
-              tc_mma(tmem + 32 + 16 * sb, smem_desc(vt + 4096 * j, 1024, 1024, 2), smem_desc(pt + 512 * j, 128, 128, 0),
-                     kIdescPV, j > 0);
-            tc_commit(bar(kBarOFull + sb));
-            tc_commit(bar(kBarEmpty + stage));
-            pv_issued = true;
-          }
+          // this warp's weights of chunk i are in (and its fold of chunk i - 2 is done): the MMA
+          // thread issues O^T (chunk i) = V^T . P'^T once all four warps have said so
+          __syncwarp();
+          if (lane == 0) mbar_arrive(bar(kBarPFull + sb));
           if (k > 0) fold(i - 1, f_prev);
 #pragma unroll
           for (int h = 0; h < 8; ++h) f_prev[h] = f[h];
@@ -687,11 +690,6 @@ __global__ void __launch_bounds__(kThreadsTc, 2)
             p.partial_lse[(int64_t)s * p.num_q_heads + row] = lse;
         }
       }
-    }
-    // drain: thread 0's P.V MMAs have completed before TMEM is freed and the stages' barriers die
-    if (t == 0 && pv_issued) {
-      tc_commit(bar(kBarDonePV));
-      mbar_wait_timeout(bar(kBarDonePV), 0, p.wait_limit_ns);
     }
   }
 
