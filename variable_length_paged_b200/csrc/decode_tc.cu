@@ -1,6 +1,6 @@
 // decode_tc.cu -- split-KV decode attention over an FP8 (E4M3) paged KV cache
 // on the 5th-generation tensor cores: tcgen05.mma with accumulators in tensor
-// memory (TMEM), operands straight from the TMA-filled shared-memory ring.
+// memory (TMEM), operands straight from the TMA-filled shared-memory rings.
 //
 // "Tencent HPC lands in SGLang, challenging default inference kernels",
 // sections "Why Tencent HPC matters for online model serving" (attention over
@@ -33,12 +33,20 @@
 // Warps: 0-3 softmax (thread t = token t of a chunk for S, dim t for O; warp w
 // reads TMEM lanes 32w..32w+31; each warp announces its weights of a chunk on an
 // mbarrier), 4 TMA producer, 5 MMA issuer (one thread: the score MMA of a chunk as
-// soon as its K/V have landed, its P.V as soon as all four warps' weights are in).
+// soon as its K tile has landed, its P.V as soon as all four warps' weights are in).
+//
+// K and V of a chunk are requested together but held in separate rings: a K
+// tile is read once, by the score MMA, and its slot is handed back when that
+// MMA completes (~2.3 us after the request under load); a V tile waits for the
+// softmax and the P.V MMA as well (~4 us).  Two K slots and four V slots (96 KB,
+// the same as three joint stages) keep up to four chunks in flight where joint
+// stages allowed three, with the K ring no longer held through the softmax.
+//
 // TMEM: 64 columns = S[2] and O[2] (16 fp32 columns each), double buffered so
 // the tensor core computes chunk i+1's scores while the softmax warps work on
 // chunk i.  The q tile is double buffered too: segment j+1's tile is written when
-// segment j starts, so the MMA thread runs on across segment boundaries.  Every wait is bounded (DecodeParams::wait_limit_ns); TMEM is freed on
-// every path out.
+// segment j starts, so the MMA thread runs on across segment boundaries.  Every
+// wait is bounded (DecodeParams::wait_limit_ns); TMEM is freed on every path out.
 #include <cuda_fp16.h>
 
 #include <cfloat>
@@ -50,31 +58,32 @@ namespace da {
 namespace {
 
 constexpr int kD = 128;               // head_dim: one 128-byte row of E4M3 codes
-constexpr int kChunk = 128;           // tokens per stage = lanes of one MMA
+constexpr int kChunk = 128;           // tokens per chunk = lanes of one MMA
 constexpr int kSoftmaxWarps = 4;
 constexpr int kProducerWarp = 4;
 constexpr int kMmaWarp = 5;
 constexpr int kThreadsTc = 6 * 32;
-constexpr int kStagesTc = 3;
+constexpr int kKSlots = 2;            // K tiles, each freed when its chunk's score MMA completes
+constexpr int kVSlots = 4;            // V tiles, each freed when its chunk's P.V MMA completes
 constexpr int kTileBytes = kChunk * 128;  // K (or V) of one chunk: 16 KB
-constexpr int kStageBytes = 2 * kTileBytes;
 constexpr uint32_t kTmemCols = 64;    // S[2] at columns 0, 16; O[2] at 32, 48
 constexpr float kPShift = 8.f;        // P' = 2^8 P
 constexpr float kFloor = 40.f;        // a chunk's reference stays within 2^40 of the running max
 
 // shared memory map (offsets from a 1024-byte aligned base)
-constexpr int kOffStages = 0;
-constexpr int kOffQ8 = kStagesTc * kStageBytes;  // [2][16 rows x 128 B], 128-byte swizzle (1024-aligned)
+constexpr int kOffK = 0;                          // [kKSlots][128 tokens x 128 B], 128-byte swizzle
+constexpr int kOffV = kOffK + kKSlots * kTileBytes;  // [kVSlots][128 tokens x 128 B], 128-byte swizzle
+constexpr int kOffQ8 = kOffV + kVSlots * kTileBytes;  // [2][16 rows x 128 B], 128-byte swizzle (1024-aligned)
 constexpr int kOffP = kOffQ8 + 2 * 2048;         // [2][128 tokens][16 B]
 constexpr int kOffRed = kOffP + 2 * 2048;        // [2][4 warps][8] floats
 constexpr int kOffRowScale = kOffRed + 2 * 32 * 4;  // [2][8] floats
 constexpr int kOffBars = kOffRowScale + 2 * 8 * 4;
-// mbarriers: full[3], empty[3], s_full[2], s_free[2], o_full[2], q_full[2], done (MMA thread),
-// p_full[2] (the four softmax warps' weights of a chunk are written)
-constexpr int kBarFull = 0, kBarEmpty = 3, kBarSFull = 6, kBarSFree = 8, kBarOFull = 10, kBarQFull = 12,
-              kBarDone = 14, kBarPFull = 15, kNumBars = 17;
-constexpr int kOffMeta = kOffBars + kNumBars * 8;  // loaded tokens per stage
-constexpr int kOffFlags = kOffMeta + kStagesTc * 4;  // abort flag, TMEM base address
+// mbarriers: k_full[2], k_empty[2], v_full[4], v_empty[4], s_full[2], s_free[2], o_full[2],
+// q_full[2], done (MMA thread), p_full[2] (the four softmax warps' weights of a chunk are written)
+constexpr int kBarKFull = 0, kBarKEmpty = 2, kBarVFull = 4, kBarVEmpty = 8, kBarSFull = 12, kBarSFree = 14,
+              kBarOFull = 16, kBarQFull = 18, kBarDone = 20, kBarPFull = 21, kNumBars = 23;
+constexpr int kOffMeta = kOffBars + kNumBars * 8;  // loaded tokens of the chunk in each V slot
+constexpr int kOffFlags = kOffMeta + kVSlots * 4;  // abort flag, TMEM base address
 constexpr int kBytesTc = kOffFlags + 16;
 constexpr int kSmemTc = kBytesTc + 1024;  // slack for the manual 1024-byte alignment
 static_assert(kOffQ8 % 1024 == 0 && kOffP % 16 == 0 && kOffBars % 8 == 0, "alignment");
@@ -254,9 +263,13 @@ __global__ void __launch_bounds__(kThreadsTc, 2)
   volatile uint32_t* tmem_slot = reinterpret_cast<volatile uint32_t*>(smem + kOffFlags + 4);
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < kStagesTc; ++s) {
-      mbar_init(bar(kBarFull + s), 1);
-      mbar_init(bar(kBarEmpty + s), 1);  // released by the tensor core (commit after P.V)
+    for (int s = 0; s < kKSlots; ++s) {
+      mbar_init(bar(kBarKFull + s), 1);
+      mbar_init(bar(kBarKEmpty + s), 1);  // released by the tensor core (commit after S)
+    }
+    for (int s = 0; s < kVSlots; ++s) {
+      mbar_init(bar(kBarVFull + s), 1);
+      mbar_init(bar(kBarVEmpty + s), 1);  // released by the tensor core (commit after P.V)
     }
     for (int j = 0; j < 2; ++j) {
       mbar_init(bar(kBarSFull + j), 1);
@@ -279,43 +292,44 @@ __global__ void __launch_bounds__(kThreadsTc, 2)
   }
   __syncthreads();
 
-  // Stage `stage` <- K and V codes of tokens [c0, c0 + n) of one request, whose 16-token
-  // pieces sit in pages pid[]; the stage's "full" barrier expects the bytes.  Lane 0 of the
-  // producer.
+  // K slot ks <- K codes, V slot vs <- V codes of tokens [c0, c0 + n) of one request, whose
+  // 16-token pieces sit in pages pid[]; each slot's "full" barrier expects its bytes.  Both
+  // tiles of a chunk are requested together.  Lane 0 of the producer.
   constexpr int kPieces = kChunk / 16;
-  auto issue_chunk = [&](int stage, int c0, int n, const int (&pid)[kPieces], bool ok, uint64_t policy) {
+  auto issue_chunk = [&](int ks, int vs, int c0, int n, const int (&pid)[kPieces], bool ok, uint64_t policy) {
     const int P = p.page_size;
-    meta[stage] = ok ? n : 0;
-    uint32_t bytes = 0;
+    meta[vs] = ok ? n : 0;
+    uint32_t bytes = 0;  // of one tile
     if (ok) {
 #pragma unroll
       for (int j = 0; j < kChunk / 64; ++j) {
         if (64 * j >= n) break;
         const bool fast = ((c0 + 64 * j) % P) + 64 <= P;
         const int pieces = fast ? 4 : min(4, (n - 64 * j + 15) >> 4);
-        bytes += (uint32_t)(pieces * 16 * 128 * 2);
+        bytes += (uint32_t)(pieces * 16 * 128);
       }
     }
-    const uint32_t full = bar(kBarFull + stage);
-    mbar_arrive_expect_tx(full, bytes);
+    const uint32_t kfull = bar(kBarKFull + ks), vfull = bar(kBarVFull + vs);
+    mbar_arrive_expect_tx(kfull, bytes);
+    mbar_arrive_expect_tx(vfull, bytes);
     if (ok) {
-      const uint32_t sk = sbase + kOffStages + stage * kStageBytes, sv = sk + kTileBytes;
+      const uint32_t sk = sbase + kOffK + ks * kTileBytes, sv = sbase + kOffV + vs * kTileBytes;
 #pragma unroll
       for (int j = 0; j < kChunk / 64; ++j) {
         if (64 * j >= n) break;
         const int tok = c0 + 64 * j;
         if ((tok % P) + 64 <= P) {
           const int row = (pid[4 * j] * p.num_kv_heads + g) * P + tok % P;
-          tma_load_2d(sk + j * 64 * 128, &k64, 0, row, full, policy);
-          tma_load_2d(sv + j * 64 * 128, &v64, 0, row, full, policy);
+          tma_load_2d(sk + j * 64 * 128, &k64, 0, row, kfull, policy);
+          tma_load_2d(sv + j * 64 * 128, &v64, 0, row, vfull, policy);
         } else {
 #pragma unroll
           for (int i = 0; i < 4; ++i) {
             if (64 * j + 16 * i >= n) break;
             const int row = (pid[4 * j + i] * p.num_kv_heads + g) * P + (tok + 16 * i) % P;
             const uint32_t off = (64 * j + 16 * i) * 128;
-            tma_load_2d(sk + off, &k16, 0, row, full, policy);
-            tma_load_2d(sv + off, &v16, 0, row, full, policy);
+            tma_load_2d(sk + off, &k16, 0, row, kfull, policy);
+            tma_load_2d(sv + off, &v16, 0, row, vfull, policy);
           }
         }
       }
@@ -340,23 +354,26 @@ __global__ void __launch_bounds__(kThreadsTc, 2)
   const int seg_hi = min(seg_next, min(h_segs, p.max_segments));
   if (seg_lo < 0 || seg_lo >= seg_hi) return;  // nothing planned for this CTA (uniform over the block)
 
-  // TMEM for this CTA (64 of the SM's 512 columns; two CTAs per SM)
-  if (warp == kMmaWarp) {
-    tmem_alloc(smem_u32(const_cast<uint32_t*>(tmem_slot)), kTmemCols);
-    tmem_relinquish();
+  // TMEM for this CTA (64 of the SM's 512 columns; two CTAs per SM).  The producer does not
+  // wait for it: its first requests go out while the MMA warp allocates and the softmax
+  // warps build the first q tile.
+  uint32_t tmem = 0;
+  if (warp != kProducerWarp) {
+    if (warp == kMmaWarp) {
+      tmem_alloc(smem_u32(const_cast<uint32_t*>(tmem_slot)), kTmemCols);
+      tmem_relinquish();
+    }
+    tc_fence_before();
+    named_barrier_sync(2, (kSoftmaxWarps + 1) * 32);
+    tc_fence_after();
+    tmem = *tmem_slot;
   }
-  tc_fence_before();
-  __syncthreads();
-  tc_fence_after();
-  const uint32_t tmem = *tmem_slot;
 
   if (warp == kProducerWarp) {
     // ------------------------------------------------------------------ TMA producer
     const uint64_t policy = policy_evict_first();
     const int P = p.page_size;
-    int stage = 0;
-    uint32_t phase = 0;
-    int fills = 0;
+    int fills = 0;  // chunks requested: chunk k goes to K slot k % kKSlots, V slot k % kVSlots
     bool aborted = p.stall_producer != 0;  // failure-path test: send nothing
     for (int s = seg_lo; s < seg_hi && !aborted; ++s) {
       const int4 sg = segs[s];
@@ -385,8 +402,14 @@ __global__ void __launch_bounds__(kThreadsTc, 2)
           pid[i] = __shfl_sync(0xffffffffu, win_val, (lp - win_base) & 31);
           if (16 * i < n) ok = ok && pid[i] >= 0 && pid[i] < p.num_pages;
         }
+        // wait until the tensor core has released both slots (S of chunk fills - kKSlots, P.V of
+        // chunk fills - kVSlots)
+        const int ks = fills % kKSlots, vs = fills % kVSlots;
         bool got = true;
-        if (lane == 0) got = mbar_wait_bounded(bar(kBarEmpty + stage), phase ^ 1, abort_flag, p.wait_limit_ns);
+        if (lane == 0) {
+          got = mbar_wait_bounded(bar(kBarKEmpty + ks), ((fills / kKSlots) & 1) ^ 1, abort_flag, p.wait_limit_ns) &&
+                mbar_wait_bounded(bar(kBarVEmpty + vs), ((fills / kVSlots) & 1) ^ 1, abort_flag, p.wait_limit_ns);
+        }
         got = __shfl_sync(0xffffffffu, got, 0);
         if (!got) {
           if (lane == 0) {
@@ -398,28 +421,27 @@ __global__ void __launch_bounds__(kThreadsTc, 2)
         }
         if (lane == 0) {
           if (!ok) record_status(hdr_w, DA_DEV_BAD_PAGE, si.b);
-          issue_chunk(stage, c0, n, pid, ok, policy);
+          issue_chunk(ks, vs, c0, n, pid, ok, policy);
         }
         __syncwarp();
         ++fills;
-        if (++stage == kStagesTc) {
-          stage = 0;
-          phase ^= 1;
-        }
       }
     }
-    // every stage's last fill must have landed before the CTA may exit (also after an abort:
+    // every slot's last fill must have landed before the CTA may exit (also after an abort:
     // the copies were requested, so they are waited for, within the limit)
     if (lane == 0) {
-      for (int k = max(0, fills - kStagesTc); k < fills; ++k)
-        mbar_wait_drain(bar(kBarFull + k % kStagesTc), (k / kStagesTc) & 1, p.wait_limit_ns);
+      for (int k = max(0, fills - kKSlots); k < fills; ++k)
+        mbar_wait_drain(bar(kBarKFull + k % kKSlots), (k / kKSlots) & 1, p.wait_limit_ns);
+      for (int k = max(0, fills - kVSlots); k < fills; ++k)
+        mbar_wait_drain(bar(kBarVFull + k % kVSlots), (k / kVSlots) & 1, p.wait_limit_ns);
     }
   } else if (warp == kMmaWarp) {
     // ------------------------------------------------------------------ MMA issuer
-    // One thread issues every MMA: S of chunk is as soon as its K/V have landed, the q tile
+    // One thread issues every MMA: S of chunk ic as soon as its K tile has landed, the q tile
     // of its segment is written and its score buffer is free; O of chunk ip (ip < is) as
-    // soon as the four softmax warps have written its weights.  Chunk ic sits in stage
-    // ic % kStagesTc, S, P and O buffers ic % 2.
+    // soon as the four softmax warps have written its weights.  Chunk k sits in K slot
+    // k % kKSlots and V slot k % kVSlots; S, P and O buffers k % 2.  The commit after S hands
+    // the K slot back to the producer, the commit after P.V the V slot.
     if (lane == 0) {
       bool aborted = false;
       auto fail = [&](int s) {
@@ -449,36 +471,40 @@ __global__ void __launch_bounds__(kThreadsTc, 2)
       uint64_t t_last = global_timer_ns();
       for (uint32_t it = 0; !aborted && (more || ip < is); ++it) {
         bool progressed = false;
-        // O^T (chunk ip) = V^T . P'^T, first (it hands the stage back to the producer).  The
+        // O^T (chunk ip) = V^T . P'^T, first (it hands a V slot back to the producer).  The
         // softmax warps announce the weights after their fold of chunk ip - 2 (the last reader
-        // of O buffer ip % 2) and after zeroing the V rows past the loaded tokens.
-        if (ip < is && mbar_test(bar(kBarPFull + (ip & 1)), (ip >> 1) & 1)) {
+        // of O buffer ip % 2) and after zeroing the V rows past the loaded tokens, which they
+        // do once the V tile has landed.
+        const int pvs = ip % kVSlots;
+        if (ip < is && mbar_test(bar(kBarPFull + (ip & 1)), (ip >> 1) & 1) &&
+            mbar_test(bar(kBarVFull + pvs), (ip / kVSlots) & 1)) {
           tc_fence_after();
-          const int pb = ip & 1, pst = ip % kStagesTc;
-          const uint32_t vt = sbase + kOffStages + pst * kStageBytes + kTileBytes;
+          const int pb = ip & 1;
+          const uint32_t vt = sbase + kOffV + pvs * kTileBytes;
           const uint32_t pt = sbase + kOffP + pb * 2048;
 #pragma unroll
           for (int j = 0; j < 4; ++j)
             tc_mma(tmem + 32 + 16 * pb, smem_desc(vt + 4096 * j, 1024, 1024, 2), smem_desc(pt + 512 * j, 128, 128, 0),
                    kIdescPV, j > 0);
           tc_commit(bar(kBarOFull + pb));
-          tc_commit(bar(kBarEmpty + pst));
+          tc_commit(bar(kBarVEmpty + pvs));
           ++ip;
           progressed = true;
         }
         // S^T (chunk ic) = K . Q8^T, with the q tile of the chunk's segment
         if (more && !q_ready) q_ready = mbar_test(bar(kBarQFull + (s_js & 1)), (s_js >> 1) & 1);
-        const int ic = is, sb = ic & 1, st = ic % kStagesTc;
-        if (more && q_ready && mbar_test(bar(kBarFull + st), (ic / kStagesTc) & 1) &&
+        const int ic = is, sb = ic & 1, ks = ic % kKSlots;
+        if (more && q_ready && mbar_test(bar(kBarKFull + ks), (ic / kKSlots) & 1) &&
             (ic < 2 || mbar_test(bar(kBarSFree + sb), ((ic >> 1) - 1) & 1))) {
           tc_fence_after();
-          const uint32_t kt = sbase + kOffStages + st * kStageBytes;
+          const uint32_t kt = sbase + kOffK + ks * kTileBytes;
           const uint32_t q8 = sbase + kOffQ8 + (s_js & 1) * 2048;
 #pragma unroll
           for (int j = 0; j < 4; ++j)
             tc_mma(tmem + 16 * sb, smem_desc(kt + 32 * j, 16, 1024, 2), smem_desc(q8 + 32 * j, 16, 1024, 2),
                    kIdescS, j > 0);
           tc_commit(bar(kBarSFull + sb));
+          tc_commit(bar(kBarKEmpty + ks));
           ++is;
           progressed = true;
           if (is == s_end) more = next_segment();
@@ -504,8 +530,6 @@ __global__ void __launch_bounds__(kThreadsTc, 2)
     float* red = reinterpret_cast<float*>(smem + kOffRed);
     float* row_scale = reinterpret_cast<float*>(smem + kOffRowScale);
     const int G = p.group;
-    int stage = 0;
-    uint32_t phase = 0;
     int i = 0, calls = 0;
     auto fail = [&](int s) {
       if (lane == 0) {
@@ -612,10 +636,11 @@ __global__ void __launch_bounds__(kThreadsTc, 2)
         for (int k = 0; k < nch; ++k, ++i) {
           const int sb = i & 1;
           int n = 0;
-          const bool landed = wait(bar(kBarFull + stage), phase, s);
-          if (landed) n = meta[stage];
+          const int vs = i % kVSlots;
+          const bool landed = wait(bar(kBarVFull + vs), (i / kVSlots) & 1, s);
+          if (landed) n = meta[vs];
           if (landed && t >= n) {  // V rows past the loaded tokens may hold anything (NaN too): zero them
-            uint4* vrow = reinterpret_cast<uint4*>(smem + kOffStages + stage * kStageBytes + kTileBytes + t * 128);
+            uint4* vrow = reinterpret_cast<uint4*>(smem + kOffV + vs * kTileBytes + t * 128);
 #pragma unroll
             for (int c = 0; c < 8; ++c) vrow[c] = make_uint4(0, 0, 0, 0);
           }
@@ -661,10 +686,6 @@ __global__ void __launch_bounds__(kThreadsTc, 2)
           if (k > 0) fold(i - 1, f_prev);
 #pragma unroll
           for (int h = 0; h < 8; ++h) f_prev[h] = f[h];
-          if (++stage == kStagesTc) {
-            stage = 0;
-            phase ^= 1;
-          }
         }
         fold(i - 1, f_prev);
       }
