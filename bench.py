@@ -150,6 +150,8 @@ def recorded_traffic(workload_name, kv="bf16", q_len=1):
             j = dict(ln.split(": ", 1) for ln in f.read().splitlines() if ln and not ln.startswith("#"))
     except Exception:
         return None, f"no ncu capture recorded ({rel} missing)"
+    if os.environ.get("DA_LIB_PATH"):
+        return None, "a library built with other definitions (DA_LIB_PATH) is loaded; the record is for the default build"
     if j.get(f"kernel_source_sha.{kv}") != kernel_source_hash(kv):
         return None, f"{kv} decode kernel changed since the ncu capture in {rel}"
     key = f"{workload_name}.{kv}"

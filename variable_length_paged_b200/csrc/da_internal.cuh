@@ -120,18 +120,27 @@ struct SegmentInfo {
   bool valid;
 };
 
-__device__ __forceinline__ SegmentInfo load_segment(const DecodeParams& p, const int4* segs, int s) {
-  const int4 sg = segs[s];
+__device__ __forceinline__ bool segment_entry_valid(const DecodeParams& p, int4 sg) {
+  return sg.x >= 0 && sg.x < p.batch && sg.z >= 0 && sg.w >= sg.z;
+}
+
+// The segment of plan entry sg, given its request's length as read from seq_lens (any value
+// for an invalid entry).  Split from the loads so that a kernel can request them early.
+__device__ __forceinline__ SegmentInfo make_segment(const DecodeParams& p, int4 sg, int L) {
   SegmentInfo r;
   r.b = sg.x;
-  r.valid = sg.x >= 0 && sg.x < p.batch && sg.z >= 0 && sg.w >= sg.z;
-  int L = r.valid ? p.seq_lens[sg.x] : 0;
-  if (L < 0 || (int64_t)L > p.capacity_tokens) L = 0;
+  r.valid = segment_entry_valid(p, sg);
+  if (!r.valid || L < 0 || (int64_t)L > p.capacity_tokens) L = 0;
   const int64_t t0 = (int64_t)sg.z * p.tile_tokens, t1 = min((int64_t)sg.w * p.tile_tokens, (int64_t)L);
   r.tok0 = (int)min(t0, (int64_t)L);
   r.tok1 = (int)t1;
   r.len = L;
   return r;
+}
+
+__device__ __forceinline__ SegmentInfo load_segment(const DecodeParams& p, const int4* segs, int s) {
+  const int4 sg = segs[s];
+  return make_segment(p, sg, segment_entry_valid(p, sg) ? p.seq_lens[sg.x] : 0);
 }
 
 // Host launchers (defined next to their kernels).

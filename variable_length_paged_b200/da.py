@@ -12,7 +12,8 @@ import ctypes
 import os
 
 HERE = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(HERE, "libda.so")
+# DA_LIB_PATH selects another build of the library (one made with `build --define ... --out`)
+LIB_PATH = os.environ.get("DA_LIB_PATH") or os.path.join(HERE, "libda.so")
 
 OK, ERR_INVALID_ARG, ERR_UNSUPPORTED, ERR_CUDA, ERR_WORKSPACE = 0, -1, -2, -3, -4
 DEV_OK, DEV_BAD_SEQLEN, DEV_BAD_PAGE, DEV_TIMEOUT, DEV_BAD_PLAN = 0, 1, 2, 3, 4
