@@ -342,7 +342,6 @@ __global__ void __launch_bounds__(kThreadsTc, 2)
   const WsLayout WL = ws_layout(p.batch, p.num_ctas, p.max_segments, p.num_kv_heads);
   const int32_t* hdr = p.ws + WL.hdr;
   const int4* segs = reinterpret_cast<const int4*>(p.ws + WL.segs);
-  const int32_t* rsb = p.ws + WL.req_seg_begin;
   const int32_t* csb = p.ws + WL.cta_seg_begin;
   int32_t* hdr_w = const_cast<int32_t*>(hdr);
   const int h_ctas = hdr[kHdrCtas], h_batch = hdr[kHdrBatch], h_ms = hdr[kHdrMaxSegments], h_kind = hdr[kHdrKind];
@@ -693,7 +692,13 @@ __global__ void __launch_bounds__(kThreadsTc, 2)
       // ---- the segment's result: per head, O / (sum of weights) and the log-sum-exp
       float lt[8];
       reduce8<false>(l_part, lt, red + 32 * (calls++ & 1), warp, lane);
-      const bool direct = rsb[b + 1] - rsb[b] == 1 && !p.out_f32;  // fp32 output: the combine writes it
+      // one segment for the request (no load of its segment count): in a dynamic plan, whose
+      // segments are never empty, when this one covers all of it; in a static plan, whose
+      // requests have S segments each (empty ones too), when S = 1.  With fp32 output the
+      // combine writes every request.
+      const bool one_segment = p.kind == DA_PLAN_DYNAMIC ? si.tok0 == 0 && si.tok1 == si.len && si.len > 0
+                                                         : p.num_ctas == p.batch;
+      const bool direct = one_segment && !p.out_f32;
 #pragma unroll
       for (int h = 0; h < 8; ++h) {
         if (h >= G) break;
