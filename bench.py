@@ -68,6 +68,8 @@ def parse_args():
     ap.add_argument("--width", type=int, default=0, help="CTAs per KV head (0 = 2 per SM / Hkv)")
     ap.add_argument("--merge-in-decode", action="store_true",
                     help="dynamic plan: merge split requests in the decode kernel instead of a combine launch")
+    ap.add_argument("--start-cost", type=int, default=None,
+                    help="dynamic plan: units charged to the CTA that starts a request (default: the library's)")
     ap.add_argument("--no-static", action="store_true", help="skip the static split-k comparison")
     ap.add_argument("--no-cpu", action="store_true", help="skip the CPU oracle baseline")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
@@ -282,7 +284,8 @@ def run_ours(args, world, rank, local):
     w8 = W.quantize_fp8(w) if args.kv == "fp8" else None
     dw = w8.to("cuda") if w8 is not None else w.to("cuda")
     prob = da.problem_from(dw.problem)
-    desc = da.da_plan_desc_init(prob, da.PLAN_DYNAMIC, args.tile, args.width, merge_in_decode=args.merge_in_decode)
+    desc = da.da_plan_desc_init(prob, da.PLAN_DYNAMIC, args.tile, args.width, merge_in_decode=args.merge_in_decode,
+                                start_cost=args.start_cost)
     bufs = da.Buffers(prob, desc, "cuda")
     kv_bytes = w8.kv_bytes if w8 is not None else w.kv_bytes
     stream = torch.cuda.Stream()
@@ -391,7 +394,7 @@ def run_ours(args, world, rank, local):
         higher_is_better=True, scaling="weak", vs_baseline=None, dtype="bf16", data="synthetic",
         config=workload_config(args.config, w, w8, args.q_len),
         launch={"tile_tokens": desc.tile_tokens, "ctas_per_kv_head": desc.num_ctas,
-                "merge_in_decode": bool(desc.merge_in_decode), "graph": True,
+                "merge_in_decode": bool(desc.merge_in_decode), "start_cost": int(desc.start_cost), "graph": True,
                 "timing": "one CUDA graph per step (plan, decode, combine), K replays between CUDA events on "
                           "the launching stream; median/p10/p90 from a second pass of K replays with an event "
                           "between replays"},
@@ -458,7 +461,8 @@ def run_trace(args, world, rank, local):
     dt = DeviceTrace(tr)
     prob = dt.prob
     stream = torch.cuda.Stream()
-    desc = da.da_plan_desc_init(prob, da.PLAN_DYNAMIC, args.tile, args.width, merge_in_decode=args.merge_in_decode)
+    desc = da.da_plan_desc_init(prob, da.PLAN_DYNAMIC, args.tile, args.width, merge_in_decode=args.merge_in_decode,
+                                start_cost=args.start_cost)
     sdesc = da.da_plan_desc_init(prob, da.PLAN_STATIC, args.tile, 0)
     bufs, sbufs = da.Buffers(prob, desc, "cuda"), da.Buffers(prob, sdesc, "cuda")
     steps, warm = min(max(1, args.steps), tr.steps), max(3, args.warmup)
@@ -523,7 +527,8 @@ def run_trace(args, world, rank, local):
         higher_is_better=True, scaling="weak", vs_baseline=None, dtype="bf16", data="synthetic",
         config={"workload": f"trace: {tr.recipe}", "batch": prob.batch, "steps_timed": steps,
                 "kv_bytes_first_last_step": [kv[0], kv[-1]], "tile_tokens": desc.tile_tokens,
-                "ctas_per_kv_head": desc.num_ctas, "merge_in_decode": bool(desc.merge_in_decode), "graph": True,
+                "ctas_per_kv_head": desc.num_ctas, "merge_in_decode": bool(desc.merge_in_decode),
+                "start_cost": int(desc.start_cost), "graph": True,
                 "untimed": "device copies of each step's changes (restarted pages, block table, lengths, q) "
                            "and the KV append kernel, enqueued between the timed steps",
                 "l2": f"inputs larger than L2 ({min(kv) / 1e9:.1f}-{max(kv) / 1e9:.1f} GB K/V per step), no flush"},

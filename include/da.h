@@ -153,10 +153,18 @@ typedef struct da_plan_desc {
                               merge.  Every segment's result then goes to the partials and
                               da_combine writes `out` for every request (also those with one
                               segment); merge_in_decode must be 0 */
+  int32_t start_cost;      /* dynamic plans: units charged, besides its tiles, to the CTA that starts
+                              a request (the fixed cost of a segment: loading the request's query,
+                              merging and writing its result).  The plan spreads tiles plus these
+                              start units evenly, so a CTA that starts many short requests gets
+                              fewer tiles.  Default 2 (measured on B200 at 64-token tiles); 0 is the
+                              tiles-only plan.  Must be 0 for a static plan. */
 } da_plan_desc;
 
 /*
- * da_plan_desc_init -- validate a problem and fix the plan geometry.
+ * da_plan_desc_init -- validate a problem and fix the plan geometry (and set
+ * merge_in_decode = 0, out_format = DA_OUT_BF16, start_cost = 2 for a dynamic
+ * plan, 0 for a static one; change those fields afterwards if wanted).
  *   kind         DA_PLAN_DYNAMIC or DA_PLAN_STATIC.
  *   tile_tokens  T > 0, a multiple of 16; 0 = default (64).
  *   width        dynamic: C, CTAs per KV head; 0 = default

@@ -68,6 +68,8 @@ def _bind(path: str):
                  _i32p, _i32p]
     lib.dao_plan.restype = ctypes.c_int
     lib.dao_plan.argtypes = plan_args
+    lib.dao_plan_start_cost.restype = ctypes.c_int
+    lib.dao_plan_start_cost.argtypes = plan_args + [ctypes.c_int32]
     lib.dao_static_plan.restype = ctypes.c_int
     lib.dao_static_plan.argtypes = plan_args
     lib.dao_num_threads.restype = ctypes.c_int
@@ -257,7 +259,7 @@ def combine(o_parts, lse_parts, lib=None):
     return out, float(lse[0])
 
 
-def _run_plan(fn, seq_lens, tile_tokens, width, capacity_tokens, max_segments, num_ctas):
+def _run_plan(fn, seq_lens, tile_tokens, width, capacity_tokens, max_segments, num_ctas, *extra):
     sl = np.ascontiguousarray(seq_lens, dtype=np.int32)
     B = sl.shape[0]
     arr = lambda n: np.zeros((n,), dtype=np.int32)
@@ -269,7 +271,7 @@ def _run_plan(fn, seq_lens, tile_tokens, width, capacity_tokens, max_segments, n
             ctypes.byref(nu), ctypes.byref(ns), *[_ptr(res[k], ctypes.c_int32) for k in
                                                    ("req_tile_prefix", "req_seg_begin", "cta_seg_begin", "seg_req",
                                                     "seg_cta", "seg_tile_begin", "seg_tile_end")],
-            ctypes.byref(bad))
+            ctypes.byref(bad), *extra)
     if st not in (OK, ERR_BAD_SEQLEN):
         raise ValueError(f"oracle plan failed with status {st}")
     S = ns.value
@@ -280,11 +282,17 @@ def _run_plan(fn, seq_lens, tile_tokens, width, capacity_tokens, max_segments, n
     return res
 
 
-def plan(seq_lens, tile_tokens: int, num_ctas: int, capacity_tokens: int, lib=None):
-    """Dynamic plan (dict of int32 arrays; see ``dao_plan`` in dao.c)."""
+def plan(seq_lens, tile_tokens: int, num_ctas: int, capacity_tokens: int, lib=None, start_cost: int = 0):
+    """Dynamic plan (dict of int32 arrays; see ``dao_plan_start_cost`` in dao.c).
+
+    start_cost: start units charged to every non-empty request (0: every unit is a tile)."""
     B = len(seq_lens)
-    return _run_plan((lib or _load()).dao_plan, seq_lens, tile_tokens, num_ctas, capacity_tokens,
-                     num_ctas + max(B, 1) - 1, num_ctas)
+    lib = lib or _load()
+    if start_cost == 0:
+        return _run_plan(lib.dao_plan, seq_lens, tile_tokens, num_ctas, capacity_tokens, num_ctas + max(B, 1) - 1,
+                         num_ctas)
+    return _run_plan(lib.dao_plan_start_cost, seq_lens, tile_tokens, num_ctas, capacity_tokens,
+                     num_ctas + max(B, 1) - 1, num_ctas, int(start_cost))
 
 
 def static_plan(seq_lens, tile_tokens: int, splits: int, capacity_tokens: int, lib=None):

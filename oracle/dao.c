@@ -314,33 +314,49 @@ static int32_t first_bad_length(int32_t batch, const int32_t* seq_lens, int64_t 
 
 /*
  * Dynamic (load-balanced) plan, written from its definition by walking the
- * global tile units in order.
+ * global units in order.
  *
- *   n_b  = ceil(L_b / T),  prefix[b] = sum_{r<b} n_r,  U = prefix[B]
- *   unit u belongs to request r with prefix[r] <= u < prefix[r+1] and to the
- *   CTA c(u) = floor(((u+1)*C - 1) / U), the unique c with
+ *   n_b  = ceil(L_b / T) tiles;  w_b = n_b + sigma when n_b > 0, else 0
+ *   prefix[b] = sum_{r<b} w_r,  U = prefix[B]
+ *   The units of request r are [prefix[r], prefix[r+1]): the first sigma of
+ *   them stand for the fixed cost of starting the request and carry no tokens
+ *   ("start units"), the rest are its tiles 0 .. n_r - 1 in order.  With
+ *   sigma = start_cost = 0 every unit is a tile.
+ *   unit u belongs to the CTA c(u) = floor(((u+1)*C - 1) / U), the unique c with
  *   floor(c*U/C) <= u < floor((c+1)*U/C).
- *   A segment is a maximal run of consecutive units with the same
+ *   A segment is a maximal run of consecutive tile units with the same
  *   (request, CTA); segments are numbered in unit order.
  *
+ * The tiles are the article's uniform units of KV-cache work, spread over the
+ * CTAs by the current lengths ("Tencent HPC lands in SGLang, challenging default
+ * inference kernels", section "Why Tencent HPC matters for online model
+ * serving").  The article gives no planner; the start units are this
+ * implementation's addition: a CTA pays a fixed cost for every request it
+ * starts (loading its query, merging and writing its result), so a CTA whose
+ * range starts many short requests is given correspondingly fewer tiles.
+ *
  * Outputs (caller-allocated):
- *   req_tile_prefix[B+1], req_seg_begin[B+1] (segments of request b are
- *   [req_seg_begin[b], req_seg_begin[b+1])), cta_seg_begin[C+1] (segments of
- *   CTA c are [cta_seg_begin[c], cta_seg_begin[c+1])), seg_req, seg_cta,
- *   seg_tile_begin, seg_tile_end [max_segments] (tile indices relative to the
- *   request), *num_units, *num_segments, *bad_index (-1 if none).
+ *   req_tile_prefix[B+1] (= prefix[], start units included), req_seg_begin[B+1]
+ *   (segments of request b are [req_seg_begin[b], req_seg_begin[b+1])),
+ *   cta_seg_begin[C+1] (segments of CTA c are [cta_seg_begin[c],
+ *   cta_seg_begin[c+1])), seg_req, seg_cta, seg_tile_begin, seg_tile_end
+ *   [max_segments] (tile indices relative to the request), *num_units (= U),
+ *   *num_segments, *bad_index (-1 if none).
  * Returns DAO_OK, DAO_ERR_BAD_SEQLEN (outputs still valid, bad requests have
  * 0 tiles) or DAO_ERR_ARG / DAO_ERR_CAPACITY.
  */
-int dao_plan(int32_t batch, const int32_t* seq_lens, int32_t tile_tokens, int32_t num_ctas,
-             int64_t capacity_tokens, int32_t max_segments, int32_t* num_units,
-             int32_t* num_segments, int32_t* req_tile_prefix, int32_t* req_seg_begin,
-             int32_t* cta_seg_begin, int32_t* seg_req, int32_t* seg_cta,
-             int32_t* seg_tile_begin, int32_t* seg_tile_end, int32_t* bad_index) {
-  if (batch < 0 || tile_tokens <= 0 || num_ctas <= 0 || capacity_tokens < 0) return DAO_ERR_ARG;
+int dao_plan_start_cost(int32_t batch, const int32_t* seq_lens, int32_t tile_tokens, int32_t num_ctas,
+                        int64_t capacity_tokens, int32_t max_segments, int32_t* num_units,
+                        int32_t* num_segments, int32_t* req_tile_prefix, int32_t* req_seg_begin,
+                        int32_t* cta_seg_begin, int32_t* seg_req, int32_t* seg_cta,
+                        int32_t* seg_tile_begin, int32_t* seg_tile_end, int32_t* bad_index,
+                        int32_t start_cost) {
+  if (batch < 0 || tile_tokens <= 0 || num_ctas <= 0 || capacity_tokens < 0 || start_cost < 0) return DAO_ERR_ARG;
   req_tile_prefix[0] = 0;
-  for (int32_t b = 0; b < batch; ++b)
-    req_tile_prefix[b + 1] = req_tile_prefix[b] + (int32_t)tiles_of(seq_lens[b], tile_tokens, capacity_tokens);
+  for (int32_t b = 0; b < batch; ++b) {
+    const int64_t n = tiles_of(seq_lens[b], tile_tokens, capacity_tokens);
+    req_tile_prefix[b + 1] = req_tile_prefix[b] + (int32_t)(n > 0 ? n + start_cost : 0);
+  }
   const int64_t U = req_tile_prefix[batch];
   const int64_t C = num_ctas;
   *num_units = (int32_t)U;
@@ -351,17 +367,19 @@ int dao_plan(int32_t batch, const int32_t* seq_lens, int32_t tile_tokens, int32_
   int32_t prev_r = -1, prev_c = -1;
   for (int64_t u = 0; u < U; ++u) {
     while (req_tile_prefix[r + 1] <= u) ++r; /* request owning unit u */
+    const int64_t t = u - req_tile_prefix[r] - start_cost; /* its tile, or < 0 for a start unit */
+    if (t < 0) continue;
     const int32_t c = (int32_t)(((u + 1) * C - 1) / U);
     if (r != prev_r || c != prev_c) {
       if (S >= max_segments) return DAO_ERR_CAPACITY;
       seg_req[S] = r;
       seg_cta[S] = c;
-      seg_tile_begin[S] = (int32_t)(u - req_tile_prefix[r]);
+      seg_tile_begin[S] = (int32_t)t;
       ++S;
       prev_r = r;
       prev_c = c;
     }
-    seg_tile_end[S - 1] = (int32_t)(u - req_tile_prefix[r] + 1);
+    seg_tile_end[S - 1] = (int32_t)(t + 1);
   }
   *num_segments = S;
   /* req_seg_begin[b] = #segments of requests < b;  cta_seg_begin[c] = #segments of CTAs < c. */
@@ -376,6 +394,17 @@ int dao_plan(int32_t batch, const int32_t* seq_lens, int32_t tile_tokens, int32_
     cta_seg_begin[c] = count;
   }
   return *bad_index >= 0 ? DAO_ERR_BAD_SEQLEN : DAO_OK;
+}
+
+/* The plan without start units (sigma = 0): every unit is a tile. */
+int dao_plan(int32_t batch, const int32_t* seq_lens, int32_t tile_tokens, int32_t num_ctas,
+             int64_t capacity_tokens, int32_t max_segments, int32_t* num_units,
+             int32_t* num_segments, int32_t* req_tile_prefix, int32_t* req_seg_begin,
+             int32_t* cta_seg_begin, int32_t* seg_req, int32_t* seg_cta,
+             int32_t* seg_tile_begin, int32_t* seg_tile_end, int32_t* bad_index) {
+  return dao_plan_start_cost(batch, seq_lens, tile_tokens, num_ctas, capacity_tokens, max_segments, num_units,
+                             num_segments, req_tile_prefix, req_seg_begin, cta_seg_begin, seg_req, seg_cta,
+                             seg_tile_begin, seg_tile_end, bad_index, 0);
 }
 
 /*

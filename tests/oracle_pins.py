@@ -403,29 +403,34 @@ ATTENTION_PINS = [pin_golden_attention, pin_length_one, pin_constant_v, pin_unif
 # Plan pins.
 
 
-def brute_force_plan(seq_lens, T, C, capacity):
-    """The dynamic plan by scanning: for each unit, search the CTA whose range holds it."""
+def brute_force_plan(seq_lens, T, C, capacity, start_cost=0):
+    """The dynamic plan by scanning: lay out every unit (a request's start units, then its tiles),
+    and for each tile unit search the CTA whose range holds it."""
     n = [(-(-L // T) if 0 <= L <= capacity else 0) for L in seq_lens]
-    U = sum(n)
+    units = []  # (request, tile or None for a start unit)
+    for r, nr in enumerate(n):
+        if nr:
+            units += [(r, None)] * start_cost + [(r, t) for t in range(nr)]
+    U = len(units)
     starts = [c * U // C for c in range(C + 1)]
     segs = []  # [req, cta, tile_begin, tile_end]
-    u = 0
-    for r, nr in enumerate(n):
-        for t in range(nr):
-            cta = next(c for c in range(C) if starts[c] <= u < starts[c + 1])
-            if segs and segs[-1][0] == r and segs[-1][1] == cta:
-                segs[-1][3] = t + 1
-            else:
-                segs.append([r, cta, t, t + 1])
-            u += 1
+    for u, (r, t) in enumerate(units):
+        if t is None:
+            continue
+        cta = next(c for c in range(C) if starts[c] <= u < starts[c + 1])
+        if segs and segs[-1][0] == r and segs[-1][1] == cta:
+            segs[-1][3] = t + 1
+        else:
+            segs.append([r, cta, t, t + 1])
     return n, U, segs
 
 
-def check_plan_invariants(p, seq_lens, T, C, capacity):
+def check_plan_invariants(p, seq_lens, T, C, capacity, start_cost=0):
     n = [(-(-L // T) if 0 <= L <= capacity else 0) for L in seq_lens]
-    B, U, S = len(seq_lens), sum(n), p["num_segments"]
+    w = [nr + start_cost if nr else 0 for nr in n]  # units per request, start units included
+    B, U, S = len(seq_lens), sum(w), p["num_segments"]
     assert p["num_units"] == U
-    assert list(p["req_tile_prefix"]) == list(np.concatenate([[0], np.cumsum(n)]))
+    assert list(p["req_tile_prefix"]) == list(np.concatenate([[0], np.cumsum(w)]))
     assert S <= C + max(B, 1) - 1
     req, cta, tb, te = p["seg_req"], p["seg_cta"], p["seg_tile_begin"], p["seg_tile_end"]
     assert np.all(te > tb)  # no empty segment in a dynamic plan
@@ -435,16 +440,26 @@ def check_plan_invariants(p, seq_lens, T, C, capacity):
         assert np.all(req[s0:s1] == b)
         cover = [t for s in range(s0, s1) for t in range(tb[s], te[s])]
         assert cover == list(range(n[b]))
-    # each CTA's load is floor or ceil of U / C, its segments are contiguous and in unit order
+    # each CTA's load (its tiles plus the start units in its range) is floor or ceil of U / C,
+    # its segments are contiguous, in unit order, and inside its range of units
+    prefix = p["req_tile_prefix"]
+    first = [c * U // C for c in range(C + 1)]
+    start_units = np.zeros(C, np.int64)
+    for b in range(B):
+        for u in range(int(prefix[b]), int(prefix[b]) + (start_cost if n[b] else 0)):
+            start_units[next(c for c in range(C) if first[c] <= u < first[c + 1])] += 1
     loads = np.zeros(C, np.int64)
     for c in range(C):
         s0, s1 = p["cta_seg_begin"][c], p["cta_seg_begin"][c + 1]
         assert np.all(cta[s0:s1] == c)
-        loads[c] = int((te[s0:s1] - tb[s0:s1]).sum())
+        loads[c] = int((te[s0:s1] - tb[s0:s1]).sum()) + start_units[c]
+        for s in range(s0, s1):
+            u0 = int(prefix[req[s]]) + start_cost + int(tb[s])
+            assert first[c] <= u0 and u0 + int(te[s] - tb[s]) <= first[c + 1]
     assert loads.sum() == U
     if U:
         assert loads.min() >= U // C and loads.max() <= -(-U // C)
-    units = [p["req_tile_prefix"][req[s]] + tb[s] for s in range(S)]
+    units = [prefix[req[s]] + start_cost + tb[s] for s in range(S)]
     assert units == sorted(units)
 
 
@@ -460,7 +475,8 @@ def pin_golden_plans(lib=None):
     with open(os.path.join(GOLDEN, "plan_hand.json")) as f:
         g = json.load(f)
     for c in g["dynamic"]:
-        p = oracle.plan(c["seq_lens"], c["tile_tokens"], c["num_ctas"], 1 << 20, lib=lib)
+        p = oracle.plan(c["seq_lens"], c["tile_tokens"], c["num_ctas"], 1 << 20, lib=lib,
+                        start_cost=c.get("start_cost", 0))
         compare_plan(p, c)
     for c in g["static"]:
         p = oracle.static_plan(c["seq_lens"], c["tile_tokens"], c["splits"], 1 << 20, lib=lib)
@@ -494,6 +510,44 @@ def pin_plan_random(lib=None):
             _, _, segs = brute_force_plan(list(lens), T, C, 1 << 20)
             got = list(zip(p["seg_req"], p["seg_cta"], p["seg_tile_begin"], p["seg_tile_end"]))
             assert got == [tuple(s) for s in segs]
+
+
+def pin_plan_start_cost_brute_force(lib=None):
+    """Start units: every small case against the explicit unit walk, sigma = 1, 2, 3."""
+    import itertools
+    for B in range(0, 4):
+        for lens in itertools.product(range(5), repeat=B):
+            for T in (1, 2):
+                for C in range(1, 7):
+                    for sc in (1, 2, 3):
+                        p = oracle.plan(list(lens), T, C, 1 << 20, lib=lib, start_cost=sc)
+                        _, _, segs = brute_force_plan(list(lens), T, C, 1 << 20, start_cost=sc)
+                        got = list(zip(p["seg_req"], p["seg_cta"], p["seg_tile_begin"], p["seg_tile_end"]))
+                        assert got == [tuple(s) for s in segs], (lens, T, C, sc)
+                        check_plan_invariants(p, list(lens), T, C, 1 << 20, start_cost=sc)
+
+
+def pin_plan_start_cost_random(lib=None):
+    """Start units at serving sizes: invariants always, the explicit walk where it is cheap;
+    sigma = 0 through the start-cost entry point is the plain plan."""
+    rng = np.random.default_rng(23)
+    lib = lib or oracle._load()
+    for _ in range(40):
+        B = int(rng.integers(1, 300))
+        C = int(rng.choice([1, 7, 37, 148, 296, 1000]))
+        T = int(rng.choice([16, 64, 128]))
+        sc = int(rng.choice([1, 2, 5]))
+        lens = rng.integers(0, 5000, size=B)
+        lens[rng.random(B) < 0.2] = 0
+        p = oracle.plan(lens, T, C, 1 << 20, lib=lib, start_cost=sc)
+        check_plan_invariants(p, list(lens), T, C, 1 << 20, start_cost=sc)
+        if B * C < 20000:
+            _, _, segs = brute_force_plan(list(lens), T, C, 1 << 20, start_cost=sc)
+            got = list(zip(p["seg_req"], p["seg_cta"], p["seg_tile_begin"], p["seg_tile_end"]))
+            assert got == [tuple(s) for s in segs]
+        plain = oracle.plan(lens, T, C, 1 << 20, lib=lib)
+        zero = oracle._run_plan(lib.dao_plan_start_cost, lens, T, C, 1 << 20, C + B - 1, C, 0)
+        compare_plan(zero, plain)
 
 
 def pin_plan_bad_lengths(lib=None):
@@ -546,5 +600,6 @@ def pin_static_empty_splits(lib=None):
     assert p["num_segments"] == 32 and empty == 19
 
 
-PLAN_PINS = [pin_golden_plans, pin_plan_brute_force, pin_plan_random, pin_plan_bad_lengths, pin_static_brute_force,
+PLAN_PINS = [pin_golden_plans, pin_plan_brute_force, pin_plan_random, pin_plan_start_cost_brute_force,
+             pin_plan_start_cost_random, pin_plan_bad_lengths, pin_static_brute_force,
              pin_static_empty_splits]

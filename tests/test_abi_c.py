@@ -30,7 +30,7 @@ int main(void) {
   CHECK(da_plan_desc_init(&p, DA_PLAN_DYNAMIC, 64, 37, &d) == DA_OK);
   CHECK(d.kind == DA_PLAN_DYNAMIC && d.batch == 32 && d.tile_tokens == 64 && d.num_ctas == 37);
   CHECK(d.splits == 0 && d.max_segments == 37 + 32 - 1 && d.num_kv_heads == 8 && d.merge_in_decode == 0);
-  CHECK(d.out_format == DA_OUT_BF16);
+  CHECK(d.out_format == DA_OUT_BF16 && d.start_cost == 2);
   CHECK(da_plan_workspace_size(&p, 64, 37, &ws, &po, &pl) == DA_OK);
   CHECK(po == (size_t)d.max_segments * 64 * 128 * 4);
   CHECK(da_workspace_size(&p, &d, &ws, &po, &pl) == DA_OK);
@@ -41,6 +41,15 @@ int main(void) {
 
   CHECK(da_plan_desc_init(&p, DA_PLAN_STATIC, 32, 3, &s) == DA_OK);
   CHECK(s.kind == DA_PLAN_STATIC && s.num_ctas == 96 && s.splits == 3 && s.max_segments == 96);
+  CHECK(s.start_cost == 0);
+  s.start_cost = 1;  /* start units belong to dynamic plans */
+  CHECK(da_workspace_size(&p, &s, &ws, &po, &pl) == DA_ERR_INVALID_ARG);
+  s.start_cost = 0;
+  d.start_cost = -1;
+  CHECK(da_workspace_size(&p, &d, &ws, &po, &pl) == DA_ERR_INVALID_ARG);
+  d.start_cost = 0;  /* the tiles-only plan: same sizes */
+  CHECK(da_workspace_size(&p, &d, &ws, &po, &pl) == DA_OK);
+  d.start_cost = 2;
 
   /* fp32 output: every request goes through the combine, which cannot run inside the decode */
   d.out_format = DA_OUT_F32;

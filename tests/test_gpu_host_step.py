@@ -161,7 +161,7 @@ def test_host_inputs_plan_matches_the_oracle_plan(kind, oracle_lib):
         out_h, lse_h, st = host_step(w, kind=kind, seq_lens=cur, state=st)
         d = st["desc"]
         got = da.read_plan(d, st["bufs"].ws)
-        want = (oracle.plan(cur, 64, d.num_ctas, cap) if kind == da.PLAN_DYNAMIC
+        want = (oracle.plan(cur, 64, d.num_ctas, cap, start_cost=d.start_cost) if kind == da.PLAN_DYNAMIC
                 else oracle.static_plan(cur, 64, d.splits, cap))
         assert_plan_equal(got, want)
         assert torch.equal(st["dw"].seq_lens.cpu(), torch.from_numpy(cur))

@@ -75,7 +75,8 @@ def test_decode_trace_256_steps(da_lib, oracle_lib):
             dt.advance()
         da.decode_step(prob, desc, dt.q, dt.k_cache, dt.v_cache, dt.block_table, dt.seq_lens, bufs)
         torch.cuda.synchronize()
-        assert_plan_equal(da.read_plan(desc, bufs.ws), oracle.plan(tr.seq_lens, 64, desc.num_ctas, cap))
+        assert_plan_equal(da.read_plan(desc, bufs.ws), oracle.plan(tr.seq_lens, 64, desc.num_ctas, cap,
+                                                                       start_cost=desc.start_cost))
         if t in (0, 1, 127, 255):
             check_against_oracle(tr.workload(), bufs.out, bufs.lse)
         if t in (0, tr.steps - 1):  # the trace's batch at both ends, over an FP8 copy of its cache
@@ -146,7 +147,8 @@ def test_fused_plan_append_matches_separate_launches(da_lib, oracle_lib):
                        planned=t > 0)
         torch.cuda.synchronize()
         assert torch.equal(b1.ws, b2.ws)
-        assert_plan_equal(da.read_plan(desc, b2.ws), oracle.plan(host.seq_lens, 64, desc.num_ctas, cap))
+        assert_plan_equal(da.read_plan(desc, b2.ws), oracle.plan(host.seq_lens, 64, desc.num_ctas, cap,
+                                                                   start_cost=desc.start_cost))
         assert same(b1.out, b2.out) and torch.equal(b1.lse, b2.lse)
         assert same(sep.k_cache, fus.k_cache) and same(sep.v_cache, fus.v_cache)
     check_against_oracle(host.workload(), b2.out, b2.lse)

@@ -43,6 +43,9 @@ MUTANTS = [
     ("static chunk floor", "const int64_t chunk = (max_tiles + splits - 1) / splits;",
      "const int64_t chunk = max_tiles / splits + (max_tiles < splits);"),
     ("bad length kept", "if (len < 0 || (int64_t)len > capacity) return 0;", "if (len < 0) return 0;"),
+    ("start units for empty requests", "(int32_t)(n > 0 ? n + start_cost : 0)", "(int32_t)(n + start_cost)"),
+    ("start units after the tiles", "const int64_t t = u - req_tile_prefix[r] - start_cost;",
+     "const int64_t t = u - req_tile_prefix[r];"),
 ]
 
 

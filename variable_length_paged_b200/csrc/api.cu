@@ -21,6 +21,10 @@ constexpr uint64_t kWaitLimitNs = 2000000000ull;  // 2 s: far beyond any legitim
 
 constexpr int kDefaultTile = 64;
 constexpr int kCtasPerSm = 2;  // decode kernel residency (shared memory sized for two)
+// Start units of a dynamic plan: the fixed cost of starting a request (query load, merge and
+// write of its result, about 2 us of one CTA's time on B200) in 64-token tiles of bf16 d 128.
+constexpr int32_t kDefaultStartCost = 2;
+constexpr int32_t kMaxStartCost = 1 << 16;
 constexpr int kMaxRows = 16;  // query heads x queries per request packed on one MMA tile
 
 int q_len_of(const da_problem* p) { return p->q_len > 1 ? p->q_len : 1; }
@@ -54,6 +58,8 @@ int check_desc(const da_problem* p, const da_plan_desc* d) {
     return DA_ERR_INVALID_ARG;
   if (d->out_format != DA_OUT_BF16 && d->out_format != DA_OUT_F32) return DA_ERR_INVALID_ARG;
   if (d->out_format == DA_OUT_F32 && d->merge_in_decode) return DA_ERR_INVALID_ARG;  // the combine writes fp32 out
+  if (d->start_cost < 0 || d->start_cost > kMaxStartCost) return DA_ERR_INVALID_ARG;
+  if (d->start_cost != 0 && d->kind != DA_PLAN_DYNAMIC) return DA_ERR_INVALID_ARG;
   if (d->kind == DA_PLAN_DYNAMIC) {
     if (d->splits != 0 || (int64_t)d->max_segments != (int64_t)d->num_ctas + (p->batch > 0 ? p->batch : 1) - 1)
       return DA_ERR_INVALID_ARG;
@@ -63,12 +69,11 @@ int check_desc(const da_problem* p, const da_plan_desc* d) {
   } else {
     return DA_ERR_INVALID_ARG;
   }
-  // every tile index and unit count stays inside int32
+  // every tile index and unit count (start units included) stays inside int32
   const int64_t cap = (int64_t)p->max_pages_per_req * p->page_size;
-  if ((int64_t)p->batch * ((cap + d->tile_tokens - 1) / d->tile_tokens) >= (int64_t)INT_MAX) return DA_ERR_UNSUPPORTED;
-  if ((int64_t)d->num_ctas * ((int64_t)p->batch * ((cap + d->tile_tokens - 1) / d->tile_tokens) + 1) >=
-      ((int64_t)1 << 62))
-    return DA_ERR_UNSUPPORTED;
+  const int64_t units = (int64_t)p->batch * ((cap + d->tile_tokens - 1) / d->tile_tokens + d->start_cost);
+  if (units >= (int64_t)INT_MAX) return DA_ERR_UNSUPPORTED;
+  if ((int64_t)d->num_ctas * (units + 1) >= ((int64_t)1 << 62)) return DA_ERR_UNSUPPORTED;
   return DA_OK;
 }
 
@@ -164,6 +169,7 @@ DA_API int da_plan_desc_init(const da_problem* prob, int32_t kind, int32_t tile_
   d.num_kv_heads = prob->num_kv_heads;
   d.merge_in_decode = 0;
   d.out_format = DA_OUT_BF16;
+  d.start_cost = kind == DA_PLAN_DYNAMIC ? kDefaultStartCost : 0;
   if (kind == DA_PLAN_DYNAMIC) {
     d.num_ctas = w;
     d.splits = 0;
@@ -238,6 +244,7 @@ static int plan_prepare(const da_problem* prob, const da_plan_desc* desc, const 
   p->num_ctas = desc->num_ctas;
   p->num_kv_heads = prob->num_kv_heads;
   p->capacity_tokens = (int64_t)prob->max_pages_per_req * prob->page_size;
+  p->start_cost = kind == DA_PLAN_DYNAMIC ? desc->start_cost : 0;
   return DA_OK;
 }
 

@@ -55,6 +55,7 @@ struct PlanParams {
   int32_t* ws;
   int32_t batch, tile_tokens, width, max_segments, num_ctas, num_kv_heads;
   int64_t capacity_tokens;
+  int32_t start_cost;  // dynamic plan: start units charged to every non-empty request
 };
 
 struct DecodeParams {

@@ -60,13 +60,16 @@ __device__ int request_tiles(const PlanParams& p, int b, int* s_bad) {
 // from global memory (written by this block and visible after __syncthreads).
 constexpr int kSmemBatch = 4096;
 
-// Phase shared by both planners: req_tile_prefix and U (and the largest n_b).
+// Phase shared by both planners: req_tile_prefix and U (and the largest n_b).  Each
+// non-empty request counts start_units more units than its tiles (the dynamic plan's start
+// cost; 0 for the static plan), so the prefix and U are in units.
 __device__ void tile_prefix(const PlanParams& p, int32_t* rtp, int32_t* s_rtp, int* warp_buf, int* s_bad, int* U,
-                            int* max_tiles) {
+                            int* max_tiles, int start_units) {
   int carry = 0, mx = 0;
   for (int base = 0; base < p.batch; base += kPlanThreads) {
     const int b = base + threadIdx.x;
-    const int n = b < p.batch ? request_tiles(p, b, s_bad) : 0;
+    const int tiles = b < p.batch ? request_tiles(p, b, s_bad) : 0;
+    const int n = tiles > 0 ? tiles + start_units : 0;
     int total;
     const int excl = block_exclusive_scan(n, &total, warp_buf);
     if (b < p.batch) {
@@ -155,20 +158,25 @@ __device__ void plan_dynamic_body(const PlanParams& p) {
   const int32_t* rsb_r = small ? s_rsb : rsb;
   const int64_t C = p.num_ctas;
 
+  // Units: every non-empty request's start units (a fixed cost charged to the CTA that
+  // starts it), then its tiles; U counts both.  Request b's tiles are units [first_tile(b),
+  // rtp[b + 1]).
+  const int sc = p.start_cost;
   int U;
-  tile_prefix(p, rtp, small ? s_rtp : nullptr, warp_buf, &s_bad, &U, nullptr);
+  tile_prefix(p, rtp, small ? s_rtp : nullptr, warp_buf, &s_bad, &U, nullptr, sc);
   const Split sp(U, C);
+  auto first_tile = [&](int b) -> int { return rtp_r[b] + (rtp_r[b + 1] > rtp_r[b] ? sc : 0); };
 
-  // Segments per request.  With U >= C every CTA owns at least one tile, so a
-  // request spanning CTAs [cf, cl] has cl - cf + 1 segments.  With U < C each
-  // non-empty CTA owns exactly one tile, so every tile is its own segment.
+  // Segments per request.  With U >= C every CTA owns at least one unit, so a
+  // request whose tiles span CTAs [cf, cl] has cl - cf + 1 segments.  With U < C each
+  // CTA owns at most one unit, so every tile is its own segment.
   const bool sparse = (int64_t)U < C;
   int carry = 0;
   for (int base = 0; base < p.batch; base += kPlanThreads) {
     const int b = base + threadIdx.x;
     int ns = 0;
     if (b < p.batch) {
-      const int p0 = rtp_r[b], n = rtp_r[b + 1] - p0;
+      const int p0 = first_tile(b), n = rtp_r[b + 1] - p0;
       if (n > 0) ns = sparse ? n : sp.owner(p0 + n - 1) - sp.owner(p0) + 1;
     }
     int total;
@@ -190,7 +198,7 @@ __device__ void plan_dynamic_body(const PlanParams& p) {
   for (int s = threadIdx.x; s < S; s += kPlanThreads) {
     const int b = last_not_above(rsb_r, p.batch, s);  // rsb[b] <= s < rsb[b+1]
     const int j = s - rsb_r[b];
-    const int p0 = rtp_r[b], n = rtp_r[b + 1] - p0;
+    const int p0 = first_tile(b), n = rtp_r[b + 1] - p0;
     if (sparse) {
       segs[s] = make_int4(b, sp.owner((int64_t)p0 + j), j, j + 1);
     } else {
@@ -200,18 +208,19 @@ __device__ void plan_dynamic_body(const PlanParams& p) {
       segs[s] = make_int4(b, c, (int)(lo - p0), (int)(hi - p0));
     }
   }
-  // One thread per CTA: its first segment.
+  // One thread per CTA: its first segment.  Request r holds CTA c's first unit u0; the
+  // segments before CTA c's are those of the requests before r and, of r's, those of the CTAs
+  // before c (dense: one per CTA from the owner of r's first tile on; sparse: one per tile
+  // before u0).  A CTA whose units are all start units gets an empty range.
   for (int c = threadIdx.x; c <= p.num_ctas; c += kPlanThreads) {
     int first;
-    if (sparse) {
-      first = (int)sp.first(c);  // every tile is a segment
-    } else if (c == p.num_ctas) {
+    const int64_t u0 = c < p.num_ctas ? sp.first(c) : (int64_t)U;
+    if (u0 >= U) {  // the end (also every CTA of an empty batch)
       first = S;
     } else {
-      // the request holding CTA c's first tile opens CTA c
-      const int64_t u0 = sp.first(c);
       const int r = last_not_above(rtp_r, p.batch, u0);
-      first = rsb_r[r] + (c - sp.owner(rtp_r[r]));
+      const int p0 = first_tile(r);
+      first = rsb_r[r] + (sparse ? (int)max((int64_t)0, u0 - p0) : max(0, c - sp.owner(p0)));
     }
     csb[c] = first;
   }
@@ -258,7 +267,7 @@ __device__ void plan_static_body(const PlanParams& p) {
   const int S = p.width;
 
   int U, max_tiles;
-  tile_prefix(p, rtp, small ? s_rtp : nullptr, warp_buf, &s_bad, &U, &max_tiles);
+  tile_prefix(p, rtp, small ? s_rtp : nullptr, warp_buf, &s_bad, &U, &max_tiles, 0);
   const int chunk = (max_tiles + S - 1) / S;
   const int total = p.batch * S;
   for (int i = threadIdx.x; i < total; i += kPlanThreads) {

@@ -41,7 +41,7 @@ class DaPlanDesc(ctypes.Structure):
     _fields_ = [("kind", ctypes.c_int32), ("batch", ctypes.c_int32), ("tile_tokens", ctypes.c_int32),
                 ("num_ctas", ctypes.c_int32), ("splits", ctypes.c_int32), ("max_segments", ctypes.c_int32),
                 ("num_kv_heads", ctypes.c_int32), ("merge_in_decode", ctypes.c_int32),
-                ("out_format", ctypes.c_int32)]
+                ("out_format", ctypes.c_int32), ("start_cost", ctypes.c_int32)]
 
 
 class DaError(RuntimeError):
@@ -148,13 +148,17 @@ def _stream(stream) -> int | None:
 # ---- the C calls -------------------------------------------------------------------------------
 
 def da_plan_desc_init(prob: DaProblem, kind: int, tile_tokens: int = 0, width: int = 0,
-                      merge_in_decode: bool = False, out_f32: bool = False) -> DaPlanDesc:
-    """The C call, then the descriptor's two switches (in-decode merge, fp32 output) set as asked."""
+                      merge_in_decode: bool = False, out_f32: bool = False,
+                      start_cost: int | None = None) -> DaPlanDesc:
+    """The C call, then the descriptor's switches set as asked: in-decode merge, fp32 output and
+    the dynamic plan's start cost (None keeps the C default)."""
     d = DaPlanDesc()
     _check("da_plan_desc_init", lib().da_plan_desc_init(ctypes.byref(prob), int(kind), int(tile_tokens), int(width),
                                                          ctypes.byref(d)))
     d.merge_in_decode = 1 if merge_in_decode else 0
     d.out_format = OUT_F32 if out_f32 else OUT_BF16
+    if start_cost is not None:
+        d.start_cost = int(start_cost)
     return d
 
 
