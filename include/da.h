@@ -146,7 +146,11 @@ typedef struct da_plan_desc {
   int32_t merge_in_decode; /* 0 (default): split requests are merged by da_combine's kernel;
                               1: by the decode kernel's last CTA for each of them (no extra launch;
                               faster for batches of many long requests, slower when one request
-                              is split over many CTAs) */
+                              is split over many CTAs).  The last CTA is found by per-request
+                              counts in the workspace that only the plan resets, so with 1 every
+                              decode launch needs its own plan launch before it (two decodes
+                              from one plan leave split requests unmerged); with 0 a plan may
+                              serve any number of decode launches */
   int32_t out_format;      /* DA_OUT_BF16 (default) or DA_OUT_F32: `out` holds fp32 values, for a
                               caller that merges this step's result with others (one slice of a
                               request's cache per GPU) and wants no bf16 rounding before that
