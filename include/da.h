@@ -150,7 +150,7 @@ typedef struct da_plan_desc {
                               counts in the workspace that only the plan resets, so with 1 every
                               decode launch needs its own plan launch before it (two decodes
                               from one plan leave split requests unmerged); with 0 a plan may
-                              serve any number of decode launches */
+                              serve several decode launches over the same seq_lens */
   int32_t out_format;      /* DA_OUT_BF16 (default) or DA_OUT_F32: `out` holds fp32 values, for a
                               caller that merges this step's result with others (one slice of a
                               request's cache per GPU) and wants no bf16 rounding before that
