@@ -70,6 +70,8 @@ def _bind(path: str):
     lib.dao_plan.argtypes = plan_args
     lib.dao_plan_start_cost.restype = ctypes.c_int
     lib.dao_plan_start_cost.argtypes = plan_args + [ctypes.c_int32]
+    lib.dao_plan_weighted.restype = ctypes.c_int
+    lib.dao_plan_weighted.argtypes = plan_args + [ctypes.c_int32, ctypes.POINTER(ctypes.c_int32)]
     lib.dao_static_plan.restype = ctypes.c_int
     lib.dao_static_plan.argtypes = plan_args
     lib.dao_num_threads.restype = ctypes.c_int
@@ -282,12 +284,19 @@ def _run_plan(fn, seq_lens, tile_tokens, width, capacity_tokens, max_segments, n
     return res
 
 
-def plan(seq_lens, tile_tokens: int, num_ctas: int, capacity_tokens: int, lib=None, start_cost: int = 0):
-    """Dynamic plan (dict of int32 arrays; see ``dao_plan_start_cost`` in dao.c).
+def plan(seq_lens, tile_tokens: int, num_ctas: int, capacity_tokens: int, lib=None, start_cost: int = 0,
+         weights=None):
+    """Dynamic plan (dict of int32 arrays; see ``dao_plan_weighted`` in dao.c).
 
-    start_cost: start units charged to every non-empty request (0: every unit is a tile)."""
+    start_cost: start units charged to every non-empty request (0: every unit is a tile).
+    weights: per-CTA weights in [1, 65536] (None: the even split)."""
     B = len(seq_lens)
     lib = lib or _load()
+    if weights is not None:
+        w = np.ascontiguousarray(weights, dtype=np.int32)
+        assert w.shape == (num_ctas,)
+        return _run_plan(lib.dao_plan_weighted, seq_lens, tile_tokens, num_ctas, capacity_tokens,
+                         num_ctas + max(B, 1) - 1, num_ctas, int(start_cost), _ptr(w, ctypes.c_int32))
     if start_cost == 0:
         return _run_plan(lib.dao_plan, seq_lens, tile_tokens, num_ctas, capacity_tokens, num_ctas + max(B, 1) - 1,
                          num_ctas)

@@ -344,14 +344,26 @@ static int32_t first_bad_length(int32_t batch, const int32_t* seq_lens, int64_t 
  *   *num_segments, *bad_index (-1 if none).
  * Returns DAO_OK, DAO_ERR_BAD_SEQLEN (outputs still valid, bad requests have
  * 0 tiles) or DAO_ERR_ARG / DAO_ERR_CAPACITY.
+ *
+ * Weighted ranges (dao_plan_weighted, cta_weights != NULL): CTA c's range is
+ *   [first(c), first(c+1)),  first(c) = c + floor((U - C) * W_c / W)  when U >= C,
+ * W_c = sum_{k<c} w_k, W = sum_k w_k: one unit each, and the other U - C units
+ * in proportion to the weights (each w_k in [1, 65536]), so a CTA that will run on a
+ * slower SM can be given less.  Equal weights give floor(c*U/C), the even split
+ * above.  With U < C the weights are not used (every CTA holds at most one unit).
+ * The weighting is this implementation's addition (the article spreads tiles
+ * evenly over CTAs); it changes only who computes which tiles.
  */
-int dao_plan_start_cost(int32_t batch, const int32_t* seq_lens, int32_t tile_tokens, int32_t num_ctas,
-                        int64_t capacity_tokens, int32_t max_segments, int32_t* num_units,
-                        int32_t* num_segments, int32_t* req_tile_prefix, int32_t* req_seg_begin,
-                        int32_t* cta_seg_begin, int32_t* seg_req, int32_t* seg_cta,
-                        int32_t* seg_tile_begin, int32_t* seg_tile_end, int32_t* bad_index,
-                        int32_t start_cost) {
+int dao_plan_weighted(int32_t batch, const int32_t* seq_lens, int32_t tile_tokens, int32_t num_ctas,
+                      int64_t capacity_tokens, int32_t max_segments, int32_t* num_units,
+                      int32_t* num_segments, int32_t* req_tile_prefix, int32_t* req_seg_begin,
+                      int32_t* cta_seg_begin, int32_t* seg_req, int32_t* seg_cta,
+                      int32_t* seg_tile_begin, int32_t* seg_tile_end, int32_t* bad_index,
+                      int32_t start_cost, const int32_t* cta_weights) {
   if (batch < 0 || tile_tokens <= 0 || num_ctas <= 0 || capacity_tokens < 0 || start_cost < 0) return DAO_ERR_ARG;
+  if (cta_weights)
+    for (int32_t c = 0; c < num_ctas; ++c)
+      if (cta_weights[c] < 1 || cta_weights[c] > 65536) return DAO_ERR_ARG;
   req_tile_prefix[0] = 0;
   for (int32_t b = 0; b < batch; ++b) {
     const int64_t n = tiles_of(seq_lens[b], tile_tokens, capacity_tokens);
@@ -362,16 +374,37 @@ int dao_plan_start_cost(int32_t batch, const int32_t* seq_lens, int32_t tile_tok
   *num_units = (int32_t)U;
   *bad_index = first_bad_length(batch, seq_lens, capacity_tokens);
 
+  /* weighted ranges: first[c] for c = 0..C, walked with the units */
+  int64_t* first = NULL;
+  const int weighted = cta_weights != NULL && U >= C;
+  if (weighted) {
+    first = (int64_t*)malloc((size_t)(C + 1) * sizeof(int64_t));
+    if (!first) return DAO_ERR_ARG;
+    int64_t W = 0;
+    for (int64_t c = 0; c < C; ++c) W += cta_weights[c];
+    int64_t Wc = 0;
+    for (int64_t c = 0; c <= C; ++c) {
+      first[c] = c + (U - C) * Wc / W;
+      if (c < C) Wc += cta_weights[c];
+    }
+  }
+
   int32_t S = 0;
   int32_t r = 0;
+  int32_t cw = 0; /* weighted: the CTA whose range holds unit u */
   int32_t prev_r = -1, prev_c = -1;
   for (int64_t u = 0; u < U; ++u) {
     while (req_tile_prefix[r + 1] <= u) ++r; /* request owning unit u */
+    if (weighted)
+      while (first[cw + 1] <= u) ++cw;
     const int64_t t = u - req_tile_prefix[r] - start_cost; /* its tile, or < 0 for a start unit */
     if (t < 0) continue;
-    const int32_t c = (int32_t)(((u + 1) * C - 1) / U);
+    const int32_t c = weighted ? cw : (int32_t)(((u + 1) * C - 1) / U);
     if (r != prev_r || c != prev_c) {
-      if (S >= max_segments) return DAO_ERR_CAPACITY;
+      if (S >= max_segments) {
+        free(first);
+        return DAO_ERR_CAPACITY;
+      }
       seg_req[S] = r;
       seg_cta[S] = c;
       seg_tile_begin[S] = (int32_t)t;
@@ -381,6 +414,7 @@ int dao_plan_start_cost(int32_t batch, const int32_t* seq_lens, int32_t tile_tok
     }
     seg_tile_end[S - 1] = (int32_t)(t + 1);
   }
+  free(first);
   *num_segments = S;
   /* req_seg_begin[b] = #segments of requests < b;  cta_seg_begin[c] = #segments of CTAs < c. */
   for (int32_t b = 0; b <= batch; ++b) {
@@ -394,6 +428,18 @@ int dao_plan_start_cost(int32_t batch, const int32_t* seq_lens, int32_t tile_tok
     cta_seg_begin[c] = count;
   }
   return *bad_index >= 0 ? DAO_ERR_BAD_SEQLEN : DAO_OK;
+}
+
+/* The even split (no weights). */
+int dao_plan_start_cost(int32_t batch, const int32_t* seq_lens, int32_t tile_tokens, int32_t num_ctas,
+                        int64_t capacity_tokens, int32_t max_segments, int32_t* num_units,
+                        int32_t* num_segments, int32_t* req_tile_prefix, int32_t* req_seg_begin,
+                        int32_t* cta_seg_begin, int32_t* seg_req, int32_t* seg_cta,
+                        int32_t* seg_tile_begin, int32_t* seg_tile_end, int32_t* bad_index,
+                        int32_t start_cost) {
+  return dao_plan_weighted(batch, seq_lens, tile_tokens, num_ctas, capacity_tokens, max_segments, num_units,
+                           num_segments, req_tile_prefix, req_seg_begin, cta_seg_begin, seg_req, seg_cta,
+                           seg_tile_begin, seg_tile_end, bad_index, start_cost, NULL);
 }
 
 /* The plan without start units (sigma = 0): every unit is a tile. */

@@ -403,7 +403,17 @@ ATTENTION_PINS = [pin_golden_attention, pin_length_one, pin_constant_v, pin_unif
 # Plan pins.
 
 
-def brute_force_plan(seq_lens, T, C, capacity, start_cost=0):
+def cta_starts(U, C, weights=None):
+    """First unit of each CTA's range (and U at the end): the even split floor(c*U/C), or with
+    weights (and U >= C) one unit per CTA plus the other U - C units dealt out in proportion."""
+    if weights is None or U < C:
+        return [c * U // C for c in range(C + 1)]
+    W = sum(weights)
+    acc = [sum(weights[:c]) for c in range(C + 1)]
+    return [c + (U - C) * acc[c] // W for c in range(C + 1)]
+
+
+def brute_force_plan(seq_lens, T, C, capacity, start_cost=0, weights=None):
     """The dynamic plan by scanning: lay out every unit (a request's start units, then its tiles),
     and for each tile unit search the CTA whose range holds it."""
     n = [(-(-L // T) if 0 <= L <= capacity else 0) for L in seq_lens]
@@ -412,7 +422,7 @@ def brute_force_plan(seq_lens, T, C, capacity, start_cost=0):
         if nr:
             units += [(r, None)] * start_cost + [(r, t) for t in range(nr)]
     U = len(units)
-    starts = [c * U // C for c in range(C + 1)]
+    starts = cta_starts(U, C, weights)
     segs = []  # [req, cta, tile_begin, tile_end]
     for u, (r, t) in enumerate(units):
         if t is None:
@@ -425,7 +435,7 @@ def brute_force_plan(seq_lens, T, C, capacity, start_cost=0):
     return n, U, segs
 
 
-def check_plan_invariants(p, seq_lens, T, C, capacity, start_cost=0):
+def check_plan_invariants(p, seq_lens, T, C, capacity, start_cost=0, weights=None):
     n = [(-(-L // T) if 0 <= L <= capacity else 0) for L in seq_lens]
     w = [nr + start_cost if nr else 0 for nr in n]  # units per request, start units included
     B, U, S = len(seq_lens), sum(w), p["num_segments"]
@@ -443,7 +453,7 @@ def check_plan_invariants(p, seq_lens, T, C, capacity, start_cost=0):
     # each CTA's load (its tiles plus the start units in its range) is floor or ceil of U / C,
     # its segments are contiguous, in unit order, and inside its range of units
     prefix = p["req_tile_prefix"]
-    first = [c * U // C for c in range(C + 1)]
+    first = cta_starts(U, C, weights)
     start_units = np.zeros(C, np.int64)
     for b in range(B):
         for u in range(int(prefix[b]), int(prefix[b]) + (start_cost if n[b] else 0)):
@@ -457,8 +467,12 @@ def check_plan_invariants(p, seq_lens, T, C, capacity, start_cost=0):
             u0 = int(prefix[req[s]]) + start_cost + int(tb[s])
             assert first[c] <= u0 and u0 + int(te[s] - tb[s]) <= first[c + 1]
     assert loads.sum() == U
-    if U:
+    if U and (weights is None or U < C):
         assert loads.min() >= U // C and loads.max() <= -(-U // C)
+    elif U:
+        # every CTA holds one unit plus, within one unit, its weight's share of the other U - C
+        share = (U - C) * np.asarray(weights, np.float64) / float(sum(weights))
+        assert np.all(loads >= 1) and np.all(np.abs(loads - 1 - share) < 1.0 + 1e-9)
     units = [prefix[req[s]] + start_cost + tb[s] for s in range(S)]
     assert units == sorted(units)
 
@@ -476,7 +490,7 @@ def pin_golden_plans(lib=None):
         g = json.load(f)
     for c in g["dynamic"]:
         p = oracle.plan(c["seq_lens"], c["tile_tokens"], c["num_ctas"], 1 << 20, lib=lib,
-                        start_cost=c.get("start_cost", 0))
+                        start_cost=c.get("start_cost", 0), weights=c.get("weights"))
         compare_plan(p, c)
     for c in g["static"]:
         p = oracle.static_plan(c["seq_lens"], c["tile_tokens"], c["splits"], 1 << 20, lib=lib)
@@ -550,6 +564,48 @@ def pin_plan_start_cost_random(lib=None):
         compare_plan(zero, plain)
 
 
+def pin_plan_weighted_brute_force(lib=None):
+    """Weighted ranges: every small case against the explicit unit walk, with weights from
+    equal to skewed by 65536 : 1, sigma = 0 and 2."""
+    import itertools
+    rng = np.random.default_rng(27)
+    for B in range(0, 4):
+        for lens in itertools.product(range(5), repeat=B):
+            for T in (1, 2):
+                for C in range(1, 6):
+                    for wv in ([1] * C, list(rng.integers(1, 10, size=C)), [65536] + [1] * (C - 1),
+                               [1] * (C - 1) + [65536]):
+                        for sc in (0, 2):
+                            p = oracle.plan(list(lens), T, C, 1 << 20, lib=lib, start_cost=sc, weights=wv)
+                            _, _, segs = brute_force_plan(list(lens), T, C, 1 << 20, start_cost=sc, weights=wv)
+                            got = list(zip(p["seg_req"], p["seg_cta"], p["seg_tile_begin"], p["seg_tile_end"]))
+                            assert got == [tuple(s) for s in segs], (lens, T, C, wv, sc)
+                            check_plan_invariants(p, list(lens), T, C, 1 << 20, start_cost=sc, weights=wv)
+
+
+def pin_plan_weighted_random(lib=None):
+    """Weighted ranges at serving sizes: invariants (each CTA within one unit of its weight's
+    share), the explicit walk where cheap, and equal weights give the even split exactly."""
+    rng = np.random.default_rng(29)
+    lib = lib or oracle._load()
+    for _ in range(30):
+        B = int(rng.integers(1, 300))
+        C = int(rng.choice([1, 7, 37, 148, 296, 1000]))
+        T = int(rng.choice([16, 64, 128]))
+        sc = int(rng.choice([0, 2]))
+        lens = rng.integers(0, 5000, size=B)
+        lens[rng.random(B) < 0.2] = 0
+        wv = rng.integers(1, 65537, size=C) if rng.random() < 0.5 else rng.integers(900, 1200, size=C)
+        p = oracle.plan(lens, T, C, 1 << 20, lib=lib, start_cost=sc, weights=wv)
+        check_plan_invariants(p, list(lens), T, C, 1 << 20, start_cost=sc, weights=list(wv))
+        if B * C < 20000:
+            _, _, segs = brute_force_plan(list(lens), T, C, 1 << 20, start_cost=sc, weights=list(wv))
+            got = list(zip(p["seg_req"], p["seg_cta"], p["seg_tile_begin"], p["seg_tile_end"]))
+            assert got == [tuple(s) for s in segs]
+        even = oracle.plan(lens, T, C, 1 << 20, lib=lib, start_cost=sc, weights=np.full(C, int(rng.integers(1, 65537))))
+        compare_plan(even, oracle.plan(lens, T, C, 1 << 20, lib=lib, start_cost=sc))
+
+
 def pin_plan_bad_lengths(lib=None):
     p = oracle.plan([5, -3, 7, 99, 2], 2, 3, 10, lib=lib)
     assert p["status"] == oracle.ERR_BAD_SEQLEN and p["bad_index"] == 1
@@ -601,5 +657,5 @@ def pin_static_empty_splits(lib=None):
 
 
 PLAN_PINS = [pin_golden_plans, pin_plan_brute_force, pin_plan_random, pin_plan_start_cost_brute_force,
-             pin_plan_start_cost_random, pin_plan_bad_lengths, pin_static_brute_force,
-             pin_static_empty_splits]
+             pin_plan_start_cost_random, pin_plan_weighted_brute_force, pin_plan_weighted_random,
+             pin_plan_bad_lengths, pin_static_brute_force, pin_static_empty_splits]

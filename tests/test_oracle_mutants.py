@@ -46,6 +46,8 @@ MUTANTS = [
     ("start units for empty requests", "(int32_t)(n > 0 ? n + start_cost : 0)", "(int32_t)(n + start_cost)"),
     ("start units after the tiles", "const int64_t t = u - req_tile_prefix[r] - start_cost;",
      "const int64_t t = u - req_tile_prefix[r];"),
+    ("weighted ranges over all units", "first[c] = c + (U - C) * Wc / W;", "first[c] = c + U * Wc / W;"),
+    ("weighted owner at a range's first unit", "while (first[cw + 1] <= u) ++cw;", "while (first[cw + 1] < u) ++cw;"),
 ]
 
 
