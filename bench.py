@@ -43,6 +43,15 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 if ROOT not in sys.path:
     sys.path.insert(0, ROOT)
 
+BALANCE_NOTE = ("measured before the timed steps: 2 rounds of 9 steps with block times, per-block medians "
+                "-> da_balance_from_times -> da_balance_set")
+
+
+def balance_wanted(args) -> bool:
+    """Whether the dynamic plan runs with a measured balance table (see --balance)."""
+    return args.balance == "measure" or (args.balance == "auto" and args.kv == "bf16")
+
+
 METRIC = "µs/decode step and KV-read HBM GB/s (% of B200 peak) vs static split-k"
 FALLBACK_HBM_GBS = 6650.0
 DATASHEET_HBM_GBS = 8000.0
@@ -70,6 +79,11 @@ def parse_args():
                     help="dynamic plan: merge split requests in the decode kernel instead of a combine launch")
     ap.add_argument("--start-cost", type=int, default=None,
                     help="dynamic plan: units charged to the CTA that starts a request (default: the library's)")
+    ap.add_argument("--balance", choices=["auto", "none", "measure"], default="auto",
+                    help="dynamic plan: measure a balance table (per-CTA weights and block placement from "
+                         "block times, untimed, before the timed steps) or keep the even split; auto = measure "
+                         "for a bf16 cache, none for FP8 (the tcgen05 kernel's blocks land on other SMs from "
+                         "step to step, so a placement measured once does not hold)")
     ap.add_argument("--no-static", action="store_true", help="skip the static split-k comparison")
     ap.add_argument("--no-cpu", action="store_true", help="skip the CPU oracle baseline")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
@@ -310,6 +324,11 @@ def run_ours(args, world, rank, local):
         with torch.cuda.stream(stream):
             for _ in range(warm):
                 step()
+            balance_table = None
+            if balance_wanted(args):  # untimed: block times of a few steps -> the table in desc
+                balance_table = da.calibrate_balance(desc, lambda d: step(d, bufs), "cuda", stream=stream)
+                for _ in range(warm):
+                    step()
             torch.cuda.synchronize()
             status = da.da_read_status(bufs.ws, stream=stream)
             # headline: the step captured in a CUDA graph (plan, decode, combine), replayed K times
@@ -395,6 +414,7 @@ def run_ours(args, world, rank, local):
         config=workload_config(args.config, w, w8, args.q_len),
         launch={"tile_tokens": desc.tile_tokens, "ctas_per_kv_head": desc.num_ctas,
                 "merge_in_decode": bool(desc.merge_in_decode), "start_cost": int(desc.start_cost), "graph": True,
+                "balance": BALANCE_NOTE if desc.balance else "none", 
                 "timing": "one CUDA graph per step (plan, decode, combine), K replays between CUDA events on "
                           "the launching stream; median/p10/p90 from a second pass of K replays with an event "
                           "between replays"},
@@ -471,6 +491,12 @@ def run_trace(args, world, rank, local):
         da.decode_step(prob, d, dt.q, dt.k_cache, dt.v_cache, dt.block_table, dt.seq_lens, b, stream=stream,
                        planned=planned)
 
+    balance_table = None
+    if balance_wanted(args):  # untimed, on the trace's first lengths
+        with torch.cuda.stream(stream):
+            balance_table = da.calibrate_balance(desc, lambda d: step(d, bufs), "cuda", stream=stream)
+        torch.cuda.synchronize()
+
     graphs = {}
     with torch.cuda.stream(stream):
         for key, d, b, planned in (("dynamic", desc, bufs, False), ("static", sdesc, sbufs, False),
@@ -528,7 +554,7 @@ def run_trace(args, world, rank, local):
         config={"workload": f"trace: {tr.recipe}", "batch": prob.batch, "steps_timed": steps,
                 "kv_bytes_first_last_step": [kv[0], kv[-1]], "tile_tokens": desc.tile_tokens,
                 "ctas_per_kv_head": desc.num_ctas, "merge_in_decode": bool(desc.merge_in_decode),
-                "start_cost": int(desc.start_cost), "graph": True,
+                "start_cost": int(desc.start_cost), "graph": True, "balance": BALANCE_NOTE if desc.balance else "none", 
                 "untimed": "device copies of each step's changes (restarted pages, block table, lengths, q) "
                            "and the KV append kernel, enqueued between the timed steps",
                 "l2": f"inputs larger than L2 ({min(kv) / 1e9:.1f}-{max(kv) / 1e9:.1f} GB K/V per step), no flush"},

@@ -76,6 +76,8 @@ extern "C" {
 #define DA_DEV_BAD_PAGE 2   /* a block-table entry outside [0, num_pages); that chunk is skipped */
 #define DA_DEV_TIMEOUT 3    /* a pipeline wait gave up after its time limit; results are incomplete */
 #define DA_DEV_BAD_PLAN 4   /* the workspace holds no plan matching this descriptor */
+#define DA_DEV_BAD_BALANCE 5 /* desc->balance is not a table for this descriptor (da_balance_set); the
+                                step ran with the even split instead */
 
 /* ---- plan kinds ---------------------------------------------------------------------- */
 #define DA_PLAN_DYNAMIC 0 /* load-balanced: U tiles over C CTAs per KV head, contiguous ranges */
@@ -163,6 +165,12 @@ typedef struct da_plan_desc {
                               start units evenly, so a CTA that starts many short requests gets
                               fewer tiles.  Default 2 (measured on B200 at 64-token tiles); 0 is the
                               tiles-only plan.  Must be 0 for a static plan. */
+  const int32_t* balance;  /* dynamic plans: dev, a table written by da_balance_set (per-CTA weights
+                              and which CTA of the plan each block of the decode grid runs), or
+                              NULL (default): every CTA gets an even share.  See da_balance_set. */
+  int64_t* block_times;    /* dev int64 [num_kv_heads][num_ctas][2], or NULL (default): every decode
+                              launch writes, for block (x, g) of its grid, the %globaltimer (ns) at
+                              its start and at its end, input to da_balance_from_times */
 } da_plan_desc;
 
 /*
@@ -250,6 +258,71 @@ DA_API int da_workspace_offsets(const da_plan_desc* desc, int64_t off[7]);
  */
 DA_API int da_plan(const da_problem* prob, const da_plan_desc* desc, const int32_t* seq_lens, void* ws,
                    size_t ws_bytes, void* stream);
+
+/*
+ * Balancing the plan against the speed of the SMs.
+ *
+ * The decode kernel streams K/V at the HBM roof while every CTA runs, but with
+ * an even split the CTAs do not end together: some SMs stream a few percent
+ * slower than others (on B200 the same SMs in every workload, within a process
+ * and on other boxes), and the last ones end up to 9 % after the median, with
+ * HBM partly idle meanwhile.  A balance table gives each CTA of the dynamic plan a
+ * weight, and places the CTAs on the blocks of the decode grid so that the
+ * blocks running one CTA (one per KV head) sit on SMs of like speed:
+ *   - CTA c's range of units is [first(c), first(c+1)) with
+ *     first(c) = c + floor((U - C) * W_c / W), W_c = sum_{k<c} w_k, W = sum w
+ *     (one unit each, the rest in proportion; equal weights give the even
+ *     split floor(c*U/C) exactly; with U < C the weights are not used);
+ *   - block (x, g) of the decode grid runs CTA perm[g][x] of the plan.
+ * The table changes who computes which tiles, never what is computed; for a
+ * given table, plan and results are deterministic.  A table is measured with
+ * desc->block_times over a few steps and da_balance_from_times.
+ * Source of the scheme it refines: "Tencent HPC lands in SGLang, challenging
+ * default inference kernels", section "Why Tencent HPC matters for online model
+ * serving" (tiles handed to CTAs by the current workload); the weighting is this
+ * implementation's addition.
+ */
+
+/* Words (int32) of a balance table: 4 + num_ctas + num_kv_heads * num_ctas.  Host only.
+   Errors: DA_ERR_INVALID_ARG (null pointer, not a dynamic descriptor), DA_ERR_UNSUPPORTED
+   (num_ctas above 2048, the planner's limit for weighted ranges). */
+DA_API int da_balance_words(const da_plan_desc* desc, size_t* words);
+
+/*
+ * da_balance_set -- check a balance table on the host and copy it to the device.
+ *   weights  host int32 [num_ctas], each in [1, 65536]
+ *   perm     host int32 [num_kv_heads][num_ctas], each row a permutation of
+ *            0 .. num_ctas-1 (row g, entry x: the CTA of the plan that block
+ *            (x, g) of the decode grid runs)
+ *   table    dev, da_balance_words(desc) int32 words, 4-byte aligned; then set
+ *            desc->balance = table
+ * Enqueues host-to-device copies on `stream` (the host arrays may be reused when
+ * the call returns).  Errors: DA_ERR_INVALID_ARG (null pointer, a weight out of
+ * range, a row that is not a permutation), DA_ERR_UNSUPPORTED as for
+ * da_balance_words, DA_ERR_CUDA (a copy refused).  A table whose header does not
+ * match the descriptor it is used with is ignored by the planner, which records
+ * DA_DEV_BAD_BALANCE.
+ */
+DA_API int da_balance_set(const da_plan_desc* desc, const int32_t* weights, const int32_t* perm, int32_t* table,
+                          void* stream);
+
+/*
+ * da_balance_from_times -- a balance table from measured block times.  Host only.
+ *   times      host int64 [num_kv_heads][num_ctas][2]: start and end (ns) of every
+ *              block, as written to desc->block_times (e.g. per-block medians over
+ *              a few steps), measured with the table (prev_weights, prev_perm)
+ *              in use, NULL for the even split and the identity placement
+ *   weights, perm  host out, as for da_balance_set
+ * Each block's speed is its CTA's share of the work (its weight) over its time.
+ * In every KV head's row the blocks are ranked by speed and block x takes CTA
+ * rank(x), so that CTA c runs on the c-th slowest block of every row; its weight
+ * is the mean speed of those blocks (relative, scaled to 4096 on average).  A block
+ * without a usable time counts at its row's median speed.  Errors:
+ * DA_ERR_INVALID_ARG (null pointer, a previous table that fails the checks of
+ * da_balance_set), DA_ERR_UNSUPPORTED as for da_balance_words.
+ */
+DA_API int da_balance_from_times(const da_plan_desc* desc, const int64_t* times, const int32_t* prev_weights,
+                                 const int32_t* prev_perm, int32_t* weights, int32_t* perm);
 
 /*
  * da_static_plan -- static split-k plan (the comparator), same work-list format.

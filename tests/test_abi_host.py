@@ -267,6 +267,72 @@ def test_status_strings(da_lib):
     assert da.status_string(0) == "ok" and "workspace" in da.status_string(-4)
     assert "length" in da.dev_status_string(1) and "page" in da.dev_status_string(2)
     assert "timed out" in da.dev_status_string(3) and "plan" in da.dev_status_string(4)
+    assert "balance" in da.dev_status_string(5)
+
+
+def test_balance_table_host_checks(da_lib):
+    """Sizes and the checks of da_balance_set that come before any copy."""
+    import ctypes
+    import numpy as np
+    da = da_lib
+    d = da.da_plan_desc_init(prob(da), da.PLAN_DYNAMIC, 64, 37)
+    assert d.balance is None and d.block_times is None
+    assert da.da_balance_words(d) == 4 + 37 + 8 * 37
+    good_w = np.full(37, 4096, np.int32)
+    good_p = np.tile(np.arange(37, dtype=np.int32), (8, 1))
+    fake = ctypes.c_void_p(1 << 20)  # never written: every call below is refused first
+    L = da.lib()
+    cases = [(np.zeros(37, np.int32), good_p), (np.full(37, 65537, np.int32), good_p)]
+    dup = good_p.copy(); dup[3, 5] = dup[3, 6]
+    neg = good_p.copy(); neg[0, 0] = -1
+    cases += [(good_w, dup), (good_w, neg)]
+    for w, p in cases:
+        assert L.da_balance_set(ctypes.byref(d), w.ctypes.data, p.ctypes.data, fake, None) == da.ERR_INVALID_ARG
+    s = da.da_plan_desc_init(prob(da), da.PLAN_STATIC, 64, 4)
+    n = ctypes.c_size_t()
+    assert L.da_balance_words(ctypes.byref(s), ctypes.byref(n)) == da.ERR_INVALID_ARG
+    big = da.da_plan_desc_init(prob(da), da.PLAN_DYNAMIC, 64, 2049)
+    assert L.da_balance_words(ctypes.byref(big), ctypes.byref(n)) == da.ERR_UNSUPPORTED
+    # descriptors carrying a table: dynamic only, aligned, at most 2048 CTAs; block times 8-byte aligned
+    for desc, field, val, code in [(s, "balance", 1 << 20, da.ERR_INVALID_ARG), (d, "balance", (1 << 20) + 2, da.ERR_INVALID_ARG),
+                                   (big, "balance", 1 << 20, da.ERR_UNSUPPORTED),
+                                   (d, "block_times", (1 << 20) + 4, da.ERR_INVALID_ARG)]:
+        setattr(desc, field, val)
+        sizes = (ctypes.c_size_t(), ctypes.c_size_t(), ctypes.c_size_t())
+        rc = L.da_workspace_size(ctypes.byref(prob(da)), ctypes.byref(desc), *map(ctypes.byref, sizes))
+        assert rc == code, (field, val, rc)
+        setattr(desc, field, None)
+
+
+def test_balance_from_times(da_lib):
+    """The table measured from block times: in each KV head's row the slowest block runs CTA 0;
+    a CTA's weight follows the speed of its blocks; a block with no time counts at its row's
+    median; the previous table's weights divide back out."""
+    import numpy as np
+    da = da_lib
+    d = da.da_plan_desc_init(prob(da), da.PLAN_DYNAMIC, 64, 37)
+    rng = np.random.default_rng(4)
+    dur = rng.uniform(90, 110, size=(8, 37))
+    t = np.zeros((8, 37, 2), np.int64)
+    t[:, :, 0] = 1000
+    t[:, :, 1] = 1000 + np.round(dur * 1000).astype(np.int64)
+    w, p = da.da_balance_from_times(d, t)
+    for g in range(8):
+        assert sorted(p[g]) == list(range(37))
+        ns = t[g, :, 1] - t[g, :, 0]
+        assert list(np.argsort(p[g])) == list(np.argsort(-ns, kind="stable"))  # slowest first
+    assert np.all(np.diff(w) >= 0)  # CTA c runs on the c-th slowest blocks: weights rise with c
+    speed = np.sort(1.0 / dur, axis=1).mean(axis=0)
+    np.testing.assert_allclose(w / w.mean(), speed / speed.mean(), rtol=2e-3)
+    assert abs(w.mean() - 4096) < 2
+    # a block without a usable time: the row's median speed
+    t2 = t.copy()
+    t2[2, 5, 1] = t2[2, 5, 0]
+    w2, p2 = da.da_balance_from_times(d, t2)
+    assert sorted(p2[2]) == list(range(37))
+    # measured with a table in use: the same times under twice the work per CTA give twice the speed
+    w3, p3 = da.da_balance_from_times(d, t, np.full(37, 2, np.int32), np.tile(np.arange(37, dtype=np.int32), (8, 1)))
+    assert np.array_equal(p3, p) and np.allclose(w3, w, atol=1)
 
 
 @pytest.mark.skipif(cuda_available(), reason="checks the no-device error path")

@@ -3,9 +3,12 @@
 // (except da_read_status, documented to synchronise its stream).
 #include <cudaTypedefs.h>
 
+#include <algorithm>
 #include <climits>
+#include <cmath>
 #include <cstring>
 #include <mutex>
+#include <vector>
 
 #include "append_rows.cuh"
 #include "da_internal.cuh"
@@ -60,6 +63,11 @@ int check_desc(const da_problem* p, const da_plan_desc* d) {
   if (d->out_format == DA_OUT_F32 && d->merge_in_decode) return DA_ERR_INVALID_ARG;  // the combine writes fp32 out
   if (d->start_cost < 0 || d->start_cost > kMaxStartCost) return DA_ERR_INVALID_ARG;
   if (d->start_cost != 0 && d->kind != DA_PLAN_DYNAMIC) return DA_ERR_INVALID_ARG;
+  if (d->balance) {  // a balance table: dynamic plans, 4-byte aligned, within the planner's limit
+    if (d->kind != DA_PLAN_DYNAMIC || reinterpret_cast<uintptr_t>(d->balance) % 4 != 0) return DA_ERR_INVALID_ARG;
+    if (d->num_ctas > da::kBalanceMaxCtas) return DA_ERR_UNSUPPORTED;
+  }
+  if (reinterpret_cast<uintptr_t>(d->block_times) % 8 != 0) return DA_ERR_INVALID_ARG;
   if (d->kind == DA_PLAN_DYNAMIC) {
     if (d->splits != 0 || (int64_t)d->max_segments != (int64_t)d->num_ctas + (p->batch > 0 ? p->batch : 1) - 1)
       return DA_ERR_INVALID_ARG;
@@ -170,6 +178,8 @@ DA_API int da_plan_desc_init(const da_problem* prob, int32_t kind, int32_t tile_
   d.merge_in_decode = 0;
   d.out_format = DA_OUT_BF16;
   d.start_cost = kind == DA_PLAN_DYNAMIC ? kDefaultStartCost : 0;
+  d.balance = nullptr;
+  d.block_times = nullptr;
   if (kind == DA_PLAN_DYNAMIC) {
     d.num_ctas = w;
     d.splits = 0;
@@ -245,6 +255,7 @@ static int plan_prepare(const da_problem* prob, const da_plan_desc* desc, const 
   p->num_kv_heads = prob->num_kv_heads;
   p->capacity_tokens = (int64_t)prob->max_pages_per_req * prob->page_size;
   p->start_cost = kind == DA_PLAN_DYNAMIC ? desc->start_cost : 0;
+  p->balance = kind == DA_PLAN_DYNAMIC ? desc->balance : nullptr;
   return DA_OK;
 }
 
@@ -323,6 +334,9 @@ static int decode_prepare(const da_problem* prob, const da_plan_desc* desc, cons
   p.stall_producer = g_stall_next_ns != 0 ? 1 : 0;
   p.wait_limit_ns = g_stall_next_ns != 0 ? g_stall_next_ns : kWaitLimitNs;
   g_stall_next_ns = 0;  // one launch only
+  // the balance table's placement part; the kernel follows it only if the plan took the table
+  p.cta_perm = desc->balance ? desc->balance + da::kBalanceHeader + desc->num_ctas : nullptr;
+  p.block_times = desc->block_times;
   return DA_OK;
 }
 
@@ -645,6 +659,106 @@ DA_API int da_read_status(const void* ws, int32_t* dev_status, int32_t* bad_inde
   return DA_OK;
 }
 
+// ---- balance tables -------------------------------------------------------------------
+
+static int balance_check_desc(const da_plan_desc* desc) {
+  if (!desc || desc->kind != DA_PLAN_DYNAMIC || desc->num_ctas <= 0 || desc->num_kv_heads <= 0)
+    return DA_ERR_INVALID_ARG;
+  if (desc->num_ctas > da::kBalanceMaxCtas) return DA_ERR_UNSUPPORTED;
+  return DA_OK;
+}
+
+// weights in range, every row of perm a permutation of 0..C-1
+static bool balance_valid(int C, int H, const int32_t* weights, const int32_t* perm) {
+  for (int c = 0; c < C; ++c)
+    if (weights[c] < 1 || weights[c] > da::kBalanceMaxWeight) return false;
+  std::vector<char> seen((size_t)C);
+  for (int g = 0; g < H; ++g) {
+    std::fill(seen.begin(), seen.end(), 0);
+    for (int x = 0; x < C; ++x) {
+      const int32_t c = perm[(size_t)g * C + x];
+      if (c < 0 || c >= C || seen[(size_t)c]) return false;
+      seen[(size_t)c] = 1;
+    }
+  }
+  return true;
+}
+
+DA_API int da_balance_words(const da_plan_desc* desc, size_t* words) {
+  const int rc = balance_check_desc(desc);
+  if (rc != DA_OK) return rc;
+  if (!words) return DA_ERR_INVALID_ARG;
+  *words = (size_t)da::kBalanceHeader + (size_t)desc->num_ctas * (1 + (size_t)desc->num_kv_heads);
+  return DA_OK;
+}
+
+DA_API int da_balance_set(const da_plan_desc* desc, const int32_t* weights, const int32_t* perm, int32_t* table,
+                          void* stream) {
+  const int rc = balance_check_desc(desc);
+  if (rc != DA_OK) return rc;
+  if (!weights || !perm || !table || reinterpret_cast<uintptr_t>(table) % 4 != 0) return DA_ERR_INVALID_ARG;
+  const int C = desc->num_ctas, H = desc->num_kv_heads;
+  if (!balance_valid(C, H, weights, perm)) return DA_ERR_INVALID_ARG;
+  const int32_t head[da::kBalanceHeader] = {da::kBalanceMagic, C, H, 0};
+  const cudaStream_t s = static_cast<cudaStream_t>(stream);
+  // from pageable host memory: each copy has taken its source when the call returns
+  cudaError_t e = cudaMemcpyAsync(table, head, sizeof(head), cudaMemcpyHostToDevice, s);
+  if (e == cudaSuccess)
+    e = cudaMemcpyAsync(table + da::kBalanceHeader, weights, (size_t)C * 4, cudaMemcpyHostToDevice, s);
+  if (e == cudaSuccess)
+    e = cudaMemcpyAsync(table + da::kBalanceHeader + C, perm, (size_t)C * H * 4, cudaMemcpyHostToDevice, s);
+  return e == cudaSuccess ? DA_OK : cuda_fail(e);
+}
+
+DA_API int da_balance_from_times(const da_plan_desc* desc, const int64_t* times, const int32_t* prev_weights,
+                                 const int32_t* prev_perm, int32_t* weights, int32_t* perm) {
+  const int rc = balance_check_desc(desc);
+  if (rc != DA_OK) return rc;
+  if (!times || !weights || !perm || (prev_weights == nullptr) != (prev_perm == nullptr)) return DA_ERR_INVALID_ARG;
+  const int C = desc->num_ctas, H = desc->num_kv_heads;
+  if (prev_weights && !balance_valid(C, H, prev_weights, prev_perm)) return DA_ERR_INVALID_ARG;
+  // speed of block (x, g): its CTA's share of the work (the weight it ran with) over its time
+  std::vector<double> speed((size_t)C * H);
+  for (int g = 0; g < H; ++g) {
+    std::vector<double> row;
+    for (int x = 0; x < C; ++x) {
+      const size_t i = (size_t)g * C + x;
+      const int c = prev_perm ? prev_perm[i] : x;
+      const double w = prev_weights ? (double)prev_weights[c] : 1.0;
+      const int64_t dt = times[2 * i + 1] - times[2 * i];
+      speed[i] = dt > 0 ? w / (double)dt : -1.0;
+      if (speed[i] > 0) row.push_back(speed[i]);
+    }
+    double med = 1.0;
+    if (!row.empty()) {
+      std::nth_element(row.begin(), row.begin() + row.size() / 2, row.end());
+      med = row[row.size() / 2];
+    }
+    for (int x = 0; x < C; ++x)
+      if (speed[(size_t)g * C + x] <= 0) speed[(size_t)g * C + x] = med;
+  }
+  // rank the blocks of each row by speed (ties by index): block x runs CTA rank(x); CTA c's
+  // speed is the mean over the rows of the c-th slowest block
+  std::vector<double> cta_speed((size_t)C, 0.0);
+  std::vector<int> order((size_t)C);
+  for (int g = 0; g < H; ++g) {
+    const double* sp = speed.data() + (size_t)g * C;
+    for (int x = 0; x < C; ++x) order[(size_t)x] = x;
+    std::stable_sort(order.begin(), order.end(), [sp](int a, int b) { return sp[a] < sp[b]; });
+    for (int r = 0; r < C; ++r) {
+      perm[(size_t)g * C + order[(size_t)r]] = r;
+      cta_speed[(size_t)r] += sp[order[(size_t)r]] / H;
+    }
+  }
+  double mean = 0.0;
+  for (int c = 0; c < C; ++c) mean += cta_speed[(size_t)c] / C;
+  for (int c = 0; c < C; ++c) {
+    const double w = mean > 0 ? 4096.0 * cta_speed[(size_t)c] / mean : 4096.0;
+    weights[c] = (int32_t)std::min<double>(std::max<double>(std::llround(w), 1.0), (double)da::kBalanceMaxWeight);
+  }
+  return DA_OK;
+}
+
 DA_API const char* da_status_string(int32_t code) {
   switch (code) {
     case DA_OK: return "ok";
@@ -663,6 +777,7 @@ DA_API const char* da_dev_status_string(int32_t code) {
     case DA_DEV_BAD_PAGE: return "block-table page id out of range";
     case DA_DEV_TIMEOUT: return "pipeline wait timed out";
     case DA_DEV_BAD_PLAN: return "workspace plan does not match the descriptor";
+    case DA_DEV_BAD_BALANCE: return "balance table does not match the descriptor (even split used)";
     default: return "unknown device status";
   }
 }

@@ -24,6 +24,7 @@ enum HeaderWord {
   kHdrBatch = 7,
   kHdrMaxSegments = 8,
   kHdrSplits = 9,
+  kHdrBalance = 10,  // 1: the plan used the descriptor's balance table (the decode follows its placement)
   kHdrWords = 16,
 };
 
@@ -56,7 +57,14 @@ struct PlanParams {
   int32_t batch, tile_tokens, width, max_segments, num_ctas, num_kv_heads;
   int64_t capacity_tokens;
   int32_t start_cost;  // dynamic plan: start units charged to every non-empty request
+  const int32_t* balance;  // dynamic plan: balance table (weights and placement), or null
 };
+
+// Balance table: [magic, num_ctas, num_kv_heads, 0, weights[C], perm[Hkv][C]].
+constexpr int32_t kBalanceMagic = 0x0DA0BA1A;
+constexpr int32_t kBalanceMaxCtas = 2048;     // weighted ranges are kept in the planner's shared memory
+constexpr int32_t kBalanceMaxWeight = 65536;
+constexpr int kBalanceHeader = 4;
 
 struct DecodeParams {
   const __nv_bfloat16* q;
@@ -79,6 +87,9 @@ struct DecodeParams {
   int32_t stall_producer;   // failure-path test: the producer sends nothing, so every wait runs out
   uint64_t wait_limit_ns;   // limit of every pipeline wait
   int32_t out_f32;          // 1: every segment's result goes to the partials (the combine writes fp32 out)
+  const int32_t* cta_perm;  // [Hkv][num_ctas]: the plan CTA block (x, g) runs, used when the plan took the
+                            // balance table (header word kHdrBalance); null: block x runs CTA x
+  int64_t* block_times;     // [Hkv][num_ctas][2]: start and end ns of every block, or null
 };
 
 struct CombineParams {
@@ -195,6 +206,24 @@ __device__ __forceinline__ uint64_t global_timer_ns() {
   uint64_t t;
   asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
   return t;
+}
+
+// ---- balance table in the decode kernels -----------------------------------------------
+// The plan CTA that block (blockIdx.x, KV head blockIdx.y) runs if the plan took the balance
+// table (read before the plan lands; an entry out of range keeps the block's own index).
+__device__ __forceinline__ int placed_cta(const DecodeParams& p) {
+  if (!p.cta_perm) return (int)blockIdx.x;
+  const int c = __ldg(p.cta_perm + (int64_t)blockIdx.y * p.num_ctas + blockIdx.x);
+  return c >= 0 && c < p.num_ctas ? c : (int)blockIdx.x;
+}
+
+// Thread 0: this block's start (t_start) and end times, when the descriptor asked for them.
+__device__ __forceinline__ void record_block_times(const DecodeParams& p, uint64_t t_start) {
+  if (p.block_times && threadIdx.x == 0) {
+    int64_t* bt = p.block_times + ((int64_t)blockIdx.y * gridDim.x + blockIdx.x) * 2;
+    bt[0] = (int64_t)t_start;
+    bt[1] = (int64_t)global_timer_ns();
+  }
 }
 
 // Bounded wait on an mbarrier phase.  Gives up (returns false) when *abort is

@@ -342,14 +342,17 @@ __global__ void __launch_bounds__(kThreads, 2)
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const uint32_t sbase = smem_u32(smem);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int cta = blockIdx.x, g = blockIdx.y;
+  const int g = blockIdx.y;
+  __shared__ unsigned long long s_t_start;
 
   // Prologue that does not depend on the plan: barriers and descriptor
   // prefetch overlap the planner kernel (programmatic dependent launch).
   const uint32_t full0 = sbase + C::kOffBars, empty0 = full0 + C::kStages * 8;
   volatile int* meta = reinterpret_cast<volatile int*>(smem + C::kOffMeta);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::kOffAbort);
+  const int placed = placed_cta(p);
   if (threadIdx.x == 0) {
+    s_t_start = p.block_times ? global_timer_ns() : 0;
     for (int s = 0; s < C::kStages; ++s) {
       mbar_init(full0 + 8 * s, 1);
       mbar_init(empty0 + 8 * s, kConsumerWarps);
@@ -425,11 +428,19 @@ __global__ void __launch_bounds__(kThreads, 2)
   const int32_t* csb = p.ws + WL.cta_seg_begin;
   int32_t* hdr_w = const_cast<int32_t*>(hdr);
 
-  // The plan must match the descriptor this launch was given.
+  // The plan must match the descriptor this launch was given.  Which plan CTA this block runs:
+  // its own index, or its place in the balance table if the plan took the table (both CTAs'
+  // ranges are loaded with the header, so the choice adds no round trip).
   const int h_ctas = hdr[kHdrCtas], h_batch = hdr[kHdrBatch], h_ms = hdr[kHdrMaxSegments], h_kind = hdr[kHdrKind];
-  const int h_segs = hdr[kHdrSegments], seg_lo = csb[cta], seg_next = csb[cta + 1];
+  const int own = blockIdx.x;
+  const int h_segs = hdr[kHdrSegments], own_lo = csb[own], own_next = csb[own + 1];
+  const int alt_lo = csb[placed], alt_next = csb[placed + 1];
+  const bool balanced = hdr[kHdrBalance] == 1;
+  const int cta = balanced ? placed : own;
+  const int seg_lo = balanced ? alt_lo : own_lo, seg_next = balanced ? alt_next : own_next;
   if (h_ctas != p.num_ctas || h_batch != p.batch || h_ms != p.max_segments || h_kind != p.kind) {
-    if (threadIdx.x == 0 && cta == 0 && g == 0) record_status(hdr_w, DA_DEV_BAD_PLAN, 0);
+    if (threadIdx.x == 0 && blockIdx.x == 0 && g == 0) record_status(hdr_w, DA_DEV_BAD_PLAN, 0);
+    record_block_times(p, s_t_start);
     return;
   }
   const int seg_hi = min(seg_next, min(h_segs, p.max_segments));
@@ -447,7 +458,10 @@ __global__ void __launch_bounds__(kThreads, 2)
       }
     }
   }
-  if (seg_lo < 0 || seg_lo >= seg_hi) return;  // nothing planned for this CTA (uniform over the block)
+  if (seg_lo < 0 || seg_lo >= seg_hi) {  // nothing planned for this CTA (uniform over the block)
+    record_block_times(p, s_t_start);
+    return;
+  }
 
   if (warp == kConsumerWarps) {
     // ------------------------------------------------------------------ producer warp
@@ -523,6 +537,7 @@ __global__ void __launch_bounds__(kThreads, 2)
 #if DA_BF16_FFMA
   if constexpr (!FP8 && !MQ && !MERGE && D == 128) {
     ffma_consumer<C>(p, smem, segs, rsb, hdr_w, full0, empty0, meta, abort_flag, seg_lo, seg_hi, g, warp, lane);
+    record_block_times(p, s_t_start);
     return;
   }
 #endif
@@ -935,6 +950,7 @@ __global__ void __launch_bounds__(kThreads, 2)
       }
     }
   }
+  record_block_times(p, s_t_start);  // thread 0 is a consumer: every segment of the block is done
 }
 
 template <int D, bool FP8, bool MQ, bool MERGE>

@@ -255,7 +255,9 @@ __global__ void __launch_bounds__(kThreadsTc, 2)
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const uint32_t sbase = smem_u32(smem);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int cta = blockIdx.x, g = blockIdx.y;
+  const int g = blockIdx.y;
+  __shared__ unsigned long long s_t_start;
+  const int placed = placed_cta(p);  // the plan CTA this block runs if the plan took the balance table
   const uint32_t bars = sbase + kOffBars;
   auto bar = [bars](int i) -> uint32_t { return bars + 8u * (uint32_t)i; };
   volatile int* meta = reinterpret_cast<volatile int*>(smem + kOffMeta);
@@ -263,6 +265,7 @@ __global__ void __launch_bounds__(kThreadsTc, 2)
   volatile uint32_t* tmem_slot = reinterpret_cast<volatile uint32_t*>(smem + kOffFlags + 4);
 
   if (threadIdx.x == 0) {
+    s_t_start = p.block_times ? global_timer_ns() : 0;
     for (int s = 0; s < kKSlots; ++s) {
       mbar_init(bar(kBarKFull + s), 1);
       mbar_init(bar(kBarKEmpty + s), 1);  // released by the tensor core (commit after S)
@@ -345,13 +348,21 @@ __global__ void __launch_bounds__(kThreadsTc, 2)
   const int32_t* csb = p.ws + WL.cta_seg_begin;
   int32_t* hdr_w = const_cast<int32_t*>(hdr);
   const int h_ctas = hdr[kHdrCtas], h_batch = hdr[kHdrBatch], h_ms = hdr[kHdrMaxSegments], h_kind = hdr[kHdrKind];
-  const int h_segs = hdr[kHdrSegments], seg_lo = csb[cta], seg_next = csb[cta + 1];
+  const int own = blockIdx.x;
+  const int h_segs = hdr[kHdrSegments], own_lo = csb[own], own_next = csb[own + 1];
+  const int alt_lo = csb[placed], alt_next = csb[placed + 1];
+  const bool balanced = hdr[kHdrBalance] == 1;  // the plan took the balance table: follow its placement
+  const int seg_lo = balanced ? alt_lo : own_lo, seg_next = balanced ? alt_next : own_next;
   if (h_ctas != p.num_ctas || h_batch != p.batch || h_ms != p.max_segments || h_kind != p.kind) {
-    if (threadIdx.x == 0 && cta == 0 && g == 0) record_status(hdr_w, DA_DEV_BAD_PLAN, 0);
+    if (threadIdx.x == 0 && blockIdx.x == 0 && g == 0) record_status(hdr_w, DA_DEV_BAD_PLAN, 0);
+    record_block_times(p, s_t_start);
     return;  // before TMEM is allocated
   }
   const int seg_hi = min(seg_next, min(h_segs, p.max_segments));
-  if (seg_lo < 0 || seg_lo >= seg_hi) return;  // nothing planned for this CTA (uniform over the block)
+  if (seg_lo < 0 || seg_lo >= seg_hi) {  // nothing planned for this CTA (uniform over the block)
+    record_block_times(p, s_t_start);
+    return;
+  }
 
   // TMEM for this CTA (64 of the SM's 512 columns; two CTAs per SM).  The producer does not
   // wait for it: its first requests go out while the MMA warp allocates and the softmax
@@ -724,6 +735,7 @@ __global__ void __launch_bounds__(kThreadsTc, 2)
   __syncthreads();
   tc_fence_after();
   if (warp == kMmaWarp) tmem_dealloc(tmem, kTmemCols);
+  record_block_times(p, s_t_start);
 }
 
 }  // namespace

@@ -96,36 +96,22 @@ __device__ void tile_prefix(const PlanParams& p, int32_t* rtp, int32_t* s_rtp, i
   __syncthreads();
 }
 
-__device__ void write_header(const PlanParams& p, int32_t* hdr, int U, int S, int kind, int splits, int bad) {
+// balance: 1 the plan used a balance table, 0 none was given, -1 one was given but refused.
+__device__ void write_header(const PlanParams& p, int32_t* hdr, int U, int S, int kind, int splits, int bad,
+                             int balance = 0) {
   hdr[kHdrUnits] = U;
   hdr[kHdrSegments] = S;
   hdr[kHdrCtas] = p.num_ctas;
   hdr[kHdrTile] = p.tile_tokens;
-  hdr[kHdrStatus] = bad == INT_MAX ? DA_DEV_OK : DA_DEV_BAD_SEQLEN;
+  hdr[kHdrStatus] = bad != INT_MAX ? DA_DEV_BAD_SEQLEN : balance < 0 ? DA_DEV_BAD_BALANCE : DA_DEV_OK;
   hdr[kHdrBadIndex] = bad == INT_MAX ? -1 : bad;
   hdr[kHdrKind] = kind;
   hdr[kHdrBatch] = p.batch;
   hdr[kHdrMaxSegments] = p.max_segments;
   hdr[kHdrSplits] = splits;
-  for (int i = kHdrSplits + 1; i < kHdrWords; ++i) hdr[i] = 0;
+  hdr[kHdrBalance] = balance > 0 ? 1 : 0;
+  for (int i = kHdrBalance + 1; i < kHdrWords; ++i) hdr[i] = 0;
 }
-
-// CTA that owns global tile u: the unique c with floor(c*U/C) <= u < floor((c+1)*U/C),
-// and the first tile of CTA c.  Every product is below C*(U+1); when that fits in 32
-// bits (the common case) the divisions are done in 32-bit integers.
-struct Split {
-  int64_t U, C;
-  bool narrow;
-  __device__ Split(int64_t u, int64_t c) : U(u), C(c), narrow(c * (u + 1) < (int64_t(1) << 31)) {}
-  __device__ __forceinline__ int owner(int64_t u) const {
-    if (narrow) return (int)(((uint32_t)(u + 1) * (uint32_t)C - 1u) / (uint32_t)U);
-    return (int)(((u + 1) * C - 1) / U);
-  }
-  __device__ __forceinline__ int64_t first(int64_t c) const {
-    if (narrow) return (int64_t)(((uint32_t)c * (uint32_t)U) / (uint32_t)C);
-    return c * U / C;
-  }
-};
 
 // Largest i in [0, n] with a[i] <= x, for a non-decreasing a[0..n] with a[0] <= x.
 __device__ __forceinline__ int last_not_above(const int32_t* a, int n, int64_t x) {
@@ -137,11 +123,96 @@ __device__ __forceinline__ int last_not_above(const int32_t* a, int n, int64_t x
   return lo;
 }
 
+// CTA that owns global unit u, and the first unit of CTA c.  Even split: the unique c with
+// floor(c*U/C) <= u < floor((c+1)*U/C); every product is below C*(U+1), and when that fits
+// in 32 bits (the common case) the divisions are done in 32-bit integers.  Weighted (a
+// balance table, U >= C): the ranges start at F[c], kept in shared memory.
+struct Split {
+  int64_t U, C;
+  bool narrow;
+  const int32_t* F;  // weighted range starts F[0..C], or null
+  __device__ Split(int64_t u, int64_t c, const int32_t* f)
+      : U(u), C(c), narrow(c * (u + 1) < (int64_t(1) << 31)), F(f) {}
+  __device__ __forceinline__ int owner(int64_t u) const {
+    if (F) return last_not_above(F, (int)C, u);
+    if (narrow) return (int)(((uint32_t)(u + 1) * (uint32_t)C - 1u) / (uint32_t)U);
+    return (int)(((u + 1) * C - 1) / U);
+  }
+  __device__ __forceinline__ int64_t first(int64_t c) const {
+    if (F) return F[c];
+    if (narrow) return (int64_t)(((uint32_t)c * (uint32_t)U) / (uint32_t)C);
+    return c * U / C;
+  }
+};
+
+// The balance table's weights, if the table fits this plan: each thread keeps the weights of
+// CTAs t, t + kPlanThreads, ... (loaded before the lengths, so the two loads overlap).
+constexpr int kBalancePerThread = (kBalanceMaxCtas + kPlanThreads - 1) / kPlanThreads;
+struct BalanceWeights {
+  int32_t w[kBalancePerThread];
+  bool given;  // a table pointer was given
+};
+
+__device__ __forceinline__ BalanceWeights load_balance(const PlanParams& p) {
+  BalanceWeights bw;
+  bw.given = p.balance != nullptr;
+#pragma unroll
+  for (int k = 0; k < kBalancePerThread; ++k) {
+    const int c = threadIdx.x + k * kPlanThreads;
+    bw.w[k] = bw.given && p.num_ctas <= kBalanceMaxCtas && c < p.num_ctas ? p.balance[kBalanceHeader + c] : 1;
+  }
+  return bw;
+}
+
+// Checks the table against the plan (header, weight range) and, when it fits and U >= C,
+// writes the weighted range starts F[c] = c + floor((U - C) * W_c / W) for c = 0..C.
+// Returns 1 (table used), 0 (no table) or -1 (table refused).  Block-wide: every thread calls.
+__device__ int weighted_starts(const PlanParams& p, const BalanceWeights& bw, int U, int32_t* F, int* warp_buf,
+                               int* s_flag) {
+  if (!bw.given) return 0;
+  const int C = p.num_ctas;
+  if (threadIdx.x == 0) {
+    const bool hdr_ok = C <= kBalanceMaxCtas && p.balance[0] == kBalanceMagic && p.balance[1] == C &&
+                        p.balance[2] == p.num_kv_heads;
+    *s_flag = hdr_ok ? 1 : -1;
+  }
+  __syncthreads();
+  int bad = 0;
+#pragma unroll
+  for (int k = 0; k < kBalancePerThread; ++k)
+    if (threadIdx.x + k * kPlanThreads < C && (bw.w[k] < 1 || bw.w[k] > kBalanceMaxWeight)) bad = 1;
+  if (__syncthreads_or(bad) && threadIdx.x == 0) *s_flag = -1;
+  __syncthreads();
+  const int flag = *s_flag;
+  if (flag < 0 || U < C) return flag;
+  // exclusive prefix of the weights (each sum below 2^28), then the range starts
+  int carry = 0, total = 0;
+#pragma unroll
+  for (int k = 0; k < kBalancePerThread; ++k) {
+    const int c = threadIdx.x + k * kPlanThreads;
+    const int v = c < C ? bw.w[k] : 0;
+    const int excl = block_exclusive_scan(v, &total, warp_buf);
+    if (c < C) F[c] = carry + excl;
+    carry += total;
+    if (k * kPlanThreads + kPlanThreads >= C) break;  // uniform over the block
+  }
+  __syncthreads();
+  const int64_t W = carry;
+  for (int c = threadIdx.x; c <= C; c += kPlanThreads) {
+    const int64_t Wc = c < C ? F[c] : W;
+    F[c] = (int32_t)(c + (int64_t)(U - C) * Wc / W);
+  }
+  __syncthreads();
+  return 1;
+}
+
 // The dynamic plan, computed by one block of kPlanThreads threads.
 __device__ void plan_dynamic_body(const PlanParams& p) {
   __shared__ int warp_buf[32];
-  __shared__ int s_bad;
+  __shared__ int s_bad, s_bal;
   __shared__ int32_t s_rtp[kSmemBatch + 1], s_rsb[kSmemBatch + 1];
+  __shared__ int32_t s_first[kBalanceMaxCtas + 1];
+  const BalanceWeights bw = load_balance(p);
   if (threadIdx.x == 0) s_bad = INT_MAX;
   __syncthreads();
 
@@ -164,7 +235,8 @@ __device__ void plan_dynamic_body(const PlanParams& p) {
   const int sc = p.start_cost;
   int U;
   tile_prefix(p, rtp, small ? s_rtp : nullptr, warp_buf, &s_bad, &U, nullptr, sc);
-  const Split sp(U, C);
+  const int balance = weighted_starts(p, bw, U, s_first, warp_buf, &s_bal);
+  const Split sp(U, C, balance > 0 && (int64_t)U >= C ? s_first : nullptr);
   auto first_tile = [&](int b) -> int { return rtp_r[b] + (rtp_r[b + 1] > rtp_r[b] ? sc : 0); };
 
   // Segments per request.  With U >= C every CTA owns at least one unit, so a
@@ -224,7 +296,7 @@ __device__ void plan_dynamic_body(const PlanParams& p) {
     }
     csb[c] = first;
   }
-  if (threadIdx.x == 0) write_header(p, hdr, U, S, DA_PLAN_DYNAMIC, 0, s_bad);
+  if (threadIdx.x == 0) write_header(p, hdr, U, S, DA_PLAN_DYNAMIC, 0, s_bad, balance);
 }
 
 __global__ void __launch_bounds__(kPlanThreads) plan_dynamic_kernel(const PlanParams p) {

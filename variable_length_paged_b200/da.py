@@ -16,7 +16,7 @@ HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.environ.get("DA_LIB_PATH") or os.path.join(HERE, "libda.so")
 
 OK, ERR_INVALID_ARG, ERR_UNSUPPORTED, ERR_CUDA, ERR_WORKSPACE = 0, -1, -2, -3, -4
-DEV_OK, DEV_BAD_SEQLEN, DEV_BAD_PAGE, DEV_TIMEOUT, DEV_BAD_PLAN = 0, 1, 2, 3, 4
+DEV_OK, DEV_BAD_SEQLEN, DEV_BAD_PAGE, DEV_TIMEOUT, DEV_BAD_PLAN, DEV_BAD_BALANCE = 0, 1, 2, 3, 4, 5
 PLAN_DYNAMIC, PLAN_STATIC = 0, 1
 OUT_BF16, OUT_F32 = 0, 1
 
@@ -26,7 +26,8 @@ EXPORTS = ("da_plan_desc_init", "da_workspace_size", "da_workspace_offsets", "da
            "da_last_cuda_error", "da_device_num_sms", "da_decode_step_noalloc", "da_append_kv",
            "da_decode_attention_fp8", "da_merge_partials", "da_decode_step_host", "da_test_stall_next_decode",
            "da_plan_append", "da_plan_workspace_size", "da_noalloc_read_status",
-           "da_merge_partials_f32", "da_decode_step")
+           "da_merge_partials_f32", "da_decode_step", "da_balance_words", "da_balance_set",
+           "da_balance_from_times")
 
 NOALLOC_SCRATCH_BYTES = 16 << 20  # DA_NOALLOC_SCRATCH_BYTES
 
@@ -41,7 +42,8 @@ class DaPlanDesc(ctypes.Structure):
     _fields_ = [("kind", ctypes.c_int32), ("batch", ctypes.c_int32), ("tile_tokens", ctypes.c_int32),
                 ("num_ctas", ctypes.c_int32), ("splits", ctypes.c_int32), ("max_segments", ctypes.c_int32),
                 ("num_kv_heads", ctypes.c_int32), ("merge_in_decode", ctypes.c_int32),
-                ("out_format", ctypes.c_int32), ("start_cost", ctypes.c_int32)]
+                ("out_format", ctypes.c_int32), ("start_cost", ctypes.c_int32),
+                ("balance", ctypes.c_void_p), ("block_times", ctypes.c_void_p)]
 
 
 class DaError(RuntimeError):
@@ -92,6 +94,9 @@ def lib():
             "da_plan_append": [P, D, _vp, _vp, _sz, _vp, _vp, _vp, _vp, _vp, _vp, _vp],
             "da_decode_step_host": [P, D, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _sz, _vp, _vp, _vp,
                                     _vp, _vp, _vp, _vp],
+            "da_balance_words": [D, ctypes.POINTER(_sz)],
+            "da_balance_set": [D, _vp, _vp, _vp, _vp],
+            "da_balance_from_times": [D, _vp, _vp, _vp, _vp, _vp],
         }
         for name, args in sig.items():
             fn = getattr(L, name)
@@ -302,6 +307,65 @@ def da_noalloc_read_status(stream=None) -> tuple[int, int]:
     return st.value, bad.value
 
 
+def da_balance_words(desc: DaPlanDesc) -> int:
+    n = _sz()
+    _check("da_balance_words", lib().da_balance_words(ctypes.byref(desc), ctypes.byref(n)))
+    return n.value
+
+
+def da_balance_set(desc: DaPlanDesc, weights, perm, table, stream=None):
+    """Check (weights [C], perm [Hkv][C], host int32 arrays) and copy them into the device table."""
+    import numpy as np
+    w = np.ascontiguousarray(weights, dtype=np.int32)
+    p = np.ascontiguousarray(perm, dtype=np.int32)
+    _check("da_balance_set", lib().da_balance_set(ctypes.byref(desc), w.ctypes.data, p.ctypes.data, _ptr(table),
+                                                  _stream(stream)))
+
+
+def da_balance_from_times(desc: DaPlanDesc, times, prev_weights=None, prev_perm=None):
+    """(weights, perm) from block times [Hkv][C][2] (host int64), measured with the previous
+    table in use (None: even split, identity placement)."""
+    import numpy as np
+    C, H = desc.num_ctas, desc.num_kv_heads
+    t = np.ascontiguousarray(times, dtype=np.int64)
+    assert t.size == 2 * C * H
+    pw = None if prev_weights is None else np.ascontiguousarray(prev_weights, dtype=np.int32)
+    pp = None if prev_perm is None else np.ascontiguousarray(prev_perm, dtype=np.int32)
+    w = np.zeros(C, np.int32)
+    p = np.zeros((H, C), np.int32)
+    _check("da_balance_from_times", lib().da_balance_from_times(
+        ctypes.byref(desc), t.ctypes.data, None if pw is None else pw.ctypes.data,
+        None if pp is None else pp.ctypes.data, w.ctypes.data, p.ctypes.data))
+    return w, p
+
+
+def calibrate_balance(desc: DaPlanDesc, run_step, device, rounds: int = 2, steps: int = 9, stream=None):
+    """Measure a balance table for `desc` and install it (sets desc.balance; returns the device
+    table, which must outlive the descriptor's use).  run_step(desc) enqueues one step with the
+    descriptor it is given.  Each round runs `steps` steps with block times, takes every block's
+    median start and end, and refines the table from them."""
+    import numpy as np
+    import torch
+    C, H = desc.num_ctas, desc.num_kv_heads
+    table = torch.zeros(da_balance_words(desc), dtype=torch.int32, device=device)
+    times = torch.zeros((steps, H, C, 2), dtype=torch.int64, device=device)
+    w = p = None
+    for _ in range(rounds):
+        for k in range(steps):
+            desc.block_times = times[k].data_ptr()
+            run_step(desc)
+        desc.block_times = None
+        torch.cuda.synchronize()
+        t = times.cpu().numpy()
+        med = np.median(t - t[:, :, :, :1].min(axis=(1, 2, 3), keepdims=True), axis=0).astype(np.int64)
+        w, p = da_balance_from_times(desc, med, w, p)
+        da_balance_set(desc, w, p, table, stream=stream)
+        if stream is None:
+            torch.cuda.synchronize()
+        desc.balance = table.data_ptr()
+    return table
+
+
 # ---- buffers and one whole step --------------------------------------------------------------------
 
 class Buffers:
@@ -357,7 +421,7 @@ def read_plan(desc: DaPlanDesc, ws) -> dict:
     B, C = desc.batch, desc.num_ctas
     return dict(num_units=int(hdr[0]), num_segments=S, num_ctas=int(hdr[2]), tile_tokens=int(hdr[3]),
                 status=int(hdr[4]), bad_index=int(hdr[5]), kind=int(hdr[6]), batch=int(hdr[7]),
-                max_segments=int(hdr[8]), splits=int(hdr[9]),
+                max_segments=int(hdr[8]), splits=int(hdr[9]), balance=int(hdr[10]),
                 seg_req=segs[:, 0].copy(), seg_cta=segs[:, 1].copy(), seg_tile_begin=segs[:, 2].copy(),
                 seg_tile_end=segs[:, 3].copy(), req_tile_prefix=w[off[2]:off[2] + B + 1].copy(),
                 req_seg_begin=w[off[3]:off[3] + B + 1].copy(), cta_seg_begin=w[off[4]:off[4] + C + 1].copy())
