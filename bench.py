@@ -52,6 +52,32 @@ def balance_wanted(args) -> bool:
     return args.balance == "measure" or (args.balance == "auto" and args.kv == "bf16")
 
 
+def measure_balance(da, desc, step, stream, reps: int = 3, n: int = 20) -> dict:
+    """Measure a balance table into desc (untimed), then keep it only if the step is faster with
+    it: a CUDA graph of the step with the table and one without, `n` replays each, alternated
+    `reps` times, best of each.  The table places the plan's CTAs by the SMs the blocks ran on
+    while it was measured; the check guards against a launch that lands them elsewhere."""
+    import torch
+    table = da.calibrate_balance(desc, step, "cuda", stream=stream)
+    graphs = {}
+    for keep in (True, False):
+        desc.balance = table.data_ptr() if keep else None
+        step(desc)
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=stream):
+            step(desc)
+        graphs[keep] = g
+    best = {True: float("inf"), False: float("inf")}
+    for _ in range(reps):
+        for keep in (True, False):
+            best[keep] = min(best[keep], time_region(stream, graphs[keep].replay, n) / n * 1e3)
+    kept = best[True] < best[False]
+    desc.balance = table.data_ptr() if kept else None
+    del graphs
+    return dict(table=table, note={"measured": BALANCE_NOTE, "kept": kept,
+                                   "check_us_per_step_with_without": [round(best[True], 2), round(best[False], 2)]})
+
+
 METRIC = "µs/decode step and KV-read HBM GB/s (% of B200 peak) vs static split-k"
 FALLBACK_HBM_GBS = 6650.0
 DATASHEET_HBM_GBS = 8000.0
@@ -324,9 +350,9 @@ def run_ours(args, world, rank, local):
         with torch.cuda.stream(stream):
             for _ in range(warm):
                 step()
-            balance_table = None
+            balance = {"note": "none"}
             if balance_wanted(args):  # untimed: block times of a few steps -> the table in desc
-                balance_table = da.calibrate_balance(desc, lambda d: step(d, bufs), "cuda", stream=stream)
+                balance = measure_balance(da, desc, lambda d: step(d, bufs), stream)
                 for _ in range(warm):
                     step()
             torch.cuda.synchronize()
@@ -414,7 +440,7 @@ def run_ours(args, world, rank, local):
         config=workload_config(args.config, w, w8, args.q_len),
         launch={"tile_tokens": desc.tile_tokens, "ctas_per_kv_head": desc.num_ctas,
                 "merge_in_decode": bool(desc.merge_in_decode), "start_cost": int(desc.start_cost), "graph": True,
-                "balance": BALANCE_NOTE if desc.balance else "none", 
+                "balance": balance["note"],
                 "timing": "one CUDA graph per step (plan, decode, combine), K replays between CUDA events on "
                           "the launching stream; median/p10/p90 from a second pass of K replays with an event "
                           "between replays"},
@@ -491,10 +517,10 @@ def run_trace(args, world, rank, local):
         da.decode_step(prob, d, dt.q, dt.k_cache, dt.v_cache, dt.block_table, dt.seq_lens, b, stream=stream,
                        planned=planned)
 
-    balance_table = None
+    balance = {"note": "none"}
     if balance_wanted(args):  # untimed, on the trace's first lengths
         with torch.cuda.stream(stream):
-            balance_table = da.calibrate_balance(desc, lambda d: step(d, bufs), "cuda", stream=stream)
+            balance = measure_balance(da, desc, lambda d: step(d, bufs), stream)
         torch.cuda.synchronize()
 
     graphs = {}
@@ -554,7 +580,7 @@ def run_trace(args, world, rank, local):
         config={"workload": f"trace: {tr.recipe}", "batch": prob.batch, "steps_timed": steps,
                 "kv_bytes_first_last_step": [kv[0], kv[-1]], "tile_tokens": desc.tile_tokens,
                 "ctas_per_kv_head": desc.num_ctas, "merge_in_decode": bool(desc.merge_in_decode),
-                "start_cost": int(desc.start_cost), "graph": True, "balance": BALANCE_NOTE if desc.balance else "none", 
+                "start_cost": int(desc.start_cost), "graph": True, "balance": balance["note"], 
                 "untimed": "device copies of each step's changes (restarted pages, block table, lengths, q) "
                            "and the KV append kernel, enqueued between the timed steps",
                 "l2": f"inputs larger than L2 ({min(kv) / 1e9:.1f}-{max(kv) / 1e9:.1f} GB K/V per step), no flush"},
