@@ -70,8 +70,27 @@ int main(void) {
   p.num_q_heads = 64; p.head_dim = 96;
   CHECK(da_plan_desc_init(&p, DA_PLAN_DYNAMIC, 64, 37, &d) == DA_ERR_UNSUPPORTED);
 
+  /* balance tables: sizes, and a table from block times (host only) */
+  p.head_dim = 128;
+  CHECK(da_plan_desc_init(&p, DA_PLAN_DYNAMIC, 64, 37, &d) == DA_OK);
+  CHECK(d.balance == NULL && d.block_times == NULL);
+  {
+    size_t words = 0;
+    int64_t times[8 * 37 * 2];
+    int32_t w[37], perm[8 * 37];
+    CHECK(da_balance_words(&d, &words) == DA_OK && words == 4 + 37 + 8 * 37);
+    CHECK(da_balance_words(&s, &words) == DA_ERR_INVALID_ARG);
+    for (int i = 0; i < 8 * 37; ++i) {
+      times[2 * i] = 1000;
+      times[2 * i + 1] = 1000 + 100000 + (i % 37) * 100;  /* block x of every row: slower as x grows */
+    }
+    CHECK(da_balance_from_times(&d, times, NULL, NULL, w, perm) == DA_OK);
+    CHECK(perm[0] == 36 && perm[36] == 0 && w[0] < w[36]);  /* the slowest block runs CTA 0 */
+    perm[1] = perm[0];  /* not a permutation: refused before any copy */
+    CHECK(da_balance_set(&d, w, perm, (int32_t*)256, NULL) == DA_ERR_INVALID_ARG);
+  }
   CHECK(strlen(da_status_string(DA_OK)) > 0 && strlen(da_status_string(DA_ERR_WORKSPACE)) > 0);
-  CHECK(strlen(da_dev_status_string(DA_DEV_TIMEOUT)) > 0);
+  CHECK(strlen(da_dev_status_string(DA_DEV_TIMEOUT)) > 0 && strlen(da_dev_status_string(DA_DEV_BAD_BALANCE)) > 0);
   printf("%s\n", fails ? "C ABI FAILED" : "C ABI OK");
   return fails != 0;
 }
