@@ -296,8 +296,9 @@ DA_API int da_balance_words(const da_plan_desc* desc, size_t* words);
  *            (x, g) of the decode grid runs)
  *   table    dev, da_balance_words(desc) int32 words, 4-byte aligned; then set
  *            desc->balance = table
- * Enqueues host-to-device copies on `stream` (the host arrays may be reused when
- * the call returns).  Errors: DA_ERR_INVALID_ARG (null pointer, a weight out of
+ * Enqueues host-to-device copies on `stream`.  Pageable host arrays may be reused
+ * when the call returns; page-locked ones must stay unchanged until the copies
+ * have run.  Errors: DA_ERR_INVALID_ARG (null pointer, a weight out of
  * range, a row that is not a permutation), DA_ERR_UNSUPPORTED as for
  * da_balance_words, DA_ERR_CUDA (a copy refused).  A table whose header does not
  * match the descriptor it is used with is ignored by the planner, which records

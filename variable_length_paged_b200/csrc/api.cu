@@ -701,7 +701,8 @@ DA_API int da_balance_set(const da_plan_desc* desc, const int32_t* weights, cons
   if (!balance_valid(C, H, weights, perm)) return DA_ERR_INVALID_ARG;
   const int32_t head[da::kBalanceHeader] = {da::kBalanceMagic, C, H, 0};
   const cudaStream_t s = static_cast<cudaStream_t>(stream);
-  // from pageable host memory: each copy has taken its source when the call returns
+  // the header is a stack array (pageable: staged before cudaMemcpyAsync returns); the caller's
+  // weights and perm follow the same rule, or, if page-locked, must outlive the copies
   cudaError_t e = cudaMemcpyAsync(table, head, sizeof(head), cudaMemcpyHostToDevice, s);
   if (e == cudaSuccess)
     e = cudaMemcpyAsync(table + da::kBalanceHeader, weights, (size_t)C * 4, cudaMemcpyHostToDevice, s);
