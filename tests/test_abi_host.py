@@ -333,6 +333,16 @@ def test_balance_from_times(da_lib):
     # measured with a table in use: the same times under twice the work per CTA give twice the speed
     w3, p3 = da.da_balance_from_times(d, t, np.full(37, 2, np.int32), np.tile(np.arange(37, dtype=np.int32), (8, 1)))
     assert np.array_equal(p3, p) and np.allclose(w3, w, atol=1)
+    # a previous table must be whole and valid
+    import ctypes
+    L = da.lib()
+    out_w, out_p = np.zeros(37, np.int32), np.zeros((8, 37), np.int32)
+    ident = np.tile(np.arange(37, dtype=np.int32), (8, 1))
+    bad = ident.copy(); bad[4, 0] = 36
+    for pw, pp in [(np.full(37, 2, np.int32), None), (np.full(37, 0, np.int32), ident), (np.full(37, 2, np.int32), bad)]:
+        rc = L.da_balance_from_times(ctypes.byref(d), t.ctypes.data, None if pw is None else pw.ctypes.data,
+                                     None if pp is None else pp.ctypes.data, out_w.ctypes.data, out_p.ctypes.data)
+        assert rc == da.ERR_INVALID_ARG
 
 
 @pytest.mark.skipif(cuda_available(), reason="checks the no-device error path")
