@@ -21,6 +21,10 @@ during the measurement.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference] [--config skewed]
 
+For a bf16 cache (`--balance auto`, the default) a balance table is measured before
+the timed steps from a few steps' block times, and kept only if the graph-replayed
+step is faster with it; `launch.balance` says what was done.
+
 With N > 1 (torchrun) every rank runs its own, differently seeded batch of the
 same shape (weak scaling: requests are independent, so there is no data-path
 collective); the step time is the max over ranks and the value is the KV bytes
